@@ -1,0 +1,564 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Closed forms, library routines for special cases, hand-worked integer values,
+central finite differences (fp64) for every backward, algebraic invariants of
+the sharded method the pages state, and brute force in pure-Python loops on
+tiny shapes. The mutation tests at the end plant plausible mistakes in copies
+of oracle functions and check that some pin catches each one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+from scipy.stats import norm
+
+import oracle as O
+import tp_synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(7)
+
+
+def randn(*shape, std=1.0):
+    return rng.standard_normal(shape) * std
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_gelu_is_z_times_normal_cdf():
+    z = np.linspace(-8, 8, 4001)
+    np.testing.assert_allclose(O.gelu(z), z * norm.cdf(z), rtol=1e-13, atol=1e-15)
+    assert O.gelu(np.array([0.0]))[0] == 0.0
+    assert abs(O.gelu(np.array([30.0]))[0] - 30.0) < 1e-12
+    assert abs(O.gelu(np.array([-30.0]))[0]) < 1e-12
+
+
+def test_silu_is_z_times_logistic():
+    z = np.linspace(-30, 30, 4001)
+    np.testing.assert_allclose(O.silu(z), z * expit(z), rtol=1e-13, atol=1e-15)
+    assert O.silu(np.array([0.0]))[0] == 0.0
+
+
+def _fd_scalar(f, z, eps=1e-6):
+    return (f(z + eps) - f(z - eps)) / (2 * eps)
+
+
+def test_activation_derivatives_by_finite_differences():
+    z = np.linspace(-6, 6, 241)
+    np.testing.assert_allclose(O.gelu_grad(z), _fd_scalar(O.gelu, z), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(O.silu_grad(z), _fd_scalar(O.silu, z), rtol=1e-7, atol=1e-9)
+    assert abs(O.gelu_grad(np.array([0.0]))[0] - 0.5) < 1e-15
+    assert abs(O.silu_grad(np.array([0.0]))[0] - 0.5) < 1e-15
+
+
+# ------------------------------------------------------- hand-worked golden
+
+def test_golden_column_and_row_split():
+    g = json.load(open(os.path.join(GOLDEN, "split_2x2_hand.json")))
+    X, A, B = (np.array(g[k], dtype=np.float64) for k in ("X", "A", "B"))
+    assert np.array_equal(O.linear(X, A), np.array(g["XAt"]))
+    for i in range(2):
+        assert np.array_equal(O.linear(X, O.shard_rows(A, 2, i)), np.array(g["XAt_shards_p2"][i]))
+    assert np.array_equal(O.linear(X, B), np.array(g["XBt"]))
+    Xs = [X[:, :2], X[:, 2:]]
+    P = [O.row_partial(Xs[i], O.shard_cols(B, 2, i)) for i in range(2)]
+    for i in range(2):
+        assert np.array_equal(P[i], np.array(g["XBt_partials_p2"][i]))
+    assert np.array_equal(O.reduce_partials(P), np.array(g["XBt"]))
+
+
+# --------------------------------------------------------- brute force (loops)
+
+def _bf_linear(X, W, b=None):
+    T, n_in = len(X), len(X[0])
+    n_out = len(W)
+    Y = [[0.0] * n_out for _ in range(T)]
+    for t in range(T):
+        for o in range(n_out):
+            acc = 0.0
+            for k in range(n_in):
+                acc += X[t][k] * W[o][k]
+            Y[t][o] = acc + (b[o] if b is not None else 0.0)
+    return np.array(Y)
+
+
+def _bf_gelu(z):
+    return z * 0.5 * (1.0 + math.erf(z / math.sqrt(2.0)))
+
+
+def _bf_silu(z):
+    return z / (1.0 + math.exp(-z))
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_brute_force_mlp_tiny(act):
+    T, h, f = 5, 8, 12
+    X = randn(T, h)
+    W1 = randn(f if act == "gelu" else 2 * f, h, std=0.3)
+    W2 = randn(h, f, std=0.3)
+    b1 = randn(W1.shape[0]) if act == "gelu" else None
+    b2 = randn(h)
+    Z = _bf_linear(X.tolist(), W1.tolist(), None if b1 is None else b1.tolist())
+    if act == "gelu":
+        H = np.vectorize(_bf_gelu)(Z)
+    else:
+        H = np.vectorize(_bf_silu)(Z[:, :f]) * Z[:, f:]
+    Y = _bf_linear(H.tolist(), W2.tolist(), b2.tolist())
+    out = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    np.testing.assert_allclose(out["Z"], Z, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(out["H"], H, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(out["Y"], Y, rtol=1e-12, atol=1e-13)
+
+
+def _bf_attention(q, k, v, causal):
+    """q, k, v: lists [s][d] for one (batch, head)."""
+    s, d = len(q), len(q[0])
+    out = []
+    for i in range(s):
+        scores = []
+        for j in range(s):
+            if causal and j > i:
+                continue
+            scores.append((j, sum(q[i][x] * k[j][x] for x in range(d)) / math.sqrt(d)))
+        m = max(sc for _, sc in scores)
+        w = [(j, math.exp(sc - m)) for j, sc in scores]
+        z = sum(e for _, e in w)
+        out.append([sum(e * v[j][x] for j, e in w) / z for x in range(d)])
+    return out
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_brute_force_attention_tiny(causal):
+    s, b, H, d = 5, 2, 3, 4
+    Q, K, V = randn(s, b, H * d), randn(s, b, H * d), randn(s, b, H * d)
+    got, _ = O.attention_fwd(Q, K, V, b, H, causal)
+    for bi in range(b):
+        for hh in range(H):
+            sl = slice(hh * d, (hh + 1) * d)
+            ref = _bf_attention(Q[:, bi, sl].tolist(), K[:, bi, sl].tolist(), V[:, bi, sl].tolist(), causal)
+            np.testing.assert_allclose(got[:, bi, sl], np.array(ref), rtol=1e-12, atol=1e-13)
+
+
+def test_brute_force_layernorm_tiny():
+    x = randn(4, 10)
+    g, b = randn(10), randn(10)
+    y, mean, rstd = O.layernorm_fwd(x, g, b)
+    for r in range(4):
+        row = x[r].tolist()
+        mu = sum(row) / len(row)
+        var = sum((v - mu) ** 2 for v in row) / len(row)
+        ref = [(v - mu) / math.sqrt(var + 1e-5) * g[c] + b[c] for c, v in enumerate(row)]
+        np.testing.assert_allclose(y[r], ref, rtol=1e-12, atol=1e-13)
+        assert abs(mean[r] - mu) < 1e-14
+
+
+# ------------------------------------------------- invariants of the method
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+@pytest.mark.parametrize("act", ["none", "gelu"])
+def test_column_split_concat_equals_full(p, act):
+    """XA = [XA_1, ..., XA_p] (wiki 两种切法; walkthrough §2.1)."""
+    X, A, a = randn(6, 16), randn(32, 16), randn(32)
+    Z, H = O.column_fwd_shard(X, A, a, act)
+    parts = [O.column_fwd_shard(X, O.shard_rows(A, p, i), O.shard_vec(a, p, i), act) for i in range(p)]
+    np.testing.assert_allclose(np.concatenate([z for z, _ in parts], axis=1), Z, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(np.concatenate([hh for _, hh in parts], axis=1), H, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_swiglu_gate_up_pairing(p):
+    """Each shard must pair gate units i with up units i (walkthrough §3.2):
+    concat of the shards' H equals the unsharded H; a naive p-way split of the
+    stacked [G; U] rows does not (for p > 1)."""
+    T, h, f = 6, 16, 24
+    X, W1 = randn(T, h), randn(2 * f, h)
+    H = O.mlp_fwd(X, W1, None, randn(h, f), None, "swiglu")["H"]
+    Hs = [O.column_fwd_shard(X, O.shard_gate_up(W1, p, i), None, "swiglu")[1] for i in range(p)]
+    np.testing.assert_allclose(np.concatenate(Hs, axis=1), H, rtol=1e-13, atol=1e-14)
+    if p > 1:
+        naive = [O.column_fwd_shard(X, O.shard_rows(W1, p, i), None, "swiglu")[1] for i in range(p)]
+        assert not np.allclose(np.concatenate(naive, axis=1), H)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4, 8])
+def test_row_partials_sum_to_full(p):
+    """XB = X_1B_1 + ... + X_pB_p (wiki 两种切法; walkthrough §2.2)."""
+    H, B = randn(7, 32), randn(16, 32)
+    P = [O.row_partial(O.shard_cols(H, p, i), O.shard_cols(B, p, i)) for i in range(p)]
+    for Pi in P:
+        assert Pi.shape == (7, 16)
+    full = H @ B.T
+    assert np.abs(O.reduce_partials(P) - full).max() <= 1e-12 * np.abs(full).max()
+
+
+@pytest.mark.parametrize("p", [2, 4, 8])
+def test_bias_added_once(p):
+    """The row bias enters once, after the sum (bjdmk 实现细节). Integer values
+    make every sum exact: a per-shard bias would differ by exactly (p-1)*b."""
+    P, b, _ = tp_synth.draw_partials(p, 5, 6, torch.float32, integer_valued=True)
+    P, b = [O.f64(x) for x in P], O.f64(b)
+    once = O.reduce_partials(P, bias=b)
+    pfold = O.reduce_partials([Pi + b[None, :] for Pi in P])
+    assert np.array_equal(pfold - once, np.broadcast_to((p - 1) * b, once.shape))
+    assert np.array_equal(once, sum(P) + b[None, :])
+
+
+def test_reduce_p1_is_copy_plus_bias():
+    P, b, r = tp_synth.draw_partials(1, 4, 8, torch.float32, residual=True)
+    P, b, r = [O.f64(x) for x in P], O.f64(b), O.f64(r)
+    assert np.array_equal(O.reduce_partials(P, b, r), (P[0] + b[None, :]) + r)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_head_split_attention_equals_unsplit(p):
+    """Attention on each shard's whole heads, concatenated, equals attention on
+    all heads (walkthrough §3.1): the per-head computation is identical."""
+    s, b, H, d = 6, 2, 4, 3
+    Q, K, V = randn(s, b, H * d), randn(s, b, H * d), randn(s, b, H * d)
+    full, lse = O.attention_fwd(Q, K, V, b, H, True)
+    hl = H // p
+    outs, lses = [], []
+    for i in range(p):
+        sl = slice(i * hl * d, (i + 1) * hl * d)
+        o, l_ = O.attention_fwd(Q[:, :, sl], K[:, :, sl], V[:, :, sl], b, hl, True)
+        outs.append(o)
+        lses.append(l_)
+    assert np.array_equal(np.concatenate(outs, axis=2), full)
+    assert np.array_equal(np.concatenate(lses, axis=1), lse)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_qkv_head_shard_feeds_local_attention(p):
+    """QKV weight sharded by whole heads gives each shard exactly its heads' Q, K, V."""
+    T, h, H = 6, 12, 4
+    u, W, bq = randn(T, h), randn(3 * h, h), randn(3 * h)
+    full = O.linear(u, W, bq)
+    d, hl = h // H, H // p
+    for i in range(p):
+        part = O.linear(u, O.shard_qkv(W, H, p, i), O.shard_qkv_vec(bq, H, p, i))
+        c0, c1 = i * hl * d, (i + 1) * hl * d
+        ref = np.concatenate([full[:, c0:c1], full[:, h + c0:h + c1], full[:, 2 * h + c0:2 * h + c1]], axis=1)
+        np.testing.assert_allclose(part, ref, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4, 8])
+def test_reduce_scatter_then_all_gather_is_all_reduce(p):
+    """AG(RS(P)) == AR(P) bit for bit (walkthrough §4.3, wiki Megatron-SP)."""
+    P, b, _ = tp_synth.draw_partials(p, 8 * p, 12, torch.float32)
+    P, b = [O.f64(x) for x in P], O.f64(b)
+    assert np.array_equal(O.all_gather_seq(O.reduce_scatter_seq(P, b)), O.reduce_partials(P, b))
+
+
+def test_layernorm_commutes_with_all_gather():
+    X = randn(16, 10)
+    g, b = randn(10), randn(10)
+    shards = [X[i * 4:(i + 1) * 4] for i in range(4)]
+    a = O.all_gather_seq([O.layernorm_fwd(s_, g, b)[0] for s_ in shards])
+    assert np.array_equal(a, O.layernorm_fwd(O.all_gather_seq(shards), g, b)[0])
+
+
+def test_layernorm_rows_standardised():
+    y, _, _ = O.layernorm_fwd(randn(8, 64, std=3.0) + 5.0, np.ones(64), np.zeros(64))
+    np.testing.assert_allclose(y.mean(axis=1), 0.0, atol=1e-13)
+    np.testing.assert_allclose(y.var(axis=1), 1.0, rtol=1e-4)
+
+
+def test_softmax_rows_sum_to_one_and_causal_row0():
+    s, d = 6, 6
+    Q, K = randn(s, 1, d), randn(s, 1, d)
+    V = np.eye(s).reshape(s, 1, s)  # O = P itself when V is the identity
+    Pm, _ = O.attention_fwd(Q, K, V, 1, 1, True)
+    Pm = Pm[:, 0, :]
+    np.testing.assert_allclose(Pm.sum(axis=1), 1.0, rtol=1e-14)
+    assert np.all(np.triu(Pm, k=1) == 0.0)
+    V2 = randn(s, 1, d)
+    out, _ = O.attention_fwd(Q, K, V2, 1, 1, True)
+    assert np.array_equal(out[0, 0], V2[0, 0])
+
+
+# ------------------------------------------- backward: finite differences
+
+def _fd_grad(fun, x, eps=1e-6, idx=None):
+    """Central differences of scalar fun() with respect to entries of x (in place)."""
+    flat = x.reshape(-1)
+    if idx is None:
+        idx = range(flat.size)
+    g = []
+    for i in idx:
+        old = flat[i]
+        flat[i] = old + eps
+        fp = fun()
+        flat[i] = old - eps
+        fm = fun()
+        flat[i] = old
+        g.append((fp - fm) / (2 * eps))
+    return np.array(g)
+
+
+def _check_fd(analytic, fun, x, n=12, rtol=1e-6):
+    idx = rng.choice(x.size, size=min(n, x.size), replace=False)
+    num = _fd_grad(fun, x, idx=idx)
+    ana = analytic.reshape(-1)[idx]
+    scale = max(np.abs(ana).max(), 1e-3)
+    assert np.abs(num - ana).max() <= rtol * scale, (num, ana)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_mlp_bwd_finite_differences(act):
+    T, h, f = 4, 6, 8
+    X = randn(T, h)
+    W1 = randn(f if act == "gelu" else 2 * f, h, std=0.5)
+    W2 = randn(h, f, std=0.5)
+    b1 = randn(W1.shape[0]) if act == "gelu" else None
+    b2 = randn(h)
+    C = randn(T, h)  # loss = sum(C * Y), so dY = C
+
+    def loss():
+        return float((O.mlp_fwd(X, W1, b1, W2, b2, act)["Y"] * C).sum())
+
+    fwd = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    g = O.mlp_bwd(X, W1, W2, fwd["Z"], fwd["H"], C, act)
+    _check_fd(g["dX"], loss, X)
+    _check_fd(g["dW1"], loss, W1)
+    _check_fd(g["dW2"], loss, W2)
+    _check_fd(g["db2"], loss, b2)
+    if b1 is not None:
+        _check_fd(g["db1"], loss, b1)
+
+
+def test_layernorm_bwd_finite_differences():
+    x, g, b = randn(5, 7), randn(7), randn(7)
+    C = randn(5, 7)
+
+    def loss():
+        return float((O.layernorm_fwd(x, g, b)[0] * C).sum())
+
+    _, mean, rstd = O.layernorm_fwd(x, g, b)
+    dx, dg, db = O.layernorm_bwd(x, g, C, mean, rstd)
+    _check_fd(dx, loss, x, n=20)
+    _check_fd(dg, loss, g, n=7)
+    _check_fd(db, loss, b, n=7)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_attention_bwd_finite_differences(causal):
+    s, b, H, d = 5, 2, 2, 3
+    Q, K, V = randn(s, b, H * d), randn(s, b, H * d), randn(s, b, H * d)
+    C = randn(s, b, H * d)
+
+    def loss():
+        return float((O.attention_fwd(Q, K, V, b, H, causal)[0] * C).sum())
+
+    dQ, dK, dV = O.attention_bwd(Q, K, V, C, b, H, causal)
+    _check_fd(dQ, loss, Q, n=20)
+    _check_fd(dK, loss, K, n=20)
+    _check_fd(dV, loss, V, n=20)
+
+
+def test_attention_lse_definition():
+    s, b, H, d = 4, 1, 1, 2
+    Q, K, V = randn(s, b, d), randn(s, b, d), randn(s, b, d)
+    _, lse = O.attention_fwd(Q, K, V, b, H, True)
+    for i in range(s):
+        sc = [float(Q[i, 0] @ K[j, 0]) / math.sqrt(d) for j in range(i + 1)]
+        assert abs(lse[0, 0, i] - math.log(sum(math.exp(x) for x in sc))) < 1e-12
+
+
+def _layer_params(h, f, H):
+    P = {"ln1_g": 1 + 0.1 * randn(h), "ln1_b": 0.1 * randn(h), "Wqkv": randn(3 * h, h, std=0.4),
+         "bqkv": 0.1 * randn(3 * h), "Wo": randn(h, h, std=0.4), "bo": 0.1 * randn(h),
+         "ln2_g": 1 + 0.1 * randn(h), "ln2_b": 0.1 * randn(h), "W1": randn(f, h, std=0.4),
+         "b1": 0.1 * randn(f), "W2": randn(h, f, std=0.4), "b2": 0.1 * randn(h)}
+    return P
+
+
+def test_layer_bwd_finite_differences():
+    batch, s, h, f, H = 2, 3, 4, 8, 2
+    x = randn(batch * s, h)
+    P = _layer_params(h, f, H)
+    C = randn(batch * s, h)
+
+    def loss():
+        return float((O.layer_fwd(x, P, batch, H)["y"] * C).sum())
+
+    cache = O.layer_fwd(x, P, batch, H)
+    g = O.layer_bwd(cache, P, C, batch, H)
+    _check_fd(g["dx"], loss, x, n=10)
+    for name, gname in [("Wqkv", "dWqkv"), ("bqkv", "dbqkv"), ("Wo", "dWo"), ("bo", "dbo"),
+                        ("W1", "dW1"), ("b1", "db1"), ("W2", "dW2"), ("b2", "db2"),
+                        ("ln1_g", "dln1_g"), ("ln1_b", "dln1_b"), ("ln2_g", "dln2_g"), ("ln2_b", "dln2_b")]:
+        _check_fd(g[gname], loss, P[name], n=6)
+
+
+def test_sp_mlp_bwd_finite_differences():
+    s, h, f = 6, 6, 8
+    X, g, b = randn(s, h), 1 + 0.1 * randn(h), 0.1 * randn(h)
+    W1, W2 = randn(2 * f, h, std=0.5), randn(h, f, std=0.5)
+    C = randn(s, h)
+
+    def loss():
+        return float((O.sp_mlp_fwd(X, g, b, W1, W2)["Y"] * C).sum())
+
+    fwd = O.sp_mlp_fwd(X, g, b, W1, W2)
+    gr = O.sp_mlp_bwd(X, g, W1, W2, fwd, C)
+    _check_fd(gr["dX"], loss, X)
+    _check_fd(gr["dg"], loss, g, n=6)
+    _check_fd(gr["db"], loss, b, n=6)
+    _check_fd(gr["dW1"], loss, W1)
+
+
+# ----------------------------------- sharded backward equals the unsharded one
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_sharded_backward_matches_unsharded(p, act):
+    """Row bwd needs no sum (dY replicated); column bwd dX partials sum to dX
+    (从零实现 Tensor Parallel §四)."""
+    T, h, f = 6, 8, 16
+    X = randn(T, h)
+    W1 = randn(f if act == "gelu" else 2 * f, h, std=0.5)
+    W2 = randn(h, f, std=0.5)
+    b1 = randn(W1.shape[0]) if act == "gelu" else None
+    dY = randn(T, h)
+    fwd = O.mlp_fwd(X, W1, b1, W2, None, act)
+    ref = O.mlp_bwd(X, W1, W2, fwd["Z"], fwd["H"], dY, act)
+    shard = (lambda W, i: O.shard_rows(W, p, i)) if act == "gelu" else (lambda W, i: O.shard_gate_up(W, p, i))
+    dXp, dW1s, dW2s, db1s = [], [], [], []
+    for i in range(p):
+        Wi = shard(W1, i)
+        bi = None if b1 is None else O.shard_vec(b1, p, i)
+        Zi, Hi = O.column_fwd_shard(X, Wi, bi, act)
+        dZi, dW2i = O.row_bwd_shard(dY, Hi, O.shard_cols(W2, p, i), Zi, act)
+        dWi, dbi, dXi = O.column_bwd_shard(X, dZi, Wi)
+        dXp.append(dXi)
+        dW1s.append(dWi)
+        dW2s.append(dW2i)
+        db1s.append(dbi)
+    np.testing.assert_allclose(O.reduce_partials(dXp), ref["dX"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(dW2s, axis=1), ref["dW2"], rtol=1e-12, atol=1e-12)
+    for i in range(p):
+        np.testing.assert_allclose(dW1s[i], shard(ref["dW1"], i), rtol=1e-12, atol=1e-12)
+        if b1 is not None:
+            np.testing.assert_allclose(db1s[i], O.shard_vec(ref["db1"], p, i), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_sp_pipeline_equals_unsharded(p):
+    """LN on sequence shards -> AG -> column -> row partials -> RS equals the
+    unsharded LN -> MLP, and the backward (AG of dY, RS of dX partials, LN bwd
+    per shard, dgamma/dbeta summed over shards) equals the unsharded backward."""
+    s, h, f = 8, 8, 16
+    X, g, b = randn(s, h), 1 + 0.1 * randn(h), 0.1 * randn(h)
+    W1, W2 = randn(2 * f, h, std=0.5), randn(h, f, std=0.5)
+    dY = randn(s, h)
+    ref = O.sp_mlp_fwd(X, g, b, W1, W2)
+    refb = O.sp_mlp_bwd(X, g, W1, W2, ref, dY)
+    t = s // p
+    Xs = [X[j * t:(j + 1) * t] for j in range(p)]
+    lns = [O.layernorm_fwd(x, g, b) for x in Xs]
+    u = O.all_gather_seq([l_[0] for l_ in lns])
+    Zs, Hs, P = [], [], []
+    for i in range(p):
+        Zi, Hi = O.column_fwd_shard(u, O.shard_gate_up(W1, p, i), None, "swiglu")
+        Zs.append(Zi)
+        Hs.append(Hi)
+        P.append(O.row_partial(Hi, O.shard_cols(W2, p, i)))
+    Ys = O.reduce_scatter_seq(P)
+    np.testing.assert_allclose(O.all_gather_seq(Ys), ref["Y"], rtol=1e-12, atol=1e-12)
+    dYfull = O.all_gather_seq([dY[j * t:(j + 1) * t] for j in range(p)])
+    dXp = []
+    for i in range(p):
+        dZi, _ = O.row_bwd_shard(dYfull, Hs[i], O.shard_cols(W2, p, i), Zs[i], "swiglu")
+        dXp.append(O.column_bwd_shard(u, dZi, O.shard_gate_up(W1, p, i))[2])
+    du_seq = O.reduce_scatter_seq(dXp)
+    dXs, dgs, dbs = [], [], []
+    for j in range(p):
+        dx, dg_, db_ = O.layernorm_bwd(Xs[j], g, du_seq[j], lns[j][1], lns[j][2])
+        dXs.append(dx)
+        dgs.append(dg_)
+        dbs.append(db_)
+    np.testing.assert_allclose(O.all_gather_seq(dXs), refb["dX"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(sum(dgs), refb["dg"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(sum(dbs), refb["db"], rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_sampled_backward_matches_full(act):
+    T, h, f = 20, 8, 12
+    X = randn(T, h)
+    W1 = randn(f if act == "gelu" else 2 * f, h, std=0.5)
+    b1 = randn(W1.shape[0]) if act == "gelu" else None
+    W2, dY = randn(h, f, std=0.5), randn(T, h)
+    fwd = O.mlp_fwd(X, W1, b1, W2, None, act)
+    ref = O.mlp_bwd(X, W1, W2, fwd["Z"], fwd["H"], dY, act)
+    rows, fcols = np.array([0, 3, 19]), np.array([1, 5, 11])
+    smp = O.mlp_bwd_sampled(X, W1, b1, W2, dY, act, rows, fcols)
+    np.testing.assert_allclose(smp["dX_rows"], ref["dX"][rows], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(smp["dW2_cols"], ref["dW2"][:, fcols], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(smp["dW1_rows"], ref["dW1"][smp["W1_rows_index"]], rtol=1e-12, atol=1e-12)
+    if act == "gelu":
+        np.testing.assert_allclose(smp["db1"], ref["db1"][fcols], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(
+        O.mlp_fwd_rows(X, W1, b1, W2, None, act, rows)["Y"], fwd["Y"][rows], rtol=1e-12, atol=1e-12)
+
+
+def test_max_row_rel_err():
+    ref = np.array([[1.0, -4.0], [0.0, 0.0], [2.0, 1.0]])
+    got = ref + np.array([[0.0, 0.04], [0.0, 0.0], [0.02, 0.0]])
+    assert abs(O.max_row_rel_err(got, ref) - 0.01) < 1e-15
+    assert O.max_row_rel_err(got * np.nan, ref) == float("inf")
+
+
+def test_divisibility_is_checked():
+    with pytest.raises(ValueError):
+        O.shard_rows(np.zeros((10, 4)), 4, 0)
+    with pytest.raises(ValueError):
+        O.shard_qkv(np.zeros((3 * 12, 12)), 3, 2, 0)
+
+
+# ------------------------------------------------ mutation checks (plant bugs)
+
+def _mut_gelu_tanh(z):
+    return 0.5 * z * (1 + np.tanh(math.sqrt(2 / math.pi) * (z + 0.044715 * z ** 3)))
+
+
+def test_mutant_tanh_gelu_fails_the_cdf_pin():
+    z = np.linspace(-8, 8, 4001)
+    assert not np.allclose(_mut_gelu_tanh(z), z * norm.cdf(z), rtol=1e-13, atol=1e-15)
+
+
+def test_mutant_layernorm_bwd_dropped_term_fails_fd():
+    x, g, b = randn(5, 7), randn(7), randn(7)
+    C = randn(5, 7)
+    _, mean, rstd = O.layernorm_fwd(x, g, b)
+    xhat = (x - mean[:, None]) * rstd[:, None]
+    gy = C * g[None, :]
+    bad_dx = rstd[:, None] * (gy - gy.mean(axis=1, keepdims=True))  # dropped the xhat term
+    with pytest.raises(AssertionError):
+        _check_fd(bad_dx, lambda: float((O.layernorm_fwd(x, g, b)[0] * C).sum()), x, n=20)
+
+
+def test_mutant_attention_missing_scale_fails_brute_force():
+    s, b, H, d = 4, 1, 1, 4
+    Q, K, V = randn(s, b, d), randn(s, b, d), randn(s, b, d)
+    bad, _ = O.attention_fwd(Q * math.sqrt(d), K, V, b, H, True)  # scale dropped
+    ref = _bf_attention(Q[:, 0].tolist(), K[:, 0].tolist(), V[:, 0].tolist(), True)
+    assert not np.allclose(bad[:, 0], np.array(ref), rtol=1e-6)
+
+
+def test_mutant_transposed_row_shard_fails_the_sum_pin():
+    H, B = randn(7, 32), randn(16, 32)
+    p = 4
+    bad = [O.shard_cols(H, p, i) @ O.shard_cols(B, p, p - 1 - i).T for i in range(p)]  # wrong shard index
+    assert not np.allclose(O.reduce_partials(bad), H @ B.T)
+
+
+def test_mutant_silu_grad_sign_fails_fd():
+    z = np.linspace(-6, 6, 241)
+    s = 1 / (1 + np.exp(-z))
+    bad = s * (1 - z * (1 - s))
+    assert not np.allclose(bad, _fd_scalar(O.silu, z), rtol=1e-7, atol=1e-9)
