@@ -1,0 +1,271 @@
+/*
+ * tp.h -- C ABI of the single-GPU tensor-parallel (TP) block library, libtp.so.
+ *
+ * The library computes the Megatron tensor-parallel MLP and attention block
+ * with all p shards held as separate buffers on ONE GPU, so each "collective"
+ * of the method (all-reduce, reduce-scatter, all-gather) is a local kernel
+ * over HBM. Sources, cited by page title and section:
+ *   [TP-blog]    "企业官网建设流程全解析" (2kiu.com), a TP walkthrough: §2.1 column
+ *                parallel, §2.2 row parallel, §2.3 pairing, §3.1 attention split
+ *                by heads, §3.2 MLP with gate/up in one column shard, §3.3
+ *                normalisation, §4.1 collectives, §4.3 sequence parallelism,
+ *                §6.1 divisibility checks before model init.
+ *   [TP-wiki]    "张量并行" (ai-infra-wiki): 两种切法 (Y = GELU(XA)B,
+ *                XA = [XA_1, XA_2], XB = X_1B_1 + X_2B_2), 序列维度的补充：Megatron-SP.
+ *   [TP-scratch] "大模型分布式训练篇——从零实现 Tensor Parallel" (makesence), §四:
+ *                column forward identity / backward all-reduce, and the mirror.
+ *   [TP-basics]  "Tensor Parallelism基础：模型切分原理" (bjdmk), 实现细节: the
+ *                F.linear [out, in] weight layout, row bias added once after the sum.
+ *
+ * Conventions for every call
+ *   - Pointers named in the argument lists are DEVICE pointers unless stated.
+ *     Arrays of per-shard pointers (`const void* const* X`) are HOST arrays of
+ *     n (= p unless stated) device pointers; the array itself is read during
+ *     the call only.
+ *   - Tensors are dense row-major. Weights use the [out, in] layout of
+ *     F.linear; activations are [T, features] with T = batch * seq tokens in
+ *     sequence-major order (row = s * batch + b), so a sequence shard is a
+ *     contiguous block of rows.
+ *   - Element types follow the plan dtype (TP_BF16: bf16 storage, fp32
+ *     accumulation; TP_F32: fp32 throughout) except where a parameter is
+ *     typed `float*`: statistics and bias / LayerNorm-parameter gradients
+ *     are always fp32.
+ *   - Every device pointer must be 16-byte aligned and every row (the
+ *     innermost extent times the element size) a multiple of 16 bytes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it; they take no locks and never synchronise.
+ *   - Ownership: the caller owns every tensor. The plan owns host metadata and
+ *     a device workspace that the library allocates (cudaMalloc) the first
+ *     time a call needs scratch space and frees in tp_plan_destroy.
+ *   - Errors: argument, shape, divisibility and alignment errors are detected
+ *     on the host and returned BEFORE any launch, with detail text available
+ *     from tp_last_error() (thread-local). A failed launch returns TP_ERR_CUDA.
+ *     Kernels never trap: a device wait that runs past its time limit sets a
+ *     device status word and the kernel returns; read it with
+ *     tp_get_device_status().
+ *   - A plan may be used from one host thread at a time.
+ */
+#ifndef TP_H_
+#define TP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TP_MAX_SHARDS 16
+
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
+typedef struct tp_plan tp_plan; /* opaque, host side */
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_ARG = 1,          /* NULL / out-of-range argument */
+  TP_ERR_DIVISIBILITY = 2, /* a dimension is not divisible by p ([TP-blog] §6.1) */
+  TP_ERR_ALIGN = 3,        /* pointer or row not 16-byte aligned */
+  TP_ERR_DTYPE = 4,        /* combination not available for this dtype */
+  TP_ERR_UNSUPPORTED = 5,  /* shape beyond what the kernels support */
+  TP_ERR_CUDA = 6,         /* CUDA runtime / driver error (detail in tp_last_error) */
+  TP_ERR_TIMEOUT = 7,      /* a device-side wait gave up (from tp_get_device_status) */
+  TP_ERR_NO_DEVICE = 8     /* no usable sm_100 device */
+} tp_status;
+
+typedef enum { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+
+/* Activation between the column and the row GEMM of the MLP.
+ * GELU is the exact erf form; SWIGLU is H = SiLU(gate) * up with the column
+ * shard holding [G_i; U_i] (gate rows first) ([TP-blog] §3.2). */
+typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU = 1, TP_ACT_SWIGLU = 2 } tp_act;
+
+/* Which projection a GEMM call is for; fixes the shard shapes.
+ *   TP_MLP:     column W1 [n1, hidden] (n1 = ffn, or 2*ffn for SwiGLU),
+ *               row W2 [hidden, ffn].
+ *   TP_QKV:     column Wqkv [3*hidden, hidden], rows [Wq; Wk; Wv], split by
+ *               whole heads ([TP-blog] §3.1). No activation.
+ *   TP_OUTPROJ: row Wo [hidden, hidden], input = local heads' outputs. */
+typedef enum { TP_MLP = 0, TP_QKV = 1, TP_OUTPROJ = 2 } tp_which;
+
+/* ---------------------------------------------------------------- plan */
+
+/* Create a plan for one block. Checks, before anything else ([TP-blog] §6.1):
+ * p in [1, TP_MAX_SHARDS]; hidden % p, heads % p, hidden % heads, ffn % p
+ * (and the doubled gate+up column count 2*ffn % p for SwiGLU) all zero.
+ * ffn may be 0 (attention-only plan); heads may be 0 (MLP-only plan).
+ * Allocates no device memory. Returns TP_ERR_DIVISIBILITY naming the failing
+ * dimension (tp_last_error), TP_ERR_ARG for non-positive sizes. */
+TP_API tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype,
+                         tp_act act, tp_plan** out);
+TP_API void tp_plan_destroy(tp_plan* plan);
+
+/* Write a text description of every shard shape into buf (host, n bytes,
+ * always NUL-terminated) -- the shape print [TP-blog] §6.1/§6.4 asks for. */
+TP_API tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n);
+
+TP_API const char* tp_status_string(tp_status s);
+TP_API const char* tp_last_error(void);
+
+/* Synchronise `stream`, read the device status word of the current device,
+ * store it in *device_status (TP_OK or TP_ERR_TIMEOUT) and clear it. */
+TP_API tp_status tp_get_device_status(void* stream, int* device_status);
+
+/* Number of kernel launches this thread has issued through the library
+ * since the last reset (host counter; used to report launch counts). */
+TP_API uint64_t tp_launch_count(int reset);
+
+/* ------------------------------------------------------------ sharding
+ * Bit-exact copies between a full weight and its p shards.
+ * [TP-blog] §2.1 (column: blocks of the output dim), §2.2 (row: blocks of the
+ * input dim), §3.1 (QKV: whole heads from each of Wq, Wk, Wv), §3.2 (SwiGLU:
+ * shard i = [G rows i*f/p.., U rows i*f/p..]).
+ *   column, TP_MLP:  W_full [n1, hidden] -> W_shards[i] [n1/p, hidden]
+ *   column, TP_QKV:  W_full [3h, h]      -> W_shards[i] [3h/p, h] = [Q_i; K_i; V_i]
+ *   row,    TP_MLP:  W_full [h, ffn]     -> W_shards[i] [h, ffn/p]
+ *   row,    TP_OUTPROJ: W_full [h, h]    -> W_shards[i] [h, h/p]
+ * The bias variants shard a column bias the same way (vectors). */
+TP_API tp_status tp_shard_column(const tp_plan* plan, tp_which which, const void* W_full,
+                          void* const* W_shards, void* stream);
+TP_API tp_status tp_unshard_column(const tp_plan* plan, tp_which which, const void* const* W_shards,
+                            void* W_full, void* stream);
+TP_API tp_status tp_shard_row(const tp_plan* plan, tp_which which, const void* W_full,
+                       void* const* W_shards, void* stream);
+TP_API tp_status tp_unshard_row(const tp_plan* plan, tp_which which, const void* const* W_shards,
+                         void* W_full, void* stream);
+TP_API tp_status tp_shard_column_bias(const tp_plan* plan, tp_which which, const void* b_full,
+                               void* const* b_shards, void* stream);
+
+/* ------------------------------------------------------------- forward */
+
+/* Column-parallel GEMM of every shard in one launch, with its epilogue.
+ * [TP-blog] §2.1, [TP-wiki] 两种切法 (XA = [XA_1, ..., XA_p], no communication),
+ * [TP-basics] (column bias sharded with its columns).
+ *   X:    [T, hidden], replicated input.
+ *   W[i]: column shard i (see the sharding calls).
+ *   bias: NULL, or bias[i] = shard i of the column bias (length of W[i]'s rows).
+ *         Not allowed with SwiGLU.
+ *   TP_MLP, GELU:   Z[i] [T, ffn/p] = X W[i]^T + bias[i] (pre-activation, may be
+ *                   NULL when no backward follows); H[i] [T, ffn/p] = GELU(Z[i]).
+ *   TP_MLP, SWIGLU: Z[i] [T, 2*ffn/p] = [Zg | Zu] (may be NULL);
+ *                   H[i] [T, ffn/p] = SiLU(Zg) * Zu.
+ *   TP_MLP, NONE:   H[i] = X W[i]^T + bias[i]; Z must be NULL.
+ *   TP_QKV:         H[i] [T, 3h/p] = [Q_i | K_i | V_i] = X W[i]^T + bias[i];
+ *                   Z must be NULL.
+ * bf16 plans run the tcgen05 tensor-core kernel; fp32 plans an fp32 FMA kernel. */
+TP_API tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                        const void* const* W, const void* const* bias, void* const* Z,
+                        void* const* H, void* stream);
+
+/* Row-parallel GEMM of every shard: P[i] [T, hidden] = H[i] W[i]^T, the
+ * full-shape partial sums, with NO bias ([TP-blog] §2.2, [TP-wiki] XB = X_1B_1 +
+ * X_2B_2). H[i] is [T, ffn/p] (TP_MLP) or [T, h/p] (TP_OUTPROJ); W[i] the row shard. */
+TP_API tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                             const void* const* W, void* const* P, void* stream);
+
+/* The all-reduce of the row layer, done locally: Y = sum_{i<n} P[i] (fp32, in
+ * order 0..n-1), then + bias once (NULL ok), then + residual (NULL ok).
+ * [TP-blog] §2.2, [TP-basics] (bias once, after the sum). P[i], residual, Y
+ * are [T, hidden]; bias [hidden]. Y may alias residual. */
+TP_API tp_status tp_reduce_partials(tp_plan* plan, int64_t T, int n, const void* const* P,
+                             const void* bias, const void* residual, void* Y, void* stream);
+
+/* Sequence-parallel form of the reduction ([TP-blog] §4.3, [TP-wiki] Megatron-SP):
+ * Y_seq[j] [T/n, hidden] = rows [j*T/n, (j+1)*T/n) of (sum_i P[i] + bias),
+ * plus residual_seq[j] (NULL array ok). T % n must be 0. */
+TP_API tp_status tp_reduce_scatter_seq(tp_plan* plan, int64_t T, int n, const void* const* P,
+                                const void* bias, const void* const* residual_seq,
+                                void* const* Y_seq, void* stream);
+
+/* All-gather along the sequence: X_full [T, hidden] = rows of X_seq[0..n-1]
+ * ([T/n, hidden] each) in order. Bit-exact copy. */
+TP_API tp_status tp_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* const* X_seq,
+                            void* X_full, void* stream);
+
+/* LayerNorm over the full hidden dim ([TP-blog] §3.3): y = (x - mean) * rstd *
+ * gamma + beta, biased variance, eps = 1e-5. x, y [rows, hidden]; gamma, beta
+ * [hidden]; mean, rstd [rows] fp32 outputs (either may be NULL). */
+TP_API tp_status tp_layernorm_fwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
+                           const void* beta, void* y, float* mean, float* rstd, void* stream);
+
+/* LayerNorm on each sequence shard fused with the all-gather that follows it
+ * in Megatron-SP ([TP-blog] §4.3): Y_full row j*T/n + r = LN(X_seq[j] row r).
+ * mean, rstd: [T] fp32 in full-sequence order (NULL ok). */
+TP_API tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* const* X_seq,
+                                      const void* gamma, const void* beta, void* Y_full,
+                                      float* mean, float* rstd, void* stream);
+
+/* Causal attention of each shard's local heads ([TP-blog] §3.1: full sequence,
+ * whole heads, no cross-shard step). QKV[i] [seq*batch, 3*h/p] = [Q_i|K_i|V_i]
+ * (the TP_QKV column output); O[i] [seq*batch, h/p] with head j of the shard
+ * in columns [j*d, (j+1)*d); LSE[i] [batch, heads/p, seq] fp32 log-sum-exp of
+ * each row's scaled, masked scores (NULL ok when no backward follows).
+ * softmax(Q K^T / sqrt(d), causal j <= i) V. */
+TP_API tp_status tp_attention_fwd(tp_plan* plan, int batch, int seq, const void* const* QKV,
+                           void* const* O, float* const* LSE, void* stream);
+
+/* ------------------------------------------------------------ backward */
+
+/* Row layer backward for every shard ([TP-scratch] §四: the input gradient of
+ * the row layer needs no reduction; dY is replicated).
+ *   dY [T, hidden]; H[i] the row input of shard i; W[i] the row shard.
+ *   TP_MLP: dZ[i] = act'(dH_i) with dH_i = dY W[i]: GELU: dZ[i] [T, ffn/p] =
+ *     dH_i * GELU'(Z[i]); SWIGLU: Z[i] = [Zg|Zu], dZ[i] [T, 2ffn/p] =
+ *     [dH_i * Zu * SiLU'(Zg) | dH_i * SiLU(Zg)]; NONE: dZ[i] = dH_i.
+ *   TP_OUTPROJ: dZ[i] [T, h/p] = dY W[i] (Z ignored).
+ *   dW[i] = dY^T H[i] (shape of W[i]; NULL array skips);
+ *   dbias [hidden] fp32 = sum over tokens of dY, computed once (NULL skips). */
+TP_API tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
+                     const void* const* H, const void* const* W, const void* const* Z,
+                     void* const* dZ, void* const* dW, float* dbias, void* stream);
+
+/* Column layer backward for every shard ([TP-scratch] §四: forward identity,
+ * backward sum of the input gradient).
+ *   X [T, hidden]; dZ[i] the gradient of shard i's pre-activation output;
+ *   W[i] the column shard. dW[i] = dZ[i]^T X (NULL array skips); dbias[i] fp32
+ *   = sum over tokens of dZ[i] (NULL array skips); dX_partials[i] [T, hidden] =
+ *   dZ[i] W[i], to be summed by tp_reduce_partials (or tp_all_gather_seq_bwd). */
+TP_API tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                        const void* const* dZ, const void* const* W, void* const* dW,
+                        float* const* dbias, void* const* dX_partials, void* stream);
+
+/* Backward of tp_reduce_scatter_seq: the all-gather of the dY sequence shards
+ * into dY_full [T, hidden] (the conjugate of the reduce-scatter, [TP-wiki]
+ * Megatron-SP). */
+TP_API tp_status tp_reduce_scatter_seq_bwd(tp_plan* plan, int64_t T, int n, const void* const* dY_seq,
+                                    void* dY_full, void* stream);
+
+/* Backward of tp_all_gather_seq: the reduce-scatter of the n full-shape dX
+ * partials into sequence shards dX_seq[j] [T/n, hidden]. */
+TP_API tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const void* const* dX_partials,
+                                void* const* dX_seq, void* stream);
+
+/* LayerNorm backward: dx [rows, hidden] (plan dtype); dgamma, dbeta [hidden]
+ * fp32 (sums over the rows; when accumulate != 0 they are added to the
+ * existing contents, so shards can be summed). mean/rstd from the forward. */
+TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
+                           const void* dy, const float* mean, const float* rstd, void* dx,
+                           float* dgamma, float* dbeta, int accumulate, void* stream);
+
+/* Attention backward of each shard's local heads: from QKV[i], O[i], dO[i]
+ * and LSE[i] of the forward, writes dQKV[i] [seq*batch, 3h/p] = [dQ|dK|dV].
+ * dV = P^T dO; dS = P * (dO V^T - rowsum(dO * O)); dQ = dS K / sqrt(d);
+ * dK = dS^T Q / sqrt(d). */
+TP_API tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void* const* QKV,
+                           const void* const* O, const void* const* dO,
+                           const float* const* LSE, void* const* dQKV, void* stream);
+
+/* Column sums over rows: out[c] = sum_r x[r, c] in fp32 (fixed order;
+ * accumulate != 0 adds to out). x [rows, cols] in the plan dtype. */
+TP_API tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const void* x, float* out,
+                        int accumulate, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_H_ */

@@ -1,0 +1,164 @@
+"""Call sequences of the tensor-parallel sublayers on one GPU.
+
+Buffers are torch CUDA tensors (device memory only); every step is one or
+more libtp.so calls. Shard i of every layer is a separate buffer, as it would
+be a separate rank's memory; the "collectives" are the library's local
+reduce / reduce-scatter / all-gather kernels.
+
+  TPMLP      column GEMM (+bias, GELU or SwiGLU) -> row GEMM partials ->
+             reduce (+bias once); backward: row bwd (act' fused) -> column bwd
+             -> reduce of the dX partials.       (TP walkthrough §2-§3.2, §四 of
+             "从零实现 Tensor Parallel" for the backward pairing)
+  SPMLP      Megatron-SP: LN on sequence shards fused with the all-gather ->
+             column -> row -> reduce-scatter; backward: all-gather of dY ->
+             row bwd -> column bwd -> reduce-scatter of dX partials -> LN bwd
+             per shard.                            (TP walkthrough §4.3, wiki Megatron-SP)
+"""
+from __future__ import annotations
+
+import torch
+
+from .tp import Plan
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+class TPMLP:
+    """One MLP sublayer split over p shards that all live on ``device``."""
+
+    def __init__(self, hidden: int, ffn: int, p: int, act: str = "gelu", dtype: str = "bf16",
+                 device="cuda", bias: bool = False, partial_dtype=None):
+        self.h, self.f, self.p, self.act = hidden, ffn, p, act
+        self.plan = Plan(hidden, ffn, 0, p, dtype, act)
+        self.dt = self.plan.torch_dtype
+        self.device = torch.device(device)
+        self.bias = bias
+        fp = ffn // p
+        self.n1 = 2 * fp if act == "swiglu" else fp
+        self.fp = fp
+        dev, dt = self.device, self.dt
+        self.W1 = [_empty((self.n1, hidden), dt, dev) for _ in range(p)]
+        self.W2 = [_empty((hidden, fp), dt, dev) for _ in range(p)]
+        self.b1 = [_empty((self.n1,), dt, dev) for _ in range(p)] if bias else None
+        self.b2 = _empty((hidden,), dt, dev) if bias else None
+        self._T = None
+
+    # --------------------------------------------------------------- weights
+    def load_weights(self, W1_full: torch.Tensor, W2_full: torch.Tensor, b1_full=None, b2_full=None):
+        """Shard full weights (already on the device) into the per-shard buffers."""
+        self.plan.shard_column("mlp", W1_full.contiguous(), self.W1)
+        self.plan.shard_row("mlp", W2_full.contiguous(), self.W2)
+        if self.bias:
+            self.plan.shard_column_bias("mlp", b1_full.contiguous(), self.b1)
+            self.b2.copy_(b2_full)
+
+    # ------------------------------------------------------------ activations
+    def alloc(self, T: int, backward: bool = True):
+        if self._T == T and (not backward or hasattr(self, "dZ")):
+            return
+        dev, dt, p = self.device, self.dt, self.p
+        self._T = T
+        self.Z = [_empty((T, self.n1), dt, dev) for _ in range(p)]
+        self.H = [_empty((T, self.fp), dt, dev) for _ in range(p)]
+        self.P = [_empty((T, self.h), dt, dev) for _ in range(p)]
+        self.Y = _empty((T, self.h), dt, dev)
+        if backward:
+            self.dZ = [_empty((T, self.n1), dt, dev) for _ in range(p)]
+            self.dXp = [_empty((T, self.h), dt, dev) for _ in range(p)]
+            self.dX = _empty((T, self.h), dt, dev)
+            self.dW1 = [torch.empty_like(w) for w in self.W1]
+            self.dW2 = [torch.empty_like(w) for w in self.W2]
+            self.db1 = [_empty((self.n1,), torch.float32, dev) for _ in range(p)] if self.bias else None
+            self.db2 = _empty((self.h,), torch.float32, dev) if self.bias else None
+
+    # ---------------------------------------------------------------- passes
+    def forward(self, X: torch.Tensor, residual=None, out=None):
+        T = X.shape[0]
+        self.alloc(T, backward=hasattr(self, "dZ") or True)
+        self.X = X
+        pl = self.plan
+        pl.column_fwd("mlp", T, X, self.W1, self.b1, self.Z if self.act != "none" else None, self.H)
+        pl.row_fwd_partial("mlp", T, self.H, self.W2, self.P)
+        Y = self.Y if out is None else out
+        pl.reduce_partials(T, self.P, self.b2, residual, Y)
+        return Y
+
+    def backward(self, dY: torch.Tensor, out=None):
+        T = dY.shape[0]
+        pl = self.plan
+        pl.row_bwd("mlp", T, dY, self.H, self.W2, self.Z if self.act != "none" else None, self.dZ,
+                   self.dW2, self.db2)
+        pl.column_bwd("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.dXp)
+        dX = self.dX if out is None else out
+        pl.reduce_partials(T, self.dXp, None, None, dX)
+        return dX
+
+    # Number of useful FLOPs in one forward + backward (three GEMMs of each layer).
+    def flops(self, T: int) -> float:
+        n1_total = self.n1 * self.p
+        fwd = 2.0 * T * self.h * n1_total + 2.0 * T * self.f * self.h
+        return 3.0 * fwd
+
+
+class SPMLP:
+    """Megatron-SP SwiGLU MLP: LayerNorm on sequence shards, all-gather, column,
+    row, reduce-scatter (and the mirrored backward)."""
+
+    def __init__(self, hidden: int, ffn: int, p: int, act: str = "swiglu", device="cuda"):
+        self.mlp = TPMLP(hidden, ffn, p, act, "bf16", device, bias=False)
+        self.plan = self.mlp.plan
+        self.h, self.p = hidden, p
+        self.gamma = torch.ones(hidden, dtype=torch.bfloat16, device=device)
+        self.beta = torch.zeros(hidden, dtype=torch.bfloat16, device=device)
+        self.device = torch.device(device)
+        self._T = None
+
+    def alloc(self, T: int):
+        if self._T == T:
+            return
+        self._T = T
+        dev, p, h = self.device, self.p, self.h
+        t = T // p
+        self.U = _empty((T, h), torch.bfloat16, dev)          # LN output, gathered
+        self.mean = _empty((T,), torch.float32, dev)
+        self.rstd = _empty((T,), torch.float32, dev)
+        self.Y_seq = [_empty((t, h), torch.bfloat16, dev) for _ in range(p)]
+        self.dY_full = _empty((T, h), torch.bfloat16, dev)
+        self.dU_seq = [_empty((t, h), torch.bfloat16, dev) for _ in range(p)]
+        self.dX_seq = [_empty((t, h), torch.bfloat16, dev) for _ in range(p)]
+        self.dgamma = _empty((h,), torch.float32, dev)
+        self.dbeta = _empty((h,), torch.float32, dev)
+        self.mlp.alloc(T)
+
+    def forward(self, X_seq):
+        p = self.p
+        T = X_seq[0].shape[0] * p
+        self.alloc(T)
+        self.X_seq = X_seq
+        pl, m = self.plan, self.mlp
+        pl.layernorm_all_gather_seq(T, X_seq, self.gamma, self.beta, self.U, self.mean, self.rstd)
+        m.X = self.U
+        pl.column_fwd("mlp", T, self.U, m.W1, None, m.Z, m.H)
+        pl.row_fwd_partial("mlp", T, m.H, m.W2, m.P)
+        pl.reduce_scatter_seq(T, m.P, None, None, self.Y_seq)
+        return self.Y_seq
+
+    def backward(self, dY_seq):
+        p = self.p
+        T = dY_seq[0].shape[0] * p
+        t = T // p
+        pl, m = self.plan, self.mlp
+        pl.reduce_scatter_seq_bwd(T, dY_seq, self.dY_full)
+        pl.row_bwd("mlp", T, self.dY_full, m.H, m.W2, m.Z, m.dZ, m.dW2, None)
+        pl.column_bwd("mlp", T, self.U, m.dZ, m.W1, m.dW1, None, m.dXp)
+        pl.all_gather_seq_bwd(T, m.dXp, self.dU_seq)
+        for j in range(p):
+            pl.layernorm_bwd(t, self.X_seq[j], self.gamma, self.dU_seq[j], self.mean[j * t:(j + 1) * t],
+                             self.rstd[j * t:(j + 1) * t], self.dX_seq[j], self.dgamma, self.dbeta,
+                             accumulate=j > 0)
+        return self.dX_seq
+
+    def flops(self, T: int) -> float:
+        return self.mlp.flops(T)

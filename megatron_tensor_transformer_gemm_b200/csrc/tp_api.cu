@@ -1,0 +1,900 @@
+// extern "C" entry points of libtp.so: plan management, host-side validation
+// and dispatch to the kernels. Every check happens before any launch.
+#include <cuda.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "tp_internal.h"
+
+namespace {
+thread_local char g_last_error[1024] = "";
+thread_local uint64_t g_launches = 0;
+
+__device__ unsigned g_device_status;  // per device: bit 0 = a wait timed out
+
+constexpr int kMaxDevices = 64;
+unsigned* g_status_addr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+}  // namespace
+
+namespace tpi {
+
+tp_status fail(tp_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+tp_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return TP_OK;
+  return fail(TP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+tp_status after_launch(const char* what, int launches) {
+  g_launches += static_cast<uint64_t>(launches);
+  return cuda_status(cudaGetLastError(), what);
+}
+
+tp_status device_status_word(unsigned** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_addr[dev]) {
+    void* p = nullptr;
+    tp_status s = cuda_status(cudaGetSymbolAddress(&p, g_device_status), "cudaGetSymbolAddress");
+    if (s != TP_OK) return s;
+    g_status_addr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = g_status_addr[dev];
+  return TP_OK;
+}
+
+tp_status workspace(tp_plan* plan, size_t bytes, void** out) {
+  int dev = 0;
+  tp_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != TP_OK) return s;
+  if (plan->ws && (plan->ws_bytes < bytes || plan->ws_device != dev)) {
+    // Grow (or move to another device): release the old block first. The
+    // caller's stream may still use it, so wait for the device.
+    cudaDeviceSynchronize();
+    int cur = dev;
+    if (plan->ws_device != dev) cudaSetDevice(plan->ws_device);
+    cudaFree(plan->ws);
+    if (plan->ws_device != dev) cudaSetDevice(cur);
+    plan->ws = nullptr;
+    plan->ws_bytes = 0;
+  }
+  if (!plan->ws) {
+    size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+    s = cuda_status(cudaMalloc(&plan->ws, want), "cudaMalloc(workspace)");
+    if (s != TP_OK) {
+      plan->ws = nullptr;
+      return s;
+    }
+    plan->ws_bytes = want;
+    plan->ws_device = dev;
+  }
+  *out = plan->ws;
+  return TP_OK;
+}
+
+tp_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(TP_ERR_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(TP_ERR_ALIGN, "%s (%p) is not 16-byte aligned", name, p);
+  return TP_OK;
+}
+
+tp_status check_ptrs(const void* const* arr, int n, const char* name, bool allow_null_array) {
+  if (!arr) {
+    if (allow_null_array) return TP_OK;
+    return fail(TP_ERR_ARG, "%s (pointer array) is NULL", name);
+  }
+  for (int i = 0; i < n; ++i) {
+    if (!arr[i]) return fail(TP_ERR_ARG, "%s[%d] is NULL", name, i);
+    if (!aligned16(arr[i]))
+      return fail(TP_ERR_ALIGN, "%s[%d] (%p) is not 16-byte aligned", name, i, arr[i]);
+  }
+  return TP_OK;
+}
+
+tp_status check_row_bytes(int64_t cols, tp_dtype t, const char* name) {
+  if ((cols * static_cast<int64_t>(dsize(t))) % 16 != 0)
+    return fail(TP_ERR_ALIGN, "%s: a row of %lld elements is not a multiple of 16 bytes", name,
+                static_cast<long long>(cols));
+  return TP_OK;
+}
+
+}  // namespace tpi
+
+using namespace tpi;
+
+#define TP_TRY(expr)                   \
+  do {                                 \
+    tp_status _s = (expr);             \
+    if (_s != TP_OK) return _s;        \
+  } while (0)
+
+namespace {
+
+tp_status check_plan(const tp_plan* plan) {
+  if (!plan) return fail(TP_ERR_ARG, "plan is NULL");
+  return TP_OK;
+}
+
+// Rows of W_i for the column layer and the matching width of Z_i / H_i.
+struct ColShape {
+  int n_w;   // rows of the column shard W_i (= columns of Z_i)
+  int n_h;   // columns of H_i
+  int k;     // hidden
+};
+
+tp_status col_shape(const tp_plan* plan, tp_which which, ColShape* cs) {
+  const int p = plan->p;
+  if (which == TP_MLP) {
+    if (plan->ffn <= 0) return fail(TP_ERR_ARG, "plan has no MLP (ffn = 0)");
+    int f = plan->ffn / p;
+    cs->n_h = f;
+    cs->n_w = plan->act == TP_ACT_SWIGLU ? 2 * f : f;
+  } else if (which == TP_QKV) {
+    if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention (heads = 0)");
+    cs->n_w = cs->n_h = 3 * plan->hidden / p;
+  } else {
+    return fail(TP_ERR_ARG, "projection %d is not column-parallel", static_cast<int>(which));
+  }
+  cs->k = plan->hidden;
+  return TP_OK;
+}
+
+// Input width K_i of the row shard.
+tp_status row_k(const tp_plan* plan, tp_which which, int* k) {
+  if (which == TP_MLP) {
+    if (plan->ffn <= 0) return fail(TP_ERR_ARG, "plan has no MLP (ffn = 0)");
+    *k = plan->ffn / plan->p;
+  } else if (which == TP_OUTPROJ) {
+    if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention (heads = 0)");
+    *k = plan->hidden / plan->p;
+  } else {
+    return fail(TP_ERR_ARG, "projection %d is not row-parallel", static_cast<int>(which));
+  }
+  return TP_OK;
+}
+
+tp_status check_T(int64_t T) {
+  if (T < 0) return fail(TP_ERR_ARG, "T = %lld is negative", static_cast<long long>(T));
+  if (T > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "T = %lld exceeds 2^31 - 1", (long long)T);
+  return TP_OK;
+}
+
+PtrArray to_arr(const void* const* a, int n) {
+  PtrArray r{};
+  for (int i = 0; i < n && a; ++i) r.p[i] = a[i];
+  return r;
+}
+MutPtrArray to_marr(void* const* a, int n) {
+  MutPtrArray r{};
+  for (int i = 0; i < n && a; ++i) r.p[i] = a[i];
+  return r;
+}
+
+// Launch grouped GEMMs in the plan dtype; fp32 takes EPI_STORE only.
+tp_status run_gemm(const tp_plan* plan, const GemmBatch& b, cudaStream_t st) {
+  if (plan->dtype == TP_BF16) return launch_gemm_bf16(b, st);
+  return launch_gemm_f32(b, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tp_status_string(tp_status s) {
+  switch (s) {
+    case TP_OK: return "TP_OK";
+    case TP_ERR_ARG: return "TP_ERR_ARG";
+    case TP_ERR_DIVISIBILITY: return "TP_ERR_DIVISIBILITY";
+    case TP_ERR_ALIGN: return "TP_ERR_ALIGN";
+    case TP_ERR_DTYPE: return "TP_ERR_DTYPE";
+    case TP_ERR_UNSUPPORTED: return "TP_ERR_UNSUPPORTED";
+    case TP_ERR_CUDA: return "TP_ERR_CUDA";
+    case TP_ERR_TIMEOUT: return "TP_ERR_TIMEOUT";
+    case TP_ERR_NO_DEVICE: return "TP_ERR_NO_DEVICE";
+  }
+  return "TP_ERR_UNKNOWN";
+}
+
+const char* tp_last_error(void) { return g_last_error; }
+
+uint64_t tp_launch_count(int reset) {
+  uint64_t n = g_launches;
+  if (reset) g_launches = 0;
+  return n;
+}
+
+tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, tp_act act,
+                         tp_plan** out) {
+  if (!out) return fail(TP_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (p < 1 || p > TP_MAX_SHARDS)
+    return fail(TP_ERR_ARG, "p = %d outside [1, %d]", p, TP_MAX_SHARDS);
+  if (hidden <= 0) return fail(TP_ERR_ARG, "hidden = %d must be positive", hidden);
+  if (ffn < 0 || heads < 0) return fail(TP_ERR_ARG, "ffn and heads must be >= 0");
+  if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_ERR_DTYPE, "unknown dtype %d", dtype);
+  if (act != TP_ACT_NONE && act != TP_ACT_GELU && act != TP_ACT_SWIGLU)
+    return fail(TP_ERR_ARG, "unknown activation %d", act);
+  if (hidden % p) return fail(TP_ERR_DIVISIBILITY, "hidden = %d is not divisible by p = %d", hidden, p);
+  if (heads > 0) {
+    if (heads % p)
+      return fail(TP_ERR_DIVISIBILITY, "heads = %d is not divisible by p = %d", heads, p);
+    if (hidden % heads)
+      return fail(TP_ERR_DIVISIBILITY, "hidden = %d is not divisible by heads = %d", hidden, heads);
+  }
+  if (ffn > 0) {
+    if (ffn % p) return fail(TP_ERR_DIVISIBILITY, "ffn = %d is not divisible by p = %d", ffn, p);
+    if (act == TP_ACT_SWIGLU && (2 * ffn) % (2 * p))
+      return fail(TP_ERR_DIVISIBILITY, "gate+up columns 2*ffn = %d do not split into p = %d pairs",
+                  2 * ffn, p);
+  }
+  tp_plan* plan = new (std::nothrow) tp_plan();
+  if (!plan) return fail(TP_ERR_ARG, "out of host memory");
+  plan->hidden = hidden;
+  plan->ffn = ffn;
+  plan->heads = heads;
+  plan->p = p;
+  plan->head_dim = heads > 0 ? hidden / heads : 0;
+  plan->dtype = dtype;
+  plan->act = act;
+  plan->ws = nullptr;
+  plan->ws_bytes = 0;
+  plan->ws_device = -1;
+  *out = plan;
+  return TP_OK;
+}
+
+void tp_plan_destroy(tp_plan* plan) {
+  if (!plan) return;
+  if (plan->ws) {
+    int cur = 0;
+    cudaGetDevice(&cur);
+    cudaSetDevice(plan->ws_device);
+    cudaDeviceSynchronize();
+    cudaFree(plan->ws);
+    cudaSetDevice(cur);
+    cudaGetLastError();
+  }
+  delete plan;
+}
+
+tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n) {
+  TP_TRY(check_plan(plan));
+  if (!buf || n == 0) return fail(TP_ERR_ARG, "buf is NULL or empty");
+  const int p = plan->p, h = plan->hidden, f = plan->ffn;
+  const char* act = plan->act == TP_ACT_GELU ? "gelu" : plan->act == TP_ACT_SWIGLU ? "swiglu" : "none";
+  int w = snprintf(buf, n,
+                   "tp_plan: hidden=%d ffn=%d heads=%d head_dim=%d p=%d dtype=%s act=%s\n", h, f,
+                   plan->heads, plan->head_dim, p, plan->dtype == TP_BF16 ? "bf16" : "f32", act);
+  auto add = [&](const char* fmt, auto... args) {
+    if (w >= 0 && static_cast<size_t>(w) < n) w += snprintf(buf + w, n - w, fmt, args...);
+  };
+  if (f > 0) {
+    int n1 = plan->act == TP_ACT_SWIGLU ? 2 * f / p : f / p;
+    add("  MLP column shard W1_i: [%d, %d]%s; Z_i: [T, %d]; H_i: [T, %d]\n", n1, h,
+        plan->act == TP_ACT_SWIGLU ? " = [G_i; U_i]" : "", n1, f / p);
+    add("  MLP row shard W2_i: [%d, %d]; partial P_i: [T, %d]\n", h, f / p, h);
+  }
+  if (plan->heads > 0) {
+    add("  QKV column shard: [%d, %d] = [Q_i; K_i; V_i], %d heads x %d each\n", 3 * h / p, h,
+        plan->heads / p, plan->head_dim);
+    add("  out-proj row shard Wo_i: [%d, %d]\n", h, h / p);
+  }
+  add("  sequence shard (SP): [T/%d, %d]\n", p, h);
+  return TP_OK;
+}
+
+tp_status tp_get_device_status(void* stream, int* device_status) {
+  if (!device_status) return fail(TP_ERR_ARG, "device_status is NULL");
+  unsigned* addr = nullptr;
+  TP_TRY(device_status_word(&addr));
+  unsigned v = 0;
+  TP_TRY(cuda_status(cudaStreamSynchronize(as_stream(stream)), "cudaStreamSynchronize"));
+  TP_TRY(cuda_status(cudaMemcpy(&v, addr, sizeof(v), cudaMemcpyDeviceToHost), "read status"));
+  unsigned zero = 0;
+  TP_TRY(cuda_status(cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status"));
+  *device_status = v ? TP_ERR_TIMEOUT : TP_OK;
+  return TP_OK;
+}
+
+// ------------------------------------------------------------------ sharding
+
+static tp_status shard_copy(const tp_plan* plan, tp_which which, bool column, const void* full,
+                            void* const* shards_out, const void* const* shards_in, bool to_shards,
+                            cudaStream_t st) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_ptr(full, to_shards ? "W_full" : "W_full (out)"));
+  const int p = plan->p, h = plan->hidden;
+  const void* const* shards = to_shards ? reinterpret_cast<const void* const*>(shards_out) : shards_in;
+  TP_TRY(check_ptrs(shards, p, "W_shards", false));
+  const size_t es = dsize(plan->dtype);
+  char* F = static_cast<char*>(const_cast<void*>(full));
+  // Each shard is a set of (src block -> dst block) 2-D copies.
+  auto copy = [&](const char* src, int64_t sld, char* dst, int64_t dld, int64_t rows, int64_t cols) {
+    return launch_copy_2d(src, sld, dst, dld, rows, cols, es, st);
+  };
+  if (column) {
+    if (which == TP_MLP) {
+      if (plan->ffn <= 0) return fail(TP_ERR_ARG, "plan has no MLP");
+      const int f = plan->ffn, k = f / p;
+      TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+      for (int i = 0; i < p; ++i) {
+        char* S = static_cast<char*>(const_cast<void*>(shards[i]));
+        if (plan->act == TP_ACT_SWIGLU) {
+          // [G_i; U_i]: gate rows then the matching up rows.
+          const int64_t rows[2] = {static_cast<int64_t>(i) * k, static_cast<int64_t>(f) + i * k};
+          for (int half = 0; half < 2; ++half) {
+            char* fb = F + rows[half] * h * es;
+            char* sb = S + static_cast<int64_t>(half) * k * h * es;
+            TP_TRY(to_shards ? copy(fb, h, sb, h, k, h) : copy(sb, h, fb, h, k, h));
+          }
+        } else {
+          char* fb = F + static_cast<int64_t>(i) * k * h * es;
+          TP_TRY(to_shards ? copy(fb, h, S, h, k, h) : copy(S, h, fb, h, k, h));
+        }
+      }
+      return TP_OK;
+    }
+    if (which == TP_QKV) {
+      if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention");
+      const int rows = h / p;  // heads/p * head_dim rows from each of Wq, Wk, Wv
+      TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+      for (int i = 0; i < p; ++i) {
+        char* S = static_cast<char*>(const_cast<void*>(shards[i]));
+        for (int part = 0; part < 3; ++part) {
+          char* fb = F + (static_cast<int64_t>(part) * h + static_cast<int64_t>(i) * rows) * h * es;
+          char* sb = S + static_cast<int64_t>(part) * rows * h * es;
+          TP_TRY(to_shards ? copy(fb, h, sb, h, rows, h) : copy(sb, h, fb, h, rows, h));
+        }
+      }
+      return TP_OK;
+    }
+    return fail(TP_ERR_ARG, "projection %d is not column-parallel", static_cast<int>(which));
+  }
+  int k = 0;
+  TP_TRY(row_k(plan, which, &k));
+  const int kin = k * p;
+  TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
+  for (int i = 0; i < p; ++i) {
+    char* S = static_cast<char*>(const_cast<void*>(shards[i]));
+    char* fb = F + static_cast<int64_t>(i) * k * es;
+    TP_TRY(to_shards ? copy(fb, kin, S, k, h, k) : copy(S, k, fb, kin, h, k));
+  }
+  return TP_OK;
+}
+
+tp_status tp_shard_column(const tp_plan* plan, tp_which which, const void* W_full,
+                          void* const* W_shards, void* stream) {
+  return shard_copy(plan, which, true, W_full, W_shards, nullptr, true, as_stream(stream));
+}
+tp_status tp_unshard_column(const tp_plan* plan, tp_which which, const void* const* W_shards,
+                            void* W_full, void* stream) {
+  return shard_copy(plan, which, true, W_full, nullptr, W_shards, false, as_stream(stream));
+}
+tp_status tp_shard_row(const tp_plan* plan, tp_which which, const void* W_full,
+                       void* const* W_shards, void* stream) {
+  return shard_copy(plan, which, false, W_full, W_shards, nullptr, true, as_stream(stream));
+}
+tp_status tp_unshard_row(const tp_plan* plan, tp_which which, const void* const* W_shards,
+                         void* W_full, void* stream) {
+  return shard_copy(plan, which, false, W_full, nullptr, W_shards, false, as_stream(stream));
+}
+
+tp_status tp_shard_column_bias(const tp_plan* plan, tp_which which, const void* b_full,
+                               void* const* b_shards, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_ptr(b_full, "b_full"));
+  const int p = plan->p;
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(b_shards), p, "b_shards", false));
+  const size_t es = dsize(plan->dtype);
+  cudaStream_t st = as_stream(stream);
+  const char* B = static_cast<const char*>(b_full);
+  auto copy = [&](const char* src, char* dst, int64_t n) {
+    return launch_copy_2d(src, n, dst, n, 1, n, es, st);
+  };
+  for (int i = 0; i < p; ++i) {
+    char* S = static_cast<char*>(b_shards[i]);
+    if (which == TP_MLP) {
+      if (plan->ffn <= 0) return fail(TP_ERR_ARG, "plan has no MLP");
+      const int f = plan->ffn, k = f / p;
+      if (plan->act == TP_ACT_SWIGLU) {
+        TP_TRY(copy(B + static_cast<int64_t>(i) * k * es, S, k));
+        TP_TRY(copy(B + (static_cast<int64_t>(f) + i * k) * es, S + k * es, k));
+      } else {
+        TP_TRY(copy(B + static_cast<int64_t>(i) * k * es, S, k));
+      }
+    } else if (which == TP_QKV) {
+      if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention");
+      const int h = plan->hidden, rows = h / p;
+      for (int part = 0; part < 3; ++part)
+        TP_TRY(copy(B + (static_cast<int64_t>(part) * h + static_cast<int64_t>(i) * rows) * es,
+                    S + static_cast<int64_t>(part) * rows * es, rows));
+    } else {
+      return fail(TP_ERR_ARG, "projection %d is not column-parallel", static_cast<int>(which));
+    }
+  }
+  return TP_OK;
+}
+
+// ------------------------------------------------------------------- forward
+
+tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                        const void* const* W, const void* const* bias, void* const* Z,
+                        void* const* H, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  ColShape cs{};
+  TP_TRY(col_shape(plan, which, &cs));
+  const int p = plan->p;
+  const tp_act act = which == TP_QKV ? TP_ACT_NONE : plan->act;
+  TP_TRY(check_ptr(X, "X"));
+  TP_TRY(check_ptrs(W, p, "W", false));
+  TP_TRY(check_ptrs(bias, p, "bias", true));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Z), p, "Z", true));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(H), p, "H", false));
+  TP_TRY(check_row_bytes(cs.k, plan->dtype, "hidden"));
+  TP_TRY(check_row_bytes(cs.n_h, plan->dtype, "H_i width"));
+  if (act == TP_ACT_SWIGLU && bias)
+    return fail(TP_ERR_ARG, "a column bias is not supported with SwiGLU");
+  if (act == TP_ACT_NONE && Z)
+    return fail(TP_ERR_ARG, "Z must be NULL when there is no activation");
+  if (T == 0) return TP_OK;
+  cudaStream_t st = as_stream(stream);
+
+  GemmBatch b{};
+  b.n = p;
+  b.a_mn = false;
+  b.b_mn = false;
+  b.out_f32 = plan->dtype == TP_F32;
+  for (int i = 0; i < p; ++i) {
+    GemmProblem& g = b.g[i];
+    g.M = static_cast<int>(T);
+    g.K = cs.k;
+    g.A = X;
+    g.lda = cs.k;
+    g.B = W[i];
+    g.ldb = cs.k;
+    g.bias = bias ? bias[i] : nullptr;
+  }
+  if (plan->dtype == TP_BF16) {
+    if (act == TP_ACT_NONE) {
+      b.epi = EPI_STORE;
+      for (int i = 0; i < p; ++i) {
+        b.g[i].N = cs.n_w;
+        b.g[i].D = H[i];
+        b.g[i].ldd = cs.n_h;
+      }
+    } else if (act == TP_ACT_GELU) {
+      b.epi = EPI_BIAS_GELU;
+      for (int i = 0; i < p; ++i) {
+        b.g[i].N = cs.n_w;
+        b.g[i].D = Z ? Z[i] : nullptr;
+        b.g[i].ldd = cs.n_w;
+        b.g[i].D2 = H[i];
+        b.g[i].ldd2 = cs.n_h;
+      }
+    } else {
+      b.epi = EPI_SWIGLU;
+      for (int i = 0; i < p; ++i) {
+        b.g[i].N = cs.n_h;  // gate/up pairs
+        b.g[i].nh = cs.n_h;
+        b.g[i].D = Z ? Z[i] : nullptr;
+        b.g[i].ldd = cs.n_w;
+        b.g[i].D2 = H[i];
+        b.g[i].ldd2 = cs.n_h;
+      }
+    }
+    return launch_gemm_bf16(b, st);
+  }
+  // fp32: the GEMM writes the pre-activation, an element-wise kernel the activation.
+  b.epi = EPI_STORE;
+  float* zbuf = nullptr;
+  if (act != TP_ACT_NONE && !Z) {
+    void* ws = nullptr;
+    TP_TRY(workspace(plan, static_cast<size_t>(T) * cs.n_w * sizeof(float), &ws));
+    zbuf = static_cast<float*>(ws);
+  }
+  for (int i = 0; i < p; ++i) {
+    GemmBatch one = b;
+    one.n = 1;
+    one.g[0] = b.g[i];
+    one.g[0].N = cs.n_w;
+    void* zi = act == TP_ACT_NONE ? H[i] : (Z ? Z[i] : zbuf);
+    one.g[0].D = zi;
+    one.g[0].ldd = cs.n_w;
+    TP_TRY(launch_gemm_f32(one, st));
+    if (act != TP_ACT_NONE)
+      TP_TRY(launch_act_fwd(act, static_cast<const float*>(zi), T, cs.n_h, cs.n_w,
+                            static_cast<float*>(H[i]), cs.n_h, st));
+  }
+  return TP_OK;
+}
+
+tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                             const void* const* W, void* const* P, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  int k = 0;
+  TP_TRY(row_k(plan, which, &k));
+  const int p = plan->p, h = plan->hidden;
+  TP_TRY(check_ptrs(H, p, "H", false));
+  TP_TRY(check_ptrs(W, p, "W", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(P), p, "P", false));
+  TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
+  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (T == 0) return TP_OK;
+  GemmBatch b{};
+  b.n = p;
+  b.epi = EPI_STORE;
+  b.out_f32 = plan->dtype == TP_F32;
+  for (int i = 0; i < p; ++i) {
+    GemmProblem& g = b.g[i];
+    g.M = static_cast<int>(T);
+    g.N = h;
+    g.K = k;
+    g.A = H[i];
+    g.lda = k;
+    g.B = W[i];
+    g.ldb = k;
+    g.D = P[i];
+    g.ldd = h;
+  }
+  return run_gemm(plan, b, as_stream(stream));
+}
+
+static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* const* P,
+                               const void* bias, const void* residual,
+                               const void* const* residual_seq, void* Y,
+                               void* const* Y_seq, bool scatter, cudaStream_t st) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "n = %d outside [1, %d]", n, TP_MAX_SHARDS);
+  const int h = plan->hidden;
+  TP_TRY(check_ptrs(P, n, "P", false));
+  if (bias) TP_TRY(check_ptr(bias, "bias"));
+  if (residual) TP_TRY(check_ptr(residual, "residual"));
+  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (scatter) {
+    if (T % n) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by n = %d", (long long)T, n);
+    TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Y_seq), n, "Y_seq", false));
+    TP_TRY(check_ptrs(residual_seq, n, "residual_seq", true));
+  } else {
+    TP_TRY(check_ptr(Y, "Y"));
+  }
+  if (T == 0) return TP_OK;
+  MutPtrArray out{};
+  int nout = 1;
+  if (scatter) {
+    out = to_marr(Y_seq, n);
+    nout = n;
+  } else {
+    out.p[0] = Y;
+  }
+  return launch_reduce(to_arr(P, n), n, bias, residual, to_arr(residual_seq, n),
+                       scatter && residual_seq != nullptr, out, nout, T, h, plan->dtype, st);
+}
+
+tp_status tp_reduce_partials(tp_plan* plan, int64_t T, int n, const void* const* P,
+                             const void* bias, const void* residual, void* Y, void* stream) {
+  return reduce_common(plan, T, n, P, bias, residual, nullptr, Y, nullptr, false,
+                       as_stream(stream));
+}
+
+tp_status tp_reduce_scatter_seq(tp_plan* plan, int64_t T, int n, const void* const* P,
+                                const void* bias, const void* const* residual_seq,
+                                void* const* Y_seq, void* stream) {
+  return reduce_common(plan, T, n, P, bias, nullptr, residual_seq, nullptr, Y_seq, true,
+                       as_stream(stream));
+}
+
+tp_status tp_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* const* X_seq,
+                            void* X_full, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "n = %d outside [1, %d]", n, TP_MAX_SHARDS);
+  if (T % n) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by n = %d", (long long)T, n);
+  TP_TRY(check_ptrs(X_seq, n, "X_seq", false));
+  TP_TRY(check_ptr(X_full, "X_full"));
+  TP_TRY(check_row_bytes(plan->hidden, plan->dtype, "hidden"));
+  if (T == 0) return TP_OK;
+  return launch_gather(to_arr(X_seq, n), n, X_full, T, plan->hidden, plan->dtype, as_stream(stream));
+}
+
+tp_status tp_reduce_scatter_seq_bwd(tp_plan* plan, int64_t T, int n, const void* const* dY_seq,
+                                    void* dY_full, void* stream) {
+  return tp_all_gather_seq(plan, T, n, dY_seq, dY_full, stream);
+}
+
+tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const void* const* dX_partials,
+                                void* const* dX_seq, void* stream) {
+  return tp_reduce_scatter_seq(plan, T, n, dX_partials, nullptr, nullptr, dX_seq, stream);
+}
+
+static tp_status check_ln(const tp_plan* plan) {
+  const int h = plan->hidden;
+  if (h % 8) return fail(TP_ERR_UNSUPPORTED, "LayerNorm needs hidden %% 8 == 0 (hidden = %d)", h);
+  if (h > 16384) return fail(TP_ERR_UNSUPPORTED, "LayerNorm supports hidden <= 16384 (got %d)", h);
+  return check_row_bytes(h, plan->dtype, "hidden");
+}
+
+tp_status tp_layernorm_fwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
+                           const void* beta, void* y, float* mean, float* rstd, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(rows));
+  TP_TRY(check_ptr(x, "x"));
+  TP_TRY(check_ptr(gamma, "gamma"));
+  TP_TRY(check_ptr(beta, "beta"));
+  TP_TRY(check_ptr(y, "y"));
+  TP_TRY(check_ln(plan));
+  if (rows == 0) return TP_OK;
+  PtrArray xs{};
+  xs.p[0] = x;
+  return launch_layernorm_fwd(xs, 1, rows, plan->hidden, gamma, beta, y, mean, rstd, plan->dtype,
+                              as_stream(stream));
+}
+
+tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* const* X_seq,
+                                      const void* gamma, const void* beta, void* Y_full,
+                                      float* mean, float* rstd, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "n = %d outside [1, %d]", n, TP_MAX_SHARDS);
+  if (T % n) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by n = %d", (long long)T, n);
+  TP_TRY(check_ptrs(X_seq, n, "X_seq", false));
+  TP_TRY(check_ptr(gamma, "gamma"));
+  TP_TRY(check_ptr(beta, "beta"));
+  TP_TRY(check_ptr(Y_full, "Y_full"));
+  TP_TRY(check_ln(plan));
+  if (T == 0) return TP_OK;
+  return launch_layernorm_fwd(to_arr(X_seq, n), n, T / n, plan->hidden, gamma, beta, Y_full, mean,
+                              rstd, plan->dtype, as_stream(stream));
+}
+
+tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
+                           const void* dy, const float* mean, const float* rstd, void* dx,
+                           float* dgamma, float* dbeta, int accumulate, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(rows));
+  TP_TRY(check_ptr(x, "x"));
+  TP_TRY(check_ptr(gamma, "gamma"));
+  TP_TRY(check_ptr(dy, "dy"));
+  TP_TRY(check_ptr(mean, "mean"));
+  TP_TRY(check_ptr(rstd, "rstd"));
+  TP_TRY(check_ptr(dx, "dx"));
+  TP_TRY(check_ptr(dgamma, "dgamma"));
+  TP_TRY(check_ptr(dbeta, "dbeta"));
+  TP_TRY(check_ln(plan));
+  return launch_layernorm_bwd(plan, x, gamma, dy, mean, rstd, dx, dgamma, dbeta, accumulate, rows,
+                              plan->hidden, plan->dtype, as_stream(stream));
+}
+
+tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const void* x, float* out,
+                        int accumulate, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(rows));
+  if (cols <= 0 || cols > 0x7fffffffLL) return fail(TP_ERR_ARG, "cols = %lld", (long long)cols);
+  if (rows > 0) TP_TRY(check_ptr(x, "x"));
+  TP_TRY(check_ptr(out, "out"));
+  TP_TRY(check_row_bytes(cols, plan->dtype, "cols"));
+  return launch_column_sum(plan, x, rows, cols, cols, out, accumulate, plan->dtype,
+                           as_stream(stream));
+}
+
+tp_status tp_attention_fwd(tp_plan* plan, int batch, int seq, const void* const* QKV,
+                           void* const* O, float* const* LSE, void* stream) {
+  TP_TRY(check_plan(plan));
+  if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention (heads = 0)");
+  if (batch <= 0 || seq <= 0) return fail(TP_ERR_ARG, "batch and seq must be positive");
+  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "attention runs in bf16 only");
+  const int p = plan->p;
+  TP_TRY(check_ptrs(QKV, p, "QKV", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(O), p, "O", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(LSE), p, "LSE", true));
+  if (plan->head_dim != 64 && plan->head_dim != 128)
+    return fail(TP_ERR_UNSUPPORTED, "attention supports head_dim 64 or 128 (got %d)", plan->head_dim);
+  return launch_attention_fwd(plan, batch, seq, to_arr(QKV, p), to_marr(O, p), LSE,
+                              as_stream(stream));
+}
+
+tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void* const* QKV,
+                           const void* const* O, const void* const* dO, const float* const* LSE,
+                           void* const* dQKV, void* stream) {
+  TP_TRY(check_plan(plan));
+  if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention (heads = 0)");
+  if (batch <= 0 || seq <= 0) return fail(TP_ERR_ARG, "batch and seq must be positive");
+  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "attention runs in bf16 only");
+  const int p = plan->p;
+  TP_TRY(check_ptrs(QKV, p, "QKV", false));
+  TP_TRY(check_ptrs(O, p, "O", false));
+  TP_TRY(check_ptrs(dO, p, "dO", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(LSE), p, "LSE", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dQKV), p, "dQKV", false));
+  if (plan->head_dim != 64 && plan->head_dim != 128)
+    return fail(TP_ERR_UNSUPPORTED, "attention supports head_dim 64 or 128 (got %d)", plan->head_dim);
+  return launch_attention_bwd(plan, batch, seq, to_arr(QKV, p), to_arr(O, p), to_arr(dO, p), LSE,
+                              to_marr(dQKV, p), as_stream(stream));
+}
+
+// ------------------------------------------------------------------ backward
+
+tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
+                     const void* const* H, const void* const* W, const void* const* Z,
+                     void* const* dZ, void* const* dW, float* dbias, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  int k = 0;
+  TP_TRY(row_k(plan, which, &k));
+  const int p = plan->p, h = plan->hidden;
+  const tp_act act = which == TP_OUTPROJ ? TP_ACT_NONE : plan->act;
+  const int nz = act == TP_ACT_SWIGLU ? 2 * k : k;  // width of Z_i / dZ_i
+  TP_TRY(check_ptr(dY, "dY"));
+  TP_TRY(check_ptrs(W, p, "W", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dZ), p, "dZ", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dW), p, "dW", true));
+  TP_TRY(check_ptrs(H, p, "H", dW == nullptr));
+  if (act != TP_ACT_NONE) TP_TRY(check_ptrs(Z, p, "Z", false));
+  if (dbias) TP_TRY(check_ptr(dbias, "dbias"));
+  TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
+  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (T == 0) return TP_OK;
+  cudaStream_t st = as_stream(stream);
+
+  // dH_i = dY W_i (W_i is [h, k]: (n = j, k = c) at W_i + c*k + j -> MN-major B),
+  // with the activation derivative fused in the epilogue.
+  GemmBatch b{};
+  b.n = p;
+  b.a_mn = false;
+  b.b_mn = true;
+  b.out_f32 = plan->dtype == TP_F32;
+  for (int i = 0; i < p; ++i) {
+    GemmProblem& g = b.g[i];
+    g.M = static_cast<int>(T);
+    g.N = k;
+    g.K = h;
+    g.A = dY;
+    g.lda = h;
+    g.B = W[i];
+    g.ldb = k;
+    g.D = dZ[i];
+    g.ldd = nz;
+    g.aux = act != TP_ACT_NONE ? Z[i] : nullptr;
+    g.ldaux = nz;
+    g.nh = k;
+  }
+  if (plan->dtype == TP_BF16) {
+    b.epi = act == TP_ACT_GELU ? EPI_DGELU : act == TP_ACT_SWIGLU ? EPI_DSWIGLU : EPI_STORE;
+    TP_TRY(launch_gemm_bf16(b, st));
+  } else {
+    b.epi = EPI_STORE;
+    float* dh = nullptr;
+    if (act == TP_ACT_SWIGLU) {
+      void* ws = nullptr;
+      TP_TRY(workspace(plan, static_cast<size_t>(T) * k * sizeof(float), &ws));
+      dh = static_cast<float*>(ws);
+    }
+    for (int i = 0; i < p; ++i) {
+      GemmBatch one = b;
+      one.n = 1;
+      one.g[0] = b.g[i];
+      void* dst = act == TP_ACT_SWIGLU ? static_cast<void*>(dh) : dZ[i];
+      one.g[0].D = dst;
+      one.g[0].ldd = act == TP_ACT_SWIGLU ? k : nz;
+      TP_TRY(launch_gemm_f32(one, st));
+      if (act != TP_ACT_NONE)
+        TP_TRY(launch_act_bwd(act, static_cast<const float*>(dst), T, k,
+                              static_cast<const float*>(Z[i]), nz, static_cast<float*>(dZ[i]), nz,
+                              st));
+    }
+  }
+  if (dW) {
+    // dW_i [h, k] = dY^T H_i: A(m, t) = dY[t, m] (MN-major), B(n, t) = H_i[t, n] (MN-major).
+    GemmBatch w{};
+    w.n = p;
+    w.a_mn = true;
+    w.b_mn = true;
+    w.epi = EPI_STORE;
+    w.out_f32 = plan->dtype == TP_F32;
+    for (int i = 0; i < p; ++i) {
+      GemmProblem& g = w.g[i];
+      g.M = h;
+      g.N = k;
+      g.K = static_cast<int>(T);
+      g.A = dY;
+      g.lda = h;
+      g.B = H[i];
+      g.ldb = k;
+      g.D = dW[i];
+      g.ldd = k;
+    }
+    TP_TRY(run_gemm(plan, w, st));
+  }
+  if (dbias) TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, st));
+  return TP_OK;
+}
+
+tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                        const void* const* dZ, const void* const* W, void* const* dW,
+                        float* const* dbias, void* const* dX_partials, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  ColShape cs{};
+  TP_TRY(col_shape(plan, which, &cs));
+  const int p = plan->p, h = plan->hidden;
+  const int n = cs.n_w;
+  TP_TRY(check_ptrs(dZ, p, "dZ", false));
+  TP_TRY(check_ptrs(W, p, "W", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dW), p, "dW", true));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dbias), p, "dbias", true));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX_partials), p, "dX_partials", true));
+  if (dW) TP_TRY(check_ptr(X, "X"));
+  TP_TRY(check_row_bytes(n, plan->dtype, "dZ_i width"));
+  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (T == 0) return TP_OK;
+  cudaStream_t st = as_stream(stream);
+  if (dW) {
+    // dW_i [n, h] = dZ_i^T X: A(m, t) = dZ_i[t, m] (MN-major), B(c, t) = X[t, c] (MN-major).
+    GemmBatch w{};
+    w.n = p;
+    w.a_mn = true;
+    w.b_mn = true;
+    w.epi = EPI_STORE;
+    w.out_f32 = plan->dtype == TP_F32;
+    for (int i = 0; i < p; ++i) {
+      GemmProblem& g = w.g[i];
+      g.M = n;
+      g.N = h;
+      g.K = static_cast<int>(T);
+      g.A = dZ[i];
+      g.lda = n;
+      g.B = X;
+      g.ldb = h;
+      g.D = dW[i];
+      g.ldd = h;
+    }
+    TP_TRY(run_gemm(plan, w, st));
+  }
+  if (dX_partials) {
+    // dX_i [T, h] = dZ_i W_i: A = dZ_i (K-major), B(c, j) = W_i[j, c] (MN-major).
+    GemmBatch d{};
+    d.n = p;
+    d.a_mn = false;
+    d.b_mn = true;
+    d.epi = EPI_STORE;
+    d.out_f32 = plan->dtype == TP_F32;
+    for (int i = 0; i < p; ++i) {
+      GemmProblem& g = d.g[i];
+      g.M = static_cast<int>(T);
+      g.N = h;
+      g.K = n;
+      g.A = dZ[i];
+      g.lda = n;
+      g.B = W[i];
+      g.ldb = h;
+      g.D = dX_partials[i];
+      g.ldd = h;
+    }
+    TP_TRY(run_gemm(plan, d, st));
+  }
+  if (dbias)
+    for (int i = 0; i < p; ++i)
+      TP_TRY(launch_column_sum(plan, dZ[i], T, n, n, dbias[i], 0, plan->dtype, st));
+  return TP_OK;
+}
+
+}  // extern "C"

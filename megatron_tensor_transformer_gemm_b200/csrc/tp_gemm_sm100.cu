@@ -1,0 +1,525 @@
+// Grouped, persistent bf16 GEMM on the sm_100a 5th-generation tensor cores.
+//
+// One launch computes every shard's GEMM of a column- or row-parallel layer
+// (the p shards are separate buffers on this GPU): D_g = A_g . B_g^T for
+// g < p, with a fused epilogue:
+//   EPI_STORE      D = acc (+ column bias)              QKV, row partials, grads
+//   EPI_BIAS_GELU  Z = acc + bias, H = GELU(Z)           column layer, GELU MLP
+//   EPI_SWIGLU     Z = [g|u], H = SiLU(g) * u            column layer, SwiGLU MLP
+//   EPI_DGELU      dZ = acc * GELU'(Z)                   row layer backward
+//   EPI_DSWIGLU    dZ = [acc*u*SiLU'(g) | acc*SiLU(g)]   row layer backward
+// (TP walkthrough 2kiu.com §2.1-§2.2 and §3.2; 张量并行 wiki, 两种切法.)
+//
+// Design (per CTA, one CTA per SM, persistent over a static tile schedule):
+//   warp 0      TMA producer: 128B-swizzled A and B tiles into a 4-stage ring
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> HBM
+// The 128x256 fp32 accumulator lives in TMEM (256 columns); two accumulators
+// (all 512 columns) let the epilogue of one tile overlap the MMAs of the next.
+// Operands may be K-major or MN-major (the backward GEMMs read dY^T, X^T and
+// W without transposes); SwiGLU stacks 128 gate rows and the 128 matching up
+// rows into one 256-wide B tile, so one accumulator holds both halves.
+// Every mbarrier wait is bounded (tp_device.cuh); on a time-out the CTA drains
+// its in-flight copies and MMAs, frees TMEM and returns with the status set.
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "tp_device.cuh"
+#include "tp_internal.h"
+
+namespace {
+
+using namespace tpd;
+using tpi::GemmBatch;
+using tpi::GemmProblem;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 16;
+constexpr int kThreads = 192;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int kBarBytes = 256;
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + kBarBytes;
+constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64-wide MN block of an MN-major tile
+
+struct GroupArgs {
+  int M, N, K;
+  int tiles_n;
+  int tile_begin;
+  int num_kb;
+  int nh;
+  int pad;
+  void* D;
+  int64_t ldd;
+  void* D2;
+  int64_t ldd2;
+  const void* bias;
+  const void* aux;
+  int64_t ldaux;
+};
+
+struct alignas(64) GemmParams {
+  CUtensorMap tmA[TP_MAX_SHARDS];
+  CUtensorMap tmB[TP_MAX_SHARDS];
+  GroupArgs g[TP_MAX_SHARDS];
+  int ngroups;
+  int total_tiles;
+  int a_mn;
+  int b_mn;
+  int epi;
+  int out_f32;
+  unsigned* status;
+};
+
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, int& mt, int& nt) {
+  g = 0;
+#pragma unroll 1
+  for (int i = 1; i < p.ngroups; ++i)
+    if (t >= p.g[i].tile_begin) g = i;
+  const int local = t - p.g[g].tile_begin;
+  mt = local / p.g[g].tiles_n;
+  nt = local - mt * p.g[g].tiles_n;
+}
+
+// ------------------------------------------------------------- epilogue math
+__device__ __forceinline__ void store_row_chunk_bf16(void* base, int64_t ld, int row, int col0,
+                                                     int N, const float (&v)[32]) {
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(base) + static_cast<int64_t>(row) * ld + col0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (col0 + q * 8 < N) {
+      uint4 u = make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]),
+                           pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                           pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]),
+                           pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+      *reinterpret_cast<uint4*>(dst + q * 8) = u;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_row_chunk_f32(void* base, int64_t ld, int row, int col0,
+                                                    int N, const float (&v)[32]) {
+  float* dst = static_cast<float*>(base) + static_cast<int64_t>(row) * ld + col0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (col0 + q * 4 < N)
+      *reinterpret_cast<float4*>(dst + q * 4) =
+          make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+}
+
+__device__ __forceinline__ void load_row_chunk_bf16(const void* base, int64_t ld, int row,
+                                                    int col0, int N, float (&v)[32]) {
+  const __nv_bfloat16* src =
+      static_cast<const __nv_bfloat16*>(base) + static_cast<int64_t>(row) * ld + col0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (col0 + q * 8 < N) u = *reinterpret_cast<const uint4*>(src + q * 8);
+    float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y), c = unpack_bf16x2(u.z),
+           d = unpack_bf16x2(u.w);
+    v[q * 8 + 0] = a.x; v[q * 8 + 1] = a.y; v[q * 8 + 2] = b.x; v[q * 8 + 3] = b.y;
+    v[q * 8 + 4] = c.x; v[q * 8 + 5] = c.y; v[q * 8 + 6] = d.x; v[q * 8 + 7] = d.y;
+  }
+}
+
+__device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t taddr, int row,
+                              int n0) {
+  const bool row_ok = row < ga.M;
+  if (p.epi == tpi::EPI_SWIGLU) {
+    // Accumulator columns [0,128) = gate units n0.., [128,256) = the same up units.
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tc_wait_ld();
+      const int j0 = n0 + c * 32;
+      if (row_ok && j0 < ga.N) {
+        if (ga.D) {
+          store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, g);
+          store_row_chunk_bf16(static_cast<__nv_bfloat16*>(ga.D) + ga.nh, ga.ldd, row, j0, ga.N, u);
+        }
+        float h[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
+        store_row_chunk_bf16(ga.D2, ga.ldd2, row, j0, ga.N, h);
+      }
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tc_wait_ld();
+    const int j0 = n0 + c * 32;
+    if (!row_ok || j0 >= ga.N) continue;
+    switch (p.epi) {
+      case tpi::EPI_STORE: {
+        if (ga.bias) {
+          float b[32];
+          load_row_chunk_bf16(ga.bias, 0, 0, j0, ga.N, b);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += b[i];
+        }
+        if (p.out_f32) store_row_chunk_f32(ga.D, ga.ldd, row, j0, ga.N, v);
+        else store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, v);
+        break;
+      }
+      case tpi::EPI_BIAS_GELU: {
+        if (ga.bias) {
+          float b[32];
+          load_row_chunk_bf16(ga.bias, 0, 0, j0, ga.N, b);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += b[i];
+        }
+        if (ga.D) store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+        store_row_chunk_bf16(ga.D2, ga.ldd2, row, j0, ga.N, v);
+        break;
+      }
+      case tpi::EPI_DGELU: {
+        float z[32];
+        load_row_chunk_bf16(ga.aux, ga.ldaux, row, j0, ga.N, z);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= gelu_grad_f(z[i]);
+        store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, v);
+        break;
+      }
+      case tpi::EPI_DSWIGLU: {
+        float zg[32], zu[32], dg[32];
+        load_row_chunk_bf16(ga.aux, ga.ldaux, row, j0, ga.N, zg);
+        load_row_chunk_bf16(static_cast<const __nv_bfloat16*>(ga.aux) + ga.nh, ga.ldaux, row, j0,
+                            ga.N, zu);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          dg[i] = v[i] * zu[i] * silu_grad_f(zg[i]);
+          v[i] = v[i] * silu_f(zg[i]);
+        }
+        store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, dg);
+        store_row_chunk_bf16(static_cast<__nv_bfloat16*>(ga.D) + ga.nh, ga.ldd, row, j0, ga.N, v);
+        break;
+      }
+      default:
+        break;
+    }
+  }
+}
+
+// -------------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < p.ngroups; ++g) {
+      tma_prefetch_desc(&p.tmA[g]);
+      tma_prefetch_desc(&p.tmB[g]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------- producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int last_parity[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+      int g, mt, nt;
+      decode_tile(p, t, g, mt, nt);
+      const GroupArgs& ga = p.g[g];
+      const int m0 = mt * BM;
+      const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
+      for (int kb = 0; kb < ga.num_kb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+        const int k0 = kb * BK;
+        uint8_t* a_dst = sA + stage * A_BYTES;
+        uint8_t* b_dst = sB + stage * B_BYTES;
+        if (!p.a_mn) {
+          tma_load_2d(a_dst, &p.tmA[g], &full[stage], k0, m0);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BM / 64; ++c)
+            tma_load_2d(a_dst + c * MN_BLOCK_BYTES, &p.tmA[g], &full[stage], m0 + c * 64, k0);
+        }
+        if (p.epi == tpi::EPI_SWIGLU) {
+          tma_load_3d(b_dst, &p.tmB[g], &full[stage], k0, n0, 0);
+          tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[g], &full[stage], k0, n0, 1);
+        } else if (!p.b_mn) {
+          tma_load_2d(b_dst, &p.tmB[g], &full[stage], k0, n0);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[g], &full[stage], n0 + c * 64, k0);
+        }
+        last_parity[stage] = static_cast<int>(phase);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Drain: every copy this thread issued has landed before the CTA exits.
+    for (int s = 0; s < STAGES; ++s)
+      if (last_parity[s] >= 0)
+        mbar_wait(&full[s], static_cast<uint32_t>(last_parity[s]), abort_flag, p.status);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16(BM, BN, p.a_mn != 0, p.b_mn != 0);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+      int g, mt, nt;
+      decode_tile(p, t, g, mt, nt);
+      const int num_kb = p.g[g].num_kb;
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          const uint64_t adesc =
+              p.a_mn ? smem_desc_sw128(a_base + k * (UMMA_K * 128), MN_BLOCK_BYTES, 1024)
+                     : smem_desc_sw128(a_base + k * (UMMA_K * 2), 16, 1024);
+          const uint64_t bdesc =
+              p.b_mn ? smem_desc_sw128(b_base + k * (UMMA_K * 128), MN_BLOCK_BYTES, 1024)
+                     : smem_desc_sw128(b_base + k * (UMMA_K * 2), 16, 1024);
+          tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        tc_commit(&empty[stage]);  // frees the smem stage when these MMAs finish
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      tc_commit(&tfull[acc]);  // accumulator ready for the epilogue
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    // Drain: no MMA of this CTA is in flight when TMEM is released.
+    tc_commit(drain);
+    mbar_wait(drain, 0, abort_flag, p.status);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------- epilogue
+    const int lg = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      int g, mt, nt;
+      decode_tile(p, t, g, mt, nt);
+      const GroupArgs& ga = p.g[g];
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int row = mt * BM + lg * 32 + lane;
+      const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      epilogue_tile(p, ga, taddr, row, n0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+tp_status get_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  if (!fn) return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *out = fn;
+  return TP_OK;
+}
+
+// 2-D bf16 tensor [outer, inner] (row stride ld elements), box {64, box_outer}.
+tp_status encode_2d(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_t inner,
+                    uint64_t outer, int64_t ld, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(2d, %llu x %llu, ld %lld) failed: %d",
+                     (unsigned long long)inner, (unsigned long long)outer, (long long)ld, (int)r);
+  return TP_OK;
+}
+
+// [2][nh][K] view of a SwiGLU column shard [G_i; U_i], box {64, 128, 1}.
+tp_status encode_gateup(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_t K,
+                        uint64_t nh, int64_t ld) {
+  cuuint64_t dims[3] = {K, nh, 2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(ld) * 2 * nh};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(3d gate/up) failed: %d", (int)r);
+  return TP_OK;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+namespace tpi {
+
+tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
+  if (b.n < 1 || b.n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "GEMM group count %d", b.n);
+  EncodeTiledFn enc = nullptr;
+  tp_status s = get_encoder(&enc);
+  if (s != TP_OK) return s;
+  static GemmParams p;  // host staging (large); launches copy it into the parameter buffer
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  memset(&p, 0, sizeof(p));
+  const bool swiglu = b.epi == EPI_SWIGLU;
+  const int tile_n = swiglu ? BN / 2 : BN;
+  int tiles = 0;
+  for (int i = 0; i < b.n; ++i) {
+    const GemmProblem& g = b.g[i];
+    if (g.M <= 0 || g.N <= 0 || g.K <= 0)
+      return fail(TP_ERR_ARG, "GEMM %d has an empty extent (%d x %d x %d)", i, g.M, g.N, g.K);
+    if (g.K % 8 || g.N % 8)
+      return fail(TP_ERR_ALIGN, "GEMM %d: N and K must be multiples of 8 (N=%d K=%d)", i, g.N, g.K);
+    GroupArgs& a = p.g[i];
+    a.M = g.M;
+    a.N = g.N;
+    a.K = g.K;
+    a.tiles_n = (g.N + tile_n - 1) / tile_n;
+    a.tile_begin = tiles;
+    a.num_kb = (g.K + BK - 1) / BK;
+    a.nh = g.nh;
+    a.D = g.D;
+    a.ldd = g.ldd;
+    a.D2 = g.D2;
+    a.ldd2 = g.ldd2;
+    a.bias = g.bias;
+    a.aux = g.aux;
+    a.ldaux = g.ldaux;
+    const int64_t t = static_cast<int64_t>((g.M + BM - 1) / BM) * a.tiles_n;
+    if (tiles + t > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "too many GEMM tiles");
+    tiles += static_cast<int>(t);
+    // A operand
+    if (!b.a_mn) s = encode_2d(enc, &p.tmA[i], g.A, g.K, g.M, g.lda, BM);
+    else s = encode_2d(enc, &p.tmA[i], g.A, g.M, g.K, g.lda, BK);
+    if (s != TP_OK) return s;
+    // B operand
+    if (swiglu) s = encode_gateup(enc, &p.tmB[i], g.B, g.K, g.nh, g.ldb);
+    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, g.N, g.ldb, BN);
+    else s = encode_2d(enc, &p.tmB[i], g.B, g.N, g.K, g.ldb, BK);
+    if (s != TP_OK) return s;
+  }
+  p.ngroups = b.n;
+  p.total_tiles = tiles;
+  p.a_mn = b.a_mn;
+  p.b_mn = b.b_mn;
+  p.epi = b.epi;
+  p.out_f32 = b.out_f32;
+  s = device_status_word(&p.status);
+  if (s != TP_OK) return s;
+  static bool attr_set = false;
+  if (!attr_set) {
+    s = cuda_status(cudaFuncSetAttribute(tp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES),
+                    "cudaFuncSetAttribute(gemm smem)");
+    if (s != TP_OK) return s;
+    attr_set = true;
+  }
+  const int grid = std::min(tiles, device_sms());
+  tp_gemm_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
+  return after_launch("gemm_bf16 (tcgen05)");
+}
+
+}  // namespace tpi

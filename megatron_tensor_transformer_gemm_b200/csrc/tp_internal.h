@@ -1,0 +1,131 @@
+// Internal host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "tp.h"
+
+struct tp_plan {
+  int hidden;
+  int ffn;
+  int heads;
+  int p;
+  int head_dim;
+  tp_dtype dtype;
+  tp_act act;
+  // Device scratch, allocated on first need (cudaMalloc), grown on demand.
+  void* ws;
+  size_t ws_bytes;
+  int ws_device;
+};
+
+namespace tpi {
+
+// Record `fmt` as this thread's last error and return `s`.
+tp_status fail(tp_status s, const char* fmt, ...);
+// TP_OK if e == cudaSuccess, else TP_ERR_CUDA with the CUDA error text.
+tp_status cuda_status(cudaError_t e, const char* what);
+// Check for a launch error right after a kernel launch; counts the launch.
+tp_status after_launch(const char* what, int launches = 1);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dsize(tp_dtype t) { return t == TP_BF16 ? 2 : 4; }
+
+// Device address of this device's status word (set by kernels on a timeout).
+tp_status device_status_word(unsigned** out);
+// Scratch of at least `bytes` on the current device, owned by the plan.
+tp_status workspace(tp_plan* plan, size_t bytes, void** out);
+
+// Validation helpers: each returns TP_OK or records an error.
+tp_status check_ptr(const void* p, const char* name);
+tp_status check_ptrs(const void* const* arr, int n, const char* name, bool allow_null_array);
+tp_status check_row_bytes(int64_t cols, tp_dtype t, const char* name);
+
+// Pointer arrays passed to kernels by value.
+struct PtrArray {
+  const void* p[TP_MAX_SHARDS];
+};
+struct MutPtrArray {
+  void* p[TP_MAX_SHARDS];
+};
+
+// ---------------------------------------------------------------- launchers
+// Element-wise / copy / reduction kernels (tp_reduce.cu).
+tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int64_t rows,
+                         int64_t cols, size_t esize, cudaStream_t st);
+tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
+                        const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out, int nout,
+                        int64_t T, int64_t cols, tp_dtype dt, cudaStream_t st);
+tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
+                        tp_dtype dt, cudaStream_t st);
+tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            float* out, int accumulate, tp_dtype dt, cudaStream_t st);
+
+// LayerNorm (tp_layernorm.cu).
+tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,
+                               const void* gamma, const void* beta, void* y, float* mean,
+                               float* rstd, tp_dtype dt, cudaStream_t st);
+tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, const void* dy,
+                               const float* mean, const float* rstd, void* dx, float* dgamma,
+                               float* dbeta, int accumulate, int64_t rows, int64_t cols,
+                               tp_dtype dt, cudaStream_t st);
+
+// Element-wise activation kernels for the fp32 path (tp_gemm_simt.cu).
+tp_status launch_act_fwd(tp_act act, const float* Z, int64_t T, int64_t nh, int64_t ldz, float* H,
+                         int64_t ldh, cudaStream_t st);
+tp_status launch_act_bwd(tp_act act, const float* dH, int64_t T, int64_t nh, const float* Z,
+                         int64_t ldz, float* dZ, int64_t lddz, cudaStream_t st);
+
+// ------------------------------------------------------------------- GEMM
+// One GEMM problem of a grouped launch: D[M, N] = A[M, K] . B[N, K]^T.
+// A element (m, k) lives at A + m*lda + k when !a_mn (K-major) and at
+// A + k*lda + m when a_mn (MN-major); likewise B with (n, k).
+enum Epi : int {
+  EPI_STORE = 0,       // D = acc (+ bias[n])
+  EPI_BIAS_GELU = 1,   // Z = acc + bias; D2 (H) = GELU(Z); D (Z) optional
+  EPI_SWIGLU = 2,      // gate/up pair: D (Z = [Zg|Zu]) optional, D2 (H) = SiLU(g) * u
+  EPI_DGELU = 3,       // dH = acc; D (dZ) = dH * GELU'(aux Z)
+  EPI_DSWIGLU = 4,     // dH = acc; aux = [Zg|Zu]; D (dZ) = [dH*u*SiLU'(g) | dH*SiLU(g)]
+};
+
+struct GemmProblem {
+  int M, N, K;
+  const void* A;
+  int64_t lda;
+  const void* B;
+  int64_t ldb;
+  void* D;
+  int64_t ldd;
+  void* D2;
+  int64_t ldd2;
+  const void* bias;  // [N] (plan dtype), EPI_STORE / EPI_BIAS_GELU only
+  const void* aux;   // Z for EPI_DGELU / EPI_DSWIGLU
+  int64_t ldaux;
+  int nh;            // SwiGLU: columns of each half ([Zg|Zu] offset of Zu)
+};
+
+struct GemmBatch {
+  int n;
+  GemmProblem g[TP_MAX_SHARDS];
+  bool a_mn;
+  bool b_mn;
+  int epi;
+  bool out_f32;  // D written as fp32 (bf16 otherwise)
+};
+
+// bf16 tcgen05 tensor-core path (tp_gemm_sm100.cu).
+tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st);
+// fp32 FMA path (tp_gemm_simt.cu): EPI_STORE only (activations run separately).
+tp_status launch_gemm_f32(const GemmBatch& b, cudaStream_t st);
+
+// Attention core (tp_attention.cu).
+tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const PtrArray& qkv,
+                               const MutPtrArray& o, float* const* lse, cudaStream_t st);
+tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray& qkv,
+                               const PtrArray& o, const PtrArray& dO, const float* const* lse,
+                               const MutPtrArray& dqkv, cudaStream_t st);
+
+}  // namespace tpi

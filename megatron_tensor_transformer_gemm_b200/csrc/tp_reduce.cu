@@ -1,0 +1,360 @@
+// HBM-streaming kernels of the TP path: the local all-reduce of the row-layer
+// partials (sum in fixed order + bias once + residual), its sequence-parallel
+// reduce-scatter form, the sequence all-gather, the bit-exact 2-D copies used
+// for sharding, and deterministic column sums (bias gradients).
+//
+// Layout: a thread owns one 16-byte column vector (8 bf16 or 4 fp32) of a row
+// and walks down the rows with a grid stride, so the column index, the bias
+// vector and the output pointer arithmetic are computed once per thread and
+// every warp touches 512 contiguous bytes per row: coalesced 128-bit traffic.
+#include <algorithm>
+
+#include "tp_device.cuh"
+#include "tp_internal.h"
+
+namespace {
+
+using tpi::MutPtrArray;
+using tpi::PtrArray;
+
+constexpr int kThreads = 256;
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+  }
+  return n;
+}
+
+// 16-byte vector <-> 8 (bf16) or 4 (fp32) floats.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const uint4& u, float* f) {
+    float2 a = tpd::unpack_bf16x2(u.x), b = tpd::unpack_bf16x2(u.y);
+    float2 c = tpd::unpack_bf16x2(u.z), d = tpd::unpack_bf16x2(u.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+  }
+  __device__ static uint4 store(const float* f) {
+    return make_uint4(tpd::pack_bf16x2(f[0], f[1]), tpd::pack_bf16x2(f[2], f[3]),
+                      tpd::pack_bf16x2(f[4], f[5]), tpd::pack_bf16x2(f[6], f[7]));
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+  __device__ static uint4 store(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));  // read once: evict-first
+}
+__device__ __forceinline__ uint4 ld_keep(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Finish one output vector: + bias, + residual, store (to the full output or
+// to the sequence shard that owns row rr).
+template <typename T>
+__device__ __forceinline__ void reduce_finish(float (&a)[Vec<T>::N], const float (&b)[Vec<T>::N],
+                                              int64_t rr, int64_t cols, int64_t cv,
+                                              const T* residual, const PtrArray& res_seq,
+                                              int res_is_seq, const MutPtrArray& out, int nout,
+                                              int64_t rows_per_out) {
+  constexpr int V = Vec<T>::N;
+#pragma unroll
+  for (int k = 0; k < V; ++k) a[k] += b[k];
+  T* dst;
+  const T* res = nullptr;
+  if (nout == 1) {
+    dst = static_cast<T*>(out.p[0]) + rr * cols + cv * V;
+    if (residual) res = residual + rr * cols + cv * V;
+  } else {
+    const int j = static_cast<int>(rr / rows_per_out);
+    const int64_t lr = rr - static_cast<int64_t>(j) * rows_per_out;
+    dst = static_cast<T*>(out.p[j]) + lr * cols + cv * V;
+    if (res_is_seq) res = static_cast<const T*>(res_seq.p[j]) + lr * cols + cv * V;
+  }
+  if (res) {
+    float f[V];
+    Vec<T>::load(ld_stream(res), f);
+#pragma unroll
+    for (int k = 0; k < V; ++k) a[k] += f[k];
+  }
+  *reinterpret_cast<uint4*>(dst) = Vec<T>::store(a);
+}
+
+// Y[rows] = sum_{i<n} P[i] in order 0..n-1 (fp32), + bias once, + residual.
+// out.p[0] is the full output when nout == 1, else out.p[j] holds rows
+// [j*rows_per_out, (j+1)*rows_per_out) (the sequence-parallel reduce-scatter).
+// Each thread walks two rows per step and issues all 2n loads before using
+// any, so 2n 16-byte loads per thread are in flight.
+template <typename T, int NMAX>
+__global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ PtrArray P, int n,
+                                                          const T* bias, const T* residual,
+                                                          const __grid_constant__ PtrArray res_seq,
+                                                          int res_is_seq,
+                                                          const __grid_constant__ MutPtrArray out,
+                                                          int nout, int64_t rows, int64_t vpr,
+                                                          int64_t rows_per_out) {
+  constexpr int V = Vec<T>::N;
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (cv >= vpr) return;
+  const int64_t cols = vpr * V;
+  float b[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) b[k] = 0.f;
+  if (bias) Vec<T>::load(ld_keep(bias + cv * V), b);
+  const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.y;
+  for (int64_t r = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; r < rows;
+       r += 2 * stride) {
+    const int64_t r2 = r + stride;
+    const bool two = r2 < rows;
+    const int64_t off1 = r * cols + cv * V, off2 = (two ? r2 : r) * cols + cv * V;
+    uint4 u1[NMAX], u2[NMAX];
+#pragma unroll
+    for (int i = 0; i < NMAX; ++i) {
+      if (i < n) {
+        u1[i] = ld_stream(static_cast<const T*>(P.p[i]) + off1);
+        if (two) u2[i] = ld_stream(static_cast<const T*>(P.p[i]) + off2);
+      }
+    }
+    float a1[V], a2[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) a1[k] = a2[k] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NMAX; ++i) {
+      if (i < n) {
+        float f[V];
+        Vec<T>::load(u1[i], f);
+#pragma unroll
+        for (int k = 0; k < V; ++k) a1[k] += f[k];
+        if (two) {
+          Vec<T>::load(u2[i], f);
+#pragma unroll
+          for (int k = 0; k < V; ++k) a2[k] += f[k];
+        }
+      }
+    }
+    reduce_finish<T>(a1, b, r, cols, cv, residual, res_seq, res_is_seq, out, nout, rows_per_out);
+    if (two)
+      reduce_finish<T>(a2, b, r2, cols, cv, residual, res_seq, res_is_seq, out, nout, rows_per_out);
+  }
+}
+
+// X_full rows [j*rows_per_src, ...) = src.p[j] rows; 16-byte vectors.
+__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ PtrArray src, void* dst, int64_t rows,
+                                                          int64_t vpr, int64_t rows_per_src) {
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (cv >= vpr) return;
+  const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.y;
+  uint4* D = static_cast<uint4*>(dst);
+  for (int64_t r = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; r < rows;
+       r += stride) {
+    const int j = static_cast<int>(r / rows_per_src);
+    const int64_t lr = r - static_cast<int64_t>(j) * rows_per_src;
+    const uint4 v = ld_stream(static_cast<const uint4*>(src.p[j]) + lr * vpr + cv);
+    D[r * vpr + cv] = v;
+  }
+}
+
+// Strided 2-D copy of 16-byte vectors.
+__global__ void copy2d_vec_kernel(const uint4* src, int64_t sld, uint4* dst, int64_t dld,
+                                  int64_t rows, int64_t vpr) {
+  const int64_t total = rows * vpr;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vpr, c = i - r * vpr;
+    dst[r * dld + c] = src[r * sld + c];
+  }
+}
+
+// Strided 2-D copy, element by element (any element size that is 2 or 4 bytes).
+template <typename E>
+__global__ void copy2d_elem_kernel(const E* src, int64_t sld, E* dst, int64_t dld, int64_t rows,
+                                   int64_t cols) {
+  const int64_t total = rows * cols;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / cols, c = i - r * cols;
+    dst[r * dld + c] = src[r * sld + c];
+  }
+}
+
+// Column sums, pass 1: block (32 column vectors x 8 row lanes) sums rows
+// [split*rows_per_split, ...) of 32*V columns; lanes are combined in a fixed
+// order and the result written to part[split][col].
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_pass1(const T* x, int64_t ld, int64_t rows,
+                                                    int64_t vpr, int64_t rows_per_split,
+                                                    float* part, int64_t cols) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[8][32 * V + 1];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(rows, r0 + rows_per_split);
+  float acc[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) acc[k] = 0.f;
+  if (cv < vpr) {
+    for (int64_t r = r0 + ty; r < r1; r += 8) {
+      float f[V];
+      Vec<T>::load(ld_stream(x + r * ld + cv * V), f);
+#pragma unroll
+      for (int k = 0; k < V; ++k) acc[k] += f[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < V; ++k) red[ty][tx * V + k] = acc[k];
+  __syncthreads();
+  for (int c = threadIdx.x; c < 32 * V; c += 256) {
+    float s = 0.f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) s += red[y][c];
+    const int64_t col = static_cast<int64_t>(blockIdx.x) * 32 * V + c;
+    if (col < cols) part[static_cast<int64_t>(blockIdx.y) * cols + col] = s;
+  }
+}
+
+// Column sums, pass 2: out[c] (+)= sum over splits in order.
+__global__ void colsum_pass2(const float* part, int splits, int64_t cols, float* out,
+                             int accumulate) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  float s = 0.f;
+  for (int k = 0; k < splits; ++k) s += part[static_cast<int64_t>(k) * cols + c];
+  out[c] = accumulate ? out[c] + s : s;
+}
+
+// Block shape for row-walking kernels: x covers column vectors, y rows.
+void row_walk_shape(int64_t vpr, int64_t rows, dim3* grid, dim3* block) {
+  int bx = static_cast<int>(std::min<int64_t>(kThreads, ((vpr + 31) / 32) * 32));
+  int by = kThreads / bx;
+  int gx = static_cast<int>((vpr + bx - 1) / bx);
+  int64_t want = static_cast<int64_t>(sm_count()) * 8;  // 8 blocks per SM
+  int64_t gy = std::max<int64_t>(1, want / gx);
+  gy = std::min<int64_t>(gy, (rows + by - 1) / by);
+  gy = std::min<int64_t>(gy, 65535);
+  *block = dim3(bx, by);
+  *grid = dim3(gx, static_cast<unsigned>(std::max<int64_t>(gy, 1)));
+}
+
+}  // namespace
+
+namespace tpi {
+
+tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int64_t rows,
+                         int64_t cols, size_t esize, cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return TP_OK;
+  const bool vec = aligned16(src) && aligned16(dst) && (cols * esize) % 16 == 0 &&
+                   (src_ld * esize) % 16 == 0 && (dst_ld * esize) % 16 == 0;
+  if (vec) {
+    const int64_t vpr = cols * esize / 16;
+    const int64_t total = rows * vpr;
+    int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 16LL));
+    copy2d_vec_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src),
+                                              src_ld * esize / 16, static_cast<uint4*>(dst),
+                                              dst_ld * esize / 16, rows, vpr);
+  } else {
+    const int64_t total = rows * cols;
+    int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 16LL));
+    if (esize == 2)
+      copy2d_elem_kernel<uint16_t><<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(src),
+                                                           src_ld, static_cast<uint16_t*>(dst),
+                                                           dst_ld, rows, cols);
+    else if (esize == 4)
+      copy2d_elem_kernel<uint32_t><<<blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src),
+                                                           src_ld, static_cast<uint32_t*>(dst),
+                                                           dst_ld, rows, cols);
+    else
+      return fail(TP_ERR_ARG, "copy of %zu-byte elements", esize);
+  }
+  return after_launch("copy_2d");
+}
+
+tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
+                        const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out,
+                        int nout, int64_t T, int64_t cols, tp_dtype dt, cudaStream_t st) {
+  const int V = dt == TP_BF16 ? 8 : 4;
+  const int64_t vpr = cols / V;
+  dim3 grid, block;
+  row_walk_shape(vpr, T, &grid, &block);
+  const int64_t rows_per_out = T / nout;
+  const int rs = res_seq ? 1 : 0;
+#define TP_REDUCE_LAUNCH(T, NM)                                                                  \
+  reduce_kernel<T, NM><<<grid, block, 0, st>>>(P, n, static_cast<const T*>(bias),                \
+                                               static_cast<const T*>(residual), residual_seq, rs, \
+                                               out, nout, T_rows, vpr, rows_per_out)
+  const int64_t T_rows = T;
+  if (dt == TP_BF16) {
+    if (n <= 4) TP_REDUCE_LAUNCH(__nv_bfloat16, 4);
+    else if (n <= 8) TP_REDUCE_LAUNCH(__nv_bfloat16, 8);
+    else TP_REDUCE_LAUNCH(__nv_bfloat16, TP_MAX_SHARDS);
+  } else {
+    if (n <= 4) TP_REDUCE_LAUNCH(float, 4);
+    else if (n <= 8) TP_REDUCE_LAUNCH(float, 8);
+    else TP_REDUCE_LAUNCH(float, TP_MAX_SHARDS);
+  }
+#undef TP_REDUCE_LAUNCH
+  return after_launch("reduce_partials");
+}
+
+tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
+                        tp_dtype dt, cudaStream_t st) {
+  const int64_t vpr = cols * static_cast<int64_t>(dsize(dt)) / 16;
+  dim3 grid, block;
+  row_walk_shape(vpr, T, &grid, &block);
+  gather_kernel<<<grid, block, 0, st>>>(src, dst, T, vpr, T / n);
+  return after_launch("all_gather_seq");
+}
+
+tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            float* out, int accumulate, tp_dtype dt, cudaStream_t st) {
+  const int V = dt == TP_BF16 ? 8 : 4;
+  const int64_t vpr = cols / V;
+  const int gx = static_cast<int>((vpr + 31) / 32);
+  int64_t splits = std::max<int64_t>(1, (static_cast<int64_t>(sm_count()) * 8) / gx);
+  splits = std::min<int64_t>(splits, std::max<int64_t>(1, (rows + 63) / 64));
+  splits = std::min<int64_t>(splits, 1024);
+  const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
+  splits = rows > 0 ? (rows + rps - 1) / rps : 1;
+  void* ws = nullptr;
+  tp_status s = workspace(plan, static_cast<size_t>(splits) * cols * sizeof(float), &ws);
+  if (s != TP_OK) return s;
+  float* part = static_cast<float*>(ws);
+  if (rows > 0) {
+    dim3 grid(gx, static_cast<unsigned>(splits));
+    if (dt == TP_BF16)
+      colsum_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), ld,
+                                                        rows, vpr, rps, part, cols);
+    else
+      colsum_pass1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), ld, rows, vpr, rps,
+                                                part, cols);
+    s = after_launch("column_sum/pass1");
+    if (s != TP_OK) return s;
+  } else {
+    splits = 0;
+  }
+  colsum_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+      part, static_cast<int>(splits), cols, out, accumulate);
+  return after_launch("column_sum/pass2");
+}
+
+}  // namespace tpi

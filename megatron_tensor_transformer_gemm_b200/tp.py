@@ -1,0 +1,250 @@
+"""Thin ctypes binding of libtp.so (include/tp.h).
+
+Argument marshalling only: torch tensors become device pointers and host
+pointer arrays, the current CUDA stream is passed through, and a non-OK status
+raises TPError with the library's message. Every step of the computation runs
+in the library's kernels; there is no fallback. Importing this module fails
+loudly when libtp.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtp.so")
+
+TP_F32, TP_BF16 = 0, 1
+ACTS = {"none": 0, "gelu": 1, "swiglu": 2}
+WHICH = {"mlp": 0, "qkv": 1, "outproj": 2}
+STATUS = ["TP_OK", "TP_ERR_ARG", "TP_ERR_DIVISIBILITY", "TP_ERR_ALIGN", "TP_ERR_DTYPE",
+          "TP_ERR_UNSUPPORTED", "TP_ERR_CUDA", "TP_ERR_TIMEOUT", "TP_ERR_NO_DEVICE"]
+MAX_SHARDS = 16
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, func: str, msg: str):
+        self.status = status
+        self.status_name = STATUS[status] if 0 <= status < len(STATUS) else f"status {status}"
+        super().__init__(f"{func}: {self.status_name}: {msg}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m megatron_tensor_transformer_gemm_b200.build`")
+    return ctypes.CDLL(LIB_PATH)
+
+
+lib = _load()
+
+_vp = ctypes.c_void_p
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_fp = ctypes.c_void_p  # float* (device)
+_plan_p = ctypes.c_void_p
+
+_SIGS = {
+    "tp_plan_create": (_int, [_int, _int, _int, _int, _int, _int, ctypes.POINTER(_plan_p)]),
+    "tp_plan_destroy": (None, [_plan_p]),
+    "tp_plan_describe": (_int, [_plan_p, ctypes.c_char_p, ctypes.c_size_t]),
+    "tp_status_string": (ctypes.c_char_p, [_int]),
+    "tp_last_error": (ctypes.c_char_p, []),
+    "tp_get_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
+    "tp_launch_count": (ctypes.c_uint64, [_int]),
+    "tp_shard_column": (_int, [_plan_p, _int, _vp, _vpp, _vp]),
+    "tp_unshard_column": (_int, [_plan_p, _int, _vpp, _vp, _vp]),
+    "tp_shard_row": (_int, [_plan_p, _int, _vp, _vpp, _vp]),
+    "tp_unshard_row": (_int, [_plan_p, _int, _vpp, _vp, _vp]),
+    "tp_shard_column_bias": (_int, [_plan_p, _int, _vp, _vpp, _vp]),
+    "tp_column_fwd": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_row_fwd_partial": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vpp, _vp]),
+    "tp_reduce_partials": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vp, _vp, _vp]),
+    "tp_reduce_scatter_seq": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vpp, _vpp, _vp]),
+    "tp_all_gather_seq": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vp]),
+    "tp_layernorm_fwd": (_int, [_plan_p, _i64, _vp, _vp, _vp, _vp, _fp, _fp, _vp]),
+    "tp_layernorm_all_gather_seq": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vp, _vp, _fp, _fp, _vp]),
+    "tp_attention_fwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vp]),
+    "tp_row_bwd": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _fp, _vp]),
+    "tp_column_bwd": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_reduce_scatter_seq_bwd": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vp]),
+    "tp_all_gather_seq_bwd": (_int, [_plan_p, _i64, _int, _vpp, _vpp, _vp]),
+    "tp_layernorm_bwd": (_int, [_plan_p, _i64, _vp, _vp, _vp, _fp, _fp, _vp, _fp, _fp, _int, _vp]),
+    "tp_attention_bwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_column_sum": (_int, [_plan_p, _i64, _i64, _vp, _fp, _int, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def last_error() -> str:
+    return (lib.tp_last_error() or b"").decode(errors="replace")
+
+
+def check(status: int, func: str) -> None:
+    if status != 0:
+        raise TPError(status, func, last_error())
+
+
+def launch_count(reset: bool = False) -> int:
+    return int(lib.tp_launch_count(1 if reset else 0))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libtp must be contiguous")
+    return t.data_ptr()
+
+
+def _arr(ts: Sequence | None):
+    if ts is None:
+        return None
+    vals = [_ptr(t) for t in ts]
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def _stream(stream=None) -> int | None:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    if torch.cuda.is_available():
+        return torch.cuda.current_stream().cuda_stream
+    return None
+
+
+class Plan:
+    """A tp_plan: block dimensions, shard count p, dtype and activation."""
+
+    def __init__(self, hidden: int, ffn: int, heads: int, p: int, dtype: str = "bf16",
+                 act: str = "gelu"):
+        self.hidden, self.ffn, self.heads, self.p = hidden, ffn, heads, p
+        self.dtype_name = dtype
+        self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.act = act
+        h = ctypes.c_void_p()
+        check(lib.tp_plan_create(hidden, ffn, heads, p, TP_BF16 if dtype == "bf16" else TP_F32,
+                                 ACTS[act], ctypes.byref(h)), "tp_plan_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            lib.tp_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self):
+        return self._h
+
+    def describe(self) -> str:
+        buf = ctypes.create_string_buffer(4096)
+        check(lib.tp_plan_describe(self._h, buf, len(buf)), "tp_plan_describe")
+        return buf.value.decode()
+
+    # ----------------------------------------------------------- sharding
+    def shard_column(self, which, W_full, W_shards, stream=None):
+        check(lib.tp_shard_column(self._h, WHICH[which], _ptr(W_full), _arr(W_shards), _stream(stream)),
+              "tp_shard_column")
+
+    def unshard_column(self, which, W_shards, W_full, stream=None):
+        check(lib.tp_unshard_column(self._h, WHICH[which], _arr(W_shards), _ptr(W_full), _stream(stream)),
+              "tp_unshard_column")
+
+    def shard_row(self, which, W_full, W_shards, stream=None):
+        check(lib.tp_shard_row(self._h, WHICH[which], _ptr(W_full), _arr(W_shards), _stream(stream)),
+              "tp_shard_row")
+
+    def unshard_row(self, which, W_shards, W_full, stream=None):
+        check(lib.tp_unshard_row(self._h, WHICH[which], _arr(W_shards), _ptr(W_full), _stream(stream)),
+              "tp_unshard_row")
+
+    def shard_column_bias(self, which, b_full, b_shards, stream=None):
+        check(lib.tp_shard_column_bias(self._h, WHICH[which], _ptr(b_full), _arr(b_shards),
+                                       _stream(stream)), "tp_shard_column_bias")
+
+    # ------------------------------------------------------------ forward
+    def column_fwd(self, which, T, X, W, bias, Z, H, stream=None):
+        check(lib.tp_column_fwd(self._h, WHICH[which], T, _ptr(X), _arr(W), _arr(bias), _arr(Z),
+                                _arr(H), _stream(stream)), "tp_column_fwd")
+
+    def row_fwd_partial(self, which, T, H, W, P, stream=None):
+        check(lib.tp_row_fwd_partial(self._h, WHICH[which], T, _arr(H), _arr(W), _arr(P),
+                                     _stream(stream)), "tp_row_fwd_partial")
+
+    def reduce_partials(self, T, P, bias, residual, Y, stream=None):
+        check(lib.tp_reduce_partials(self._h, T, len(P), _arr(P), _ptr(bias), _ptr(residual),
+                                     _ptr(Y), _stream(stream)), "tp_reduce_partials")
+
+    def reduce_scatter_seq(self, T, P, bias, residual_seq, Y_seq, stream=None):
+        check(lib.tp_reduce_scatter_seq(self._h, T, len(P), _arr(P), _ptr(bias), _arr(residual_seq),
+                                        _arr(Y_seq), _stream(stream)), "tp_reduce_scatter_seq")
+
+    def all_gather_seq(self, T, X_seq, X_full, stream=None):
+        check(lib.tp_all_gather_seq(self._h, T, len(X_seq), _arr(X_seq), _ptr(X_full),
+                                    _stream(stream)), "tp_all_gather_seq")
+
+    def layernorm_fwd(self, rows, x, gamma, beta, y, mean=None, rstd=None, stream=None):
+        check(lib.tp_layernorm_fwd(self._h, rows, _ptr(x), _ptr(gamma), _ptr(beta), _ptr(y),
+                                   _ptr(mean), _ptr(rstd), _stream(stream)), "tp_layernorm_fwd")
+
+    def layernorm_all_gather_seq(self, T, X_seq, gamma, beta, Y_full, mean=None, rstd=None,
+                                 stream=None):
+        check(lib.tp_layernorm_all_gather_seq(self._h, T, len(X_seq), _arr(X_seq), _ptr(gamma),
+                                              _ptr(beta), _ptr(Y_full), _ptr(mean), _ptr(rstd),
+                                              _stream(stream)), "tp_layernorm_all_gather_seq")
+
+    def attention_fwd(self, batch, seq, QKV, O, LSE=None, stream=None):
+        check(lib.tp_attention_fwd(self._h, batch, seq, _arr(QKV), _arr(O), _arr(LSE),
+                                   _stream(stream)), "tp_attention_fwd")
+
+    # ----------------------------------------------------------- backward
+    def row_bwd(self, which, T, dY, H, W, Z, dZ, dW=None, dbias=None, stream=None):
+        check(lib.tp_row_bwd(self._h, WHICH[which], T, _ptr(dY), _arr(H), _arr(W), _arr(Z),
+                             _arr(dZ), _arr(dW), _ptr(dbias), _stream(stream)), "tp_row_bwd")
+
+    def column_bwd(self, which, T, X, dZ, W, dW=None, dbias=None, dX_partials=None, stream=None):
+        check(lib.tp_column_bwd(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
+                                _arr(dbias), _arr(dX_partials), _stream(stream)), "tp_column_bwd")
+
+    def reduce_scatter_seq_bwd(self, T, dY_seq, dY_full, stream=None):
+        check(lib.tp_reduce_scatter_seq_bwd(self._h, T, len(dY_seq), _arr(dY_seq), _ptr(dY_full),
+                                            _stream(stream)), "tp_reduce_scatter_seq_bwd")
+
+    def all_gather_seq_bwd(self, T, dX_partials, dX_seq, stream=None):
+        check(lib.tp_all_gather_seq_bwd(self._h, T, len(dX_partials), _arr(dX_partials),
+                                        _arr(dX_seq), _stream(stream)), "tp_all_gather_seq_bwd")
+
+    def layernorm_bwd(self, rows, x, gamma, dy, mean, rstd, dx, dgamma, dbeta, accumulate=False,
+                      stream=None):
+        check(lib.tp_layernorm_bwd(self._h, rows, _ptr(x), _ptr(gamma), _ptr(dy), _ptr(mean),
+                                   _ptr(rstd), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
+                                   1 if accumulate else 0, _stream(stream)), "tp_layernorm_bwd")
+
+    def attention_bwd(self, batch, seq, QKV, O, dO, LSE, dQKV, stream=None):
+        check(lib.tp_attention_bwd(self._h, batch, seq, _arr(QKV), _arr(O), _arr(dO), _arr(LSE),
+                                   _arr(dQKV), _stream(stream)), "tp_attention_bwd")
+
+    def column_sum(self, rows, cols, x, out, accumulate=False, stream=None):
+        check(lib.tp_column_sum(self._h, rows, cols, _ptr(x), _ptr(out), 1 if accumulate else 0,
+                                _stream(stream)), "tp_column_sum")
+
+
+def device_status(stream=None) -> str:
+    """Read and clear the device status word ("TP_OK" or "TP_ERR_TIMEOUT")."""
+    v = ctypes.c_int(0)
+    check(lib.tp_get_device_status(_stream(stream), ctypes.byref(v)), "tp_get_device_status")
+    return STATUS[v.value]

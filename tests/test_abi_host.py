@@ -1,0 +1,156 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/tp.h declares, and rejects bad arguments on the host before any launch.
+
+Every call here either fails validation or has T = 0, so no kernel is ever
+launched (the fake pointers below are never dereferenced)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from megatron_tensor_transformer_gemm_b200 import tp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"TP_API\s+[\w\s\*]+?\b(tp_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_north_star_calls():
+    names = declared_functions()
+    for must in ["tp_plan_create", "tp_column_fwd", "tp_row_fwd_partial", "tp_reduce_partials",
+                 "tp_reduce_scatter_seq", "tp_all_gather_seq", "tp_row_bwd", "tp_column_bwd",
+                 "tp_reduce_scatter_seq_bwd", "tp_all_gather_seq_bwd"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 25
+    out = subprocess.run(["nm", "-D", "--defined-only", tp.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(tp_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(tp.lib, n)
+
+
+def _create(h, f, H, p, dtype=1, act=1):
+    ptr = ctypes.c_void_p()
+    st = tp.lib.tp_plan_create(h, f, H, p, dtype, act, ctypes.byref(ptr))
+    return st, ptr
+
+
+@pytest.mark.parametrize("args,status,needle", [
+    ((4096, 11008, 32, 0), 1, "p = 0"),
+    ((4096, 11008, 32, 17), 1, "p = 17"),
+    ((4100, 11008, 32, 8), 2, "hidden"),
+    ((4096, 11008, 20, 8), 2, "heads = 20"),      # the 20-heads-on-TP8 case of the walkthrough §6.1
+    ((4096, 11010, 32, 8), 2, "ffn"),
+    ((4096, 11008, 48, 8), 2, "hidden = 4096 is not divisible by heads = 48"),
+    ((0, 11008, 32, 8), 1, "hidden"),
+])
+def test_plan_create_divisibility(args, status, needle):
+    st, ptr = _create(*args)
+    assert st == status
+    assert not ptr.value
+    assert needle in tp.last_error()
+
+
+def test_plan_describe_prints_shard_shapes():
+    p = tp.Plan(4096, 11008, 32, 8, "bf16", "swiglu")
+    d = p.describe()
+    assert "[2752, 4096] = [G_i; U_i]" in d
+    assert "W2_i: [4096, 1376]" in d
+    assert "4 heads x 128" in d
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced (every call below stops before launch)
+
+
+def _arr(vals):
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+@pytest.fixture()
+def plan():
+    p = tp.Plan(256, 512, 4, 2, "bf16", "gelu")
+    yield p
+    p.close()
+
+
+def test_column_fwd_rejects_null_and_misaligned(plan):
+    L, h = tp.lib, plan.handle
+    W = _arr([FAKE, FAKE])
+    H = _arr([FAKE, FAKE])
+    assert L.tp_column_fwd(h, 0, 64, None, W, None, None, H, None) == 1           # X NULL
+    assert "X is NULL" in tp.last_error()
+    assert L.tp_column_fwd(h, 0, 64, FAKE + 2, W, None, None, H, None) == 3      # misaligned X
+    assert L.tp_column_fwd(h, 0, 64, FAKE, _arr([FAKE, 0]), None, None, H, None) == 1
+    assert "W[1] is NULL" in tp.last_error()
+    assert L.tp_column_fwd(h, 0, 64, FAKE, W, None, None, _arr([FAKE, FAKE + 8]), None) == 3
+    assert L.tp_column_fwd(h, 0, -1, FAKE, W, None, None, H, None) == 1           # negative T
+    assert L.tp_column_fwd(h, 1, 64, FAKE, W, None, _arr([FAKE, FAKE]), H, None) == 1  # Z with no activation
+    assert L.tp_column_fwd(h, 2, 64, FAKE, W, None, None, H, None) == 1           # outproj is not column
+    assert L.tp_column_fwd(None, 0, 64, FAKE, W, None, None, H, None) == 1
+
+
+def test_zero_tokens_is_a_no_op(plan):
+    L, h = tp.lib, plan.handle
+    W = _arr([FAKE, FAKE])
+    assert L.tp_column_fwd(h, 0, 0, FAKE, W, None, None, _arr([FAKE, FAKE]), None) == 0
+    assert L.tp_row_fwd_partial(h, 0, 0, W, W, W, None) == 0
+    assert L.tp_reduce_partials(h, 0, 2, W, None, None, FAKE, None) == 0
+    assert L.tp_all_gather_seq(h, 0, 2, W, FAKE, None) == 0
+    assert L.tp_row_bwd(h, 0, 0, FAKE, W, W, W, W, None, None, None) == 0
+    assert L.tp_column_bwd(h, 0, 0, FAKE, W, W, None, None, None, None) == 0
+
+
+def test_reduce_and_sequence_calls_validate(plan):
+    L, h = tp.lib, plan.handle
+    P = _arr([FAKE, FAKE])
+    assert L.tp_reduce_partials(h, 64, 0, P, None, None, FAKE, None) == 1          # n = 0
+    assert L.tp_reduce_partials(h, 64, 17, P, None, None, FAKE, None) == 1         # n > max
+    assert L.tp_reduce_partials(h, 64, 2, P, FAKE + 4, None, FAKE, None) == 3      # bias misaligned
+    assert L.tp_reduce_scatter_seq(h, 63, 2, P, None, None, P, None) == 2          # T % n
+    assert "not divisible" in tp.last_error()
+    assert L.tp_all_gather_seq(h, 63, 2, P, FAKE, None) == 2
+    assert L.tp_all_gather_seq(h, 64, 2, _arr([FAKE, 0]), FAKE, None) == 1
+
+
+def test_row_width_must_be_16_bytes():
+    p = tp.Plan(256, 24, 0, 2, "bf16", "gelu")  # ffn/p = 12 bf16 = 24 bytes per row
+    W = _arr([FAKE, FAKE])
+    assert tp.lib.tp_column_fwd(p.handle, 0, 64, FAKE, W, None, None, W, None) == 3
+    assert "16 bytes" in tp.last_error()
+
+
+def test_plan_without_attention_rejects_attention_calls():
+    p = tp.Plan(256, 512, 0, 2, "bf16", "gelu")
+    A = _arr([FAKE, FAKE])
+    assert tp.lib.tp_attention_fwd(p.handle, 2, 64, A, A, None, None) == 1
+    assert tp.lib.tp_column_fwd(p.handle, 1, 64, FAKE, A, None, None, A, None) == 1
+
+
+def test_swiglu_rejects_column_bias():
+    p = tp.Plan(256, 512, 0, 2, "bf16", "swiglu")
+    A = _arr([FAKE, FAKE])
+    assert tp.lib.tp_column_fwd(p.handle, 0, 64, FAKE, A, A, None, A, None) == 1
+    assert "SwiGLU" in tp.last_error()
+
+
+def test_status_strings():
+    for i, name in enumerate(tp.STATUS):
+        assert tp.lib.tp_status_string(i).decode() == name
+
+
+def test_binding_raises_tperror():
+    with pytest.raises(tp.TPError) as e:
+        tp.Plan(4096, 11008, 20, 8)
+    assert e.value.status_name == "TP_ERR_DIVISIBILITY"

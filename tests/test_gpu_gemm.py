@@ -1,0 +1,210 @@
+"""GPU parity of the tensor-core GEMM paths against the oracle's sharded steps.
+
+Shapes span several 128x256 tiles and end in ragged tails in M (tokens), N
+(output features) and K (reduction), including a final K block that is
+partly out of bounds."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import tp_synth
+from gpu_helpers import TOL_BF16, TOL_F32, assert_close, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _tp():
+    from megatron_tensor_transformer_gemm_b200 import tp
+    return tp
+
+
+def _empty(*shape, dtype=torch.bfloat16):
+    return torch.empty(*shape, dtype=dtype, device="cuda")
+
+
+def _shard_w1(W1, act, p, i):
+    return O.shard_gate_up(W1, p, i) if act == "swiglu" else O.shard_rows(W1, p, i)
+
+
+CASES = [
+    # (T, h, f, p, act, bias)
+    (300, 192, 528, 2, "gelu", True),     # M tail 44, N = 264 (tail 8), K = 3 blocks
+    (300, 200, 528, 2, "gelu", False),    # K = 200: last K block 8 wide
+    (257, 256, 272, 2, "swiglu", False),  # 136 gate/up pairs: 128 + 8
+    (129, 128, 1024, 4, "swiglu", False),
+    (513, 136, 512, 1, "none", True),
+]
+
+
+@pytest.mark.parametrize("T,h,f,p,act,bias", CASES)
+def test_column_forward(T, h, f, p, act, bias):
+    tp = _tp()
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=T + h, bias=bias, dy=False)
+    plan = tp.Plan(h, f, 0, p, "bf16", act)
+    n1 = (2 if act == "swiglu" else 1) * f // p
+    W1s = [_empty(n1, h) for _ in range(p)]
+    plan.shard_column("mlp", dev(inp.W1), W1s)
+    b1s = None
+    if bias:
+        b1s = [_empty(n1) for _ in range(p)]
+        plan.shard_column_bias("mlp", dev(inp.b1), b1s)
+    Z = [_empty(T, n1) for _ in range(p)] if act != "none" else None
+    H = [_empty(T, f // p) for _ in range(p)]
+    plan.column_fwd("mlp", T, dev(inp.X), W1s, b1s, Z, H)
+    X, W1 = O.f64(inp.X), O.f64(inp.W1)
+    for i in range(p):
+        bi = O.shard_vec(O.f64(inp.b1), p, i) if bias else None
+        rz, rh = O.column_fwd_shard(X, _shard_w1(W1, act, p, i), bi, act)
+        if Z is not None:
+            assert_close(Z[i], rz, TOL_BF16, f"Z[{i}]")
+        assert_close(H[i], rh, TOL_BF16, f"H[{i}]")
+    # Z may be omitted (inference): H unchanged
+    if Z is not None:
+        H2 = [_empty(T, f // p) for _ in range(p)]
+        plan.column_fwd("mlp", T, dev(inp.X), W1s, b1s, None, H2)
+        for i in range(p):
+            assert torch.equal(H2[i], H[i])
+
+
+@pytest.mark.parametrize("T,K,h,p", [(300, 264, 192, 2), (129, 1376, 4096, 1), (1, 64, 256, 8)])
+def test_row_forward_partials(T, K, h, p):
+    tp = _tp()
+    g = torch.Generator().manual_seed(T)
+    Hs = [torch.randn(T, K, generator=g).to(torch.bfloat16) for _ in range(p)]
+    W2 = (torch.randn(h, K * p, generator=g) * 0.02).to(torch.bfloat16)
+    plan = tp.Plan(h, K * p, 0, p, "bf16", "gelu")
+    W2s = [_empty(h, K) for _ in range(p)]
+    plan.shard_row("mlp", dev(W2), W2s)
+    P = [_empty(T, h) for _ in range(p)]
+    plan.row_fwd_partial("mlp", T, [dev(x) for x in Hs], W2s, P)
+    for i in range(p):
+        assert_close(P[i], O.row_partial(O.f64(Hs[i]), O.shard_cols(O.f64(W2), p, i)), TOL_BF16, f"P[{i}]")
+
+
+@pytest.mark.parametrize("T,h,f,p,act", [(300, 192, 528, 2, "gelu"), (257, 256, 272, 2, "swiglu"),
+                                         (200, 128, 512, 4, "none")])
+def test_row_backward(T, h, f, p, act):
+    """dZ_i = act'(dY W2_i), dW2_i = dY^T H_i, db2 = sum dY, from independent
+    inputs (Z_i, H_i drawn, not produced by the forward)."""
+    tp = _tp()
+    g = torch.Generator().manual_seed(T + 1)
+    k = f // p
+    nz = 2 * k if act == "swiglu" else k
+    dY = torch.randn(T, h, generator=g).to(torch.bfloat16)
+    W2 = (torch.randn(h, f, generator=g) * 0.05).to(torch.bfloat16)
+    Zs = [torch.randn(T, nz, generator=g).to(torch.bfloat16) for _ in range(p)]
+    Hs = [torch.randn(T, k, generator=g).to(torch.bfloat16) for _ in range(p)]
+    plan = tp.Plan(h, f, 0, p, "bf16", act)
+    W2s = [_empty(h, k) for _ in range(p)]
+    plan.shard_row("mlp", dev(W2), W2s)
+    dZ = [_empty(T, nz) for _ in range(p)]
+    dW = [_empty(h, k) for _ in range(p)]
+    db = torch.empty(h, dtype=torch.float32, device="cuda")
+    plan.row_bwd("mlp", T, dev(dY), [dev(x) for x in Hs], W2s,
+                 [dev(z) for z in Zs] if act != "none" else None, dZ, dW, db)
+    for i in range(p):
+        rdz, rdw = O.row_bwd_shard(O.f64(dY), O.f64(Hs[i]), O.shard_cols(O.f64(W2), p, i), O.f64(Zs[i]), act)
+        assert_close(dZ[i], rdz, TOL_BF16, f"dZ[{i}]")
+        assert_close(dW[i], rdw, TOL_BF16, f"dW2[{i}]")
+    assert_close(db[None, :], O.bias_grad(O.f64(dY))[None, :], 1e-4, "db2")
+
+
+@pytest.mark.parametrize("T,h,f,p,act,which", [(300, 192, 528, 2, "gelu", "mlp"),
+                                               (257, 256, 272, 2, "swiglu", "mlp"),
+                                               (130, 256, 0, 4, "none", "qkv")])
+def test_column_backward(T, h, f, p, act, which):
+    tp = _tp()
+    g = torch.Generator().manual_seed(T + 2)
+    heads = 8 if which == "qkv" else 0
+    if which == "qkv":
+        n = 3 * h // p
+        Wfull = (torch.randn(3 * h, h, generator=g) * 0.05).to(torch.bfloat16)
+    else:
+        n = (2 if act == "swiglu" else 1) * f // p
+        Wfull = (torch.randn(n * p, h, generator=g) * 0.05).to(torch.bfloat16)
+    X = torch.randn(T, h, generator=g).to(torch.bfloat16)
+    dZs = [torch.randn(T, n, generator=g).to(torch.bfloat16) for _ in range(p)]
+    plan = tp.Plan(h, f, heads, p, "bf16", act)
+    Ws = [_empty(n, h) for _ in range(p)]
+    plan.shard_column(which, dev(Wfull), Ws)
+    dW = [_empty(n, h) for _ in range(p)]
+    db = [torch.empty(n, dtype=torch.float32, device="cuda") for _ in range(p)]
+    dXp = [_empty(T, h) for _ in range(p)]
+    plan.column_bwd(which, T, dev(X), [dev(z) for z in dZs], Ws, dW, db, dXp)
+    Wf = O.f64(Wfull)
+    for i in range(p):
+        if which == "qkv":
+            Wi = O.shard_qkv(Wf, heads, p, i)
+        else:
+            Wi = _shard_w1(Wf, act, p, i)
+        rdw, rdb, rdx = O.column_bwd_shard(O.f64(X), O.f64(dZs[i]), Wi)
+        assert_close(dW[i], rdw, TOL_BF16, f"dW1[{i}]")
+        assert_close(db[i][None, :], rdb[None, :], 1e-4, f"db1[{i}]")
+        assert_close(dXp[i], rdx, TOL_BF16, f"dX partial {i}")
+
+
+@pytest.mark.parametrize("T,p", [(512, 8), (300, 2)])
+def test_qkv_column_forward_by_heads(T, p):
+    tp = _tp()
+    h, H = 512, 8
+    a = tp_synth.draw_attn_block(1, T, h, torch.bfloat16, seed=T, bias=True)
+    plan = tp.Plan(h, 0, H, p, "bf16", "none")
+    n = 3 * h // p
+    Ws = [_empty(n, h) for _ in range(p)]
+    bs = [_empty(n) for _ in range(p)]
+    plan.shard_column("qkv", dev(a.Wqkv), Ws)
+    plan.shard_column_bias("qkv", dev(a.bqkv), bs)
+    out = [_empty(T, n) for _ in range(p)]
+    plan.column_fwd("qkv", T, dev(a.X), Ws, bs, None, out)
+    full = O.linear(O.f64(a.X), O.f64(a.Wqkv), O.f64(a.bqkv))
+    d, hl = h // H, H // p
+    for i in range(p):
+        c0, c1 = i * hl * d, (i + 1) * hl * d
+        ref = np.concatenate([full[:, c0:c1], full[:, h + c0:h + c1], full[:, 2 * h + c0:2 * h + c1]], axis=1)
+        assert_close(out[i], ref, TOL_BF16, f"QKV shard {i}")
+
+
+def test_tiny_fp32_mlp_forward_backward():
+    """The tiny fp32 MLP (X 64x128, A 128x512, B 512x128, p = 2) against the
+    unsharded definition, fwd + bwd, within 1e-4."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    inp = tp_synth.draw_tiny_fp32_mlp(0)
+    m = TPMLP(128, 512, 2, "gelu", "f32", bias=True)
+    m.load_weights(dev(inp.W1), dev(inp.W2), dev(inp.b1), dev(inp.b2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    X, W1, W2, b1, b2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.b1, inp.b2, inp.dY))
+    ref = O.mlp_fwd(X, W1, b1, W2, b2, "gelu")
+    g = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, "gelu")
+    assert_close(Y, ref["Y"], TOL_F32, "Y")
+    assert_close(dX, g["dX"], TOL_F32, "dX")
+    assert_close(torch.cat(m.dW1, 0), g["dW1"], TOL_F32, "dW1")
+    assert_close(torch.cat(m.dW2, 1), g["dW2"], TOL_F32, "dW2")
+    assert_close(torch.cat(m.db1, 0)[None, :], g["db1"][None, :], TOL_F32, "db1")
+    assert_close(m.db2[None, :], g["db2"][None, :], TOL_F32, "db2")
+
+
+@pytest.mark.parametrize("act,bias", [("gelu", True), ("swiglu", False)])
+def test_bf16_mlp_end_to_end_small(act, bias):
+    """Whole sharded MLP (forward + backward through TPMLP) against the unsharded
+    definition on a small multi-tile case."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 384, 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=5, bias=bias)
+    m = TPMLP(h, f, p, act, "bf16", bias=bias)
+    m.load_weights(dev(inp.W1), dev(inp.W2), dev(inp.b1), dev(inp.b2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    b1, b2 = (O.f64(inp.b1), O.f64(inp.b2)) if bias else (None, None)
+    ref = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    g = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
+    assert_close(Y, ref["Y"], TOL_BF16, "Y")
+    assert_close(dX, g["dX"], TOL_BF16, "dX")
+    dW1 = torch.empty(W1.shape, dtype=torch.bfloat16, device="cuda")
+    m.plan.unshard_column("mlp", m.dW1, dW1)
+    assert_close(dW1, g["dW1"], TOL_BF16, "dW1")
+    dW2 = torch.empty(W2.shape, dtype=torch.bfloat16, device="cuda")
+    m.plan.unshard_row("mlp", m.dW2, dW2)
+    assert_close(dW2, g["dW2"], TOL_BF16, "dW2")
