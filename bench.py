@@ -1,0 +1,408 @@
+#!/usr/bin/env python3
+"""Benchmark of the tensor-parallel MLP hot path on B200.
+
+Default workload: the 7B-shaped SwiGLU MLP, forward + backward: hidden 4096,
+ffn 11008 (gate and up fused into column shards of 2 x 11008/p), tokens
+8 x 4096 = 32768, p = 8 shards held as separate buffers on one GPU, bf16
+storage with fp32 accumulation. One step = column GEMM (+SwiGLU) -> row GEMM
+partials -> reduce of the partials -> row backward (dSwiGLU fused) -> column
+backward -> reduce of the dX partials.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). For N > 1 (torchrun, one process per GPU) every
+rank runs its own replica of the workload (weak scaling; the path's shards all
+live on one GPU, so there is no data-path collective); time is the max over
+ranks of the device-timed region.
+
+--impl reference times the CPU oracle (fp64 numpy, the machine's host cores) on
+a bounded sample of the same workload: each step is the full forward and
+backward of the MLP on a fixed sample of token rows.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HIDDEN, FFN, TOKENS, P = 4096, 11008, 8 * 4096, 8
+METRIC = "sharded MLP fwd+bwd TFLOP/s at p shards on 1 B200; partial-reduce HBM GB/s"
+WORKLOAD = "7B-shaped SwiGLU MLP fwd+bwd: hidden 4096, ffn 11008, tokens 8x4096, p=8 shards on one GPU"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def mlp_flops(T, h, f):
+    # SwiGLU: forward 2*T*h*(2f) + 2*T*f*h; backward twice the forward.
+    return 3.0 * (2.0 * T * h * 2 * f + 2.0 * T * f * h)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle leg
+def oracle_sample(rows, seed=0):
+    """Inputs for the oracle sample: the first `rows` token rows of the same
+    seeded draw and the full weights."""
+    import torch
+    import tp_synth
+    inp = tp_synth.draw_mlp(TOKENS, HIDDEN, FFN, "swiglu", torch.bfloat16, seed=seed)
+    import oracle as O
+    return (O.f64(inp.X[:rows]), O.f64(inp.W1), O.f64(inp.W2), O.f64(inp.dY[:rows]))
+
+
+def oracle_step(X, W1, W2, dY):
+    import oracle as O
+    fwd = O.mlp_fwd(X, W1, None, W2, None, "swiglu")
+    O.mlp_bwd(X, W1, W2, fwd["Z"], fwd["H"], dY, "swiglu")
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_cpu_baseline(rows=256, seed=0):
+    X, W1, W2, dY = oracle_sample(rows, seed)
+    t0 = time.perf_counter()
+    oracle_step(X, W1, W2, dY)
+    dt = time.perf_counter() - t0
+    fl = mlp_flops(rows, HIDDEN, FFN)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"full fwd+bwd of the MLP on {rows} of the {TOKENS} token rows (fp64 numpy), "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    X, W1, W2, dY = oracle_sample(rows)
+    fl = mlp_flops(rows, HIDDEN, FFN)
+    for _ in range(args.warmup):
+        oracle_step(X, W1, W2, dY)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(X, W1, W2, dY)
+    dt = time.perf_counter() - t0
+    value = fl * args.steps / dt / 1e12
+    cores = oracle_threads()
+    sample = f"each step: full fwd+bwd of the MLP on {rows} of the {TOKENS} token rows (fp64 numpy)"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded; tp_synth)",
+           "config": {"workload": WORKLOAD, "hidden": HIDDEN, "ffn": FFN, "tokens": TOKENS, "p": P,
+                      "act": "swiglu", "sample_rows": rows},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- GPU leg
+def run_ours(args, world, rank, local):
+    import torch
+    import tp_synth
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    T = args.tokens
+    inp = tp_synth.draw_mlp(T, HIDDEN, FFN, "swiglu", torch.bfloat16, seed=rank)
+    X_h = inp.X.pin_memory()
+    dY_h = inp.dY.pin_memory()
+    m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev)
+    m.load_weights(inp.W1.to(dev), inp.W2.to(dev))
+    del inp
+    X = X_h.to(dev)
+    dY = dY_h.to(dev)
+    m.alloc(T)
+    stream = torch.cuda.current_stream()
+
+    # Per-launch CUDA events around the GEMM and reduce calls (same stream).
+    gemm_ev, red_ev = [], []
+    pl = m.plan
+    orig = {name: getattr(pl, name) for name in ("column_fwd", "row_fwd_partial", "row_bwd",
+                                                 "column_bwd", "reduce_partials")}
+
+    def timed(name, bucket):
+        fn = orig[name]
+
+        def wrapper(*a, **k):
+            if bucket is None:
+                return fn(*a, **k)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(*a, **k)
+            e1.record(stream)
+            bucket.append((name, e0, e1))
+        return wrapper
+
+    def step(instrument=False):
+        g = gemm_ev if instrument else None
+        r = red_ev if instrument else None
+        for name in ("column_fwd", "row_fwd_partial", "row_bwd", "column_bwd"):
+            setattr(pl, name, timed(name, g))
+        pl.reduce_partials = timed("reduce_partials", r)
+        m.forward(X)
+        m.backward(dY)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    tp.launch_count(reset=True)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        step(instrument=True)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    launches = tp.launch_count(reset=True)
+    barrier(world)
+    clk = clocks.stop()
+    ms_local = s0.elapsed_time(s1)
+    ms = max_over_ranks(ms_local, world)
+    flops = mlp_flops(T, HIDDEN, FFN)
+    value = world * flops * args.steps / (ms / 1e3) / 1e12
+
+    # GEMM launches (the dominant kernel): algorithmic FLOPs / summed launch time.
+    # The row_bwd and column_bwd calls each hold two GEMM launches plus a small
+    # column-sum (db) only when biases exist (not in this workload).
+    gemm_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in gemm_ev)
+    n_gemm_launches = args.steps * 6
+    gemm_tflops = flops * args.steps / (gemm_ms / 1e3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    red_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in red_ev)
+    red_bytes = 2 * (P * T * HIDDEN * 2 + T * HIDDEN * 2)  # two reduces per step
+    red_gbs = red_bytes * args.steps / (red_ms / 1e3) / 1e9
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        e2e = run_e2e(m, X_h, dY_h, T, flops, args, world, stream)
+    status = tp.device_status()
+    if rank != 0:
+        return 0
+    return report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t,
+                  red_gbs, red_bytes, e2e, launches, clk, status, orig, pl)
+
+
+def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
+    import torch
+    pl = m.plan
+    X = m.X
+    Y_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
+    dX_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(X)
+    dYd = torch.empty_like(X)
+
+    def e2e_step():
+        Xd.copy_(X_h, non_blocking=True)
+        dYd.copy_(dY_h, non_blocking=True)
+        Y = m.forward(Xd)
+        dX = m.backward(dYd)
+        Y_h.copy_(Y, non_blocking=True)
+        dX_h.copy_(dX, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * flops * args.steps / (e2e_ms / 1e3) / 1e12
+    h2d = X_h.numel() * 2 + dY_h.numel() * 2
+    d2h = Y_h.numel() * 2 + dX_h.numel() * 2
+    return {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+
+def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t, red_gbs,
+           red_bytes, e2e, launches, clk, status, orig, pl):
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(tr_path):
+        try:
+            traffic = json.load(open(tr_path)).get("bytes_per_launch")
+        except Exception:
+            traffic = None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(rows=args.cpu_rows)
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded tp_synth draws: X, dY ~ N(0,1), W ~ N(0,0.02))",
+        "config": {"workload": WORKLOAD if T == TOKENS else WORKLOAD.replace("tokens 8x4096", f"tokens {T}"),
+                   "hidden": HIDDEN, "ffn": FFN, "tokens": T, "p": P,
+                   "act": "swiglu", "global_batch": world * 8, "seq_len": 4096,
+                   "parallelism": f"{P} TP shards per GPU x {world} replicas",
+                   "l2": "inputs larger than L2 (X and dY 268 MB each); no flush"},
+        "roofline": {"bound": "tensor", "kernel": "tp_gemm_kernel (tcgen05)",
+                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak_t,
+                     "peak_kind": f"bf16 sustained ({peaks['source']})",
+                     "frac_of_burst_peak": gemm_tflops / peaks["bf16_tflops"],
+                     "launches_timed": n_gemm_launches, "traffic": traffic},
+        "reduce": {"kernel": "reduce_kernel", "achieved": red_gbs, "unit": "GB/s",
+                   "peak": peaks["hbm_gbs"], "frac": red_gbs / peaks["hbm_gbs"],
+                   "frac_of_8TBs": red_gbs / 8000.0, "bytes_per_launch": red_bytes // 2},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "device_status": status,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=8192, help="token rows in the oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="token rows per oracle step (--impl reference)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=TOKENS,
+                    help="token rows (default 8x4096; smaller values are for profiling only)")
+    ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = (1, int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        # The oracle runs on rank 0's host cores only; no GPU or process group needed.
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+    world, rank, local = dist_setup()
+    rc = run_ours(args, world, rank, local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -162,3 +162,62 @@ class SPMLP:
 
     def flops(self, T: int) -> float:
         return self.mlp.flops(T)
+
+
+class TPAttention:
+    """Attention sublayer split by whole heads over p shards on one GPU:
+    QKV column GEMM -> causal attention on local heads -> out-projection row
+    GEMM partials -> reduce (+bias once, +residual).   (TP walkthrough §3.1)"""
+
+    def __init__(self, hidden: int, heads: int, p: int, device="cuda", bias: bool = False):
+        self.h, self.H, self.p = hidden, heads, p
+        self.plan = Plan(hidden, 0, heads, p, "bf16", "none")
+        self.device = torch.device(device)
+        self.d = hidden // heads
+        self.hl = heads // p
+        n = 3 * hidden // p
+        dev = self.device
+        self.Wqkv = [_empty((n, hidden), torch.bfloat16, dev) for _ in range(p)]
+        self.Wo = [_empty((hidden, hidden // p), torch.bfloat16, dev) for _ in range(p)]
+        self.bias = bias
+        self.bqkv = [_empty((n,), torch.bfloat16, dev) for _ in range(p)] if bias else None
+        self.bo = _empty((hidden,), torch.bfloat16, dev) if bias else None
+        self._key = None
+
+    def load_weights(self, Wqkv_full, Wo_full, bqkv_full=None, bo_full=None):
+        self.plan.shard_column("qkv", Wqkv_full.contiguous(), self.Wqkv)
+        self.plan.shard_row("outproj", Wo_full.contiguous(), self.Wo)
+        if self.bias:
+            self.plan.shard_column_bias("qkv", bqkv_full.contiguous(), self.bqkv)
+            self.bo.copy_(bo_full)
+
+    def alloc(self, batch: int, seq: int):
+        if self._key == (batch, seq):
+            return
+        self._key = (batch, seq)
+        T, p, dev = batch * seq, self.p, self.device
+        n = 3 * self.h // p
+        self.QKV = [_empty((T, n), torch.bfloat16, dev) for _ in range(p)]
+        self.O = [_empty((T, self.h // p), torch.bfloat16, dev) for _ in range(p)]
+        self.LSE = [_empty((batch, self.hl, seq), torch.float32, dev) for _ in range(p)]
+        self.P = [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
+        self.Y = _empty((T, self.h), torch.bfloat16, dev)
+
+    def forward(self, X: torch.Tensor, batch: int, seq: int, residual=None, out=None):
+        self.alloc(batch, seq)
+        T = batch * seq
+        pl = self.plan
+        self.X = X
+        pl.column_fwd("qkv", T, X, self.Wqkv, self.bqkv, None, self.QKV)
+        pl.attention_fwd(batch, seq, self.QKV, self.O, self.LSE)
+        pl.row_fwd_partial("outproj", T, self.O, self.Wo, self.P)
+        Y = self.Y if out is None else out
+        pl.reduce_partials(T, self.P, self.bo, residual, Y)
+        return Y
+
+    def flops_fwd(self, batch: int, seq: int, causal: bool = True) -> float:
+        T = batch * seq
+        proj = 2.0 * T * self.h * 3 * self.h + 2.0 * T * self.h * self.h
+        pairs = seq * (seq + 1) / 2 if causal else seq * seq
+        att = 4.0 * batch * self.H * pairs * self.d
+        return proj + att

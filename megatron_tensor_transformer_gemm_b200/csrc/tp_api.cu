@@ -587,7 +587,8 @@ static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* cons
     out.p[0] = Y;
   }
   return launch_reduce(to_arr(P, n), n, bias, residual, to_arr(residual_seq, n),
-                       scatter && residual_seq != nullptr, out, nout, T, h, plan->dtype, st);
+                       scatter && residual_seq != nullptr, out, scatter, nout, T, h, plan->dtype,
+                       st);
 }
 
 tp_status tp_reduce_partials(tp_plan* plan, int64_t T, int n, const void* const* P,

@@ -471,8 +471,13 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     const GemmProblem& g = b.g[i];
     if (g.M <= 0 || g.N <= 0 || g.K <= 0)
       return fail(TP_ERR_ARG, "GEMM %d has an empty extent (%d x %d x %d)", i, g.M, g.N, g.K);
-    if (g.K % 8 || g.N % 8)
-      return fail(TP_ERR_ALIGN, "GEMM %d: N and K must be multiples of 8 (N=%d K=%d)", i, g.N, g.K);
+    // TMA needs 16-byte row strides; the epilogue stores 8-column vectors, so N
+    // and the output strides must be multiples of 8. K and M may be ragged.
+    if (g.N % 8 || g.lda % 8 || g.ldb % 8 || (g.D && g.ldd % 8) || (g.D2 && g.ldd2 % 8) ||
+        (g.aux && g.ldaux % 8))
+      return fail(TP_ERR_ALIGN, "GEMM %d: N and every leading dimension must be multiples of 8 "
+                  "(N=%d lda=%lld ldb=%lld ldd=%lld)", i, g.N, (long long)g.lda, (long long)g.ldb,
+                  (long long)g.ldd);
     GroupArgs& a = p.g[i];
     a.M = g.M;
     a.N = g.N;

@@ -57,8 +57,9 @@ struct MutPtrArray {
 tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int64_t rows,
                          int64_t cols, size_t esize, cudaStream_t st);
 tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
-                        const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out, int nout,
-                        int64_t T, int64_t cols, tp_dtype dt, cudaStream_t st);
+                        const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out,
+                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype dt,
+                        cudaStream_t st);
 tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
                         tp_dtype dt, cudaStream_t st);
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,

@@ -69,20 +69,20 @@ __device__ __forceinline__ uint4 ld_keep(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
-// Finish one output vector: + bias, + residual, store (to the full output or
-// to the sequence shard that owns row rr).
+// Finish one output vector: + bias, + residual, store (to the full output, or
+// in the reduce-scatter (scatter != 0) to the sequence shard that owns row rr).
 template <typename T>
 __device__ __forceinline__ void reduce_finish(float (&a)[Vec<T>::N], const float (&b)[Vec<T>::N],
                                               int64_t rr, int64_t cols, int64_t cv,
                                               const T* residual, const PtrArray& res_seq,
-                                              int res_is_seq, const MutPtrArray& out, int nout,
-                                              int64_t rows_per_out) {
+                                              int res_is_seq, const MutPtrArray& out,
+                                              int scatter, int64_t rows_per_out) {
   constexpr int V = Vec<T>::N;
 #pragma unroll
   for (int k = 0; k < V; ++k) a[k] += b[k];
   T* dst;
   const T* res = nullptr;
-  if (nout == 1) {
+  if (!scatter) {
     dst = static_cast<T*>(out.p[0]) + rr * cols + cv * V;
     if (residual) res = residual + rr * cols + cv * V;
   } else {
@@ -101,7 +101,7 @@ __device__ __forceinline__ void reduce_finish(float (&a)[Vec<T>::N], const float
 }
 
 // Y[rows] = sum_{i<n} P[i] in order 0..n-1 (fp32), + bias once, + residual.
-// out.p[0] is the full output when nout == 1, else out.p[j] holds rows
+// out.p[0] is the full output when scatter == 0, else out.p[j] holds rows
 // [j*rows_per_out, (j+1)*rows_per_out) (the sequence-parallel reduce-scatter).
 // Each thread walks two rows per step and issues all 2n loads before using
 // any, so 2n 16-byte loads per thread are in flight.
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
                                                           const __grid_constant__ PtrArray res_seq,
                                                           int res_is_seq,
                                                           const __grid_constant__ MutPtrArray out,
-                                                          int nout, int64_t rows, int64_t vpr,
+                                                          int scatter, int64_t rows, int64_t vpr,
                                                           int64_t rows_per_out) {
   constexpr int V = Vec<T>::N;
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -152,9 +152,9 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
         }
       }
     }
-    reduce_finish<T>(a1, b, r, cols, cv, residual, res_seq, res_is_seq, out, nout, rows_per_out);
+    reduce_finish<T>(a1, b, r, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
     if (two)
-      reduce_finish<T>(a2, b, r2, cols, cv, residual, res_seq, res_is_seq, out, nout, rows_per_out);
+      reduce_finish<T>(a2, b, r2, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
   }
 }
 
@@ -291,17 +291,19 @@ tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst
 
 tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
                         const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out,
-                        int nout, int64_t T, int64_t cols, tp_dtype dt, cudaStream_t st) {
+                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype dt,
+                        cudaStream_t st) {
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   dim3 grid, block;
   row_walk_shape(vpr, T, &grid, &block);
   const int64_t rows_per_out = T / nout;
   const int rs = res_seq ? 1 : 0;
+  const int scatter = out_is_seq ? 1 : 0;
 #define TP_REDUCE_LAUNCH(T, NM)                                                                  \
   reduce_kernel<T, NM><<<grid, block, 0, st>>>(P, n, static_cast<const T*>(bias),                \
                                                static_cast<const T*>(residual), residual_seq, rs, \
-                                               out, nout, T_rows, vpr, rows_per_out)
+                                               out, scatter, T_rows, vpr, rows_per_out)
   const int64_t T_rows = T;
   if (dt == TP_BF16) {
     if (n <= 4) TP_REDUCE_LAUNCH(__nv_bfloat16, 4);

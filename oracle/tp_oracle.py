@@ -46,7 +46,7 @@ __all__ = [
     "shard_qkv", "shard_qkv_vec", "unshard_rows", "unshard_cols",
     "column_fwd_shard", "row_partial", "reduce_partials", "reduce_scatter_seq",
     "all_gather_seq", "row_bwd_shard", "column_bwd_shard", "bias_grad",
-    "attention_fwd", "attention_bwd", "layernorm_fwd", "layernorm_bwd",
+    "attention_fwd", "attention_fwd_rows", "attention_bwd", "layernorm_fwd", "layernorm_bwd",
     "attn_sublayer_fwd", "attn_sublayer_bwd", "layer_fwd", "layer_bwd",
     "sp_mlp_fwd", "sp_mlp_bwd", "max_row_rel_err", "LN_EPS",
 ]
@@ -426,6 +426,26 @@ def attention_fwd(Q, K, V, batch, heads, causal=True):
     O = np.einsum("bhij,bhjd->bhid", P, v)
     lse = (m + np.log(L))[..., 0]
     return _merge_heads(O), lse
+
+
+def attention_fwd_rows(Q, K, V, batch, heads, rows, causal=True):
+    """attention_fwd restricted to the query positions ``rows`` (each output row
+    depends only on its own query and the keys it may see).
+
+    Returns O [len(rows), batch, heads*d] and lse [batch, heads, len(rows)].
+    """
+    q, k, v = (_split_heads(a, batch, heads) for a in (Q, K, V))
+    d = q.shape[-1]
+    rows = np.asarray(rows)
+    S = np.einsum("bhid,bhjd->bhij", q[:, :, rows], k) / math.sqrt(d)
+    if causal:
+        mask = np.arange(k.shape[2])[None, :] > rows[:, None]
+        S = np.where(mask[None, None], -np.inf, S)
+    m = S.max(axis=-1, keepdims=True)
+    E = np.exp(S - m)
+    L = E.sum(axis=-1, keepdims=True)
+    O = np.einsum("bhij,bhjd->bhid", E / L, v)
+    return _merge_heads(O), (m + np.log(L))[..., 0]
 
 
 def attention_bwd(Q, K, V, dO, batch, heads, causal=True):

@@ -1,0 +1,65 @@
+"""GPU parity of the attention core on local heads and of the attention
+sublayer (QKV by whole heads -> attention -> out-projection partials -> reduce)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import tp_synth
+from gpu_helpers import TOL_BF16, assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _tp():
+    from megatron_tensor_transformer_gemm_b200 import tp
+    return tp
+
+
+@pytest.mark.parametrize("batch,seq,heads,d,p", [
+    (2, 300, 4, 64, 2),     # 3 query tiles, ragged last tile and key block
+    (1, 256, 2, 128, 1),
+    (3, 129, 8, 64, 4),
+    (2, 512, 4, 128, 2),
+])
+def test_attention_fwd_local_heads(batch, seq, heads, d, p):
+    tp = _tp()
+    h = heads * d
+    Q, K, V, _ = tp_synth.draw_qkv_activations(batch, seq, heads, d, torch.bfloat16, seed=seq, dy=False)
+    hl = heads // p
+    plan = tp.Plan(h, 0, heads, p, "bf16", "none")
+    qkv, outs, lses = [], [], []
+    for i in range(p):
+        sl = slice(i * hl * d, (i + 1) * hl * d)
+        qkv.append(dev(torch.cat([Q[:, :, sl], K[:, :, sl], V[:, :, sl]], dim=2).reshape(seq * batch, 3 * hl * d)))
+        outs.append(torch.empty(seq * batch, hl * d, dtype=torch.bfloat16, device="cuda"))
+        lses.append(torch.empty(batch, hl, seq, dtype=torch.float32, device="cuda"))
+    plan.attention_fwd(batch, seq, qkv, outs, lses)
+    ref, ref_lse = O.attention_fwd(O.f64(Q), O.f64(K), O.f64(V), batch, heads, True)
+    got = np.concatenate([host(o).reshape(seq, batch, hl * d) for o in outs], axis=2)
+    assert_close(got.reshape(seq * batch, h), ref.reshape(seq * batch, h), TOL_BF16, "O")
+    got_lse = np.concatenate([host(l_) for l_ in lses], axis=1)
+    np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-2)
+
+
+def test_attention_block_full_size_sampled():
+    """hidden 4096, 32 heads x 128, seq 4096, batch 2, p 8 (4 heads per shard),
+    causal; QKV -> attention -> out-projection partials -> reduce + residual."""
+    from megatron_tensor_transformer_gemm_b200.block import TPAttention
+    batch, seq, h, H, p = 2, 4096, 4096, 32, 8
+    a = tp_synth.draw_attn_block(batch, seq, h, torch.bfloat16, seed=0)
+    blk = TPAttention(h, H, p)
+    blk.load_weights(dev(a.Wqkv), dev(a.Wo))
+    X = dev(a.X)
+    Y = blk.forward(X, batch, seq, residual=X)
+    rows_s = tp_synth.sample_rows(seq, 16, seed=5).numpy()
+    X64 = O.f64(a.X)
+    QKV = O.linear(X64, O.f64(a.Wqkv))
+    Qf = QKV[:, :h].reshape(seq, batch, h)
+    Kf = QKV[:, h:2 * h].reshape(seq, batch, h)
+    Vf = QKV[:, 2 * h:].reshape(seq, batch, h)
+    Osub, _ = O.attention_fwd_rows(Qf, Kf, Vf, batch, H, rows_s, True)
+    Yref = O.linear(Osub.reshape(-1, h), O.f64(a.Wo)) + X64.reshape(seq, batch, h)[rows_s].reshape(-1, h)
+    got = host(Y).reshape(seq, batch, h)[rows_s].reshape(-1, h)
+    assert_close(got, Yref, TOL_BF16, "Y sampled rows")
+    assert _tp().device_status() == "TP_OK"

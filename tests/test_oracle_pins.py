@@ -359,6 +359,16 @@ def test_attention_bwd_finite_differences(causal):
     _check_fd(dV, loss, V, n=20)
 
 
+def test_attention_rows_matches_full():
+    s, b, H, d = 9, 2, 2, 3
+    Q, K, V = randn(s, b, H * d), randn(s, b, H * d), randn(s, b, H * d)
+    full, lse = O.attention_fwd(Q, K, V, b, H, True)
+    rows = np.array([0, 4, 8])
+    part, lse_r = O.attention_fwd_rows(Q, K, V, b, H, rows, True)
+    np.testing.assert_allclose(part, full[rows], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse_r, lse[:, :, rows], rtol=1e-13, atol=1e-14)
+
+
 def test_attention_lse_definition():
     s, b, H, d = 4, 1, 1, 2
     Q, K, V = randn(s, b, d), randn(s, b, d), randn(s, b, d)

@@ -51,11 +51,11 @@ def draw_mlp(T: int, h: int, f: int, act: str, dtype: torch.dtype, seed: int = 0
              x_std: float = 1.0, w_std: float = 0.02, bias: bool = False,
              dy: bool = True) -> MLPInputs:
     """Draw X, W1, W2, b1, b2, dY in that order from one seeded generator."""
-    if act not in ("gelu", "swiglu"):
+    if act not in ("gelu", "swiglu", "none"):
         raise ValueError(f"unknown activation {act!r}")
     gen = torch.Generator().manual_seed(seed)
     X = _normal(gen, (T, h), x_std)
-    n1 = f if act == "gelu" else 2 * f
+    n1 = 2 * f if act == "swiglu" else f
     W1 = _normal(gen, (n1, h), w_std)
     W2 = _normal(gen, (h, f), w_std)
     b1 = _uniform(gen, (n1,), -0.1, 0.1) if bias else None
