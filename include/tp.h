@@ -264,6 +264,28 @@ TP_API tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void*
 TP_API tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const void* x, float* out,
                         int accumulate, void* stream);
 
+/* Column sums that allocate nothing: same result as tp_column_sum (out[c] =
+ * sum_r x[r, c] in fp32, x [rows, cols] of `dtype`, accumulate != 0 adds to
+ * out), for callers that cannot call cudaMalloc -- for example a framework
+ * whose caching allocator already owns the device memory (a cudaMalloc from
+ * the side can fail or fragment its pool), or a latency-sensitive loop that
+ * must not pay cudaMalloc's implicit device synchronisation. It takes no plan.
+ * The pages have no counterpart of this call; it exists for such callers only.
+ *   - Scratch: a fixed device array inside libtp.so of 512 Ki floats (2 MiB);
+ *     every GPU that loads the library holds it until the process exits.
+ *     cols > 524288 returns TP_ERR_UNSUPPORTED; larger column counts lower the
+ *     number of row splits (each split needs cols floats).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, so calls that overlap on the GPU (two
+ *     streams, or two host threads) race and corrupt each other's sums:
+ *     serialise them. Each call overwrites every scratch entry it reads, so
+ *     nothing from an earlier call leaks into a later one.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+TP_API tp_status tp_column_sum_static(int64_t rows, int64_t cols, tp_dtype dtype, const void* x,
+                                      float* out, int accumulate, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

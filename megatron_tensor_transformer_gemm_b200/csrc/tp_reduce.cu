@@ -8,6 +8,7 @@
 // vector and the output pointer arithmetic are computed once per thread and
 // every warp touches 512 contiguous bytes per row: coalesced 128-bit traffic.
 #include <algorithm>
+#include <mutex>
 
 #include "tp_device.cuh"
 #include "tp_internal.h"
@@ -360,3 +361,93 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
 }
 
 }  // namespace tpi
+
+// ---------------------------------------------------------------------------
+// Column sums without any allocation: the scratch of the two-pass sum lives in
+// a fixed file-scope device array instead of a cudaMalloc'd workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Capacity of the static scratch in floats (2 MiB). Every GPU that loads the
+// library holds this array until the process exits.
+constexpr int64_t kStaticScratchFloats = 512 * 1024;
+static __device__ __align__(256) float g_colsum_scratch[kStaticScratchFloats];
+
+constexpr int kMaxDevicesStatic = 64;
+float* g_scratch_addr[kMaxDevicesStatic] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_colsum_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+tp_status static_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesStatic) {
+    cudaGetLastError();
+    return tpi::fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    float* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_colsum_scratch);
+    if (e != cudaSuccess || !ptr)
+      return tpi::cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                              "cudaGetSymbolAddress(static column-sum scratch)");
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return TP_OK;
+}
+
+}  // namespace
+
+extern "C" tp_status tp_column_sum_static(int64_t rows, int64_t cols, tp_dtype dtype,
+                                          const void* x, float* out, int accumulate,
+                                          void* stream) {
+  using namespace tpi;
+  if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_ERR_DTYPE, "unknown dtype %d", dtype);
+  if (rows < 0 || rows > 0x7fffffffLL) return fail(TP_ERR_ARG, "rows = %lld", (long long)rows);
+  if (cols <= 0 || cols > 0x7fffffffLL) return fail(TP_ERR_ARG, "cols = %lld", (long long)cols);
+  if (cols > kStaticScratchFloats)
+    return fail(TP_ERR_UNSUPPORTED,
+                "cols = %lld exceeds the static scratch of tp_column_sum_static (%lld columns max)",
+                (long long)cols, (long long)kStaticScratchFloats);
+  if (rows > 0) {
+    tp_status s = check_ptr(x, "x");
+    if (s != TP_OK) return s;
+  }
+  tp_status s = check_ptr(out, "out");
+  if (s != TP_OK) return s;
+  s = check_row_bytes(cols, dtype, "cols");
+  if (s != TP_OK) return s;
+  float* part = nullptr;
+  s = static_scratch(&part);
+  if (s != TP_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int V = dtype == TP_BF16 ? 8 : 4;
+  const int64_t vpr = cols / V;
+  const int gx = static_cast<int>((vpr + 31) / 32);
+  // Same split heuristic as the workspace version, capped so that
+  // splits x cols floats fit in the static scratch.
+  int64_t splits = std::max<int64_t>(1, (static_cast<int64_t>(sm_count()) * 8) / gx);
+  splits = std::min<int64_t>(splits, std::max<int64_t>(1, (rows + 63) / 64));
+  splits = std::min<int64_t>(splits, kStaticScratchFloats / cols);
+  const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
+  splits = rows > 0 ? (rows + rps - 1) / rps : 0;
+  if (rows > 0) {
+    // Pass 1 writes every scratch entry pass 2 reads (splits x cols), so
+    // nothing left from an earlier call is ever read.
+    dim3 grid(gx, static_cast<unsigned>(splits));
+    if (dtype == TP_BF16)
+      colsum_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                        cols, rows, vpr, rps, part, cols);
+    else
+      colsum_pass1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), cols, rows, vpr,
+                                                rps, part, cols);
+    s = after_launch("column_sum_static/pass1");
+    if (s != TP_OK) return s;
+  }
+  colsum_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+      part, static_cast<int>(splits), cols, out, accumulate);
+  return after_launch("column_sum_static/pass2");
+}

@@ -76,6 +76,7 @@ _SIGS = {
     "tp_layernorm_bwd": (_int, [_plan_p, _i64, _vp, _vp, _vp, _fp, _fp, _vp, _fp, _fp, _int, _vp]),
     "tp_attention_bwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_column_sum": (_int, [_plan_p, _i64, _i64, _vp, _fp, _int, _vp]),
+    "tp_column_sum_static": (_int, [_i64, _i64, _int, _vp, _fp, _int, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -241,6 +242,14 @@ class Plan:
     def column_sum(self, rows, cols, x, out, accumulate=False, stream=None):
         check(lib.tp_column_sum(self._h, rows, cols, _ptr(x), _ptr(out), 1 if accumulate else 0,
                                 _stream(stream)), "tp_column_sum")
+
+
+def column_sum_static(rows, cols, x, out, accumulate=False, stream=None):
+    """tp_column_sum_static: column sums with the library's fixed device scratch
+    (no allocation); see include/tp.h for its limits."""
+    dt = TP_BF16 if x.dtype == torch.bfloat16 else TP_F32
+    check(lib.tp_column_sum_static(rows, cols, dt, _ptr(x), _ptr(out), 1 if accumulate else 0,
+                                   _stream(stream)), "tp_column_sum_static")
 
 
 def device_status(stream=None) -> str:
