@@ -5,8 +5,15 @@ Default workload: the 7B-shaped SwiGLU MLP, forward + backward: hidden 4096,
 ffn 11008 (gate and up fused into column shards of 2 x 11008/p), tokens
 8 x 4096 = 32768, p = 8 shards held as separate buffers on one GPU, bf16
 storage with fp32 accumulation. One step = column GEMM (+SwiGLU) -> row GEMM
-partials -> reduce of the partials -> row backward (dSwiGLU fused) -> column
-backward -> reduce of the dX partials.
+-> sum over shards (+bias once) -> row backward (dSwiGLU fused) -> column
+backward -> sum of the dX partials.
+
+--variant fused (default): the sums over shards happen inside the row GEMM and
+the column-backward dX GEMM (one TMEM accumulator over all shards' K slices).
+--variant partials: the row GEMM writes p full-shape partials and the reduce
+kernel sums them (and likewise for dX). In both variants the standalone
+partial-reduce kernel's HBM GB/s is reported: measured inside the step for
+"partials", and in its own timed loop over the same partial sizes for "fused".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -129,13 +136,22 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank float over all ranks (device tensor for NCCL, host for gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(flops_per_step, steps, ms_local, world):
+    """Whole-job throughput (TFLOP/s) of N weak-scaling replicas: every rank
+    processes the same work, and the job takes as long as the slowest rank."""
+    ms = max_over_ranks(ms_local, world)
+    return world * flops_per_step * steps / (ms / 1e3) / 1e12, ms
 
 
 # --------------------------------------------------------------- CPU oracle leg
@@ -216,7 +232,8 @@ def run_ours(args, world, rank, local):
     inp = tp_synth.draw_mlp(T, HIDDEN, FFN, "swiglu", torch.bfloat16, seed=rank)
     X_h = inp.X.pin_memory()
     dY_h = inp.dY.pin_memory()
-    m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev)
+    fused = args.variant == "fused"
+    m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev, fused=fused)
     m.load_weights(inp.W1.to(dev), inp.W2.to(dev))
     del inp
     X = X_h.to(dev)
@@ -227,8 +244,9 @@ def run_ours(args, world, rank, local):
     # Per-launch CUDA events around the GEMM and reduce calls (same stream).
     gemm_ev, red_ev = [], []
     pl = m.plan
-    orig = {name: getattr(pl, name) for name in ("column_fwd", "row_fwd_partial", "row_bwd",
-                                                 "column_bwd", "reduce_partials")}
+    gemm_calls = ("column_fwd", "row_fwd_partial", "row_bwd", "column_bwd", "row_fwd_reduce",
+                  "column_bwd_reduce")
+    orig = {name: getattr(pl, name) for name in gemm_calls + ("reduce_partials",)}
 
     def timed(name, bucket):
         fn = orig[name]
@@ -247,7 +265,7 @@ def run_ours(args, world, rank, local):
     def step(instrument=False):
         g = gemm_ev if instrument else None
         r = red_ev if instrument else None
-        for name in ("column_fwd", "row_fwd_partial", "row_bwd", "column_bwd"):
+        for name in gemm_calls:
             setattr(pl, name, timed(name, g))
         pl.reduce_partials = timed("reduce_partials", r)
         m.forward(X)
@@ -275,9 +293,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     clk = clocks.stop()
     ms_local = s0.elapsed_time(s1)
-    ms = max_over_ranks(ms_local, world)
     flops = mlp_flops(T, HIDDEN, FFN)
-    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    value, ms = aggregate(flops, args.steps, ms_local, world)
 
     # GEMM launches (the dominant kernel): algorithmic FLOPs / summed launch time.
     # The row_bwd and column_bwd calls each hold two GEMM launches plus a small
@@ -286,9 +303,15 @@ def run_ours(args, world, rank, local):
     n_gemm_launches = args.steps * 6
     gemm_tflops = flops * args.steps / (gemm_ms / 1e3) / 1e12
     peak_t = peaks["bf16_tflops_sustained"]
-    red_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in red_ev)
-    red_bytes = 2 * (P * T * HIDDEN * 2 + T * HIDDEN * 2)  # two reduces per step
-    red_gbs = red_bytes * args.steps / (red_ms / 1e3) / 1e9
+    red_bytes_launch = P * T * HIDDEN * 2 + T * HIDDEN * 2
+    if red_ev:
+        red_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in red_ev)
+        red_gbs = red_bytes_launch * len(red_ev) / (red_ms / 1e3) / 1e9
+        red_where = "inside the timed steps (2 per step)"
+    else:
+        red_gbs = time_standalone_reduce(pl, T, args.steps, stream)
+        red_where = "standalone loop over the same partial sizes (p=8 x [T, 4096] bf16)"
+    red_bytes = red_bytes_launch
 
     # ---- end-to-end through the public API with host buffers
     e2e = None
@@ -298,7 +321,30 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return 0
     return report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t,
-                  red_gbs, red_bytes, e2e, launches, clk, status, orig, pl)
+                  red_gbs, red_bytes, e2e, launches, clk, status, red_where)
+
+
+def time_standalone_reduce(pl, T, steps, stream):
+    """HBM GB/s of tp_reduce_partials summing p = 8 bf16 partials [T, 4096]."""
+    import torch
+    Pt = [torch.randn(T, HIDDEN, device="cuda", dtype=torch.bfloat16) for _ in range(P)]
+    Y = torch.empty(T, HIDDEN, device="cuda", dtype=torch.bfloat16)
+    for _ in range(3):
+        pl.reduce_partials(T, Pt, None, None, Y)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n = max(2 * steps, 4)
+    e0.record(stream)
+    for _ in range(n):
+        pl.reduce_partials(T, Pt, None, None, Y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    nbytes = (P + 1) * T * HIDDEN * 2
+    gbs = nbytes * n / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del Pt, Y
+    torch.cuda.empty_cache()
+    return gbs
 
 
 def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
@@ -328,8 +374,7 @@ def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * flops * args.steps / (e2e_ms / 1e3) / 1e12
+    e2e_value, e2e_ms = aggregate(flops, args.steps, e0.elapsed_time(e1), world)
     h2d = X_h.numel() * 2 + dY_h.numel() * 2
     d2h = Y_h.numel() * 2 + dX_h.numel() * 2
     return {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -337,7 +382,7 @@ def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
 
 
 def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t, red_gbs,
-           red_bytes, e2e, launches, clk, status, orig, pl):
+           red_bytes, e2e, launches, clk, status, red_where):
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(tr_path):
@@ -357,6 +402,7 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
                    "hidden": HIDDEN, "ffn": FFN, "tokens": T, "p": P,
                    "act": "swiglu", "global_batch": world * 8, "seq_len": 4096,
                    "parallelism": f"{P} TP shards per GPU x {world} replicas",
+                   "variant": args.variant,
                    "l2": "inputs larger than L2 (X and dY 268 MB each); no flush"},
         "roofline": {"bound": "tensor", "kernel": "tp_gemm_kernel (tcgen05)",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
@@ -366,7 +412,9 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
                      "launches_timed": n_gemm_launches, "traffic": traffic},
         "reduce": {"kernel": "reduce_kernel", "achieved": red_gbs, "unit": "GB/s",
                    "peak": peaks["hbm_gbs"], "frac": red_gbs / peaks["hbm_gbs"],
-                   "frac_of_8TBs": red_gbs / 8000.0, "bytes_per_launch": red_bytes // 2},
+                   "peak_kind": f"HBM copy ({peaks['source']})",
+                   "frac_of_8TBs": red_gbs / 8000.0, "bytes_per_launch": red_bytes,
+                   "measured": red_where},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
@@ -380,7 +428,7 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=8192, help="token rows in the oracle baseline sample")
@@ -389,6 +437,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=TOKENS,
                     help="token rows (default 8x4096; smaller values are for profiling only)")
     ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--variant", choices=["fused", "partials"], default="fused",
+                    help="sum over shards inside the GEMMs (fused) or via p partials + reduce")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -167,6 +167,25 @@ TP_API tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const v
 TP_API tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
                              const void* const* W, void* const* P, void* stream);
 
+/* Row-parallel GEMM with the sum over shards fused into it: one launch in
+ * which every output tile accumulates all p shards' K-slices in the same TMEM
+ * accumulator, Y = sum_i H[i] W[i]^T (fp32) + bias once (NULL ok) + residual
+ * (NULL ok), rounded once. Same result as tp_row_fwd_partial followed by
+ * tp_reduce_partials (TP-blog §2.2, TP-basics: bias once after the sum)
+ * without writing or re-reading the p partials. Y [T, hidden]; Y must not
+ * alias an input. bf16 plans only. */
+TP_API tp_status tp_row_fwd_reduce(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                                   const void* const* W, const void* bias, const void* residual,
+                                   void* Y, void* stream);
+
+/* The same with the sequence-parallel reduce-scatter fused in (TP-blog §4.3):
+ * rows [j*T/p, (j+1)*T/p) of the sum (+ bias, + residual_seq[j]) go to
+ * Y_seq[j] [T/p, hidden]. residual_seq may be NULL. */
+TP_API tp_status tp_row_fwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_t T,
+                                               const void* const* H, const void* const* W,
+                                               const void* bias, const void* const* residual_seq,
+                                               void* const* Y_seq, void* stream);
+
 /* The all-reduce of the row layer, done locally: Y = sum_{i<n} P[i] (fp32, in
  * order 0..n-1), then + bias once (NULL ok), then + residual (NULL ok).
  * [TP-blog] §2.2, [TP-basics] (bias once, after the sum). P[i], residual, Y
@@ -232,6 +251,22 @@ TP_API tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void
 TP_API tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
                         const void* const* dZ, const void* const* W, void* const* dW,
                         float* const* dbias, void* const* dX_partials, void* stream);
+
+/* Column layer backward with the sum of the input gradient fused into its
+ * GEMM ([TP-scratch] §四: the column layer's backward all-reduces dX): dW[i],
+ * dbias[i] as in tp_column_bwd; dX [T, hidden] = sum_i dZ[i] W[i] accumulated
+ * over all shards in one TMEM accumulator and rounded once. bf16 plans only. */
+TP_API tp_status tp_column_bwd_reduce(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                                      const void* const* dZ, const void* const* W, void* const* dW,
+                                      float* const* dbias, void* dX, void* stream);
+
+/* The same with the sequence-parallel reduce-scatter fused in: rows
+ * [j*T/p, (j+1)*T/p) of dX go to dX_seq[j] [T/p, hidden]. */
+TP_API tp_status tp_column_bwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_t T,
+                                                  const void* X, const void* const* dZ,
+                                                  const void* const* W, void* const* dW,
+                                                  float* const* dbias, void* const* dX_seq,
+                                                  void* stream);
 
 /* Backward of tp_reduce_scatter_seq: the all-gather of the dY sequence shards
  * into dY_full [T, hidden] (the conjugate of the reduce-scatter, [TP-wiki]

@@ -9,6 +9,10 @@ reduce / reduce-scatter / all-gather kernels.
              reduce (+bias once); backward: row bwd (act' fused) -> column bwd
              -> reduce of the dX partials.       (TP walkthrough §2-§3.2, §四 of
              "从零实现 Tensor Parallel" for the backward pairing)
+  TPAttention  QKV column GEMM (by whole heads) -> causal attention on local
+             heads -> out-projection partials -> reduce (+bias, +residual), and
+             its backward.                         (TP walkthrough §3.1)
+  TPLayer    pre-LN layer: x1 = x + Attn(LN1(x)); y = x1 + MLP(LN2(x1)).
   SPMLP      Megatron-SP: LN on sequence shards fused with the all-gather ->
              column -> row -> reduce-scatter; backward: all-gather of dY ->
              row bwd -> column bwd -> reduce-scatter of dX partials -> LN bwd
@@ -29,8 +33,12 @@ class TPMLP:
     """One MLP sublayer split over p shards that all live on ``device``."""
 
     def __init__(self, hidden: int, ffn: int, p: int, act: str = "gelu", dtype: str = "bf16",
-                 device="cuda", bias: bool = False, partial_dtype=None):
+                 device="cuda", bias: bool = False, fused: bool = False):
+        """fused: sum the shards inside the row GEMM and the column-backward dX
+        GEMM (tp_row_fwd_reduce / tp_column_bwd_reduce) instead of writing p
+        partials and reducing them (tp_row_fwd_partial + tp_reduce_partials)."""
         self.h, self.f, self.p, self.act = hidden, ffn, p, act
+        self.fused = fused
         self.plan = Plan(hidden, ffn, 0, p, dtype, act)
         self.dt = self.plan.torch_dtype
         self.device = torch.device(device)
@@ -62,11 +70,11 @@ class TPMLP:
         self._T = T
         self.Z = [_empty((T, self.n1), dt, dev) for _ in range(p)]
         self.H = [_empty((T, self.fp), dt, dev) for _ in range(p)]
-        self.P = [_empty((T, self.h), dt, dev) for _ in range(p)]
+        self.P = None if self.fused else [_empty((T, self.h), dt, dev) for _ in range(p)]
         self.Y = _empty((T, self.h), dt, dev)
         if backward:
             self.dZ = [_empty((T, self.n1), dt, dev) for _ in range(p)]
-            self.dXp = [_empty((T, self.h), dt, dev) for _ in range(p)]
+            self.dXp = None if self.fused else [_empty((T, self.h), dt, dev) for _ in range(p)]
             self.dX = _empty((T, self.h), dt, dev)
             self.dW1 = [torch.empty_like(w) for w in self.W1]
             self.dW2 = [torch.empty_like(w) for w in self.W2]
@@ -80,9 +88,12 @@ class TPMLP:
         self.X = X
         pl = self.plan
         pl.column_fwd("mlp", T, X, self.W1, self.b1, self.Z if self.act != "none" else None, self.H)
-        pl.row_fwd_partial("mlp", T, self.H, self.W2, self.P)
         Y = self.Y if out is None else out
-        pl.reduce_partials(T, self.P, self.b2, residual, Y)
+        if self.fused:
+            pl.row_fwd_reduce("mlp", T, self.H, self.W2, self.b2, residual, Y)
+        else:
+            pl.row_fwd_partial("mlp", T, self.H, self.W2, self.P)
+            pl.reduce_partials(T, self.P, self.b2, residual, Y)
         return Y
 
     def backward(self, dY: torch.Tensor, out=None):
@@ -90,9 +101,12 @@ class TPMLP:
         pl = self.plan
         pl.row_bwd("mlp", T, dY, self.H, self.W2, self.Z if self.act != "none" else None, self.dZ,
                    self.dW2, self.db2)
-        pl.column_bwd("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.dXp)
         dX = self.dX if out is None else out
-        pl.reduce_partials(T, self.dXp, None, None, dX)
+        if self.fused:
+            pl.column_bwd_reduce("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, dX)
+        else:
+            pl.column_bwd("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.dXp)
+            pl.reduce_partials(T, self.dXp, None, None, dX)
         return dX
 
     # Number of useful FLOPs in one forward + backward (three GEMMs of each layer).
@@ -106,8 +120,10 @@ class SPMLP:
     """Megatron-SP SwiGLU MLP: LayerNorm on sequence shards, all-gather, column,
     row, reduce-scatter (and the mirrored backward)."""
 
-    def __init__(self, hidden: int, ffn: int, p: int, act: str = "swiglu", device="cuda"):
-        self.mlp = TPMLP(hidden, ffn, p, act, "bf16", device, bias=False)
+    def __init__(self, hidden: int, ffn: int, p: int, act: str = "swiglu", device="cuda",
+                 fused: bool = False):
+        self.fused = fused
+        self.mlp = TPMLP(hidden, ffn, p, act, "bf16", device, bias=False, fused=fused)
         self.plan = self.mlp.plan
         self.h, self.p = hidden, p
         self.gamma = torch.ones(hidden, dtype=torch.bfloat16, device=device)
@@ -141,8 +157,11 @@ class SPMLP:
         pl.layernorm_all_gather_seq(T, X_seq, self.gamma, self.beta, self.U, self.mean, self.rstd)
         m.X = self.U
         pl.column_fwd("mlp", T, self.U, m.W1, None, m.Z, m.H)
-        pl.row_fwd_partial("mlp", T, m.H, m.W2, m.P)
-        pl.reduce_scatter_seq(T, m.P, None, None, self.Y_seq)
+        if self.fused:
+            pl.row_fwd_reduce_scatter_seq("mlp", T, m.H, m.W2, None, None, self.Y_seq)
+        else:
+            pl.row_fwd_partial("mlp", T, m.H, m.W2, m.P)
+            pl.reduce_scatter_seq(T, m.P, None, None, self.Y_seq)
         return self.Y_seq
 
     def backward(self, dY_seq):
@@ -152,8 +171,11 @@ class SPMLP:
         pl, m = self.plan, self.mlp
         pl.reduce_scatter_seq_bwd(T, dY_seq, self.dY_full)
         pl.row_bwd("mlp", T, self.dY_full, m.H, m.W2, m.Z, m.dZ, m.dW2, None)
-        pl.column_bwd("mlp", T, self.U, m.dZ, m.W1, m.dW1, None, m.dXp)
-        pl.all_gather_seq_bwd(T, m.dXp, self.dU_seq)
+        if self.fused:
+            pl.column_bwd_reduce_scatter_seq("mlp", T, self.U, m.dZ, m.W1, m.dW1, None, self.dU_seq)
+        else:
+            pl.column_bwd("mlp", T, self.U, m.dZ, m.W1, m.dW1, None, m.dXp)
+            pl.all_gather_seq_bwd(T, m.dXp, self.dU_seq)
         for j in range(p):
             pl.layernorm_bwd(t, self.X_seq[j], self.gamma, self.dU_seq[j], self.mean[j * t:(j + 1) * t],
                              self.rstd[j * t:(j + 1) * t], self.dX_seq[j], self.dgamma, self.dbeta,
@@ -215,9 +237,102 @@ class TPAttention:
         pl.reduce_partials(T, self.P, self.bo, residual, Y)
         return Y
 
+    def alloc_bwd(self):
+        if hasattr(self, "dQKV") and self.dQKV[0].shape == self.QKV[0].shape:
+            return
+        T, p, dev = self.QKV[0].shape[0], self.p, self.device
+        self.dO = [_empty((T, self.h // p), torch.bfloat16, dev) for _ in range(p)]
+        self.dQKV = [torch.empty_like(x) for x in self.QKV]
+        self.dXp = [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
+        self.dX = _empty((T, self.h), torch.bfloat16, dev)
+        self.dWqkv = [torch.empty_like(w) for w in self.Wqkv]
+        self.dWo = [torch.empty_like(w) for w in self.Wo]
+        self.dbqkv = [_empty((w.shape[0],), torch.float32, dev) for w in self.Wqkv] if self.bias else None
+        self.dbo = _empty((self.h,), torch.float32, dev) if self.bias else None
+
+    def backward(self, dY: torch.Tensor, batch: int, seq: int, out=None):
+        """dY -> (out-proj row bwd) dO_i, dWo_i, dbo -> (attention bwd) dQKV_i ->
+        (QKV column bwd) dWqkv_i, dbqkv_i, dX partials -> reduce."""
+        self.alloc_bwd()
+        T = batch * seq
+        pl = self.plan
+        pl.row_bwd("outproj", T, dY, self.O, self.Wo, None, self.dO, self.dWo, self.dbo)
+        pl.attention_bwd(batch, seq, self.QKV, self.O, self.dO, self.LSE, self.dQKV)
+        pl.column_bwd("qkv", T, self.X, self.dQKV, self.Wqkv, self.dWqkv, self.dbqkv, self.dXp)
+        dX = self.dX if out is None else out
+        pl.reduce_partials(T, self.dXp, None, None, dX)
+        return dX
+
     def flops_fwd(self, batch: int, seq: int, causal: bool = True) -> float:
         T = batch * seq
         proj = 2.0 * T * self.h * 3 * self.h + 2.0 * T * self.h * self.h
         pairs = seq * (seq + 1) / 2 if causal else seq * seq
         att = 4.0 * batch * self.H * pairs * self.d
         return proj + att
+
+
+class TPLayer:
+    """Pre-LN transformer layer with a GELU MLP, every sublayer split over p
+    shards on one GPU: x1 = x + Attn(LN1(x)); y = x1 + MLP(LN2(x1)).
+    Biases on every projection (TP-basics' row bias enters once, in the reduce)."""
+
+    def __init__(self, hidden: int, ffn: int, heads: int, p: int, device="cuda"):
+        self.h = hidden
+        self.attn = TPAttention(hidden, heads, p, device, bias=True)
+        self.mlp = TPMLP(hidden, ffn, p, "gelu", "bf16", device, bias=True)
+        self.ln = Plan(hidden, 0, 0, 1, "bf16", "none")  # LayerNorm / elementwise calls
+        self.device = torch.device(device)
+        dev = self.device
+        self.ln1_g = torch.ones(hidden, dtype=torch.bfloat16, device=dev)
+        self.ln1_b = torch.zeros(hidden, dtype=torch.bfloat16, device=dev)
+        self.ln2_g = torch.ones(hidden, dtype=torch.bfloat16, device=dev)
+        self.ln2_b = torch.zeros(hidden, dtype=torch.bfloat16, device=dev)
+        self._T = None
+
+    def load(self, prm):
+        """prm: a tp_synth.LayerParams with tensors already on the device."""
+        self.ln1_g.copy_(prm.ln1_g)
+        self.ln1_b.copy_(prm.ln1_b)
+        self.ln2_g.copy_(prm.ln2_g)
+        self.ln2_b.copy_(prm.ln2_b)
+        self.attn.load_weights(prm.Wqkv, prm.Wo, prm.bqkv, prm.bo)
+        self.mlp.load_weights(prm.W1, prm.W2, prm.b1, prm.b2)
+
+    def alloc(self, T: int):
+        if self._T == T:
+            return
+        self._T = T
+        dev, h = self.device, self.h
+        bf, f32 = torch.bfloat16, torch.float32
+        self.u1, self.u2 = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
+        self.x1, self.y = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
+        self.m1, self.r1 = _empty((T,), f32, dev), _empty((T,), f32, dev)
+        self.m2, self.r2 = _empty((T,), f32, dev), _empty((T,), f32, dev)
+        self.dx1_ln, self.dx1 = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
+        self.dx_ln, self.dx = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
+        self.dln1_g, self.dln1_b = _empty((h,), f32, dev), _empty((h,), f32, dev)
+        self.dln2_g, self.dln2_b = _empty((h,), f32, dev), _empty((h,), f32, dev)
+
+    def forward(self, x: torch.Tensor, batch: int, seq: int):
+        T = batch * seq
+        self.alloc(T)
+        self.x = x
+        ln = self.ln
+        ln.layernorm_fwd(T, x, self.ln1_g, self.ln1_b, self.u1, self.m1, self.r1)
+        self.attn.forward(self.u1, batch, seq, residual=x, out=self.x1)
+        ln.layernorm_fwd(T, self.x1, self.ln2_g, self.ln2_b, self.u2, self.m2, self.r2)
+        self.mlp.forward(self.u2, residual=self.x1, out=self.y)
+        return self.y
+
+    def backward(self, dy: torch.Tensor, batch: int, seq: int):
+        T = batch * seq
+        ln = self.ln
+        du2 = self.mlp.backward(dy)
+        ln.layernorm_bwd(T, self.x1, self.ln2_g, du2, self.m2, self.r2, self.dx1_ln,
+                         self.dln2_g, self.dln2_b)
+        ln.reduce_partials(T, [dy, self.dx1_ln], None, None, self.dx1)        # residual branch
+        du1 = self.attn.backward(self.dx1, batch, seq)
+        ln.layernorm_bwd(T, self.x, self.ln1_g, du1, self.m1, self.r1, self.dx_ln,
+                         self.dln1_g, self.dln1_b)
+        ln.reduce_partials(T, [self.dx1, self.dx_ln], None, None, self.dx)
+        return self.dx

@@ -558,6 +558,77 @@ tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const voi
   return run_gemm(plan, b, as_stream(stream));
 }
 
+// Row GEMM with the shard sum fused (K-concatenated over shards), writing the
+// full output or (scatter) its sequence shards.
+static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
+                                       const void* const* H, const void* const* W, const void* bias,
+                                       const void* residual, const void* const* residual_seq,
+                                       void* Y, void* const* Y_seq, bool scatter, cudaStream_t st) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "the fused reduce runs on bf16 plans");
+  int k = 0;
+  TP_TRY(row_k(plan, which, &k));
+  const int p = plan->p, h = plan->hidden;
+  TP_TRY(check_ptrs(H, p, "H", false));
+  TP_TRY(check_ptrs(W, p, "W", false));
+  if (bias) TP_TRY(check_ptr(bias, "bias"));
+  TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
+  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (scatter) {
+    if (T % p) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by p = %d", (long long)T, p);
+    TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Y_seq), p, "Y_seq", false));
+    TP_TRY(check_ptrs(residual_seq, p, "residual_seq", true));
+  } else {
+    TP_TRY(check_ptr(Y, "Y"));
+    if (residual) TP_TRY(check_ptr(residual, "residual"));
+  }
+  if (T == 0) return TP_OK;
+  GemmBatch b{};
+  b.n = p;
+  b.kcat = true;
+  b.epi = EPI_STORE;
+  for (int i = 0; i < p; ++i) {
+    GemmProblem& g = b.g[i];
+    g.M = static_cast<int>(T);
+    g.N = h;
+    g.K = k;
+    g.A = H[i];
+    g.lda = k;
+    g.B = W[i];
+    g.ldb = k;
+  }
+  b.g[0].D = scatter ? Y_seq[0] : Y;
+  b.g[0].ldd = h;
+  b.g[0].bias = bias;
+  b.g[0].aux = scatter ? nullptr : residual;
+  b.g[0].ldaux = h;
+  if (scatter) {
+    b.scatter_n = p;
+    b.rows_per_out = T / p;
+    for (int j = 0; j < p; ++j) {
+      b.out_seq[j] = Y_seq[j];
+      b.res_seq[j] = residual_seq ? residual_seq[j] : nullptr;
+    }
+  }
+  return launch_gemm_bf16(b, st);
+}
+
+tp_status tp_row_fwd_reduce(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                            const void* const* W, const void* bias, const void* residual, void* Y,
+                            void* stream) {
+  return row_fwd_reduce_common(plan, which, T, H, W, bias, residual, nullptr, Y, nullptr, false,
+                               as_stream(stream));
+}
+
+tp_status tp_row_fwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_t T,
+                                        const void* const* H, const void* const* W,
+                                        const void* bias, const void* const* residual_seq,
+                                        void* const* Y_seq, void* stream) {
+  return row_fwd_reduce_common(plan, which, T, H, W, bias, nullptr, residual_seq, nullptr, Y_seq,
+                               true, as_stream(stream));
+}
+
 static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* const* P,
                                const void* bias, const void* residual,
                                const void* const* residual_seq, void* Y,
@@ -829,25 +900,31 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
   return TP_OK;
 }
 
-tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
-                        const void* const* dZ, const void* const* W, void* const* dW,
-                        float* const* dbias, void* const* dX_partials, void* stream) {
+// dX mode: 0 = partials (dX_out[i] per shard), 1 = summed (dX_out[0] full),
+// 2 = summed and scattered by sequence (dX_out[j] = rows of shard j).
+static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                                   const void* const* dZ, const void* const* W, void* const* dW,
+                                   float* const* dbias, void* const* dX_out, int mode,
+                                   cudaStream_t st) {
   TP_TRY(check_plan(plan));
   TP_TRY(check_T(T));
   ColShape cs{};
   TP_TRY(col_shape(plan, which, &cs));
   const int p = plan->p, h = plan->hidden;
   const int n = cs.n_w;
+  if (mode != 0 && plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "the fused reduce runs on bf16 plans");
   TP_TRY(check_ptrs(dZ, p, "dZ", false));
   TP_TRY(check_ptrs(W, p, "W", false));
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dW), p, "dW", true));
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dbias), p, "dbias", true));
-  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX_partials), p, "dX_partials", true));
+  const int nout = mode == 1 ? 1 : p;
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX_out), nout, "dX", mode == 0));
+  if (mode == 2 && T % p)
+    return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by p = %d", (long long)T, p);
   if (dW) TP_TRY(check_ptr(X, "X"));
   TP_TRY(check_row_bytes(n, plan->dtype, "dZ_i width"));
   TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
   if (T == 0) return TP_OK;
-  cudaStream_t st = as_stream(stream);
   if (dW) {
     // dW_i [n, h] = dZ_i^T X: A(m, t) = dZ_i[t, m] (MN-major), B(c, t) = X[t, c] (MN-major).
     GemmBatch w{};
@@ -870,7 +947,7 @@ tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
     }
     TP_TRY(run_gemm(plan, w, st));
   }
-  if (dX_partials) {
+  if (dX_out) {
     // dX_i [T, h] = dZ_i W_i: A = dZ_i (K-major), B(c, j) = W_i[j, c] (MN-major).
     GemmBatch d{};
     d.n = p;
@@ -878,6 +955,7 @@ tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
     d.b_mn = true;
     d.epi = EPI_STORE;
     d.out_f32 = plan->dtype == TP_F32;
+    d.kcat = mode != 0;
     for (int i = 0; i < p; ++i) {
       GemmProblem& g = d.g[i];
       g.M = static_cast<int>(T);
@@ -887,8 +965,13 @@ tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
       g.lda = n;
       g.B = W[i];
       g.ldb = h;
-      g.D = dX_partials[i];
+      g.D = mode == 0 ? dX_out[i] : dX_out[0];
       g.ldd = h;
+    }
+    if (mode == 2) {
+      d.scatter_n = p;
+      d.rows_per_out = T / p;
+      for (int j = 0; j < p; ++j) d.out_seq[j] = dX_out[j];
     }
     TP_TRY(run_gemm(plan, d, st));
   }
@@ -896,6 +979,27 @@ tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
     for (int i = 0; i < p; ++i)
       TP_TRY(launch_column_sum(plan, dZ[i], T, n, n, dbias[i], 0, plan->dtype, st));
   return TP_OK;
+}
+
+tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                        const void* const* dZ, const void* const* W, void* const* dW,
+                        float* const* dbias, void* const* dX_partials, void* stream) {
+  return column_bwd_common(plan, which, T, X, dZ, W, dW, dbias, dX_partials, 0, as_stream(stream));
+}
+
+tp_status tp_column_bwd_reduce(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                               const void* const* dZ, const void* const* W, void* const* dW,
+                               float* const* dbias, void* dX, void* stream) {
+  void* out[1] = {dX};
+  return column_bwd_common(plan, which, T, X, dZ, W, dW, dbias, out, 1, as_stream(stream));
+}
+
+tp_status tp_column_bwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_t T,
+                                           const void* X, const void* const* dZ,
+                                           const void* const* W, void* const* dW,
+                                           float* const* dbias, void* const* dX_seq,
+                                           void* stream) {
+  return column_bwd_common(plan, which, T, X, dZ, W, dW, dbias, dX_seq, 2, as_stream(stream));
 }
 
 }  // extern "C"

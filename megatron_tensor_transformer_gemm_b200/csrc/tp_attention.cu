@@ -15,7 +15,7 @@
 //               state (m, l) stay in registers and are rescaled per block.
 // Blocks are causal: the tile's last key block is the diagonal one and is
 // masked (key > query -> probability 0); keys and queries past seq are masked.
-// The backward recomputes P from the saved row log-sum-exp.
+// The backward (tp_attention_bwd.cu) recomputes P from the saved row log-sum-exp.
 #include <cuda.h>
 
 #include <algorithm>
@@ -23,6 +23,7 @@
 
 #include "tp_device.cuh"
 #include "tp_internal.h"
+#include "tp_tma.h"
 
 namespace {
 
@@ -307,26 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-tp_status get_encoder(EncodeTiledFn* out) {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  if (!fn) return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  *out = fn;
-  return TP_OK;
-}
-
 template <int D>
 tp_status launch_fwd_d(AttnParams& prm, cudaStream_t st) {
   static bool attr = false;
@@ -351,9 +332,7 @@ tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const Pt
                                const MutPtrArray& o, float* const* lse, cudaStream_t st) {
   const int p = plan->p, d = plan->head_dim, hl = plan->heads / plan->p;
   const int64_t C = 3LL * hl * d;
-  EncodeTiledFn enc = nullptr;
-  tp_status s = get_encoder(&enc);
-  if (s != TP_OK) return s;
+  tp_status s = TP_OK;
   static AttnParams prm;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
@@ -363,12 +342,8 @@ tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const Pt
                           static_cast<cuuint64_t>(seq)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * batch};
     cuuint32_t box[3] = {64, 1, 128};
-    cuuint32_t es[3] = {1, 1, 1};
-    CUresult r = enc(&prm.tm[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv.p[i]),
-                     dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(QKV %d) failed: %d", i, (int)r);
+    s = encode_bf16(&prm.tm[i], qkv.p[i], 3, dims, strides, box, "QKV");
+    if (s != TP_OK) return s;
     prm.O[i] = o.p[i];
     prm.lse[i] = lse ? lse[i] : nullptr;
   }
@@ -386,12 +361,6 @@ tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const Pt
   if (d == 64) return launch_fwd_d<64>(prm, st);
   if (d == 128) return launch_fwd_d<128>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
-}
-
-tp_status launch_attention_bwd(tp_plan*, int, int, const PtrArray&, const PtrArray&,
-                               const PtrArray&, const float* const*, const MutPtrArray&,
-                               cudaStream_t) {
-  return fail(TP_ERR_UNSUPPORTED, "attention backward is not built yet");
 }
 
 }  // namespace tpi

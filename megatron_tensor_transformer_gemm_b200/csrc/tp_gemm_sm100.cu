@@ -13,7 +13,8 @@
 // Design (per CTA, one CTA per SM, persistent over a static tile schedule):
 //   warp 0      TMA producer: 128B-swizzled A and B tiles into a 4-stage ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> HBM
+//   warps 2..9  epilogue: tcgen05.ld TMEM -> registers -> fused math -> HBM;
+//               two warps per TMEM lane quarter, each taking half of the columns
 // The 128x256 fp32 accumulator lives in TMEM (256 columns); two accumulators
 // (all 512 columns) let the epilogue of one tile overlap the MMAs of the next.
 // Operands may be K-major or MN-major (the backward GEMMs read dY^T, X^T and
@@ -28,6 +29,7 @@
 
 #include "tp_device.cuh"
 #include "tp_internal.h"
+#include "tp_tma.h"
 
 namespace {
 
@@ -40,7 +42,8 @@ constexpr int BN = 256;
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int STAGES = 4;
 constexpr int UMMA_K = 16;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -75,6 +78,17 @@ struct alignas(64) GemmParams {
   int b_mn;
   int epi;
   int out_f32;
+  // K-concatenated mode (kcat > 0): one output problem (g[0]) whose K loop runs
+  // over kcat segments, segment s reading tmA[s] / tmB[s] for seg_kb[s] blocks:
+  // D = sum_s A_s B_s^T, i.e. the sum over shards happens in the accumulator.
+  int kcat;
+  int seg_kb[TP_MAX_SHARDS];
+  // Row scatter (scatter > 0): output row r goes to out_seq[r / rows_per_out]
+  // at row r % rows_per_out, with residual rows from res_seq (if non-NULL).
+  int scatter;
+  int rows_per_out;
+  void* out_seq[TP_MAX_SHARDS];
+  const void* res_seq[TP_MAX_SHARDS];
   unsigned* status;
 };
 
@@ -129,13 +143,15 @@ __device__ __forceinline__ void load_row_chunk_bf16(const void* base, int64_t ld
   }
 }
 
+// Columns [half * BN/2, (half + 1) * BN/2) of the accumulator row this thread owns.
 __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t taddr, int row,
-                              int n0) {
+                              int n0, int half) {
   const bool row_ok = row < ga.M;
   if (p.epi == tpi::EPI_SWIGLU) {
-    // Accumulator columns [0,128) = gate units n0.., [128,256) = the same up units.
+    // Accumulator columns [0,128) = gate units n0.., [128,256) = the same up units;
+    // this thread handles gate/up pairs [half * 64, half * 64 + 64).
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = half * 2; c < half * 2 + 2; ++c) {
       float g[32], u[32];
       tmem_ld32(taddr + c * 32, g);
       tmem_ld32(taddr + 128 + c * 32, u);
@@ -155,7 +171,7 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
     return;
   }
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
     tc_wait_ld();
@@ -169,8 +185,23 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] += b[i];
         }
-        if (p.out_f32) store_row_chunk_f32(ga.D, ga.ldd, row, j0, ga.N, v);
-        else store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, v);
+        void* dst = ga.D;
+        const void* res = ga.aux;
+        int orow = row;
+        if (p.scatter) {
+          const int j = row / p.rows_per_out;
+          orow = row - j * p.rows_per_out;
+          dst = p.out_seq[j];
+          res = p.res_seq[j];
+        }
+        if (res) {
+          float r[32];
+          load_row_chunk_bf16(res, ga.ldaux, orow, j0, ga.N, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += r[i];
+        }
+        if (p.out_f32) store_row_chunk_f32(dst, ga.ldd, orow, j0, ga.N, v);
+        else store_row_chunk_bf16(dst, ga.ldd, orow, j0, ga.N, v);
         break;
       }
       case tpi::EPI_BIAS_GELU: {
@@ -239,14 +270,15 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    for (int g = 0; g < p.ngroups; ++g) {
+    const int nmaps = p.kcat ? p.kcat : p.ngroups;
+    for (int g = 0; g < nmaps; ++g) {
       tma_prefetch_desc(&p.tmA[g]);
       tma_prefetch_desc(&p.tmB[g]);
     }
@@ -274,36 +306,41 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const GroupArgs& ga = p.g[g];
       const int m0 = mt * BM;
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
-      for (int kb = 0; kb < ga.num_kb; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-        const int k0 = kb * BK;
-        uint8_t* a_dst = sA + stage * A_BYTES;
-        uint8_t* b_dst = sB + stage * B_BYTES;
-        if (!p.a_mn) {
-          tma_load_2d(a_dst, &p.tmA[g], &full[stage], k0, m0);
-        } else {
+      const int nseg = p.kcat ? p.kcat : 1;
+      for (int sg = 0; sg < nseg && ok; ++sg) {
+        const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
+        const int nkb = p.kcat ? p.seg_kb[sg] : ga.num_kb;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          const int k0 = kb * BK;
+          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* b_dst = sB + stage * B_BYTES;
+          if (!p.a_mn) {
+            tma_load_2d(a_dst, &p.tmA[gi], &full[stage], k0, m0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BM / 64; ++c)
-            tma_load_2d(a_dst + c * MN_BLOCK_BYTES, &p.tmA[g], &full[stage], m0 + c * 64, k0);
-        }
-        if (p.epi == tpi::EPI_SWIGLU) {
-          tma_load_3d(b_dst, &p.tmB[g], &full[stage], k0, n0, 0);
-          tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[g], &full[stage], k0, n0, 1);
-        } else if (!p.b_mn) {
-          tma_load_2d(b_dst, &p.tmB[g], &full[stage], k0, n0);
-        } else {
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(a_dst + c * MN_BLOCK_BYTES, &p.tmA[gi], &full[stage], m0 + c * 64, k0);
+          }
+          if (p.epi == tpi::EPI_SWIGLU) {
+            tma_load_3d(b_dst, &p.tmB[gi], &full[stage], k0, n0, 0);
+            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[gi], &full[stage], k0, n0, 1);
+          } else if (!p.b_mn) {
+            tma_load_2d(b_dst, &p.tmB[gi], &full[stage], k0, n0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c)
-            tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[g], &full[stage], n0 + c * 64, k0);
-        }
-        last_parity[stage] = static_cast<int>(phase);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], &full[stage], n0 + c * 64, k0);
+          }
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
     }
@@ -322,7 +359,11 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
-      const int num_kb = p.g[g].num_kb;
+      int num_kb = p.g[g].num_kb;
+      if (p.kcat) {
+        num_kb = 0;
+        for (int sg = 0; sg < p.kcat; ++sg) num_kb += p.seg_kb[sg];
+      }
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -361,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   } else if (warp >= 2) {
     // ------------------------------------------------------------- epilogue
     const int lg = warp & 3;  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) / 4;  // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
@@ -373,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_tile(p, ga, taddr, row, n0);
+      epilogue_tile(p, ga, taddr, row, n0, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -391,25 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-tp_status get_encoder(EncodeTiledFn* out) {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  static cudaError_t err = cudaSuccess;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
-    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  if (!fn) return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
-  *out = fn;
-  return TP_OK;
-}
+using tpi::EncodeTiledFn;
 
 // 2-D bf16 tensor [outer, inner] (row stride ld elements), box {64, box_outer}.
 tp_status encode_2d(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_t inner,
@@ -458,7 +482,7 @@ namespace tpi {
 tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   if (b.n < 1 || b.n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "GEMM group count %d", b.n);
   EncodeTiledFn enc = nullptr;
-  tp_status s = get_encoder(&enc);
+  tp_status s = tma_encoder(&enc);
   if (s != TP_OK) return s;
   static GemmParams p;  // host staging (large); launches copy it into the parameter buffer
   static std::mutex mu;
@@ -466,47 +490,64 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   memset(&p, 0, sizeof(p));
   const bool swiglu = b.epi == EPI_SWIGLU;
   const int tile_n = swiglu ? BN / 2 : BN;
+  if (b.kcat && b.epi != EPI_STORE)
+    return fail(TP_ERR_ARG, "K-concatenated GEMM supports the plain epilogue only");
   int tiles = 0;
+  const int nout = b.kcat ? 1 : b.n;
   for (int i = 0; i < b.n; ++i) {
     const GemmProblem& g = b.g[i];
-    if (g.M <= 0 || g.N <= 0 || g.K <= 0)
-      return fail(TP_ERR_ARG, "GEMM %d has an empty extent (%d x %d x %d)", i, g.M, g.N, g.K);
+    const GemmProblem& o = b.kcat ? b.g[0] : g;  // the output this segment feeds
+    if (o.M <= 0 || o.N <= 0 || g.K <= 0)
+      return fail(TP_ERR_ARG, "GEMM %d has an empty extent (%d x %d x %d)", i, o.M, o.N, g.K);
     // TMA needs 16-byte row strides; the epilogue stores 8-column vectors, so N
     // and the output strides must be multiples of 8. K and M may be ragged.
-    if (g.N % 8 || g.lda % 8 || g.ldb % 8 || (g.D && g.ldd % 8) || (g.D2 && g.ldd2 % 8) ||
-        (g.aux && g.ldaux % 8))
+    if (o.N % 8 || g.lda % 8 || g.ldb % 8 || (o.D && o.ldd % 8) || (o.D2 && o.ldd2 % 8) ||
+        (o.aux && o.ldaux % 8))
       return fail(TP_ERR_ALIGN, "GEMM %d: N and every leading dimension must be multiples of 8 "
-                  "(N=%d lda=%lld ldb=%lld ldd=%lld)", i, g.N, (long long)g.lda, (long long)g.ldb,
-                  (long long)g.ldd);
-    GroupArgs& a = p.g[i];
-    a.M = g.M;
-    a.N = g.N;
-    a.K = g.K;
-    a.tiles_n = (g.N + tile_n - 1) / tile_n;
-    a.tile_begin = tiles;
-    a.num_kb = (g.K + BK - 1) / BK;
-    a.nh = g.nh;
-    a.D = g.D;
-    a.ldd = g.ldd;
-    a.D2 = g.D2;
-    a.ldd2 = g.ldd2;
-    a.bias = g.bias;
-    a.aux = g.aux;
-    a.ldaux = g.ldaux;
-    const int64_t t = static_cast<int64_t>((g.M + BM - 1) / BM) * a.tiles_n;
-    if (tiles + t > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "too many GEMM tiles");
-    tiles += static_cast<int>(t);
-    // A operand
-    if (!b.a_mn) s = encode_2d(enc, &p.tmA[i], g.A, g.K, g.M, g.lda, BM);
-    else s = encode_2d(enc, &p.tmA[i], g.A, g.M, g.K, g.lda, BK);
+                  "(N=%d lda=%lld ldb=%lld ldd=%lld)", i, o.N, (long long)g.lda, (long long)g.ldb,
+                  (long long)o.ldd);
+    if (i < nout) {
+      GroupArgs& a = p.g[i];
+      a.M = o.M;
+      a.N = o.N;
+      a.K = g.K;
+      a.tiles_n = (o.N + tile_n - 1) / tile_n;
+      a.tile_begin = tiles;
+      a.num_kb = (g.K + BK - 1) / BK;
+      a.nh = o.nh;
+      a.D = o.D;
+      a.ldd = o.ldd;
+      a.D2 = o.D2;
+      a.ldd2 = o.ldd2;
+      a.bias = o.bias;
+      a.aux = o.aux;
+      a.ldaux = o.ldaux;
+      const int64_t t = static_cast<int64_t>((o.M + BM - 1) / BM) * a.tiles_n;
+      if (tiles + t > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "too many GEMM tiles");
+      tiles += static_cast<int>(t);
+    }
+    if (b.kcat) p.seg_kb[i] = (g.K + BK - 1) / BK;
+    // A operand: [M, K] (K-major) or [K, M] (MN-major)
+    if (!b.a_mn) s = encode_2d(enc, &p.tmA[i], g.A, g.K, o.M, g.lda, BM);
+    else s = encode_2d(enc, &p.tmA[i], g.A, o.M, g.K, g.lda, BK);
     if (s != TP_OK) return s;
     // B operand
-    if (swiglu) s = encode_gateup(enc, &p.tmB[i], g.B, g.K, g.nh, g.ldb);
-    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, g.N, g.ldb, BN);
-    else s = encode_2d(enc, &p.tmB[i], g.B, g.N, g.K, g.ldb, BK);
+    if (swiglu) s = encode_gateup(enc, &p.tmB[i], g.B, g.K, o.nh, g.ldb);
+    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, o.N, g.ldb, BN);
+    else s = encode_2d(enc, &p.tmB[i], g.B, o.N, g.K, g.ldb, BK);
     if (s != TP_OK) return s;
   }
-  p.ngroups = b.n;
+  p.kcat = b.kcat ? b.n : 0;
+  if (b.scatter_n > 0) {
+    if (!b.kcat && b.n != 1) return fail(TP_ERR_ARG, "row scatter needs a single output");
+    p.scatter = 1;
+    p.rows_per_out = static_cast<int>(b.rows_per_out);
+    for (int j = 0; j < b.scatter_n; ++j) {
+      p.out_seq[j] = b.out_seq[j];
+      p.res_seq[j] = b.res_seq[j];
+    }
+  }
+  p.ngroups = nout;
   p.total_tiles = tiles;
   p.a_mn = b.a_mn;
   p.b_mn = b.b_mn;
@@ -525,6 +566,41 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   const int grid = std::min(tiles, device_sms());
   tp_gemm_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
   return after_launch("gemm_bf16 (tcgen05)");
+}
+
+}  // namespace tpi
+
+namespace tpi {
+
+tp_status tma_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  if (!fn)
+    return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *out = fn;
+  return TP_OK;
+}
+
+tp_status encode_bf16(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+                      const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+  EncodeTiledFn enc = nullptr;
+  tp_status s = tma_encoder(&enc);
+  if (s != TP_OK) return s;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                   const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+  return TP_OK;
 }
 
 }  // namespace tpi

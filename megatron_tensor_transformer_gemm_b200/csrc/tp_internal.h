@@ -115,6 +115,17 @@ struct GemmBatch {
   bool b_mn;
   int epi;
   bool out_f32;  // D written as fp32 (bf16 otherwise)
+  // K-concatenated: the n problems are K segments of ONE output, D = sum_i
+  // A_i B_i^T (the shards' sum happens in the accumulator). M, N, D, ldd,
+  // bias and aux (a residual added in the epilogue) come from g[0]; each
+  // g[i] gives A, lda, B, ldb, K of its segment. EPI_STORE only.
+  bool kcat;
+  // Row scatter of that single output: row r goes to out_seq[r / rows_per_out]
+  // (row r % rows_per_out, stride g[0].ldd), plus res_seq[j] rows if given.
+  int scatter_n;  // 0 = off, else number of output blocks
+  int64_t rows_per_out;
+  void* out_seq[TP_MAX_SHARDS];
+  const void* res_seq[TP_MAX_SHARDS];
 };
 
 // bf16 tcgen05 tensor-core path (tp_gemm_sm100.cu).

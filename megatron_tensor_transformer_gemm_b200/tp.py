@@ -77,6 +77,10 @@ _SIGS = {
     "tp_attention_bwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_column_sum": (_int, [_plan_p, _i64, _i64, _vp, _fp, _int, _vp]),
     "tp_column_sum_static": (_int, [_i64, _i64, _int, _vp, _fp, _int, _vp]),
+    "tp_row_fwd_reduce": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vp, _vp, _vp, _vp]),
+    "tp_row_fwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vp, _vpp, _vpp, _vp]),
+    "tp_column_bwd_reduce": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp]),
+    "tp_column_bwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -186,6 +190,15 @@ class Plan:
         check(lib.tp_row_fwd_partial(self._h, WHICH[which], T, _arr(H), _arr(W), _arr(P),
                                      _stream(stream)), "tp_row_fwd_partial")
 
+    def row_fwd_reduce(self, which, T, H, W, bias, residual, Y, stream=None):
+        check(lib.tp_row_fwd_reduce(self._h, WHICH[which], T, _arr(H), _arr(W), _ptr(bias),
+                                    _ptr(residual), _ptr(Y), _stream(stream)), "tp_row_fwd_reduce")
+
+    def row_fwd_reduce_scatter_seq(self, which, T, H, W, bias, residual_seq, Y_seq, stream=None):
+        check(lib.tp_row_fwd_reduce_scatter_seq(self._h, WHICH[which], T, _arr(H), _arr(W), _ptr(bias),
+                                                _arr(residual_seq), _arr(Y_seq), _stream(stream)),
+              "tp_row_fwd_reduce_scatter_seq")
+
     def reduce_partials(self, T, P, bias, residual, Y, stream=None):
         check(lib.tp_reduce_partials(self._h, T, len(P), _arr(P), _ptr(bias), _ptr(residual),
                                      _ptr(Y), _stream(stream)), "tp_reduce_partials")
@@ -220,6 +233,16 @@ class Plan:
     def column_bwd(self, which, T, X, dZ, W, dW=None, dbias=None, dX_partials=None, stream=None):
         check(lib.tp_column_bwd(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
                                 _arr(dbias), _arr(dX_partials), _stream(stream)), "tp_column_bwd")
+
+    def column_bwd_reduce(self, which, T, X, dZ, W, dW=None, dbias=None, dX=None, stream=None):
+        check(lib.tp_column_bwd_reduce(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
+                                       _arr(dbias), _ptr(dX), _stream(stream)), "tp_column_bwd_reduce")
+
+    def column_bwd_reduce_scatter_seq(self, which, T, X, dZ, W, dW=None, dbias=None, dX_seq=None,
+                                      stream=None):
+        check(lib.tp_column_bwd_reduce_scatter_seq(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W),
+                                                   _arr(dW), _arr(dbias), _arr(dX_seq), _stream(stream)),
+              "tp_column_bwd_reduce_scatter_seq")
 
     def reduce_scatter_seq_bwd(self, T, dY_seq, dY_full, stream=None):
         check(lib.tp_reduce_scatter_seq_bwd(self._h, T, len(dY_seq), _arr(dY_seq), _ptr(dY_full),

@@ -414,7 +414,7 @@ def attention_fwd(Q, K, V, batch, heads, causal=True):
     """
     q, k, v = (_split_heads(a, batch, heads) for a in (Q, K, V))
     d = q.shape[-1]
-    S = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(d)
+    S = np.matmul(q, k.swapaxes(-1, -2)) / math.sqrt(d)
     s = S.shape[-1]
     if causal:
         mask = np.triu(np.ones((s, s), dtype=bool), k=1)
@@ -423,7 +423,7 @@ def attention_fwd(Q, K, V, batch, heads, causal=True):
     E = np.exp(S - m)
     L = E.sum(axis=-1, keepdims=True)
     P = E / L
-    O = np.einsum("bhij,bhjd->bhid", P, v)
+    O = np.matmul(P, v)
     lse = (m + np.log(L))[..., 0]
     return _merge_heads(O), lse
 
@@ -437,14 +437,14 @@ def attention_fwd_rows(Q, K, V, batch, heads, rows, causal=True):
     q, k, v = (_split_heads(a, batch, heads) for a in (Q, K, V))
     d = q.shape[-1]
     rows = np.asarray(rows)
-    S = np.einsum("bhid,bhjd->bhij", q[:, :, rows], k) / math.sqrt(d)
+    S = np.matmul(q[:, :, rows], k.swapaxes(-1, -2)) / math.sqrt(d)
     if causal:
         mask = np.arange(k.shape[2])[None, :] > rows[:, None]
         S = np.where(mask[None, None], -np.inf, S)
     m = S.max(axis=-1, keepdims=True)
     E = np.exp(S - m)
     L = E.sum(axis=-1, keepdims=True)
-    O = np.einsum("bhij,bhjd->bhid", E / L, v)
+    O = np.matmul(E / L, v)
     return _merge_heads(O), (m + np.log(L))[..., 0]
 
 
@@ -456,7 +456,7 @@ def attention_bwd(Q, K, V, dO, batch, heads, causal=True):
     """
     q, k, v, do = (_split_heads(a, batch, heads) for a in (Q, K, V, dO))
     d = q.shape[-1]
-    S = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(d)
+    S = np.matmul(q, k.swapaxes(-1, -2)) / math.sqrt(d)
     s = S.shape[-1]
     if causal:
         mask = np.triu(np.ones((s, s), dtype=bool), k=1)
@@ -464,13 +464,13 @@ def attention_bwd(Q, K, V, dO, batch, heads, causal=True):
     m = S.max(axis=-1, keepdims=True)
     E = np.exp(S - m)
     P = E / E.sum(axis=-1, keepdims=True)
-    O = np.einsum("bhij,bhjd->bhid", P, v)
-    dV = np.einsum("bhij,bhid->bhjd", P, do)
-    dP = np.einsum("bhid,bhjd->bhij", do, v)
+    O = np.matmul(P, v)
+    dV = np.matmul(P.swapaxes(-1, -2), do)
+    dP = np.matmul(do, v.swapaxes(-1, -2))
     Dr = (do * O).sum(axis=-1, keepdims=True)
     dS = P * (dP - Dr)
-    dQ = np.einsum("bhij,bhjd->bhid", dS, k) / math.sqrt(d)
-    dK = np.einsum("bhij,bhid->bhjd", dS, q) / math.sqrt(d)
+    dQ = np.matmul(dS, k) / math.sqrt(d)
+    dK = np.matmul(dS.swapaxes(-1, -2), q) / math.sqrt(d)
     return _merge_heads(dQ), _merge_heads(dK), _merge_heads(dV)
 
 

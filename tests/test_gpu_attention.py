@@ -63,3 +63,33 @@ def test_attention_block_full_size_sampled():
     got = host(Y).reshape(seq, batch, h)[rows_s].reshape(-1, h)
     assert_close(got, Yref, TOL_BF16, "Y sampled rows")
     assert _tp().device_status() == "TP_OK"
+
+
+@pytest.mark.parametrize("batch,seq,heads,d,p", [
+    (2, 300, 4, 64, 2),
+    (1, 256, 2, 128, 1),
+    (3, 129, 8, 64, 4),
+])
+def test_attention_bwd_local_heads(batch, seq, heads, d, p):
+    """dQ, dK, dV of each shard's heads from independent Q, K, V, dO; O and LSE
+    come from the GPU forward of those inputs (the oracle computes its own)."""
+    tp = _tp()
+    h = heads * d
+    Q, K, V, dO = tp_synth.draw_qkv_activations(batch, seq, heads, d, torch.bfloat16, seed=seq + 7)
+    hl = heads // p
+    plan = tp.Plan(h, 0, heads, p, "bf16", "none")
+    qkv, outs, lses, dos, dqkv = [], [], [], [], []
+    for i in range(p):
+        sl = slice(i * hl * d, (i + 1) * hl * d)
+        qkv.append(dev(torch.cat([Q[:, :, sl], K[:, :, sl], V[:, :, sl]], dim=2).reshape(seq * batch, 3 * hl * d)))
+        outs.append(torch.empty(seq * batch, hl * d, dtype=torch.bfloat16, device="cuda"))
+        lses.append(torch.empty(batch, hl, seq, dtype=torch.float32, device="cuda"))
+        dos.append(dev(dO[:, :, sl].reshape(seq * batch, hl * d)))
+        dqkv.append(torch.empty(seq * batch, 3 * hl * d, dtype=torch.bfloat16, device="cuda"))
+    plan.attention_fwd(batch, seq, qkv, outs, lses)
+    plan.attention_bwd(batch, seq, qkv, outs, dos, lses, dqkv)
+    rq, rk, rv = O.attention_bwd(O.f64(Q), O.f64(K), O.f64(V), O.f64(dO), batch, heads, True)
+    got = [host(x).reshape(seq, batch, 3, hl * d) for x in dqkv]
+    for name, idx, ref in (("dQ", 0, rq), ("dK", 1, rk), ("dV", 2, rv)):
+        g = np.concatenate([x[:, :, idx, :] for x in got], axis=2)
+        assert_close(g.reshape(seq * batch, h), ref.reshape(seq * batch, h), TOL_BF16, name)

@@ -86,3 +86,40 @@ def test_sp_mlp_full_size_sampled():
     assert_close(host(Y)[rows], ref["Y"], TOL_BF16, "Y rows")
     rb = O.sp_mlp_bwd(Xr, g64, W1f, W2f, ref, O.f64(dY[rows]))
     assert_close(host(dX)[rows], rb["dX"], TOL_BF16, "dX rows")
+
+
+def test_mlp_7b_swiglu_full_size_sampled_fused():
+    """The same full-size check with the shard sums fused into the row GEMM and
+    the column-backward dX GEMM."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 32768, 4096, 11008, 8
+    inp = tp_synth.draw_mlp(T, h, f, "swiglu", torch.bfloat16, seed=0)
+    m = TPMLP(h, f, p, "swiglu", "bf16", fused=True)
+    m.load_weights(dev(inp.W1), dev(inp.W2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    rows = _rows(T, 48)
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    ref = O.mlp_fwd_rows(X, W1, None, W2, None, "swiglu", rows)
+    assert_close(host(Y)[rows], ref["Y"], TOL_BF16, "Y rows")
+    smp = O.mlp_bwd_sampled(X, W1, None, W2, dY, "swiglu", rows, np.array([0, 5000, 11007]))
+    assert_close(host(dX)[rows], smp["dX_rows"], TOL_BF16, "dX rows")
+
+
+def test_sp_mlp_reduced_size_fused():
+    from megatron_tensor_transformer_gemm_b200.block import SPMLP
+    seq, h, f, p = 512, 1024, 3584, 8
+    X, g, b, W1, W2, dY = tp_synth.draw_sp_mlp(seq, h, f, p, torch.bfloat16, seed=4, ln_affine_random=True)
+    sp = SPMLP(h, f, p, "swiglu", fused=True)
+    sp.mlp.load_weights(dev(W1), dev(W2))
+    sp.gamma.copy_(dev(g))
+    sp.beta.copy_(dev(b))
+    t = seq // p
+    Y = torch.cat(sp.forward([dev(X[j * t:(j + 1) * t]) for j in range(p)]), 0)
+    dX = torch.cat(sp.backward([dev(dY[j * t:(j + 1) * t]) for j in range(p)]), 0)
+    X, g, b, W1, W2, dY = (O.f64(x) for x in (X, g, b, W1, W2, dY))
+    ref = O.sp_mlp_fwd(X, g, b, W1, W2)
+    rb = O.sp_mlp_bwd(X, g, W1, W2, ref, dY)
+    assert_close(Y, ref["Y"], TOL_BF16, "Y")
+    assert_close(dX, rb["dX"], TOL_BF16, "dX")
+    assert_close(sp.dgamma[None, :], rb["dg"][None, :], TOL_BF16, "dgamma")

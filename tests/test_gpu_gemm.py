@@ -208,3 +208,71 @@ def test_bf16_mlp_end_to_end_small(act, bias):
     dW2 = torch.empty(W2.shape, dtype=torch.bfloat16, device="cuda")
     m.plan.unshard_row("mlp", m.dW2, dW2)
     assert_close(dW2, g["dW2"], TOL_BF16, "dW2")
+
+
+@pytest.mark.parametrize("T,K,h,p", [(300, 264, 192, 2), (257, 1376, 512, 8), (64, 128, 256, 1)])
+def test_row_forward_fused_reduce(T, K, h, p):
+    """The row GEMM with the shard sum fused: sum_i H_i W2_i^T + b + residual."""
+    tp = _tp()
+    g = torch.Generator().manual_seed(T + 11)
+    Hs = [torch.randn(T, K, generator=g).to(torch.bfloat16) for _ in range(p)]
+    W2 = (torch.randn(h, K * p, generator=g) * 0.02).to(torch.bfloat16)
+    b = (torch.rand(h, generator=g) * 0.2 - 0.1).to(torch.bfloat16)
+    r = torch.randn(T, h, generator=g).to(torch.bfloat16)
+    plan = tp.Plan(h, K * p, 0, p, "bf16", "gelu")
+    W2s = [_empty(h, K) for _ in range(p)]
+    plan.shard_row("mlp", dev(W2), W2s)
+    Y = _empty(T, h)
+    plan.row_fwd_reduce("mlp", T, [dev(x) for x in Hs], W2s, dev(b), dev(r), Y)
+    P = [O.row_partial(O.f64(Hs[i]), O.shard_cols(O.f64(W2), p, i)) for i in range(p)]
+    ref = O.reduce_partials(P, O.f64(b), O.f64(r))
+    assert_close(Y, ref, TOL_BF16, "fused row fwd")
+    if T % p == 0:
+        t = T // p
+        Ys = [_empty(t, h) for _ in range(p)]
+        rs = [dev(r[j * t:(j + 1) * t]) for j in range(p)]
+        plan.row_fwd_reduce_scatter_seq("mlp", T, [dev(x) for x in Hs], W2s, dev(b), rs, Ys)
+        refs = O.reduce_scatter_seq(P, O.f64(b), [O.f64(r[j * t:(j + 1) * t]) for j in range(p)])
+        for j in range(p):
+            assert_close(Ys[j], refs[j], TOL_BF16, f"fused RS shard {j}")
+
+
+@pytest.mark.parametrize("T,h,f,p,act", [(300, 192, 528, 2, "gelu"), (256, 256, 272, 2, "swiglu")])
+def test_column_backward_fused_reduce(T, h, f, p, act):
+    tp = _tp()
+    g = torch.Generator().manual_seed(T + 12)
+    n = (2 if act == "swiglu" else 1) * f // p
+    Wfull = (torch.randn(n * p, h, generator=g) * 0.05).to(torch.bfloat16)
+    X = torch.randn(T, h, generator=g).to(torch.bfloat16)
+    dZs = [torch.randn(T, n, generator=g).to(torch.bfloat16) for _ in range(p)]
+    plan = tp.Plan(h, f, 0, p, "bf16", act)
+    Ws = [_empty(n, h) for _ in range(p)]
+    plan.shard_column("mlp", dev(Wfull), Ws)
+    dX = _empty(T, h)
+    plan.column_bwd_reduce("mlp", T, dev(X), [dev(z) for z in dZs], Ws, None, None, dX)
+    Wf = O.f64(Wfull)
+    parts = [O.column_bwd_shard(O.f64(X), O.f64(dZs[i]), _shard_w1(Wf, act, p, i))[2] for i in range(p)]
+    assert_close(dX, O.reduce_partials(parts), TOL_BF16, "fused dX")
+    t = T // p
+    dXs = [_empty(t, h) for _ in range(p)]
+    plan.column_bwd_reduce_scatter_seq("mlp", T, dev(X), [dev(z) for z in dZs], Ws, None, None, dXs)
+    refs = O.reduce_scatter_seq(parts)
+    for j in range(p):
+        assert_close(dXs[j], refs[j], TOL_BF16, f"fused dX RS shard {j}")
+
+
+@pytest.mark.parametrize("act,bias", [("gelu", True), ("swiglu", False)])
+def test_bf16_mlp_end_to_end_small_fused(act, bias):
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 384, 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=6, bias=bias)
+    m = TPMLP(h, f, p, act, "bf16", bias=bias, fused=True)
+    m.load_weights(dev(inp.W1), dev(inp.W2), dev(inp.b1), dev(inp.b2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    b1, b2 = (O.f64(inp.b1), O.f64(inp.b2)) if bias else (None, None)
+    ref = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    gr = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
+    assert_close(Y, ref["Y"], TOL_BF16, "Y")
+    assert_close(dX, gr["dX"], TOL_BF16, "dX")
