@@ -25,6 +25,8 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -37,20 +39,29 @@ using namespace tpd;
 using tpi::GemmBatch;
 using tpi::GemmProblem;
 
-constexpr int BM = 128;
+constexpr int BM = 128;  // accumulator rows per CTA
 constexpr int BN = 256;
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
 constexpr int UMMA_K = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int kBarBytes = 256;
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + kBarBytes;
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64-wide MN block of an MN-major tile
+
+// Per-CTA tile geometry. PAIR = 1: one CTA computes a 128 x 256 tile.
+// PAIR = 2: a (2,1,1) cluster computes a 256 x 256 tile with cta_group::2
+// MMAs; each CTA loads its 128 rows of A and its 128 rows of B.
+template <int PAIR>
+struct Cfg {
+  static constexpr int TILE_M = BM * PAIR;
+  static constexpr int B_ROWS = BN / PAIR;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR == 1 ? 4 : 6;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + kBarBytes;
+};
 
 struct GroupArgs {
   int M, N, K;
@@ -246,13 +257,16 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
 }
 
 // -------------------------------------------------------------------- kernel
+template <int PAIR>
 __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<PAIR>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -262,6 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;  // 0 = MMA leader of the pair
+  const int first_tile = static_cast<int>(blockIdx.x) / PAIR;
+  const int tile_stride = static_cast<int>(gridDim.x) / PAIR;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -270,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], PAIR * kEpiWarps);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -284,11 +301,17 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR == 2) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync_all();  // the peer's barriers are initialised before any signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -300,12 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+    for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
       const GroupArgs& ga = p.g[g];
-      const int m0 = mt * BM;
+      const int m0 = mt * C::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
+      const int nb0 = n0 + static_cast<int>(rank) * C::B_ROWS;      // this CTA's B rows
       const int nseg = p.kcat ? p.kcat : 1;
       for (int sg = 0; sg < nseg && ok; ++sg) {
         const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
@@ -315,26 +339,50 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           const int k0 = kb * BK;
-          uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
-          if (!p.a_mn) {
-            tma_load_2d(a_dst, &p.tmA[gi], &full[stage], k0, m0);
-          } else {
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+          if (PAIR == 1) {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            if (!p.a_mn) {
+              tma_load_2d(a_dst, &p.tmA[gi], &full[stage], k0, m0);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BM / 64; ++c)
-              tma_load_2d(a_dst + c * MN_BLOCK_BYTES, &p.tmA[gi], &full[stage], m0 + c * 64, k0);
-          }
-          if (p.epi == tpi::EPI_SWIGLU) {
-            tma_load_3d(b_dst, &p.tmB[gi], &full[stage], k0, n0, 0);
-            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[gi], &full[stage], k0, n0, 1);
-          } else if (!p.b_mn) {
-            tma_load_2d(b_dst, &p.tmB[gi], &full[stage], k0, n0);
-          } else {
+              for (int c = 0; c < BM / 64; ++c)
+                tma_load_2d(a_dst + c * MN_BLOCK_BYTES, &p.tmA[gi], &full[stage], m0 + c * 64, k0);
+            }
+            if (p.epi == tpi::EPI_SWIGLU) {
+              tma_load_3d(b_dst, &p.tmB[gi], &full[stage], k0, n0, 0);
+              tma_load_3d(b_dst + C::B_BYTES / 2, &p.tmB[gi], &full[stage], k0, n0, 1);
+            } else if (!p.b_mn) {
+              tma_load_2d(b_dst, &p.tmB[gi], &full[stage], k0, n0);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], &full[stage], n0 + c * 64, k0);
+              for (int c = 0; c < BN / 64; ++c)
+                tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], &full[stage], n0 + c * 64, k0);
+            }
+          } else {
+            // Both CTAs' copies complete on the leader's full barrier, which
+            // expects the bytes of the whole pair.
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], PAIR * C::STAGE_BYTES);
+            const uint32_t fb = map_shared(smem_u32(&full[stage]), 0);
+            if (!p.a_mn) {
+              tma_load_2d_pair(a_dst, &p.tmA[gi], fb, k0, m0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < BM / 64; ++c)
+                tma_load_2d_pair(a_dst + c * MN_BLOCK_BYTES, &p.tmA[gi], fb, m0 + c * 64, k0);
+            }
+            if (p.epi == tpi::EPI_SWIGLU) {
+              // rank 0 holds the 128 gate rows, rank 1 the matching 128 up rows
+              tma_load_3d_pair(b_dst, &p.tmB[gi], fb, k0, n0, static_cast<int>(rank));
+            } else if (!p.b_mn) {
+              tma_load_2d_pair(b_dst, &p.tmB[gi], fb, k0, nb0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < C::B_ROWS / 64; ++c)
+                tma_load_2d_pair(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], fb, nb0 + c * 64, k0);
+            }
           }
           last_parity[stage] = static_cast<int>(phase);
           if (++stage == STAGES) {
@@ -344,19 +392,22 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
         }
       }
     }
-    // Drain: every copy this thread issued has landed before the CTA exits.
-    for (int s = 0; s < STAGES; ++s)
-      if (last_parity[s] >= 0)
-        mbar_wait(&full[s], static_cast<uint32_t>(last_parity[s]), abort_flag, p.status);
-  } else if (warp == 1 && lane == 0) {
+    // Drain: every copy of this CTA (and, for the leader, of the pair) has
+    // landed before the CTA exits. The peer's copies complete on the leader's
+    // barriers, which the leader drains.
+    if (rank == 0)
+      for (int s = 0; s < STAGES; ++s)
+        if (last_parity[s] >= 0)
+          mbar_wait(&full[s], static_cast<uint32_t>(last_parity[s]), abort_flag, p.status);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_bf16(BM, BN, p.a_mn != 0, p.b_mn != 0);
+    const uint32_t idesc = idesc_bf16(C::TILE_M, BN, p.a_mn != 0, p.b_mn != 0);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+    for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
       int num_kb = p.g[g].num_kb;
@@ -373,8 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
-        const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+        const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t adesc =
@@ -383,42 +434,52 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
           const uint64_t bdesc =
               p.b_mn ? smem_desc_sw128(b_base + k * (UMMA_K * 128), MN_BLOCK_BYTES, 1024)
                      : smem_desc_sw128(b_base + k * (UMMA_K * 2), 16, 1024);
-          tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          if (PAIR == 2) tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          else tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
         }
-        tc_commit(&empty[stage]);  // frees the smem stage when these MMAs finish
+        // frees the smem stage (in both CTAs of a pair) when these MMAs finish
+        if (PAIR == 2) tc_commit_pair_mc(&empty[stage], 0x3);
+        else tc_commit(&empty[stage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      tc_commit(&tfull[acc]);  // accumulator ready for the epilogue
+      // accumulator ready for the epilogue (of both CTAs of a pair)
+      if (PAIR == 2) tc_commit_pair_mc(&tfull[acc], 0x3);
+      else tc_commit(&tfull[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    // Drain: no MMA of this CTA is in flight when TMEM is released.
-    tc_commit(drain);
+    // Drain: no MMA of this CTA (pair) is in flight when TMEM is released.
+    if (PAIR == 2) tc_commit_pair_mc(drain, 0x1);
+    else tc_commit(drain);
     mbar_wait(drain, 0, abort_flag, p.status);
   } else if (warp >= 2) {
     // ------------------------------------------------------------- epilogue
-    const int lg = warp & 3;  // TMEM lane quarter this warp may access
+    const int lg = warp & 3;          // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;  // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+    const uint32_t tempty_leader = PAIR == 2 ? map_shared(smem_u32(&tempty[0]), 0) : 0u;
+    for (int t = first_tile; t < p.total_tiles; t += tile_stride) {
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
       const GroupArgs& ga = p.g[g];
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const int row = mt * BM + lg * 32 + lane;
+      const int row = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32 + lane;
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       epilogue_tile(p, ga, taddr, row, n0, half);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR == 2) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
+        else mbar_arrive(&tempty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -426,9 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) cluster_sync_all();  // neither CTA leaves while its pair may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -465,6 +528,44 @@ tp_status encode_gateup(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint
   return TP_OK;
 }
 
+// CTA pairing of the bf16 GEMM: 2 (cta_group::2, 256-row tiles) unless the
+// environment variable TP_GEMM_CTA_PAIR is "1" (one CTA per 128-row tile).
+int gemm_pair() {
+  const char* e = getenv("TP_GEMM_CTA_PAIR");
+  return (e && e[0] == '1') ? 1 : 2;
+}
+
+template <int PAIR>
+tp_status launch_kernel(const GemmParams& p, int tiles, int sms, cudaStream_t st) {
+  using C = Cfg<PAIR>;
+  static bool attr_set[2] = {false, false};
+  if (!attr_set[PAIR - 1]) {
+    tp_status s = tpi::cuda_status(
+        cudaFuncSetAttribute(tp_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES),
+        "cudaFuncSetAttribute(gemm smem)");
+    if (s != TP_OK) return s;
+    attr_set[PAIR - 1] = true;
+  }
+  const int clusters = std::max(1, std::min(tiles, sms / PAIR));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(clusters * PAIR);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  tp_status s = tpi::cuda_status(cudaLaunchKernelEx(&cfg, tp_gemm_kernel<PAIR>, p),
+                                 "cudaLaunchKernelEx(gemm)");
+  if (s != TP_OK) return s;
+  return tpi::after_launch(PAIR == 2 ? "gemm_bf16 (tcgen05, CTA pair)" : "gemm_bf16 (tcgen05)");
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -490,6 +591,8 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   memset(&p, 0, sizeof(p));
   const bool swiglu = b.epi == EPI_SWIGLU;
   const int tile_n = swiglu ? BN / 2 : BN;
+  const int pair = gemm_pair();
+  const int tile_m = BM * pair;
   if (b.kcat && b.epi != EPI_STORE)
     return fail(TP_ERR_ARG, "K-concatenated GEMM supports the plain epilogue only");
   int tiles = 0;
@@ -522,7 +625,7 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
       a.bias = o.bias;
       a.aux = o.aux;
       a.ldaux = o.ldaux;
-      const int64_t t = static_cast<int64_t>((o.M + BM - 1) / BM) * a.tiles_n;
+      const int64_t t = static_cast<int64_t>((o.M + tile_m - 1) / tile_m) * a.tiles_n;
       if (tiles + t > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "too many GEMM tiles");
       tiles += static_cast<int>(t);
     }
@@ -533,7 +636,7 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     if (s != TP_OK) return s;
     // B operand
     if (swiglu) s = encode_gateup(enc, &p.tmB[i], g.B, g.K, o.nh, g.ldb);
-    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, o.N, g.ldb, BN);
+    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, o.N, g.ldb, BN / pair);
     else s = encode_2d(enc, &p.tmB[i], g.B, o.N, g.K, g.ldb, BK);
     if (s != TP_OK) return s;
   }
@@ -555,17 +658,8 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   p.out_f32 = b.out_f32;
   s = device_status_word(&p.status);
   if (s != TP_OK) return s;
-  static bool attr_set = false;
-  if (!attr_set) {
-    s = cuda_status(cudaFuncSetAttribute(tp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES),
-                    "cudaFuncSetAttribute(gemm smem)");
-    if (s != TP_OK) return s;
-    attr_set = true;
-  }
-  const int grid = std::min(tiles, device_sms());
-  tp_gemm_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(p);
-  return after_launch("gemm_bf16 (tcgen05)");
+  if (pair == 2) return launch_kernel<2>(p, tiles, device_sms(), st);
+  return launch_kernel<1>(p, tiles, device_sms(), st);
 }
 
 }  // namespace tpi
