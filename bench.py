@@ -381,15 +381,34 @@ def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
 
+def gemm_source_hash():
+    """sha256 of the GEMM kernel sources: ncu traffic figures taken on other
+    sources are not reported."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("tp_gemm_sm100.cu", "tp_device.cuh"):
+        with open(os.path.join(ROOT, "megatron_tensor_transformer_gemm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(T, variant):
+    """DRAM bytes per GEMM launch (mean over the six launches of one step) from
+    the committed ncu capture, if it was taken on this workload, variant and
+    kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        return None
+    if d.get("tokens") != T or d.get("variant") != variant or d.get("source_sha256") != gemm_source_hash():
+        return None
+    return d.get("bytes_per_launch")
+
+
 def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t, red_gbs,
            red_bytes, e2e, launches, clk, status, red_where):
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(tr_path):
-        try:
-            traffic = json.load(open(tr_path)).get("bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = measured_traffic(T, args.variant)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(rows=args.cpu_rows)
@@ -425,6 +444,113 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
     return 0
 
 
+def run_other(args, world, rank, local):
+    """Device-timed throughput of the other workloads (parity cases of the
+    suite), printed in the same JSON form: the attention block forward
+    (hidden 4096, 32 heads x 128, seq 4096, batch 2, p 8), the Megatron-SP
+    SwiGLU MLP fwd+bwd (hidden 8192, ffn 28672, seq 8192, p 8) and the
+    12-layer stack fwd+bwd (hidden 512, MLP 2048, 8 heads, tokens 8x512, p 4)."""
+    import torch
+    import tp_synth
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.block import SPMLP, TPAttention, TPLayer
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    if args.workload == "attn":
+        b, s, h, H, p = 2, 4096, 4096, 32, 8
+        a = tp_synth.draw_attn_block(b, s, h, torch.bfloat16, seed=rank)
+        blk = TPAttention(h, H, p, dev)
+        blk.load_weights(a.Wqkv.to(dev), a.Wo.to(dev))
+        X = a.X.to(dev)
+        flops = blk.flops_fwd(b, s)
+        step = lambda: blk.forward(X, b, s, residual=X)
+        name = "attention block fwd: hidden 4096, 32 heads x 128, seq 4096, batch 2, p=8, causal"
+        # attention-core launches alone, for the roofline of the dominant kernel
+        core = lambda: blk.plan.attention_fwd(b, s, blk.QKV, blk.O, blk.LSE)
+        core_flops = 4.0 * b * H * (s * (s + 1) / 2) * (h // H)
+    elif args.workload == "sp":
+        s_, h, f, p = 8192, 8192, 28672, 8
+        X, g, be, W1, W2, dY = tp_synth.draw_sp_mlp(s_, h, f, p, torch.bfloat16, seed=rank)
+        sp = SPMLP(h, f, p, "swiglu", dev, fused=args.variant == "fused")
+        sp.mlp.load_weights(W1.to(dev), W2.to(dev))
+        t = s_ // p
+        Xs = [X[j * t:(j + 1) * t].to(dev) for j in range(p)]
+        dYs = [dY[j * t:(j + 1) * t].to(dev) for j in range(p)]
+        flops = sp.flops(s_)
+
+        def step():
+            sp.forward(Xs)
+            sp.backward(dYs)
+        name = "Megatron-SP SwiGLU MLP fwd+bwd: hidden 8192, ffn 28672, seq 8192, batch 1, p=8"
+        core, core_flops = None, None
+    else:
+        L, b, s_, h, f, H, p = 12, 8, 512, 512, 2048, 8, 4
+        X, layers, dY = tp_synth.draw_block_stack(L, b, s_, h, f, torch.bfloat16, seed=rank)
+        lays = []
+        for prm in layers:
+            lay = TPLayer(h, f, H, p, dev)
+            lay.load(type(prm)(**{k: getattr(prm, k).to(dev) for k in prm.__dataclass_fields__}))
+            lays.append(lay)
+        Xd, dYd = X.to(dev), dY.to(dev)
+        T = b * s_
+        per_layer = (3.0 * (2.0 * T * h * f * 2) + 3.0 * (2.0 * T * h * 3 * h + 2.0 * T * h * h)
+                     + 3.0 * 4.0 * b * H * (s_ * (s_ + 1) / 2) * (h // H) * 1.0)
+        flops = L * per_layer
+
+        def step():
+            x = Xd
+            for lay in lays:
+                x = lay.forward(x, b, s_)
+            g = dYd
+            for lay in reversed(lays):
+                g = lay.backward(g, b, s_)
+        name = "12-layer block stack fwd+bwd: hidden 512, MLP 2048, 8 heads x 64, tokens 8x512, p=4"
+        core, core_flops = None, None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    tp.launch_count(reset=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = tp.launch_count(reset=True)
+    clk = clocks.stop()
+    value, ms = aggregate(flops, args.steps, e0.elapsed_time(e1), world)
+    roof = None
+    if core is not None:
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            core()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        ach = core_flops * args.steps / (c0.elapsed_time(c1) / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": "attn_fwd_kernel (tcgen05)", "achieved": ach,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "peak_kind": f"bf16 burst ({peaks['source']}; timed alone)", "traffic": None}
+    if rank != 0:
+        return 0
+    print(json.dumps({"metric": f"{args.workload} TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded tp_synth)",
+                      "config": {"workload": name, "variant": args.variant}, "roofline": roof,
+                      "gpu_launches": launches, "clocks": clk,
+                      "device_status": tp.device_status()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,6 +565,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--variant", choices=["fused", "partials"], default="fused",
                     help="sum over shards inside the GEMMs (fused) or via p partials + reduce")
+    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack"], default="mlp7b",
+                    help="mlp7b (the metric's workload) or another config of the suite")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -447,7 +575,7 @@ def main():
         # The oracle runs on rank 0's host cores only; no GPU or process group needed.
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
     world, rank, local = dist_setup()
-    rc = run_ours(args, world, rank, local)
+    rc = run_ours(args, world, rank, local) if args.workload == "mlp7b" else run_other(args, world, rank, local)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -22,7 +22,7 @@ def declared_functions():
     return sorted(set(re.findall(r"TP_API\s+[\w\s\*]+?\b(tp_\w+)\s*\(", src)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_layer_and_collective_calls():
     names = declared_functions()
     for must in ["tp_plan_create", "tp_column_fwd", "tp_row_fwd_partial", "tp_reduce_partials",
                  "tp_reduce_scatter_seq", "tp_all_gather_seq", "tp_row_bwd", "tp_column_bwd",
