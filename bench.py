@@ -453,7 +453,7 @@ def run_other(args, world, rank, local):
     import torch
     import tp_synth
     from megatron_tensor_transformer_gemm_b200 import tp
-    from megatron_tensor_transformer_gemm_b200.block import SPMLP, TPAttention, TPLayer
+    from megatron_tensor_transformer_gemm_b200.block import CapturedStep, SPMLP, TPAttention, TPLayer
 
     peaks = load_peaks()
     dev = torch.device("cuda", local)
@@ -511,6 +511,13 @@ def run_other(args, world, rank, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    graph = None
+    if args.graph:
+        graph = CapturedStep(step)
+        step = graph
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
@@ -524,6 +531,8 @@ def run_other(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     launches = tp.launch_count(reset=True)
+    if graph is not None:
+        launches = graph.launches * args.steps  # replays launch the captured kernels
     clk = clocks.stop()
     value, ms = aggregate(flops, args.steps, e0.elapsed_time(e1), world)
     roof = None
@@ -545,7 +554,8 @@ def run_other(args, world, rank, local):
                       "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                       "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                       "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded tp_synth)",
-                      "config": {"workload": name, "variant": args.variant}, "roofline": roof,
+                      "config": {"workload": name, "variant": args.variant,
+                                 "cuda_graph": bool(args.graph)}, "roofline": roof,
                       "gpu_launches": launches, "clocks": clk,
                       "device_status": tp.device_status()}), flush=True)
     return 0
@@ -567,6 +577,8 @@ def main():
                     help="sum over shards inside the GEMMs (fused) or via p partials + reduce")
     ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack"], default="mlp7b",
                     help="mlp7b (the metric's workload) or another config of the suite")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step as one captured CUDA graph (other workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -336,3 +336,29 @@ class TPLayer:
                          self.dln1_g, self.dln1_b)
         ln.reduce_partials(T, [self.dx1, self.dx_ln], None, None, self.dx)
         return self.dx
+
+
+class CapturedStep:
+    """A step (a callable that only issues libtp.so launches on the current
+    stream) captured once into a CUDA graph and replayed: one graph launch
+    instead of one host call per kernel. The step runs eagerly `warmup` times
+    first, on the capture stream, so every workspace the library allocates on
+    first use exists before capture starts."""
+
+    def __init__(self, fn, warmup: int = 2):
+        from .tp import launch_count
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        before = launch_count()
+        with torch.cuda.graph(self.graph):
+            fn()
+        self.launches = launch_count() - before  # kernel launches per replay
+
+    def __call__(self):
+        self.graph.replay()

@@ -2,20 +2,25 @@
 // tensor cores (TP walkthrough 2kiu.com §3.1: every shard runs full-sequence
 // attention on its own whole heads, with no cross-shard step).
 //
-// One CTA computes one 128-query tile of one (shard, batch, head):
-//   warp 0      TMA producer: the Q tile once, then K and V blocks of 128 keys
-//               into a 2-stage ring (3-D tensor map over the sequence-major
-//               [seq, batch, 3*heads_local*d] QKV buffer of the shard)
-//   warp 1      TMEM allocator + MMA issuer: S = Q K^T (128 x 128, fp32 in
-//               TMEM), then O_j = P V_j (128 x d, fp32 in TMEM)
-//   warps 2..5  softmax: thread r owns query row r; two passes over its row of
-//               S in TMEM (row max, then exp2 and the row sum), P rounded to
-//               bf16 and written to shared memory in the 128-byte-swizzled
-//               K-major layout the PV MMA reads; O and the online-softmax
-//               state (m, l) stay in registers and are rescaled per block.
-// Blocks are causal: the tile's last key block is the diagonal one and is
-// masked (key > query -> probability 0); keys and queries past seq are masked.
-// The backward (tp_attention_bwd.cu) recomputes P from the saved row log-sum-exp.
+// One CTA computes two adjacent 128-query tiles (A = 2i, B = 2i + 1) of one
+// (shard, batch, head); both read every K/V block once from shared memory:
+//   warp 0      TMA producer: both Q tiles, then each 128-key block's K and V
+//               (single buffers released separately, so K_{j+1} loads while
+//               block j's softmax and P.V run) from a 3-D tensor map over the
+//               sequence-major [seq, batch, 3*heads_local*d] QKV of the shard
+//   warp 1      TMEM allocator + MMA issuer, ping-pong order: S_A(0), S_B(0),
+//               then per block PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one
+//               tile's MMAs run while the other tile's softmax works
+//   warps 2..5  softmax of tile A, warps 6..9 of tile B: thread r owns query
+//               row r; two passes over its row of S in TMEM (row max, then
+//               exp2 and the row sum), P rounded to bf16 and written to shared
+//               memory in the 128-byte-swizzled K-major layout of the PV MMA.
+// O accumulates in TMEM across key blocks. P is taken relative to a reference
+// max m that is raised (and O, l rescaled in place) only when a row's max
+// exceeds it by more than 2^8; P <= 2^8 stays exact in fp32/bf16 range and the
+// final O / l is independent of the reference, so this is exact, not an
+// approximation. Blocks are causal: the diagonal block of each tile is masked
+// (key > query -> probability 0); keys and queries past seq are masked.
 #include <cuda.h>
 
 #include <algorithm>
@@ -31,19 +36,19 @@ using namespace tpd;
 using tpi::MutPtrArray;
 using tpi::PtrArray;
 
-constexpr int BQ = 128;        // queries per tile
-constexpr int BKV = 128;       // keys per block
-constexpr int KV_STAGES = 2;
-constexpr int kThreads = 192;
+constexpr int BQ = 128;   // queries per tile
+constexpr int BKV = 128;  // keys per block
+constexpr int kThreads = 320;
 constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-atom column)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;  // raise the reference max when exceeded by > 2^8
 
 struct AttnParams {
   CUtensorMap tm[TP_MAX_SHARDS];  // QKV_i as {3*Hl*d, batch, seq}, box {64, 1, 128}
   void* O[TP_MAX_SHARDS];
   float* lse[TP_MAX_SHARDS];
   int p, batch, seq, heads_local, d;
-  int n_qtiles;
+  int n_qtiles, n_pairs;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned* status;
 };
@@ -53,7 +58,7 @@ struct AttnSmem {
   static constexpr int Q_BYTES = BQ * D * 2;
   static constexpr int KV_BYTES = BKV * D * 2;
   static constexpr int P_BYTES = BQ * BKV * 2;
-  static constexpr int TOTAL = 1024 + Q_BYTES + 2 * KV_STAGES * KV_BYTES + P_BYTES + 256;
+  static constexpr int TOTAL = 1024 + 2 * Q_BYTES + 2 * KV_BYTES + 2 * P_BYTES + 256;
 };
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -66,192 +71,244 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + SM::Q_BYTES;
-  uint8_t* sV = sK + KV_STAGES * SM::KV_BYTES;
-  uint8_t* sP = sV + KV_STAGES * SM::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + SM::P_BYTES);
+  uint8_t* sQ = smem;                     // [2] tiles
+  uint8_t* sK = sQ + 2 * SM::Q_BYTES;
+  uint8_t* sV = sK + SM::KV_BYTES;
+  uint8_t* sP = sV + SM::KV_BYTES;        // [2] tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SM::P_BYTES);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                  // [KV_STAGES]
-  uint64_t* v_full = k_full + KV_STAGES;        // [KV_STAGES]
-  uint64_t* kv_empty = v_full + KV_STAGES;      // [KV_STAGES]
-  uint64_t* s_full = kv_empty + KV_STAGES;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* o_full = p_full + 1;
-  uint64_t* o_empty = o_full + 1;
-  uint64_t* drain = o_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* s_full = bars + 5;   // [2]
+  uint64_t* p_full = bars + 7;   // [2]
+  uint64_t* o_done = bars + 9;   // [2]
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Tile decode: heaviest (last) query tiles first.
-  const int per_qt = p.p * p.batch * p.heads_local;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / per_qt;
-  int rest = static_cast<int>(blockIdx.x) % per_qt;
+  // Work decode: heaviest (last) tile pairs first.
+  const int per = p.p * p.batch * p.heads_local;
+  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x) / per;
+  int rest = static_cast<int>(blockIdx.x) % per;
   const int hh = rest % p.heads_local;
   rest /= p.heads_local;
   const int b = rest % p.batch;
   const int shard = rest / p.batch;
-  const int q0 = qt * BQ;
   const int n_kv_total = (p.seq + BKV - 1) / BKV;
-  const int nb = min(qt + 1, n_kv_total);  // causal: key blocks 0..qt
+  int nbt[2];
+  int q0t[2];
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * pair + t;
+    q0t[t] = qt * BQ;
+    nbt[t] = qt < p.n_qtiles ? min(qt + 1, n_kv_total) : 0;  // causal: key blocks 0..qt
+  }
+  const int nb = max(nbt[0], nbt[1]);
   const int hl_d = p.heads_local * D;
   const CUtensorMap* tm = &p.tm[shard];
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&o_done[t], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(o_full, 1);
-    mbar_init(o_empty, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;        // columns [0, 128)
-  const uint32_t tO = tmem + 128;  // columns [128, 128 + D)
+  // S of tile t in columns [128 t, 128 t + 128); O of tile t in [256 + D t, 256 + D (t + 1)).
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------- producer
     tma_prefetch_desc(tm);
-    mbar_arrive_expect_tx(q_full, SM::Q_BYTES);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c)
-      tma_load_3d(sQ + c * CHUNK_BYTES, tm, q_full, hh * D + c * 64, b, q0);
-    int last_par[KV_STAGES];
-    for (int s = 0; s < KV_STAGES; ++s) last_par[s] = -1;
-    for (int j = 0; j < nb; ++j) {
-      const int st = j % KV_STAGES;
-      const uint32_t ph = static_cast<uint32_t>(j / KV_STAGES) & 1u;
-      if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status)) break;
-      const int k0 = j * BKV;
-      mbar_arrive_expect_tx(&k_full[st], SM::KV_BYTES);
+    mbar_arrive_expect_tx(q_full, (nbt[1] > 0 ? 2 : 1) * SM::Q_BYTES);
+    for (int t = 0; t < 2; ++t) {
+      if (nbt[t] == 0) continue;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sK + st * SM::KV_BYTES + c * CHUNK_BYTES, tm, &k_full[st],
-                    hl_d + hh * D + c * 64, b, k0);
-      mbar_arrive_expect_tx(&v_full[st], SM::KV_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sV + st * SM::KV_BYTES + c * CHUNK_BYTES, tm, &v_full[st],
-                    2 * hl_d + hh * D + c * 64, b, k0);
-      last_par[st] = static_cast<int>(ph);
+        tma_load_3d(sQ + t * SM::Q_BYTES + c * CHUNK_BYTES, tm, q_full, hh * D + c * 64, b, q0t[t]);
     }
-    mbar_wait(q_full, 0, abort_flag, p.status);
-    for (int s = 0; s < KV_STAGES; ++s)
-      if (last_par[s] >= 0) {
-        mbar_wait(&k_full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
-        mbar_wait(&v_full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
+    int issued = 0;
+    for (int j = 0; j < nb; ++j) {
+      const uint32_t ph = static_cast<uint32_t>(j) & 1u;
+      const int k0 = j * BKV;
+      if (!mbar_wait(k_empty, ph ^ 1u, abort_flag, p.status)) break;
+      mbar_arrive_expect_tx(k_full, SM::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sK + c * CHUNK_BYTES, tm, k_full, hl_d + hh * D + c * 64, b, k0);
+      if (!mbar_wait(v_empty, ph ^ 1u, abort_flag, p.status)) {
+        issued = -(j + 1);  // K of block j issued, V not
+        break;
       }
+      mbar_arrive_expect_tx(v_full, SM::KV_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sV + c * CHUNK_BYTES, tm, v_full, 2 * hl_d + hh * D + c * 64, b, k0);
+      issued = j + 1;
+    }
+    // Drain: every copy issued has landed before the CTA exits.
+    mbar_wait(q_full, 0, abort_flag, p.status);
+    const int nk = issued >= 0 ? issued : -issued;
+    const int nv = issued >= 0 ? issued : -issued - 1;
+    if (nk > 0) mbar_wait(k_full, static_cast<uint32_t>(nk - 1) & 1u, abort_flag, p.status);
+    if (nv > 0) mbar_wait(v_full, static_cast<uint32_t>(nv - 1) & 1u, abort_flag, p.status);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
     const uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
-    const uint32_t q_base = smem_u32(sQ), p_base = smem_u32(sP);
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-    auto issue_s = [&](int j) -> bool {
-      const int st = j % KV_STAGES;
-      if (!mbar_wait(&k_full[st], static_cast<uint32_t>(j / KV_STAGES) & 1u, abort_flag, p.status))
-        return false;
-      tc_fence_after();
-      const uint32_t k_base = smem_u32(sK + st * SM::KV_BYTES);
+    const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+    auto issue_s = [&](int t) {
+      const uint32_t q_base = smem_u32(sQ + t * SM::Q_BYTES);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk / 4) * CHUNK_BYTES + (kk % 4) * 32;
-        tc_mma_bf16(tS, smem_desc_sw128(q_base + off, 16, 1024),
+        tc_mma_bf16(tmem + 128 * t, smem_desc_sw128(q_base + off, 16, 1024),
                     smem_desc_sw128(k_base + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
       }
-      tc_commit(s_full);
-      return true;
+      tc_commit(&s_full[t]);
     };
-    if (ok && nb > 0) ok = issue_s(0);
-    for (int j = 0; ok && j < nb; ++j) {
-      const int st = j % KV_STAGES;
-      const uint32_t ph = static_cast<uint32_t>(j) & 1u;
-      if (!mbar_wait(p_full, ph, abort_flag, p.status)) break;
-      if (!mbar_wait(&v_full[st], static_cast<uint32_t>(j / KV_STAGES) & 1u, abort_flag, p.status)) break;
-      if (!mbar_wait(o_empty, ph ^ 1u, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t v_base = smem_u32(sV + st * SM::KV_BYTES);
+    auto issue_pv = [&](int t, bool first) {
+      const uint32_t p_base = smem_u32(sP + t * SM::P_BYTES);
 #pragma unroll
       for (int kk = 0; kk < BKV / 16; ++kk) {
         const uint64_t adesc = smem_desc_sw128(p_base + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
         const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, CHUNK_BYTES, 1024);
-        tc_mma_bf16(tO, adesc, bdesc, idesc_o, kk > 0 ? 1u : 0u);
+        tc_mma_bf16(tmem + 256 + D * t, adesc, bdesc, idesc_o, (first && kk == 0) ? 0u : 1u);
       }
-      tc_commit(o_full);
-      tc_commit(&kv_empty[st]);
-      if (j + 1 < nb) ok = issue_s(j + 1);
+      tc_commit(&o_done[t]);
+    };
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full, 0, abort_flag, p.status);
+    if (ok) {
+      tc_fence_after();
+      for (int t = 0; t < 2; ++t)
+        if (nbt[t] > 0) issue_s(t);
+      tc_commit(k_empty);  // K_0 free once both S MMAs finish
+    }
+    for (int j = 0; ok && j < nb; ++j) {
+      if (!mbar_wait(v_full, static_cast<uint32_t>(j) & 1u, abort_flag, p.status)) break;
+      bool have_k_next = false;
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (j >= nbt[t]) continue;
+        if (!mbar_wait(&p_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(t, j == 0);
+        if (j + 1 < nbt[t]) {
+          if (!have_k_next) {
+            if (!mbar_wait(k_full, static_cast<uint32_t>(j + 1) & 1u, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            have_k_next = true;
+          }
+          issue_s(t);
+        }
+      }
+      if (!ok) break;
+      tc_commit(v_empty);                 // V_j free once both P.V MMAs finish
+      if (have_k_next) tc_commit(k_empty);  // K_{j+1} free once both S MMAs finish
     }
     tc_commit(drain);
     mbar_wait(drain, 0, abort_flag, p.status);
   } else if (warp >= 2) {
     // ------------------------------------------------------------- softmax
+    const int t = (warp - 2) / 4;  // query tile of this warpgroup
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
-    const int q = q0 + r;
+    const int q = q0t[t] + r;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-    float o[D];
-#pragma unroll
-    for (int i = 0; i < D; ++i) o[i] = 0.f;
+    const uint32_t tS = tmem + 128 * t + lane_off;
+    const uint32_t tO = tmem + 256 + D * t + lane_off;
+    uint8_t* sPt = sP + t * SM::P_BYTES;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nb && ok; ++j) {
-      const uint32_t ph = static_cast<uint32_t>(j) & 1u;
-      if (!mbar_wait(s_full, ph, abort_flag, p.status)) {
+    for (int j = 0; j < nbt[t] && ok; ++j) {
+      // The whole warp proceeds together (tcgen05.ld below is warp-collective).
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag,
+                                              p.status))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int k0 = j * BKV;
-      // keys visible to this row: k <= q and k < seq
-      const int kmax = min(q, p.seq - 1) - k0;  // last visible column in this block
+      const int kmax = min(q, p.seq - 1) - k0;  // last visible column of this block
       float mx = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < BKV / 32; ++c) {
-        float s[32];
-        tmem_ld32(tS + lane_off + c * 32, s);
+        float sv[32];
+        tmem_ld32(tS + c * 32, sv);
         tc_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (c * 32 + i <= kmax) mx = fmaxf(mx, s[i] * p.scale_log2);
+          if (c * 32 + i <= kmax) mx = fmaxf(mx, sv[i] * p.scale_log2);
       }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
-      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
+      if (j > 0) {
+        // P.V of the previous block done: the P buffer is free and O is stable.
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], static_cast<uint32_t>(j - 1) & 1u,
+                                                abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kRescale)) {
+        // tcgen05.ld / st are warp-collective: the whole warp rescales, each
+        // row by its own factor (1 for rows whose max did not move).
+        const float m_new = fmaxf(m, mx);
+        const float alpha = exp2f(m - m_new);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(tO + c * 32, ov);
+        }
+        tc_wait_st();
+        l *= alpha;
+        m = m_new;
+      }
       float rs = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BKV / 32; ++c) {
-        float s[32];
-        tmem_ld32(tS + lane_off + c * 32, s);
+        float sv[32];
+        tmem_ld32(tS + c * 32, sv);
         tc_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float a = (c * 32 + i <= kmax) ? exp2f(s[i] * p.scale_log2 - msub) : 0.f;
-          const float bb = (c * 32 + i + 1 <= kmax) ? exp2f(s[i + 1] * p.scale_log2 - msub) : 0.f;
+          const float a = (c * 32 + i <= kmax) ? exp2f(sv[i] * p.scale_log2 - m) : 0.f;
+          const float bb = (c * 32 + i + 1 <= kmax) ? exp2f(sv[i + 1] * p.scale_log2 - m) : 0.f;
           const uint32_t u = pack_bf16x2(a, bb);
           pk[i / 2] = u;
-          // the row sum uses the rounded probabilities the PV product sees
-          const float2 f = unpack_bf16x2(u);
+          const float2 f = unpack_bf16x2(u);  // the row sum uses the rounded P of the PV MMA
           rs += f.x + f.y;
         }
-        // 4 16-byte vectors: keys c*32 .. c*32+31 -> chunk (c/2), vectors (c%2)*4 .. +3
-        uint8_t* rowp = sP + (c / 2) * CHUNK_BYTES + r * 128;
+        uint8_t* rowp = sPt + (c / 2) * CHUNK_BYTES + r * 128;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int qv = (c % 2) * 4 + v;
@@ -259,42 +316,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
               make_uint4(pk[v * 4 + 0], pk[v * 4 + 1], pk[v * 4 + 2], pk[v * 4 + 3]);
         }
       }
-      l = l * alpha + rs;
-      m = m_new;
+      l += rs;
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      // O_j = P_j V_j is ready: O <- alpha * O + O_j
-      if (!mbar_wait(o_full, ph, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float ov[32];
-        tmem_ld32(tO + lane_off + c * 32, ov);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c * 32 + i] = o[c * 32 + i] * alpha + ov[i];
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && q < p.seq) {
+    if (ok && nbt[t] > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&o_done[t], static_cast<uint32_t>(nbt[t] - 1) & 1u,
+                                          abort_flag, p.status))) {
+      tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.O[shard]) +
                            (static_cast<int64_t>(q) * p.batch + b) * hl_d + hh * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tc_wait_ld();
+        if (q < p.seq) {
 #pragma unroll
-      for (int v = 0; v < D / 8; ++v)
-        *reinterpret_cast<uint4*>(dst + v * 8) = make_uint4(
-            pack_bf16x2(o[v * 8 + 0] * inv, o[v * 8 + 1] * inv),
-            pack_bf16x2(o[v * 8 + 2] * inv, o[v * 8 + 3] * inv),
-            pack_bf16x2(o[v * 8 + 4] * inv, o[v * 8 + 5] * inv),
-            pack_bf16x2(o[v * 8 + 6] * inv, o[v * 8 + 7] * inv));
-      if (p.lse[shard])
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(dst + c * 32 + v * 8) = make_uint4(
+                pack_bf16x2(ov[v * 8 + 0] * inv, ov[v * 8 + 1] * inv),
+                pack_bf16x2(ov[v * 8 + 2] * inv, ov[v * 8 + 3] * inv),
+                pack_bf16x2(ov[v * 8 + 4] * inv, ov[v * 8 + 5] * inv),
+                pack_bf16x2(ov[v * 8 + 6] * inv, ov[v * 8 + 7] * inv));
+        }
+      }
+      if (q < p.seq && p.lse[shard])
         p.lse[shard][(static_cast<int64_t>(b) * p.heads_local + hh) * p.seq + q] =
             (m + log2f(l)) * 0.69314718055994531f;
     }
@@ -304,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -319,7 +369,7 @@ tp_status launch_fwd_d(AttnParams& prm, cudaStream_t st) {
     if (s != TP_OK) return s;
     attr = true;
   }
-  const int grid = prm.n_qtiles * prm.p * prm.batch * prm.heads_local;
+  const int grid = prm.n_pairs * prm.p * prm.batch * prm.heads_local;
   attn_fwd_kernel<D><<<grid, kThreads, smem, st>>>(prm);
   return tpi::after_launch("attention_fwd (tcgen05)");
 }
@@ -353,10 +403,11 @@ tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const Pt
   prm.heads_local = hl;
   prm.d = d;
   prm.n_qtiles = (seq + BQ - 1) / BQ;
+  prm.n_pairs = (prm.n_qtiles + 1) / 2;
   prm.scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
   s = device_status_word(&prm.status);
   if (s != TP_OK) return s;
-  if (static_cast<int64_t>(prm.n_qtiles) * p * batch * hl > 0x7fffffffLL)
+  if (static_cast<int64_t>(prm.n_pairs) * p * batch * hl > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "attention grid too large");
   if (d == 64) return launch_fwd_d<64>(prm, st);
   if (d == 128) return launch_fwd_d<128>(prm, st);

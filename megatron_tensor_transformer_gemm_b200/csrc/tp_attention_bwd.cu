@@ -283,8 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
       const int q = (j + it) * BQ + r;
       const float lse2 = q < p.seq ? lse[q] * kLog2e : 0.f;
       const float Dq = q < p.seq ? dv[q] : 0.f;
-      if (!mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status) ||
-          !mbar_wait(pds_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, p.status)) {
+      // warp-uniform: p_ds_row's tcgen05.ld is warp-collective
+      const bool got = mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status) &&
+                       mbar_wait(pds_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
@@ -295,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(acc_full, 0, abort_flag, p.status)) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
       tc_fence_after();
       const int key = k0 + r;  // accumulator lane = key row
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
@@ -456,8 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
     const float Dq = q < p.seq ? dv[q] : 0.f;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
-      if (!mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status) ||
-          !mbar_wait(ds_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, p.status)) {
+      // warp-uniform: p_ds_row's tcgen05.ld is warp-collective
+      const bool got = mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status) &&
+                       mbar_wait(ds_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(acc_full, 0, abort_flag, p.status)) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
       tc_fence_after();
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
                             (static_cast<int64_t>(q) * p.batch + b) * (3 * hl_d) + hh * D;

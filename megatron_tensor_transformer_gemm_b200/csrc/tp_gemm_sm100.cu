@@ -467,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
       const GroupArgs& ga = p.g[g];
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status)) break;
+      // warp-uniform: the epilogue's tcgen05.ld is warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) break;
       tc_fence_after();
       const int row = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32 + lane;
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);

@@ -42,6 +42,29 @@ def test_attention_fwd_local_heads(batch, seq, heads, d, p):
     np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=2e-2)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_attention_fwd_growing_scores_rescale(d):
+    """Keys scaled up along the sequence so that every row's max grows by far
+    more than 2^8 from one key block to the next: exercises the in-place
+    rescale of O (and l) in TMEM."""
+    tp = _tp()
+    batch, seq, heads, p = 1, 1024, 2, 1
+    h = heads * d
+    Q, K, V, _ = tp_synth.draw_qkv_activations(batch, seq, heads, d, torch.bfloat16, seed=d, dy=False)
+    ramp = (1.0 + torch.arange(seq, dtype=torch.float32) / 16.0).view(seq, 1, 1)
+    Q = (Q.float() * 2.0).to(torch.bfloat16)
+    K = (K.float() * ramp).to(torch.bfloat16)
+    plan = tp.Plan(h, 0, heads, p, "bf16", "none")
+    qkv = dev(torch.cat([Q, K, V], dim=2).reshape(seq * batch, 3 * h))
+    out = torch.empty(seq * batch, h, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(batch, heads, seq, dtype=torch.float32, device="cuda")
+    plan.attention_fwd(batch, seq, [qkv], [out], [lse])
+    ref, ref_lse = O.attention_fwd(O.f64(Q), O.f64(K), O.f64(V), batch, heads, True)
+    assert_close(out, ref.reshape(seq * batch, h), TOL_BF16, "O")
+    np.testing.assert_allclose(host(lse), ref_lse, rtol=1e-4, atol=5e-2)
+    assert tp.device_status() == "TP_OK"
+
+
 def test_attention_block_full_size_sampled():
     """hidden 4096, 32 heads x 128, seq 4096, batch 2, p 8 (4 heads per shard),
     causal; QKV -> attention -> out-projection partials -> reduce + residual."""
