@@ -49,6 +49,7 @@ __all__ = [
     "attention_fwd", "attention_fwd_rows", "attention_bwd", "layernorm_fwd", "layernorm_bwd",
     "attn_sublayer_fwd", "attn_sublayer_bwd", "layer_fwd", "layer_bwd",
     "sp_mlp_fwd", "sp_mlp_bwd", "max_row_rel_err", "LN_EPS",
+    "rmsnorm_fwd", "rmsnorm_bwd", "norm_sharded_fwd", "norm_sharded_bwd",
 ]
 
 LN_EPS = 1e-5
@@ -501,6 +502,58 @@ def layernorm_bwd(x, g, dy, mean, rstd):
     dx = rstd[:, None] * (gy - gy.mean(axis=1, keepdims=True)
                           - xhat * (gy * xhat).mean(axis=1, keepdims=True))
     return dx, (dy * xhat).sum(axis=0), dy.sum(axis=0)
+
+
+def rmsnorm_fwd(x, g, eps=LN_EPS):
+    """y = x / sqrt(mean(x^2) + eps) * g per row (RMSNorm over the full hidden dim)."""
+    rstd = 1.0 / np.sqrt((x * x).mean(axis=1, keepdims=True) + eps)
+    return x * rstd * g[None, :], rstd[:, 0]
+
+
+def rmsnorm_bwd(x, g, dy, rstd):
+    """dx, dg of rmsnorm_fwd: with xhat = x * rstd and gy = dy * g,
+    dx = rstd * (gy - xhat * mean_row(gy * xhat)); dg = sum_rows dy * xhat."""
+    xhat = x * rstd[:, None]
+    gy = dy * g[None, :]
+    dx = rstd[:, None] * (gy - xhat * (gy * xhat).mean(axis=1, keepdims=True))
+    return dx, (dy * xhat).sum(axis=0)
+
+
+def norm_sharded_fwd(x_shards, g_shards, b_shards, kind):
+    """LayerNorm / RMSNorm whose input is split over the hidden dim, the way
+    [TP-blog] §3.3 describes: every shard forms its local sums (sum x and
+    sum x^2 for LayerNorm, sum x^2 for RMSNorm), the per-row scalars are summed
+    over shards, and the resulting statistics normalise each shard's slice.
+    Returns the output shards and (mean, rstd) (mean is None for RMSNorm)."""
+    h = sum(xs.shape[1] for xs in x_shards)
+    s2 = sum((xs * xs).sum(axis=1) for xs in x_shards)
+    if kind == "rms":
+        rstd = 1.0 / np.sqrt(s2 / h + LN_EPS)
+        return [xs * rstd[:, None] * gs[None, :] for xs, gs in zip(x_shards, g_shards)], (None, rstd)
+    s1 = sum(xs.sum(axis=1) for xs in x_shards)
+    mean = s1 / h
+    var = s2 / h - mean * mean
+    rstd = 1.0 / np.sqrt(var + LN_EPS)
+    return ([(xs - mean[:, None]) * rstd[:, None] * gs[None, :] + bs[None, :]
+             for xs, gs, bs in zip(x_shards, g_shards, b_shards)], (mean, rstd))
+
+
+def norm_sharded_bwd(x_shards, g_shards, dy_shards, stats, kind):
+    """Backward of norm_sharded_fwd: the two per-row means of the backward
+    (of gy and of gy * xhat) are again local sums reduced over shards.
+    Returns dx shards and dg (and db for LayerNorm) shards."""
+    mean, rstd = stats
+    h = sum(xs.shape[1] for xs in x_shards)
+    xh = [(xs if mean is None else xs - mean[:, None]) * rstd[:, None] for xs in x_shards]
+    gy = [dys * gs[None, :] for dys, gs in zip(dy_shards, g_shards)]
+    m2 = sum((a * b).sum(axis=1) for a, b in zip(gy, xh)) / h
+    if kind == "rms":
+        dx = [rstd[:, None] * (a - b * m2[:, None]) for a, b in zip(gy, xh)]
+        return dx, [(d * b).sum(axis=0) for d, b in zip(dy_shards, xh)], None
+    m1 = sum(a.sum(axis=1) for a in gy) / h
+    dx = [rstd[:, None] * (a - m1[:, None] - b * m2[:, None]) for a, b in zip(gy, xh)]
+    return (dx, [(d * b).sum(axis=0) for d, b in zip(dy_shards, xh)],
+            [d.sum(axis=0) for d in dy_shards])
 
 
 # ---------------------------------------------------------------------------

@@ -572,3 +572,54 @@ def test_mutant_silu_grad_sign_fails_fd():
     s = 1 / (1 + np.exp(-z))
     bad = s * (1 - z * (1 - s))
     assert not np.allclose(bad, _fd_scalar(O.silu, z), rtol=1e-7, atol=1e-9)
+
+
+# --------------------------------------------- hidden-sharded norm statistics
+
+def test_rmsnorm_brute_force_and_fd():
+    x, g = randn(4, 9), randn(9)
+    y, rstd = O.rmsnorm_fwd(x, g)
+    for r in range(4):
+        ms = sum(v * v for v in x[r].tolist()) / 9
+        ref = [v / math.sqrt(ms + 1e-5) * g[c] for c, v in enumerate(x[r].tolist())]
+        np.testing.assert_allclose(y[r], ref, rtol=1e-12, atol=1e-13)
+    C = randn(4, 9)
+    dx, dg = O.rmsnorm_bwd(x, g, C, rstd)
+    _check_fd(dx, lambda: float((O.rmsnorm_fwd(x, g)[0] * C).sum()), x, n=20)
+    _check_fd(dg, lambda: float((O.rmsnorm_fwd(x, g)[0] * C).sum()), g, n=9)
+
+
+def test_rmsnorm_rows_have_unit_rms():
+    y, _ = O.rmsnorm_fwd(randn(6, 64, std=4.0), np.ones(64))
+    np.testing.assert_allclose(np.sqrt((y * y).mean(axis=1)), 1.0, rtol=1e-5)
+
+
+@pytest.mark.parametrize("kind", ["rms", "ln"])
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_hidden_sharded_norm_equals_full_norm(kind, p):
+    """Local sums reduced over shards give the full-row statistics (walkthrough §3.3)."""
+    T, h = 5, 16
+    x, g, b, dy = randn(T, h, std=2.0) + 0.3, 1 + 0.1 * randn(h), 0.1 * randn(h), randn(T, h)
+    xs, gs, bs, dys = ([O.shard_cols(a, p, i) for i in range(p)] for a in (x, g[None, :], b[None, :], dy))
+    gs, bs = [a[0] for a in gs], [a[0] for a in bs]
+    ys, stats = O.norm_sharded_fwd(xs, gs, bs, kind)
+    dxs, dgs, dbs = O.norm_sharded_bwd(xs, gs, dys, stats, kind)
+    if kind == "rms":
+        y, rstd = O.rmsnorm_fwd(x, g)
+        dx, dg = O.rmsnorm_bwd(x, g, dy, rstd)
+    else:
+        y, mean, rstd = O.layernorm_fwd(x, g, b)
+        dx, dg, db = O.layernorm_bwd(x, g, dy, mean, rstd)
+        np.testing.assert_allclose(np.concatenate(dbs), db, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(ys, axis=1), y, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(dxs, axis=1), dx, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(dgs), dg, rtol=1e-10, atol=1e-12)
+
+
+def test_mutant_local_only_statistics_fail_the_sharded_norm_pin():
+    """Normalising each shard by its own statistics (the mistake the walkthrough
+    §3.3 warns about) does not reproduce the full-row norm."""
+    x, g = randn(5, 16, std=2.0) + 1.0, np.ones(16)
+    y, _ = O.rmsnorm_fwd(x, g)
+    bad = np.concatenate([O.rmsnorm_fwd(O.shard_cols(x, 2, i), g[:8])[0] for i in range(2)], axis=1)
+    assert not np.allclose(bad, y, rtol=1e-6)
