@@ -50,6 +50,8 @@ __all__ = [
     "attn_sublayer_fwd", "attn_sublayer_bwd", "layer_fwd", "layer_bwd",
     "sp_mlp_fwd", "sp_mlp_bwd", "max_row_rel_err", "LN_EPS",
     "rmsnorm_fwd", "rmsnorm_bwd", "norm_sharded_fwd", "norm_sharded_bwd",
+    "vocab_padded", "embedding_fwd", "embedding_fwd_sharded", "embedding_bwd",
+    "cross_entropy", "cross_entropy_vocab_parallel",
 ]
 
 LN_EPS = 1e-5
@@ -554,6 +556,104 @@ def norm_sharded_bwd(x_shards, g_shards, dy_shards, stats, kind):
     dx = [rstd[:, None] * (a - m1[:, None] - b * m2[:, None]) for a, b in zip(gy, xh)]
     return (dx, [(d * b).sum(axis=0) for d, b in zip(dy_shards, xh)],
             [d.sum(axis=0) for d in dy_shards])
+
+
+# ---------------------------------------------------------------------------
+# Vocab-parallel embedding and cross-entropy. [TP-blog] §6.2: the vocab dim is
+# split over shards, padded up to a size the split divides; the output head
+# computes only its own vocab slice of the logits and its partial loss, and the
+# partials are reduced instead of gathering the full logits. [TP-wiki] 工程实践
+# (vocab-parallel embedding).
+# ---------------------------------------------------------------------------
+
+def vocab_padded(vocab, p, align=8):
+    """Smallest padded vocab >= vocab whose p shards each hold a multiple of
+    `align` rows (the split must divide it; the alignment keeps shard rows at
+    16-byte multiples for bf16)."""
+    unit = p * align
+    return ((vocab + unit - 1) // unit) * unit
+
+
+def embedding_fwd(ids, E):
+    """Y[t] = E[ids[t]]: the plain definition of the lookup."""
+    return E[np.asarray(ids)]
+
+
+def embedding_fwd_sharded(ids, E_shards):
+    """The vocab-parallel lookup: shard i holds rows [i*Vs, (i+1)*Vs) and
+    returns the row for tokens in its range and zeros otherwise; the sum over
+    shards (the all-reduce) gives the lookup."""
+    ids = np.asarray(ids)
+    Vs = E_shards[0].shape[0]
+    parts = []
+    for i, Ei in enumerate(E_shards):
+        loc = ids - i * Vs
+        own = (loc >= 0) & (loc < Vs)
+        part = np.zeros((len(ids), Ei.shape[1]))
+        part[own] = Ei[loc[own]]
+        parts.append(part)
+    return reduce_partials(parts)
+
+
+def embedding_bwd(ids, dY, vocab_rows):
+    """dE[v] = sum over tokens t with ids[t] == v of dY[t]."""
+    dE = np.zeros((vocab_rows, dY.shape[1]))
+    for t, v in enumerate(np.asarray(ids)):
+        dE[v] += dY[t]
+    return dE
+
+
+def cross_entropy(logits, labels, vocab):
+    """Per-token loss log(sum_v exp(z_v)) - z_label over the first `vocab`
+    columns (padding columns excluded), and d(mean loss)/d logits =
+    (softmax - onehot) / T (zero on padding columns)."""
+    z = logits[:, :vocab]
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    S = e.sum(axis=1, keepdims=True)
+    labels = np.asarray(labels)
+    T = z.shape[0]
+    loss = (np.log(S) + m)[:, 0] - z[np.arange(T), labels]
+    g = np.zeros_like(logits)
+    g[:, :vocab] = e / S
+    g[np.arange(T), labels] -= 1.0
+    return loss, g / T
+
+
+def cross_entropy_vocab_parallel(logit_shards, labels, vocab):
+    """The pages' way: every shard forms its local row max, its local sum of
+    exp(z - local max) over its real (non-padding) columns and, if it owns the
+    label, the target logit; the per-row scalars are reduced over shards
+    (max, rescaled sum, target). Returns per-token loss and per-shard gradients
+    of the mean loss."""
+    labels = np.asarray(labels)
+    Vs = logit_shards[0].shape[1]
+    T = logit_shards[0].shape[0]
+    ms, ss, zt = [], [], np.zeros(T)
+    for i, Li in enumerate(logit_shards):
+        real = max(0, min(Vs, vocab - i * Vs))
+        zi = Li[:, :real]
+        mi = zi.max(axis=1) if real > 0 else np.full(T, -np.inf)
+        si = np.exp(zi - mi[:, None]).sum(axis=1) if real > 0 else np.zeros(T)
+        ms.append(mi)
+        ss.append(si)
+        loc = labels - i * Vs
+        own = (loc >= 0) & (loc < real)
+        zt[own] = Li[np.arange(T)[own], loc[own]]
+    m = np.max(np.stack(ms), axis=0)
+    S = sum(si * np.exp(mi - m) for mi, si in zip(ms, ss))
+    lse = np.log(S) + m
+    loss = lse - zt
+    grads = []
+    for i, Li in enumerate(logit_shards):
+        real = max(0, min(Vs, vocab - i * Vs))
+        g = np.zeros_like(Li)
+        g[:, :real] = np.exp(Li[:, :real] - lse[:, None])
+        loc = labels - i * Vs
+        own = (loc >= 0) & (loc < real)
+        g[np.arange(T)[own], loc[own]] -= 1.0
+        grads.append(g / T)
+    return loss, grads
 
 
 # ---------------------------------------------------------------------------

@@ -623,3 +623,75 @@ def test_mutant_local_only_statistics_fail_the_sharded_norm_pin():
     y, _ = O.rmsnorm_fwd(x, g)
     bad = np.concatenate([O.rmsnorm_fwd(O.shard_cols(x, 2, i), g[:8])[0] for i in range(2)], axis=1)
     assert not np.allclose(bad, y, rtol=1e-6)
+
+
+# ------------------------------------------ vocab-parallel embedding and loss
+
+def test_vocab_padding():
+    assert O.vocab_padded(32000, 8) == 32000
+    assert O.vocab_padded(32001, 8) == 32064
+    assert O.vocab_padded(50257, 4) == 50272
+    assert O.vocab_padded(10, 3, align=1) == 12
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_vocab_parallel_embedding_equals_lookup(p):
+    V, h, T = 40, 6, 25
+    E = randn(V, h)
+    ids = rng.integers(0, V, size=T)
+    shards = [E[i * V // p:(i + 1) * V // p] for i in range(p)]
+    assert np.array_equal(O.embedding_fwd_sharded(ids, shards), O.embedding_fwd(ids, E))
+    assert np.array_equal(O.embedding_fwd(ids, E)[3], E[ids[3]])
+
+
+def test_embedding_bwd_by_finite_differences_and_counting():
+    V, h, T = 7, 3, 12
+    E, C = randn(V, h), randn(T, h)
+    ids = rng.integers(0, V, size=T)
+    dE = O.embedding_bwd(ids, C, V)
+    _check_fd(dE, lambda: float((O.embedding_fwd(ids, E) * C).sum()), E, n=21)
+    ones = O.embedding_bwd(ids, np.ones((T, 1)), V)[:, 0]
+    assert np.array_equal(ones, np.bincount(ids, minlength=V).astype(float))
+
+
+def test_cross_entropy_brute_force_and_closed_forms():
+    T, V = 4, 5
+    z = randn(T, V + 3)   # 3 padding columns
+    labels = rng.integers(0, V, size=T)
+    loss, g = O.cross_entropy(z, labels, V)
+    for t in range(T):
+        row = z[t, :V].tolist()
+        ref = math.log(sum(math.exp(v) for v in row)) - row[labels[t]]
+        assert abs(loss[t] - ref) < 1e-12
+    assert np.all(loss >= 0)
+    assert np.all(g[:, V:] == 0)
+    np.testing.assert_allclose(g.sum(axis=1), 0.0, atol=1e-15)
+    u, _ = O.cross_entropy(np.zeros((2, V)), [0, 3], V)
+    np.testing.assert_allclose(u, math.log(V), rtol=1e-15)
+    _check_fd(g, lambda: float(O.cross_entropy(z, labels, V)[0].mean()), z, n=20)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_vocab_parallel_cross_entropy_equals_full(p):
+    """Local max / sum / target per shard, reduced over shards, equals the
+    cross-entropy on the full logits (walkthrough §6.2), padding excluded."""
+    T, V = 9, 37
+    Vp = O.vocab_padded(V, p, align=2)
+    z = randn(T, Vp, std=3.0)
+    labels = rng.integers(0, V, size=T)
+    labels[0] = V - 1                      # a label in the last, padded shard
+    Vs = Vp // p
+    shards = [z[:, i * Vs:(i + 1) * Vs] for i in range(p)]
+    loss, grads = O.cross_entropy_vocab_parallel(shards, labels, V)
+    rl, rg = O.cross_entropy(z, labels, V)
+    np.testing.assert_allclose(loss, rl, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.concatenate(grads, axis=1), rg, rtol=1e-12, atol=1e-14)
+
+
+def test_mutant_padding_included_fails_the_ce_pin():
+    T, V = 6, 10
+    z = randn(T, 16)
+    labels = rng.integers(0, V, size=T)
+    bad, _ = O.cross_entropy(z, labels, 16)   # padding columns wrongly in the softmax
+    good, _ = O.cross_entropy(z, labels, V)
+    assert not np.allclose(bad, good)
