@@ -89,8 +89,13 @@ typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU = 1, TP_ACT_SWIGLU = 2 } tp_act;
  *               row W2 [hidden, ffn].
  *   TP_QKV:     column Wqkv [3*hidden, hidden], rows [Wq; Wk; Wv], split by
  *               whole heads ([TP-blog] §3.1). No activation.
- *   TP_OUTPROJ: row Wo [hidden, hidden], input = local heads' outputs. */
-typedef enum { TP_MLP = 0, TP_QKV = 1, TP_OUTPROJ = 2 } tp_which;
+ *   TP_OUTPROJ: row Wo [hidden, hidden], input = local heads' outputs.
+ *   TP_VOCAB:   column output head W [Vp, hidden] split by vocab rows (Vp the
+ *               padded vocab, see tp_plan_set_vocab); no activation. */
+typedef enum { TP_MLP = 0, TP_QKV = 1, TP_OUTPROJ = 2, TP_VOCAB = 3 } tp_which;
+
+/* Norm of a hidden-sharded activation (tp_norm_sharded_*). */
+typedef enum { TP_NORM_LAYER = 0, TP_NORM_RMS = 1 } tp_norm_kind;
 
 /* ---------------------------------------------------------------- plan */
 
@@ -104,6 +109,13 @@ TP_API tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype 
                          tp_act act, tp_plan** out);
 TP_API void tp_plan_destroy(tp_plan* plan);
 
+/* Vocab of the embedding / output head ([TP-blog] §6.2: the vocab is padded
+ * up to a size the split divides). Sets the plan's padded vocab Vp, the
+ * smallest multiple of 8*p >= vocab (each shard then holds Vp/p rows, a
+ * multiple of 8, i.e. 16-byte rows in bf16), and writes it to *vocab_padded
+ * (NULL ok). */
+TP_API tp_status tp_plan_set_vocab(tp_plan* plan, int vocab, int* vocab_padded);
+
 /* Write a text description of every shard shape into buf (host, n bytes,
  * always NUL-terminated) -- the shape print [TP-blog] §6.1/§6.4 asks for. */
 TP_API tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n);
@@ -112,7 +124,8 @@ TP_API const char* tp_status_string(tp_status s);
 TP_API const char* tp_last_error(void);
 
 /* Synchronise `stream`, read the device status word of the current device,
- * store it in *device_status (TP_OK or TP_ERR_TIMEOUT) and clear it. */
+ * store it in *device_status (TP_OK, TP_ERR_TIMEOUT if a kernel wait gave up,
+ * TP_ERR_ARG if a kernel met an out-of-range token id / label) and clear it. */
 TP_API tp_status tp_get_device_status(void* stream, int* device_status);
 
 /* Number of kernel launches this thread has issued through the library
@@ -218,6 +231,47 @@ TP_API tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, co
                                       const void* gamma, const void* beta, void* Y_full,
                                       float* mean, float* rstd, void* stream);
 
+/* Vocab-parallel embedding lookup ([TP-blog] §6.2, [TP-wiki] 工程实践): E[i]
+ * [Vp/p, hidden] is shard i of the padded embedding (vocab ids [i*Vp/p,
+ * (i+1)*Vp/p)); ids [T] int32 (device). Y [T, hidden] = the row of the owning
+ * shard, i.e. the sum over shards of the partial lookups (each shard
+ * contributes zeros outside its range). Ids outside [0, vocab) give a zero
+ * row and set the device status word (tp_get_device_status -> TP_ERR_ARG). */
+TP_API tp_status tp_embedding_fwd(tp_plan* plan, int64_t T, const int32_t* ids,
+                                  const void* const* E, void* Y, void* stream);
+
+/* Backward of the lookup: dE[i] [Vp/p, hidden] (plan dtype, overwritten) =
+ * for each vocab row v of shard i, the sum over tokens with id == v of dY[t]
+ * (fp32, in token order, deterministic); rows no token uses are zero. */
+TP_API tp_status tp_embedding_bwd(tp_plan* plan, int64_t T, const int32_t* ids, const void* dY,
+                                  void* const* dE, void* stream);
+
+/* Vocab-parallel cross-entropy on sharded logits ([TP-blog] §6.2: each shard
+ * computes only its vocab slice's logits and partial loss; the per-row
+ * scalars -- local max, local sum of exponentials, target logit -- are
+ * reduced over shards). logits[i] [T, Vp/p] (e.g. from tp_column_fwd with
+ * TP_VOCAB); labels [T] int32 (device; < 0 = ignored token). loss [T] fp32 =
+ * logsumexp over the real vocab columns (padding excluded) minus the target
+ * logit (0 for ignored tokens); lse [T] fp32 (NULL ok). dlogits[i] (NULL array
+ * skips; may alias logits[i]) = (softmax - onehot) * grad_scale, zero on
+ * padding columns and ignored tokens. Labels >= vocab set the device status. */
+TP_API tp_status tp_vocab_cross_entropy(tp_plan* plan, int64_t T, const void* const* logits,
+                                        const int32_t* labels, float grad_scale, float* loss,
+                                        float* lse, void* const* dlogits, void* stream);
+
+/* LayerNorm / RMSNorm of rows whose hidden dim is split over the p shards,
+ * with the statistics formed the way [TP-blog] §3.3 describes: every shard's
+ * local sums (sum x and sum x^2; RMSNorm only sum x^2) are summed over shards
+ * into one scalar per row, and every shard normalises its slice with them.
+ *   X[i], Y[i]: [rows, hidden/p] (columns [i*h/p, (i+1)*h/p) of the row);
+ *   gamma[i], beta[i]: [hidden/p] (beta ignored, may be NULL, for RMSNorm);
+ *   mean (LayerNorm only), rstd: [rows] fp32 outputs (NULL ok).
+ * LayerNorm uses var = E[x^2] - mean^2 (the local-sums form), eps = 1e-5. */
+TP_API tp_status tp_norm_sharded_fwd(tp_plan* plan, tp_norm_kind kind, int64_t rows,
+                                     const void* const* X, const void* const* gamma,
+                                     const void* const* beta, void* const* Y, float* mean,
+                                     float* rstd, void* stream);
+
 /* Causal attention of each shard's local heads ([TP-blog] §3.1: full sequence,
  * whole heads, no cross-shard step). QKV[i] [seq*batch, 3*h/p] = [Q_i|K_i|V_i]
  * (the TP_QKV column output); O[i] [seq*batch, h/p] with head j of the shard
@@ -285,6 +339,15 @@ TP_API tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const vo
 TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
                            const void* dy, const float* mean, const float* rstd, void* dx,
                            float* dgamma, float* dbeta, int accumulate, void* stream);
+
+/* Backward of tp_norm_sharded_fwd: dX[i] [rows, hidden/p]; dgamma[i] (and
+ * dbeta[i] for LayerNorm; NULL array ok) [hidden/p] fp32 sums over rows. The
+ * per-row means of the backward are again local sums reduced over shards. */
+TP_API tp_status tp_norm_sharded_bwd(tp_plan* plan, tp_norm_kind kind, int64_t rows,
+                                     const void* const* X, const void* const* gamma,
+                                     const void* const* dY, const float* mean, const float* rstd,
+                                     void* const* dX, float* const* dgamma, float* const* dbeta,
+                                     void* stream);
 
 /* Attention backward of each shard's local heads: from QKV[i], O[i], dO[i]
  * and LSE[i] of the forward, writes dQKV[i] [seq*batch, 3h/p] = [dQ|dK|dV].

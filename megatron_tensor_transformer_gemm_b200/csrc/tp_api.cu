@@ -149,6 +149,9 @@ tp_status col_shape(const tp_plan* plan, tp_which which, ColShape* cs) {
   } else if (which == TP_QKV) {
     if (plan->heads <= 0) return fail(TP_ERR_ARG, "plan has no attention (heads = 0)");
     cs->n_w = cs->n_h = 3 * plan->hidden / p;
+  } else if (which == TP_VOCAB) {
+    if (plan->vocab_padded <= 0) return fail(TP_ERR_ARG, "plan has no vocab (tp_plan_set_vocab)");
+    cs->n_w = cs->n_h = plan->vocab_padded / p;
   } else {
     return fail(TP_ERR_ARG, "projection %d is not column-parallel", static_cast<int>(which));
   }
@@ -251,6 +254,8 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   plan->heads = heads;
   plan->p = p;
   plan->head_dim = heads > 0 ? hidden / heads : 0;
+  plan->vocab = 0;
+  plan->vocab_padded = 0;
   plan->dtype = dtype;
   plan->act = act;
   plan->ws = nullptr;
@@ -296,6 +301,9 @@ tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n) {
         plan->heads / p, plan->head_dim);
     add("  out-proj row shard Wo_i: [%d, %d]\n", h, h / p);
   }
+  if (plan->vocab_padded > 0)
+    add("  vocab shard (embedding / output head): [%d, %d] (vocab %d padded to %d)\n",
+        plan->vocab_padded / p, h, plan->vocab, plan->vocab_padded);
   add("  sequence shard (SP): [T/%d, %d]\n", p, h);
   return TP_OK;
 }
@@ -309,7 +317,7 @@ tp_status tp_get_device_status(void* stream, int* device_status) {
   TP_TRY(cuda_status(cudaMemcpy(&v, addr, sizeof(v), cudaMemcpyDeviceToHost), "read status"));
   unsigned zero = 0;
   TP_TRY(cuda_status(cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status"));
-  *device_status = v ? TP_ERR_TIMEOUT : TP_OK;
+  *device_status = (v & 1u) ? TP_ERR_TIMEOUT : (v & 2u) ? TP_ERR_ARG : TP_OK;
   return TP_OK;
 }
 
@@ -362,6 +370,17 @@ static tp_status shard_copy(const tp_plan* plan, tp_which which, bool column, co
           char* sb = S + static_cast<int64_t>(part) * rows * h * es;
           TP_TRY(to_shards ? copy(fb, h, sb, h, rows, h) : copy(sb, h, fb, h, rows, h));
         }
+      }
+      return TP_OK;
+    }
+    if (which == TP_VOCAB) {
+      if (plan->vocab_padded <= 0) return fail(TP_ERR_ARG, "plan has no vocab (tp_plan_set_vocab)");
+      const int rows = plan->vocab_padded / p;
+      TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+      for (int i = 0; i < p; ++i) {
+        char* S = static_cast<char*>(const_cast<void*>(shards[i]));
+        char* fb = F + static_cast<int64_t>(i) * rows * h * es;
+        TP_TRY(to_shards ? copy(fb, h, S, h, rows, h) : copy(S, h, fb, h, rows, h));
       }
       return TP_OK;
     }
@@ -442,7 +461,7 @@ tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
   ColShape cs{};
   TP_TRY(col_shape(plan, which, &cs));
   const int p = plan->p;
-  const tp_act act = which == TP_QKV ? TP_ACT_NONE : plan->act;
+  const tp_act act = which == TP_MLP ? plan->act : TP_ACT_NONE;
   TP_TRY(check_ptr(X, "X"));
   TP_TRY(check_ptrs(W, p, "W", false));
   TP_TRY(check_ptrs(bias, p, "bias", true));
@@ -754,6 +773,119 @@ tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const voi
   TP_TRY(check_ln(plan));
   return launch_layernorm_bwd(plan, x, gamma, dy, mean, rstd, dx, dgamma, dbeta, accumulate, rows,
                               plan->hidden, plan->dtype, as_stream(stream));
+}
+
+tp_status tp_plan_set_vocab(tp_plan* plan, int vocab, int* vocab_padded) {
+  TP_TRY(check_plan(plan));
+  if (vocab <= 0) return fail(TP_ERR_ARG, "vocab = %d must be positive", vocab);
+  const int64_t unit = 8LL * plan->p;
+  const int64_t vp = ((vocab + unit - 1) / unit) * unit;
+  if (vp > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "vocab too large");
+  plan->vocab = vocab;
+  plan->vocab_padded = static_cast<int>(vp);
+  if (vocab_padded) *vocab_padded = plan->vocab_padded;
+  return TP_OK;
+}
+
+static tp_status check_vocab(const tp_plan* plan, int64_t T) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (plan->vocab_padded <= 0) return fail(TP_ERR_ARG, "plan has no vocab (tp_plan_set_vocab)");
+  return check_row_bytes(plan->hidden, plan->dtype, "hidden");
+}
+
+tp_status tp_embedding_fwd(tp_plan* plan, int64_t T, const int32_t* ids, const void* const* E,
+                           void* Y, void* stream) {
+  TP_TRY(check_vocab(plan, T));
+  const int p = plan->p;
+  TP_TRY(check_ptr(ids, "ids"));
+  TP_TRY(check_ptrs(E, p, "E", false));
+  TP_TRY(check_ptr(Y, "Y"));
+  if (T == 0) return TP_OK;
+  return launch_embedding_fwd(ids, to_arr(E, p), plan->vocab, plan->vocab_padded / p, T,
+                              plan->hidden, plan->dtype, Y, as_stream(stream));
+}
+
+tp_status tp_embedding_bwd(tp_plan* plan, int64_t T, const int32_t* ids, const void* dY,
+                           void* const* dE, void* stream) {
+  TP_TRY(check_vocab(plan, T));
+  const int p = plan->p;
+  if (T > 0) {
+    TP_TRY(check_ptr(ids, "ids"));
+    TP_TRY(check_ptr(dY, "dY"));
+  }
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dE), p, "dE", false));
+  return launch_embedding_bwd(ids, T, dY, plan->hidden, plan->vocab, plan->vocab_padded,
+                              plan->vocab_padded / p, to_marr(dE, p), plan->dtype,
+                              as_stream(stream));
+}
+
+tp_status tp_vocab_cross_entropy(tp_plan* plan, int64_t T, const void* const* logits,
+                                 const int32_t* labels, float grad_scale, float* loss, float* lse,
+                                 void* const* dlogits, void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(T));
+  if (plan->vocab_padded <= 0) return fail(TP_ERR_ARG, "plan has no vocab (tp_plan_set_vocab)");
+  const int p = plan->p;
+  TP_TRY(check_ptrs(logits, p, "logits", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dlogits), p, "dlogits", true));
+  TP_TRY(check_ptr(labels, "labels"));
+  TP_TRY(check_ptr(loss, "loss"));
+  if (T == 0) return TP_OK;
+  MutPtrArray g{};
+  if (dlogits)
+    for (int i = 0; i < p; ++i) g.p[i] = dlogits[i];
+  return launch_vocab_ce(to_arr(logits, p), g, p, plan->vocab_padded / p, plan->vocab, labels,
+                         grad_scale, loss, lse, T, plan->dtype, as_stream(stream));
+}
+
+static tp_status check_norm_sharded(const tp_plan* plan, tp_norm_kind kind, int64_t rows) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(rows));
+  if (kind != TP_NORM_LAYER && kind != TP_NORM_RMS) return fail(TP_ERR_ARG, "unknown norm kind %d", kind);
+  const int h = plan->hidden, p = plan->p;
+  if ((h / p) % 8) return fail(TP_ERR_UNSUPPORTED, "hidden/p = %d must be a multiple of 8", h / p);
+  if (h > 16384) return fail(TP_ERR_UNSUPPORTED, "norms support hidden <= 16384 (got %d)", h);
+  return TP_OK;
+}
+
+tp_status tp_norm_sharded_fwd(tp_plan* plan, tp_norm_kind kind, int64_t rows, const void* const* X,
+                              const void* const* gamma, const void* const* beta, void* const* Y,
+                              float* mean, float* rstd, void* stream) {
+  TP_TRY(check_norm_sharded(plan, kind, rows));
+  const int p = plan->p;
+  TP_TRY(check_ptrs(X, p, "X", false));
+  TP_TRY(check_ptrs(gamma, p, "gamma", false));
+  if (kind == TP_NORM_LAYER) TP_TRY(check_ptrs(beta, p, "beta", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Y), p, "Y", false));
+  if (rows == 0) return TP_OK;
+  return launch_norm_sharded_fwd(kind == TP_NORM_RMS, to_arr(X, p), to_arr(gamma, p),
+                                 to_arr(kind == TP_NORM_LAYER ? beta : nullptr, p), to_marr(Y, p), p,
+                                 rows, plan->hidden, mean, rstd, plan->dtype, as_stream(stream));
+}
+
+tp_status tp_norm_sharded_bwd(tp_plan* plan, tp_norm_kind kind, int64_t rows, const void* const* X,
+                              const void* const* gamma, const void* const* dY, const float* mean,
+                              const float* rstd, void* const* dX, float* const* dgamma,
+                              float* const* dbeta, void* stream) {
+  TP_TRY(check_norm_sharded(plan, kind, rows));
+  const int p = plan->p;
+  TP_TRY(check_ptrs(X, p, "X", false));
+  TP_TRY(check_ptrs(gamma, p, "gamma", false));
+  TP_TRY(check_ptrs(dY, p, "dY", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX), p, "dX", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dgamma), p, "dgamma", false));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dbeta), p, "dbeta", true));
+  TP_TRY(check_ptr(rstd, "rstd"));
+  if (kind == TP_NORM_LAYER) TP_TRY(check_ptr(mean, "mean"));
+  MutPtrArray dg{}, db{};
+  for (int i = 0; i < p; ++i) {
+    dg.p[i] = dgamma[i];
+    db.p[i] = dbeta ? dbeta[i] : nullptr;
+  }
+  return launch_norm_sharded_bwd(plan, kind == TP_NORM_RMS, to_arr(X, p), to_arr(gamma, p),
+                                 to_arr(dY, p), to_marr(dX, p), dg, db, p, rows, plan->hidden, mean,
+                                 rstd, plan->dtype, as_stream(stream));
 }
 
 tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const void* x, float* out,

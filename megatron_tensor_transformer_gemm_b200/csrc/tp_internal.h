@@ -14,6 +14,8 @@ struct tp_plan {
   int heads;
   int p;
   int head_dim;
+  int vocab;         // 0 until tp_plan_set_vocab
+  int vocab_padded;  // multiple of 8 * p
   tp_dtype dtype;
   tp_act act;
   // Device scratch, allocated on first need (cudaMalloc), grown on demand.
@@ -73,6 +75,27 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
                                const float* mean, const float* rstd, void* dx, float* dgamma,
                                float* dbeta, int accumulate, int64_t rows, int64_t cols,
                                tp_dtype dt, cudaStream_t st);
+
+// Vocab-parallel embedding and cross-entropy (tp_vocab.cu).
+tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab, int64_t Vs,
+                               int64_t T, int64_t h, tp_dtype dt, void* Y, cudaStream_t st);
+tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, int64_t h, int vocab,
+                               int64_t Vp, int64_t Vs, const MutPtrArray& dE, tp_dtype dt,
+                               cudaStream_t st);
+tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
+                          const int32_t* labels, float scale, float* loss, float* lse, int64_t T,
+                          tp_dtype dt, cudaStream_t st);
+
+// Norms of hidden-sharded rows (tp_layernorm.cu).
+tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G,
+                                  const PtrArray& B, const MutPtrArray& Y, int p, int64_t rows,
+                                  int64_t h, float* mean, float* rstd, tp_dtype dt,
+                                  cudaStream_t st);
+tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, const PtrArray& G,
+                                  const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
+                                  const MutPtrArray& db, int p, int64_t rows, int64_t h,
+                                  const float* mean, const float* rstd, tp_dtype dt,
+                                  cudaStream_t st);
 
 // Element-wise activation kernels for the fp32 path (tp_gemm_simt.cu).
 tp_status launch_act_fwd(tp_act act, const float* Z, int64_t T, int64_t nh, int64_t ldz, float* H,

@@ -328,3 +328,264 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
 }
 
 }  // namespace tpi
+
+// ---------------------------------------------------------------------------
+// Norms of rows whose hidden dim is split over p shards (each shard holds
+// columns [i*h/p, (i+1)*h/p) in its own buffer). The row statistics are sums
+// of the shards' local sums -- on one GPU that reduction over shards is part
+// of the CTA's row reduction -- and each shard's slice is normalised with them.
+// LayerNorm uses the one-pass variance E[x^2] - mean^2 that the local-sums
+// method implies; RMSNorm needs only sum x^2.
+// ---------------------------------------------------------------------------
+namespace {
+
+using tpi::MutPtrArray;
+
+template <typename T, int THREADS, bool RMS>
+__global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
+    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
+    const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int vps,
+    int64_t hs, int64_t h, float* mean_out, float* rstd_out) {
+  constexpr int V = LnVec<T>::N;
+  __shared__ float red[THREADS / 32];
+  const int64_t r = blockIdx.x;
+  const int vpr = static_cast<int>(h / V);
+  float v[kVptMax][V];
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    if (c < vpr) {
+      const int sh = c / vps, lc = c - sh * vps;
+      LnVec<T>::load(static_cast<const T*>(X.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, v[i]);
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        s1 += v[i][k];
+        s2 += v[i][k] * v[i][k];
+      }
+    }
+  }
+  const float S2 = block_sum<THREADS>(s2, red);
+  float mean = 0.f;
+  if (!RMS) mean = block_sum<THREADS>(s1, red) / static_cast<float>(h);
+  const float var = RMS ? S2 / static_cast<float>(h) : fmaxf(S2 / static_cast<float>(h) - mean * mean, 0.f);
+  const float rstd = rsqrtf(var + kEps);
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    if (c < vpr) {
+      const int sh = c / vps, lc = c - sh * vps;
+      float g[V], b[V], o[V];
+      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+      if (!RMS) LnVec<T>::load(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V, b);
+#pragma unroll
+      for (int k = 0; k < V; ++k) o[k] = (v[i][k] - mean) * rstd * g[k] + (RMS ? 0.f : b[k]);
+      LnVec<T>::store(static_cast<T*>(Y.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (mean_out && !RMS) mean_out[r] = mean;
+    if (rstd_out) rstd_out[r] = rstd;
+  }
+}
+
+template <typename T, int THREADS, bool RMS>
+__global__ void __launch_bounds__(THREADS) norm_hsh_bwd_dx_kernel(
+    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
+    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int vps,
+    int64_t hs, int64_t h, const float* mean_in, const float* rstd_in) {
+  constexpr int V = LnVec<T>::N;
+  __shared__ float red[THREADS / 32];
+  const int64_t r = blockIdx.x;
+  const int vpr = static_cast<int>(h / V);
+  const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+  float xh[kVptMax][V], gy[kVptMax][V];
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    if (c < vpr) {
+      const int sh = c / vps, lc = c - sh * vps;
+      float g[V], d[V];
+      LnVec<T>::load(static_cast<const T*>(X.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, xh[i]);
+      LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, d);
+      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        xh[i][k] = (xh[i][k] - mean) * rstd;
+        gy[i][k] = d[k] * g[k];
+        s1 += gy[i][k];
+        s2 += gy[i][k] * xh[i][k];
+      }
+    }
+  }
+  const float m2 = block_sum<THREADS>(s2, red) / static_cast<float>(h);
+  const float m1 = RMS ? 0.f : block_sum<THREADS>(s1, red) / static_cast<float>(h);
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    if (c < vpr) {
+      const int sh = c / vps, lc = c - sh * vps;
+      float o[V];
+#pragma unroll
+      for (int k = 0; k < V; ++k) o[k] = rstd * (gy[i][k] - m1 - xh[i][k] * m2);
+      LnVec<T>::store(static_cast<T*>(DX.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+    }
+  }
+}
+
+// dgamma / dbeta of a hidden-sharded norm, pass 1: block (32 column vectors x
+// 8 row lanes) of shard blockIdx.z over rows [split*rps, ...):
+// part[split][0][col] = sum dy * xhat, part[split][1][col] = sum dy (col in 0..h).
+template <typename T, bool RMS>
+__global__ void __launch_bounds__(256) norm_hsh_param_pass1(
+    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray DY, const float* mean_in,
+    const float* rstd_in, int64_t rows, int64_t hs, int64_t h, int64_t rps, float* part) {
+  constexpr int V = LnVec<T>::N;
+  __shared__ float red[2][8][32 * V + 1];
+  const int sh = blockIdx.z;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t vps = hs / V;
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rps;
+  const int64_t r1 = min(rows, r0 + rps);
+  const T* x = static_cast<const T*>(X.p[sh]);
+  const T* dy = static_cast<const T*>(DY.p[sh]);
+  float ag[V], ab[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) ag[k] = ab[k] = 0.f;
+  if (cv < vps) {
+    for (int64_t r = r0 + ty; r < r1; r += 8) {
+      float xv[V], dv[V];
+      LnVec<T>::load(x + r * hs + cv * V, xv);
+      LnVec<T>::load(dy + r * hs + cv * V, dv);
+      const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        ag[k] += dv[k] * ((xv[k] - mean) * rstd);
+        ab[k] += dv[k];
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    red[0][ty][tx * V + k] = ag[k];
+    red[1][ty][tx * V + k] = ab[k];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 32 * V; c += 256) {
+    float sg = 0.f, sb = 0.f;
+#pragma unroll
+    for (int yy = 0; yy < 8; ++yy) {
+      sg += red[0][yy][c];
+      sb += red[1][yy][c];
+    }
+    const int64_t lcol = static_cast<int64_t>(blockIdx.x) * 32 * V + c;
+    if (lcol < hs) {
+      const int64_t col = static_cast<int64_t>(sh) * hs + lcol;
+      part[(static_cast<int64_t>(blockIdx.y) * 2 + 0) * h + col] = sg;
+      part[(static_cast<int64_t>(blockIdx.y) * 2 + 1) * h + col] = sb;
+    }
+  }
+}
+
+__global__ void norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
+                                     const __grid_constant__ MutPtrArray dg,
+                                     const __grid_constant__ MutPtrArray db) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= h) return;
+  float sg = 0.f, sb = 0.f;
+  for (int k = 0; k < splits; ++k) {
+    sg += part[(static_cast<int64_t>(k) * 2 + 0) * h + c];
+    sb += part[(static_cast<int64_t>(k) * 2 + 1) * h + c];
+  }
+  const int sh = static_cast<int>(c / hs);
+  const int64_t lc = c - sh * hs;
+  static_cast<float*>(dg.p[sh])[lc] = sg;
+  if (db.p[sh]) static_cast<float*>(db.p[sh])[lc] = sb;
+}
+
+}  // namespace
+
+namespace tpi {
+
+tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G,
+                                  const PtrArray& B, const MutPtrArray& Y, int p, int64_t rows,
+                                  int64_t h, float* mean, float* rstd, tp_dtype dt,
+                                  cudaStream_t st) {
+  const int V = dt == TP_BF16 ? 8 : 4;
+  const int64_t vpr = h / V, hs = h / p;
+  if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
+  const int vps = static_cast<int>(hs / V);
+  const int th = threads_for(vpr);
+#define TP_NH_FWD(T, TH, R)                                                                        \
+  norm_hsh_fwd_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, B, Y, vps, hs, h, \
+                                                                          mean, rstd)
+#define TP_NH_FWD_T(T, R)              \
+  if (th == 64) TP_NH_FWD(T, 64, R);   \
+  else if (th == 128) TP_NH_FWD(T, 128, R); \
+  else TP_NH_FWD(T, 256, R)
+  if (dt == TP_BF16) {
+    if (rms) { TP_NH_FWD_T(__nv_bfloat16, true); } else { TP_NH_FWD_T(__nv_bfloat16, false); }
+  } else {
+    if (rms) { TP_NH_FWD_T(float, true); } else { TP_NH_FWD_T(float, false); }
+  }
+#undef TP_NH_FWD_T
+#undef TP_NH_FWD
+  return after_launch("norm_sharded_fwd");
+}
+
+tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, const PtrArray& G,
+                                  const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
+                                  const MutPtrArray& db, int p, int64_t rows, int64_t h,
+                                  const float* mean, const float* rstd, tp_dtype dt,
+                                  cudaStream_t st) {
+  const int V = dt == TP_BF16 ? 8 : 4;
+  const int64_t vpr = h / V, hs = h / p;
+  if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
+  const int vps = static_cast<int>(hs / V);
+  const int gx = static_cast<int>((hs / V + 31) / 32);
+  int64_t splits = std::max<int64_t>(1, (static_cast<int64_t>(num_sms()) * 8) / (gx * p));
+  splits = std::min<int64_t>(splits, std::max<int64_t>(1, (rows + 63) / 64));
+  splits = std::min<int64_t>(splits, 1024);
+  const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
+  splits = rows > 0 ? (rows + rps - 1) / rps : 0;
+  void* ws = nullptr;
+  tp_status s = workspace(plan, static_cast<size_t>(std::max<int64_t>(splits, 1)) * 2 * h * sizeof(float), &ws);
+  if (s != TP_OK) return s;
+  float* part = static_cast<float*>(ws);
+  if (rows > 0) {
+    const int th = threads_for(vpr);
+#define TP_NH_BWD(T, TH, R)                                                                 \
+  norm_hsh_bwd_dx_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, DY, DX, \
+                                                                              vps, hs, h, mean, rstd)
+#define TP_NH_BWD_T(T, R)              \
+  if (th == 64) TP_NH_BWD(T, 64, R);   \
+  else if (th == 128) TP_NH_BWD(T, 128, R); \
+  else TP_NH_BWD(T, 256, R)
+    if (dt == TP_BF16) {
+      if (rms) { TP_NH_BWD_T(__nv_bfloat16, true); } else { TP_NH_BWD_T(__nv_bfloat16, false); }
+    } else {
+      if (rms) { TP_NH_BWD_T(float, true); } else { TP_NH_BWD_T(float, false); }
+    }
+#undef TP_NH_BWD_T
+#undef TP_NH_BWD
+    s = after_launch("norm_sharded_bwd/dx");
+    if (s != TP_OK) return s;
+    dim3 grid(gx, static_cast<unsigned>(splits), p);
+    if (dt == TP_BF16) {
+      if (rms) norm_hsh_param_pass1<__nv_bfloat16, true><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
+      else norm_hsh_param_pass1<__nv_bfloat16, false><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
+    } else {
+      if (rms) norm_hsh_param_pass1<float, true><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
+      else norm_hsh_param_pass1<float, false><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
+    }
+    s = after_launch("norm_sharded_bwd/param1");
+    if (s != TP_OK) return s;
+  }
+  norm_hsh_param_pass2<<<static_cast<unsigned>((h + 255) / 256), 256, 0, st>>>(
+      part, static_cast<int>(splits), hs, h, dg, db);
+  return after_launch("norm_sharded_bwd/param2");
+}
+
+}  // namespace tpi

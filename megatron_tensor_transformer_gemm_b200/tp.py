@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libtp.so")
 
 TP_F32, TP_BF16 = 0, 1
 ACTS = {"none": 0, "gelu": 1, "swiglu": 2}
-WHICH = {"mlp": 0, "qkv": 1, "outproj": 2}
+WHICH = {"mlp": 0, "qkv": 1, "outproj": 2, "vocab": 3}
+NORMS = {"layer": 0, "rms": 1}
 STATUS = ["TP_OK", "TP_ERR_ARG", "TP_ERR_DIVISIBILITY", "TP_ERR_ALIGN", "TP_ERR_DTYPE",
           "TP_ERR_UNSUPPORTED", "TP_ERR_CUDA", "TP_ERR_TIMEOUT", "TP_ERR_NO_DEVICE"]
 MAX_SHARDS = 16
@@ -77,6 +78,12 @@ _SIGS = {
     "tp_attention_bwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_column_sum": (_int, [_plan_p, _i64, _i64, _vp, _fp, _int, _vp]),
     "tp_column_sum_static": (_int, [_i64, _i64, _int, _vp, _fp, _int, _vp]),
+    "tp_plan_set_vocab": (_int, [_plan_p, _int, ctypes.POINTER(_int)]),
+    "tp_embedding_fwd": (_int, [_plan_p, _i64, _vp, _vpp, _vp, _vp]),
+    "tp_embedding_bwd": (_int, [_plan_p, _i64, _vp, _vp, _vpp, _vp]),
+    "tp_vocab_cross_entropy": (_int, [_plan_p, _i64, _vpp, _vp, ctypes.c_float, _fp, _fp, _vpp, _vp]),
+    "tp_norm_sharded_fwd": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vpp, _vpp, _fp, _fp, _vp]),
+    "tp_norm_sharded_bwd": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vpp, _fp, _fp, _vpp, _vpp, _vpp, _vp]),
     "tp_row_fwd_reduce": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vp, _vp, _vp, _vp]),
     "tp_row_fwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vp, _vpp, _vpp, _vp]),
     "tp_column_bwd_reduce": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp]),
@@ -155,6 +162,27 @@ class Plan:
     def handle(self):
         return self._h
 
+    def set_vocab(self, vocab: int) -> int:
+        """Pad the vocab so the p shards split it; returns the padded size."""
+        vp = ctypes.c_int(0)
+        check(lib.tp_plan_set_vocab(self._h, vocab, ctypes.byref(vp)), "tp_plan_set_vocab")
+        self.vocab, self.vocab_padded = vocab, vp.value
+        return vp.value
+
+    def embedding_fwd(self, T, ids, E, Y, stream=None):
+        check(lib.tp_embedding_fwd(self._h, T, _ptr(ids), _arr(E), _ptr(Y), _stream(stream)),
+              "tp_embedding_fwd")
+
+    def embedding_bwd(self, T, ids, dY, dE, stream=None):
+        check(lib.tp_embedding_bwd(self._h, T, _ptr(ids), _ptr(dY), _arr(dE), _stream(stream)),
+              "tp_embedding_bwd")
+
+    def vocab_cross_entropy(self, T, logits, labels, grad_scale, loss, lse=None, dlogits=None,
+                            stream=None):
+        check(lib.tp_vocab_cross_entropy(self._h, T, _arr(logits), _ptr(labels), float(grad_scale),
+                                         _ptr(loss), _ptr(lse), _arr(dlogits), _stream(stream)),
+              "tp_vocab_cross_entropy")
+
     def describe(self) -> str:
         buf = ctypes.create_string_buffer(4096)
         check(lib.tp_plan_describe(self._h, buf, len(buf)), "tp_plan_describe")
@@ -220,6 +248,18 @@ class Plan:
         check(lib.tp_layernorm_all_gather_seq(self._h, T, len(X_seq), _arr(X_seq), _ptr(gamma),
                                               _ptr(beta), _ptr(Y_full), _ptr(mean), _ptr(rstd),
                                               _stream(stream)), "tp_layernorm_all_gather_seq")
+
+    def norm_sharded_fwd(self, kind, rows, X, gamma, beta, Y, mean=None, rstd=None, stream=None):
+        """kind: "layer" or "rms"; X, gamma, beta, Y: per-shard tensors (hidden split)."""
+        check(lib.tp_norm_sharded_fwd(self._h, NORMS[kind], rows, _arr(X), _arr(gamma), _arr(beta),
+                                      _arr(Y), _ptr(mean), _ptr(rstd), _stream(stream)),
+              "tp_norm_sharded_fwd")
+
+    def norm_sharded_bwd(self, kind, rows, X, gamma, dY, mean, rstd, dX, dgamma, dbeta=None,
+                         stream=None):
+        check(lib.tp_norm_sharded_bwd(self._h, NORMS[kind], rows, _arr(X), _arr(gamma), _arr(dY),
+                                      _ptr(mean), _ptr(rstd), _arr(dX), _arr(dgamma), _arr(dbeta),
+                                      _stream(stream)), "tp_norm_sharded_bwd")
 
     def attention_fwd(self, batch, seq, QKV, O, LSE=None, stream=None):
         check(lib.tp_attention_fwd(self._h, batch, seq, _arr(QKV), _arr(O), _arr(LSE),

@@ -154,3 +154,14 @@ def test_binding_raises_tperror():
     with pytest.raises(tp.TPError) as e:
         tp.Plan(4096, 11008, 20, 8)
     assert e.value.status_name == "TP_ERR_DIVISIBILITY"
+
+
+def test_vocab_padding_on_the_plan():
+    p = tp.Plan(4096, 0, 0, 8, "bf16", "none")
+    assert p.set_vocab(32000) == 32000
+    assert p.set_vocab(32001) == 32064
+    assert "vocab 32001 padded to 32064" in p.describe()
+    q = tp.Plan(384, 0, 0, 3, "bf16", "none")
+    assert q.set_vocab(100) == 120
+    with pytest.raises(tp.TPError):
+        q.set_vocab(0)
