@@ -233,7 +233,8 @@ def run_ours(args, world, rank, local):
     X_h = inp.X.pin_memory()
     dY_h = inp.dY.pin_memory()
     fused = args.variant == "fused"
-    m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev, fused=fused)
+    m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev, fused=fused,
+              overlap_chunks=4 if args.variant == "overlap" else 0)
     m.load_weights(inp.W1.to(dev), inp.W2.to(dev))
     del inp
     X = X_h.to(dev)
@@ -248,6 +249,8 @@ def run_ours(args, world, rank, local):
                   "column_bwd_reduce")
     orig = {name: getattr(pl, name) for name in gemm_calls + ("reduce_partials",)}
 
+    n_gemm = [0]
+
     def timed(name, bucket):
         fn = orig[name]
 
@@ -256,15 +259,20 @@ def run_ours(args, world, rank, local):
                 return fn(*a, **k)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
+            c0 = tp.launch_count()
             e0.record(stream)
             fn(*a, **k)
             e1.record(stream)
+            if bucket is gemm_ev:
+                n_gemm[0] += tp.launch_count() - c0
             bucket.append((name, e0, e1))
         return wrapper
 
     def step(instrument=False):
         g = gemm_ev if instrument else None
-        r = red_ev if instrument else None
+        # the overlapped variant launches its reduces on a side stream, where
+        # events on this stream would not bracket them: time those standalone
+        r = red_ev if instrument and args.variant != "overlap" else None
         for name in gemm_calls:
             setattr(pl, name, timed(name, g))
         pl.reduce_partials = timed("reduce_partials", r)
@@ -300,7 +308,7 @@ def run_ours(args, world, rank, local):
     # The row_bwd and column_bwd calls each hold two GEMM launches plus a small
     # column-sum (db) only when biases exist (not in this workload).
     gemm_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in gemm_ev)
-    n_gemm_launches = args.steps * 6
+    n_gemm_launches = n_gemm[0]
     gemm_tflops = flops * args.steps / (gemm_ms / 1e3) / 1e12
     peak_t = peaks["bf16_tflops_sustained"]
     red_bytes_launch = P * T * HIDDEN * 2 + T * HIDDEN * 2
@@ -561,6 +569,119 @@ def run_other(args, world, rank, local):
     return 0
 
 
+def run_hbm(args, world, rank, local):
+    """Device-timed HBM throughput of the memory-bound rows, each kernel timed
+    on its own over the same buffers (algorithmic bytes / event time):
+    vocab -- embedding lookup, vocab-parallel cross-entropy (loss + dlogits,
+    in place) and embedding gradient; Llama-7B shapes: vocab 32000, hidden
+    4096, tokens 8x4096, p 8.
+    norm -- hidden-sharded RMSNorm and LayerNorm forward + backward; hidden
+    8192 split over p 8, tokens 8x4096."""
+    import torch
+    from megatron_tensor_transformer_gemm_b200 import tp
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device="cpu").manual_seed(1000 + rank)
+    kernels = []   # (name, fn, algorithmic bytes per launch)
+    if args.workload == "vocab":
+        T, V, h, p = 32768, 32000, 4096, 8
+        plan = tp.Plan(h, 0, 0, p, "bf16", "none")
+        Vp = plan.set_vocab(V)
+        Vs = Vp // p
+        E = [(torch.randn(Vs, h, generator=g) * 0.02).to(torch.bfloat16).to(dev) for _ in range(p)]
+        ids = torch.randint(0, V, (T,), generator=g, dtype=torch.int32).to(dev)
+        Y = torch.empty(T, h, dtype=torch.bfloat16, device=dev)
+        L = [(torch.randn(T, Vs, generator=g) * 2).to(torch.bfloat16).to(dev) for _ in range(p)]
+        loss = torch.empty(T, dtype=torch.float32, device=dev)
+        lse = torch.empty(T, dtype=torch.float32, device=dev)
+        dY = torch.randn(T, h, generator=g).to(torch.bfloat16).to(dev)
+        dE = [torch.empty(Vs, h, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+        kernels = [
+            ("vocab_ce_kernel", lambda: plan.vocab_cross_entropy(T, L, ids, 1.0 / T, loss, lse, L),
+             T * Vp * 2 * 2 + T * 12),
+            ("embed_fwd_kernel", lambda: plan.embedding_fwd(T, ids, E, Y), T * h * 2 * 2 + T * 4),
+            ("embed_bwd_kernel", lambda: plan.embedding_bwd(T, ids, dY, dE), T * h * 2 + Vp * h * 2 + T * 4),
+        ]
+        name = "vocab-parallel embedding + cross-entropy: vocab 32000 (padded to a multiple of 8p), hidden 4096, tokens 8x4096, p=8"
+    else:
+        T, h, p = 32768, 8192, 8
+        plan = tp.Plan(h, 0, 0, p, "bf16", "none")
+        hs = h // p
+        X = [torch.randn(T, hs, generator=g).to(torch.bfloat16).to(dev) for _ in range(p)]
+        gam = [(1 + 0.1 * torch.randn(hs, generator=g)).to(torch.bfloat16).to(dev) for _ in range(p)]
+        bet = [(0.1 * torch.randn(hs, generator=g)).to(torch.bfloat16).to(dev) for _ in range(p)]
+        Yn = [torch.empty_like(x) for x in X]
+        dYn = [torch.randn(T, hs, generator=g).to(torch.bfloat16).to(dev) for _ in range(p)]
+        dXn = [torch.empty_like(x) for x in X]
+        dg = [torch.empty(hs, dtype=torch.float32, device=dev) for _ in range(p)]
+        db = [torch.empty(hs, dtype=torch.float32, device=dev) for _ in range(p)]
+        mean = torch.empty(T, dtype=torch.float32, device=dev)
+        rstd = torch.empty(T, dtype=torch.float32, device=dev)
+        kernels = [
+            ("norm_hsh_fwd_kernel (rms)", lambda: plan.norm_sharded_fwd("rms", T, X, gam, None, Yn, None, rstd),
+             T * h * 2 * 2 + T * 4),
+            ("norm_hsh_bwd (rms)", lambda: plan.norm_sharded_bwd("rms", T, X, gam, dYn, None, rstd, dXn, dg),
+             T * h * 2 * 3 + T * 4),
+            ("norm_hsh_fwd_kernel (layer)", lambda: plan.norm_sharded_fwd("layer", T, X, gam, bet, Yn, mean, rstd),
+             T * h * 2 * 2 + T * 8),
+            ("norm_hsh_bwd (layer)", lambda: plan.norm_sharded_bwd("layer", T, X, gam, dYn, mean, rstd, dXn, dg, db),
+             T * h * 2 * 3 + T * 8),
+        ]
+        name = "hidden-sharded RMSNorm + LayerNorm fwd+bwd: hidden 8192 over p=8, tokens 8x4096"
+
+    def step():
+        for _, fn, _ in kernels:
+            fn()
+    step_bytes = sum(b for _, _, b in kernels)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    tp.launch_count(reset=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = tp.launch_count(reset=True)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    value = step_bytes * args.steps * world / (ms / 1e3) / 1e9
+    per = []
+    for kname, fn, nbytes in kernels:
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        sec = c0.elapsed_time(c1) / 1e3 / args.steps
+        per.append({"kernel": kname, "bytes_per_launch": nbytes, "us": sec * 1e6,
+                    "achieved": nbytes / sec / 1e9, "frac": nbytes / sec / 1e9 / peaks["hbm_gbs"]})
+    top = per[0]
+    if rank != 0:
+        return 0
+    print(json.dumps({"metric": f"{args.workload} algorithmic HBM GB/s on 1 B200", "value": value,
+                      "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch draws)",
+                      "config": {"workload": name, "l2": "every buffer set larger than L2; no flush"},
+                      "roofline": {"bound": "hbm", "kernel": top["kernel"], "achieved": top["achieved"],
+                                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": top["frac"],
+                                   "peak_kind": f"HBM copy ({peaks['source']})", "traffic": None},
+                      "kernels": per, "gpu_launches": launches, "clocks": clk,
+                      "device_status": tp.device_status()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -573,9 +694,11 @@ def main():
     ap.add_argument("--tokens", type=int, default=TOKENS,
                     help="token rows (default 8x4096; smaller values are for profiling only)")
     ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--variant", choices=["fused", "partials"], default="fused",
-                    help="sum over shards inside the GEMMs (fused) or via p partials + reduce")
-    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack"], default="mlp7b",
+    ap.add_argument("--variant", choices=["fused", "partials", "overlap"], default="fused",
+                    help="sum over shards inside the GEMMs (fused), via p partials + reduce, "
+                         "or partials with each token block's reduce overlapped with the next "
+                         "block's GEMM (overlap)")
+    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm"], default="mlp7b",
                     help="mlp7b (the metric's workload) or another config of the suite")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph (other workloads)")
@@ -587,7 +710,12 @@ def main():
         # The oracle runs on rank 0's host cores only; no GPU or process group needed.
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
     world, rank, local = dist_setup()
-    rc = run_ours(args, world, rank, local) if args.workload == "mlp7b" else run_other(args, world, rank, local)
+    if args.workload == "mlp7b":
+        rc = run_ours(args, world, rank, local)
+    elif args.workload in ("vocab", "norm"):
+        rc = run_hbm(args, world, rank, local)
+    else:
+        rc = run_other(args, world, rank, local)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -242,7 +242,10 @@ TP_API tp_status tp_embedding_fwd(tp_plan* plan, int64_t T, const int32_t* ids,
 
 /* Backward of the lookup: dE[i] [Vp/p, hidden] (plan dtype, overwritten) =
  * for each vocab row v of shard i, the sum over tokens with id == v of dY[t]
- * (fp32, in token order, deterministic); rows no token uses are zero. */
+ * (fp32, in token order, deterministic); rows no token uses are zero; ids
+ * outside [0, vocab) are skipped. Uses the plan's device workspace (a stable
+ * bucket sort of the token indices, about Vp/16 * ceil(T/1024) + 2 T ints).
+ * TP_ERR_UNSUPPORTED for Vp > 196608 or T > 2^31 - 1. */
 TP_API tp_status tp_embedding_bwd(tp_plan* plan, int64_t T, const int32_t* ids, const void* dY,
                                   void* const* dE, void* stream);
 
@@ -266,7 +269,9 @@ TP_API tp_status tp_vocab_cross_entropy(tp_plan* plan, int64_t T, const void* co
  *   X[i], Y[i]: [rows, hidden/p] (columns [i*h/p, (i+1)*h/p) of the row);
  *   gamma[i], beta[i]: [hidden/p] (beta ignored, may be NULL, for RMSNorm);
  *   mean (LayerNorm only), rstd: [rows] fp32 outputs (NULL ok).
- * LayerNorm uses var = E[x^2] - mean^2 (the local-sums form), eps = 1e-5. */
+ * LayerNorm uses var = E[x^2] - mean^2 (the local-sums form), eps = 1e-5.
+ * hidden/p must be a multiple of 8; hidden <= 16384 (bf16) or 8192 (fp32),
+ * else TP_ERR_UNSUPPORTED. */
 TP_API tp_status tp_norm_sharded_fwd(tp_plan* plan, tp_norm_kind kind, int64_t rows,
                                      const void* const* X, const void* const* gamma,
                                      const void* const* beta, void* const* Y, float* mean,
@@ -341,8 +346,10 @@ TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, co
                            float* dgamma, float* dbeta, int accumulate, void* stream);
 
 /* Backward of tp_norm_sharded_fwd: dX[i] [rows, hidden/p]; dgamma[i] (and
- * dbeta[i] for LayerNorm; NULL array ok) [hidden/p] fp32 sums over rows. The
- * per-row means of the backward are again local sums reduced over shards. */
+ * dbeta[i] for LayerNorm; NULL array ok) [hidden/p] fp32 sums over rows
+ * (deterministic: fixed per-CTA partials in the plan's workspace, summed in a
+ * fixed order). The per-row means of the backward are again local sums
+ * reduced over shards. One pass over X and dY. */
 TP_API tp_status tp_norm_sharded_bwd(tp_plan* plan, tp_norm_kind kind, int64_t rows,
                                      const void* const* X, const void* const* gamma,
                                      const void* const* dY, const float* mean, const float* rstd,

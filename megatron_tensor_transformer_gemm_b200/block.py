@@ -33,12 +33,18 @@ class TPMLP:
     """One MLP sublayer split over p shards that all live on ``device``."""
 
     def __init__(self, hidden: int, ffn: int, p: int, act: str = "gelu", dtype: str = "bf16",
-                 device="cuda", bias: bool = False, fused: bool = False):
+                 device="cuda", bias: bool = False, fused: bool = False, overlap_chunks: int = 0):
         """fused: sum the shards inside the row GEMM and the column-backward dX
         GEMM (tp_row_fwd_reduce / tp_column_bwd_reduce) instead of writing p
-        partials and reducing them (tp_row_fwd_partial + tp_reduce_partials)."""
+        partials and reducing them (tp_row_fwd_partial + tp_reduce_partials).
+        overlap_chunks > 1 (partials only): split the tokens into that many
+        blocks and reduce block c on a second stream while the GEMM of block
+        c + 1 runs (the compute / communication overlap of "从零实现 Tensor
+        Parallel" §三, with the local reduce in place of the collective)."""
         self.h, self.f, self.p, self.act = hidden, ffn, p, act
         self.fused = fused
+        self.chunks = overlap_chunks if (overlap_chunks > 1 and not fused) else 0
+        self._side = None
         self.plan = Plan(hidden, ffn, 0, p, dtype, act)
         self.dt = self.plan.torch_dtype
         self.device = torch.device(device)
@@ -91,10 +97,44 @@ class TPMLP:
         Y = self.Y if out is None else out
         if self.fused:
             pl.row_fwd_reduce("mlp", T, self.H, self.W2, self.b2, residual, Y)
+        elif self.chunks:
+            self._overlapped(T, lambda r0, r1: pl.row_fwd_partial(
+                                 "mlp", r1 - r0, [h[r0:r1] for h in self.H], self.W2,
+                                 [q[r0:r1] for q in self.P]),
+                             lambda r0, r1: pl.reduce_partials(
+                                 r1 - r0, [q[r0:r1] for q in self.P], self.b2,
+                                 None if residual is None else residual[r0:r1], Y[r0:r1]))
         else:
             pl.row_fwd_partial("mlp", T, self.H, self.W2, self.P)
             pl.reduce_partials(T, self.P, self.b2, residual, Y)
         return Y
+
+    def _overlapped(self, T, gemm, reduce, tail=None):
+        """gemm(r0, r1) on the current stream for token block after block; each
+        block's reduce(r0, r1) on a side stream as soon as its GEMM is done, so
+        it runs under the next block's GEMM (and under tail(), if given, after
+        the last block). The current stream waits for the last reduce before
+        returning."""
+        main = torch.cuda.current_stream()
+        if self._side is None:
+            self._side = torch.cuda.Stream(device=self.device)
+        side = self._side
+        step = -(-T // self.chunks)
+        step = -(-step // 128) * 128           # whole 128-row tiles per block
+        r0 = 0
+        side.wait_stream(main)
+        while r0 < T:
+            r1 = min(T, r0 + step)
+            gemm(r0, r1)
+            ev = torch.cuda.Event()
+            ev.record(main)
+            side.wait_event(ev)
+            with torch.cuda.stream(side):
+                reduce(r0, r1)
+            r0 = r1
+        if tail is not None:
+            tail()
+        main.wait_stream(side)
 
     def backward(self, dY: torch.Tensor, out=None):
         T = dY.shape[0]
@@ -104,6 +144,16 @@ class TPMLP:
         dX = self.dX if out is None else out
         if self.fused:
             pl.column_bwd_reduce("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, dX)
+        elif self.chunks:
+            # dX block by block with the reduces overlapped; the weight gradient
+            # last, so the final block's reduce runs under it too.
+            self._overlapped(T, lambda r0, r1: pl.column_bwd(
+                                 "mlp", r1 - r0, None, [z[r0:r1] for z in self.dZ], self.W1, None,
+                                 None, [q[r0:r1] for q in self.dXp]),
+                             lambda r0, r1: pl.reduce_partials(
+                                 r1 - r0, [q[r0:r1] for q in self.dXp], None, None, dX[r0:r1]),
+                             tail=lambda: pl.column_bwd("mlp", T, self.X, self.dZ, self.W1,
+                                                        self.dW1, self.db1, None))
         else:
             pl.column_bwd("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.dXp)
             pl.reduce_partials(T, self.dXp, None, None, dX)

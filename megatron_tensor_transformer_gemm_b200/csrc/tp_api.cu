@@ -815,8 +815,12 @@ tp_status tp_embedding_bwd(tp_plan* plan, int64_t T, const int32_t* ids, const v
     TP_TRY(check_ptr(dY, "dY"));
   }
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dE), p, "dE", false));
+  size_t bytes = 0;
+  TP_TRY(embedding_bwd_workspace(T, plan->vocab_padded, &bytes));
+  void* ws = nullptr;
+  TP_TRY(workspace(plan, bytes, &ws));
   return launch_embedding_bwd(ids, T, dY, plan->hidden, plan->vocab, plan->vocab_padded,
-                              plan->vocab_padded / p, to_marr(dE, p), plan->dtype,
+                              plan->vocab_padded / p, to_marr(dE, p), plan->dtype, ws,
                               as_stream(stream));
 }
 
@@ -845,7 +849,8 @@ static tp_status check_norm_sharded(const tp_plan* plan, tp_norm_kind kind, int6
   if (kind != TP_NORM_LAYER && kind != TP_NORM_RMS) return fail(TP_ERR_ARG, "unknown norm kind %d", kind);
   const int h = plan->hidden, p = plan->p;
   if ((h / p) % 8) return fail(TP_ERR_UNSUPPORTED, "hidden/p = %d must be a multiple of 8", h / p);
-  if (h > 16384) return fail(TP_ERR_UNSUPPORTED, "norms support hidden <= 16384 (got %d)", h);
+  const int hmax = plan->dtype == TP_BF16 ? 16384 : 8192;  // 2048 16-byte vectors a row
+  if (h > hmax) return fail(TP_ERR_UNSUPPORTED, "norms support hidden <= %d (got %d)", hmax, h);
   return TP_OK;
 }
 

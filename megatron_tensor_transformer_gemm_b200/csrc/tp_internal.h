@@ -79,9 +79,10 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
 // Vocab-parallel embedding and cross-entropy (tp_vocab.cu).
 tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab, int64_t Vs,
                                int64_t T, int64_t h, tp_dtype dt, void* Y, cudaStream_t st);
+tp_status embedding_bwd_workspace(int64_t T, int64_t Vp, size_t* bytes);
 tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, int64_t h, int vocab,
                                int64_t Vp, int64_t Vs, const MutPtrArray& dE, tp_dtype dt,
-                               cudaStream_t st);
+                               void* ws, cudaStream_t st);
 tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
                           const int32_t* labels, float scale, float* loss, float* lse, int64_t T,
                           tp_dtype dt, cudaStream_t st);

@@ -23,8 +23,8 @@ struct LnVec;
 template <>
 struct LnVec<__nv_bfloat16> {
   static constexpr int N = 8;
-  __device__ static void load(const void* p, float* f) {
-    uint4 u = *reinterpret_cast<const uint4*>(p);
+  __device__ static void load(const void* p, float* f) { unpack(*reinterpret_cast<const uint4*>(p), f); }
+  __device__ static void unpack(const uint4 u, float* f) {
     float2 a = tpd::unpack_bf16x2(u.x), b = tpd::unpack_bf16x2(u.y);
     float2 c = tpd::unpack_bf16x2(u.z), d = tpd::unpack_bf16x2(u.w);
     f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
@@ -39,9 +39,10 @@ struct LnVec<__nv_bfloat16> {
 template <>
 struct LnVec<float> {
   static constexpr int N = 4;
-  __device__ static void load(const void* p, float* f) {
-    float4 v = *reinterpret_cast<const float4*>(p);
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  __device__ static void load(const void* p, float* f) { unpack(*reinterpret_cast<const uint4*>(p), f); }
+  __device__ static void unpack(const uint4 u, float* f) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
   }
   __device__ static void store(void* p, const float* f) {
     *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
@@ -341,7 +342,7 @@ namespace {
 
 using tpi::MutPtrArray;
 
-template <typename T, int THREADS, bool RMS>
+template <typename T, int THREADS, int VPT, bool RMS>
 __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
     const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int vps,
@@ -350,10 +351,10 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
   __shared__ float red[THREADS / 32];
   const int64_t r = blockIdx.x;
   const int vpr = static_cast<int>(h / V);
-  float v[kVptMax][V];
+  float v[VPT][V];
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int i = 0; i < kVptMax; ++i) {
+  for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * THREADS;
     if (c < vpr) {
       const int sh = c / vps, lc = c - sh * vps;
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
   const float var = RMS ? S2 / static_cast<float>(h) : fmaxf(S2 / static_cast<float>(h) - mean * mean, 0.f);
   const float rstd = rsqrtf(var + kEps);
 #pragma unroll
-  for (int i = 0; i < kVptMax; ++i) {
+  for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * THREADS;
     if (c < vpr) {
       const int sh = c / vps, lc = c - sh * vps;
@@ -389,102 +390,105 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
   }
 }
 
-template <typename T, int THREADS, bool RMS>
-__global__ void __launch_bounds__(THREADS) norm_hsh_bwd_dx_kernel(
-    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
-    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int vps,
-    int64_t hs, int64_t h, const float* mean_in, const float* rstd_in) {
-  constexpr int V = LnVec<T>::N;
-  __shared__ float red[THREADS / 32];
-  const int64_t r = blockIdx.x;
-  const int vpr = static_cast<int>(h / V);
-  const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
-  float xh[kVptMax][V], gy[kVptMax][V];
-  float s1 = 0.f, s2 = 0.f;
+// Sum of a float pair over the CTA, same result in every thread.
+template <int THREADS>
+__device__ __forceinline__ float2 block_sum2(float2 v, float2* red) {
 #pragma unroll
-  for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
-      const int sh = c / vps, lc = c - sh * vps;
-      float g[V], d[V];
-      LnVec<T>::load(static_cast<const T*>(X.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, xh[i]);
-      LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, d);
-      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
-#pragma unroll
-      for (int k = 0; k < V; ++k) {
-        xh[i][k] = (xh[i][k] - mean) * rstd;
-        gy[i][k] = d[k] * g[k];
-        s1 += gy[i][k];
-        s2 += gy[i][k] * xh[i][k];
-      }
-    }
+  for (int o = 16; o > 0; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
   }
-  const float m2 = block_sum<THREADS>(s2, red) / static_cast<float>(h);
-  const float m1 = RMS ? 0.f : block_sum<THREADS>(s1, red) / static_cast<float>(h);
+  constexpr int W = THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red may still be read by the previous row
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float2 s = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
-      const int sh = c / vps, lc = c - sh * vps;
-      float o[V];
-#pragma unroll
-      for (int k = 0; k < V; ++k) o[k] = rstd * (gy[i][k] - m1 - xh[i][k] * m2);
-      LnVec<T>::store(static_cast<T*>(DX.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
-    }
+  for (int w = 0; w < W; ++w) {
+    s.x += red[w].x;
+    s.y += red[w].y;
   }
+  return s;
 }
 
-// dgamma / dbeta of a hidden-sharded norm, pass 1: block (32 column vectors x
-// 8 row lanes) of shard blockIdx.z over rows [split*rps, ...):
-// part[split][0][col] = sum dy * xhat, part[split][1][col] = sum dy (col in 0..h).
-template <typename T, bool RMS>
-__global__ void __launch_bounds__(256) norm_hsh_param_pass1(
-    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray DY, const float* mean_in,
-    const float* rstd_in, int64_t rows, int64_t hs, int64_t h, int64_t rps, float* part) {
+// Backward of a hidden-sharded norm in one pass over x and dy. CTA b takes
+// rows b, b + gridDim.x, ... in order; thread tid owns the same 16-byte column
+// vectors tid + i * THREADS of every row, so besides dx it keeps running
+// column partials dgamma = sum dy * xhat and dbeta = sum dy in registers and
+// writes them once: part[b][0][col], part[b][1][col]. A second kernel sums the
+// partials over b in order, so the parameter gradients are deterministic.
+// The row is read from HBM once; the dx pass reads it again from L1 / L2.
+template <typename T, int THREADS, int VPT, bool RMS>
+__global__ void __launch_bounds__(THREADS, VPT >= 8 ? 1 : 512 / THREADS) norm_hsh_bwd_fused_kernel(
+    const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
+    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int vps,
+    int64_t hs, int64_t h, int64_t rows, const float* mean_in, const float* rstd_in,
+    float* part) {
   constexpr int V = LnVec<T>::N;
-  __shared__ float red[2][8][32 * V + 1];
-  const int sh = blockIdx.z;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int64_t vps = hs / V;
-  const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + tx;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rps;
-  const int64_t r1 = min(rows, r0 + rps);
-  const T* x = static_cast<const T*>(X.p[sh]);
-  const T* dy = static_cast<const T*>(DY.p[sh]);
-  float ag[V], ab[V];
+  __shared__ float2 red[THREADS / 32];
+  const int vpr = static_cast<int>(h / V);
+  const float inv_h = 1.f / static_cast<float>(h);
+  float pg[VPT][V], pb[VPT][V];
 #pragma unroll
-  for (int k = 0; k < V; ++k) ag[k] = ab[k] = 0.f;
-  if (cv < vps) {
-    for (int64_t r = r0 + ty; r < r1; r += 8) {
-      float xv[V], dv[V];
-      LnVec<T>::load(x + r * hs + cv * V, xv);
-      LnVec<T>::load(dy + r * hs + cv * V, dv);
-      const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+  for (int i = 0; i < VPT; ++i)
 #pragma unroll
-      for (int k = 0; k < V; ++k) {
-        ag[k] += dv[k] * ((xv[k] - mean) * rstd);
-        ab[k] += dv[k];
+    for (int k = 0; k < V; ++k) pg[i][k] = pb[i][k] = 0.f;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+    float2 acc = make_float2(0.f, 0.f);  // (sum g dy, sum g dy xhat) of this thread's columns
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * THREADS;
+      if (c < vpr) {
+        const int sh = c / vps, lc = c - sh * vps;
+        const int64_t off = r * hs + static_cast<int64_t>(lc) * V;
+        float x[V], d[V], g[V];
+        LnVec<T>::load(static_cast<const T*>(X.p[sh]) + off, x);
+        LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + off, d);
+        LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+          const float xh = (x[k] - mean) * rstd;
+          const float gy = d[k] * g[k];
+          acc.x += gy;
+          acc.y += gy * xh;
+          pg[i][k] += d[k] * xh;
+          pb[i][k] += d[k];
+        }
+      }
+    }
+    const float2 tot = block_sum2<THREADS>(acc, red);
+    const float m1 = RMS ? 0.f : tot.x * inv_h, m2 = tot.y * inv_h;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * THREADS;
+      if (c < vpr) {
+        const int sh = c / vps, lc = c - sh * vps;
+        const int64_t off = r * hs + static_cast<int64_t>(lc) * V;
+        float x[V], d[V], g[V], o[V];
+        LnVec<T>::load(static_cast<const T*>(X.p[sh]) + off, x);  // again: an L1 / L2 hit
+        LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + off, d);
+        LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] = rstd * (d[k] * g[k] - m1 - (x[k] - mean) * rstd * m2);
+        LnVec<T>::store(static_cast<T*>(DX.p[sh]) + off, o);
       }
     }
   }
+  float* pgo = part + (static_cast<int64_t>(blockIdx.x) * 2 + 0) * h;
+  float* pbo = part + (static_cast<int64_t>(blockIdx.x) * 2 + 1) * h;
 #pragma unroll
-  for (int k = 0; k < V; ++k) {
-    red[0][ty][tx * V + k] = ag[k];
-    red[1][ty][tx * V + k] = ab[k];
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < 32 * V; c += 256) {
-    float sg = 0.f, sb = 0.f;
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    if (c < vpr) {
 #pragma unroll
-    for (int yy = 0; yy < 8; ++yy) {
-      sg += red[0][yy][c];
-      sb += red[1][yy][c];
-    }
-    const int64_t lcol = static_cast<int64_t>(blockIdx.x) * 32 * V + c;
-    if (lcol < hs) {
-      const int64_t col = static_cast<int64_t>(sh) * hs + lcol;
-      part[(static_cast<int64_t>(blockIdx.y) * 2 + 0) * h + col] = sg;
-      part[(static_cast<int64_t>(blockIdx.y) * 2 + 1) * h + col] = sb;
+      for (int k = 0; k < V; k += 4) {
+        *reinterpret_cast<float4*>(pgo + static_cast<int64_t>(c) * V + k) =
+            make_float4(pg[i][k], pg[i][k + 1], pg[i][k + 2], pg[i][k + 3]);
+        *reinterpret_cast<float4*>(pbo + static_cast<int64_t>(c) * V + k) =
+            make_float4(pb[i][k], pb[i][k + 1], pb[i][k + 2], pb[i][k + 3]);
+      }
     }
   }
 }
@@ -509,6 +513,24 @@ __global__ void norm_hsh_param_pass2(const float* part, int splits, int64_t hs, 
 
 namespace tpi {
 
+// Threads for the sharded norms: up to 256, so a thread holds at most 4
+// vectors up to 1024 vectors a row (8 beyond).
+int hsh_threads(int64_t vpr) { return vpr <= 64 ? 64 : vpr <= 128 ? 128 : 256; }
+
+// Vectors per thread for a row of vpr vectors over th threads: 1, 2, 4 or 8.
+int vpt_for(int64_t vpr, int th) {
+  const int64_t need = (vpr + th - 1) / th;
+  return need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
+}
+
+#define TP_NH_DISPATCH(LAUNCH, T, R)                 \
+  if (th == 64) LAUNCH(T, 64, 1, R);                 \
+  else if (th == 128) LAUNCH(T, 128, 1, R);          \
+  else if (vpt == 1) LAUNCH(T, 256, 1, R);           \
+  else if (vpt == 2) LAUNCH(T, 256, 2, R);           \
+  else if (vpt == 4) LAUNCH(T, 256, 4, R);           \
+  else LAUNCH(T, 256, 8, R)
+
 tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G,
                                   const PtrArray& B, const MutPtrArray& Y, int p, int64_t rows,
                                   int64_t h, float* mean, float* rstd, tp_dtype dt,
@@ -517,20 +539,18 @@ tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G
   const int64_t vpr = h / V, hs = h / p;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
   const int vps = static_cast<int>(hs / V);
-  const int th = threads_for(vpr);
-#define TP_NH_FWD(T, TH, R)                                                                        \
-  norm_hsh_fwd_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, B, Y, vps, hs, h, \
-                                                                          mean, rstd)
-#define TP_NH_FWD_T(T, R)              \
-  if (th == 64) TP_NH_FWD(T, 64, R);   \
-  else if (th == 128) TP_NH_FWD(T, 128, R); \
-  else TP_NH_FWD(T, 256, R)
+  const int th = hsh_threads(vpr);
+  const int vpt = vpt_for(vpr, th);
+#define TP_NH_FWD(T, TH, VP, R)                                                   \
+  norm_hsh_fwd_kernel<T, TH, VP, R><<<static_cast<unsigned>(rows), TH, 0, st>>>( \
+      X, G, B, Y, vps, hs, h, mean, rstd)
   if (dt == TP_BF16) {
-    if (rms) { TP_NH_FWD_T(__nv_bfloat16, true); } else { TP_NH_FWD_T(__nv_bfloat16, false); }
+    if (rms) { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, true); }
+    else { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, false); }
   } else {
-    if (rms) { TP_NH_FWD_T(float, true); } else { TP_NH_FWD_T(float, false); }
+    if (rms) { TP_NH_DISPATCH(TP_NH_FWD, float, true); }
+    else { TP_NH_DISPATCH(TP_NH_FWD, float, false); }
   }
-#undef TP_NH_FWD_T
 #undef TP_NH_FWD
   return after_launch("norm_sharded_fwd");
 }
@@ -544,48 +564,35 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   const int64_t vpr = h / V, hs = h / p;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
   const int vps = static_cast<int>(hs / V);
-  const int gx = static_cast<int>((hs / V + 31) / 32);
-  int64_t splits = std::max<int64_t>(1, (static_cast<int64_t>(num_sms()) * 8) / (gx * p));
-  splits = std::min<int64_t>(splits, std::max<int64_t>(1, (rows + 63) / 64));
-  splits = std::min<int64_t>(splits, 1024);
-  const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
-  splits = rows > 0 ? (rows + rps - 1) / rps : 0;
+  const int th = hsh_threads(vpr);
+  const int vpt = vpt_for(vpr, th);
+  // As many CTAs as the launch bounds fit at once, at most one per row.
+  const int per_sm = vpt >= 8 ? 1 : 512 / th;
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rows, static_cast<int64_t>(num_sms()) * per_sm));
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(std::max<int64_t>(splits, 1)) * 2 * h * sizeof(float), &ws);
+  tp_status s = workspace(plan, static_cast<size_t>(grid) * 2 * h * sizeof(float), &ws);
   if (s != TP_OK) return s;
   float* part = static_cast<float*>(ws);
   if (rows > 0) {
-    const int th = threads_for(vpr);
-#define TP_NH_BWD(T, TH, R)                                                                 \
-  norm_hsh_bwd_dx_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, DY, DX, \
-                                                                              vps, hs, h, mean, rstd)
-#define TP_NH_BWD_T(T, R)              \
-  if (th == 64) TP_NH_BWD(T, 64, R);   \
-  else if (th == 128) TP_NH_BWD(T, 128, R); \
-  else TP_NH_BWD(T, 256, R)
+#define TP_NH_BWD(T, TH, VP, R)                                                       \
+  norm_hsh_bwd_fused_kernel<T, TH, VP, R><<<static_cast<unsigned>(grid), TH, 0, st>>>( \
+      X, G, DY, DX, vps, hs, h, rows, mean, rstd, part)
     if (dt == TP_BF16) {
-      if (rms) { TP_NH_BWD_T(__nv_bfloat16, true); } else { TP_NH_BWD_T(__nv_bfloat16, false); }
+      if (rms) { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
+      else { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, false); }
     } else {
-      if (rms) { TP_NH_BWD_T(float, true); } else { TP_NH_BWD_T(float, false); }
+      if (rms) { TP_NH_DISPATCH(TP_NH_BWD, float, true); }
+      else { TP_NH_DISPATCH(TP_NH_BWD, float, false); }
     }
-#undef TP_NH_BWD_T
 #undef TP_NH_BWD
-    s = after_launch("norm_sharded_bwd/dx");
-    if (s != TP_OK) return s;
-    dim3 grid(gx, static_cast<unsigned>(splits), p);
-    if (dt == TP_BF16) {
-      if (rms) norm_hsh_param_pass1<__nv_bfloat16, true><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
-      else norm_hsh_param_pass1<__nv_bfloat16, false><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
-    } else {
-      if (rms) norm_hsh_param_pass1<float, true><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
-      else norm_hsh_param_pass1<float, false><<<grid, 256, 0, st>>>(X, DY, mean, rstd, rows, hs, h, rps, part);
-    }
-    s = after_launch("norm_sharded_bwd/param1");
+    s = after_launch("norm_sharded_bwd");
     if (s != TP_OK) return s;
   }
   norm_hsh_param_pass2<<<static_cast<unsigned>((h + 255) / 256), 256, 0, st>>>(
-      part, static_cast<int>(splits), hs, h, dg, db);
-  return after_launch("norm_sharded_bwd/param2");
+      part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg, db);
+  return after_launch("norm_sharded_bwd/param");
 }
+
+#undef TP_NH_DISPATCH
 
 }  // namespace tpi

@@ -11,7 +11,8 @@
 //              memory (no atomics), then writes its rows to the owning shard.
 //  ce          per token row: max, sum of exp and the target logit over the
 //              real (non-padding) columns of all shards -- the shards' local
-//              max / sum / target reduced over shards -- then loss = lse - z_t
+//              max / sum / target reduced over shards, here merged as running
+//              (max, sum) pairs in one streaming pass -- then loss = lse - z_t
 //              and the gradient of the scaled loss, (softmax - onehot) * scale,
 //              written to dlogits (which may alias the logits).
 #include <algorithm>
@@ -45,113 +46,170 @@ __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ Ptr
   }
 }
 
-constexpr int kEmbRows = 32;    // vocab rows per CTA
-constexpr int kEmbCols = 512;   // columns per CTA (2 per thread)
+// Embedding gradient as a stable bucket sort of the tokens, then a gather-sum:
+//   count    per 1024-token block, how many of its tokens fall in each bucket of
+//            16 vocab ids (cnt[bucket][block], bucket-major);
+//   scan     exclusive prefix over cnt in that order: the start of each
+//            (bucket, block) run in the sorted token list;
+//   scatter  each token's slot = its run start + the number of earlier tokens
+//            of its block in the same bucket, so every bucket lists its tokens
+//            in token order;
+//   accum    one CTA per (bucket, 512-column tile) sums the listed dY rows in
+//            that order in fp32 and writes its 16 rows of dE (zeros if none).
+// No atomics touch the sums, so the result is deterministic.
+constexpr int kEmbRows = 16;    // vocab ids per bucket
+constexpr int kEmbCols = 512;   // columns per accumulating CTA (2 per thread)
 constexpr int kEmbThreads = 256;
-constexpr int kIdTile = 1024;
+constexpr int kTokBlock = 1024; // tokens per count / scatter CTA
+constexpr int kEmbMaxBuckets = 12288;  // 48 KB of shared counters (padded vocab <= 196608)
+constexpr int kListChunk = 512;
 
-// dE rows [v0, v0 + 32) x columns [c0, c0 + 512) of the padded vocab.
-template <typename T>
-__global__ void __launch_bounds__(kEmbThreads) embed_bwd_kernel(
-    const int32_t* ids, int64_t ntok, const T* dY, int64_t h, int vocab, int64_t Vs, int64_t Vp,
-    const __grid_constant__ MutPtrArray dE) {
-  extern __shared__ float acc[];  // [kEmbRows][kEmbCols]
-  __shared__ int match[kIdTile];
-  __shared__ int nmatch;
-  __shared__ int wcount[kEmbThreads / 32];
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kEmbRows;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kEmbCols;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kEmbRows * kEmbCols; i += kEmbThreads) acc[i] = 0.f;
+__device__ __forceinline__ bool valid_id(int id, int vocab) { return id >= 0 && id < vocab; }
+
+__global__ void __launch_bounds__(kTokBlock) emb_bucket_count(const int32_t* ids, int64_t ntok,
+                                                              int vocab, int nb, int nblk,
+                                                              int* cnt) {
+  __shared__ int hist[kEmbMaxBuckets];
+  for (int i = threadIdx.x; i < nb; i += kTokBlock) hist[i] = 0;
   __syncthreads();
-  for (int64_t base = 0; base < ntok; base += kIdTile) {
-    // Ordered compaction of this tile's matching tokens: thread tid checks
-    // tokens base + tid*4 .. +3, warp ballots give each match its rank.
-    int mine[4], cnt = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t t = base + tid * 4 + k;
-      mine[k] = -1;
-      if (t < ntok) {
-        const int id = ids[t];
-        if (id >= v0 && id < v0 + kEmbRows && id < vocab) {
-          mine[k] = static_cast<int>(t - base);
-          ++cnt;
-        }
-      }
-    }
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane == 31) wcount[warp] = incl;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kTokBlock + threadIdx.x;
+  if (t < ntok) {
+    const int id = ids[t];
+    if (valid_id(id, vocab)) atomicAdd(&hist[id / kEmbRows], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nb; i += kTokBlock)
+    cnt[static_cast<int64_t>(i) * nblk + blockIdx.x] = hist[i];
+}
+
+// One CTA: a[0..n) <- exclusive prefix sums, a[n] <- the total.
+__global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
+  __shared__ int part[1024];
+  const int tid = threadIdx.x;
+  const int64_t chunk = (n + 1023) / 1024;
+  const int64_t lo = tid * chunk, hi = lo + chunk < n ? lo + chunk : n;
+  int sum = 0;
+  for (int64_t i = lo; i < hi; ++i) sum += a[i];
+  part[tid] = sum;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive Hillis-Steele scan of the partial sums
+    const int v = tid >= o ? part[tid - o] : 0;
     __syncthreads();
-    int woff = 0, total = 0;
-    for (int w = 0; w < kEmbThreads / 32; ++w) {
-      if (w < warp) woff += wcount[w];
-      total += wcount[w];
-    }
-    int pos = woff + incl - cnt;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if (mine[k] >= 0) match[pos++] = mine[k];
-    if (tid == 0) nmatch = total;
+    part[tid] += v;
     __syncthreads();
-    // Accumulate the matches in token order; thread tid owns columns 2 tid, 2 tid + 1.
-    const int64_t col = c0 + 2 * tid;
-    for (int m = 0; m < nmatch; ++m) {
-      const int64_t t = base + match[m];
-      const int r = ids[t] - static_cast<int>(v0);
-      if (col < h) {
-        float a, b;
-        if constexpr (sizeof(T) == 2) {
-          const float2 f = tpd::unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dY + t * h + col));
-          a = f.x;
-          b = f.y;
-        } else {
-          a = dY[t * h + col];
-          b = dY[t * h + col + 1];
-        }
-        acc[r * kEmbCols + 2 * tid] += a;
-        acc[r * kEmbCols + 2 * tid + 1] += b;
-      }
+  }
+  int run = part[tid] - sum;
+  for (int64_t i = lo; i < hi; ++i) {
+    const int v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  if (tid == 1023) a[n] = part[1023];
+}
+
+// sorted[k] = (token, id - bucket * kEmbRows) of the k-th entry of the sorted list.
+__global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* ids, int64_t ntok,
+                                                                int vocab, int nb, int nblk,
+                                                                const int* off, int2* sorted) {
+  __shared__ int seen[kEmbMaxBuckets];
+  for (int i = threadIdx.x; i < nb; i += kTokBlock) seen[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kTokBlock + threadIdx.x;
+  const int id = t < ntok ? ids[t] : -1;
+  const bool valid = valid_id(id, vocab);
+  const int b = valid ? id / kEmbRows : -1;
+  const unsigned peers = __match_any_sync(0xffffffffu, b);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  int base = 0;
+  // Warps in order: each reads how many tokens of its bucket earlier warps
+  // placed, then the first lane of each bucket group adds its group's size.
+  for (int w = 0; w < kTokBlock / 32; ++w) {
+    if (warp == w) {
+      if (valid) base = seen[b];
+      __syncwarp();
+      if (valid && rank == 0) seen[b] += __popc(peers);
     }
     __syncthreads();
   }
-  // Write the rows to their shards (every padded row gets written: zeros if unused).
+  if (valid)
+    sorted[off[static_cast<int64_t>(b) * nblk + blockIdx.x] + base + rank] =
+        make_int2(static_cast<int>(t), id - b * kEmbRows);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kEmbThreads) emb_bucket_accum(
+    const int2* sorted, const int* off, int nb, int nblk, const T* dY, int64_t h, int64_t Vs,
+    int64_t Vp, const __grid_constant__ MutPtrArray dE) {
+  extern __shared__ float acc[];  // [kEmbRows][kEmbCols]; thread tid owns columns 2 tid, 2 tid + 1
+  __shared__ int ltok[kListChunk];
+  __shared__ int lrow[kListChunk];
+  const int b = blockIdx.x;
+  const int64_t v0 = static_cast<int64_t>(b) * kEmbRows;
+  const int tid = threadIdx.x;
+  const int64_t col = static_cast<int64_t>(blockIdx.y) * kEmbCols + 2 * tid;
+  const bool col_ok = col < h;
+#pragma unroll 4
+  for (int r = 0; r < kEmbRows; ++r) {
+    acc[r * kEmbCols + 2 * tid] = 0.f;
+    acc[r * kEmbCols + 2 * tid + 1] = 0.f;
+  }
+  const int start = off[static_cast<int64_t>(b) * nblk];
+  const int end = off[static_cast<int64_t>(b + 1) * nblk];  // off[nb * nblk] is the total
+  for (int c0 = start; c0 < end; c0 += kListChunk) {
+    const int n = end - c0 < kListChunk ? end - c0 : kListChunk;
+    __syncthreads();  // the previous chunk's list is consumed
+    for (int k = tid; k < n; k += kEmbThreads) {
+      const int2 e = sorted[c0 + k];
+      ltok[k] = e.x;
+      lrow[k] = e.y;
+    }
+    __syncthreads();
+    if (!col_ok) continue;
+    int k = 0;
+    for (; k + 8 <= n; k += 8) {  // eight independent row loads in flight, summed in list order
+      float2 f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t off_t = static_cast<int64_t>(ltok[k + u]) * h + col;
+        if constexpr (sizeof(T) == 2) {
+          f[u] = tpd::unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dY + off_t));
+        } else {
+          f[u] = *reinterpret_cast<const float2*>(dY + off_t);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float* a2 = acc + lrow[k + u] * kEmbCols + 2 * tid;
+        a2[0] += f[u].x;
+        a2[1] += f[u].y;
+      }
+    }
+    for (; k < n; ++k) {
+      const int64_t off_t = static_cast<int64_t>(ltok[k]) * h + col;
+      float2 f;
+      if constexpr (sizeof(T) == 2) f = tpd::unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dY + off_t));
+      else f = *reinterpret_cast<const float2*>(dY + off_t);
+      float* a2 = acc + lrow[k] * kEmbCols + 2 * tid;
+      a2[0] += f.x;
+      a2[1] += f.y;
+    }
+  }
+  if (!col_ok) return;
+  // Write the bucket's rows to their shards (every padded row: zeros if unused).
   for (int r = 0; r < kEmbRows; ++r) {
     const int64_t v = v0 + r;
     if (v >= Vp) break;
     const int s = static_cast<int>(v / Vs);
-    const int64_t col = c0 + 2 * tid;
-    if (col < h) {
-      T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + col;
-      if constexpr (sizeof(T) == 2) {
-        *reinterpret_cast<uint32_t*>(dst) =
-            tpd::pack_bf16x2(acc[r * kEmbCols + 2 * tid], acc[r * kEmbCols + 2 * tid + 1]);
-      } else {
-        dst[0] = acc[r * kEmbCols + 2 * tid];
-        dst[1] = acc[r * kEmbCols + 2 * tid + 1];
-      }
+    T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + col;
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint32_t*>(dst) =
+          tpd::pack_bf16x2(acc[r * kEmbCols + 2 * tid], acc[r * kEmbCols + 2 * tid + 1]);
+    } else {
+      *reinterpret_cast<float2*>(dst) =
+          make_float2(acc[r * kEmbCols + 2 * tid], acc[r * kEmbCols + 2 * tid + 1]);
     }
   }
-}
-
-template <int THREADS>
-__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float u = __shfl_xor_sync(0xffffffffu, v, o);
-    v = is_max ? fmaxf(v, u) : v + u;
-  }
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = red[0];
-  for (int w = 1; w < THREADS / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
-  return r;
 }
 
 template <typename T>
@@ -160,60 +218,249 @@ __device__ __forceinline__ float ld_logit(const void* p, int64_t i) {
   else return static_cast<const float*>(p)[i];
 }
 
-template <typename T>
-__device__ __forceinline__ void st_grad(void* p, int64_t i, float v) {
-  if constexpr (sizeof(T) == 2) static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
-  else static_cast<float*>(p)[i] = v;
+// Running (max, sum of exp2) pair in the log2 domain: the pair (m, s) stands
+// for s * 2^m. Merging rescales the smaller side; an empty side is (-inf, 0).
+struct MaxSum {
+  float m, s;
+};
+
+__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b) {
+  const float m = fmaxf(a.m, b.m);
+  if (m == -INFINITY) return {m, 0.f};
+  return {m, a.s * exp2f(a.m - m) + b.s * exp2f(b.m - m)};
 }
 
-// One CTA per token row t.
+template <int THREADS>
+__device__ __forceinline__ MaxSum block_merge(MaxSum v, float2* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    MaxSum u{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
+    v = merge(v, u);
+  }
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(v.m, v.s);
+  __syncthreads();
+  MaxSum r{red[0].x, red[0].y};
+  for (int w = 1; w < THREADS / 32; ++w) r = merge(r, MaxSum{red[w].x, red[w].y});
+  return r;
+}
+
+// 16 bytes of logits as floats (8 bf16 or 4 fp32).
+template <typename T>
+struct Vec {
+  static constexpr int N = 16 / sizeof(T);
+  float v[N];
+  __device__ __forceinline__ void load(const void* base, int64_t i) {
+    // plain load: the gradient may overwrite the logits in place
+    unpack(reinterpret_cast<const uint4*>(base)[i]);
+  }
+  __device__ __forceinline__ void unpack(const uint4 u) {
+    if constexpr (sizeof(T) == 2) {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = tpd::unpack_bf16x2(w[k]);
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+      }
+    } else {
+      v[0] = __uint_as_float(u.x);
+      v[1] = __uint_as_float(u.y);
+      v[2] = __uint_as_float(u.z);
+      v[3] = __uint_as_float(u.w);
+    }
+  }
+  __device__ __forceinline__ void store(void* base, int64_t i) const {
+    uint4 u;
+    if constexpr (sizeof(T) == 2) {
+      u.x = tpd::pack_bf16x2(v[0], v[1]);
+      u.y = tpd::pack_bf16x2(v[2], v[3]);
+      u.z = tpd::pack_bf16x2(v[4], v[5]);
+      u.w = tpd::pack_bf16x2(v[6], v[7]);
+    } else {
+      u = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                     __float_as_uint(v[3]));
+    }
+    reinterpret_cast<uint4*>(base)[i] = u;
+  }
+};
+
+// One CTA per token row t. Pass 1 streams every shard's slice of the row once
+// in 16-byte vectors and keeps a running (max, sum of exp) per thread; pass 2
+// re-reads it (mostly from L2) to write the gradient. Exponentials are taken
+// as exp2 of logits scaled by log2(e). Vs is a multiple of 8 (the vocab is
+// padded to a multiple of 8 p), so every shard row starts on 16 bytes.
 template <typename T, int THREADS>
 __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
     const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
     int vocab, const int32_t* labels, float scale, float* loss, float* lse_out,
     unsigned* status) {
-  __shared__ float red[THREADS / 32];
+  constexpr int N = Vec<T>::N;
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ float2 red[THREADS / 32];
   __shared__ float ztarget;
   const int64_t t = blockIdx.x;
   const int label = labels[t];
-  const int64_t row_total = static_cast<int64_t>(p) * Vs;
+  const bool ignore = label < 0 || label >= vocab;
   if (threadIdx.x == 0) {
     ztarget = 0.f;
     if (label >= vocab) atomicOr(status, kStatusBadIndex);
+    if (!ignore) {
+      const int s = static_cast<int>(label / Vs);
+      ztarget = ld_logit<T>(L.p[s], t * Vs + (label - s * Vs));
+    }
   }
-  // pass 1: max over real columns (and the target logit)
-  float mx = -INFINITY;
-  for (int64_t v = threadIdx.x; v < row_total; v += THREADS) {
-    if (v >= vocab) break;
-    const int s = static_cast<int>(v / Vs);
-    const float z = ld_logit<T>(L.p[s], t * Vs + (v - s * Vs));
-    mx = fmaxf(mx, z);
-    if (v == label) ztarget = z;
+  const int64_t nv = Vs / N;  // vectors per shard row
+  MaxSum acc{-INFINITY, 0.f};
+  for (int s = 0; s < p; ++s) {
+    const int64_t col0 = static_cast<int64_t>(s) * Vs;
+    if (col0 >= vocab) break;
+    const int64_t row = t * nv;
+    for (int64_t j = threadIdx.x; j < nv; j += THREADS) {
+      Vec<T> x;
+      x.load(L.p[s], row + j);
+      const int64_t c = col0 + j * N;
+      float lm = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < N; ++k) {
+        x.v[k] = (c + k < vocab) ? x.v[k] * kLog2e : -INFINITY;
+        lm = fmaxf(lm, x.v[k]);
+      }
+      if (lm == -INFINITY) continue;  // all padding
+      if (lm > acc.m) {
+        acc.s *= exp2f(acc.m - lm);
+        acc.m = lm;
+      }
+#pragma unroll
+      for (int k = 0; k < N; ++k) acc.s += exp2f(x.v[k] - acc.m);
+    }
   }
-  const float m = block_reduce<THREADS>(mx, red, true);
-  // pass 2: sum of exp(z - m)
-  float se = 0.f;
-  for (int64_t v = threadIdx.x; v < vocab; v += THREADS) {
-    const int s = static_cast<int>(v / Vs);
-    se += expf(ld_logit<T>(L.p[s], t * Vs + (v - s * Vs)) - m);
-  }
-  const float S = block_reduce<THREADS>(se, red, false);
-  const float lse = m + logf(S);
-  const bool ignore = label < 0 || label >= vocab;
+  const MaxSum tot = block_merge<THREADS>(acc, red);
+  const float lse2 = tot.m + log2f(tot.s);  // log2 of the sum of exp
   if (threadIdx.x == 0) {
+    const float lse = lse2 * 0.6931471805599453f;
     loss[t] = ignore ? 0.f : lse - ztarget;
     if (lse_out) lse_out[t] = lse;
   }
-  // pass 3: gradient of scale * loss (zero for ignored tokens and padding columns)
+  // pass 2: gradient of scale * loss (zero for ignored tokens and padding columns)
   if (G.p[0] == nullptr) return;
-  for (int64_t v = threadIdx.x; v < row_total; v += THREADS) {
-    const int s = static_cast<int>(v / Vs);
-    const int64_t off = t * Vs + (v - s * Vs);
-    float g = 0.f;
-    if (!ignore && v < vocab) g = (expf(ld_logit<T>(L.p[s], off) - lse) - (v == label ? 1.f : 0.f)) * scale;
-    st_grad<T>(G.p[s], off, g);
+  for (int s = 0; s < p; ++s) {
+    const int64_t col0 = static_cast<int64_t>(s) * Vs;
+    const int64_t row = t * nv;
+    for (int64_t j = threadIdx.x; j < nv; j += THREADS) {
+      Vec<T> x;
+      const int64_t c = col0 + j * N;
+      if (!ignore && c < vocab) x.load(L.p[s], row + j);
+#pragma unroll
+      for (int k = 0; k < N; ++k) {
+        float g = 0.f;
+        if (!ignore && c + k < vocab)
+          g = (exp2f(fmaf(x.v[k], kLog2e, -lse2)) - (c + k == label ? 1.f : 0.f)) * scale;
+        x.v[k] = g;
+      }
+      x.store(G.p[s], row + j);
+    }
   }
 }
+
+// Rows of up to kCeSmemMax bytes: one CTA per token row copies the row's p
+// shard slices into shared memory with bulk copies (one per shard, completing
+// on one mbarrier), takes each thread's max and sum of exp2 relative to it
+// from there, merges the (max, sum) pairs over the CTA and writes the gradient
+// from the same shared copy, so the logits cross HBM exactly once and no
+// registers hold the row. The shards are contiguous slices of the padded
+// vocab, so 16-byte vector i of the row holds columns [i * N, (i + 1) * N).
+template <typename T, int THREADS>
+__global__ void __launch_bounds__(THREADS) vocab_ce_smem_kernel(
+    const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
+    int vocab, const int32_t* labels, float scale, float* loss, float* lse_out,
+    unsigned* status) {
+  constexpr int N = Vec<T>::N;
+  constexpr float kLog2e = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t srow[];
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  __shared__ float2 red[THREADS / 32];
+  const int64_t t = blockIdx.x;
+  const uint32_t shard_bytes = static_cast<uint32_t>(Vs * sizeof(T));
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    tpd::mbar_init(&bar, 1);
+    tpd::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tpd::mbar_arrive_expect_tx(&bar, shard_bytes * static_cast<uint32_t>(p));
+    for (int s = 0; s < p; ++s)
+      tpd::bulk_load(srow + static_cast<size_t>(s) * shard_bytes,
+                     static_cast<const uint8_t*>(L.p[s]) + t * shard_bytes, shard_bytes, &bar);
+  }
+  const int label = labels[t];
+  const bool ignore = label < 0 || label >= vocab;
+  const bool ok = tpd::mbar_wait(&bar, 0, &abort_flag, status);
+  if (!__syncthreads_and(ok)) {
+    // The copies did not land in time: give them one more bounded wait so
+    // none is still writing this CTA's shared memory when it exits.
+    if (threadIdx.x == 0) {
+      int again = 0;
+      tpd::mbar_wait(&bar, 0, &again, nullptr);
+    }
+    __syncthreads();
+    return;
+  }
+  const int nv = static_cast<int>(Vs / N);
+  const int total = p * nv;
+  const uint4* row = reinterpret_cast<const uint4*>(srow);
+  float m = -INFINITY;
+  for (int i = threadIdx.x; i < total; i += THREADS) {
+    Vec<T> x;
+    x.unpack(row[i]);
+#pragma unroll
+    for (int e = 0; e < N; ++e)
+      if (i * N + e < vocab) m = fmaxf(m, x.v[e] * kLog2e);
+  }
+  float sum = 0.f;
+  if (m != -INFINITY) {
+    for (int i = threadIdx.x; i < total; i += THREADS) {
+      Vec<T> x;
+      x.unpack(row[i]);
+#pragma unroll
+      for (int e = 0; e < N; ++e)
+        if (i * N + e < vocab) sum += exp2f(fmaf(x.v[e], kLog2e, -m));
+    }
+  }
+  const MaxSum tot = block_merge<THREADS>(MaxSum{m, sum}, red);
+  const float lse2 = tot.m + log2f(tot.s);
+  if (threadIdx.x == 0) {
+    if (label >= vocab) atomicOr(status, kStatusBadIndex);
+    float zt = 0.f;
+    if (!ignore) {
+      Vec<T> x;
+      x.unpack(row[label / N]);
+      zt = x.v[label % N];
+    }
+    const float lse = lse2 * 0.6931471805599453f;
+    loss[t] = ignore ? 0.f : lse - zt;
+    if (lse_out) lse_out[t] = lse;
+  }
+  if (G.p[0] == nullptr) return;
+  for (int i = threadIdx.x; i < total; i += THREADS) {
+    Vec<T> x;
+    x.unpack(row[i]);
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+      const int c = i * N + e;
+      float g = 0.f;
+      if (!ignore && c < vocab)
+        g = (exp2f(fmaf(x.v[e], kLog2e, -lse2)) - (c == label ? 1.f : 0.f)) * scale;
+      x.v[e] = g;
+    }
+    const int s = i / nv;
+    x.store(G.p[s], t * nv + (i - s * nv));
+  }
+}
+
+constexpr int kCeSmemSmall = 64 * 1024;    // up to 3 CTAs per SM
+constexpr int kCeSmemMax = 200 * 1024;     // one CTA per SM
 
 int sms() {
   int dev = 0, n = 0;
@@ -241,29 +488,58 @@ tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab,
   return after_launch("embedding_fwd");
 }
 
+tp_status embedding_bwd_workspace(int64_t T, int64_t Vp, size_t* bytes) {
+  const int64_t nb = (Vp + kEmbRows - 1) / kEmbRows;
+  const int64_t nblk = (T + kTokBlock - 1) / kTokBlock;
+  if (nb > kEmbMaxBuckets)
+    return fail(TP_ERR_UNSUPPORTED, "embedding backward supports a padded vocab of at most %d rows",
+                kEmbMaxBuckets * kEmbRows);
+  if (T > 0x7fffffffLL || nb * nblk + 1 > 0x7fffffffLL)
+    return fail(TP_ERR_UNSUPPORTED, "embedding backward: %lld tokens is too many", (long long)T);
+  *bytes = static_cast<size_t>(nb * nblk + 1 + 1 + 2 * T) * sizeof(int);  // + 1: int2 alignment
+  return TP_OK;
+}
+
 tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, int64_t h, int vocab,
                                int64_t Vp, int64_t Vs, const MutPtrArray& dE, tp_dtype dt,
-                               cudaStream_t st) {
+                               void* ws, cudaStream_t st) {
+  const int nb = static_cast<int>((Vp + kEmbRows - 1) / kEmbRows);
+  const int nblk = static_cast<int>((T + kTokBlock - 1) / kTokBlock);
+  int* cnt = static_cast<int*>(ws);
+  const int64_t ncnt = static_cast<int64_t>(nb) * nblk + 1;
+  int2* sorted = reinterpret_cast<int2*>(cnt + ncnt + (ncnt & 1));
   const int smem = kEmbRows * kEmbCols * 4;
   static bool attr[2] = {false, false};
   const int k = dt == TP_BF16 ? 0 : 1;
   if (!attr[k]) {
     cudaError_t e = dt == TP_BF16
-        ? cudaFuncSetAttribute(embed_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-        : cudaFuncSetAttribute(embed_bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        ? cudaFuncSetAttribute(emb_bucket_accum<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+        : cudaFuncSetAttribute(emb_bucket_accum<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     tp_status s = cuda_status(e, "cudaFuncSetAttribute(embedding_bwd)");
     if (s != TP_OK) return s;
     attr[k] = true;
   }
-  dim3 grid(static_cast<unsigned>((Vp + kEmbRows - 1) / kEmbRows),
-            static_cast<unsigned>((h + kEmbCols - 1) / kEmbCols));
+  if (T > 0) {
+    emb_bucket_count<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt);
+    tp_status s = after_launch("embedding_bwd count");
+    if (s != TP_OK) return s;
+  }
+  emb_scan<<<1, 1024, 0, st>>>(cnt, static_cast<int64_t>(nb) * nblk);
+  tp_status s = after_launch("embedding_bwd scan");
+  if (s != TP_OK) return s;
+  if (T > 0) {
+    emb_bucket_scatter<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt, sorted);
+    s = after_launch("embedding_bwd scatter");
+    if (s != TP_OK) return s;
+  }
+  dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((h + kEmbCols - 1) / kEmbCols));
   if (dt == TP_BF16)
-    embed_bwd_kernel<__nv_bfloat16><<<grid, kEmbThreads, smem, st>>>(
-        ids, T, static_cast<const __nv_bfloat16*>(dY), h, vocab, Vs, Vp, dE);
+    emb_bucket_accum<__nv_bfloat16><<<grid, kEmbThreads, smem, st>>>(
+        sorted, cnt, nb, nblk, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
   else
-    embed_bwd_kernel<float><<<grid, kEmbThreads, smem, st>>>(ids, T, static_cast<const float*>(dY), h,
-                                                            vocab, Vs, Vp, dE);
-  return after_launch("embedding_bwd");
+    emb_bucket_accum<float><<<grid, kEmbThreads, smem, st>>>(sorted, cnt, nb, nblk,
+                                                            static_cast<const float*>(dY), h, Vs, Vp, dE);
+  return after_launch("embedding_bwd accumulate");
 }
 
 tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
@@ -272,12 +548,49 @@ tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_
   unsigned* status = nullptr;
   tp_status s = device_status_word(&status);
   if (s != TP_OK) return s;
-  if (dt == TP_BF16)
-    vocab_ce_kernel<__nv_bfloat16, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(
-        L, G, p, Vs, vocab, labels, scale, loss, lse, status);
-  else
-    vocab_ce_kernel<float, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(L, G, p, Vs, vocab, labels,
+  const int64_t row_bytes = static_cast<int64_t>(p) * Vs * static_cast<int64_t>(dsize(dt));
+  const unsigned grid = static_cast<unsigned>(T);
+  static bool attr[4] = {false, false, false, false};
+  auto set_attr = [&](const void* fn, int k) -> tp_status {
+    if (attr[k]) return TP_OK;
+    tp_status r = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kCeSmemMax),
+                              "cudaFuncSetAttribute(vocab_cross_entropy)");
+    if (r == TP_OK) attr[k] = true;
+    return r;
+  };
+  const int smem = static_cast<int>(row_bytes);
+  if (row_bytes <= kCeSmemSmall) {
+    if (dt == TP_BF16) {
+      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<__nv_bfloat16, 256>), 0);
+      if (s != TP_OK) return s;
+      vocab_ce_smem_kernel<__nv_bfloat16, 256><<<grid, 256, smem, st>>>(L, G, p, Vs, vocab, labels,
                                                                          scale, loss, lse, status);
+    } else {
+      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<float, 256>), 1);
+      if (s != TP_OK) return s;
+      vocab_ce_smem_kernel<float, 256><<<grid, 256, smem, st>>>(L, G, p, Vs, vocab, labels, scale,
+                                                                 loss, lse, status);
+    }
+  } else if (row_bytes <= kCeSmemMax) {
+    if (dt == TP_BF16) {
+      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<__nv_bfloat16, 1024>), 2);
+      if (s != TP_OK) return s;
+      vocab_ce_smem_kernel<__nv_bfloat16, 1024><<<grid, 1024, smem, st>>>(
+          L, G, p, Vs, vocab, labels, scale, loss, lse, status);
+    } else {
+      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<float, 1024>), 3);
+      if (s != TP_OK) return s;
+      vocab_ce_smem_kernel<float, 1024><<<grid, 1024, smem, st>>>(L, G, p, Vs, vocab, labels, scale,
+                                                                   loss, lse, status);
+    }
+  } else if (dt == TP_BF16) {
+    vocab_ce_kernel<__nv_bfloat16, 256><<<grid, 256, 0, st>>>(L, G, p, Vs, vocab, labels, scale,
+                                                              loss, lse, status);
+  } else {
+    vocab_ce_kernel<float, 256><<<grid, 256, 0, st>>>(L, G, p, Vs, vocab, labels, scale, loss,
+                                                      lse, status);
+  }
   return after_launch("vocab_cross_entropy");
 }
 

@@ -276,3 +276,22 @@ def test_bf16_mlp_end_to_end_small_fused(act, bias):
     gr = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
     assert_close(Y, ref["Y"], TOL_BF16, "Y")
     assert_close(dX, gr["dX"], TOL_BF16, "dX")
+
+
+def test_overlapped_reduce_matches_sequential_bit_for_bit():
+    """Token blocks reduced on a side stream under the next block's GEMM give
+    exactly the sequential partials result (same kernels, same sums)."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 1000, 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, "swiglu", torch.bfloat16, seed=8)
+    outs = []
+    for chunks in (0, 3):
+        m = TPMLP(h, f, p, "swiglu", "bf16", overlap_chunks=chunks)
+        m.load_weights(dev(inp.W1), dev(inp.W2))
+        Y = m.forward(dev(inp.X)).clone()
+        dX = m.backward(dev(inp.dY)).clone()
+        torch.cuda.synchronize()
+        outs.append((Y, dX, torch.cat(m.dW1, 0).clone()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
+    assert torch.equal(outs[0][2], outs[1][2])

@@ -48,14 +48,19 @@ def test_embedding_fwd_bwd(p, dtype):
     assert _tp().device_status() == "TP_OK"
 
 
-@pytest.mark.parametrize("p,V", [(1, 1000), (4, 1001), (8, 32000)])
-def test_vocab_parallel_cross_entropy(p, V):
+@pytest.mark.parametrize("p,V,dtype", [(1, 1000, "bf16"), (4, 1001, "bf16"), (8, 32000, "bf16"),
+                                       (4, 50000, "bf16"), (8, 128000, "bf16"), (3, 997, "f32"),
+                                       (8, 32000, "f32")])
+def test_vocab_parallel_cross_entropy(p, V, dtype):
+    """Rows up to 64 KB and up to 200 KB (the shared-memory kernels) and wider
+    (the streaming kernel), padded and unpadded vocabularies, bf16 and fp32."""
     tp = _tp()
-    T, h = 300, 64
-    plan = tp.Plan(h, 0, 0, p, "bf16", "none")
+    T, h = (300, 64) if V <= 50000 else (40, 64)
+    plan = tp.Plan(h if h % p == 0 else 3 * h, 0, 0, p, dtype, "none")
     Vp = plan.set_vocab(V)
     g = torch.Generator().manual_seed(V)
-    z = (torch.randn(T, Vp, generator=g) * 3).to(torch.bfloat16)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    z = (torch.randn(T, Vp, generator=g) * 3).to(torch.bfloat16 if dtype == "bf16" else torch.float32)
     labels = torch.randint(0, V, (T,), generator=g, dtype=torch.int32)
     labels[0] = V - 1
     labels[5] = -1                    # ignored token
@@ -75,10 +80,47 @@ def test_vocab_parallel_cross_entropy(p, V):
     gg = np.concatenate([host(x) for x in G], axis=1)
     assert np.all(gg[5] == 0) and np.all(gg[:, V:] == 0)
     # oracle gradient of the mean over the kept tokens, rescaled to 1/T
-    assert_close(gg[keep] * T, rg * keep.sum(), TOL_BF16, "dlogits")
+    assert_close(gg[keep] * T, rg * keep.sum(), tol, "dlogits")
     # in place (dlogits aliasing the logits)
     plan.vocab_cross_entropy(T, L, labels.cuda(), 1.0 / T, loss, None, L)
-    assert_close(np.concatenate([host(x) for x in L], axis=1)[keep] * T, rg * keep.sum(), TOL_BF16, "in place")
+    assert_close(np.concatenate([host(x) for x in L], axis=1)[keep] * T, rg * keep.sum(), tol, "in place")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_embedding_bwd_many_blocks_heavy_id_and_ignored_ids(dtype):
+    """Tokens spanning several 1024-token blocks, one id repeated 2000 times (a
+    token list longer than one chunk), ids outside [0, vocab) ignored, a hidden
+    size with a ragged 512-column tile; integer-valued dY makes every sum exact,
+    so the result is bit for bit, and two calls agree bit for bit."""
+    tp = _tp()
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    T, V, h, p = 5000, 3000, 1032, 4
+    plan = tp.Plan(h, 0, 0, p, dtype, "none")
+    Vp = plan.set_vocab(V)
+    g = torch.Generator().manual_seed(5)
+    ids = torch.randint(0, V, (T,), generator=g, dtype=torch.int32)
+    heavy = torch.randperm(T, generator=g)[:2000]
+    ids[heavy] = V - 1
+    ids[17] = -1
+    ids[4000] = -5
+    dY = torch.randint(-1, 2, (T, h), generator=g).to(tdt)
+    dE = [torch.full((Vp // p, h), 7.0, dtype=tdt, device="cuda") for _ in range(p)]
+    idd = ids.cuda()
+    plan.embedding_bwd(T, idd, dev(dY), dE)
+    keep = (ids >= 0).numpy()
+    ref = O.embedding_bwd(ids.numpy()[keep], O.f64(dY)[keep], Vp)
+    assert np.abs(ref).max() <= 256      # every sum is an integer that bf16 holds exactly
+    assert_bitexact(torch.cat(dE, 0), ref, "embedding grad")
+    dY = torch.randn(T, h, generator=g).to(tdt)
+    first = [torch.empty_like(x) for x in dE]
+    plan.embedding_bwd(T, idd, dev(dY), first)
+    plan.embedding_bwd(T, idd, dev(dY), dE)
+    for a, b in zip(first, dE):
+        assert torch.equal(a, b)
+    ref = O.embedding_bwd(ids.numpy()[keep], O.f64(dY)[keep], Vp)
+    used = np.unique(ids.numpy()[keep])
+    assert_close(host(torch.cat(dE, 0))[used], ref[used], TOL_BF16 if dtype == "bf16" else TOL_F32, "dE")
+    assert tp.device_status() == "TP_OK"
 
 
 def test_output_head_logits_loss_and_gradients():
