@@ -4,10 +4,11 @@
 //
 // One CTA computes two adjacent 128-query tiles (A = 2i, B = 2i + 1) of one
 // (shard, batch, head); both read every K/V block once from shared memory:
-//   warp 0      TMA producer: both Q tiles, then each 128-key block's K and V
-//               (single buffers released separately, so K_{j+1} loads while
-//               block j's softmax and P.V run) from a 3-D tensor map over the
-//               sequence-major [seq, batch, 3*heads_local*d] QKV of the shard
+//   warp 0      TMA producer: both Q tiles, then K_0, V_0, K_1, V_1, ... into a
+//               ring of three K/V buffers (item n waits only for item n - 3 to
+//               be released, so V_j lands while block j - 1 is still in flight)
+//               from a 3-D tensor map over the sequence-major
+//               [seq, batch, 3*heads_local*d] QKV of the shard
 //   warp 1      TMEM allocator + MMA issuer, ping-pong order: S_A(0), S_B(0),
 //               then per block PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one
 //               tile's MMAs run while the other tile's softmax works
@@ -15,6 +16,7 @@
 //               row r; two passes over its row of S in TMEM (row max, then
 //               exp2 and the row sum), P rounded to bf16 and written to shared
 //               memory in the 128-byte-swizzled K-major layout of the PV MMA.
+//               Only the diagonal block (and a ragged last block) is masked.
 // O accumulates in TMEM across key blocks. P is taken relative to a reference
 // max m that is raised (and O, l rescaled in place) only when a row's max
 // exceeds it by more than 2^8; P <= 2^8 stays exact in fp32/bf16 range and the
@@ -58,11 +60,19 @@ struct AttnSmem {
   static constexpr int Q_BYTES = BQ * D * 2;
   static constexpr int KV_BYTES = BKV * D * 2;
   static constexpr int P_BYTES = BQ * BKV * 2;
-  static constexpr int TOTAL = 1024 + 2 * Q_BYTES + 2 * KV_BYTES + 2 * P_BYTES + 256;
+  static constexpr int KV_SLOTS = 3;
+  static constexpr int TOTAL = 1024 + 2 * Q_BYTES + KV_SLOTS * KV_BYTES + 2 * P_BYTES + 256;
 };
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 2^x by the hardware approximation (inputs here are <= 2^3; denormal results flush to 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int D>
@@ -72,20 +82,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   uint8_t* sQ = smem;                     // [2] tiles
-  uint8_t* sK = sQ + 2 * SM::Q_BYTES;
-  uint8_t* sV = sK + SM::KV_BYTES;
-  uint8_t* sP = sV + SM::KV_BYTES;        // [2] tiles
+  uint8_t* sKV = sQ + 2 * SM::Q_BYTES;    // [KV_SLOTS] K or V blocks
+  uint8_t* sP = sKV + SM::KV_SLOTS * SM::KV_BYTES;  // [2] tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SM::P_BYTES);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 2;
-  uint64_t* v_full = bars + 3;
-  uint64_t* v_empty = bars + 4;
-  uint64_t* s_full = bars + 5;   // [2]
-  uint64_t* p_full = bars + 7;   // [2]
-  uint64_t* o_done = bars + 9;   // [2]
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* kv_full = bars + 1;   // [KV_SLOTS]
+  uint64_t* kv_empty = bars + 4;  // [KV_SLOTS]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* o_done = bars + 11;   // [2]
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -112,10 +119,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(k_full, 1);
-    mbar_init(k_empty, 1);
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
+    for (int k = 0; k < SM::KV_SLOTS; ++k) {
+      mbar_init(&kv_full[k], 1);
+      mbar_init(&kv_empty[k], 1);
+    }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 4);
@@ -145,38 +152,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int c = 0; c < D / 64; ++c)
         tma_load_3d(sQ + t * SM::Q_BYTES + c * CHUNK_BYTES, tm, q_full, hh * D + c * 64, b, q0t[t]);
     }
+    // Ring items: 2j = K_j, 2j + 1 = V_j, in slot n % KV_SLOTS.
+    const int n_items = 2 * nb;
     int issued = 0;
-    for (int j = 0; j < nb; ++j) {
-      const uint32_t ph = static_cast<uint32_t>(j) & 1u;
-      const int k0 = j * BKV;
-      if (!mbar_wait(k_empty, ph ^ 1u, abort_flag, p.status)) break;
-      mbar_arrive_expect_tx(k_full, SM::KV_BYTES);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sK + c * CHUNK_BYTES, tm, k_full, hl_d + hh * D + c * 64, b, k0);
-      if (!mbar_wait(v_empty, ph ^ 1u, abort_flag, p.status)) {
-        issued = -(j + 1);  // K of block j issued, V not
+    for (int n = 0; n < n_items; ++n) {
+      const int slot = n % SM::KV_SLOTS, use = n / SM::KV_SLOTS;
+      if (use > 0 && !mbar_wait(&kv_empty[slot], static_cast<uint32_t>(use - 1) & 1u, abort_flag,
+                                p.status))
         break;
-      }
-      mbar_arrive_expect_tx(v_full, SM::KV_BYTES);
+      mbar_arrive_expect_tx(&kv_full[slot], SM::KV_BYTES);
+      const int col0 = ((n & 1) ? 2 * hl_d : hl_d) + hh * D;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sV + c * CHUNK_BYTES, tm, v_full, 2 * hl_d + hh * D + c * 64, b, k0);
-      issued = j + 1;
+        tma_load_3d(sKV + slot * SM::KV_BYTES + c * CHUNK_BYTES, tm, &kv_full[slot], col0 + c * 64, b,
+                    (n >> 1) * BKV);
+      issued = n + 1;
     }
     // Drain: every copy issued has landed before the CTA exits.
     mbar_wait(q_full, 0, abort_flag, p.status);
-    const int nk = issued >= 0 ? issued : -issued;
-    const int nv = issued >= 0 ? issued : -issued - 1;
-    if (nk > 0) mbar_wait(k_full, static_cast<uint32_t>(nk - 1) & 1u, abort_flag, p.status);
-    if (nv > 0) mbar_wait(v_full, static_cast<uint32_t>(nv - 1) & 1u, abort_flag, p.status);
+    for (int k = 0; k < SM::KV_SLOTS; ++k) {
+      const int uses = issued > k ? (issued - 1 - k) / SM::KV_SLOTS + 1 : 0;
+      if (uses > 0) mbar_wait(&kv_full[k], static_cast<uint32_t>(uses - 1) & 1u, abort_flag, p.status);
+    }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
     const uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
-    const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
-    auto issue_s = [&](int t) {
+    auto slot_of = [](int n) { return n % SM::KV_SLOTS; };
+    auto full_parity = [](int n) { return static_cast<uint32_t>(n / SM::KV_SLOTS) & 1u; };
+    auto issue_s = [&](int t, int j) {
       const uint32_t q_base = smem_u32(sQ + t * SM::Q_BYTES);
+      const uint32_t k_base = smem_u32(sKV + slot_of(2 * j) * SM::KV_BYTES);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk / 4) * CHUNK_BYTES + (kk % 4) * 32;
@@ -185,8 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       tc_commit(&s_full[t]);
     };
-    auto issue_pv = [&](int t, bool first) {
+    auto issue_pv = [&](int t, int j) {
+      const bool first = j == 0;
       const uint32_t p_base = smem_u32(sP + t * SM::P_BYTES);
+      const uint32_t v_base = smem_u32(sKV + slot_of(2 * j + 1) * SM::KV_BYTES);
 #pragma unroll
       for (int kk = 0; kk < BKV / 16; ++kk) {
         const uint64_t adesc = smem_desc_sw128(p_base + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
@@ -195,15 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       tc_commit(&o_done[t]);
     };
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && mbar_wait(k_full, 0, abort_flag, p.status);
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.status) &&
+              mbar_wait(&kv_full[slot_of(0)], full_parity(0), abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       for (int t = 0; t < 2; ++t)
-        if (nbt[t] > 0) issue_s(t);
-      tc_commit(k_empty);  // K_0 free once both S MMAs finish
+        if (nbt[t] > 0) issue_s(t, 0);
+      tc_commit(&kv_empty[slot_of(0)]);  // K_0 free once both S MMAs finish
     }
     for (int j = 0; ok && j < nb; ++j) {
-      if (!mbar_wait(v_full, static_cast<uint32_t>(j) & 1u, abort_flag, p.status)) break;
+      if (!mbar_wait(&kv_full[slot_of(2 * j + 1)], full_parity(2 * j + 1), abort_flag, p.status)) break;
+      tc_fence_after();
       bool have_k_next = false;
       for (int t = 0; t < 2 && ok; ++t) {
         if (j >= nbt[t]) continue;
@@ -212,22 +222,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           break;
         }
         tc_fence_after();
-        issue_pv(t, j == 0);
+        issue_pv(t, j);
         if (j + 1 < nbt[t]) {
           if (!have_k_next) {
-            if (!mbar_wait(k_full, static_cast<uint32_t>(j + 1) & 1u, abort_flag, p.status)) {
+            if (!mbar_wait(&kv_full[slot_of(2 * j + 2)], full_parity(2 * j + 2), abort_flag,
+                           p.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
             have_k_next = true;
           }
-          issue_s(t);
+          issue_s(t, j + 1);
         }
       }
       if (!ok) break;
-      tc_commit(v_empty);                 // V_j free once both P.V MMAs finish
-      if (have_k_next) tc_commit(k_empty);  // K_{j+1} free once both S MMAs finish
+      tc_commit(&kv_empty[slot_of(2 * j + 1)]);                 // V_j free after both P.V MMAs
+      if (have_k_next) tc_commit(&kv_empty[slot_of(2 * j + 2)]);  // K_{j+1} after both S MMAs
     }
     tc_commit(drain);
     mbar_wait(drain, 0, abort_flag, p.status);
@@ -253,16 +264,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       tc_fence_after();
       const int k0 = j * BKV;
       const int kmax = min(q, p.seq - 1) - k0;  // last visible column of this block
+      // No column of this block is masked for any row of the warp (every block
+      // but the diagonal one and a ragged last one): skip the per-column tests.
+      const bool full = k0 + BKV - 1 <= min(q0t[t] + lg * 32, p.seq - 1);
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < BKV / 32; ++c) {
-        float sv[32];
+      for (int c = 0; c < BKV / 32; c += 2) {
+        float sv[32], sw[32];
         tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tS + c * 32 + 32, sw);
         tc_wait_ld();
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i <= kmax) mx = fmaxf(mx, sv[i] * p.scale_log2);
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(sv[i], sw[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (c * 32 + i <= kmax) mx = fmaxf(mx, sv[i]);
+            if (c * 32 + 32 + i <= kmax) mx = fmaxf(mx, sw[i]);
+          }
+        }
       }
+      mx *= p.scale_log2;  // the scale is positive: max of the scaled scores
       if (j > 0) {
         // P.V of the previous block done: the P buffer is free and O is stable.
         if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], static_cast<uint32_t>(j - 1) & 1u,
@@ -293,27 +316,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         m = m_new;
       }
       float rs = 0.f;
+      const float sc = p.scale_log2;
 #pragma unroll 1
-      for (int c = 0; c < BKV / 32; ++c) {
-        float sv[32];
-        tmem_ld32(tS + c * 32, sv);
+      for (int c = 0; c < BKV / 32; c += 2) {
+        float sv[2][32];
+        tmem_ld32(tS + c * 32, sv[0]);
+        tmem_ld32(tS + c * 32 + 32, sv[1]);
         tc_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float a = (c * 32 + i <= kmax) ? exp2f(sv[i] * p.scale_log2 - m) : 0.f;
-          const float bb = (c * 32 + i + 1 <= kmax) ? exp2f(sv[i + 1] * p.scale_log2 - m) : 0.f;
-          const uint32_t u = pack_bf16x2(a, bb);
-          pk[i / 2] = u;
-          const float2 f = unpack_bf16x2(u);  // the row sum uses the rounded P of the PV MMA
-          rs += f.x + f.y;
-        }
-        uint8_t* rowp = sPt + (c / 2) * CHUNK_BYTES + r * 128;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int cc = c + h2;
+          uint32_t pk[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int qv = (c % 2) * 4 + v;
-          *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) =
-              make_uint4(pk[v * 4 + 0], pk[v * 4 + 1], pk[v * 4 + 2], pk[v * 4 + 3]);
+          for (int i = 0; i < 32; i += 2) {
+            float a = ex2(fmaf(sv[h2][i], sc, -m));
+            float bb = ex2(fmaf(sv[h2][i + 1], sc, -m));
+            if (!full) {
+              a = (cc * 32 + i <= kmax) ? a : 0.f;
+              bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
+            }
+            const uint32_t u = pack_bf16x2(a, bb);
+            pk[i / 2] = u;
+            const float2 f = unpack_bf16x2(u);  // the row sum uses the rounded P of the PV MMA
+            rs += f.x + f.y;
+          }
+          uint8_t* rowp = sPt + (cc / 2) * CHUNK_BYTES + r * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int qv = (cc % 2) * 4 + v;
+            *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) =
+                make_uint4(pk[v * 4 + 0], pk[v * 4 + 1], pk[v * 4 + 2], pk[v * 4 + 3]);
+          }
         }
       }
       l += rs;
