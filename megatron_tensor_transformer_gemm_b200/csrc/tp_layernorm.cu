@@ -342,51 +342,121 @@ namespace {
 
 using tpi::MutPtrArray;
 
-template <typename T, int THREADS, int VPT, bool RMS>
+// Rows staged in shared memory: CTA b takes rows b, b + G, b + 2G, ... and
+// keeps STAGES of them in flight; a row's p shard slices arrive by bulk copy
+// (one per shard, completing on the stage's mbarrier) while the CTA works on
+// the rows before it. Thread tid owns the row's 16-byte vectors
+// tid + i * THREADS (vector c lies in shard c / vps), the same for every row.
+// thread 0: start the copies of row r of `a` (and, if given, of `b`: placed
+// after a's row) into `dst`, one bulk copy per shard slice, completing on `bar`.
+__device__ __forceinline__ void issue_row(const PtrArray& a, const PtrArray* b, int p, int64_t r,
+                                          uint32_t shard_bytes, uint8_t* dst, uint64_t* bar) {
+  const int nbuf = b ? 2 : 1;
+  tpd::mbar_arrive_expect_tx(bar, shard_bytes * static_cast<uint32_t>(p * nbuf));
+  for (int s = 0; s < p; ++s)
+    tpd::bulk_load(dst + static_cast<size_t>(s) * shard_bytes,
+                   static_cast<const uint8_t*>(a.p[s]) + r * shard_bytes, shard_bytes, bar);
+  if (b)
+    for (int s = 0; s < p; ++s)
+      tpd::bulk_load(dst + static_cast<size_t>(p + s) * shard_bytes,
+                     static_cast<const uint8_t*>(b->p[s]) + r * shard_bytes, shard_bytes, bar);
+}
+
+template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
 __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
-    const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int vps,
-    int64_t hs, int64_t h, float* mean_out, float* rstd_out) {
+    const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int p, int vps,
+    int64_t hs, int64_t h, int64_t rows, float* mean_out, float* rstd_out, unsigned* status) {
   constexpr int V = LnVec<T>::N;
+  extern __shared__ __align__(128) uint8_t sbuf[];
+  __shared__ uint64_t bar[STAGES];
+  __shared__ int abort_flag;
   __shared__ float red[THREADS / 32];
-  const int64_t r = blockIdx.x;
+  const uint32_t shard_bytes = static_cast<uint32_t>(hs * sizeof(T));
+  const size_t stage_bytes = static_cast<size_t>(h) * sizeof(T);
   const int vpr = static_cast<int>(h / V);
-  float v[VPT][V];
-  float s1 = 0.f, s2 = 0.f;
+  const int64_t G0 = blockIdx.x, GS = gridDim.x;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < STAGES; ++st) tpd::mbar_init(&bar[st], 1);
+    tpd::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < STAGES && G0 + k * GS < rows; ++k)
+      issue_row(X, nullptr, p, G0 + k * GS, shard_bytes, sbuf + k * stage_bytes, &bar[k]);
+  // gamma (and beta) of this thread's columns, packed, for every row
+  uint4 gp[VPT], bp[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = threadIdx.x + i * THREADS;
+    gp[i] = bp[i] = make_uint4(0, 0, 0, 0);
     if (c < vpr) {
       const int sh = c / vps, lc = c - sh * vps;
-      LnVec<T>::load(static_cast<const T*>(X.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, v[i]);
+      gp[i] = *reinterpret_cast<const uint4*>(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V);
+      if (!RMS) bp[i] = *reinterpret_cast<const uint4*>(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V);
+    }
+  }
+  int64_t k = 0;
+  for (;; ++k) {
+    const int64_t r = G0 + k * GS;
+    if (r >= rows) break;
+    const int st = static_cast<int>(k % STAGES);
+    const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
+    if (!__syncthreads_and(ok)) break;
+    const uint4* row = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes);
+    float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-      for (int k = 0; k < V; ++k) {
-        s1 += v[i][k];
-        s2 += v[i][k] * v[i][k];
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * THREADS;
+      if (c < vpr) {
+        float x[V];
+        LnVec<T>::unpack(row[c], x);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          s1 += x[e];
+          s2 += x[e] * x[e];
+        }
       }
     }
-  }
-  const float S2 = block_sum<THREADS>(s2, red);
-  float mean = 0.f;
-  if (!RMS) mean = block_sum<THREADS>(s1, red) / static_cast<float>(h);
-  const float var = RMS ? S2 / static_cast<float>(h) : fmaxf(S2 / static_cast<float>(h) - mean * mean, 0.f);
-  const float rstd = rsqrtf(var + kEps);
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
-      const int sh = c / vps, lc = c - sh * vps;
-      float g[V], b[V], o[V];
-      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
-      if (!RMS) LnVec<T>::load(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V, b);
-#pragma unroll
-      for (int k = 0; k < V; ++k) o[k] = (v[i][k] - mean) * rstd * g[k] + (RMS ? 0.f : b[k]);
-      LnVec<T>::store(static_cast<T*>(Y.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+    float2 tot;
+    if (RMS) {
+      tot = make_float2(0.f, block_sum<THREADS>(s2, red));
+    } else {
+      tot = make_float2(block_sum<THREADS>(s1, red), 0.f);
+      tot.y = block_sum<THREADS>(s2, red);
     }
+    const float mean = RMS ? 0.f : tot.x / static_cast<float>(h);
+    const float var = RMS ? tot.y / static_cast<float>(h)
+                          : fmaxf(tot.y / static_cast<float>(h) - mean * mean, 0.f);
+    const float rstd = rsqrtf(var + kEps);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * THREADS;
+      if (c < vpr) {
+        const int sh = c / vps, lc = c - sh * vps;
+        float x[V], g[V], bb[V], o[V];
+        LnVec<T>::unpack(row[c], x);
+        LnVec<T>::unpack(gp[i], g);
+        if (!RMS) LnVec<T>::unpack(bp[i], bb);
+#pragma unroll
+        for (int e = 0; e < V; ++e) o[e] = (x[e] - mean) * rstd * g[e] + (RMS ? 0.f : bb[e]);
+        LnVec<T>::store(static_cast<T*>(Y.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+      }
+    }
+    if (threadIdx.x == 0) {
+      if (mean_out && !RMS) mean_out[r] = mean;
+      if (rstd_out) rstd_out[r] = rstd;
+    }
+    __syncthreads();  // every thread is done with this stage
+    if (threadIdx.x == 0 && G0 + (k + STAGES) * GS < rows)
+      issue_row(X, nullptr, p, G0 + (k + STAGES) * GS, shard_bytes, sbuf + st * stage_bytes, &bar[st]);
   }
-  if (threadIdx.x == 0) {
-    if (mean_out && !RMS) mean_out[r] = mean;
-    if (rstd_out) rstd_out[r] = rstd;
+  if (threadIdx.x == 0 && abort_flag) {  // let copies still in flight land (bounded)
+    for (int64_t kk = k; kk < k + STAGES && G0 + kk * GS < rows; ++kk) {
+      int again = 0;
+      tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+    }
   }
 }
 
@@ -412,49 +482,78 @@ __device__ __forceinline__ float2 block_sum2(float2 v, float2* red) {
   return s;
 }
 
-// Backward of a hidden-sharded norm in one pass over x and dy. CTA b takes
-// rows b, b + gridDim.x, ... in order; thread tid owns the same 16-byte column
-// vectors tid + i * THREADS of every row, so besides dx it keeps running
+// Backward of a hidden-sharded norm in one pass over x and dy, staged like
+// the forward (a stage holds a row of x and the same row of dy). Thread tid
+// owns the same column vectors of every row, so besides dx it keeps running
 // column partials dgamma = sum dy * xhat and dbeta = sum dy in registers and
 // writes them once: part[b][0][col], part[b][1][col]. A second kernel sums the
 // partials over b in order, so the parameter gradients are deterministic.
-// The row is read from HBM once; the dx pass reads it again from L1 / L2.
-template <typename T, int THREADS, int VPT, bool RMS>
-__global__ void __launch_bounds__(THREADS, VPT >= 8 ? 1 : 512 / THREADS) norm_hsh_bwd_fused_kernel(
+template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
+__global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
-    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int vps,
+    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int p, int vps,
     int64_t hs, int64_t h, int64_t rows, const float* mean_in, const float* rstd_in,
-    float* part) {
+    float* part, unsigned* status) {
   constexpr int V = LnVec<T>::N;
+  extern __shared__ __align__(128) uint8_t sbuf[];
+  __shared__ uint64_t bar[STAGES];
+  __shared__ int abort_flag;
   __shared__ float2 red[THREADS / 32];
+  const uint32_t shard_bytes = static_cast<uint32_t>(hs * sizeof(T));
+  const size_t row_bytes = static_cast<size_t>(h) * sizeof(T);
+  const size_t stage_bytes = 2 * row_bytes;
   const int vpr = static_cast<int>(h / V);
   const float inv_h = 1.f / static_cast<float>(h);
+  const int64_t G0 = blockIdx.x, GS = gridDim.x;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < STAGES; ++st) tpd::mbar_init(&bar[st], 1);
+    tpd::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < STAGES && G0 + k * GS < rows; ++k)
+      issue_row(X, &DY, p, G0 + k * GS, shard_bytes, sbuf + k * stage_bytes, &bar[k]);
+  uint4 gp[VPT];
   float pg[VPT][V], pb[VPT][V];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i)
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    gp[i] = make_uint4(0, 0, 0, 0);
+    if (c < vpr) {
+      const int sh = c / vps, lc = c - sh * vps;
+      gp[i] = *reinterpret_cast<const uint4*>(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V);
+    }
 #pragma unroll
-    for (int k = 0; k < V; ++k) pg[i][k] = pb[i][k] = 0.f;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    for (int e = 0; e < V; ++e) pg[i][e] = pb[i][e] = 0.f;
+  }
+  int64_t k = 0;
+  for (;; ++k) {
+    const int64_t r = G0 + k * GS;
+    if (r >= rows) break;
+    const int st = static_cast<int>(k % STAGES);
     const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+    const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
+    if (!__syncthreads_and(ok)) break;
+    const uint4* xrow = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes);
+    const uint4* drow = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes + row_bytes);
     float2 acc = make_float2(0.f, 0.f);  // (sum g dy, sum g dy xhat) of this thread's columns
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * THREADS;
       if (c < vpr) {
-        const int sh = c / vps, lc = c - sh * vps;
-        const int64_t off = r * hs + static_cast<int64_t>(lc) * V;
         float x[V], d[V], g[V];
-        LnVec<T>::load(static_cast<const T*>(X.p[sh]) + off, x);
-        LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + off, d);
-        LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+        LnVec<T>::unpack(xrow[c], x);
+        LnVec<T>::unpack(drow[c], d);
+        LnVec<T>::unpack(gp[i], g);
 #pragma unroll
-        for (int k = 0; k < V; ++k) {
-          const float xh = (x[k] - mean) * rstd;
-          const float gy = d[k] * g[k];
+        for (int e = 0; e < V; ++e) {
+          const float xh = (x[e] - mean) * rstd;
+          const float gy = d[e] * g[e];
           acc.x += gy;
           acc.y += gy * xh;
-          pg[i][k] += d[k] * xh;
-          pb[i][k] += d[k];
+          pg[i][e] += d[e] * xh;
+          pb[i][e] += d[e];
         }
       }
     }
@@ -465,15 +564,23 @@ __global__ void __launch_bounds__(THREADS, VPT >= 8 ? 1 : 512 / THREADS) norm_hs
       const int c = threadIdx.x + i * THREADS;
       if (c < vpr) {
         const int sh = c / vps, lc = c - sh * vps;
-        const int64_t off = r * hs + static_cast<int64_t>(lc) * V;
         float x[V], d[V], g[V], o[V];
-        LnVec<T>::load(static_cast<const T*>(X.p[sh]) + off, x);  // again: an L1 / L2 hit
-        LnVec<T>::load(static_cast<const T*>(DY.p[sh]) + off, d);
-        LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+        LnVec<T>::unpack(xrow[c], x);
+        LnVec<T>::unpack(drow[c], d);
+        LnVec<T>::unpack(gp[i], g);
 #pragma unroll
-        for (int k = 0; k < V; ++k) o[k] = rstd * (d[k] * g[k] - m1 - (x[k] - mean) * rstd * m2);
-        LnVec<T>::store(static_cast<T*>(DX.p[sh]) + off, o);
+        for (int e = 0; e < V; ++e) o[e] = rstd * (d[e] * g[e] - m1 - (x[e] - mean) * rstd * m2);
+        LnVec<T>::store(static_cast<T*>(DX.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
       }
+    }
+    __syncthreads();  // every thread is done with this stage
+    if (threadIdx.x == 0 && G0 + (k + STAGES) * GS < rows)
+      issue_row(X, &DY, p, G0 + (k + STAGES) * GS, shard_bytes, sbuf + st * stage_bytes, &bar[st]);
+  }
+  if (threadIdx.x == 0 && abort_flag) {  // let copies still in flight land (bounded)
+    for (int64_t kk = k; kk < k + STAGES && G0 + kk * GS < rows; ++kk) {
+      int again = 0;
+      tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
     }
   }
   float* pgo = part + (static_cast<int64_t>(blockIdx.x) * 2 + 0) * h;
@@ -483,11 +590,11 @@ __global__ void __launch_bounds__(THREADS, VPT >= 8 ? 1 : 512 / THREADS) norm_hs
     const int c = threadIdx.x + i * THREADS;
     if (c < vpr) {
 #pragma unroll
-      for (int k = 0; k < V; k += 4) {
-        *reinterpret_cast<float4*>(pgo + static_cast<int64_t>(c) * V + k) =
-            make_float4(pg[i][k], pg[i][k + 1], pg[i][k + 2], pg[i][k + 3]);
-        *reinterpret_cast<float4*>(pbo + static_cast<int64_t>(c) * V + k) =
-            make_float4(pb[i][k], pb[i][k + 1], pb[i][k + 2], pb[i][k + 3]);
+      for (int e = 0; e < V; e += 4) {
+        *reinterpret_cast<float4*>(pgo + static_cast<int64_t>(c) * V + e) =
+            make_float4(pg[i][e], pg[i][e + 1], pg[i][e + 2], pg[i][e + 3]);
+        *reinterpret_cast<float4*>(pbo + static_cast<int64_t>(c) * V + e) =
+            make_float4(pb[i][e], pb[i][e + 1], pb[i][e + 2], pb[i][e + 3]);
       }
     }
   }
@@ -523,6 +630,9 @@ int vpt_for(int64_t vpr, int th) {
   return need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
 }
 
+constexpr int kNormFwdStages = 4;
+constexpr int kNormBwdStages = 3;
+
 #define TP_NH_DISPATCH(LAUNCH, T, R)                 \
   if (th == 64) LAUNCH(T, 64, 1, R);                 \
   else if (th == 128) LAUNCH(T, 128, 1, R);          \
@@ -531,6 +641,21 @@ int vpt_for(int64_t vpr, int th) {
   else if (vpt == 4) LAUNCH(T, 256, 4, R);           \
   else LAUNCH(T, 256, 8, R)
 
+// Persistent grid for a staged row kernel: as many CTAs as are resident at
+// once (at most one per row), with its dynamic shared memory opted in.
+template <typename K>
+tp_status pipe_grid(K kernel, int threads, int smem, int64_t rows, int64_t* grid) {
+  tp_status s = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                            "cudaFuncSetAttribute(norm)");
+  if (s != TP_OK) return s;
+  int per_sm = 0;
+  s = cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem),
+                  "cudaOccupancyMaxActiveBlocksPerMultiprocessor(norm)");
+  if (s != TP_OK) return s;
+  *grid = std::max<int64_t>(1, std::min<int64_t>(rows, static_cast<int64_t>(num_sms()) * std::max(per_sm, 1)));
+  return TP_OK;
+}
+
 tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G,
                                   const PtrArray& B, const MutPtrArray& Y, int p, int64_t rows,
                                   int64_t h, float* mean, float* rstd, tp_dtype dt,
@@ -538,12 +663,23 @@ tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = h / V, hs = h / p;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
+  if (rows == 0) return TP_OK;
   const int vps = static_cast<int>(hs / V);
   const int th = hsh_threads(vpr);
   const int vpt = vpt_for(vpr, th);
-#define TP_NH_FWD(T, TH, VP, R)                                                   \
-  norm_hsh_fwd_kernel<T, TH, VP, R><<<static_cast<unsigned>(rows), TH, 0, st>>>( \
-      X, G, B, Y, vps, hs, h, mean, rstd)
+  const int smem = static_cast<int>(kNormFwdStages * h * static_cast<int64_t>(dsize(dt)));
+  unsigned* status = nullptr;
+  tp_status s = device_status_word(&status);
+  if (s != TP_OK) return s;
+  int64_t grid = 1;
+#define TP_NH_FWD(T, TH, VP, R)                                                                    \
+  do {                                                                                             \
+    auto kern = norm_hsh_fwd_kernel<T, TH, VP, kNormFwdStages, R>;                                 \
+    s = pipe_grid(kern, TH, smem, rows, &grid);                                                    \
+    if (s != TP_OK) return s;                                                                      \
+    kern<<<static_cast<unsigned>(grid), TH, smem, st>>>(X, G, B, Y, p, vps, hs, h, rows, mean,     \
+                                                        rstd, status);                             \
+  } while (0)
   if (dt == TP_BF16) {
     if (rms) { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, true); }
     else { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, false); }
@@ -566,17 +702,34 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   const int vps = static_cast<int>(hs / V);
   const int th = hsh_threads(vpr);
   const int vpt = vpt_for(vpr, th);
-  // As many CTAs as the launch bounds fit at once, at most one per row.
-  const int per_sm = vpt >= 8 ? 1 : 512 / th;
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(rows, static_cast<int64_t>(num_sms()) * per_sm));
+  const int smem = static_cast<int>(kNormBwdStages * 2 * h * static_cast<int64_t>(dsize(dt)));
+  unsigned* status = nullptr;
+  tp_status s = device_status_word(&status);
+  if (s != TP_OK) return s;
+  // The grid (and so the partials' size) depends only on the kernel, not on
+  // the data: size it first, then the workspace.
+  int64_t grid = 1;
+#define TP_NH_GRID(T, TH, VP, R)                                                          \
+  s = pipe_grid(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R>, TH, smem,         \
+                std::max<int64_t>(rows, 1), &grid)
+  if (dt == TP_BF16) {
+    if (rms) { TP_NH_DISPATCH(TP_NH_GRID, __nv_bfloat16, true); }
+    else { TP_NH_DISPATCH(TP_NH_GRID, __nv_bfloat16, false); }
+  } else {
+    if (rms) { TP_NH_DISPATCH(TP_NH_GRID, float, true); }
+    else { TP_NH_DISPATCH(TP_NH_GRID, float, false); }
+  }
+#undef TP_NH_GRID
+  if (s != TP_OK) return s;
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(grid) * 2 * h * sizeof(float), &ws);
+  s = workspace(plan, static_cast<size_t>(grid) * 2 * h * sizeof(float), &ws);
   if (s != TP_OK) return s;
   float* part = static_cast<float*>(ws);
   if (rows > 0) {
-#define TP_NH_BWD(T, TH, VP, R)                                                       \
-  norm_hsh_bwd_fused_kernel<T, TH, VP, R><<<static_cast<unsigned>(grid), TH, 0, st>>>( \
-      X, G, DY, DX, vps, hs, h, rows, mean, rstd, part)
+#define TP_NH_BWD(T, TH, VP, R)                                                               \
+  norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R><<<static_cast<unsigned>(grid), TH,   \
+                                                            smem, st>>>(                       \
+      X, G, DY, DX, p, vps, hs, h, rows, mean, rstd, part, status)
     if (dt == TP_BF16) {
       if (rms) { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
       else { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, false); }
