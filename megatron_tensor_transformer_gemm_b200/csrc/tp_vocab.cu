@@ -58,8 +58,8 @@ __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ Ptr
 //            that order in fp32 and writes its 16 rows of dE (zeros if none).
 // No atomics touch the sums, so the result is deterministic.
 constexpr int kEmbRows = 16;    // vocab ids per bucket
-constexpr int kEmbCols = 512;   // columns per accumulating CTA (2 per thread)
-constexpr int kEmbThreads = 256;
+constexpr int kEmbCols = 512;   // columns per accumulating CTA (4 per thread)
+constexpr int kEmbThreads = 128;
 constexpr int kTokBlock = 1024; // tokens per count / scatter CTA
 constexpr int kEmbMaxBuckets = 12288;  // 48 KB of shared counters (padded vocab <= 196608)
 constexpr int kListChunk = 512;
@@ -82,29 +82,56 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_count(const int32_t* ids
     cnt[static_cast<int64_t>(i) * nblk + blockIdx.x] = hist[i];
 }
 
-// One CTA: a[0..n) <- exclusive prefix sums, a[n] <- the total.
+// One CTA: a[0..n) <- exclusive prefix sums, a[n] <- the total. Thread tid
+// owns the contiguous chunk [tid * C, (tid + 1) * C), C a multiple of 4, read
+// and written as 16-byte vectors (a is 16-byte aligned).
 __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
-  __shared__ int part[1024];
-  const int tid = threadIdx.x;
-  const int64_t chunk = (n + 1023) / 1024;
-  const int64_t lo = tid * chunk, hi = lo + chunk < n ? lo + chunk : n;
+  __shared__ int wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t C = ((n + 1023) / 1024 + 3) / 4 * 4;
+  const int64_t lo = tid * C < n ? tid * C : n;
+  const int64_t hi = lo + C < n ? lo + C : n;
+  const int64_t hv = lo + (hi - lo) / 4 * 4;  // [lo, hv) as int4
   int sum = 0;
-  for (int64_t i = lo; i < hi; ++i) sum += a[i];
-  part[tid] = sum;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {  // inclusive Hillis-Steele scan of the partial sums
-    const int v = tid >= o ? part[tid - o] : 0;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
+#pragma unroll 4
+  for (int64_t i = lo; i < hv; i += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(a + i);
+    sum += v.x + v.y + v.z + v.w;
   }
-  int run = part[tid] - sum;
-  for (int64_t i = lo; i < hi; ++i) {
+  for (int64_t i = hv; i < hi; ++i) sum += a[i];
+  // exclusive scan of the per-thread sums: within the warp, then over warps
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    wsum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = (warp > 0 ? wsum[warp - 1] : 0) + incl - sum;
+#pragma unroll 4
+  for (int64_t i = lo; i < hv; i += 4) {
+    int4 v = *reinterpret_cast<const int4*>(a + i);
+    const int4 o = make_int4(run, run + v.x, run + v.x + v.y, run + v.x + v.y + v.z);
+    run += v.x + v.y + v.z + v.w;
+    *reinterpret_cast<int4*>(a + i) = o;
+  }
+  for (int64_t i = hv; i < hi; ++i) {
     const int v = a[i];
     a[i] = run;
     run += v;
   }
-  if (tid == 1023) a[n] = part[1023];
+  if (tid == 1023) a[n] = wsum[31];
 }
 
 // sorted[k] = (token, id - bucket * kEmbRows) of the k-th entry of the sorted list.
@@ -137,23 +164,33 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* i
         make_int2(static_cast<int>(t), id - b * kEmbRows);
 }
 
+// Four consecutive columns of dY row t as floats.
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* dY, int64_t off) {
+  if constexpr (sizeof(T) == 2) {
+    const uint2 u = *reinterpret_cast<const uint2*>(dY + off);
+    const float2 a = tpd::unpack_bf16x2(u.x), b = tpd::unpack_bf16x2(u.y);
+    return make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    return *reinterpret_cast<const float4*>(dY + off);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kEmbThreads) emb_bucket_accum(
     const int2* sorted, const int* off, int nb, int nblk, const T* dY, int64_t h, int64_t Vs,
     int64_t Vp, const __grid_constant__ MutPtrArray dE) {
-  extern __shared__ float acc[];  // [kEmbRows][kEmbCols]; thread tid owns columns 2 tid, 2 tid + 1
+  extern __shared__ float4 acc[];  // [kEmbRows][kEmbCols / 4]; thread tid owns columns 4 tid .. 4 tid + 3
   __shared__ int ltok[kListChunk];
   __shared__ int lrow[kListChunk];
+  constexpr int CV = kEmbCols / 4;  // float4 per accumulator row
   const int b = blockIdx.x;
   const int64_t v0 = static_cast<int64_t>(b) * kEmbRows;
   const int tid = threadIdx.x;
-  const int64_t col = static_cast<int64_t>(blockIdx.y) * kEmbCols + 2 * tid;
+  const int64_t col = static_cast<int64_t>(blockIdx.y) * kEmbCols + 4 * tid;
   const bool col_ok = col < h;
-#pragma unroll 4
-  for (int r = 0; r < kEmbRows; ++r) {
-    acc[r * kEmbCols + 2 * tid] = 0.f;
-    acc[r * kEmbCols + 2 * tid + 1] = 0.f;
-  }
+#pragma unroll
+  for (int r = 0; r < kEmbRows; ++r) acc[r * CV + tid] = make_float4(0.f, 0.f, 0.f, 0.f);
   const int start = off[static_cast<int64_t>(b) * nblk];
   const int end = off[static_cast<int64_t>(b + 1) * nblk];  // off[nb * nblk] is the total
   for (int c0 = start; c0 < end; c0 += kListChunk) {
@@ -167,32 +204,26 @@ __global__ void __launch_bounds__(kEmbThreads) emb_bucket_accum(
     __syncthreads();
     if (!col_ok) continue;
     int k = 0;
-    for (; k + 8 <= n; k += 8) {  // eight independent row loads in flight, summed in list order
-      float2 f[8];
+    for (; k + 16 <= n; k += 16) {  // sixteen independent row loads in flight, summed in list order
+      float4 f[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t off_t = static_cast<int64_t>(ltok[k + u]) * h + col;
-        if constexpr (sizeof(T) == 2) {
-          f[u] = tpd::unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dY + off_t));
-        } else {
-          f[u] = *reinterpret_cast<const float2*>(dY + off_t);
-        }
-      }
+      for (int u = 0; u < 16; ++u) f[u] = load4(dY, static_cast<int64_t>(ltok[k + u]) * h + col);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float* a2 = acc + lrow[k + u] * kEmbCols + 2 * tid;
-        a2[0] += f[u].x;
-        a2[1] += f[u].y;
+      for (int u = 0; u < 16; ++u) {
+        float4& a4 = acc[lrow[k + u] * CV + tid];
+        a4.x += f[u].x;
+        a4.y += f[u].y;
+        a4.z += f[u].z;
+        a4.w += f[u].w;
       }
     }
     for (; k < n; ++k) {
-      const int64_t off_t = static_cast<int64_t>(ltok[k]) * h + col;
-      float2 f;
-      if constexpr (sizeof(T) == 2) f = tpd::unpack_bf16x2(*reinterpret_cast<const uint32_t*>(dY + off_t));
-      else f = *reinterpret_cast<const float2*>(dY + off_t);
-      float* a2 = acc + lrow[k] * kEmbCols + 2 * tid;
-      a2[0] += f.x;
-      a2[1] += f.y;
+      const float4 f = load4(dY, static_cast<int64_t>(ltok[k]) * h + col);
+      float4& a4 = acc[lrow[k] * CV + tid];
+      a4.x += f.x;
+      a4.y += f.y;
+      a4.z += f.z;
+      a4.w += f.w;
     }
   }
   if (!col_ok) return;
@@ -202,12 +233,11 @@ __global__ void __launch_bounds__(kEmbThreads) emb_bucket_accum(
     if (v >= Vp) break;
     const int s = static_cast<int>(v / Vs);
     T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + col;
+    const float4 a4 = acc[r * CV + tid];
     if constexpr (sizeof(T) == 2) {
-      *reinterpret_cast<uint32_t*>(dst) =
-          tpd::pack_bf16x2(acc[r * kEmbCols + 2 * tid], acc[r * kEmbCols + 2 * tid + 1]);
+      *reinterpret_cast<uint2*>(dst) = make_uint2(tpd::pack_bf16x2(a4.x, a4.y), tpd::pack_bf16x2(a4.z, a4.w));
     } else {
-      *reinterpret_cast<float2*>(dst) =
-          make_float2(acc[r * kEmbCols + 2 * tid], acc[r * kEmbCols + 2 * tid + 1]);
+      *reinterpret_cast<float4*>(dst) = a4;
     }
   }
 }
@@ -218,30 +248,81 @@ __device__ __forceinline__ float ld_logit(const void* p, int64_t i) {
   else return static_cast<const float*>(p)[i];
 }
 
+// 2^x by the hardware approximation (denormal results flush to 0).
+__device__ __forceinline__ float ex2f_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Running (max, sum of exp2) pair in the log2 domain: the pair (m, s) stands
 // for s * 2^m. Merging rescales the smaller side; an empty side is (-inf, 0).
 struct MaxSum {
   float m, s;
 };
 
-__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b) {
-  const float m = fmaxf(a.m, b.m);
-  if (m == -INFINITY) return {m, 0.f};
-  return {m, a.s * exp2f(a.m - m) + b.s * exp2f(b.m - m)};
-}
-
-template <int THREADS>
-__device__ __forceinline__ MaxSum block_merge(MaxSum v, float2* red) {
+// CTA-wide max or sum: warp shuffles, then warp 0 combines the warps' values;
+// every thread gets the result. red holds THREADS / 32 + 1 floats.
+template <int THREADS, bool MAX>
+__device__ __forceinline__ float block_reduce(float v, float* red) {
+  constexpr int W = THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    MaxSum u{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
-    v = merge(v, u);
+    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = MAX ? fmaxf(v, u) : v + u;
   }
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(v.m, v.s);
+  __syncthreads();  // red may still be read from the previous use
+  if (lane == 0) red[warp] = v;
   __syncthreads();
-  MaxSum r{red[0].x, red[0].y};
-  for (int w = 1; w < THREADS / 32; ++w) r = merge(r, MaxSum{red[w].x, red[w].y});
-  return r;
+  if (warp == 0) {
+    float x = lane < W ? red[lane] : (MAX ? -INFINITY : 0.f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float u = __shfl_xor_sync(0xffffffffu, x, o);
+      x = MAX ? fmaxf(x, u) : x + u;
+    }
+    if (lane == 0) red[W] = x;
+  }
+  __syncthreads();
+  return red[W];
+}
+
+// Merge of every thread's (max m, sum s of 2^(x - m)): the CTA max M, then
+// the sum of s * 2^(m - M) (threads that saw no column hold (-inf, 0)).
+template <int THREADS>
+__device__ __forceinline__ MaxSum block_merge(MaxSum v, float* red) {
+  const float M = block_reduce<THREADS, true>(v.m, red);
+  const float s = v.m == -INFINITY ? 0.f : v.s * exp2f(v.m - M);
+  return {M, block_reduce<THREADS, false>(s, red)};
+}
+
+// Two (max, sum of 2^(x - max)) pairs as one.
+__device__ __forceinline__ MaxSum merge2(MaxSum a, MaxSum b) {
+  const float m = fmaxf(a.m, b.m);
+  if (m == -INFINITY) return {m, 0.f};
+  return {m, a.s * ex2f_fast(a.m - m) + b.s * ex2f_fast(b.m - m)};
+}
+
+// The same merge with one barrier: pairs merged within each warp by
+// shuffles, one pair per warp through shared memory (red2 holds THREADS / 32
+// pairs), then every warp merges those by shuffles again. red2 must not be
+// written again before every thread has returned (the caller's next barrier).
+template <int THREADS>
+__device__ __forceinline__ MaxSum block_merge1(MaxSum v, float2* red2) {
+  constexpr int W = THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    v = merge2(v, MaxSum{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)});
+  if (lane == 0) red2[warp] = make_float2(v.m, v.s);
+  __syncthreads();
+  const float2 w = lane < W ? red2[lane] : make_float2(-INFINITY, 0.f);
+  MaxSum u{w.x, w.y};
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    u = merge2(u, MaxSum{__shfl_xor_sync(0xffffffffu, u.m, o), __shfl_xor_sync(0xffffffffu, u.s, o)});
+  return u;
 }
 
 // 16 bytes of logits as floats (8 bf16 or 4 fp32).
@@ -296,7 +377,7 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
     unsigned* status) {
   constexpr int N = Vec<T>::N;
   constexpr float kLog2e = 1.4426950408889634f;
-  __shared__ float2 red[THREADS / 32];
+  __shared__ float red[THREADS / 32 + 1];
   __shared__ float ztarget;
   const int64_t t = blockIdx.x;
   const int label = labels[t];
@@ -362,105 +443,162 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
   }
 }
 
-// Rows of up to kCeSmemMax bytes: one CTA per token row copies the row's p
-// shard slices into shared memory with bulk copies (one per shard, completing
-// on one mbarrier), takes each thread's max and sum of exp2 relative to it
-// from there, merges the (max, sum) pairs over the CTA and writes the gradient
-// from the same shared copy, so the logits cross HBM exactly once and no
-// registers hold the row. The shards are contiguous slices of the padded
-// vocab, so 16-byte vector i of the row holds columns [i * N, (i + 1) * N).
-template <typename T, int THREADS>
-__global__ void __launch_bounds__(THREADS) vocab_ce_smem_kernel(
+// Rows of up to kCeSmemMax / 2 bytes, persistent CTAs: CTA b takes rows
+// b, b + G, b + 2G, ... and keeps STAGES of them in flight in shared memory.
+// Each row's p shard slices arrive by bulk copy (one per shard, completing on
+// the stage's mbarrier) while the CTA works on the rows before it; each
+// thread takes its max and sum of exp2 from the shared copy, the CTA merges
+// the (max, sum) pairs and writes the gradient from the same copy, so the
+// logits cross HBM exactly once and loads overlap the exponentials. The
+// shards are contiguous slices of the padded vocab, so 16-byte vector i of
+// a row holds columns [i * N, (i + 1) * N).
+template <typename T, int THREADS, int STAGES>
+__global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
-    int vocab, const int32_t* labels, float scale, float* loss, float* lse_out,
-    unsigned* status) {
+    int vocab, int64_t T_rows, uint32_t stage_bytes, const int32_t* labels, float scale,
+    float* loss, float* lse_out, unsigned* status) {
   constexpr int N = Vec<T>::N;
   constexpr float kLog2e = 1.4426950408889634f;
-  extern __shared__ __align__(128) uint8_t srow[];
-  __shared__ uint64_t bar;
+  extern __shared__ __align__(128) uint8_t sbuf[];
+  __shared__ uint64_t bar[STAGES];
   __shared__ int abort_flag;
-  __shared__ float2 red[THREADS / 32];
-  const int64_t t = blockIdx.x;
+  __shared__ float2 red2[THREADS / 32];
   const uint32_t shard_bytes = static_cast<uint32_t>(Vs * sizeof(T));
+  const int64_t G0 = blockIdx.x, GS = gridDim.x;
+  auto issue = [&](int64_t k) {  // thread 0: start loading the CTA's k-th row
+    const int64_t t = G0 + k * GS;
+    if (t >= T_rows) return;
+    const int st = static_cast<int>(k % STAGES);
+    uint8_t* dst = sbuf + static_cast<size_t>(st) * stage_bytes;
+    tpd::mbar_arrive_expect_tx(&bar[st], shard_bytes * static_cast<uint32_t>(p));
+    for (int s = 0; s < p; ++s)
+      tpd::bulk_load(dst + static_cast<size_t>(s) * shard_bytes,
+                     static_cast<const uint8_t*>(L.p[s]) + t * shard_bytes, shard_bytes, &bar[st]);
+  };
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    tpd::mbar_init(&bar, 1);
+    for (int st = 0; st < STAGES; ++st) tpd::mbar_init(&bar[st], 1);
     tpd::fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    tpd::mbar_arrive_expect_tx(&bar, shard_bytes * static_cast<uint32_t>(p));
-    for (int s = 0; s < p; ++s)
-      tpd::bulk_load(srow + static_cast<size_t>(s) * shard_bytes,
-                     static_cast<const uint8_t*>(L.p[s]) + t * shard_bytes, shard_bytes, &bar);
-  }
-  const int label = labels[t];
-  const bool ignore = label < 0 || label >= vocab;
-  const bool ok = tpd::mbar_wait(&bar, 0, &abort_flag, status);
-  if (!__syncthreads_and(ok)) {
-    // The copies did not land in time: give them one more bounded wait so
-    // none is still writing this CTA's shared memory when it exits.
-    if (threadIdx.x == 0) {
-      int again = 0;
-      tpd::mbar_wait(&bar, 0, &again, nullptr);
-    }
-    __syncthreads();
-    return;
-  }
+  if (threadIdx.x == 0)
+    for (int k = 0; k < STAGES; ++k) issue(k);
   const int nv = static_cast<int>(Vs / N);
   const int total = p * nv;
-  const uint4* row = reinterpret_cast<const uint4*>(srow);
-  float m = -INFINITY;
-  for (int i = threadIdx.x; i < total; i += THREADS) {
-    Vec<T> x;
-    x.unpack(row[i]);
-#pragma unroll
-    for (int e = 0; e < N; ++e)
-      if (i * N + e < vocab) m = fmaxf(m, x.v[e] * kLog2e);
-  }
-  float sum = 0.f;
-  if (m != -INFINITY) {
+  int64_t k = 0;
+  for (;; ++k) {
+    const int64_t t = G0 + k * GS;
+    if (t >= T_rows) break;
+    const int st = static_cast<int>(k % STAGES);
+    const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
+    if (!__syncthreads_and(ok)) break;
+    const uint4* row = reinterpret_cast<const uint4*>(sbuf + static_cast<size_t>(st) * stage_bytes);
+    const int label = labels[t];
+    const bool ignore = label < 0 || label >= vocab;
+    // Vectors below nfull hold no padding column: no per-column tests there.
+    const int nfull = vocab / N;
+    // One pass: this thread's running max (log2 domain) and sum of 2^(x - max).
+    float m = -INFINITY, sum = 0.f;
     for (int i = threadIdx.x; i < total; i += THREADS) {
       Vec<T> x;
       x.unpack(row[i]);
+      if (i >= nfull) {
 #pragma unroll
-      for (int e = 0; e < N; ++e)
-        if (i * N + e < vocab) sum += exp2f(fmaf(x.v[e], kLog2e, -m));
-    }
-  }
-  const MaxSum tot = block_merge<THREADS>(MaxSum{m, sum}, red);
-  const float lse2 = tot.m + log2f(tot.s);
-  if (threadIdx.x == 0) {
-    if (label >= vocab) atomicOr(status, kStatusBadIndex);
-    float zt = 0.f;
-    if (!ignore) {
-      Vec<T> x;
-      x.unpack(row[label / N]);
-      zt = x.v[label % N];
-    }
-    const float lse = lse2 * 0.6931471805599453f;
-    loss[t] = ignore ? 0.f : lse - zt;
-    if (lse_out) lse_out[t] = lse;
-  }
-  if (G.p[0] == nullptr) return;
-  for (int i = threadIdx.x; i < total; i += THREADS) {
-    Vec<T> x;
-    x.unpack(row[i]);
+        for (int e = 0; e < N; ++e)
+          if (i * N + e >= vocab) x.v[e] = -INFINITY;
+      }
+      float lm = x.v[0];
 #pragma unroll
-    for (int e = 0; e < N; ++e) {
-      const int c = i * N + e;
-      float g = 0.f;
-      if (!ignore && c < vocab)
-        g = (exp2f(fmaf(x.v[e], kLog2e, -lse2)) - (c == label ? 1.f : 0.f)) * scale;
-      x.v[e] = g;
+      for (int e = 1; e < N; ++e) lm = fmaxf(lm, x.v[e]);
+      lm *= kLog2e;
+      if (lm == -INFINITY) continue;  // all padding
+      if (lm > m) {
+        sum *= ex2f_fast(m - lm);
+        m = lm;
+      }
+#pragma unroll
+      for (int e = 0; e < N; ++e) sum += ex2f_fast(fmaf(x.v[e], kLog2e, -m));
     }
-    const int s = i / nv;
-    x.store(G.p[s], t * nv + (i - s * nv));
+    const MaxSum tot = block_merge1<THREADS>(MaxSum{m, sum}, red2);
+    const float lse2 = tot.m + log2f(tot.s);
+    if (threadIdx.x == 0) {
+      if (label >= vocab) atomicOr(status, kStatusBadIndex);
+      float zt = 0.f;
+      if (!ignore) {
+        Vec<T> x;
+        x.unpack(row[label / N]);
+        zt = x.v[label % N];
+      }
+      const float lse = lse2 * 0.6931471805599453f;
+      loss[t] = ignore ? 0.f : lse - zt;
+      if (lse_out) lse_out[t] = lse;
+    }
+    if (G.p[0] != nullptr) {
+      const int lab_vec = ignore ? -1 : label / N;
+      for (int i = threadIdx.x; i < total; i += THREADS) {
+        Vec<T> x;
+        x.unpack(row[i]);
+        if (ignore) {
+#pragma unroll
+          for (int e = 0; e < N; ++e) x.v[e] = 0.f;
+        } else if (i < nfull) {
+#pragma unroll
+          for (int e = 0; e < N; ++e) x.v[e] = ex2f_fast(fmaf(x.v[e], kLog2e, -lse2)) * scale;
+        } else {
+#pragma unroll
+          for (int e = 0; e < N; ++e)
+            x.v[e] = i * N + e < vocab ? ex2f_fast(fmaf(x.v[e], kLog2e, -lse2)) * scale : 0.f;
+        }
+        if (i == lab_vec) {  // minus the one-hot target
+#pragma unroll
+          for (int e = 0; e < N; ++e)
+            if (e == label - i * N) x.v[e] -= scale;
+        }
+        const int s = i / nv;
+        x.store(G.p[s], t * nv + (i - s * nv));
+      }
+    }
+    __syncthreads();  // every thread is done with this stage
+    if (threadIdx.x == 0) issue(k + STAGES);
+  }
+  // On a time-out, let the copies still in flight land (bounded) before exit.
+  if (threadIdx.x == 0 && abort_flag) {
+    for (int64_t kk = k; kk < k + STAGES; ++kk) {
+      if (G0 + kk * GS >= T_rows) break;
+      int again = 0;
+      tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+    }
   }
 }
 
-constexpr int kCeSmemSmall = 64 * 1024;    // up to 3 CTAs per SM
-constexpr int kCeSmemMax = 200 * 1024;     // one CTA per SM
+constexpr int kCeSmemMax = 200 * 1024;  // shared memory for the staged rows
+
+template <typename E, int THREADS, int STAGES>
+tp_status launch_ce_pipe(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
+                         const int32_t* labels, float scale, float* loss, float* lse, int64_t T,
+                         uint32_t stage_bytes, unsigned* status, cudaStream_t st) {
+  static bool attr = false;
+  auto fn = vocab_ce_pipe_kernel<E, THREADS, STAGES>;
+  if (!attr) {
+    tp_status r = tpi::cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kCeSmemMax),
+                              "cudaFuncSetAttribute(vocab_cross_entropy)");
+    if (r != TP_OK) return r;
+    attr = true;
+  }
+  const int smem = static_cast<int>(stage_bytes) * STAGES;
+  int per_sm = 0;
+  tp_status r = tpi::cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, THREADS, smem),
+                            "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (r != TP_OK) return r;
+  int dev = 0, n_sm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(T, static_cast<int64_t>(n_sm) * std::max(per_sm, 1)));
+  fn<<<static_cast<unsigned>(grid), THREADS, smem, st>>>(L, G, p, Vs, vocab, T, stage_bytes, labels,
+                                                         scale, loss, lse, status);
+  return TP_OK;
+}
 
 int sms() {
   int dev = 0, n = 0;
@@ -549,48 +687,21 @@ tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_
   tp_status s = device_status_word(&status);
   if (s != TP_OK) return s;
   const int64_t row_bytes = static_cast<int64_t>(p) * Vs * static_cast<int64_t>(dsize(dt));
-  const unsigned grid = static_cast<unsigned>(T);
-  static bool attr[4] = {false, false, false, false};
-  auto set_attr = [&](const void* fn, int k) -> tp_status {
-    if (attr[k]) return TP_OK;
-    tp_status r = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   kCeSmemMax),
-                              "cudaFuncSetAttribute(vocab_cross_entropy)");
-    if (r == TP_OK) attr[k] = true;
-    return r;
-  };
-  const int smem = static_cast<int>(row_bytes);
-  if (row_bytes <= kCeSmemSmall) {
-    if (dt == TP_BF16) {
-      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<__nv_bfloat16, 256>), 0);
-      if (s != TP_OK) return s;
-      vocab_ce_smem_kernel<__nv_bfloat16, 256><<<grid, 256, smem, st>>>(L, G, p, Vs, vocab, labels,
-                                                                         scale, loss, lse, status);
-    } else {
-      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<float, 256>), 1);
-      if (s != TP_OK) return s;
-      vocab_ce_smem_kernel<float, 256><<<grid, 256, smem, st>>>(L, G, p, Vs, vocab, labels, scale,
-                                                                 loss, lse, status);
-    }
-  } else if (row_bytes <= kCeSmemMax) {
-    if (dt == TP_BF16) {
-      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<__nv_bfloat16, 1024>), 2);
-      if (s != TP_OK) return s;
-      vocab_ce_smem_kernel<__nv_bfloat16, 1024><<<grid, 1024, smem, st>>>(
-          L, G, p, Vs, vocab, labels, scale, loss, lse, status);
-    } else {
-      s = set_attr(reinterpret_cast<const void*>(vocab_ce_smem_kernel<float, 1024>), 3);
-      if (s != TP_OK) return s;
-      vocab_ce_smem_kernel<float, 1024><<<grid, 1024, smem, st>>>(L, G, p, Vs, vocab, labels, scale,
-                                                                   loss, lse, status);
-    }
+  const uint32_t sb = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
+  if (3 * row_bytes <= kCeSmemMax) {
+    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 3>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
+                      : launch_ce_pipe<float, 1024, 3>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
+  } else if (2 * row_bytes <= kCeSmemMax) {
+    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 2>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
+                      : launch_ce_pipe<float, 1024, 2>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
   } else if (dt == TP_BF16) {
-    vocab_ce_kernel<__nv_bfloat16, 256><<<grid, 256, 0, st>>>(L, G, p, Vs, vocab, labels, scale,
-                                                              loss, lse, status);
+    vocab_ce_kernel<__nv_bfloat16, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(
+        L, G, p, Vs, vocab, labels, scale, loss, lse, status);
   } else {
-    vocab_ce_kernel<float, 256><<<grid, 256, 0, st>>>(L, G, p, Vs, vocab, labels, scale, loss,
-                                                      lse, status);
+    vocab_ce_kernel<float, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(L, G, p, Vs, vocab, labels,
+                                                                         scale, loss, lse, status);
   }
+  if (s != TP_OK) return s;
   return after_launch("vocab_cross_entropy");
 }
 

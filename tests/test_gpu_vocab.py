@@ -52,10 +52,11 @@ def test_embedding_fwd_bwd(p, dtype):
                                        (4, 50000, "bf16"), (8, 128000, "bf16"), (3, 997, "f32"),
                                        (8, 32000, "f32")])
 def test_vocab_parallel_cross_entropy(p, V, dtype):
-    """Rows up to 64 KB and up to 200 KB (the shared-memory kernels) and wider
-    (the streaming kernel), padded and unpadded vocabularies, bf16 and fp32."""
+    """Rows staged three or two deep in shared memory (up to 66 KB / 100 KB)
+    and wider rows (the streaming kernel), padded and unpadded vocabularies,
+    bf16 and fp32; 1000 rows so every persistent CTA recycles its stages."""
     tp = _tp()
-    T, h = (300, 64) if V <= 50000 else (40, 64)
+    T, h = (1000, 64) if V <= 50000 else (40, 64)
     plan = tp.Plan(h if h % p == 0 else 3 * h, 0, 0, p, dtype, "none")
     Vp = plan.set_vocab(V)
     g = torch.Generator().manual_seed(V)
