@@ -13,8 +13,8 @@
 //               then per block PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one
 //               tile's MMAs run while the other tile's softmax works
 //   warps 2..5  softmax of tile A, warps 6..9 of tile B: thread r owns query
-//               row r; two passes over its row of S in TMEM (row max, then
-//               exp2 and the row sum), P rounded to bf16 and written to shared
+//               row r; its 128 scores of a block come from TMEM in one read
+//               (row max, then exp2 and the row sum), P rounded to bf16 and written to shared
 //               memory in the 128-byte-swizzled K-major layout of the PV MMA.
 //               Only the diagonal block (and a ragged last block) is masked.
 // O accumulates in TMEM across key blocks. P is taken relative to a reference
@@ -40,7 +40,10 @@ using tpi::PtrArray;
 
 constexpr int BQ = 128;   // queries per tile
 constexpr int BKV = 128;  // keys per block
+// Warps 0-3 softmax of tile A, 4-7 of tile B (warp w reads TMEM lanes
+// 32 (w % 4) ..), warp 8 TMA producer, warp 9 TMEM owner and MMA issuer.
 constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-atom column)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // raise the reference max when exceeded by > 2^8
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t tmem = *tmem_slot;
   // S of tile t in columns [128 t, 128 t + 128); O of tile t in [256 + D t, 256 + D (t + 1)).
 
-  if (warp == 0 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     // ------------------------------------------------------------- producer
     tma_prefetch_desc(tm);
     mbar_arrive_expect_tx(q_full, (nbt[1] > 0 ? 2 : 1) * SM::Q_BYTES);
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int uses = issued > k ? (issued - 1 - k) / SM::KV_SLOTS + 1 : 0;
       if (uses > 0) mbar_wait(&kv_full[k], static_cast<uint32_t>(uses - 1) & 1u, abort_flag, p.status);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == kMmaWarp && lane == 0) {
     // ---------------------------------------------------------- MMA issuer
     const uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
     const uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
@@ -242,9 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     tc_commit(drain);
     mbar_wait(drain, 0, abort_flag, p.status);
-  } else if (warp >= 2) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------- softmax
-    const int t = (warp - 2) / 4;  // query tile of this warpgroup
+    const int t = warp / 4;  // query tile of this warpgroup
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
     const int q = q0t[t] + r;
@@ -267,23 +270,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       // No column of this block is masked for any row of the warp (every block
       // but the diagonal one and a ragged last one): skip the per-column tests.
       const bool full = k0 + BKV - 1 <= min(q0t[t] + lg * 32, p.seq - 1);
+      // The whole 128-column row of S into registers with one wait; both
+      // passes below work from there.
+      float sv[BKV / 32][32];
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) tmem_ld32(tS + c * 32, sv[c]);
+      tc_wait_ld();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BKV / 32; c += 2) {
-        float sv[32], sw[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tS + c * 32 + 32, sw);
-        tc_wait_ld();
-        if (full) {
+      if (full) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(sv[i], sw[i]));
-        } else {
+        for (int c = 0; c < BKV / 32; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (c * 32 + i <= kmax) mx = fmaxf(mx, sv[i]);
-            if (c * 32 + 32 + i <= kmax) mx = fmaxf(mx, sw[i]);
-          }
-        }
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, sv[c][i]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BKV / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i <= kmax) mx = fmaxf(mx, sv[c][i]);
       }
       mx *= p.scale_log2;  // the scale is positive: max of the scaled scores
       if (j > 0) {
@@ -295,13 +299,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         tc_fence_after();
       }
+      // Raise the reference max only when some row of the warp outgrew it by
+      // more than 2^kRescale (warp-uniform: the O rescale below is a
+      // warp-collective TMEM access); rows whose max did not move get alpha 1.
+      float alpha = 1.f;
+      const bool rescale = j > 0 && __any_sync(0xffffffffu, mx > m + kRescale);
       if (j == 0) {
         m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + kRescale)) {
-        // tcgen05.ld / st are warp-collective: the whole warp rescales, each
-        // row by its own factor (1 for rows whose max did not move).
+      } else if (rescale) {
         const float m_new = fmaxf(m, mx);
-        const float alpha = exp2f(m - m_new);
+        alpha = exp2f(m - m_new);
+        m = m_new;
+      }
+      float rs = 0.f;
+      const float sc = p.scale_log2;
+#pragma unroll
+      for (int cc = 0; cc < BKV / 32; ++cc) {
+        uint8_t* rowp = sPt + (cc / 2) * CHUNK_BYTES + r * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {  // 8 columns -> one 16-byte store of P
+          uint32_t pk[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int i = v * 8 + 2 * w;
+            float a = ex2(fmaf(sv[cc][i], sc, -m));
+            float bb = ex2(fmaf(sv[cc][i + 1], sc, -m));
+            if (!full) {
+              a = (cc * 32 + i <= kmax) ? a : 0.f;
+              bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
+            }
+            pk[w] = pack_bf16x2(a, bb);
+            const float2 f = unpack_bf16x2(pk[w]);  // the row sum uses the rounded P of the PV MMA
+            rs += f.x + f.y;
+          }
+          const int qv = (cc % 2) * 4 + v;
+          *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      if (rescale) {
+        // O of the previous blocks (stable: their P.V is done) to the new reference.
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float ov[32];
@@ -312,44 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           tmem_st32(tO + c * 32, ov);
         }
         tc_wait_st();
-        l *= alpha;
-        m = m_new;
       }
-      float rs = 0.f;
-      const float sc = p.scale_log2;
-#pragma unroll 1
-      for (int c = 0; c < BKV / 32; c += 2) {
-        float sv[2][32];
-        tmem_ld32(tS + c * 32, sv[0]);
-        tmem_ld32(tS + c * 32 + 32, sv[1]);
-        tc_wait_ld();
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int cc = c + h2;
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float a = ex2(fmaf(sv[h2][i], sc, -m));
-            float bb = ex2(fmaf(sv[h2][i + 1], sc, -m));
-            if (!full) {
-              a = (cc * 32 + i <= kmax) ? a : 0.f;
-              bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
-            }
-            const uint32_t u = pack_bf16x2(a, bb);
-            pk[i / 2] = u;
-            const float2 f = unpack_bf16x2(u);  // the row sum uses the rounded P of the PV MMA
-            rs += f.x + f.y;
-          }
-          uint8_t* rowp = sPt + (cc / 2) * CHUNK_BYTES + r * 128;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int qv = (cc % 2) * 4 + v;
-            *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) =
-                make_uint4(pk[v * 4 + 0], pk[v * 4 + 1], pk[v * 4 + 2], pk[v * 4 + 3]);
-          }
-        }
-      }
-      l += rs;
+      l = l * alpha + rs;
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
