@@ -362,6 +362,16 @@ __device__ __forceinline__ void issue_row(const PtrArray& a, const PtrArray* b, 
                      static_cast<const uint8_t*>(b->p[s]) + r * shard_bytes, shard_bytes, bar);
 }
 
+// thread 0: store row r of the p shard buffers of `y` from `src` (its shard
+// slices back to back), one bulk copy per shard, as one bulk group.
+__device__ __forceinline__ void store_row(const MutPtrArray& y, int p, int64_t r, uint32_t shard_bytes,
+                                          const uint8_t* src) {
+  for (int s = 0; s < p; ++s)
+    tpd::bulk_store(static_cast<uint8_t*>(y.p[s]) + r * shard_bytes, src + static_cast<size_t>(s) * shard_bytes,
+                    shard_bytes);
+  tpd::bulk_commit();
+}
+
 template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
 __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
@@ -382,9 +392,10 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     tpd::fence_barrier_init();
   }
   __syncthreads();
+  int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
   if (threadIdx.x == 0)
-    for (int k = 0; k < STAGES && G0 + k * GS < rows; ++k)
-      issue_row(X, nullptr, p, G0 + k * GS, shard_bytes, sbuf + k * stage_bytes, &bar[k]);
+    for (; issued < STAGES && G0 + issued * GS < rows; ++issued)
+      issue_row(X, nullptr, p, G0 + issued * GS, shard_bytes, sbuf + issued * stage_bytes, &bar[issued]);
   // gamma (and beta) of this thread's columns, packed, for every row
   uint4 gp[VPT], bp[VPT];
 #pragma unroll
@@ -441,22 +452,34 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
         if (!RMS) LnVec<T>::unpack(bp[i], bb);
 #pragma unroll
         for (int e = 0; e < V; ++e) o[e] = (x[e] - mean) * rstd * g[e] + (RMS ? 0.f : bb[e]);
-        LnVec<T>::store(static_cast<T*>(Y.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+        LnVec<T>::store(const_cast<uint4*>(row) + c, o);  // y replaces x in the stage
       }
     }
     if (threadIdx.x == 0) {
       if (mean_out && !RMS) mean_out[r] = mean;
       if (rstd_out) rstd_out[r] = rstd;
     }
-    __syncthreads();  // every thread is done with this stage
-    if (threadIdx.x == 0 && G0 + (k + STAGES) * GS < rows)
-      issue_row(X, nullptr, p, G0 + (k + STAGES) * GS, shard_bytes, sbuf + st * stage_bytes, &bar[st]);
-  }
-  if (threadIdx.x == 0 && abort_flag) {  // let copies still in flight land (bounded)
-    for (int64_t kk = k; kk < k + STAGES && G0 + kk * GS < rows; ++kk) {
-      int again = 0;
-      tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+    tpd::fence_proxy_async_smem();
+    __syncthreads();  // the stage holds the row's y
+    if (threadIdx.x == 0) {
+      // y leaves by bulk copies; the previous row's stage is reloaded once its
+      // store has read it.
+      store_row(Y, p, r, shard_bytes, sbuf + st * stage_bytes);
+      tpd::bulk_wait_read<1>();
+      if (k >= 1 && G0 + (k - 1 + STAGES) * GS < rows) {
+        const int s2 = static_cast<int>((k - 1) % STAGES);
+        issue_row(X, nullptr, p, G0 + (k - 1 + STAGES) * GS, shard_bytes, sbuf + s2 * stage_bytes, &bar[s2]);
+        issued = k - 1 + STAGES + 1;
+      }
     }
+  }
+  if (threadIdx.x == 0) {
+    tpd::bulk_wait_all();  // every store has landed
+    if (abort_flag)        // let loads still in flight land (bounded)
+      for (int64_t kk = k; kk < issued; ++kk) {
+        int again = 0;
+        tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+      }
   }
 }
 
@@ -511,9 +534,10 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     tpd::fence_barrier_init();
   }
   __syncthreads();
+  int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
   if (threadIdx.x == 0)
-    for (int k = 0; k < STAGES && G0 + k * GS < rows; ++k)
-      issue_row(X, &DY, p, G0 + k * GS, shard_bytes, sbuf + k * stage_bytes, &bar[k]);
+    for (; issued < STAGES && G0 + issued * GS < rows; ++issued)
+      issue_row(X, &DY, p, G0 + issued * GS, shard_bytes, sbuf + issued * stage_bytes, &bar[issued]);
   uint4 gp[VPT];
   float pg[VPT][V], pb[VPT][V];
 #pragma unroll
@@ -570,18 +594,28 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
         LnVec<T>::unpack(gp[i], g);
 #pragma unroll
         for (int e = 0; e < V; ++e) o[e] = rstd * (d[e] * g[e] - m1 - (x[e] - mean) * rstd * m2);
-        LnVec<T>::store(static_cast<T*>(DX.p[sh]) + r * hs + static_cast<int64_t>(lc) * V, o);
+        LnVec<T>::store(const_cast<uint4*>(xrow) + c, o);  // dx replaces x in the stage
       }
     }
-    __syncthreads();  // every thread is done with this stage
-    if (threadIdx.x == 0 && G0 + (k + STAGES) * GS < rows)
-      issue_row(X, &DY, p, G0 + (k + STAGES) * GS, shard_bytes, sbuf + st * stage_bytes, &bar[st]);
-  }
-  if (threadIdx.x == 0 && abort_flag) {  // let copies still in flight land (bounded)
-    for (int64_t kk = k; kk < k + STAGES && G0 + kk * GS < rows; ++kk) {
-      int again = 0;
-      tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+    tpd::fence_proxy_async_smem();
+    __syncthreads();  // the stage holds the row's dx
+    if (threadIdx.x == 0) {
+      store_row(DX, p, r, shard_bytes, sbuf + st * stage_bytes);
+      tpd::bulk_wait_read<1>();
+      if (k >= 1 && G0 + (k - 1 + STAGES) * GS < rows) {
+        const int s2 = static_cast<int>((k - 1) % STAGES);
+        issue_row(X, &DY, p, G0 + (k - 1 + STAGES) * GS, shard_bytes, sbuf + s2 * stage_bytes, &bar[s2]);
+        issued = k - 1 + STAGES + 1;
+      }
     }
+  }
+  if (threadIdx.x == 0) {
+    tpd::bulk_wait_all();  // every store has landed
+    if (abort_flag)        // let loads still in flight land (bounded)
+      for (int64_t kk = k; kk < issued; ++kk) {
+        int again = 0;
+        tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
+      }
   }
   float* pgo = part + (static_cast<int64_t>(blockIdx.x) * 2 + 0) * h;
   float* pbo = part + (static_cast<int64_t>(blockIdx.x) * 2 + 1) * h;
