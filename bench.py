@@ -356,30 +356,27 @@ def time_standalone_reduce(pl, T, steps, stream):
 
 
 def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
+    """Every step copies X and dY in from pinned host memory and Y and dX
+    out, through HostStepPipeline (the copies of one step overlap the GEMMs
+    of its neighbours); the timed region ends when the last copy-out has
+    landed."""
     import torch
-    pl = m.plan
-    X = m.X
+    from megatron_tensor_transformer_gemm_b200.block import HostStepPipeline
     Y_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
     dX_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(X)
-    dYd = torch.empty_like(X)
-
-    def e2e_step():
-        Xd.copy_(X_h, non_blocking=True)
-        dYd.copy_(dY_h, non_blocking=True)
-        Y = m.forward(Xd)
-        dX = m.backward(dYd)
-        Y_h.copy_(Y, non_blocking=True)
-        dX_h.copy_(dX, non_blocking=True)
-
-    e2e_step()
+    pipe = HostStepPipeline(m, T)
+    for _ in range(2):
+        pipe.step(X_h, dY_h, Y_h, dX_h)
+    pipe.finish()
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    pipe.h2d.wait_stream(stream)  # the first copy-in starts inside the timed region
     for _ in range(args.steps):
-        e2e_step()
+        pipe.step(X_h, dY_h, Y_h, dX_h)
+    pipe.finish()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_value, e2e_ms = aggregate(flops, args.steps, e0.elapsed_time(e1), world)
@@ -556,6 +553,26 @@ def run_other(args, world, rank, local):
         roof = {"bound": "tensor", "kernel": "attn_fwd_kernel (tcgen05)", "achieved": ach,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
                 "peak_kind": f"bf16 burst ({peaks['source']}; timed alone)", "traffic": None}
+        if args.workload == "attn":
+            # The attention backward core alone (D prep + dK/dV + dQ launches):
+            # 2.5x the forward's FLOPs (S recomputed, dV, dP, dQ, dK).
+            blk.alloc_bwd()
+            g = torch.Generator(device="cpu").manual_seed(7 + rank)
+            for x in blk.dO:
+                x.copy_(torch.randn(x.shape, generator=g).to(torch.bfloat16))
+            bwd = lambda: blk.plan.attention_bwd(b, s, blk.QKV, blk.O, blk.dO, blk.LSE, blk.dQKV)
+            for _ in range(3):
+                bwd()
+            torch.cuda.synchronize()
+            c0.record(stream)
+            for _ in range(args.steps):
+                bwd()
+            c1.record(stream)
+            torch.cuda.synchronize()
+            achb = 2.5 * core_flops * args.steps / (c0.elapsed_time(c1) / 1e3) / 1e12
+            roof["backward"] = {"kernel": "attn_bwd_prep + attn_bwd_dkdv + attn_bwd_dq (tcgen05)",
+                                "achieved": achb, "unit": "TFLOP/s", "frac": achb / peaks["bf16_tflops"],
+                                "flops_per_launch_set": 2.5 * core_flops}
     if rank != 0:
         return 0
     print(json.dumps({"metric": f"{args.workload} TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",

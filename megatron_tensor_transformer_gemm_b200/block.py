@@ -166,6 +166,67 @@ class TPMLP:
         return 3.0 * fwd
 
 
+class HostStepPipeline:
+    """Training steps of a TPMLP fed from and drained to pinned host memory,
+    with the transfers overlapped with the compute: step(X_h, dY_h, Y_h, dX_h)
+    enqueues the host-to-device copies of X and dY on one stream, the
+    forward and backward on the current stream and the device-to-host copies
+    of Y and dX on another, with two device buffer sets so the copies of one
+    step run under the GEMMs of its neighbours. Every call returns at once;
+    finish() makes the current stream wait for all outstanding copies."""
+
+    def __init__(self, mlp: "TPMLP", T: int):
+        dev, dt, h = mlp.device, mlp.dt, mlp.h
+        self.m = mlp
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        self.X = [_empty((T, h), dt, dev) for _ in range(2)]
+        self.dY = [_empty((T, h), dt, dev) for _ in range(2)]
+        self.Y = [_empty((T, h), dt, dev) for _ in range(2)]
+        self.dX = [_empty((T, h), dt, dev) for _ in range(2)]
+        self.in_free = [None, None]   # compute done with input slot s
+        self.out_free = [None, None]  # copy-out done with output slot s
+        self.i = 0
+
+    def step(self, X_h, dY_h, Y_h, dX_h):
+        s = self.i % 2
+        self.i += 1
+        main = torch.cuda.current_stream()
+        with torch.cuda.stream(self.h2d):
+            if self.in_free[s] is not None:
+                self.h2d.wait_event(self.in_free[s])
+            self.X[s].copy_(X_h, non_blocking=True)
+            x_in = torch.cuda.Event()
+            x_in.record(self.h2d)
+            self.dY[s].copy_(dY_h, non_blocking=True)
+            dy_in = torch.cuda.Event()
+            dy_in.record(self.h2d)
+        main.wait_event(x_in)
+        if self.out_free[s] is not None:
+            main.wait_event(self.out_free[s])
+        self.m.forward(self.X[s], out=self.Y[s])
+        y_done = torch.cuda.Event()
+        y_done.record(main)
+        main.wait_event(dy_in)
+        self.m.backward(self.dY[s], out=self.dX[s])
+        dx_done = torch.cuda.Event()
+        dx_done.record(main)
+        self.in_free[s] = dx_done  # the backward reads X (weight gradient) and dY
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(y_done)
+            Y_h.copy_(self.Y[s], non_blocking=True)
+            self.d2h.wait_event(dx_done)
+            dX_h.copy_(self.dX[s], non_blocking=True)
+            out = torch.cuda.Event()
+            out.record(self.d2h)
+        self.out_free[s] = out
+
+    def finish(self):
+        main = torch.cuda.current_stream()
+        main.wait_stream(self.h2d)
+        main.wait_stream(self.d2h)
+
+
 class SPMLP:
     """Megatron-SP SwiGLU MLP: LayerNorm on sequence shards, all-gather, column,
     row, reduce-scatter (and the mirrored backward)."""

@@ -297,33 +297,36 @@ __device__ __forceinline__ MaxSum block_merge(MaxSum v, float* red) {
   return {M, block_reduce<THREADS, false>(s, red)};
 }
 
-// Two (max, sum of 2^(x - max)) pairs as one.
-__device__ __forceinline__ MaxSum merge2(MaxSum a, MaxSum b) {
-  const float m = fmaxf(a.m, b.m);
-  if (m == -INFINITY) return {m, 0.f};
-  return {m, a.s * ex2f_fast(a.m - m) + b.s * ex2f_fast(b.m - m)};
-}
-
-// The same merge with one barrier: pairs merged within each warp by
-// shuffles, one pair per warp through shared memory (red2 holds THREADS / 32
-// pairs), then every warp merges those by shuffles again. red2 must not be
-// written again before every thread has returned (the caller's next barrier).
+// The same merge with one barrier, which also carries every thread's wait
+// result: each warp merges its threads' pairs by shuffles, one pair per warp
+// goes through shared memory, and every warp merges those pairs again by
+// shuffles. Returns false (for every thread) if any thread's ok is false.
+// red2 holds THREADS / 32 pairs; it is written again only after the caller's
+// next barrier.
 template <int THREADS>
-__device__ __forceinline__ MaxSum block_merge1(MaxSum v, float2* red2) {
+__device__ __forceinline__ bool block_merge_ok(MaxSum& v, bool ok, float2* red2) {
   constexpr int W = THREADS / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float M = v.m;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-    v = merge2(v, MaxSum{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)});
-  if (lane == 0) red2[warp] = make_float2(v.m, v.s);
-  __syncthreads();
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float S = v.m == -INFINITY ? 0.f : v.s * ex2f_fast(v.m - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  if (lane == 0) red2[warp] = make_float2(M, S);
+  if (!__syncthreads_and(ok)) return false;
   const float2 w = lane < W ? red2[lane] : make_float2(-INFINITY, 0.f);
-  MaxSum u{w.x, w.y};
+  float M2 = w.x;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-    u = merge2(u, MaxSum{__shfl_xor_sync(0xffffffffu, u.m, o), __shfl_xor_sync(0xffffffffu, u.s, o)});
-  return u;
+  for (int o = 16; o > 0; o >>= 1) M2 = fmaxf(M2, __shfl_xor_sync(0xffffffffu, M2, o));
+  float S2 = w.x == -INFINITY ? 0.f : w.y * ex2f_fast(w.x - M2);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S2 += __shfl_xor_sync(0xffffffffu, S2, o);
+  v = MaxSum{M2, S2};
+  return true;
 }
+
+
 
 // 16 bytes of logits as floats (8 bf16 or 4 fp32).
 template <typename T>
@@ -448,8 +451,10 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
 // Each row's p shard slices arrive by bulk copy (one per shard, completing on
 // the stage's mbarrier) while the CTA works on the rows before it; each
 // thread takes its max and sum of exp2 from the shared copy, the CTA merges
-// the (max, sum) pairs and writes the gradient from the same copy, so the
-// logits cross HBM exactly once and loads overlap the exponentials. The
+// the (max, sum) pairs, the gradient overwrites the shared copy and leaves by
+// bulk copies too (a stage is reloaded once its store has read it), so the
+// logits cross HBM exactly once each way and the SM's load/store units stay
+// out of the stream. The
 // shards are contiguous slices of the padded vocab, so 16-byte vector i of
 // a row holds columns [i * N, (i + 1) * N).
 template <typename T, int THREADS, int STAGES>
@@ -465,9 +470,11 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
   __shared__ float2 red2[THREADS / 32];
   const uint32_t shard_bytes = static_cast<uint32_t>(Vs * sizeof(T));
   const int64_t G0 = blockIdx.x, GS = gridDim.x;
+  int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
   auto issue = [&](int64_t k) {  // thread 0: start loading the CTA's k-th row
     const int64_t t = G0 + k * GS;
     if (t >= T_rows) return;
+    issued = k + 1;
     const int st = static_cast<int>(k % STAGES);
     uint8_t* dst = sbuf + static_cast<size_t>(st) * stage_bytes;
     tpd::mbar_arrive_expect_tx(&bar[st], shard_bytes * static_cast<uint32_t>(p));
@@ -485,15 +492,18 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     for (int k = 0; k < STAGES; ++k) issue(k);
   const int nv = static_cast<int>(Vs / N);
   const int total = p * nv;
+  int next_label = G0 < T_rows ? labels[G0] : 0;  // the next row's label, loaded a row early
   int64_t k = 0;
   for (;; ++k) {
     const int64_t t = G0 + k * GS;
     if (t >= T_rows) break;
+    const int label = next_label;
+    if (t + GS < T_rows) next_label = labels[t + GS];
     const int st = static_cast<int>(k % STAGES);
+    // A thread whose wait gave up reads a stage that may not have landed; its
+    // values are discarded: the merge's barrier tells every thread to stop.
     const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
-    if (!__syncthreads_and(ok)) break;
     const uint4* row = reinterpret_cast<const uint4*>(sbuf + static_cast<size_t>(st) * stage_bytes);
-    const int label = labels[t];
     const bool ignore = label < 0 || label >= vocab;
     // Vectors below nfull hold no padding column: no per-column tests there.
     const int nfull = vocab / N;
@@ -519,7 +529,8 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
 #pragma unroll
       for (int e = 0; e < N; ++e) sum += ex2f_fast(fmaf(x.v[e], kLog2e, -m));
     }
-    const MaxSum tot = block_merge1<THREADS>(MaxSum{m, sum}, red2);
+    MaxSum tot{m, sum};
+    if (!block_merge_ok<THREADS>(tot, ok, red2)) break;
     const float lse2 = tot.m + log2f(tot.s);
     if (threadIdx.x == 0) {
       if (label >= vocab) atomicOr(status, kStatusBadIndex);
@@ -533,8 +544,10 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
       loss[t] = ignore ? 0.f : lse - zt;
       if (lse_out) lse_out[t] = lse;
     }
-    if (G.p[0] != nullptr) {
+    const bool grad = G.p[0] != nullptr;
+    if (grad) {
       const int lab_vec = ignore ? -1 : label / N;
+      uint4* out = const_cast<uint4*>(row);  // the gradient replaces the staged row
       for (int i = threadIdx.x; i < total; i += THREADS) {
         Vec<T> x;
         x.unpack(row[i]);
@@ -554,17 +567,31 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
           for (int e = 0; e < N; ++e)
             if (e == label - i * N) x.v[e] -= scale;
         }
-        const int s = i / nv;
-        x.store(G.p[s], t * nv + (i - s * nv));
+        x.store(out, i);
+      }
+      tpd::fence_proxy_async_smem();
+    }
+    __syncthreads();  // every thread is done with this stage (and its gradient is in it)
+    if (threadIdx.x == 0) {
+      if (grad) {
+        // Store the row's gradient from shared memory, one bulk copy per shard;
+        // then reload the stage of the previous row once its store has read it.
+        const uint8_t* src = sbuf + static_cast<size_t>(st) * stage_bytes;
+        for (int s = 0; s < p; ++s)
+          tpd::bulk_store(static_cast<uint8_t*>(G.p[s]) + t * shard_bytes, src + static_cast<size_t>(s) * shard_bytes,
+                          shard_bytes);
+        tpd::bulk_commit();
+        tpd::bulk_wait_read<1>();
+        if (k >= 1) issue(k - 1 + STAGES);
+      } else {
+        issue(k + STAGES);
       }
     }
-    __syncthreads();  // every thread is done with this stage
-    if (threadIdx.x == 0) issue(k + STAGES);
   }
-  // On a time-out, let the copies still in flight land (bounded) before exit.
+  if (threadIdx.x == 0) tpd::bulk_wait_all();  // every gradient store has landed
+  // On a time-out, let the loads still in flight land (bounded) before exit.
   if (threadIdx.x == 0 && abort_flag) {
-    for (int64_t kk = k; kk < k + STAGES; ++kk) {
-      if (G0 + kk * GS >= T_rows) break;
+    for (int64_t kk = k; kk < issued; ++kk) {
       int again = 0;
       tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
     }
