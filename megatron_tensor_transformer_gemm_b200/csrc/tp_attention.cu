@@ -250,14 +250,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int t = warp / 4;  // query tile of this warpgroup
     const int lg = warp & 3;
     const int r = lg * 32 + lane;
-    const int q = q0t[t] + r;
+    // this tile's first query and key-block count as scalars (an index by t
+    // into the two-entry arrays would place them in local memory)
+    const int my_q0 = t ? q0t[1] : q0t[0];
+    const int my_nb = t ? nbt[1] : nbt[0];
+    const int q = my_q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const uint32_t tS = tmem + 128 * t + lane_off;
     const uint32_t tO = tmem + 256 + D * t + lane_off;
     uint8_t* sPt = sP + t * SM::P_BYTES;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nbt[t] && ok; ++j) {
+    for (int j = 0; j < my_nb && ok; ++j) {
       // The whole warp proceeds together (tcgen05.ld below is warp-collective).
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag,
                                               p.status))) {
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const int kmax = min(q, p.seq - 1) - k0;  // last visible column of this block
       // No column of this block is masked for any row of the warp (every block
       // but the diagonal one and a ragged last one): skip the per-column tests.
-      const bool full = k0 + BKV - 1 <= min(q0t[t] + lg * 32, p.seq - 1);
+      const bool full = k0 + BKV - 1 <= min(my_q0 + lg * 32, p.seq - 1);
       // The whole 128-column row of S into registers with one wait; both
       // passes below work from there.
       float sv[BKV / 32][32];
@@ -355,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && nbt[t] > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&o_done[t], static_cast<uint32_t>(nbt[t] - 1) & 1u,
+    if (ok && my_nb > 0 &&
+        __all_sync(0xffffffffu, mbar_wait(&o_done[t], static_cast<uint32_t>(my_nb - 1) & 1u,
                                           abort_flag, p.status))) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;

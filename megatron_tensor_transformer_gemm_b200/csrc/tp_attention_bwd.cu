@@ -12,7 +12,8 @@
 //   attn_bwd_dq     one CTA per 128-query block: loops over its key blocks;
 //                   dS to shared memory (K-major) for dQ += dS K (TMEM)
 // Warp roles in both main kernels: warp 0 TMA, warp 1 TMEM + MMA issue, warps
-// 2..5 one row each (softmax recompute, dS, epilogue). Waits are bounded.
+// 2..9 the element-wise work (softmax recompute, dS, epilogue), two warps per
+// TMEM lane quarter, each on half of the 128 columns. Waits are bounded.
 #include <cuda.h>
 
 #include <algorithm>
@@ -29,7 +30,9 @@ using tpi::MutPtrArray;
 using tpi::PtrArray;
 
 constexpr int BQ = 128, BKV = 128;
-constexpr int kThreads = 192;
+// Warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..9 the element-wise work:
+// warp w takes TMEM lane quarter w % 4 and column half (w - 2) / 4.
+constexpr int kThreads = 320;
 constexpr int CHUNK = 128 * 128;  // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -110,13 +113,14 @@ __global__ void attn_bwd_prep(const __grid_constant__ PtrArray O, const __grid_c
   if (lane == 0) static_cast<float*>(dvec.p[shard])[(static_cast<int64_t>(b) * hl + hh) * seq + q] = s;
 }
 
-// Row r of this CTA's 128 x 128 (query x key) block: P and dS recomputed from
-// S and dP in TMEM. Writes P (if sP) and dS as bf16 into 128B-swizzled tiles.
+// Row r of this CTA's 128 x 128 (query x key) block, 32-column chunks
+// [c0, c0 + 2): P and dS recomputed from S and dP in TMEM. Writes P (if sP)
+// and dS as bf16 into 128B-swizzled tiles.
 __device__ __forceinline__ void p_ds_row(uint32_t tS, uint32_t tdP, uint32_t lane_off, int r, int q,
                                          int k0, int seq, float scale_log2, float lse2, float Dq,
-                                         uint8_t* sP, uint8_t* sdS) {
+                                         uint8_t* sP, uint8_t* sdS, int c0) {
 #pragma unroll 1
-  for (int c = 0; c < BKV / 32; ++c) {
+  for (int c = c0; c < c0 + 2; ++c) {
     float s[32], dp[32];
     tmem_ld32(tS + lane_off + c * 32, s);
     tmem_ld32(tdP + lane_off + c * 32, dp);
@@ -188,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(pds_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -274,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
     mbar_wait(drain, 0, abort_flag, p.status);
   } else if (warp >= 2) {
     const int lg = warp & 3;
+    const int half = (warp - 2) / 4;
     const int r = lg * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const float* lse = p.lse[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
         break;
       }
       tc_fence_after();
-      p_ds_row(tS, tdP, lane_off, r, q, k0, p.seq, p.scale_log2, lse2, Dq, sP, sdS);
+      p_ds_row(tS, tdP, lane_off, r, q, k0, p.seq, p.scale_log2, lse2, Dq, sP, sdS, 2 * half);
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -303,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
                             (static_cast<int64_t>(key) * p.batch + b) * (3 * hl_d) + hh * D;
       const bool st_ok = key < p.seq;
-      tmem_row_to_global<D>(tdV + lane_off, base + 2 * hl_d, 1.f, st_ok);
-      tmem_row_to_global<D>(tdK + lane_off, base + hl_d, p.scale, st_ok);
+      if (half == 0) tmem_row_to_global<D>(tdV + lane_off, base + 2 * hl_d, 1.f, st_ok);
+      else tmem_row_to_global<D>(tdK + lane_off, base + hl_d, p.scale, st_ok);
     }
   }
   tc_fence_before();
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(ds_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -449,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
     mbar_wait(drain, 0, abort_flag, p.status);
   } else if (warp >= 2) {
     const int lg = warp & 3;
+    const int half = (warp - 2) / 4;
     const int r = lg * 32 + lane;
     const int q = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
         break;
       }
       tc_fence_after();
-      p_ds_row(tS, tdP, lane_off, r, q, it * BKV, p.seq, p.scale_log2, lse2, Dq, nullptr, sdS);
+      p_ds_row(tS, tdP, lane_off, r, q, it * BKV, p.seq, p.scale_log2, lse2, Dq, nullptr, sdS, 2 * half);
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -476,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
       tc_fence_after();
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
                             (static_cast<int64_t>(q) * p.batch + b) * (3 * hl_d) + hh * D;
-      tmem_row_to_global<D>(tdQ + lane_off, base, p.scale, q < p.seq);
+      // each column half of warps stores half of dQ's D columns
+      tmem_row_to_global<D / 2>(tdQ + lane_off + half * (D / 2), base + half * (D / 2), p.scale, q < p.seq);
     }
   }
   tc_fence_before();

@@ -255,6 +255,30 @@ __device__ __forceinline__ float ex2f_fast(float x) {
   return y;
 }
 
+// 16 bytes as floats (8 bf16, widened exactly by shifts, or 4 fp32) and back.
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4 u, float (&x)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+    x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+    x[4] = __uint_as_float(u.z << 16); x[5] = __uint_as_float(u.z & 0xffff0000u);
+    x[6] = __uint_as_float(u.w << 16); x[7] = __uint_as_float(u.w & 0xffff0000u);
+  } else {
+    x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+  }
+}
+template <typename T>
+__device__ __forceinline__ uint4 pack16(const float (&x)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    return make_uint4(tpd::pack_bf16x2(x[0], x[1]), tpd::pack_bf16x2(x[2], x[3]),
+                      tpd::pack_bf16x2(x[4], x[5]), tpd::pack_bf16x2(x[6], x[7]));
+  } else {
+    return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
+                      __float_as_uint(x[3]));
+  }
+}
+
 // Running (max, sum of exp2) pair in the log2 domain: the pair (m, s) stands
 // for s * 2^m. Merging rescales the smaller side; an empty side is (-inf, 0).
 struct MaxSum {
@@ -446,6 +470,22 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
   }
 }
 
+// thread 0: start loading token row t (the CTA's k-th row) into stage
+// k % STAGES, one bulk copy per shard slice. False if t is past the rows.
+template <int STAGES>
+__device__ __forceinline__ bool ce_issue_row(const PtrArray& L, int p, int64_t t, int64_t T_rows,
+                                             uint32_t shard_bytes, uint8_t* sbuf, uint32_t stage_bytes,
+                                             uint64_t* bar, int64_t k) {
+  if (t >= T_rows) return false;
+  const int st = static_cast<int>(k % STAGES);
+  uint8_t* dst = sbuf + static_cast<size_t>(st) * stage_bytes;
+  tpd::mbar_arrive_expect_tx(&bar[st], shard_bytes * static_cast<uint32_t>(p));
+  for (int s = 0; s < p; ++s)
+    tpd::bulk_load(dst + static_cast<size_t>(s) * shard_bytes,
+                   static_cast<const uint8_t*>(L.p[s]) + t * shard_bytes, shard_bytes, &bar[st]);
+  return true;
+}
+
 // Rows of up to kCeSmemMax / 2 bytes, persistent CTAs: CTA b takes rows
 // b, b + G, b + 2G, ... and keeps STAGES of them in flight in shared memory.
 // Each row's p shard slices arrive by bulk copy (one per shard, completing on
@@ -471,17 +511,6 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
   const uint32_t shard_bytes = static_cast<uint32_t>(Vs * sizeof(T));
   const int64_t G0 = blockIdx.x, GS = gridDim.x;
   int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
-  auto issue = [&](int64_t k) {  // thread 0: start loading the CTA's k-th row
-    const int64_t t = G0 + k * GS;
-    if (t >= T_rows) return;
-    issued = k + 1;
-    const int st = static_cast<int>(k % STAGES);
-    uint8_t* dst = sbuf + static_cast<size_t>(st) * stage_bytes;
-    tpd::mbar_arrive_expect_tx(&bar[st], shard_bytes * static_cast<uint32_t>(p));
-    for (int s = 0; s < p; ++s)
-      tpd::bulk_load(dst + static_cast<size_t>(s) * shard_bytes,
-                     static_cast<const uint8_t*>(L.p[s]) + t * shard_bytes, shard_bytes, &bar[st]);
-  };
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int st = 0; st < STAGES; ++st) tpd::mbar_init(&bar[st], 1);
@@ -489,7 +518,8 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    for (int k = 0; k < STAGES; ++k) issue(k);
+    for (int k = 0; k < STAGES; ++k)
+      if (ce_issue_row<STAGES>(L, p, G0 + k * GS, T_rows, shard_bytes, sbuf, stage_bytes, bar, k)) issued = k + 1;
   const int nv = static_cast<int>(Vs / N);
   const int total = p * nv;
   int next_label = G0 < T_rows ? labels[G0] : 0;  // the next row's label, loaded a row early
@@ -510,24 +540,25 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     // One pass: this thread's running max (log2 domain) and sum of 2^(x - max).
     float m = -INFINITY, sum = 0.f;
     for (int i = threadIdx.x; i < total; i += THREADS) {
-      Vec<T> x;
-      x.unpack(row[i]);
+      float x[N];
+      unpack16<T>(row[i], x);
       if (i >= nfull) {
 #pragma unroll
         for (int e = 0; e < N; ++e)
-          if (i * N + e >= vocab) x.v[e] = -INFINITY;
+          if (i * N + e >= vocab) x[e] = -INFINITY;
       }
-      float lm = x.v[0];
+      float lm = x[0];
 #pragma unroll
-      for (int e = 1; e < N; ++e) lm = fmaxf(lm, x.v[e]);
+      for (int e = 1; e < N; ++e) lm = fmaxf(lm, x[e]);
       lm *= kLog2e;
-      if (lm == -INFINITY) continue;  // all padding
-      if (lm > m) {
+      if (lm > m) {  // (an all-padding vector has lm = -inf and adds nothing below)
         sum *= ex2f_fast(m - lm);
         m = lm;
       }
+      if (lm != -INFINITY) {
 #pragma unroll
-      for (int e = 0; e < N; ++e) sum += ex2f_fast(fmaf(x.v[e], kLog2e, -m));
+        for (int e = 0; e < N; ++e) sum += ex2f_fast(fmaf(x[e], kLog2e, -m));
+      }
     }
     MaxSum tot{m, sum};
     if (!block_merge_ok<THREADS>(tot, ok, red2)) break;
@@ -536,9 +567,12 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
       if (label >= vocab) atomicOr(status, kStatusBadIndex);
       float zt = 0.f;
       if (!ignore) {
-        Vec<T> x;
-        x.unpack(row[label / N]);
-        zt = x.v[label % N];
+        float x[N];
+        unpack16<T>(row[label / N], x);
+        // a bit test per element, not an index into x (which would put x in local memory)
+        const uint32_t bit = 1u << (label % N);
+#pragma unroll
+        for (int e = 0; e < N; ++e) zt += ((bit >> e) & 1u) ? x[e] : 0.f;
       }
       const float lse = lse2 * 0.6931471805599453f;
       loss[t] = ignore ? 0.f : lse - zt;
@@ -546,28 +580,37 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     }
     const bool grad = G.p[0] != nullptr;
     if (grad) {
+      // scale * softmax = 2^(x log2e - lse2 + log2 scale): the scale rides in
+      // the exponent when it is positive.
+      const bool fold = scale > 0.f;
+      const float bias = fold ? lse2 - log2f(scale) : lse2;
+      const float mul = fold ? 1.f : scale;
       const int lab_vec = ignore ? -1 : label / N;
       uint4* out = const_cast<uint4*>(row);  // the gradient replaces the staged row
       for (int i = threadIdx.x; i < total; i += THREADS) {
-        Vec<T> x;
-        x.unpack(row[i]);
+        float x[N];
+        unpack16<T>(row[i], x);
         if (ignore) {
 #pragma unroll
-          for (int e = 0; e < N; ++e) x.v[e] = 0.f;
+          for (int e = 0; e < N; ++e) x[e] = 0.f;
         } else if (i < nfull) {
 #pragma unroll
-          for (int e = 0; e < N; ++e) x.v[e] = ex2f_fast(fmaf(x.v[e], kLog2e, -lse2)) * scale;
+          for (int e = 0; e < N; ++e) x[e] = ex2f_fast(fmaf(x[e], kLog2e, -bias));
+          if (!fold) {
+#pragma unroll
+            for (int e = 0; e < N; ++e) x[e] *= mul;
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < N; ++e)
-            x.v[e] = i * N + e < vocab ? ex2f_fast(fmaf(x.v[e], kLog2e, -lse2)) * scale : 0.f;
+            x[e] = i * N + e < vocab ? ex2f_fast(fmaf(x[e], kLog2e, -bias)) * mul : 0.f;
         }
-        if (i == lab_vec) {  // minus the one-hot target
+        if (i == lab_vec) {  // minus the one-hot target (a bit test per element, as above)
+          const uint32_t bit = 1u << (label - i * N);
 #pragma unroll
-          for (int e = 0; e < N; ++e)
-            if (e == label - i * N) x.v[e] -= scale;
+          for (int e = 0; e < N; ++e) x[e] -= ((bit >> e) & 1u) ? scale : 0.f;
         }
-        x.store(out, i);
+        out[i] = pack16<T>(x);
       }
       tpd::fence_proxy_async_smem();
     }
@@ -582,9 +625,12 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
                           shard_bytes);
         tpd::bulk_commit();
         tpd::bulk_wait_read<1>();
-        if (k >= 1) issue(k - 1 + STAGES);
-      } else {
-        issue(k + STAGES);
+        if (k >= 1 && ce_issue_row<STAGES>(L, p, G0 + (k - 1 + STAGES) * GS, T_rows, shard_bytes, sbuf,
+                                           stage_bytes, bar, k - 1 + STAGES))
+          issued = k + STAGES;
+      } else if (ce_issue_row<STAGES>(L, p, G0 + (k + STAGES) * GS, T_rows, shard_bytes, sbuf, stage_bytes,
+                                      bar, k + STAGES)) {
+        issued = k + STAGES + 1;
       }
     }
   }
