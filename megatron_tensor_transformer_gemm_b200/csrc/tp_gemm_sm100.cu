@@ -113,6 +113,15 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, 
   nt = local - mt * p.g[g].tiles_n;
 }
 
+// A tile with at most BN / 2 valid columns left (the ragged last N tile of a
+// problem, e.g. N = 1376 = 5 x 256 + 96) runs narrow: an N = BN / 2 MMA over
+// the first BN / 2 rows of B, so the tensor cores skip the empty half. In a
+// CTA pair each CTA then supplies BN / 4 rows of B (its half of the narrow N).
+// SwiGLU tiles (gate and up halves of one B tile) never run narrow.
+__device__ __forceinline__ bool narrow_tile(const GemmParams& p, const GroupArgs& ga, int n0) {
+  return p.epi != tpi::EPI_SWIGLU && ga.N - n0 <= BN / 2;
+}
+
 // ------------------------------------------------------------- epilogue math
 __device__ __forceinline__ void store_row_chunk_bf16(void* base, int64_t ld, int row, int col0,
                                                      int N, const float (&v)[32]) {
@@ -156,7 +165,7 @@ __device__ __forceinline__ void load_row_chunk_bf16(const void* base, int64_t ld
 
 // Columns [half * BN/2, (half + 1) * BN/2) of the accumulator row this thread owns.
 __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t taddr, int row,
-                              int n0, int half) {
+                              int n0, int half, bool narrow) {
   const bool row_ok = row < ga.M;
   if (p.epi == tpi::EPI_SWIGLU) {
     // Accumulator columns [0,128) = gate units n0.., [128,256) = the same up units;
@@ -181,8 +190,9 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
     }
     return;
   }
+  const int cpw = narrow ? BN / 128 : BN / 64;  // 32-column chunks per warp half
 #pragma unroll 1
-  for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+  for (int c = half * cpw; c < (half + 1) * cpw; ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
     tc_wait_ld();
@@ -329,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const GroupArgs& ga = p.g[g];
       const int m0 = mt * C::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
-      const int nb0 = n0 + static_cast<int>(rank) * C::B_ROWS;      // this CTA's B rows
+      // this CTA's B rows (in a narrow tile of a pair, each CTA's first BN / 4)
+      const int nb0 = n0 + static_cast<int>(rank) * (narrow_tile(p, ga, n0) ? BN / (2 * PAIR) : C::B_ROWS);
       const int nseg = p.kcat ? p.kcat : 1;
       for (int sg = 0; sg < nseg && ok; ++sg) {
         const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
@@ -401,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
           mbar_wait(&full[s], static_cast<uint32_t>(last_parity[s]), abort_flag, p.status);
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_bf16(C::TILE_M, BN, p.a_mn != 0, p.b_mn != 0);
+    const uint32_t idesc_full = idesc_bf16(C::TILE_M, BN, p.a_mn != 0, p.b_mn != 0);
+    const uint32_t idesc_narrow = idesc_bf16(C::TILE_M, BN / 2, p.a_mn != 0, p.b_mn != 0);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -410,6 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
+      const uint32_t idesc =
+          narrow_tile(p, p.g[g], nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN)) ? idesc_narrow : idesc_full;
       int num_kb = p.g[g].num_kb;
       if (p.kcat) {
         num_kb = 0;
@@ -474,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_tile(p, ga, taddr, row, n0, half);
+      epilogue_tile(p, ga, taddr, row, n0, half, narrow_tile(p, ga, n0));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
