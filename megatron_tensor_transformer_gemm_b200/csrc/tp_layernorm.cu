@@ -372,6 +372,31 @@ __device__ __forceinline__ void store_row(const MutPtrArray& y, int p, int64_t r
   tpd::bulk_commit();
 }
 
+// Sum of a float pair over the CTA with one barrier, which also carries every
+// thread's wait result (false for all if any thread's ok is false). The
+// caller's previous barrier (end of the previous row) keeps red from being
+// overwritten while still read.
+template <int THREADS>
+__device__ __forceinline__ bool block_sum2_ok(float2& v, bool ok, float2* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+  }
+  constexpr int W = THREADS / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  if (!__syncthreads_and(ok)) return false;
+  float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    s.x += red[w].x;
+    s.y += red[w].y;
+  }
+  v = s;
+  return true;
+}
+
 template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
 __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
@@ -381,7 +406,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
   extern __shared__ __align__(128) uint8_t sbuf[];
   __shared__ uint64_t bar[STAGES];
   __shared__ int abort_flag;
-  __shared__ float red[THREADS / 32];
+  __shared__ float2 red[THREADS / 32];
   const uint32_t shard_bytes = static_cast<uint32_t>(hs * sizeof(T));
   const size_t stage_bytes = static_cast<size_t>(h) * sizeof(T);
   const int vpr = static_cast<int>(h / V);
@@ -413,8 +438,9 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     const int64_t r = G0 + k * GS;
     if (r >= rows) break;
     const int st = static_cast<int>(k % STAGES);
+    // a thread whose wait gave up computes on an unfinished stage; the sum's
+    // barrier then stops every thread before anything is written
     const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
-    if (!__syncthreads_and(ok)) break;
     const uint4* row = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes);
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
@@ -430,13 +456,8 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
         }
       }
     }
-    float2 tot;
-    if (RMS) {
-      tot = make_float2(0.f, block_sum<THREADS>(s2, red));
-    } else {
-      tot = make_float2(block_sum<THREADS>(s1, red), 0.f);
-      tot.y = block_sum<THREADS>(s2, red);
-    }
+    float2 tot = make_float2(s1, s2);
+    if (!block_sum2_ok<THREADS>(tot, ok, red)) break;
     const float mean = RMS ? 0.f : tot.x / static_cast<float>(h);
     const float var = RMS ? tot.y / static_cast<float>(h)
                           : fmaxf(tot.y / static_cast<float>(h) - mean * mean, 0.f);
@@ -445,7 +466,6 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
     for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * THREADS;
       if (c < vpr) {
-        const int sh = c / vps, lc = c - sh * vps;
         float x[V], g[V], bb[V], o[V];
         LnVec<T>::unpack(row[c], x);
         LnVec<T>::unpack(gp[i], g);
@@ -483,27 +503,6 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
   }
 }
 
-// Sum of a float pair over the CTA, same result in every thread.
-template <int THREADS>
-__device__ __forceinline__ float2 block_sum2(float2 v, float2* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
-    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
-  }
-  constexpr int W = THREADS / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();  // red may still be read by the previous row
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float2 s = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int w = 0; w < W; ++w) {
-    s.x += red[w].x;
-    s.y += red[w].y;
-  }
-  return s;
-}
 
 // Backward of a hidden-sharded norm in one pass over x and dy, staged like
 // the forward (a stage holds a row of x and the same row of dy). Thread tid
@@ -557,8 +556,9 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     if (r >= rows) break;
     const int st = static_cast<int>(k % STAGES);
     const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+    // a thread whose wait gave up computes on an unfinished stage; the sum's
+    // barrier then stops every thread before anything is written
     const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
-    if (!__syncthreads_and(ok)) break;
     const uint4* xrow = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes);
     const uint4* drow = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes + row_bytes);
     float2 acc = make_float2(0.f, 0.f);  // (sum g dy, sum g dy xhat) of this thread's columns
@@ -581,13 +581,13 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
         }
       }
     }
-    const float2 tot = block_sum2<THREADS>(acc, red);
+    float2 tot = acc;
+    if (!block_sum2_ok<THREADS>(tot, ok, red)) break;
     const float m1 = RMS ? 0.f : tot.x * inv_h, m2 = tot.y * inv_h;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * THREADS;
       if (c < vpr) {
-        const int sh = c / vps, lc = c - sh * vps;
         float x[V], d[V], g[V], o[V];
         LnVec<T>::unpack(xrow[c], x);
         LnVec<T>::unpack(drow[c], d);
