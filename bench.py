@@ -603,7 +603,7 @@ def run_hbm(args, world, rank, local):
     g = torch.Generator(device="cpu").manual_seed(1000 + rank)
     kernels = []   # (name, fn, algorithmic bytes per launch)
     if args.workload == "vocab":
-        T, V, h, p = 32768, 32000, 4096, 8
+        T, V, h, p = args.tokens, 32000, 4096, 8
         plan = tp.Plan(h, 0, 0, p, "bf16", "none")
         Vp = plan.set_vocab(V)
         Vs = Vp // p
@@ -621,9 +621,9 @@ def run_hbm(args, world, rank, local):
             ("embed_fwd_kernel", lambda: plan.embedding_fwd(T, ids, E, Y), T * h * 2 * 2 + T * 4),
             ("embed_bwd_kernel", lambda: plan.embedding_bwd(T, ids, dY, dE), T * h * 2 + Vp * h * 2 + T * 4),
         ]
-        name = "vocab-parallel embedding + cross-entropy: vocab 32000 (padded to a multiple of 8p), hidden 4096, tokens 8x4096, p=8"
+        name = f"vocab-parallel embedding + cross-entropy: vocab 32000 (padded to a multiple of 8p), hidden 4096, tokens {T}, p=8"
     else:
-        T, h, p = 32768, 8192, 8
+        T, h, p = args.tokens, 8192, 8
         plan = tp.Plan(h, 0, 0, p, "bf16", "none")
         hs = h // p
         X = [torch.randn(T, hs, generator=g).to(torch.bfloat16).to(dev) for _ in range(p)]
@@ -646,7 +646,7 @@ def run_hbm(args, world, rank, local):
             ("norm_hsh_bwd (layer)", lambda: plan.norm_sharded_bwd("layer", T, X, gam, dYn, mean, rstd, dXn, dg, db),
              T * h * 2 * 3 + T * 8),
         ]
-        name = "hidden-sharded RMSNorm + LayerNorm fwd+bwd: hidden 8192 over p=8, tokens 8x4096"
+        name = f"hidden-sharded RMSNorm + LayerNorm fwd+bwd: hidden 8192 over p=8, tokens {T}"
 
     def step():
         for _, fn, _ in kernels:

@@ -54,12 +54,11 @@ __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ Ptr
 //   scatter  each token's slot = its run start + the number of earlier tokens
 //            of its block in the same bucket, so every bucket lists its tokens
 //            in token order;
-//   accum    one CTA per (bucket, 512-column tile) sums the listed dY rows in
-//            that order in fp32 and writes its 16 rows of dE (zeros if none).
+//   accum    one CTA per (bucket, 1024-column slice), one warp per vocab row:
+//            each warp sums its row's listed dY rows in that order in fp32
+//            registers and writes the row of dE (zeros if none).
 // No atomics touch the sums, so the result is deterministic.
 constexpr int kEmbRows = 16;    // vocab ids per bucket
-constexpr int kEmbCols = 512;   // columns per accumulating CTA (4 per thread)
-constexpr int kEmbThreads = 128;
 constexpr int kTokBlock = 1024; // tokens per count / scatter CTA
 constexpr int kEmbMaxBuckets = 12288;  // 48 KB of shared counters (padded vocab <= 196608)
 constexpr int kListChunk = 512;
@@ -93,7 +92,7 @@ __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
   const int64_t hi = lo + C < n ? lo + C : n;
   const int64_t hv = lo + (hi - lo) / 4 * 4;  // [lo, hv) as int4
   int sum = 0;
-#pragma unroll 4
+#pragma unroll 16
   for (int64_t i = lo; i < hv; i += 4) {
     const int4 v = *reinterpret_cast<const int4*>(a + i);
     sum += v.x + v.y + v.z + v.w;
@@ -119,7 +118,7 @@ __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
   }
   __syncthreads();
   int run = (warp > 0 ? wsum[warp - 1] : 0) + incl - sum;
-#pragma unroll 4
+#pragma unroll 16
   for (int64_t i = lo; i < hv; i += 4) {
     int4 v = *reinterpret_cast<const int4*>(a + i);
     const int4 o = make_int4(run, run + v.x, run + v.x + v.y, run + v.x + v.y + v.z);
@@ -164,97 +163,6 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* i
         make_int2(static_cast<int>(t), id - b * kEmbRows);
 }
 
-// Four consecutive columns of dY row t as floats.
-template <typename T>
-__device__ __forceinline__ float4 load4(const T* dY, int64_t off) {
-  if constexpr (sizeof(T) == 2) {
-    const uint2 u = *reinterpret_cast<const uint2*>(dY + off);
-    const float2 a = tpd::unpack_bf16x2(u.x), b = tpd::unpack_bf16x2(u.y);
-    return make_float4(a.x, a.y, b.x, b.y);
-  } else {
-    return *reinterpret_cast<const float4*>(dY + off);
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kEmbThreads) emb_bucket_accum(
-    const int2* sorted, const int* off, int nb, int nblk, const T* dY, int64_t h, int64_t Vs,
-    int64_t Vp, const __grid_constant__ MutPtrArray dE) {
-  extern __shared__ float4 acc[];  // [kEmbRows][kEmbCols / 4]; thread tid owns columns 4 tid .. 4 tid + 3
-  __shared__ int ltok[kListChunk];
-  __shared__ int lrow[kListChunk];
-  constexpr int CV = kEmbCols / 4;  // float4 per accumulator row
-  const int b = blockIdx.x;
-  const int64_t v0 = static_cast<int64_t>(b) * kEmbRows;
-  const int tid = threadIdx.x;
-  const int64_t col = static_cast<int64_t>(blockIdx.y) * kEmbCols + 4 * tid;
-  const bool col_ok = col < h;
-#pragma unroll
-  for (int r = 0; r < kEmbRows; ++r) acc[r * CV + tid] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int start = off[static_cast<int64_t>(b) * nblk];
-  const int end = off[static_cast<int64_t>(b + 1) * nblk];  // off[nb * nblk] is the total
-  for (int c0 = start; c0 < end; c0 += kListChunk) {
-    const int n = end - c0 < kListChunk ? end - c0 : kListChunk;
-    __syncthreads();  // the previous chunk's list is consumed
-    for (int k = tid; k < n; k += kEmbThreads) {
-      const int2 e = sorted[c0 + k];
-      ltok[k] = e.x;
-      lrow[k] = e.y;
-    }
-    __syncthreads();
-    if (!col_ok) continue;
-    int k = 0;
-    for (; k + 16 <= n; k += 16) {  // sixteen independent row loads in flight, summed in list order
-      float4 f[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) f[u] = load4(dY, static_cast<int64_t>(ltok[k + u]) * h + col);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        float4& a4 = acc[lrow[k + u] * CV + tid];
-        a4.x += f[u].x;
-        a4.y += f[u].y;
-        a4.z += f[u].z;
-        a4.w += f[u].w;
-      }
-    }
-    for (; k < n; ++k) {
-      const float4 f = load4(dY, static_cast<int64_t>(ltok[k]) * h + col);
-      float4& a4 = acc[lrow[k] * CV + tid];
-      a4.x += f.x;
-      a4.y += f.y;
-      a4.z += f.z;
-      a4.w += f.w;
-    }
-  }
-  if (!col_ok) return;
-  // Write the bucket's rows to their shards (every padded row: zeros if unused).
-  for (int r = 0; r < kEmbRows; ++r) {
-    const int64_t v = v0 + r;
-    if (v >= Vp) break;
-    const int s = static_cast<int>(v / Vs);
-    T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + col;
-    const float4 a4 = acc[r * CV + tid];
-    if constexpr (sizeof(T) == 2) {
-      *reinterpret_cast<uint2*>(dst) = make_uint2(tpd::pack_bf16x2(a4.x, a4.y), tpd::pack_bf16x2(a4.z, a4.w));
-    } else {
-      *reinterpret_cast<float4*>(dst) = a4;
-    }
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ float ld_logit(const void* p, int64_t i) {
-  if constexpr (sizeof(T) == 2) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
-  else return static_cast<const float*>(p)[i];
-}
-
-// 2^x by the hardware approximation (denormal results flush to 0).
-__device__ __forceinline__ float ex2f_fast(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // 16 bytes as floats (8 bf16, widened exactly by shifts, or 4 fp32) and back.
 template <typename T>
 __device__ __forceinline__ void unpack16(const uint4 u, float (&x)[16 / sizeof(T)]) {
@@ -277,6 +185,82 @@ __device__ __forceinline__ uint4 pack16(const float (&x)[16 / sizeof(T)]) {
     return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
                       __float_as_uint(x[3]));
   }
+}
+
+// One CTA per (bucket of 16 vocab rows, 1024-column slice): warp w owns vocab
+// row v0 + w; every lane owns 32 consecutive columns of the slice and sums,
+// in registers, the dY rows of the tokens listed for its row, in list (token)
+// order; then the warp writes its row (zeros if no token uses it).
+constexpr int kAccCols = 1024;                 // columns per CTA
+constexpr int kAccThreads = 32 * kEmbRows;     // one warp per vocab row of the bucket
+
+template <typename T>
+__global__ void __launch_bounds__(kAccThreads) emb_bucket_accum(
+    const int2* sorted, const int* off, int nb, int nblk, const T* dY, int64_t h, int64_t Vs,
+    int64_t Vp, const __grid_constant__ MutPtrArray dE) {
+  constexpr int E = 16 / sizeof(T);   // elements per 16-byte vector
+  constexpr int NV = 32 / E;          // 16-byte vectors per lane (32 columns)
+  __shared__ int ltok[kListChunk];
+  __shared__ int lrow[kListChunk];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kAccCols + lane * 32;  // this lane's columns
+  float acc[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  const int start = off[static_cast<int64_t>(b) * nblk];
+  const int end = off[static_cast<int64_t>(b + 1) * nblk];  // off[nb * nblk] is the total
+  for (int k0 = start; k0 < end; k0 += kListChunk) {
+    const int n = end - k0 < kListChunk ? end - k0 : kListChunk;
+    __syncthreads();  // the previous chunk's list is consumed
+    for (int k = threadIdx.x; k < n; k += kAccThreads) {
+      const int2 e = sorted[k0 + k];
+      ltok[k] = e.x;
+      lrow[k] = e.y;
+    }
+    __syncthreads();
+    for (int k = 0; k < n; ++k) {
+      if (lrow[k] != warp) continue;  // warp-uniform
+      const T* src = dY + static_cast<int64_t>(ltok[k]) * h + c0;
+      uint4 u[NV];
+#pragma unroll
+      for (int q = 0; q < NV; ++q)
+        u[q] = c0 + q * E < h ? reinterpret_cast<const uint4*>(src)[q] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        float x[E];
+        unpack16<T>(u[q], x);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[q * E + e] += x[e];
+      }
+    }
+  }
+  const int64_t v = static_cast<int64_t>(b) * kEmbRows + warp;
+  if (v >= Vp) return;
+  const int s = static_cast<int>(v / Vs);
+  T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + c0;
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    if (c0 + q * E < h) {
+      float x[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = acc[q * E + e];
+      reinterpret_cast<uint4*>(dst)[q] = pack16<T>(x);
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_logit(const void* p, int64_t i) {
+  if constexpr (sizeof(T) == 2) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+  else return static_cast<const float*>(p)[i];
+}
+
+// 2^x by the hardware approximation (denormal results flush to 0).
+__device__ __forceinline__ float ex2f_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Running (max, sum of exp2) pair in the log2 domain: the pair (m, s) stands
@@ -719,17 +703,6 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
   int* cnt = static_cast<int*>(ws);
   const int64_t ncnt = static_cast<int64_t>(nb) * nblk + 1;
   int2* sorted = reinterpret_cast<int2*>(cnt + ncnt + (ncnt & 1));
-  const int smem = kEmbRows * kEmbCols * 4;
-  static bool attr[2] = {false, false};
-  const int k = dt == TP_BF16 ? 0 : 1;
-  if (!attr[k]) {
-    cudaError_t e = dt == TP_BF16
-        ? cudaFuncSetAttribute(emb_bucket_accum<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-        : cudaFuncSetAttribute(emb_bucket_accum<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    tp_status s = cuda_status(e, "cudaFuncSetAttribute(embedding_bwd)");
-    if (s != TP_OK) return s;
-    attr[k] = true;
-  }
   if (T > 0) {
     emb_bucket_count<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt);
     tp_status s = after_launch("embedding_bwd count");
@@ -743,13 +716,13 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
     s = after_launch("embedding_bwd scatter");
     if (s != TP_OK) return s;
   }
-  dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((h + kEmbCols - 1) / kEmbCols));
+  dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((h + kAccCols - 1) / kAccCols));
   if (dt == TP_BF16)
-    emb_bucket_accum<__nv_bfloat16><<<grid, kEmbThreads, smem, st>>>(
+    emb_bucket_accum<__nv_bfloat16><<<grid, kAccThreads, 0, st>>>(
         sorted, cnt, nb, nblk, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
   else
-    emb_bucket_accum<float><<<grid, kEmbThreads, smem, st>>>(sorted, cnt, nb, nblk,
-                                                            static_cast<const float*>(dY), h, Vs, Vp, dE);
+    emb_bucket_accum<float><<<grid, kAccThreads, 0, st>>>(sorted, cnt, nb, nblk,
+                                                         static_cast<const float*>(dY), h, Vs, Vp, dE);
   return after_launch("embedding_bwd accumulate");
 }
 
