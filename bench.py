@@ -466,7 +466,7 @@ def run_other(args, world, rank, local):
     if args.workload == "attn":
         b, s, h, H, p = 2, 4096, 4096, 32, 8
         a = tp_synth.draw_attn_block(b, s, h, torch.bfloat16, seed=rank)
-        blk = TPAttention(h, H, p, dev)
+        blk = TPAttention(h, H, p, dev, fused=args.variant == "fused")
         blk.load_weights(a.Wqkv.to(dev), a.Wo.to(dev))
         X = a.X.to(dev)
         flops = blk.flops_fwd(b, s)
@@ -495,7 +495,7 @@ def run_other(args, world, rank, local):
         X, layers, dY = tp_synth.draw_block_stack(L, b, s_, h, f, torch.bfloat16, seed=rank)
         lays = []
         for prm in layers:
-            lay = TPLayer(h, f, H, p, dev)
+            lay = TPLayer(h, f, H, p, dev, fused=args.variant == "fused")
             lay.load(type(prm)(**{k: getattr(prm, k).to(dev) for k in prm.__dataclass_fields__}))
             lays.append(lay)
         Xd, dYd = X.to(dev), dY.to(dev)

@@ -300,9 +300,14 @@ class SPMLP:
 class TPAttention:
     """Attention sublayer split by whole heads over p shards on one GPU:
     QKV column GEMM -> causal attention on local heads -> out-projection row
-    GEMM partials -> reduce (+bias once, +residual).   (TP walkthrough §3.1)"""
+    GEMM partials -> reduce (+bias once, +residual).   (TP walkthrough §3.1)
+    fused: the out-projection (forward) and the QKV dX (backward) sum the
+    shards in the GEMM accumulator (tp_row_fwd_reduce / tp_column_bwd_reduce)
+    instead of writing p partials and reducing them."""
 
-    def __init__(self, hidden: int, heads: int, p: int, device="cuda", bias: bool = False):
+    def __init__(self, hidden: int, heads: int, p: int, device="cuda", bias: bool = False,
+                 fused: bool = False):
+        self.fused = fused
         self.h, self.H, self.p = hidden, heads, p
         self.plan = Plan(hidden, 0, heads, p, "bf16", "none")
         self.device = torch.device(device)
@@ -333,7 +338,7 @@ class TPAttention:
         self.QKV = [_empty((T, n), torch.bfloat16, dev) for _ in range(p)]
         self.O = [_empty((T, self.h // p), torch.bfloat16, dev) for _ in range(p)]
         self.LSE = [_empty((batch, self.hl, seq), torch.float32, dev) for _ in range(p)]
-        self.P = [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
+        self.P = None if self.fused else [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
         self.Y = _empty((T, self.h), torch.bfloat16, dev)
 
     def forward(self, X: torch.Tensor, batch: int, seq: int, residual=None, out=None):
@@ -343,9 +348,12 @@ class TPAttention:
         self.X = X
         pl.column_fwd("qkv", T, X, self.Wqkv, self.bqkv, None, self.QKV)
         pl.attention_fwd(batch, seq, self.QKV, self.O, self.LSE)
-        pl.row_fwd_partial("outproj", T, self.O, self.Wo, self.P)
         Y = self.Y if out is None else out
-        pl.reduce_partials(T, self.P, self.bo, residual, Y)
+        if self.fused:
+            pl.row_fwd_reduce("outproj", T, self.O, self.Wo, self.bo, residual, Y)
+        else:
+            pl.row_fwd_partial("outproj", T, self.O, self.Wo, self.P)
+            pl.reduce_partials(T, self.P, self.bo, residual, Y)
         return Y
 
     def alloc_bwd(self):
@@ -354,7 +362,7 @@ class TPAttention:
         T, p, dev = self.QKV[0].shape[0], self.p, self.device
         self.dO = [_empty((T, self.h // p), torch.bfloat16, dev) for _ in range(p)]
         self.dQKV = [torch.empty_like(x) for x in self.QKV]
-        self.dXp = [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
+        self.dXp = None if self.fused else [_empty((T, self.h), torch.bfloat16, dev) for _ in range(p)]
         self.dX = _empty((T, self.h), torch.bfloat16, dev)
         self.dWqkv = [torch.empty_like(w) for w in self.Wqkv]
         self.dWo = [torch.empty_like(w) for w in self.Wo]
@@ -369,9 +377,12 @@ class TPAttention:
         pl = self.plan
         pl.row_bwd("outproj", T, dY, self.O, self.Wo, None, self.dO, self.dWo, self.dbo)
         pl.attention_bwd(batch, seq, self.QKV, self.O, self.dO, self.LSE, self.dQKV)
-        pl.column_bwd("qkv", T, self.X, self.dQKV, self.Wqkv, self.dWqkv, self.dbqkv, self.dXp)
         dX = self.dX if out is None else out
-        pl.reduce_partials(T, self.dXp, None, None, dX)
+        if self.fused:
+            pl.column_bwd_reduce("qkv", T, self.X, self.dQKV, self.Wqkv, self.dWqkv, self.dbqkv, dX)
+        else:
+            pl.column_bwd("qkv", T, self.X, self.dQKV, self.Wqkv, self.dWqkv, self.dbqkv, self.dXp)
+            pl.reduce_partials(T, self.dXp, None, None, dX)
         return dX
 
     def flops_fwd(self, batch: int, seq: int, causal: bool = True) -> float:
@@ -387,10 +398,11 @@ class TPLayer:
     shards on one GPU: x1 = x + Attn(LN1(x)); y = x1 + MLP(LN2(x1)).
     Biases on every projection (TP-basics' row bias enters once, in the reduce)."""
 
-    def __init__(self, hidden: int, ffn: int, heads: int, p: int, device="cuda"):
+    def __init__(self, hidden: int, ffn: int, heads: int, p: int, device="cuda", fused: bool = True):
+        """fused: both sublayers sum their shards inside the GEMMs (no partials)."""
         self.h = hidden
-        self.attn = TPAttention(hidden, heads, p, device, bias=True)
-        self.mlp = TPMLP(hidden, ffn, p, "gelu", "bf16", device, bias=True)
+        self.attn = TPAttention(hidden, heads, p, device, bias=True, fused=fused)
+        self.mlp = TPMLP(hidden, ffn, p, "gelu", "bf16", device, bias=True, fused=fused)
         self.ln = Plan(hidden, 0, 0, 1, "bf16", "none")  # LayerNorm / elementwise calls
         self.device = torch.device(device)
         dev = self.device

@@ -65,13 +65,15 @@ def test_attention_fwd_growing_scores_rescale(d):
     assert tp.device_status() == "TP_OK"
 
 
-def test_attention_block_full_size_sampled():
+@pytest.mark.parametrize("fused", [False, True])
+def test_attention_block_full_size_sampled(fused):
     """hidden 4096, 32 heads x 128, seq 4096, batch 2, p 8 (4 heads per shard),
-    causal; QKV -> attention -> out-projection partials -> reduce + residual."""
+    causal; QKV -> attention -> out-projection partials -> reduce + residual
+    (fused: the out-projection sums the shards in its accumulator)."""
     from megatron_tensor_transformer_gemm_b200.block import TPAttention
     batch, seq, h, H, p = 2, 4096, 4096, 32, 8
     a = tp_synth.draw_attn_block(batch, seq, h, torch.bfloat16, seed=0)
-    blk = TPAttention(h, H, p)
+    blk = TPAttention(h, H, p, fused=fused)
     blk.load_weights(dev(a.Wqkv), dev(a.Wo))
     X = dev(a.X)
     Y = blk.forward(X, batch, seq, residual=X)

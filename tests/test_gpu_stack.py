@@ -30,9 +30,9 @@ def _params64(prm):
     return {k: O.f64(getattr(prm, k)) for k in prm.__dataclass_fields__}
 
 
-def _gpu_layer(prm, p):
+def _gpu_layer(prm, p, fused=True):
     from megatron_tensor_transformer_gemm_b200.block import TPLayer
-    lay = TPLayer(H_, F_, HEADS, p)
+    lay = TPLayer(H_, F_, HEADS, p, fused=fused)
     lay.load(type(prm)(**{k: dev(getattr(prm, k)) for k in prm.__dataclass_fields__}))
     return lay
 
@@ -70,8 +70,8 @@ def _grad_errors(lay, gr, p):
     return errs
 
 
-@pytest.mark.parametrize("p", [1, 2, 4])
-def test_every_layer_fwd_bwd_from_independent_inputs(p):
+@pytest.mark.parametrize("p,fused", [(1, True), (2, True), (4, True), (2, False), (4, False)])
+def test_every_layer_fwd_bwd_from_independent_inputs(p, fused):
     _, layers, _ = tp_synth.draw_block_stack(L, BATCH, SEQ, H_, F_, torch.bfloat16, seed=0,
                                              ln_affine_random=True)
     report, worst = [], 0.0
@@ -79,7 +79,7 @@ def test_every_layer_fwd_bwd_from_independent_inputs(p):
         g = torch.Generator().manual_seed(1000 + l_)
         x = torch.randn(BATCH * SEQ, H_, generator=g).to(torch.bfloat16)
         dy = torch.randn(BATCH * SEQ, H_, generator=g).to(torch.bfloat16)
-        lay = _gpu_layer(prm, p)
+        lay = _gpu_layer(prm, p, fused)
         y = lay.forward(dev(x), BATCH, SEQ)
         dx = lay.backward(dev(dy), BATCH, SEQ)
         P = _params64(prm)
