@@ -494,24 +494,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
   }
 }
 
-template <int D, int ST>
+// STK / STQ: stages of the streamed Q, dO blocks (dK/dV kernel) and K, V
+// blocks (dQ kernel); as many as fit the 227 KB of shared memory.
+template <int D, int STK, int STQ>
 tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
+  static_assert(DkdvSmem<D, STK>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448,
+                "shared memory of the backward kernels");
   static bool attr = false;
   if (!attr) {
     tp_status s = tpi::cuda_status(
-        cudaFuncSetAttribute(attn_bwd_dkdv<D, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DkdvSmem<D, ST>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
+        cudaFuncSetAttribute(attn_bwd_dkdv<D, STK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvSmem<D, STK>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
     if (s != TP_OK) return s;
-    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq<D, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              DqSmem<D, ST>::TOTAL), "cudaFuncSetAttribute(attention dq)");
+    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq<D, STQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              DqSmem<D, STQ>::TOTAL), "cudaFuncSetAttribute(attention dq)");
     if (s != TP_OK) return s;
     attr = true;
   }
   const int per = prm.p * prm.batch * prm.hl;
-  attn_bwd_dkdv<D, ST><<<prm.nkv * per, kThreads, DkdvSmem<D, ST>::TOTAL, st>>>(prm);
+  attn_bwd_dkdv<D, STK><<<prm.nkv * per, kThreads, DkdvSmem<D, STK>::TOTAL, st>>>(prm);
   tp_status s = tpi::after_launch("attention_bwd dK/dV (tcgen05)");
   if (s != TP_OK) return s;
-  attn_bwd_dq<D, ST><<<prm.nq * per, kThreads, DqSmem<D, ST>::TOTAL, st>>>(prm);
+  attn_bwd_dq<D, STQ><<<prm.nq * per, kThreads, DqSmem<D, STQ>::TOTAL, st>>>(prm);
   return tpi::after_launch("attention_bwd dQ (tcgen05)");
 }
 
@@ -564,8 +568,8 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   attn_bwd_prep<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dO, dvec, p, batch, seq, hl, d);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;
-  if (d == 64) return launch_bwd_d<64, 2>(prm, st);
-  if (d == 128) return launch_bwd_d<128, 1>(prm, st);
+  if (d == 64) return launch_bwd_d<64, 2, 2>(prm, st);
+  if (d == 128) return launch_bwd_d<128, 1, 2>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
 }
 
