@@ -588,7 +588,8 @@ def run_other(args, world, rank, local):
 
 def run_hbm(args, world, rank, local):
     """Device-timed HBM throughput of the memory-bound rows, each kernel timed
-    on its own over the same buffers (algorithmic bytes / event time):
+    on its own over the same buffers (algorithmic bytes / event time; sp_hbm:
+    the sequence-parallel collectives and LayerNorm of the SP config):
     vocab -- embedding lookup, vocab-parallel cross-entropy (loss + dlogits,
     in place) and embedding gradient; Llama-7B shapes: vocab 32000, hidden
     4096, tokens 8x4096, p 8.
@@ -622,6 +623,42 @@ def run_hbm(args, world, rank, local):
             ("embed_bwd_kernel", lambda: plan.embedding_bwd(T, ids, dY, dE), T * h * 2 + Vp * h * 2 + T * 4),
         ]
         name = f"vocab-parallel embedding + cross-entropy: vocab 32000 (padded to a multiple of 8p), hidden 4096, tokens {T}, p=8"
+    elif args.workload == "sp_hbm":
+        # Megatron-SP's memory-bound steps at the SP config's sizes (seq 8192,
+        # hidden 8192, p 8): S1 LayerNorm fused with the sequence all-gather,
+        # S4' reduce-scatter of the row partials, S9 all-gather of dY, S8's
+        # reduce-scatter of the dX partials, and a LayerNorm backward over all
+        # rows (every buffer set larger than L2).
+        T, h, p = min(args.tokens, 8192), 8192, 8
+        t = T // p
+        plan = tp.Plan(h, 0, 0, p, "bf16", "none")
+        xs = [torch.randn(t, h, generator=g).to(torch.bfloat16).to(dev) for _ in range(p)]
+        gam = (1 + 0.1 * torch.randn(h, generator=g)).to(torch.bfloat16).to(dev)
+        bet = (0.1 * torch.randn(h, generator=g)).to(torch.bfloat16).to(dev)
+        U = torch.empty(T, h, dtype=torch.bfloat16, device=dev)
+        mean = torch.empty(T, dtype=torch.float32, device=dev)
+        rstd = torch.empty(T, dtype=torch.float32, device=dev)
+        parts = [torch.randn(T, h, generator=g).to(torch.bfloat16).to(dev) for _ in range(p)]
+        outs = [torch.empty(t, h, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+        full = torch.empty(T, h, dtype=torch.bfloat16, device=dev)
+        dxf = torch.empty(T, h, dtype=torch.bfloat16, device=dev)
+        dgam = torch.empty(h, dtype=torch.float32, device=dev)
+        dbet = torch.empty(h, dtype=torch.float32, device=dev)
+        plan.layernorm_all_gather_seq(T, xs, gam, bet, U, mean, rstd)
+        kernels = [
+            ("ln_fwd_kernel (LayerNorm + sequence all-gather)",
+             lambda: plan.layernorm_all_gather_seq(T, xs, gam, bet, U, mean, rstd), T * h * 2 * 2 + T * 8),
+            ("reduce_kernel (reduce-scatter of the row partials)",
+             lambda: plan.reduce_scatter_seq(T, parts, None, None, outs), p * T * h * 2 + T * h * 2),
+            ("gather_kernel (all-gather of dY)",
+             lambda: plan.reduce_scatter_seq_bwd(T, outs, full), T * h * 2 * 2),
+            ("reduce_kernel (reduce-scatter of the dX partials)",
+             lambda: plan.all_gather_seq_bwd(T, parts, outs), p * T * h * 2 + T * h * 2),
+            ("ln_bwd (all T rows: dx + dgamma, dbeta)",
+             lambda: plan.layernorm_bwd(T, full, gam, U, mean, rstd, dxf, dgam, dbet),
+             T * h * 2 * 3 + T * 8),
+        ]
+        name = f"Megatron-SP memory-bound steps: seq {T}, hidden 8192, p=8 (LN+AG, RS, AG, RS, LN bwd)"
     else:
         T, h, p = args.tokens, 8192, 8
         plan = tp.Plan(h, 0, 0, p, "bf16", "none")
@@ -715,7 +752,8 @@ def main():
                     help="sum over shards inside the GEMMs (fused), via p partials + reduce, "
                          "or partials with each token block's reduce overlapped with the next "
                          "block's GEMM (overlap)")
-    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm"], default="mlp7b",
+    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm", "sp_hbm"],
+                    default="mlp7b",
                     help="mlp7b (the metric's workload) or another config of the suite")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph (other workloads)")
@@ -729,7 +767,7 @@ def main():
     world, rank, local = dist_setup()
     if args.workload == "mlp7b":
         rc = run_ours(args, world, rank, local)
-    elif args.workload in ("vocab", "norm"):
+    elif args.workload in ("vocab", "norm", "sp_hbm"):
         rc = run_hbm(args, world, rank, local)
     else:
         rc = run_other(args, world, rank, local)

@@ -96,7 +96,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
                                   const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
                                   const MutPtrArray& db, int p, int64_t rows, int64_t h,
                                   const float* mean, const float* rstd, tp_dtype dt,
-                                  cudaStream_t st);
+                                  cudaStream_t st, int accumulate = 0);
 
 // Element-wise activation kernels for the fp32 path (tp_gemm_simt.cu).
 tp_status launch_act_fwd(tp_act act, const float* Z, int64_t T, int64_t nh, int64_t ldz, float* H,

@@ -280,6 +280,21 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
                                const float* mean, const float* rstd, void* dx, float* dgamma,
                                float* dbeta, int accumulate, int64_t rows, int64_t cols,
                                tp_dtype dt, cudaStream_t st) {
+  // The backward formula takes the saved mean and rstd, so a LayerNorm over the
+  // whole row is the hidden-sharded one with a single shard: its one-pass,
+  // staged kernel serves whenever the row fits it.
+  if (cols % 8 == 0 && cols <= (dt == TP_BF16 ? 16384 : 8192)) {
+    PtrArray X{}, G{}, DY{};
+    MutPtrArray DX{}, dg{}, db{};
+    X.p[0] = x;
+    G.p[0] = gamma;
+    DY.p[0] = dy;
+    DX.p[0] = dx;
+    dg.p[0] = dgamma;
+    db.p[0] = dbeta;
+    return launch_norm_sharded_bwd(plan, false, X, G, DY, DX, dg, db, 1, rows, cols, mean, rstd, dt, st,
+                                   accumulate);
+  }
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "LayerNorm row too long (%lld)", (long long)cols);
@@ -634,9 +649,11 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
   }
 }
 
+// dgamma[c] (and dbeta[c]) = the fixed-order sum over the CTAs' partials
+// (added to the existing value when accumulate is set).
 __global__ void norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
                                      const __grid_constant__ MutPtrArray dg,
-                                     const __grid_constant__ MutPtrArray db) {
+                                     const __grid_constant__ MutPtrArray db, int accumulate) {
   const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (c >= h) return;
   float sg = 0.f, sb = 0.f;
@@ -646,8 +663,12 @@ __global__ void norm_hsh_param_pass2(const float* part, int splits, int64_t hs, 
   }
   const int sh = static_cast<int>(c / hs);
   const int64_t lc = c - sh * hs;
-  static_cast<float*>(dg.p[sh])[lc] = sg;
-  if (db.p[sh]) static_cast<float*>(db.p[sh])[lc] = sb;
+  float* g = static_cast<float*>(dg.p[sh]) + lc;
+  *g = accumulate ? *g + sg : sg;
+  if (db.p[sh]) {
+    float* bp = static_cast<float*>(db.p[sh]) + lc;
+    *bp = accumulate ? *bp + sb : sb;
+  }
 }
 
 }  // namespace
@@ -729,7 +750,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
                                   const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
                                   const MutPtrArray& db, int p, int64_t rows, int64_t h,
                                   const float* mean, const float* rstd, tp_dtype dt,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, int accumulate) {
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = h / V, hs = h / p;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
@@ -776,7 +797,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
     if (s != TP_OK) return s;
   }
   norm_hsh_param_pass2<<<static_cast<unsigned>((h + 255) / 256), 256, 0, st>>>(
-      part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg, db);
+      part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg, db, accumulate);
   return after_launch("norm_sharded_bwd/param");
 }
 
