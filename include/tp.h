@@ -339,8 +339,9 @@ TP_API tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const vo
                                 void* const* dX_seq, void* stream);
 
 /* LayerNorm backward: dx [rows, hidden] (plan dtype); dgamma, dbeta [hidden]
- * fp32 (sums over the rows; when accumulate != 0 they are added to the
- * existing contents, so shards can be summed). mean/rstd from the forward. */
+ * fp32 (sums over the rows, deterministic; when accumulate != 0 they are
+ * added to the existing contents, so shards can be summed). mean/rstd from
+ * the forward. Uses the plan's device workspace for per-CTA partials. */
 TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
                            const void* dy, const float* mean, const float* rstd, void* dx,
                            float* dgamma, float* dbeta, int accumulate, void* stream);
