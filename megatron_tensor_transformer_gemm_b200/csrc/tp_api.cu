@@ -2,10 +2,13 @@
 // and dispatch to the kernels. Every check happens before any launch.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <new>
 
 #include "tp_internal.h"
@@ -41,6 +44,47 @@ tp_status cuda_status(cudaError_t e, const char* what) {
 tp_status after_launch(const char* what, int launches) {
   g_launches += static_cast<uint64_t>(launches);
   return cuda_status(cudaGetLastError(), what);
+}
+
+namespace {
+std::mutex g_occ_mu;
+std::map<std::tuple<int, const void*, int, int>, int> g_occ;  // (dev, kernel, threads, smem) -> CTAs per SM
+std::map<std::pair<int, const void*>, int> g_smem_limit;        // (dev, kernel) -> dynamic smem limit set
+int g_sms[kMaxDevices] = {};
+}  // namespace
+
+tp_status persistent_grid(const void* kernel, int threads, int smem, int64_t units, int64_t* grid) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  if (!g_sms[dev]) {
+    int n = 0;
+    tp_status s = cuda_status(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev),
+                              "cudaDeviceGetAttribute(SM count)");
+    if (s != TP_OK) return s;
+    g_sms[dev] = n > 0 ? n : 1;
+  }
+  const auto key = std::make_tuple(dev, kernel, threads, smem);
+  auto it = g_occ.find(key);
+  if (it == g_occ.end()) {
+    int& lim = g_smem_limit[std::make_pair(dev, kernel)];
+    if (smem > lim) {
+      tp_status s = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                                "cudaFuncSetAttribute(dynamic shared memory)");
+      if (s != TP_OK) return s;
+      lim = smem;
+    }
+    int per_sm = 0;
+    tp_status s = cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem),
+                              "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (s != TP_OK) return s;
+    it = g_occ.emplace(key, per_sm > 0 ? per_sm : 1).first;
+  }
+  *grid = std::max<int64_t>(1, std::min<int64_t>(units, static_cast<int64_t>(g_sms[dev]) * it->second));
+  return TP_OK;
 }
 
 tp_status device_status_word(unsigned** out) {

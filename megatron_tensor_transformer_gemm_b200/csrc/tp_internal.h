@@ -36,6 +36,13 @@ tp_status after_launch(const char* what, int launches = 1);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t dsize(tp_dtype t) { return t == TP_BF16 ? 2 : 4; }
 
+// Grid of a persistent kernel: min(units, SMs x resident CTAs of `kernel` at
+// `threads` and `smem` bytes of dynamic shared memory), at least 1. Raises the
+// kernel's dynamic shared-memory limit to `smem` when needed. Both the limit
+// and the occupancy are cached per device, kernel and size, so a repeated call
+// makes no driver query.
+tp_status persistent_grid(const void* kernel, int threads, int smem, int64_t units, int64_t* grid);
+
 // Device address of this device's status word (set by kernels on a timeout).
 tp_status device_status_word(unsigned** out);
 // Scratch of at least `bytes` on the current device, owned by the plan.

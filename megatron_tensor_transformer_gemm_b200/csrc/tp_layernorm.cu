@@ -65,55 +65,80 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
-// y row r = LN(x row r); x row r is row (r - j*rows_per_src) of src.p[j].
+// y row r = LN(x row r); x row r is row (r - j*rows_per_src) of src.p[j], so a
+// sequence all-gather is part of the load. One CTA per row, many resident per
+// SM: each row's chain (load, two sums, store) overlaps the other rows' loads.
+// The slice stays packed in registers; the mean and the biased variance about
+// it are two exact passes over those registers, each summed over the CTA with
+// one barrier (each sum has a buffer of its own, and a CTA takes one row).
 template <typename T, int THREADS>
 __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__ PtrArray src, int64_t rows_per_src,
                                                          int64_t cols, const T* gamma,
                                                          const T* beta, T* y, float* mean_out,
                                                          float* rstd_out) {
   constexpr int V = LnVec<T>::N;
-  __shared__ float red[THREADS / 32];
+  constexpr int W = THREADS / 32;
+  __shared__ float red1[W], red2[W];
   const int64_t r = blockIdx.x;
-  const int j = static_cast<int>(r / rows_per_src);
-  const T* x = static_cast<const T*>(src.p[j]) + (r - j * rows_per_src) * cols;
+  const int64_t j = r / rows_per_src;
+  const uint4* x = reinterpret_cast<const uint4*>(static_cast<const T*>(src.p[j]) + (r - j * rows_per_src) * cols);
   const int vpr = static_cast<int>(cols / V);
-  float v[kVptMax][V];
+  const float inv_h = 1.f / static_cast<float>(cols);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4 xr[kVptMax];
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
+    xr[i] = c < vpr ? __ldcs(x + c) : make_uint4(0, 0, 0, 0);  // read once: streaming
+  }
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
-      LnVec<T>::load(x + static_cast<int64_t>(c) * V, v[i]);
+    if (threadIdx.x + i * THREADS < vpr) {
+      float v[V];
+      LnVec<T>::unpack(xr[i], v);
 #pragma unroll
-      for (int k = 0; k < V; ++k) s += v[i][k];
+      for (int e = 0; e < V; ++e) s += v[e];
     }
   }
-  const float mean = block_sum<THREADS>(s, red) / static_cast<float>(cols);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red1[warp] = s;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < W; ++w) t += red1[w];
+  const float mean = t * inv_h;
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
+    if (threadIdx.x + i * THREADS < vpr) {
+      float v[V];
+      LnVec<T>::unpack(xr[i], v);
 #pragma unroll
-      for (int k = 0; k < V; ++k) {
-        const float d = v[i][k] - mean;
-        q += d * d;
-      }
+      for (int e = 0; e < V; ++e) q += (v[e] - mean) * (v[e] - mean);
     }
   }
-  const float var = block_sum<THREADS>(q, red) / static_cast<float>(cols);
-  const float rstd = rsqrtf(var + kEps);
-  T* yr = y + r * cols;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  if (lane == 0) red2[warp] = q;
+  __syncthreads();
+  float u = 0.f;
+#pragma unroll
+  for (int w = 0; w < W; ++w) u += red2[w];
+  const float rstd = rsqrtf(u * inv_h + kEps);
+  uint4* yr = reinterpret_cast<uint4*>(y + r * cols);
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
     const int c = threadIdx.x + i * THREADS;
     if (c < vpr) {
-      float g[V], b[V], o[V];
+      float v[V], g[V], b[V], o[V];
+      LnVec<T>::unpack(xr[i], v);
       LnVec<T>::load(gamma + static_cast<int64_t>(c) * V, g);
       LnVec<T>::load(beta + static_cast<int64_t>(c) * V, b);
 #pragma unroll
-      for (int k = 0; k < V; ++k) o[k] = (v[i][k] - mean) * rstd * g[k] + b[k];
-      LnVec<T>::store(yr + static_cast<int64_t>(c) * V, o);
+      for (int e = 0; e < V; ++e) o[e] = (v[e] - mean) * rstd * g[e] + b[e];
+      LnVec<T>::store(yr + c, o);
     }
   }
   if (threadIdx.x == 0) {
@@ -255,6 +280,7 @@ tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_sr
                                const void* gamma, const void* beta, void* y, float* mean,
                                float* rstd, tp_dtype dt, cudaStream_t st) {
   const int64_t rows = rows_per_src * n;
+  if (rows == 0) return TP_OK;
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "LayerNorm row too long (%lld)", (long long)cols);
@@ -412,115 +438,84 @@ __device__ __forceinline__ bool block_sum2_ok(float2& v, bool ok, float2* red) {
   return true;
 }
 
-template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
-__global__ void __launch_bounds__(THREADS) norm_hsh_fwd_kernel(
+// Forward of a hidden-sharded norm, one CTA per row: vector c of the row is
+// vector c - j*vps of shard j = c / vps. The slice stays packed in registers;
+// one barrier sums (sum x, sum x^2) over the CTA, the local sums of every shard
+// reduced in one step.
+template <typename T, int THREADS, bool RMS>
+__global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
-    const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int p, int vps,
-    int64_t hs, int64_t h, int64_t rows, float* mean_out, float* rstd_out, unsigned* status) {
+    const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int vps, int64_t h,
+    float* mean_out, float* rstd_out) {
   constexpr int V = LnVec<T>::N;
-  extern __shared__ __align__(128) uint8_t sbuf[];
-  __shared__ uint64_t bar[STAGES];
-  __shared__ int abort_flag;
-  __shared__ float2 red[THREADS / 32];
-  const uint32_t shard_bytes = static_cast<uint32_t>(hs * sizeof(T));
-  const size_t stage_bytes = static_cast<size_t>(h) * sizeof(T);
+  constexpr int W = THREADS / 32;
+  __shared__ float2 red[W];
+  const int64_t r = blockIdx.x;
   const int vpr = static_cast<int>(h / V);
-  const int64_t G0 = blockIdx.x, GS = gridDim.x;
-  if (threadIdx.x == 0) {
-    abort_flag = 0;
-    for (int st = 0; st < STAGES; ++st) tpd::mbar_init(&bar[st], 1);
-    tpd::fence_barrier_init();
-  }
-  __syncthreads();
-  int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
-  if (threadIdx.x == 0)
-    for (; issued < STAGES && G0 + issued * GS < rows; ++issued)
-      issue_row(X, nullptr, p, G0 + issued * GS, shard_bytes, sbuf + issued * stage_bytes, &bar[issued]);
-  // gamma (and beta) of this thread's columns, packed, for every row
-  uint4 gp[VPT], bp[VPT];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4 xr[kVptMax];
+  float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
+  for (int i = 0; i < kVptMax; ++i) {
     const int c = threadIdx.x + i * THREADS;
-    gp[i] = bp[i] = make_uint4(0, 0, 0, 0);
+    xr[i] = make_uint4(0, 0, 0, 0);
+    if (c < vpr) {
+      const int sh = c / vps;
+      xr[i] = __ldcs(reinterpret_cast<const uint4*>(X.p[sh]) + r * vps + (c - sh * vps));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    if (threadIdx.x + i * THREADS < vpr) {
+      float x[V];
+      LnVec<T>::unpack(xr[i], x);
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        s1 += x[e];
+        s2 += x[e] * x[e];
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  if (lane == 0) red[warp] = make_float2(s1, s2);
+  __syncthreads();
+  float2 tot = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < W; ++w) {
+    tot.x += red[w].x;
+    tot.y += red[w].y;
+  }
+  const float mean = RMS ? 0.f : tot.x / static_cast<float>(h);
+  const float var = RMS ? tot.y / static_cast<float>(h) : fmaxf(tot.y / static_cast<float>(h) - mean * mean, 0.f);
+  const float rstd = rsqrtf(var + kEps);
+#pragma unroll
+  for (int i = 0; i < kVptMax; ++i) {
+    const int c = threadIdx.x + i * THREADS;
     if (c < vpr) {
       const int sh = c / vps, lc = c - sh * vps;
-      gp[i] = *reinterpret_cast<const uint4*>(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V);
-      if (!RMS) bp[i] = *reinterpret_cast<const uint4*>(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V);
-    }
-  }
-  int64_t k = 0;
-  for (;; ++k) {
-    const int64_t r = G0 + k * GS;
-    if (r >= rows) break;
-    const int st = static_cast<int>(k % STAGES);
-    // a thread whose wait gave up computes on an unfinished stage; the sum's
-    // barrier then stops every thread before anything is written
-    const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
-    const uint4* row = reinterpret_cast<const uint4*>(sbuf + st * stage_bytes);
-    float s1 = 0.f, s2 = 0.f;
+      float x[V], g[V], bb[V], o[V];
+      LnVec<T>::unpack(xr[i], x);
+      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
+      if (!RMS) LnVec<T>::load(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V, bb);
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int c = threadIdx.x + i * THREADS;
-      if (c < vpr) {
-        float x[V];
-        LnVec<T>::unpack(row[c], x);
-#pragma unroll
-        for (int e = 0; e < V; ++e) {
-          s1 += x[e];
-          s2 += x[e] * x[e];
-        }
-      }
-    }
-    float2 tot = make_float2(s1, s2);
-    if (!block_sum2_ok<THREADS>(tot, ok, red)) break;
-    const float mean = RMS ? 0.f : tot.x / static_cast<float>(h);
-    const float var = RMS ? tot.y / static_cast<float>(h)
-                          : fmaxf(tot.y / static_cast<float>(h) - mean * mean, 0.f);
-    const float rstd = rsqrtf(var + kEps);
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int c = threadIdx.x + i * THREADS;
-      if (c < vpr) {
-        float x[V], g[V], bb[V], o[V];
-        LnVec<T>::unpack(row[c], x);
-        LnVec<T>::unpack(gp[i], g);
-        if (!RMS) LnVec<T>::unpack(bp[i], bb);
-#pragma unroll
-        for (int e = 0; e < V; ++e) o[e] = (x[e] - mean) * rstd * g[e] + (RMS ? 0.f : bb[e]);
-        LnVec<T>::store(const_cast<uint4*>(row) + c, o);  // y replaces x in the stage
-      }
-    }
-    if (threadIdx.x == 0) {
-      if (mean_out && !RMS) mean_out[r] = mean;
-      if (rstd_out) rstd_out[r] = rstd;
-    }
-    tpd::fence_proxy_async_smem();
-    __syncthreads();  // the stage holds the row's y
-    if (threadIdx.x == 0) {
-      // y leaves by bulk copies; the previous row's stage is reloaded once its
-      // store has read it.
-      store_row(Y, p, r, shard_bytes, sbuf + st * stage_bytes);
-      tpd::bulk_wait_read<1>();
-      if (k >= 1 && G0 + (k - 1 + STAGES) * GS < rows) {
-        const int s2 = static_cast<int>((k - 1) % STAGES);
-        issue_row(X, nullptr, p, G0 + (k - 1 + STAGES) * GS, shard_bytes, sbuf + s2 * stage_bytes, &bar[s2]);
-        issued = k - 1 + STAGES + 1;
-      }
+      for (int e = 0; e < V; ++e) o[e] = (x[e] - mean) * rstd * g[e] + (RMS ? 0.f : bb[e]);
+      LnVec<T>::store(reinterpret_cast<uint4*>(Y.p[sh]) + r * vps + lc, o);
     }
   }
   if (threadIdx.x == 0) {
-    tpd::bulk_wait_all();  // every store has landed
-    if (abort_flag)        // let loads still in flight land (bounded)
-      for (int64_t kk = k; kk < issued; ++kk) {
-        int again = 0;
-        tpd::mbar_wait(&bar[kk % STAGES], static_cast<uint32_t>(kk / STAGES) & 1u, &again, nullptr);
-      }
+    if (mean_out && !RMS) mean_out[r] = mean;
+    if (rstd_out) rstd_out[r] = rstd;
   }
 }
 
 
-// Backward of a hidden-sharded norm in one pass over x and dy, staged like
-// the forward (a stage holds a row of x and the same row of dy). Thread tid
+
+// Backward of a hidden-sharded norm in one pass over x and dy, with the rows
+// staged as above (a stage holds a row of x and the same row of dy). Thread tid
 // owns the same column vectors of every row, so besides dx it keeps running
 // column partials dgamma = sum dy * xhat and dbeta = sum dy in registers and
 // writes them once: part[b][0][col], part[b][1][col]. A second kernel sums the
@@ -685,7 +680,6 @@ int vpt_for(int64_t vpr, int th) {
   return need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : 8;
 }
 
-constexpr int kNormFwdStages = 4;
 constexpr int kNormBwdStages = 3;
 
 #define TP_NH_DISPATCH(LAUNCH, T, R)                 \
@@ -700,15 +694,7 @@ constexpr int kNormBwdStages = 3;
 // once (at most one per row), with its dynamic shared memory opted in.
 template <typename K>
 tp_status pipe_grid(K kernel, int threads, int smem, int64_t rows, int64_t* grid) {
-  tp_status s = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-                            "cudaFuncSetAttribute(norm)");
-  if (s != TP_OK) return s;
-  int per_sm = 0;
-  s = cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem),
-                  "cudaOccupancyMaxActiveBlocksPerMultiprocessor(norm)");
-  if (s != TP_OK) return s;
-  *grid = std::max<int64_t>(1, std::min<int64_t>(rows, static_cast<int64_t>(num_sms()) * std::max(per_sm, 1)));
-  return TP_OK;
+  return persistent_grid(reinterpret_cast<const void*>(kernel), threads, smem, rows, grid);
 }
 
 tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G,
@@ -720,28 +706,24 @@ tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
   if (rows == 0) return TP_OK;
   const int vps = static_cast<int>(hs / V);
-  const int th = hsh_threads(vpr);
-  const int vpt = vpt_for(vpr, th);
-  const int smem = static_cast<int>(kNormFwdStages * h * static_cast<int64_t>(dsize(dt)));
-  unsigned* status = nullptr;
-  tp_status s = device_status_word(&status);
-  if (s != TP_OK) return s;
-  int64_t grid = 1;
-#define TP_NH_FWD(T, TH, VP, R)                                                                    \
-  do {                                                                                             \
-    auto kern = norm_hsh_fwd_kernel<T, TH, VP, kNormFwdStages, R>;                                 \
-    s = pipe_grid(kern, TH, smem, rows, &grid);                                                    \
-    if (s != TP_OK) return s;                                                                      \
-    kern<<<static_cast<unsigned>(grid), TH, smem, st>>>(X, G, B, Y, p, vps, hs, h, rows, mean,     \
-                                                        rstd, status);                             \
+  const int th = threads_for(vpr);
+#define TP_NH_FWD(T, TH, R)                                                                      \
+  norm_hsh_row_fwd_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, B, Y, vps, h, \
+                                                                               mean, rstd)
+#define TP_NH_FWD_TH(T, R)          \
+  do {                              \
+    if (th == 64) TP_NH_FWD(T, 64, R);       \
+    else if (th == 128) TP_NH_FWD(T, 128, R); \
+    else TP_NH_FWD(T, 256, R);               \
   } while (0)
   if (dt == TP_BF16) {
-    if (rms) { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, true); }
-    else { TP_NH_DISPATCH(TP_NH_FWD, __nv_bfloat16, false); }
+    if (rms) TP_NH_FWD_TH(__nv_bfloat16, true);
+    else TP_NH_FWD_TH(__nv_bfloat16, false);
   } else {
-    if (rms) { TP_NH_DISPATCH(TP_NH_FWD, float, true); }
-    else { TP_NH_DISPATCH(TP_NH_FWD, float, false); }
+    if (rms) TP_NH_FWD_TH(float, true);
+    else TP_NH_FWD_TH(float, false);
   }
+#undef TP_NH_FWD_TH
 #undef TP_NH_FWD
   return after_launch("norm_sharded_fwd");
 }

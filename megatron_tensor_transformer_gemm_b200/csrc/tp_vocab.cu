@@ -634,24 +634,11 @@ template <typename E, int THREADS, int STAGES>
 tp_status launch_ce_pipe(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
                          const int32_t* labels, float scale, float* loss, float* lse, int64_t T,
                          uint32_t stage_bytes, unsigned* status, cudaStream_t st) {
-  static bool attr = false;
   auto fn = vocab_ce_pipe_kernel<E, THREADS, STAGES>;
-  if (!attr) {
-    tp_status r = tpi::cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   kCeSmemMax),
-                              "cudaFuncSetAttribute(vocab_cross_entropy)");
-    if (r != TP_OK) return r;
-    attr = true;
-  }
   const int smem = static_cast<int>(stage_bytes) * STAGES;
-  int per_sm = 0;
-  tp_status r = tpi::cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, THREADS, smem),
-                            "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  int64_t grid = 1;
+  tp_status r = tpi::persistent_grid(reinterpret_cast<const void*>(fn), THREADS, smem, T, &grid);
   if (r != TP_OK) return r;
-  int dev = 0, n_sm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(T, static_cast<int64_t>(n_sm) * std::max(per_sm, 1)));
   fn<<<static_cast<unsigned>(grid), THREADS, smem, st>>>(L, G, p, Vs, vocab, T, stage_bytes, labels,
                                                          scale, loss, lse, status);
   return TP_OK;
