@@ -453,16 +453,28 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
   const int64_t r = blockIdx.x;
   const int vpr = static_cast<int>(h / V);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // shard and offset of vector c = tid + i*THREADS, stepped from i to i + 1
+  // (one division per thread instead of one per vector)
+  const int step_sh = THREADS / vps, step_lc = THREADS - step_sh * vps;
+  int sh[kVptMax], lc[kVptMax];
+  sh[0] = static_cast<int>(threadIdx.x) / vps;
+  lc[0] = static_cast<int>(threadIdx.x) - sh[0] * vps;
+#pragma unroll
+  for (int i = 1; i < kVptMax; ++i) {
+    sh[i] = sh[i - 1] + step_sh;
+    lc[i] = lc[i - 1] + step_lc;
+    if (lc[i] >= vps) {
+      lc[i] -= vps;
+      ++sh[i];
+    }
+  }
   uint4 xr[kVptMax];
   float s1 = 0.f, s2 = 0.f;
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
     xr[i] = make_uint4(0, 0, 0, 0);
-    if (c < vpr) {
-      const int sh = c / vps;
-      xr[i] = __ldcs(reinterpret_cast<const uint4*>(X.p[sh]) + r * vps + (c - sh * vps));
-    }
+    if (threadIdx.x + i * THREADS < vpr)
+      xr[i] = __ldcs(reinterpret_cast<const uint4*>(X.p[sh[i]]) + r * vps + lc[i]);
   }
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
@@ -494,16 +506,14 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
   const float rstd = rsqrtf(var + kEps);
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
-    const int c = threadIdx.x + i * THREADS;
-    if (c < vpr) {
-      const int sh = c / vps, lc = c - sh * vps;
+    if (threadIdx.x + i * THREADS < vpr) {
       float x[V], g[V], bb[V], o[V];
       LnVec<T>::unpack(xr[i], x);
-      LnVec<T>::load(static_cast<const T*>(G.p[sh]) + static_cast<int64_t>(lc) * V, g);
-      if (!RMS) LnVec<T>::load(static_cast<const T*>(B.p[sh]) + static_cast<int64_t>(lc) * V, bb);
+      LnVec<T>::load(static_cast<const T*>(G.p[sh[i]]) + static_cast<int64_t>(lc[i]) * V, g);
+      if (!RMS) LnVec<T>::load(static_cast<const T*>(B.p[sh[i]]) + static_cast<int64_t>(lc[i]) * V, bb);
 #pragma unroll
       for (int e = 0; e < V; ++e) o[e] = (x[e] - mean) * rstd * g[e] + (RMS ? 0.f : bb[e]);
-      LnVec<T>::store(reinterpret_cast<uint4*>(Y.p[sh]) + r * vps + lc, o);
+      LnVec<T>::store(reinterpret_cast<uint4*>(Y.p[sh[i]]) + r * vps + lc[i], o);
     }
   }
   if (threadIdx.x == 0) {

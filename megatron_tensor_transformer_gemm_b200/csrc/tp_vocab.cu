@@ -481,7 +481,12 @@ __device__ __forceinline__ bool ce_issue_row(const PtrArray& L, int p, int64_t t
 // out of the stream. The
 // shards are contiguous slices of the padded vocab, so 16-byte vector i of
 // a row holds columns [i * N, (i + 1) * N).
-template <typename T, int THREADS, int STAGES>
+//
+// VPT > 0: every thread's vectors of a row (at most VPT) are held in registers
+// through the row: its own max first, then one exp2 per logit relative to it,
+// kept for the gradient, which is that exp2 times 2^(own max - lse2) * scale:
+// one exponential per logit instead of two.
+template <typename T, int THREADS, int STAGES, int VPT>
 __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
     int vocab, int64_t T_rows, uint32_t stage_bytes, const int32_t* labels, float scale,
@@ -492,6 +497,9 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
   __shared__ uint64_t bar[STAGES];
   __shared__ int abort_flag;
   __shared__ float2 red2[THREADS / 32];
+  // the label's logit, handed to thread 0 by the thread that owns its vector
+  // (before the merge's barrier: after it, the owner may overwrite the stage)
+  __shared__ float s_zt;
   const uint32_t shard_bytes = static_cast<uint32_t>(Vs * sizeof(T));
   const int64_t G0 = blockIdx.x, GS = gridDim.x;
   int64_t issued = 0;  // thread 0: rows [0, issued) of this CTA have their loads issued
@@ -519,57 +527,115 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
     const uint4* row = reinterpret_cast<const uint4*>(sbuf + static_cast<size_t>(st) * stage_bytes);
     const bool ignore = label < 0 || label >= vocab;
+    const int lab_vec = ignore ? -1 : label / N;
+    // a bit test per element, not an index into x (which would put x in local memory)
+    const uint32_t lab_bit = ignore ? 0u : 1u << (label % N);
     // Vectors below nfull hold no padding column: no per-column tests there.
     const int nfull = vocab / N;
-    // One pass: this thread's running max (log2 domain) and sum of 2^(x - max).
+    float e[VPT > 0 ? VPT : 1][N];  // VPT > 0: 2^(x log2e - m) of this thread's columns
     float m = -INFINITY, sum = 0.f;
-    for (int i = threadIdx.x; i < total; i += THREADS) {
-      float x[N];
-      unpack16<T>(row[i], x);
-      if (i >= nfull) {
+    if constexpr (VPT > 0) {
 #pragma unroll
-        for (int e = 0; e < N; ++e)
-          if (i * N + e >= vocab) x[e] = -INFINITY;
+      for (int j = 0; j < VPT; ++j) {
+        const int i = threadIdx.x + j * THREADS;
+        if (i < total) {
+          unpack16<T>(row[i], e[j]);
+          if (i == lab_vec) {
+            float z = 0.f;
+#pragma unroll
+            for (int q = 0; q < N; ++q) z += ((lab_bit >> q) & 1u) ? e[j][q] : 0.f;
+            s_zt = z;
+          }
+          if (i >= nfull) {
+#pragma unroll
+            for (int q = 0; q < N; ++q)
+              if (i * N + q >= vocab) e[j][q] = -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < N; ++q) e[j][q] = -INFINITY;
+        }
+#pragma unroll
+        for (int q = 0; q < N; ++q) m = fmaxf(m, e[j][q]);
       }
-      float lm = x[0];
+      m *= kLog2e;
+      const float mo = m == -INFINITY ? 0.f : m;  // no column: every term is 2^-inf = 0
 #pragma unroll
-      for (int e = 1; e < N; ++e) lm = fmaxf(lm, x[e]);
-      lm *= kLog2e;
-      if (lm > m) {  // (an all-padding vector has lm = -inf and adds nothing below)
-        sum *= ex2f_fast(m - lm);
-        m = lm;
-      }
-      if (lm != -INFINITY) {
+      for (int j = 0; j < VPT; ++j)
 #pragma unroll
-        for (int e = 0; e < N; ++e) sum += ex2f_fast(fmaf(x[e], kLog2e, -m));
+        for (int q = 0; q < N; ++q) {
+          e[j][q] = ex2f_fast(fmaf(e[j][q], kLog2e, -mo));
+          sum += e[j][q];
+        }
+    } else {
+      // One pass: this thread's running max (log2 domain) and sum of 2^(x - max).
+      for (int i = threadIdx.x; i < total; i += THREADS) {
+        float x[N];
+        unpack16<T>(row[i], x);
+        if (i == lab_vec) {
+          float z = 0.f;
+#pragma unroll
+          for (int q = 0; q < N; ++q) z += ((lab_bit >> q) & 1u) ? x[q] : 0.f;
+          s_zt = z;
+        }
+        if (i >= nfull) {
+#pragma unroll
+          for (int q = 0; q < N; ++q)
+            if (i * N + q >= vocab) x[q] = -INFINITY;
+        }
+        float lm = x[0];
+#pragma unroll
+        for (int q = 1; q < N; ++q) lm = fmaxf(lm, x[q]);
+        lm *= kLog2e;
+        if (lm > m) {  // (an all-padding vector has lm = -inf and adds nothing below)
+          sum *= ex2f_fast(m - lm);
+          m = lm;
+        }
+        if (lm != -INFINITY) {
+#pragma unroll
+          for (int q = 0; q < N; ++q) sum += ex2f_fast(fmaf(x[q], kLog2e, -m));
+        }
       }
     }
+    const float m_own = m;
     MaxSum tot{m, sum};
     if (!block_merge_ok<THREADS>(tot, ok, red2)) break;
     const float lse2 = tot.m + log2f(tot.s);
     if (threadIdx.x == 0) {
       if (label >= vocab) atomicOr(status, kStatusBadIndex);
-      float zt = 0.f;
-      if (!ignore) {
-        float x[N];
-        unpack16<T>(row[label / N], x);
-        // a bit test per element, not an index into x (which would put x in local memory)
-        const uint32_t bit = 1u << (label % N);
-#pragma unroll
-        for (int e = 0; e < N; ++e) zt += ((bit >> e) & 1u) ? x[e] : 0.f;
-      }
       const float lse = lse2 * 0.6931471805599453f;
-      loss[t] = ignore ? 0.f : lse - zt;
+      loss[t] = ignore ? 0.f : lse - s_zt;
       if (lse_out) lse_out[t] = lse;
     }
     const bool grad = G.p[0] != nullptr;
-    if (grad) {
+    if (grad && VPT > 0) {
+      // scale * softmax = e * 2^(m_own - lse2) * scale (the scale in the
+      // exponent when it is positive); padding columns hold e = 0
+      const float f = ignore || m_own == -INFINITY
+                          ? 0.f
+                          : (scale > 0.f ? ex2f_fast(m_own - lse2 + log2f(scale)) : ex2f_fast(m_own - lse2) * scale);
+      uint4* out = const_cast<uint4*>(row);  // the gradient replaces the staged row
+#pragma unroll
+      for (int j = 0; j < (VPT > 0 ? VPT : 1); ++j) {
+        const int i = threadIdx.x + j * THREADS;
+        if (i < total) {
+          float g[N];
+#pragma unroll
+          for (int q = 0; q < N; ++q) g[q] = e[j][q] * f;
+          if (i == lab_vec) {  // minus the one-hot target
+#pragma unroll
+            for (int q = 0; q < N; ++q) g[q] -= ((lab_bit >> q) & 1u) ? scale : 0.f;
+          }
+          out[i] = pack16<T>(g);
+        }
+      }
+      tpd::fence_proxy_async_smem();
+    } else if (grad) {
       // scale * softmax = 2^(x log2e - lse2 + log2 scale): the scale rides in
       // the exponent when it is positive.
       const bool fold = scale > 0.f;
       const float bias = fold ? lse2 - log2f(scale) : lse2;
       const float mul = fold ? 1.f : scale;
-      const int lab_vec = ignore ? -1 : label / N;
       uint4* out = const_cast<uint4*>(row);  // the gradient replaces the staged row
       for (int i = threadIdx.x; i < total; i += THREADS) {
         float x[N];
@@ -589,10 +655,9 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
           for (int e = 0; e < N; ++e)
             x[e] = i * N + e < vocab ? ex2f_fast(fmaf(x[e], kLog2e, -bias)) * mul : 0.f;
         }
-        if (i == lab_vec) {  // minus the one-hot target (a bit test per element, as above)
-          const uint32_t bit = 1u << (label - i * N);
+        if (i == lab_vec) {  // minus the one-hot target
 #pragma unroll
-          for (int e = 0; e < N; ++e) x[e] -= ((bit >> e) & 1u) ? scale : 0.f;
+          for (int q = 0; q < N; ++q) x[q] -= ((lab_bit >> q) & 1u) ? scale : 0.f;
         }
         out[i] = pack16<T>(x);
       }
@@ -629,12 +694,13 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
 }
 
 constexpr int kCeSmemMax = 200 * 1024;  // shared memory for the staged rows
+constexpr int kCeVpt = 4;                // vectors per thread of the register-resident rows
 
-template <typename E, int THREADS, int STAGES>
+template <typename E, int THREADS, int STAGES, int VPT>
 tp_status launch_ce_pipe(const PtrArray& L, const MutPtrArray& G, int p, int64_t Vs, int vocab,
                          const int32_t* labels, float scale, float* loss, float* lse, int64_t T,
                          uint32_t stage_bytes, unsigned* status, cudaStream_t st) {
-  auto fn = vocab_ce_pipe_kernel<E, THREADS, STAGES>;
+  auto fn = vocab_ce_pipe_kernel<E, THREADS, STAGES, VPT>;
   const int smem = static_cast<int>(stage_bytes) * STAGES;
   int64_t grid = 1;
   tp_status r = tpi::persistent_grid(reinterpret_cast<const void*>(fn), THREADS, smem, T, &grid);
@@ -721,12 +787,16 @@ tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_
   if (s != TP_OK) return s;
   const int64_t row_bytes = static_cast<int64_t>(p) * Vs * static_cast<int64_t>(dsize(dt));
   const uint32_t sb = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
-  if (3 * row_bytes <= kCeSmemMax) {
-    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 3>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
-                      : launch_ce_pipe<float, 1024, 3>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
+  const int64_t vecs = row_bytes / 16;  // 16-byte vectors per row
+  if (3 * row_bytes <= kCeSmemMax && vecs <= kCeVpt * 1024) {
+    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 3, kCeVpt>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
+                      : launch_ce_pipe<float, 1024, 3, kCeVpt>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
+  } else if (3 * row_bytes <= kCeSmemMax) {
+    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 3, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
+                      : launch_ce_pipe<float, 1024, 3, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
   } else if (2 * row_bytes <= kCeSmemMax) {
-    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 2>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
-                      : launch_ce_pipe<float, 1024, 2>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
+    s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 2, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
+                      : launch_ce_pipe<float, 1024, 2, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
   } else if (dt == TP_BF16) {
     vocab_ce_kernel<__nv_bfloat16, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(
         L, G, p, Vs, vocab, labels, scale, loss, lse, status);

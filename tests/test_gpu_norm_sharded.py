@@ -11,7 +11,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("kind", ["rms", "layer"])
-@pytest.mark.parametrize("p,h", [(1, 512), (2, 512), (4, 4096), (8, 8192), (8, 128), (8, 16384)])
+@pytest.mark.parametrize("p,h", [(1, 512), (2, 512), (3, 1152), (4, 4096), (8, 8192), (8, 128), (8, 16384)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_norm_sharded_fwd_bwd(kind, p, h, dtype):
     """1500 rows: more than the backward's CTAs at every width, so each CTA
