@@ -244,7 +244,7 @@ TP_API tp_status tp_embedding_fwd(tp_plan* plan, int64_t T, const int32_t* ids,
  * for each vocab row v of shard i, the sum over tokens with id == v of dY[t]
  * (fp32, in token order, deterministic); rows no token uses are zero; ids
  * outside [0, vocab) are skipped. Uses the plan's device workspace (a stable
- * bucket sort of the token indices, about Vp/16 * ceil(T/1024) + 2 T ints).
+ * bucket sort of the token indices, about Vp/16 * (ceil(T/1024) + 1) + 2 T ints).
  * TP_ERR_UNSUPPORTED for Vp > 196608 or T > 2^31 - 1. */
 TP_API tp_status tp_embedding_bwd(tp_plan* plan, int64_t T, const int32_t* ids, const void* dY,
                                   void* const* dE, void* stream);

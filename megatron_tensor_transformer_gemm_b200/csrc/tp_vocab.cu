@@ -48,12 +48,14 @@ __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ Ptr
 
 // Embedding gradient as a stable bucket sort of the tokens, then a gather-sum:
 //   count    per 1024-token block, how many of its tokens fall in each bucket of
-//            16 vocab ids (cnt[bucket][block], bucket-major);
-//   scan     exclusive prefix over cnt in that order: the start of each
-//            (bucket, block) run in the sorted token list;
-//   scatter  each token's slot = its run start + the number of earlier tokens
-//            of its block in the same bucket, so every bucket lists its tokens
-//            in token order;
+//            16 vocab ids (cnt[block][bucket], block-major);
+//   scan     per bucket, the exclusive prefix of its counts over the blocks
+//            (in place) and the bucket's total; then one CTA turns the totals
+//            into each bucket's start in the sorted list (tot[bucket], with
+//            tot[nb] the number of listed tokens);
+//   scatter  each token's slot = its bucket's start + its block's prefix + the
+//            number of earlier tokens of its block in the same bucket, so
+//            every bucket lists its tokens in token order;
 //   accum    one CTA per (bucket, 1024-column slice), one warp per vocab row:
 //            each warp sums its row's listed dY rows in that order in fp32
 //            registers and writes the row of dE (zeros if none).
@@ -77,8 +79,22 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_count(const int32_t* ids
     if (valid_id(id, vocab)) atomicAdd(&hist[id / kEmbRows], 1);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < nb; i += kTokBlock)
-    cnt[static_cast<int64_t>(i) * nblk + blockIdx.x] = hist[i];
+  for (int i = threadIdx.x; i < nb; i += kTokBlock) cnt[static_cast<int64_t>(blockIdx.x) * nb + i] = hist[i];
+}
+
+// Thread b: bucket b's counts over the blocks become their exclusive prefix
+// (in place); tot[b] = the bucket's total.
+__global__ void __launch_bounds__(256) emb_bucket_prefix(int* cnt, int nb, int nblk, int* tot) {
+  const int b = blockIdx.x * 256 + threadIdx.x;
+  if (b >= nb) return;
+  int run = 0;
+  for (int k = 0; k < nblk; ++k) {
+    const int64_t i = static_cast<int64_t>(k) * nb + b;
+    const int c = cnt[i];
+    cnt[i] = run;
+    run += c;
+  }
+  tot[b] = run;
 }
 
 // One CTA: a[0..n) <- exclusive prefix sums, a[n] <- the total. Thread tid
@@ -135,8 +151,8 @@ __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
 
 // sorted[k] = (token, id - bucket * kEmbRows) of the k-th entry of the sorted list.
 __global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* ids, int64_t ntok,
-                                                                int vocab, int nb, int nblk,
-                                                                const int* off, int2* sorted) {
+                                                                int vocab, int nb, const int* off,
+                                                                const int* tot, int2* sorted) {
   __shared__ int seen[kEmbMaxBuckets];
   for (int i = threadIdx.x; i < nb; i += kTokBlock) seen[i] = 0;
   __syncthreads();
@@ -159,7 +175,7 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* i
     __syncthreads();
   }
   if (valid)
-    sorted[off[static_cast<int64_t>(b) * nblk + blockIdx.x] + base + rank] =
+    sorted[tot[b] + off[static_cast<int64_t>(blockIdx.x) * nb + b] + base + rank] =
         make_int2(static_cast<int>(t), id - b * kEmbRows);
 }
 
@@ -188,7 +204,8 @@ __device__ __forceinline__ uint4 pack16(const float (&x)[16 / sizeof(T)]) {
 }
 
 // One CTA per (bucket of 16 vocab rows, 1024-column slice): warp w owns vocab
-// row v0 + w; every lane owns 32 consecutive columns of the slice and sums,
+// row v0 + w; lane l owns the 16-byte vectors l, l + 32, ... of the slice (so
+// each of the warp's loads and stores covers 512 contiguous bytes) and sums,
 // in registers, the dY rows of the tokens listed for its row, in list (token)
 // order; then the warp writes its row (zeros if no token uses it).
 constexpr int kAccCols = 1024;                 // columns per CTA
@@ -196,20 +213,21 @@ constexpr int kAccThreads = 32 * kEmbRows;     // one warp per vocab row of the 
 
 template <typename T>
 __global__ void __launch_bounds__(kAccThreads) emb_bucket_accum(
-    const int2* sorted, const int* off, int nb, int nblk, const T* dY, int64_t h, int64_t Vs,
-    int64_t Vp, const __grid_constant__ MutPtrArray dE) {
+    const int2* sorted, const int* tot, const T* dY, int64_t h, int64_t Vs, int64_t Vp,
+    const __grid_constant__ MutPtrArray dE) {
   constexpr int E = 16 / sizeof(T);   // elements per 16-byte vector
   constexpr int NV = 32 / E;          // 16-byte vectors per lane (32 columns)
+  constexpr int STRIDE = 32 * E;      // columns between a lane's vectors
   __shared__ int ltok[kListChunk];
   __shared__ int lrow[kListChunk];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kAccCols + lane * 32;  // this lane's columns
+  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kAccCols + lane * E;  // this lane's first column
   float acc[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-  const int start = off[static_cast<int64_t>(b) * nblk];
-  const int end = off[static_cast<int64_t>(b + 1) * nblk];  // off[nb * nblk] is the total
+  const int start = tot[b];
+  const int end = tot[b + 1];  // tot[nb] is the number of listed tokens
   for (int k0 = start; k0 < end; k0 += kListChunk) {
     const int n = end - k0 < kListChunk ? end - k0 : kListChunk;
     __syncthreads();  // the previous chunk's list is consumed
@@ -225,7 +243,7 @@ __global__ void __launch_bounds__(kAccThreads) emb_bucket_accum(
       uint4 u[NV];
 #pragma unroll
       for (int q = 0; q < NV; ++q)
-        u[q] = c0 + q * E < h ? reinterpret_cast<const uint4*>(src)[q] : make_uint4(0, 0, 0, 0);
+        u[q] = c0 + q * STRIDE < h ? *reinterpret_cast<const uint4*>(src + q * STRIDE) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int q = 0; q < NV; ++q) {
         float x[E];
@@ -241,11 +259,11 @@ __global__ void __launch_bounds__(kAccThreads) emb_bucket_accum(
   T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + c0;
 #pragma unroll
   for (int q = 0; q < NV; ++q) {
-    if (c0 + q * E < h) {
+    if (c0 + q * STRIDE < h) {
       float x[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) x[e] = acc[q * E + e];
-      reinterpret_cast<uint4*>(dst)[q] = pack16<T>(x);
+      *reinterpret_cast<uint4*>(dst + q * STRIDE) = pack16<T>(x);
     }
   }
 }
@@ -736,6 +754,8 @@ tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab,
   return after_launch("embedding_fwd");
 }
 
+static int64_t round4(int64_t n) { return (n + 3) / 4 * 4; }
+
 tp_status embedding_bwd_workspace(int64_t T, int64_t Vp, size_t* bytes) {
   const int64_t nb = (Vp + kEmbRows - 1) / kEmbRows;
   const int64_t nblk = (T + kTokBlock - 1) / kTokBlock;
@@ -744,7 +764,8 @@ tp_status embedding_bwd_workspace(int64_t T, int64_t Vp, size_t* bytes) {
                 kEmbMaxBuckets * kEmbRows);
   if (T > 0x7fffffffLL || nb * nblk + 1 > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "embedding backward: %lld tokens is too many", (long long)T);
-  *bytes = static_cast<size_t>(nb * nblk + 1 + 1 + 2 * T) * sizeof(int);  // + 1: int2 alignment
+  // cnt[nblk][nb], tot[nb + 1], sorted[T] (int2), each starting on 16 bytes
+  *bytes = static_cast<size_t>(round4(nb * nblk) + round4(nb + 1) + 2 * T) * sizeof(int);
   return TP_OK;
 }
 
@@ -754,28 +775,33 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
   const int nb = static_cast<int>((Vp + kEmbRows - 1) / kEmbRows);
   const int nblk = static_cast<int>((T + kTokBlock - 1) / kTokBlock);
   int* cnt = static_cast<int*>(ws);
-  const int64_t ncnt = static_cast<int64_t>(nb) * nblk + 1;
-  int2* sorted = reinterpret_cast<int2*>(cnt + ncnt + (ncnt & 1));
+  int* tot = cnt + round4(static_cast<int64_t>(nb) * nblk);
+  int2* sorted = reinterpret_cast<int2*>(tot + round4(nb + 1));
+  tp_status s = TP_OK;
   if (T > 0) {
     emb_bucket_count<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt);
-    tp_status s = after_launch("embedding_bwd count");
+    s = after_launch("embedding_bwd count");
     if (s != TP_OK) return s;
-  }
-  emb_scan<<<1, 1024, 0, st>>>(cnt, static_cast<int64_t>(nb) * nblk);
-  tp_status s = after_launch("embedding_bwd scan");
-  if (s != TP_OK) return s;
-  if (T > 0) {
-    emb_bucket_scatter<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt, sorted);
+    emb_bucket_prefix<<<(nb + 255) / 256, 256, 0, st>>>(cnt, nb, nblk, tot);
+    s = after_launch("embedding_bwd prefix");
+    if (s != TP_OK) return s;
+    emb_scan<<<1, 1024, 0, st>>>(tot, nb);
+    s = after_launch("embedding_bwd scan");
+    if (s != TP_OK) return s;
+    emb_bucket_scatter<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, cnt, tot, sorted);
     s = after_launch("embedding_bwd scatter");
+    if (s != TP_OK) return s;
+  } else {
+    s = cuda_status(cudaMemsetAsync(tot, 0, static_cast<size_t>(nb + 1) * sizeof(int), st), "embedding_bwd");
     if (s != TP_OK) return s;
   }
   dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((h + kAccCols - 1) / kAccCols));
   if (dt == TP_BF16)
     emb_bucket_accum<__nv_bfloat16><<<grid, kAccThreads, 0, st>>>(
-        sorted, cnt, nb, nblk, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
+        sorted, tot, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
   else
-    emb_bucket_accum<float><<<grid, kAccThreads, 0, st>>>(sorted, cnt, nb, nblk,
-                                                         static_cast<const float*>(dY), h, Vs, Vp, dE);
+    emb_bucket_accum<float><<<grid, kAccThreads, 0, st>>>(sorted, tot, static_cast<const float*>(dY), h, Vs,
+                                                         Vp, dE);
   return after_launch("embedding_bwd accumulate");
 }
 
