@@ -56,9 +56,9 @@ __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ Ptr
 //   scatter  each token's slot = its bucket's start + its block's prefix + the
 //            number of earlier tokens of its block in the same bucket, so
 //            every bucket lists its tokens in token order;
-//   accum    one CTA per (bucket, 1024-column slice), one warp per vocab row:
-//            each warp sums its row's listed dY rows in that order in fp32
-//            registers and writes the row of dE (zeros if none).
+//   accum    one CTA per bucket, one warp per vocab row: each warp sums its
+//            row's listed dY rows in that order in fp32 registers and writes
+//            the row of dE (zeros if none; a copy if one).
 // No atomics touch the sums, so the result is deterministic.
 constexpr int kEmbRows = 16;    // vocab ids per bucket
 constexpr int kTokBlock = 1024; // tokens per count / scatter CTA
@@ -203,68 +203,137 @@ __device__ __forceinline__ uint4 pack16(const float (&x)[16 / sizeof(T)]) {
   }
 }
 
-// One CTA per (bucket of 16 vocab rows, 1024-column slice): warp w owns vocab
-// row v0 + w; lane l owns the 16-byte vectors l, l + 32, ... of the slice (so
-// each of the warp's loads and stores covers 512 contiguous bytes) and sums,
-// in registers, the dY rows of the tokens listed for its row, in list (token)
-// order; then the warp writes its row (zeros if no token uses it).
-constexpr int kAccCols = 1024;                 // columns per CTA
+// One CTA per bucket of 16 vocab rows, all h columns: warp w owns vocab row
+// v0 + w. The bucket's token list comes into shared memory once; each warp
+// counts its own entries (ballots over the list) and then
+//   - no token: writes a zero row;
+//   - one token: copies that token's dY row (a sum of one term in fp32,
+//     rounded back to the same type, is that term), 8 vectors per lane in
+//     flight;
+//   - more: passes of kAccCols columns, lane l owning vectors l, l + 32, ...
+//     of the pass (each load and store of the warp covers 512 contiguous
+//     bytes), summing the listed dY rows in list (token) order in fp32
+//     registers.
+// A bucket listed by more than kListChunk tokens takes the list in chunks,
+// pass by pass, with every warp summing.
+constexpr int kAccCols = 1024;                 // columns per accumulation pass
 constexpr int kAccThreads = 32 * kEmbRows;     // one warp per vocab row of the bucket
+constexpr int kCopyVec = 8;                    // vectors per lane in flight when copying a row
 
 template <typename T>
-__global__ void __launch_bounds__(kAccThreads) emb_bucket_accum(
-    const int2* sorted, const int* tot, const T* dY, int64_t h, int64_t Vs, int64_t Vp,
-    const __grid_constant__ MutPtrArray dE) {
+__device__ __forceinline__ void emb_accum_pass(const int* ltok, const int* lrow, int n, int warp, int lane,
+                                               const T* dY, int64_t h, int64_t cs, float (&acc)[32]) {
   constexpr int E = 16 / sizeof(T);   // elements per 16-byte vector
-  constexpr int NV = 32 / E;          // 16-byte vectors per lane (32 columns)
+  constexpr int NV = 32 / E;          // vectors per lane in a pass
   constexpr int STRIDE = 32 * E;      // columns between a lane's vectors
-  __shared__ int ltok[kListChunk];
-  __shared__ int lrow[kListChunk];
-  const int b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t c0 = static_cast<int64_t>(blockIdx.y) * kAccCols + lane * E;  // this lane's first column
-  float acc[32];
+  const int64_t c0 = cs + lane * E;
+  for (int k = 0; k < n; ++k) {
+    if (lrow[k] != warp) continue;  // warp-uniform
+    const T* src = dY + static_cast<int64_t>(ltok[k]) * h + c0;
+    uint4 u[NV];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-  const int start = tot[b];
-  const int end = tot[b + 1];  // tot[nb] is the number of listed tokens
-  for (int k0 = start; k0 < end; k0 += kListChunk) {
-    const int n = end - k0 < kListChunk ? end - k0 : kListChunk;
-    __syncthreads();  // the previous chunk's list is consumed
-    for (int k = threadIdx.x; k < n; k += kAccThreads) {
-      const int2 e = sorted[k0 + k];
-      ltok[k] = e.x;
-      lrow[k] = e.y;
-    }
-    __syncthreads();
-    for (int k = 0; k < n; ++k) {
-      if (lrow[k] != warp) continue;  // warp-uniform
-      const T* src = dY + static_cast<int64_t>(ltok[k]) * h + c0;
-      uint4 u[NV];
+    for (int q = 0; q < NV; ++q)
+      u[q] = c0 + q * STRIDE < h ? *reinterpret_cast<const uint4*>(src + q * STRIDE) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int q = 0; q < NV; ++q)
-        u[q] = c0 + q * STRIDE < h ? *reinterpret_cast<const uint4*>(src + q * STRIDE) : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < NV; ++q) {
+      float x[E];
+      unpack16<T>(u[q], x);
 #pragma unroll
-      for (int q = 0; q < NV; ++q) {
-        float x[E];
-        unpack16<T>(u[q], x);
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[q * E + e] += x[e];
-      }
+      for (int e = 0; e < E; ++e) acc[q * E + e] += x[e];
     }
   }
-  const int64_t v = static_cast<int64_t>(b) * kEmbRows + warp;
-  if (v >= Vp) return;
-  const int s = static_cast<int>(v / Vs);
-  T* dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h + c0;
+}
+
+template <typename T>
+__device__ __forceinline__ void emb_store_pass(T* dst, int64_t h, int64_t cs, int lane, const float (&acc)[32]) {
+  constexpr int E = 16 / sizeof(T);
+  constexpr int NV = 32 / E;
+  constexpr int STRIDE = 32 * E;
+  const int64_t c0 = cs + lane * E;
 #pragma unroll
   for (int q = 0; q < NV; ++q) {
     if (c0 + q * STRIDE < h) {
       float x[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) x[e] = acc[q * E + e];
-      *reinterpret_cast<uint4*>(dst + q * STRIDE) = pack16<T>(x);
+      *reinterpret_cast<uint4*>(dst + c0 + q * STRIDE) = pack16<T>(x);
     }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kAccThreads, 2) emb_bucket_accum(
+    const int2* sorted, const int* tot, const T* dY, int64_t h, int64_t Vs, int64_t Vp,
+    const __grid_constant__ MutPtrArray dE) {
+  constexpr int E = 16 / sizeof(T);
+  __shared__ int ltok[kListChunk];
+  __shared__ int lrow[kListChunk];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t v = static_cast<int64_t>(b) * kEmbRows + warp;
+  const bool has_row = v < Vp;
+  T* dst = nullptr;
+  if (has_row) {
+    const int s = static_cast<int>(v / Vs);
+    dst = static_cast<T*>(dE.p[s]) + (v - s * Vs) * h;
+  }
+  const int start = tot[b];
+  const int n = tot[b + 1] - start;  // tot[nb] is the number of listed tokens
+  float acc[32];
+  if (n <= kListChunk) {
+    for (int k = threadIdx.x; k < n; k += kAccThreads) {
+      const int2 e = sorted[start + k];
+      ltok[k] = e.x;
+      lrow[k] = e.y;
+    }
+    __syncthreads();
+    if (!has_row) return;
+    int cnt = 0, first = 0;
+    for (int k0 = 0; k0 < n; k0 += 32) {
+      const int k = k0 + lane;
+      const unsigned m = __ballot_sync(0xffffffffu, k < n && lrow[k] == warp);
+      if (cnt == 0 && m) first = k0 + __ffs(m) - 1;
+      cnt += __popc(m);
+    }
+    const int vpr = static_cast<int>(h / E);
+    uint4* dv = reinterpret_cast<uint4*>(dst);
+    if (cnt == 0) {
+      for (int c = lane; c < vpr; c += 32) dv[c] = make_uint4(0, 0, 0, 0);
+    } else if (cnt == 1) {
+      const uint4* sv = reinterpret_cast<const uint4*>(dY + static_cast<int64_t>(ltok[first]) * h);
+      for (int c0 = lane; c0 < vpr; c0 += 32 * kCopyVec) {
+        uint4 u[kCopyVec];
+#pragma unroll
+        for (int j = 0; j < kCopyVec; ++j) u[j] = c0 + 32 * j < vpr ? sv[c0 + 32 * j] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < kCopyVec; ++j)
+          if (c0 + 32 * j < vpr) dv[c0 + 32 * j] = u[j];
+      }
+    } else {
+      for (int64_t cs = 0; cs < h; cs += kAccCols) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        emb_accum_pass<T>(ltok, lrow, n, warp, lane, dY, h, cs, acc);
+        emb_store_pass<T>(dst, h, cs, lane, acc);
+      }
+    }
+    return;
+  }
+  for (int64_t cs = 0; cs < h; cs += kAccCols) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int k0 = 0; k0 < n; k0 += kListChunk) {
+      const int nn = n - k0 < kListChunk ? n - k0 : kListChunk;
+      __syncthreads();  // the previous chunk's list is consumed
+      for (int k = threadIdx.x; k < nn; k += kAccThreads) {
+        const int2 e = sorted[start + k0 + k];
+        ltok[k] = e.x;
+        lrow[k] = e.y;
+      }
+      __syncthreads();
+      emb_accum_pass<T>(ltok, lrow, nn, warp, lane, dY, h, cs, acc);
+    }
+    if (has_row) emb_store_pass<T>(dst, h, cs, lane, acc);
   }
 }
 
@@ -795,7 +864,7 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
     s = cuda_status(cudaMemsetAsync(tot, 0, static_cast<size_t>(nb + 1) * sizeof(int), st), "embedding_bwd");
     if (s != TP_OK) return s;
   }
-  dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>((h + kAccCols - 1) / kAccCols));
+  const unsigned grid = static_cast<unsigned>(nb);
   if (dt == TP_BF16)
     emb_bucket_accum<__nv_bfloat16><<<grid, kAccThreads, 0, st>>>(
         sorted, tot, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
