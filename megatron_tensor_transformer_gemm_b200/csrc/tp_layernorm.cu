@@ -243,15 +243,45 @@ __global__ void __launch_bounds__(256) ln_bwd_param_pass1(const T* x, const T* d
   }
 }
 
-__global__ void ln_bwd_param_pass2(const float* part, int splits, int64_t cols, float* dgamma,
-                                   float* dbeta, int accumulate) {
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
+// Sums of the per-CTA partials part[k][0|1][c] over k for kPass2Cols columns
+// c0 + lane: warp w takes k = w, w + 8, ... in increasing order, then the
+// eight warps' sums are added in warp order (fixed order: deterministic).
+// Lane 0..31 of warp 0 returns true with the column's two sums.
+constexpr int kPass2Cols = 32;
+__device__ __forceinline__ bool param_colsum(const float* part, int splits, int64_t cols, int64_t c,
+                                             float* sg_out, float* sb_out) {
+  __shared__ float rg[8][32], rb[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float sg = 0.f, sb = 0.f;
-  for (int k = 0; k < splits; ++k) {
-    sg += part[(static_cast<int64_t>(k) * 2 + 0) * cols + c];
-    sb += part[(static_cast<int64_t>(k) * 2 + 1) * cols + c];
+  if (c < cols) {
+#pragma unroll 4
+    for (int k = warp; k < splits; k += 8) {
+      sg += part[(static_cast<int64_t>(k) * 2 + 0) * cols + c];
+      sb += part[(static_cast<int64_t>(k) * 2 + 1) * cols + c];
+    }
   }
+  rg[warp][lane] = sg;
+  rb[warp][lane] = sb;
+  __syncthreads();
+  if (warp != 0 || c >= cols) return false;
+  sg = rg[0][lane];
+  sb = rb[0][lane];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) {
+    sg += rg[w][lane];
+    sb += rb[w][lane];
+  }
+  *sg_out = sg;
+  *sb_out = sb;
+  return true;
+}
+
+// 256 threads per CTA, kPass2Cols columns per CTA.
+__global__ void __launch_bounds__(256) ln_bwd_param_pass2(const float* part, int splits, int64_t cols,
+                                                          float* dgamma, float* dbeta, int accumulate) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
+  float sg, sb;
+  if (!param_colsum(part, splits, cols, c, &sg, &sb)) return;
   dgamma[c] = accumulate ? dgamma[c] + sg : sg;
   dbeta[c] = accumulate ? dbeta[c] + sb : sb;
 }
@@ -364,7 +394,7 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
     s = after_launch("layernorm_bwd/param1");
     if (s != TP_OK) return s;
   }
-  ln_bwd_param_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+  ln_bwd_param_pass2<<<static_cast<unsigned>((cols + kPass2Cols - 1) / kPass2Cols), 256, 0, st>>>(
       part, static_cast<int>(splits), cols, dgamma, dbeta, accumulate);
   return after_launch("layernorm_bwd/param2");
 }
@@ -656,16 +686,12 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
 
 // dgamma[c] (and dbeta[c]) = the fixed-order sum over the CTAs' partials
 // (added to the existing value when accumulate is set).
-__global__ void norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
-                                     const __grid_constant__ MutPtrArray dg,
-                                     const __grid_constant__ MutPtrArray db, int accumulate) {
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (c >= h) return;
-  float sg = 0.f, sb = 0.f;
-  for (int k = 0; k < splits; ++k) {
-    sg += part[(static_cast<int64_t>(k) * 2 + 0) * h + c];
-    sb += part[(static_cast<int64_t>(k) * 2 + 1) * h + c];
-  }
+__global__ void __launch_bounds__(256) norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
+                                                            const __grid_constant__ MutPtrArray dg,
+                                                            const __grid_constant__ MutPtrArray db, int accumulate) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
+  float sg, sb;
+  if (!param_colsum(part, splits, h, c, &sg, &sb)) return;
   const int sh = static_cast<int>(c / hs);
   const int64_t lc = c - sh * hs;
   float* g = static_cast<float*>(dg.p[sh]) + lc;
@@ -788,7 +814,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
     s = after_launch("norm_sharded_bwd");
     if (s != TP_OK) return s;
   }
-  norm_hsh_param_pass2<<<static_cast<unsigned>((h + 255) / 256), 256, 0, st>>>(
+  norm_hsh_param_pass2<<<static_cast<unsigned>((h + kPass2Cols - 1) / kPass2Cols), 256, 0, st>>>(
       part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg, db, accumulate);
   return after_launch("norm_sharded_bwd/param");
 }

@@ -88,11 +88,15 @@ __global__ void __launch_bounds__(256) emb_bucket_prefix(int* cnt, int nb, int n
   const int b = blockIdx.x * 256 + threadIdx.x;
   if (b >= nb) return;
   int run = 0;
-  for (int k = 0; k < nblk; ++k) {
-    const int64_t i = static_cast<int64_t>(k) * nb + b;
-    const int c = cnt[i];
-    cnt[i] = run;
-    run += c;
+  for (int k0 = 0; k0 < nblk; k0 += 8) {  // eight loads in flight, then their stores
+    int c[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c[j] = k0 + j < nblk ? cnt[static_cast<int64_t>(k0 + j) * nb + b] : 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (k0 + j < nblk) cnt[static_cast<int64_t>(k0 + j) * nb + b] = run;
+      run += c[j];
+    }
   }
   tot[b] = run;
 }
