@@ -220,13 +220,18 @@ TP_API tp_status tp_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* 
 
 /* LayerNorm over the full hidden dim ([TP-blog] §3.3): y = (x - mean) * rstd *
  * gamma + beta, biased variance, eps = 1e-5. x, y [rows, hidden]; gamma, beta
- * [hidden]; mean, rstd [rows] fp32 outputs (either may be NULL). */
+ * [hidden]; mean, rstd [rows] fp32 outputs (either may be NULL). The mean and
+ * then the variance about it are two exact passes over the row (fp32).
+ * hidden a multiple of 8 and <= 16384 (bf16) or 8192 (fp32), else
+ * TP_ERR_UNSUPPORTED. */
 TP_API tp_status tp_layernorm_fwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
                            const void* beta, void* y, float* mean, float* rstd, void* stream);
 
 /* LayerNorm on each sequence shard fused with the all-gather that follows it
- * in Megatron-SP ([TP-blog] §4.3): Y_full row j*T/n + r = LN(X_seq[j] row r).
- * mean, rstd: [T] fp32 in full-sequence order (NULL ok). */
+ * in Megatron-SP ([TP-blog] §4.3): Y_full row j*T/n + r = LN(X_seq[j] row r)
+ * (each row is read from its shard once and written to Y_full once).
+ * mean, rstd: [T] fp32 in full-sequence order (NULL ok). Limits and numerics
+ * as tp_layernorm_fwd. */
 TP_API tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, const void* const* X_seq,
                                       const void* gamma, const void* beta, void* Y_full,
                                       float* mean, float* rstd, void* stream);
