@@ -413,7 +413,7 @@ namespace {
 
 using tpi::MutPtrArray;
 
-// Rows staged in shared memory: CTA b takes rows b, b + G, b + 2G, ... and
+// Rows staged in shared memory (the backward): CTA b takes rows b, b + G, ... and
 // keeps STAGES of them in flight; a row's p shard slices arrive by bulk copy
 // (one per shard, completing on the stage's mbarrier) while the CTA works on
 // the rows before it. Thread tid owns the row's 16-byte vectors
