@@ -165,3 +165,16 @@ def test_vocab_padding_on_the_plan():
     assert q.set_vocab(100) == 120
     with pytest.raises(tp.TPError):
         q.set_vocab(0)
+
+
+@pytest.mark.parametrize("dtype,hidden", [("bf16", 1004), ("bf16", 16392), ("f32", 16384)])
+def test_layernorm_row_limits(dtype, hidden):
+    """LayerNorm rows: hidden a multiple of 8 and at most 16384 bf16 / 8192 fp32
+    columns; anything else is TP_ERR_UNSUPPORTED before any launch."""
+    p = tp.Plan(hidden, 0, 0, 1, dtype, "none")
+    try:
+        L, h = tp.lib, p.handle
+        assert L.tp_layernorm_fwd(h, 4, FAKE, FAKE, FAKE, FAKE, None, None, None) == 5
+        assert L.tp_layernorm_all_gather_seq(h, 4, 1, _arr([FAKE]), FAKE, FAKE, FAKE, None, None, None) == 5
+    finally:
+        p.close()
