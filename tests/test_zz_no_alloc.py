@@ -8,7 +8,6 @@ The new call is checked through the C ABI against the existing tp_column_sum
 (which uses a plan's cudaMalloc'd workspace) on two calls in a row, so the
 second call also shows that nothing left in the shared scratch by the first
 leaks into its result."""
-import ctypes
 
 import pytest
 import torch
