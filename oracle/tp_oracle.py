@@ -43,7 +43,7 @@ __all__ = [
     "f64", "gelu", "gelu_grad", "silu", "silu_grad", "linear",
     "mlp_fwd", "mlp_bwd", "mlp_fwd_rows", "mlp_bwd_sampled",
     "shard_rows", "shard_cols", "shard_vec", "shard_gate_up", "shard_gate_up_vec",
-    "shard_qkv", "shard_qkv_vec", "unshard_rows", "unshard_cols",
+    "shard_qkv", "shard_qkv_vec",
     "column_fwd_shard", "row_partial", "reduce_partials", "reduce_scatter_seq",
     "all_gather_seq", "row_bwd_shard", "column_bwd_shard", "bias_grad",
     "attention_fwd", "attention_fwd_rows", "attention_bwd", "layernorm_fwd", "layernorm_bwd",
@@ -228,14 +228,6 @@ def shard_vec(b, p, i):
     return b[i * n:(i + 1) * n]
 
 
-def unshard_rows(shards):
-    return np.concatenate(shards, axis=0)
-
-
-def unshard_cols(shards):
-    return np.concatenate(shards, axis=1)
-
-
 def shard_gate_up(W1, p, i):
     """[G_i; U_i] for W1 = [G; U] ([2f, h]): gate rows i*f/p.. and the same up rows.
 
@@ -249,7 +241,10 @@ def shard_gate_up(W1, p, i):
 
 
 def shard_gate_up_vec(b1, p, i):
+    """The column bias of shard i of a SwiGLU MLP, paired like its weight rows:
+    [b_gate entries i*f/p.., b_up entries i*f/p..] for b1 = [b_gate; b_up] ([2f])."""
     f = b1.shape[0] // 2
+    _check_div(f, p, "ffn")
     k = f // p
     return np.concatenate([b1[i * k:(i + 1) * k], b1[f + i * k:f + (i + 1) * k]])
 

@@ -17,14 +17,9 @@ def _rows(T, n):
     return tp_synth.sample_rows(T, n).numpy()
 
 
-def test_mlp_7b_swiglu_full_size_sampled():
-    from megatron_tensor_transformer_gemm_b200.block import TPMLP
-    T, h, f, p = 32768, 4096, 11008, 8
-    inp = tp_synth.draw_mlp(T, h, f, "swiglu", torch.bfloat16, seed=0)
-    m = TPMLP(h, f, p, "swiglu", "bf16")
-    m.load_weights(dev(inp.W1), dev(inp.W2))
-    Y = m.forward(dev(inp.X))
-    dX = m.backward(dev(inp.dY))
+def _check_mlp_7b_sampled(m, inp, T, h, f, p, Y, dX):
+    """Sampled rows of Y and dX and sampled units of dW1 and dW2 against the
+    oracle (each sample computed exactly from its definition)."""
     rows = _rows(T, 48)
     fcols = np.sort(tp_synth.sample_rows(f, 12, seed=99).numpy())
     X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
@@ -46,6 +41,21 @@ def test_mlp_7b_swiglu_full_size_sampled():
     assert_close(got_w2.T, smp["dW2_cols"].T, TOL_BF16, "dW2 sampled columns")
     from megatron_tensor_transformer_gemm_b200 import tp
     assert tp.device_status() == "TP_OK"
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["partials", "fused"])
+def test_mlp_7b_swiglu_full_size_sampled(fused):
+    """hidden 4096, ffn 11008, tokens 32768, p 8; fused: the shard sums run
+    inside the row GEMM and the column-backward dX GEMM (the launch
+    configuration bench.py times by default)."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 32768, 4096, 11008, 8
+    inp = tp_synth.draw_mlp(T, h, f, "swiglu", torch.bfloat16, seed=0)
+    m = TPMLP(h, f, p, "swiglu", "bf16", fused=fused)
+    m.load_weights(dev(inp.W1), dev(inp.W2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    _check_mlp_7b_sampled(m, inp, T, h, f, p, Y, dX)
 
 
 def _run_sp(seq, h, f, p, ln_random, seed=0):
@@ -86,24 +96,6 @@ def test_sp_mlp_full_size_sampled():
     assert_close(host(Y)[rows], ref["Y"], TOL_BF16, "Y rows")
     rb = O.sp_mlp_bwd(Xr, g64, W1f, W2f, ref, O.f64(dY[rows]))
     assert_close(host(dX)[rows], rb["dX"], TOL_BF16, "dX rows")
-
-
-def test_mlp_7b_swiglu_full_size_sampled_fused():
-    """The same full-size check with the shard sums fused into the row GEMM and
-    the column-backward dX GEMM."""
-    from megatron_tensor_transformer_gemm_b200.block import TPMLP
-    T, h, f, p = 32768, 4096, 11008, 8
-    inp = tp_synth.draw_mlp(T, h, f, "swiglu", torch.bfloat16, seed=0)
-    m = TPMLP(h, f, p, "swiglu", "bf16", fused=True)
-    m.load_weights(dev(inp.W1), dev(inp.W2))
-    Y = m.forward(dev(inp.X))
-    dX = m.backward(dev(inp.dY))
-    rows = _rows(T, 48)
-    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
-    ref = O.mlp_fwd_rows(X, W1, None, W2, None, "swiglu", rows)
-    assert_close(host(Y)[rows], ref["Y"], TOL_BF16, "Y rows")
-    smp = O.mlp_bwd_sampled(X, W1, None, W2, dY, "swiglu", rows, np.array([0, 5000, 11007]))
-    assert_close(host(dX)[rows], smp["dX_rows"], TOL_BF16, "dX rows")
 
 
 def test_sp_mlp_reduced_size_fused():

@@ -297,6 +297,35 @@ def test_overlapped_reduce_matches_sequential_bit_for_bit():
     assert torch.equal(outs[0][2], outs[1][2])
 
 
+@pytest.mark.parametrize("chunks", [2, 3])
+@pytest.mark.parametrize("act,bias", [("gelu", True), ("swiglu", False)])
+def test_overlap_chunks_vs_oracle(chunks, act, bias):
+    """f2 (token blocks, each block's reduce on a side stream under the next
+    block's GEMM) against the oracle. T = 1000 is not a multiple of the
+    128-row blocks (2 chunks: 512 + 488 rows; 3 chunks: 384 + 384 + 232)."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 1000, 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=21, bias=bias)
+    m = TPMLP(h, f, p, act, "bf16", bias=bias, overlap_chunks=chunks)
+    assert m.chunks == chunks
+    m.load_weights(dev(inp.W1), dev(inp.W2), dev(inp.b1), dev(inp.b2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    b1, b2 = (O.f64(inp.b1), O.f64(inp.b2)) if bias else (None, None)
+    ref = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    gr = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
+    assert_close(Y, ref["Y"], TOL_BF16, "Y")
+    assert_close(dX, gr["dX"], TOL_BF16, "dX")
+    for i in range(p):
+        assert_close(m.dW1[i], _shard_w1(gr["dW1"], act, p, i), TOL_BF16, f"dW1 shard {i}")
+        assert_close(m.dW2[i], O.shard_cols(gr["dW2"], p, i), TOL_BF16, f"dW2 shard {i}")
+    if bias:
+        for i in range(p):
+            assert_close(m.db1[i][None, :], O.shard_vec(gr["db1"], p, i)[None, :], TOL_BF16, f"db1 shard {i}")
+        assert_close(m.db2[None, :], gr["db2"][None, :], 1e-4, "db2")
+
+
 def test_host_step_pipeline_matches_direct_steps():
     """Three overlapped host-fed steps with different inputs give, bit for
     bit, the outputs of the same steps run directly on device tensors."""

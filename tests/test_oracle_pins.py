@@ -530,6 +530,94 @@ def test_divisibility_is_checked():
         O.shard_qkv(np.zeros((3 * 12, 12)), 3, 2, 0)
 
 
+# ------------------------------- bias gradient, gate/up bias shard, RS residual
+
+def test_bias_grad_hand_worked():
+    """A bias added to every token row receives the column sums of dY over the
+    tokens (chain rule through Y = ... + 1 b^T); integers worked by hand."""
+    dY = np.array([[1.0, 2.0, 3.0], [4.0, 5.0, 6.0], [-2.0, 0.0, 7.0]])
+    assert np.array_equal(O.bias_grad(dY), np.array([3.0, 7.0, 16.0]))
+
+
+def test_bias_grad_brute_force_and_fd():
+    T, n = 9, 5
+    dY, X, b = randn(T, n), randn(T, n), randn(1, n)
+    got = O.bias_grad(dY)
+    assert got.shape == (n,)
+    loops = [sum(dY[t, c] for t in range(T)) for c in range(n)]
+    np.testing.assert_allclose(got, loops, rtol=1e-14, atol=1e-14)
+    # d/db of sum(dY * (X + 1 b^T)) by central differences
+    _check_fd(got, lambda: float((dY * (X + b)).sum()), b, n=n)
+
+
+def test_mutant_bias_grad_mean_or_wrong_axis_fails():
+    dY = np.array([[1.0, 2.0, 3.0], [4.0, 5.0, 6.0], [-2.0, 0.0, 7.0]])
+    ref = np.array([3.0, 7.0, 16.0])
+    assert not np.array_equal(dY.mean(axis=0), ref)
+    assert not np.array_equal(dY.sum(axis=1), ref)
+
+
+def test_shard_gate_up_vec_hand_worked_and_matches_weight_rows():
+    """The bias of a SwiGLU column shard pairs gate entries i*f/p.. with the
+    same up entries, exactly like the weight rows of [G_i; U_i] (walkthrough §3.2)."""
+    b1 = np.array([10.0, 11.0, 12.0, 13.0, 20.0, 21.0, 22.0, 23.0])  # gate 10.., up 20..
+    assert np.array_equal(O.shard_gate_up_vec(b1, 2, 0), [10.0, 11.0, 20.0, 21.0])
+    assert np.array_equal(O.shard_gate_up_vec(b1, 2, 1), [12.0, 13.0, 22.0, 23.0])
+    for p in (1, 2, 4):
+        b = randn(2 * 8)
+        for i in range(p):
+            as_rows = O.shard_gate_up(b[:, None], p, i)[:, 0]
+            assert np.array_equal(O.shard_gate_up_vec(b, p, i), as_rows)
+    with pytest.raises(ValueError):
+        O.shard_gate_up_vec(np.zeros(2 * 6), 4, 0)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4])
+def test_gate_up_bias_shards_give_the_full_swiglu(p):
+    """Column shards of W1 and of its bias, each paired gate/up, reproduce the
+    full SwiGLU activation's columns i*f/p.. of shard i."""
+    T, h, f = 5, 6, 8
+    X, W1, b1 = randn(T, h), randn(2 * f, h), randn(2 * f)
+    Z = X @ W1.T + b1[None, :]
+    H_full = O.silu(Z[:, :f]) * Z[:, f:]
+    k = f // p
+    for i in range(p):
+        _, H_i = O.column_fwd_shard(X, O.shard_gate_up(W1, p, i), O.shard_gate_up_vec(b1, p, i), "swiglu")
+        np.testing.assert_allclose(H_i, H_full[:, i * k:(i + 1) * k], rtol=1e-13, atol=1e-14)
+
+
+def test_reduce_scatter_residual_hand_worked():
+    """Each sequence shard j adds ITS residual rows after the sum and the bias
+    (walkthrough §4.3); integers worked by hand, T = 4 rows over n = 2 shards."""
+    P0 = np.array([[1.0, 2.0], [3.0, 4.0], [5.0, 6.0], [7.0, 8.0]])
+    P1 = np.array([[10.0, 20.0], [30.0, 40.0], [50.0, 60.0], [70.0, 80.0]])
+    b = np.array([100.0, 200.0])
+    r = [np.array([[1000.0, 2000.0], [3000.0, 4000.0]]),
+         np.array([[5000.0, 6000.0], [7000.0, 8000.0]])]
+    out = O.reduce_scatter_seq([P0, P1], b, r)
+    assert np.array_equal(out[0], [[1111.0, 2222.0], [3133.0, 4244.0]])
+    assert np.array_equal(out[1], [[5155.0, 6266.0], [7177.0, 8288.0]])
+
+
+@pytest.mark.parametrize("p", [1, 2, 4, 8])
+def test_reduce_scatter_residual_brute_force(p):
+    """Integer-valued partials, bias and residual shards: element by element in
+    pure Python, shard j row r = sum_i P_i[j*t + r] + b + R_j[r]."""
+    t, h = 3, 4
+    P, b, _ = tp_synth.draw_partials(p, p * t, h, torch.float32, integer_valued=True)
+    P, b = [O.f64(x) for x in P], O.f64(b)
+    R = [rng.integers(-8, 9, (t, h)).astype(np.float64) for _ in range(p)]
+    out = O.reduce_scatter_seq(P, b, R)
+    for j in range(p):
+        for r in range(t):
+            for c in range(h):
+                want = sum(P[i][j * t + r, c] for i in range(p)) + b[c] + R[j][r, c]
+                assert out[j][r, c] == want
+    if p > 1:  # a residual taken from the wrong shard gives a different result
+        bad = O.reduce_scatter_seq(P, b, R[::-1])
+        assert any(not np.array_equal(x, y) for x, y in zip(bad, out))
+
+
 # ------------------------------------------------ mutation checks (plant bugs)
 
 def _mut_gelu_tanh(z):
