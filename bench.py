@@ -62,6 +62,20 @@ def mlp_flops(T, h, f):
     return 3.0 * (2.0 * T * h * 2 * f + 2.0 * T * f * h)
 
 
+def gemm_algorithmic_bytes(T, h, f):
+    """Bytes each of the six GEMM launches of the fused step must move at least
+    once (bf16): its operands read once and its outputs written once.
+      column fwd + SwiGLU: X, W1 -> Z, H;   row fwd (shard sum fused): H, W2 -> Y;
+      row bwd dgrad + dSwiGLU: dY, W2, Z -> dZ;   dW2: dY, H -> dW2;
+      dW1: dZ, X -> dW1;   column bwd dX (shard sum fused): dZ, W1 -> dX."""
+    X = Y = dY = dX = T * h * 2
+    Z = dZ = T * 2 * f * 2
+    H = T * f * 2
+    W1 = dW1 = 2 * f * h * 2
+    W2 = dW2 = h * f * 2
+    return [X + W1 + Z + H, H + W2 + Y, dY + W2 + Z + dZ, dY + H + dW2, dZ + X + dW1, dZ + W1 + dX]
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
@@ -310,7 +324,6 @@ def run_ours(args, world, rank, local):
     gemm_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in gemm_ev)
     n_gemm_launches = n_gemm[0]
     gemm_tflops = flops * args.steps / (gemm_ms / 1e3) / 1e12
-    peak_t = peaks["bf16_tflops_sustained"]
     red_bytes_launch = P * T * HIDDEN * 2 + T * HIDDEN * 2
     if red_ev:
         red_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in red_ev)
@@ -325,11 +338,12 @@ def run_ours(args, world, rank, local):
     e2e = None
     if not args.skip_e2e:
         e2e = run_e2e(m, X_h, dY_h, T, flops, args, world, stream)
+    coll = None if args.skip_collectives else time_sp_collectives(peaks, stream, rank)
     status = tp.device_status()
     if rank != 0:
         return 0
-    return report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t,
-                  red_gbs, red_bytes, e2e, launches, clk, status, red_where)
+    return report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks,
+                  red_gbs, red_bytes, e2e, launches, clk, status, red_where, coll)
 
 
 def time_standalone_reduce(pl, T, steps, stream):
@@ -353,6 +367,65 @@ def time_standalone_reduce(pl, T, steps, stream):
     del Pt, Y
     torch.cuda.empty_cache()
     return gbs
+
+
+def time_sp_collectives(peaks, stream, rank):
+    """HBM GB/s of the Megatron-SP collectives at the SP workload's sizes (seq
+    8192, hidden 8192, p 8, bf16): S4' reduce-scatter of the row partials, S9
+    all-gather of dY, S1 LayerNorm fused with the sequence all-gather. Each is
+    timed as a replayed CUDA graph of 10 launches (algorithmic bytes / device
+    time); every buffer set is larger than L2."""
+    import torch
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.block import CapturedStep
+    T, h, p = 8192, 8192, 8
+    t = T // p
+    g = torch.Generator(device="cpu").manual_seed(500 + rank)
+    plan = tp.Plan(h, 0, 0, p, "bf16", "none")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    bf = torch.bfloat16
+    parts = [torch.randn(T, h, generator=g).to(bf).to(dev) for _ in range(p)]
+    outs = [torch.empty(t, h, dtype=bf, device=dev) for _ in range(p)]
+    full = torch.empty(T, h, dtype=bf, device=dev)
+    xs = [torch.randn(t, h, generator=g).to(bf).to(dev) for _ in range(p)]
+    gam = (1 + 0.1 * torch.randn(h, generator=g)).to(bf).to(dev)
+    bet = (0.1 * torch.randn(h, generator=g)).to(bf).to(dev)
+    mean = torch.empty(T, dtype=torch.float32, device=dev)
+    rstd = torch.empty(T, dtype=torch.float32, device=dev)
+    cases = [
+        ("reduce_scatter", "reduce_kernel (S4' reduce-scatter of 8 partials [8192, 8192])",
+         lambda: plan.reduce_scatter_seq(T, parts, None, None, outs), p * T * h * 2 + T * h * 2),
+        ("all_gather", "gather_kernel (S9 all-gather of dY, 8 x [1024, 8192])",
+         lambda: plan.reduce_scatter_seq_bwd(T, outs, full), 2 * T * h * 2),
+        ("ln_all_gather", "ln_fwd_kernel (S1 LayerNorm fused with the sequence all-gather)",
+         lambda: plan.layernorm_all_gather_seq(T, xs, gam, bet, full, mean, rstd), 2 * T * h * 2 + T * 8),
+    ]
+    res = {}
+    reps = 10
+    for key, kname, fn, nbytes in cases:
+        def rep(fn=fn):
+            for _ in range(reps):
+                fn()
+        graph = CapturedStep(rep)
+        for _ in range(2):
+            graph()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            graph()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sec = e0.elapsed_time(e1) / 1e3 / (3 * reps)
+        gbs = nbytes / sec / 1e9
+        res[key] = {"kernel": kname, "achieved": gbs, "unit": "GB/s", "us": sec * 1e6,
+                    "bytes_per_launch": nbytes, "frac": gbs / peaks["hbm_gbs"],
+                    "frac_of_8TBs": gbs / 8000.0}
+        del graph
+    del parts, outs, full, xs
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(m, X_h, dY_h, T, flops, args, world, stream):
@@ -408,12 +481,17 @@ def measured_traffic(T, variant):
         return None
     if d.get("tokens") != T or d.get("variant") != variant or d.get("source_sha256") != gemm_source_hash():
         return None
-    return d.get("bytes_per_launch")
+    return d.get("bytes_per_launch"), d.get("per_launch_bytes")
 
 
-def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, peak_t, red_gbs,
-           red_bytes, e2e, launches, clk, status, red_where):
-    traffic = measured_traffic(T, args.variant)
+def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, red_gbs,
+           red_bytes, e2e, launches, clk, status, red_where, coll):
+    traffic, per_launch = measured_traffic(T, args.variant) or (None, None)
+    alg = gemm_algorithmic_bytes(T, HIDDEN, FFN)
+    alg_mean = sum(alg) / len(alg)
+    ratios = None
+    if per_launch and len(per_launch) == len(alg) and args.variant == "fused":
+        ratios = [round(m / a, 2) for m, a in zip(per_launch, alg)]
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(rows=args.cpu_rows)
@@ -429,16 +507,20 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
                    "variant": args.variant,
                    "l2": "inputs larger than L2 (X and dY 268 MB each); no flush"},
         "roofline": {"bound": "tensor", "kernel": "tp_gemm_kernel (tcgen05)",
-                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / peak_t,
-                     "peak_kind": f"bf16 sustained ({peaks['source']})",
-                     "frac_of_burst_peak": gemm_tflops / peaks["bf16_tflops"],
-                     "launches_timed": n_gemm_launches, "traffic": traffic},
+                     "achieved": gemm_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peaks["bf16_tflops"],
+                     "peak_kind": f"bf16 burst ({peaks['source']}): the timed region lasts under a second",
+                     "frac_of_sustained_peak": gemm_tflops / peaks["bf16_tflops_sustained"],
+                     "launches_timed": n_gemm_launches, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg_mean,
+                     "traffic_ratio": None if traffic is None else traffic / alg_mean,
+                     "traffic_ratio_per_launch": ratios},
         "reduce": {"kernel": "reduce_kernel", "achieved": red_gbs, "unit": "GB/s",
                    "peak": peaks["hbm_gbs"], "frac": red_gbs / peaks["hbm_gbs"],
                    "peak_kind": f"HBM copy ({peaks['source']})",
                    "frac_of_8TBs": red_gbs / 8000.0, "bytes_per_launch": red_bytes,
                    "measured": red_where},
+        "collectives": coll,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
@@ -759,6 +841,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=TOKENS,
                     help="token rows (default 8x4096; smaller values are for profiling only)")
     ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--skip-collectives", action="store_true",
+                    help="skip the Megatron-SP collective GB/s measurements")
     ap.add_argument("--variant", choices=["fused", "partials", "overlap"], default="fused",
                     help="sum over shards inside the GEMMs (fused), via p partials + reduce, "
                          "or partials with each token block's reduce overlapped with the next "

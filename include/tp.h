@@ -103,10 +103,19 @@ typedef enum { TP_NORM_LAYER = 0, TP_NORM_RMS = 1 } tp_norm_kind;
  * p in [1, TP_MAX_SHARDS]; hidden % p, heads % p, hidden % heads, ffn % p
  * (and the doubled gate+up column count 2*ffn % p for SwiGLU) all zero.
  * ffn may be 0 (attention-only plan); heads may be 0 (MLP-only plan).
+ *   partial_dtype: element type of the full-shape partial sums that
+ *     tp_row_fwd_partial and tp_column_bwd write and tp_reduce_partials,
+ *     tp_reduce_scatter_seq and tp_all_gather_seq_bwd read. Either `dtype`
+ *     (the partials travel in the activation type, as an all-reduce of the
+ *     layer output would carry them) or TP_F32 (twice the bytes, but each
+ *     partial reaches the fp32 sum unrounded: [TP-wiki] notes that the
+ *     all-reduce changes the floating-point summation, and this bounds the
+ *     change to the one final rounding). TP_F32 plans take TP_F32 only;
+ *     anything else returns TP_ERR_DTYPE.
  * Allocates no device memory. Returns TP_ERR_DIVISIBILITY naming the failing
  * dimension (tp_last_error), TP_ERR_ARG for non-positive sizes. */
 TP_API tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype,
-                         tp_act act, tp_plan** out);
+                         tp_act act, tp_dtype partial_dtype, tp_plan** out);
 TP_API void tp_plan_destroy(tp_plan* plan);
 
 /* Vocab of the embedding / output head ([TP-blog] §6.2: the vocab is padded
@@ -123,10 +132,25 @@ TP_API tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n);
 TP_API const char* tp_status_string(tp_status s);
 TP_API const char* tp_last_error(void);
 
-/* Synchronise `stream`, read the device status word of the current device,
- * store it in *device_status (TP_OK, TP_ERR_TIMEOUT if a kernel wait gave up,
- * TP_ERR_ARG if a kernel met an out-of-range token id / label) and clear it. */
-TP_API tp_status tp_get_device_status(void* stream, int* device_status);
+/* Device-side error report ([TP-blog] §6: fail fast and say why). Synchronises
+ * `stream`, reads the device status word of the current device, clears it and
+ * returns what it held: TP_OK (nothing happened), TP_ERR_TIMEOUT (a kernel's
+ * bounded wait gave up; the kernel returned early and its outputs are
+ * undefined) or TP_ERR_ARG (a kernel met an out-of-range token id or label).
+ * The word is per device and shared by every plan, so `plan` may be NULL; a
+ * non-NULL plan is only validated. If the read itself fails the call returns
+ * TP_ERR_CUDA or TP_ERR_NO_DEVICE and leaves the word unchanged. */
+TP_API tp_status tp_get_device_status(const tp_plan* plan, void* stream);
+
+/* Self-test of the device-side failure path ([TP-blog] §6: fail fast, never
+ * hang). Launches one CTA whose single thread waits, through the same bounded
+ * wait every pipelined kernel of the library uses, on an mbarrier that no one
+ * will arrive at. After limit_ns nanoseconds (0 < limit_ns <= 1e9, else
+ * TP_ERR_ARG) the wait gives up, sets TP_ERR_TIMEOUT in the device status
+ * word (read it with tp_get_device_status) and the kernel returns; the
+ * context stays usable. gave_up (device int*, NULL ok) receives 1. Faults,
+ * traps and hangs nothing. */
+TP_API tp_status tp_selftest_wait_timeout(int64_t limit_ns, int* gave_up, void* stream);
 
 /* Number of kernel launches this thread has issued through the library
  * since the last reset (host counter; used to report launch counts). */
@@ -176,7 +200,8 @@ TP_API tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const v
 
 /* Row-parallel GEMM of every shard: P[i] [T, hidden] = H[i] W[i]^T, the
  * full-shape partial sums, with NO bias ([TP-blog] §2.2, [TP-wiki] XB = X_1B_1 +
- * X_2B_2). H[i] is [T, ffn/p] (TP_MLP) or [T, h/p] (TP_OUTPROJ); W[i] the row shard. */
+ * X_2B_2). H[i] is [T, ffn/p] (TP_MLP) or [T, h/p] (TP_OUTPROJ); W[i] the row
+ * shard; P[i] is stored in the plan's partial dtype. */
 TP_API tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
                              const void* const* W, void* const* P, void* stream);
 
@@ -201,14 +226,16 @@ TP_API tp_status tp_row_fwd_reduce_scatter_seq(tp_plan* plan, tp_which which, in
 
 /* The all-reduce of the row layer, done locally: Y = sum_{i<n} P[i] (fp32, in
  * order 0..n-1), then + bias once (NULL ok), then + residual (NULL ok).
- * [TP-blog] §2.2, [TP-basics] (bias once, after the sum). P[i], residual, Y
- * are [T, hidden]; bias [hidden]. Y may alias residual. */
+ * [TP-blog] §2.2, [TP-basics] (bias once, after the sum). P[i] [T, hidden] in
+ * the plan's partial dtype; residual, Y [T, hidden] and bias [hidden] in the
+ * plan dtype. Y may alias residual. */
 TP_API tp_status tp_reduce_partials(tp_plan* plan, int64_t T, int n, const void* const* P,
                              const void* bias, const void* residual, void* Y, void* stream);
 
 /* Sequence-parallel form of the reduction ([TP-blog] §4.3, [TP-wiki] Megatron-SP):
  * Y_seq[j] [T/n, hidden] = rows [j*T/n, (j+1)*T/n) of (sum_i P[i] + bias),
- * plus residual_seq[j] (NULL array ok). T % n must be 0. */
+ * plus residual_seq[j] (NULL array ok). T % n must be 0. Types as
+ * tp_reduce_partials (P[i] in the partial dtype). */
 TP_API tp_status tp_reduce_scatter_seq(tp_plan* plan, int64_t T, int n, const void* const* P,
                                 const void* bias, const void* const* residual_seq,
                                 void* const* Y_seq, void* stream);
@@ -311,7 +338,8 @@ TP_API tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void
  *   X [T, hidden]; dZ[i] the gradient of shard i's pre-activation output;
  *   W[i] the column shard. dW[i] = dZ[i]^T X (NULL array skips); dbias[i] fp32
  *   = sum over tokens of dZ[i] (NULL array skips); dX_partials[i] [T, hidden] =
- *   dZ[i] W[i], to be summed by tp_reduce_partials (or tp_all_gather_seq_bwd). */
+ *   dZ[i] W[i] in the plan's partial dtype, to be summed by tp_reduce_partials
+ *   (or tp_all_gather_seq_bwd). */
 TP_API tp_status tp_column_bwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
                         const void* const* dZ, const void* const* W, void* const* dW,
                         float* const* dbias, void* const* dX_partials, void* stream);
@@ -339,14 +367,21 @@ TP_API tp_status tp_reduce_scatter_seq_bwd(tp_plan* plan, int64_t T, int n, cons
                                     void* dY_full, void* stream);
 
 /* Backward of tp_all_gather_seq: the reduce-scatter of the n full-shape dX
- * partials into sequence shards dX_seq[j] [T/n, hidden]. */
+ * partials (partial dtype) into sequence shards dX_seq[j] [T/n, hidden]
+ * (plan dtype). */
 TP_API tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const void* const* dX_partials,
                                 void* const* dX_seq, void* stream);
 
-/* LayerNorm backward: dx [rows, hidden] (plan dtype); dgamma, dbeta [hidden]
- * fp32 (sums over the rows, deterministic; when accumulate != 0 they are
- * added to the existing contents, so shards can be summed). mean/rstd from
- * the forward. Uses the plan's device workspace for per-CTA partials. */
+/* LayerNorm backward ([TP-blog] §3.3: the statistics span the whole hidden
+ * dim, so dx of a row needs the row's two reductions; §4.3 / [TP-wiki]
+ * Megatron-SP: LayerNorm runs on sequence shards with replicated gamma and
+ * beta, so their gradients are sums over every shard's rows).
+ * dx [rows, hidden] (plan dtype) = rstd * (g - mean_h(g) - xhat * mean_h(g *
+ * xhat)) with g = dy * gamma and xhat = (x - mean) * rstd; dgamma = sum_rows
+ * dy * xhat, dbeta = sum_rows dy, [hidden] fp32 (deterministic; when
+ * accumulate != 0 they are added to the existing contents, so the sequence
+ * shards' sums can be chained). mean/rstd from the forward. Uses the plan's
+ * device workspace for per-CTA partials. */
 TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
                            const void* dy, const float* mean, const float* rstd, void* dx,
                            float* dgamma, float* dbeta, int accumulate, void* stream);
@@ -362,10 +397,14 @@ TP_API tp_status tp_norm_sharded_bwd(tp_plan* plan, tp_norm_kind kind, int64_t r
                                      void* const* dX, float* const* dgamma, float* const* dbeta,
                                      void* stream);
 
-/* Attention backward of each shard's local heads: from QKV[i], O[i], dO[i]
- * and LSE[i] of the forward, writes dQKV[i] [seq*batch, 3h/p] = [dQ|dK|dV].
+/* Attention backward of each shard's local heads ([TP-blog] §3.1: a shard's
+ * attention touches only its own whole heads over the full sequence, so the
+ * backward, like the forward, has no cross-shard step; the shard sum follows
+ * in the QKV column backward). From QKV[i], O[i], dO[i] and LSE[i] of the
+ * forward, writes dQKV[i] [seq*batch, 3h/p] = [dQ|dK|dV], the chain rule of
+ * softmax(Q K^T / sqrt(d), causal) V with P recomputed from LSE:
  * dV = P^T dO; dS = P * (dO V^T - rowsum(dO * O)); dQ = dS K / sqrt(d);
- * dK = dS^T Q / sqrt(d). */
+ * dK = dS^T Q / sqrt(d). bf16 plans, head_dim 64 or 128. */
 TP_API tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void* const* QKV,
                            const void* const* O, const void* const* dO,
                            const float* const* LSE, void* const* dQKV, void* stream);
@@ -388,12 +427,21 @@ TP_API tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const 
  *     number of row splits (each split needs cols floats).
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     stream capture. Under CUDA's lazy module loading that first call is
+ *     also where the library's module, and with it the array, is loaded onto
+ *     the device: the driver reserves the 2 MiB then, and the call may
+ *     synchronise. A caller that needs no allocation at all inside some
+ *     section makes one call first (rows = 0 is enough: it writes zeros, or
+ *     nothing in accumulate mode, to out) before entering it.
+ *   - x must be dense: row r starts at x + r * cols (no leading dimension).
+ *   - The cached address belongs to the device's current context: calls
+ *     after cudaDeviceReset in the same process are not supported.
  *   - Every call shares the one array, so calls that overlap on the GPU (two
  *     streams, or two host threads) race and corrupt each other's sums:
  *     serialise them. Each call overwrites every scratch entry it reads, so
  *     nothing from an earlier call leaks into a later one.
- *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call
+ *     (beyond the module load of the first call, above). */
 TP_API tp_status tp_column_sum_static(int64_t rows, int64_t cols, tp_dtype dtype, const void* x,
                                       float* out, int accumulate, void* stream);
 

@@ -11,6 +11,7 @@
 #include <tuple>
 #include <new>
 
+#include "tp_device.cuh"
 #include "tp_internal.h"
 
 namespace {
@@ -25,6 +26,22 @@ std::mutex g_status_mu;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 }  // namespace
+
+namespace tp_selftest {
+// One thread waits, through the same bounded wait the pipelined kernels use,
+// on an mbarrier that expects one arrival which never comes: the wait gives
+// up after limit_ns, sets the status word and the kernel returns.
+__global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns, int* gave_up) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  tpd::mbar_init(&bar, 1);
+  abort_flag = 0;
+  tpd::fence_barrier_init();
+  const bool ok = tpd::mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  if (gave_up) *gave_up = ok ? 0 : 1;
+}
+}  // namespace tp_selftest
 
 namespace tpi {
 
@@ -268,7 +285,7 @@ uint64_t tp_launch_count(int reset) {
 }
 
 tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, tp_act act,
-                         tp_plan** out) {
+                         tp_dtype partial_dtype, tp_plan** out) {
   if (!out) return fail(TP_ERR_ARG, "out is NULL");
   *out = nullptr;
   if (p < 1 || p > TP_MAX_SHARDS)
@@ -276,6 +293,9 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   if (hidden <= 0) return fail(TP_ERR_ARG, "hidden = %d must be positive", hidden);
   if (ffn < 0 || heads < 0) return fail(TP_ERR_ARG, "ffn and heads must be >= 0");
   if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_ERR_DTYPE, "unknown dtype %d", dtype);
+  if (partial_dtype != dtype && partial_dtype != TP_F32)
+    return fail(TP_ERR_DTYPE, "partial dtype %d: the partials are stored in the plan dtype or in fp32",
+                partial_dtype);
   if (act != TP_ACT_NONE && act != TP_ACT_GELU && act != TP_ACT_SWIGLU)
     return fail(TP_ERR_ARG, "unknown activation %d", act);
   if (hidden % p) return fail(TP_ERR_DIVISIBILITY, "hidden = %d is not divisible by p = %d", hidden, p);
@@ -301,6 +321,7 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   plan->vocab = 0;
   plan->vocab_padded = 0;
   plan->dtype = dtype;
+  plan->partial_dtype = partial_dtype;
   plan->act = act;
   plan->ws = nullptr;
   plan->ws_bytes = 0;
@@ -329,8 +350,9 @@ tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n) {
   const int p = plan->p, h = plan->hidden, f = plan->ffn;
   const char* act = plan->act == TP_ACT_GELU ? "gelu" : plan->act == TP_ACT_SWIGLU ? "swiglu" : "none";
   int w = snprintf(buf, n,
-                   "tp_plan: hidden=%d ffn=%d heads=%d head_dim=%d p=%d dtype=%s act=%s\n", h, f,
-                   plan->heads, plan->head_dim, p, plan->dtype == TP_BF16 ? "bf16" : "f32", act);
+                   "tp_plan: hidden=%d ffn=%d heads=%d head_dim=%d p=%d dtype=%s partials=%s act=%s\n",
+                   h, f, plan->heads, plan->head_dim, p, plan->dtype == TP_BF16 ? "bf16" : "f32",
+                   plan->partial_dtype == TP_BF16 ? "bf16" : "f32", act);
   auto add = [&](const char* fmt, auto... args) {
     if (w >= 0 && static_cast<size_t>(w) < n) w += snprintf(buf + w, n - w, fmt, args...);
   };
@@ -352,8 +374,8 @@ tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n) {
   return TP_OK;
 }
 
-tp_status tp_get_device_status(void* stream, int* device_status) {
-  if (!device_status) return fail(TP_ERR_ARG, "device_status is NULL");
+tp_status tp_get_device_status(const tp_plan* plan, void* stream) {
+  (void)plan;  // the word is per device, shared by every plan
   unsigned* addr = nullptr;
   TP_TRY(device_status_word(&addr));
   unsigned v = 0;
@@ -361,8 +383,20 @@ tp_status tp_get_device_status(void* stream, int* device_status) {
   TP_TRY(cuda_status(cudaMemcpy(&v, addr, sizeof(v), cudaMemcpyDeviceToHost), "read status"));
   unsigned zero = 0;
   TP_TRY(cuda_status(cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status"));
-  *device_status = (v & 1u) ? TP_ERR_TIMEOUT : (v & 2u) ? TP_ERR_ARG : TP_OK;
+  if (v & 1u) return fail(TP_ERR_TIMEOUT, "a kernel's bounded wait gave up (status word 0x%x)", v);
+  if (v & 2u) return fail(TP_ERR_ARG, "a kernel met an out-of-range token id or label (status word 0x%x)", v);
   return TP_OK;
+}
+
+tp_status tp_selftest_wait_timeout(int64_t limit_ns, int* gave_up, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 1000000000LL)
+    return fail(TP_ERR_ARG, "limit_ns = %lld outside (0, 1e9]", (long long)limit_ns);
+  if (gave_up && (reinterpret_cast<uintptr_t>(gave_up) & 3u))
+    return fail(TP_ERR_ALIGN, "gave_up is not 4-byte aligned");
+  unsigned* addr = nullptr;
+  TP_TRY(device_status_word(&addr));
+  tp_selftest::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(addr, static_cast<uint64_t>(limit_ns), gave_up);
+  return after_launch("selftest_wait_timeout");
 }
 
 // ------------------------------------------------------------------ sharding
@@ -600,12 +634,12 @@ tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const voi
   TP_TRY(check_ptrs(W, p, "W", false));
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(P), p, "P", false));
   TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
-  TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  TP_TRY(check_row_bytes(h, plan->partial_dtype, "hidden"));
   if (T == 0) return TP_OK;
   GemmBatch b{};
   b.n = p;
   b.epi = EPI_STORE;
-  b.out_f32 = plan->dtype == TP_F32;
+  b.out_f32 = plan->partial_dtype == TP_F32;
   for (int i = 0; i < p; ++i) {
     GemmProblem& g = b.g[i];
     g.M = static_cast<int>(T);
@@ -704,6 +738,7 @@ static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* cons
   if (bias) TP_TRY(check_ptr(bias, "bias"));
   if (residual) TP_TRY(check_ptr(residual, "residual"));
   TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  TP_TRY(check_row_bytes(h, plan->partial_dtype, "hidden (partials)"));
   if (scatter) {
     if (T % n) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by n = %d", (long long)T, n);
     TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Y_seq), n, "Y_seq", false));
@@ -721,8 +756,8 @@ static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* cons
     out.p[0] = Y;
   }
   return launch_reduce(to_arr(P, n), n, bias, residual, to_arr(residual_seq, n),
-                       scatter && residual_seq != nullptr, out, scatter, nout, T, h, plan->dtype,
-                       st);
+                       scatter && residual_seq != nullptr, out, scatter, nout, T, h,
+                       plan->partial_dtype, plan->dtype, st);
 }
 
 tp_status tp_reduce_partials(tp_plan* plan, int64_t T, int n, const void* const* P,
@@ -1105,6 +1140,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   if (dW) TP_TRY(check_ptr(X, "X"));
   TP_TRY(check_row_bytes(n, plan->dtype, "dZ_i width"));
   TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
+  if (mode == 0) TP_TRY(check_row_bytes(h, plan->partial_dtype, "hidden (dX partials)"));
   if (T == 0) return TP_OK;
   if (dW) {
     // dW_i [n, h] = dZ_i^T X: A(m, t) = dZ_i[t, m] (MN-major), B(c, t) = X[t, c] (MN-major).
@@ -1135,7 +1171,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     d.a_mn = false;
     d.b_mn = true;
     d.epi = EPI_STORE;
-    d.out_f32 = plan->dtype == TP_F32;
+    d.out_f32 = (mode == 0 ? plan->partial_dtype : plan->dtype) == TP_F32;
     d.kcat = mode != 0;
     for (int i = 0; i < p; ++i) {
       GemmProblem& g = d.g[i];

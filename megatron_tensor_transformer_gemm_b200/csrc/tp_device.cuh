@@ -66,17 +66,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete. On time-out
-// (or when another thread of the CTA already gave up, *abort != 0) it sets
-// *abort and the device status word and returns false.
+// (limit_ns of wall time, or kWaitLimitPolls polls), or when another thread of
+// the CTA already gave up (*abort != 0), it sets *abort and the device status
+// word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned* status) {
+                                          unsigned* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   for (uint32_t it = 1; it < kWaitLimitPolls; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) break;
+      if (globaltimer() - t0 > limit_ns) break;
     }
   }
   *abort = 1;

@@ -17,6 +17,7 @@ struct tp_plan {
   int vocab;         // 0 until tp_plan_set_vocab
   int vocab_padded;  // multiple of 8 * p
   tp_dtype dtype;
+  tp_dtype partial_dtype;  // element type of the full-shape partial sums
   tp_act act;
   // Device scratch, allocated on first need (cudaMalloc), grown on demand.
   void* ws;
@@ -65,10 +66,11 @@ struct MutPtrArray {
 // Element-wise / copy / reduction kernels (tp_reduce.cu).
 tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int64_t rows,
                          int64_t cols, size_t esize, cudaStream_t st);
+// P[i] are of type `pt`; bias, residual and the outputs of type `dt`.
 tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
                         const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out,
-                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype dt,
-                        cudaStream_t st);
+                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype pt,
+                        tp_dtype dt, cudaStream_t st);
 tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
                         tp_dtype dt, cudaStream_t st);
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,

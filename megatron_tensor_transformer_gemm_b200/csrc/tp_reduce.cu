@@ -20,17 +20,24 @@ using tpi::PtrArray;
 
 constexpr int kThreads = 256;
 
+// SM count of the current device, queried once per device and cached.
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (cached[dev] == 0) {
+    int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       n = 148;
     }
+    cached[dev] = n;
   }
-  return n;
+  return cached[dev];
 }
 
 // 16-byte vector <-> 8 (bf16) or 4 (fp32) floats.
@@ -104,36 +111,45 @@ __device__ __forceinline__ void reduce_finish(float (&a)[Vec<T>::N], const float
 // Y[rows] = sum_{i<n} P[i] in order 0..n-1 (fp32), + bias once, + residual.
 // out.p[0] is the full output when scatter == 0, else out.p[j] holds rows
 // [j*rows_per_out, (j+1)*rows_per_out) (the sequence-parallel reduce-scatter).
-// Each thread walks two rows per step and issues all 2n loads before using
-// any, so 2n 16-byte loads per thread are in flight.
-template <typename T, int NMAX>
+// A thread owns one 16-byte vector of the output (V elements of OT); the
+// partials are of type PT, so each contributes W = V * sizeof(PT) / 16
+// 16-byte loads per row (W = 2 for fp32 partials of a bf16 output). Each
+// thread walks two rows per step and issues all 2nW loads before using any.
+template <typename PT, typename OT, int NMAX>
 __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ PtrArray P, int n,
-                                                          const T* bias, const T* residual,
+                                                          const OT* bias, const OT* residual,
                                                           const __grid_constant__ PtrArray res_seq,
                                                           int res_is_seq,
                                                           const __grid_constant__ MutPtrArray out,
                                                           int scatter, int64_t rows, int64_t vpr,
                                                           int64_t rows_per_out) {
-  constexpr int V = Vec<T>::N;
+  constexpr int V = Vec<OT>::N;
+  constexpr int W = V * static_cast<int>(sizeof(PT)) / 16;
+  constexpr int VP = Vec<PT>::N;  // partial elements per 16-byte load
+  static_assert(W * VP == V, "a partial vector spans whole 16-byte loads");
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (cv >= vpr) return;
   const int64_t cols = vpr * V;
   float b[V];
 #pragma unroll
   for (int k = 0; k < V; ++k) b[k] = 0.f;
-  if (bias) Vec<T>::load(ld_keep(bias + cv * V), b);
+  if (bias) Vec<OT>::load(ld_keep(bias + cv * V), b);
   const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.y;
   for (int64_t r = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; r < rows;
        r += 2 * stride) {
     const int64_t r2 = r + stride;
     const bool two = r2 < rows;
     const int64_t off1 = r * cols + cv * V, off2 = (two ? r2 : r) * cols + cv * V;
-    uint4 u1[NMAX], u2[NMAX];
+    uint4 u1[NMAX][W], u2[NMAX][W];
 #pragma unroll
     for (int i = 0; i < NMAX; ++i) {
       if (i < n) {
-        u1[i] = ld_stream(static_cast<const T*>(P.p[i]) + off1);
-        if (two) u2[i] = ld_stream(static_cast<const T*>(P.p[i]) + off2);
+        const PT* base = static_cast<const PT*>(P.p[i]);
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          u1[i][w] = ld_stream(base + off1 + w * VP);
+          if (two) u2[i][w] = ld_stream(base + off2 + w * VP);
+        }
       }
     }
     float a1[V], a2[V];
@@ -142,20 +158,23 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
 #pragma unroll
     for (int i = 0; i < NMAX; ++i) {
       if (i < n) {
-        float f[V];
-        Vec<T>::load(u1[i], f);
 #pragma unroll
-        for (int k = 0; k < V; ++k) a1[k] += f[k];
-        if (two) {
-          Vec<T>::load(u2[i], f);
+        for (int w = 0; w < W; ++w) {
+          float f[VP];
+          Vec<PT>::load(u1[i][w], f);
 #pragma unroll
-          for (int k = 0; k < V; ++k) a2[k] += f[k];
+          for (int k = 0; k < VP; ++k) a1[w * VP + k] += f[k];
+          if (two) {
+            Vec<PT>::load(u2[i][w], f);
+#pragma unroll
+            for (int k = 0; k < VP; ++k) a2[w * VP + k] += f[k];
+          }
         }
       }
     }
-    reduce_finish<T>(a1, b, r, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
+    reduce_finish<OT>(a1, b, r, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
     if (two)
-      reduce_finish<T>(a2, b, r2, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
+      reduce_finish<OT>(a2, b, r2, cols, cv, residual, res_seq, res_is_seq, out, scatter, rows_per_out);
   }
 }
 
@@ -292,8 +311,8 @@ tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst
 
 tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* residual,
                         const PtrArray& residual_seq, bool res_seq, const MutPtrArray& out,
-                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype dt,
-                        cudaStream_t st) {
+                        bool out_is_seq, int nout, int64_t T, int64_t cols, tp_dtype pt,
+                        tp_dtype dt, cudaStream_t st) {
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   dim3 grid, block;
@@ -301,20 +320,23 @@ tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* 
   const int64_t rows_per_out = T / nout;
   const int rs = res_seq ? 1 : 0;
   const int scatter = out_is_seq ? 1 : 0;
-#define TP_REDUCE_LAUNCH(T, NM)                                                                  \
-  reduce_kernel<T, NM><<<grid, block, 0, st>>>(P, n, static_cast<const T*>(bias),                \
-                                               static_cast<const T*>(residual), residual_seq, rs, \
-                                               out, scatter, T_rows, vpr, rows_per_out)
   const int64_t T_rows = T;
-  if (dt == TP_BF16) {
-    if (n <= 4) TP_REDUCE_LAUNCH(__nv_bfloat16, 4);
-    else if (n <= 8) TP_REDUCE_LAUNCH(__nv_bfloat16, 8);
-    else TP_REDUCE_LAUNCH(__nv_bfloat16, TP_MAX_SHARDS);
-  } else {
-    if (n <= 4) TP_REDUCE_LAUNCH(float, 4);
-    else if (n <= 8) TP_REDUCE_LAUNCH(float, 8);
-    else TP_REDUCE_LAUNCH(float, TP_MAX_SHARDS);
-  }
+#define TP_REDUCE_LAUNCH(PT, OT, NM)                                                            \
+  reduce_kernel<PT, OT, NM><<<grid, block, 0, st>>>(P, n, static_cast<const OT*>(bias),          \
+                                                    static_cast<const OT*>(residual),            \
+                                                    residual_seq, rs, out, scatter, T_rows, vpr, \
+                                                    rows_per_out)
+#define TP_REDUCE_BY_N(PT, OT)                    \
+  do {                                            \
+    if (n <= 4) TP_REDUCE_LAUNCH(PT, OT, 4);      \
+    else if (n <= 8) TP_REDUCE_LAUNCH(PT, OT, 8); \
+    else TP_REDUCE_LAUNCH(PT, OT, TP_MAX_SHARDS); \
+  } while (0)
+  if (dt == TP_BF16 && pt == TP_BF16) TP_REDUCE_BY_N(__nv_bfloat16, __nv_bfloat16);
+  else if (dt == TP_BF16 && pt == TP_F32) TP_REDUCE_BY_N(float, __nv_bfloat16);
+  else if (dt == TP_F32 && pt == TP_F32) TP_REDUCE_BY_N(float, float);
+  else return fail(TP_ERR_DTYPE, "reduce of partials of dtype %d into dtype %d", pt, dt);
+#undef TP_REDUCE_BY_N
 #undef TP_REDUCE_LAUNCH
   return after_launch("reduce_partials");
 }

@@ -50,13 +50,14 @@ _fp = ctypes.c_void_p  # float* (device)
 _plan_p = ctypes.c_void_p
 
 _SIGS = {
-    "tp_plan_create": (_int, [_int, _int, _int, _int, _int, _int, ctypes.POINTER(_plan_p)]),
+    "tp_plan_create": (_int, [_int, _int, _int, _int, _int, _int, _int, ctypes.POINTER(_plan_p)]),
     "tp_plan_destroy": (None, [_plan_p]),
     "tp_plan_describe": (_int, [_plan_p, ctypes.c_char_p, ctypes.c_size_t]),
     "tp_status_string": (ctypes.c_char_p, [_int]),
     "tp_last_error": (ctypes.c_char_p, []),
-    "tp_get_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
+    "tp_get_device_status": (_int, [_plan_p, _vp]),
     "tp_launch_count": (ctypes.c_uint64, [_int]),
+    "tp_selftest_wait_timeout": (_int, [_i64, _vp, _vp]),
     "tp_shard_column": (_int, [_plan_p, _int, _vp, _vpp, _vp]),
     "tp_unshard_column": (_int, [_plan_p, _int, _vpp, _vp, _vp]),
     "tp_shard_row": (_int, [_plan_p, _int, _vp, _vpp, _vp]),
@@ -133,18 +134,24 @@ def _stream(stream=None) -> int | None:
     return None
 
 
+DTYPES = {"bf16": TP_BF16, "f32": TP_F32}
+
+
 class Plan:
-    """A tp_plan: block dimensions, shard count p, dtype and activation."""
+    """A tp_plan: block dimensions, shard count p, dtype, activation and the
+    dtype of the full-shape partial sums (default: the plan dtype)."""
 
     def __init__(self, hidden: int, ffn: int, heads: int, p: int, dtype: str = "bf16",
-                 act: str = "gelu"):
+                 act: str = "gelu", partial_dtype: str | None = None):
         self.hidden, self.ffn, self.heads, self.p = hidden, ffn, heads, p
         self.dtype_name = dtype
         self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.partial_dtype_name = partial_dtype or dtype
+        self.partial_torch_dtype = torch.bfloat16 if self.partial_dtype_name == "bf16" else torch.float32
         self.act = act
         h = ctypes.c_void_p()
-        check(lib.tp_plan_create(hidden, ffn, heads, p, TP_BF16 if dtype == "bf16" else TP_F32,
-                                 ACTS[act], ctypes.byref(h)), "tp_plan_create")
+        check(lib.tp_plan_create(hidden, ffn, heads, p, DTYPES[dtype], ACTS[act],
+                                 DTYPES[self.partial_dtype_name], ctypes.byref(h)), "tp_plan_create")
         self._h = h
 
     def close(self):
@@ -309,14 +316,26 @@ class Plan:
 
 def column_sum_static(rows, cols, x, out, accumulate=False, stream=None):
     """tp_column_sum_static: column sums with the library's fixed device scratch
-    (no allocation); see include/tp.h for its limits."""
+    (no allocation); see include/tp.h for its limits. x must be a dense
+    [rows, cols] tensor (row stride == cols)."""
     dt = TP_BF16 if x.dtype == torch.bfloat16 else TP_F32
     check(lib.tp_column_sum_static(rows, cols, dt, _ptr(x), _ptr(out), 1 if accumulate else 0,
                                    _stream(stream)), "tp_column_sum_static")
 
 
-def device_status(stream=None) -> str:
-    """Read and clear the device status word ("TP_OK" or "TP_ERR_TIMEOUT")."""
-    v = ctypes.c_int(0)
-    check(lib.tp_get_device_status(_stream(stream), ctypes.byref(v)), "tp_get_device_status")
-    return STATUS[v.value]
+def device_status(stream=None, plan: "Plan | None" = None) -> str:
+    """Read and clear the device status word: "TP_OK", "TP_ERR_TIMEOUT" (a
+    kernel's bounded wait gave up) or "TP_ERR_ARG" (a kernel met an
+    out-of-range id or label). A failure to read it raises TPError."""
+    st = lib.tp_get_device_status(plan.handle if plan is not None else None, _stream(stream))
+    if st in (0, 1, 7):
+        return STATUS[st]
+    check(st, "tp_get_device_status")
+    return STATUS[st]
+
+
+def selftest_wait_timeout(limit_ns: int, gave_up=None, stream=None) -> None:
+    """Launch the library's self-test kernel whose bounded wait runs out after
+    limit_ns (<= 1 s): it sets TP_ERR_TIMEOUT in the device status word."""
+    check(lib.tp_selftest_wait_timeout(int(limit_ns), _ptr(gave_up), _stream(stream)),
+          "tp_selftest_wait_timeout")

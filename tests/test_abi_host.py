@@ -9,6 +9,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from megatron_tensor_transformer_gemm_b200 import tp
 
@@ -41,9 +42,10 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(tp.lib, n)
 
 
-def _create(h, f, H, p, dtype=1, act=1):
+def _create(h, f, H, p, dtype=1, act=1, partial=None):
     ptr = ctypes.c_void_p()
-    st = tp.lib.tp_plan_create(h, f, H, p, dtype, act, ctypes.byref(ptr))
+    st = tp.lib.tp_plan_create(h, f, H, p, dtype, act, dtype if partial is None else partial,
+                               ctypes.byref(ptr))
     return st, ptr
 
 
@@ -61,6 +63,21 @@ def test_plan_create_divisibility(args, status, needle):
     assert st == status
     assert not ptr.value
     assert needle in tp.last_error()
+
+
+def test_plan_partial_dtype():
+    """Partials are stored in the plan dtype or in fp32; fp32 plans take fp32."""
+    st, ptr = _create(4096, 11008, 32, 8, dtype=1, partial=0)   # bf16 plan, fp32 partials
+    assert st == 0 and ptr.value
+    tp.lib.tp_plan_destroy(ptr)
+    st, ptr = _create(4096, 11008, 32, 8, dtype=0, partial=1)   # fp32 plan, bf16 partials
+    assert st == 4 and not ptr.value
+    assert "partial dtype" in tp.last_error()
+    st, ptr = _create(4096, 11008, 32, 8, dtype=1, partial=7)
+    assert st == 4 and not ptr.value
+    p = tp.Plan(4096, 11008, 32, 8, "bf16", "swiglu", partial_dtype="f32")
+    assert "partials=f32" in p.describe()
+    assert p.partial_torch_dtype == torch.float32
 
 
 def test_plan_describe_prints_shard_shapes():
@@ -143,6 +160,24 @@ def test_swiglu_rejects_column_bias():
     A = _arr([FAKE, FAKE])
     assert tp.lib.tp_column_fwd(p.handle, 0, 64, FAKE, A, A, None, A, None) == 1
     assert "SwiGLU" in tp.last_error()
+
+
+def test_device_status_without_a_device_is_a_host_error():
+    """With no usable GPU the status read fails on the host (TP_ERR_NO_DEVICE or
+    TP_ERR_CUDA), never with one of the device-reported codes."""
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = tp.lib.tp_get_device_status(None, None)
+    assert st in (6, 8)
+    with pytest.raises(tp.TPError):
+        tp.device_status()
+
+
+def test_selftest_wait_limit_is_validated_before_launch():
+    assert tp.lib.tp_selftest_wait_timeout(0, None, None) == 1
+    assert tp.lib.tp_selftest_wait_timeout(2_000_000_000, None, None) == 1
+    assert "limit_ns" in tp.last_error()
+    assert tp.lib.tp_selftest_wait_timeout(1000, FAKE + 2, None) == 3
 
 
 def test_status_strings():

@@ -221,3 +221,108 @@ def test_layernorm_all_gather_equals_gather_of_layernorm(n):
 def test_device_status_is_clean():
     tp = _tp()
     assert tp.device_status() == "TP_OK"
+
+
+@pytest.mark.parametrize("p", [2, 8, 16])
+@pytest.mark.parametrize("T,h", [(1000, 136), (33, 4096)])
+def test_fp32_partials_reduce_bitexact(p, T, h):
+    """A bf16 plan with fp32 partials: integer-valued partials (exact in both
+    types) sum bit for bit, with the bias once and the residual, and the
+    sequence reduce-scatter scatters the same rows."""
+    tp = _tp()
+    P, b, r = tp_synth.draw_partials(p, T, h, torch.float32, seed=p, integer_valued=True, residual=True)
+    plan = tp.Plan(h, 0, 0, 1, "bf16", "none", partial_dtype="f32")
+    Pd = [dev(x) for x in P]
+    Y = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+    plan.reduce_partials(T, Pd, dev(b.bfloat16()), dev(r.bfloat16()), Y)
+    ref = O.reduce_partials([O.f64(x) for x in P], O.f64(b), O.f64(r))
+    assert np.abs(ref).max() < 256  # every value exact in bf16
+    assert_bitexact(Y, ref, "reduce, fp32 partials")
+    if T % p == 0:
+        t = T // p
+        outs = [torch.empty(t, h, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+        plan.reduce_scatter_seq(T, Pd, dev(b.bfloat16()), None, outs)
+        refs = O.reduce_scatter_seq([O.f64(x) for x in P], O.f64(b))
+        for j in range(p):
+            assert_bitexact(outs[j], refs[j], f"RS shard {j}, fp32 partials")
+
+
+def test_fp32_partials_row_layer_against_oracle_and_bf16_partials():
+    """Row GEMM partials stored in fp32 (the plan's partial dtype) and summed:
+    within tolerance of the oracle, the partials themselves within the fp32
+    bound, and the summed output measurably closer to the oracle than with
+    bf16 partials (only the final rounding remains: RMS error about 1/sqrt(2)
+    of the bf16-partials path, where each partial is rounded once more)."""
+    tp = _tp()
+    T, h, f, p = 512, 1024, 4096, 8
+    g = torch.Generator().manual_seed(41)
+    fp = f // p
+    Hs = [torch.randn(T, fp, generator=g).to(torch.bfloat16) for _ in range(p)]
+    W2 = (torch.randn(h, f, generator=g) * 0.02).to(torch.bfloat16)
+    b2 = (torch.rand(h, generator=g) * 0.2 - 0.1).to(torch.bfloat16)
+    W2f = O.f64(W2)
+    parts = [O.row_partial(O.f64(Hs[i]), O.shard_cols(W2f, p, i)) for i in range(p)]
+    ref = O.reduce_partials(parts, O.f64(b2))
+    rms = {}
+    for pd in ("bf16", "f32"):
+        plan = tp.Plan(h, f, 0, p, "bf16", "gelu", partial_dtype=pd)
+        Ws = [torch.empty(h, fp, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+        plan.shard_row("mlp", dev(W2), Ws)
+        P = [torch.empty(T, h, dtype=plan.partial_torch_dtype, device="cuda") for _ in range(p)]
+        plan.row_fwd_partial("mlp", T, [dev(x) for x in Hs], Ws, P)
+        if pd == "f32":
+            for i in range(p):
+                assert_close(P[i], parts[i], TOL_F32, f"fp32 partial {i}")
+        Y = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+        plan.reduce_partials(T, P, dev(b2), None, Y)
+        assert_close(Y, ref, TOL_BF16, f"Y ({pd} partials)")
+        d = host(Y) - ref
+        rms[pd] = float(np.sqrt((d * d).mean() / (ref * ref).mean()))
+    assert rms["f32"] < 0.85 * rms["bf16"], rms
+
+
+def test_fp32_partials_column_backward_dx():
+    """dX partials of the column backward in fp32, reduce-scattered along the
+    sequence into bf16 shards, against the oracle."""
+    tp = _tp()
+    T, h, f, p = 256, 512, 1024, 4
+    g = torch.Generator().manual_seed(43)
+    n = f // p
+    W1 = (torch.randn(f, h, generator=g) * 0.05).to(torch.bfloat16)
+    dZs = [torch.randn(T, n, generator=g).to(torch.bfloat16) for _ in range(p)]
+    plan = tp.Plan(h, f, 0, p, "bf16", "gelu", partial_dtype="f32")
+    Ws = [torch.empty(n, h, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+    plan.shard_column("mlp", dev(W1), Ws)
+    dXp = [torch.empty(T, h, dtype=torch.float32, device="cuda") for _ in range(p)]
+    plan.column_bwd("mlp", T, None, [dev(z) for z in dZs], Ws, None, None, dXp)
+    W1f = O.f64(W1)
+    parts = [O.column_bwd_shard(np.zeros((T, h)), O.f64(dZs[i]), O.shard_rows(W1f, p, i))[2]
+             for i in range(p)]
+    for i in range(p):
+        assert_close(dXp[i], parts[i], TOL_F32, f"fp32 dX partial {i}")
+    t = T // p
+    outs = [torch.empty(t, h, dtype=torch.bfloat16, device="cuda") for _ in range(p)]
+    plan.all_gather_seq_bwd(T, dXp, outs)
+    refs = O.reduce_scatter_seq(parts)
+    for j in range(p):
+        assert_close(outs[j], refs[j], TOL_BF16, f"dX RS shard {j}")
+
+
+def test_bounded_wait_times_out_and_reports():
+    """The device-side failure path: a kernel whose bounded wait (1 ms here)
+    never sees its arrival gives up, returns, and the status word reads
+    TP_ERR_TIMEOUT once; the next read is clean and the context still works."""
+    tp = _tp()
+    assert tp.device_status() == "TP_OK"
+    flag = torch.zeros(4, dtype=torch.int32, device="cuda")
+    tp.selftest_wait_timeout(1_000_000, flag)
+    assert tp.device_status() == "TP_ERR_TIMEOUT"
+    assert int(flag[0]) == 1
+    assert tp.device_status() == "TP_OK"
+    # the context is intact: an ordinary call still runs and is correct
+    P, b, _ = tp_synth.draw_partials(2, 16, 64, torch.bfloat16, integer_valued=True)
+    plan = tp.Plan(64, 0, 0, 1, "bf16", "none")
+    Y = torch.empty(16, 64, dtype=torch.bfloat16, device="cuda")
+    plan.reduce_partials(16, [dev(x) for x in P], dev(b), None, Y)
+    assert_bitexact(Y, O.reduce_partials([O.f64(x) for x in P], O.f64(b)), "reduce after a timeout")
+    assert tp.device_status(plan=plan) == "TP_OK"

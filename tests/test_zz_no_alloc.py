@@ -61,3 +61,30 @@ def test_static_scratch_rejects_too_many_columns():
     cols = 512 * 1024 + 8
     assert tp.lib.tp_column_sum_static(1, cols, tp.TP_BF16, x.data_ptr(), out.data_ptr(), 0, None) == 5
     assert "static scratch" in tp.last_error()
+
+
+def test_static_scratch_allocates_nothing_after_the_first_call():
+    """After one warm-up call per shape (the first call on a device may load
+    the library's module, which reserves the array), repeated calls leave the
+    device's free memory unchanged: every input is allocated beforehand and no
+    plan call runs inside the window."""
+    tp = _lib()
+    big = torch.ones(32768, 4096, dtype=torch.bfloat16, device="cuda")
+    wide_cols = 512 * 1024  # the static scratch's limit: a single row split
+    wide = torch.ones(8, wide_cols, dtype=torch.float32, device="cuda")
+    out_big = torch.empty(4096, dtype=torch.float32, device="cuda")
+    out_wide = torch.empty(wide_cols, dtype=torch.float32, device="cuda")
+    calls = [(32768, 4096, big, out_big), (8, wide_cols, wide, out_wide), (0, 4096, big, out_big)]
+    for rows, cols, x, out in calls:
+        assert _static(tp, rows, cols, x, out) == 0, tp.last_error()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        for rows, cols, x, out in calls[:2]:
+            assert _static(tp, rows, cols, x, out) == 0, tp.last_error()
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free1 == free0, f"free device memory changed by {free0 - free1} bytes"
+    # the values are still the column sums (every sum of ones is exact)
+    assert torch.equal(out_big, torch.full_like(out_big, 32768.0))
+    assert torch.equal(out_wide, torch.full_like(out_wide, 8.0))
