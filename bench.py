@@ -17,10 +17,13 @@ partial-reduce kernel's HBM GB/s is reported: measured inside the step for
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Prints one JSON line (rank 0). For N > 1 (torchrun, one process per GPU) every
-rank runs its own replica of the workload (weak scaling; the path's shards all
-live on one GPU, so there is no data-path collective); time is the max over
-ranks of the device-timed region.
+Prints one JSON line (rank 0). For N > 1 (torchrun, one process per GPU) the
+p = 8 shards of the one workload split over the N ranks, 8/N per GPU
+(dist.DistTPMLP): inside a GPU the shards' sums run in the fused GEMMs, between
+GPUs the row layer's all-reduce and the dX all-reduce are NCCL collectives
+(strong scaling: the total work is fixed). --replicas instead runs one
+independent full replica per GPU (weak scaling, no data-path collective).
+Time is the max over ranks of the device-timed region.
 
 --impl reference times the CPU oracle (fp64 numpy, the machine's host cores) on
 a bounded sample of the same workload: each step is the full forward and
@@ -234,6 +237,130 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------------- GPU leg
+def run_dist(args, world, rank, local):
+    """The 7B SwiGLU MLP with its p = 8 shards split over the N ranks (8/N per
+    GPU), NCCL all-reduces between them; strong scaling."""
+    import torch
+    import tp_synth
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.dist import DistTPMLP
+
+    if P % world:
+        raise SystemExit(f"--gpus {world}: the {P} shards do not split over {world} GPUs")
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    T = args.tokens
+    inp = tp_synth.draw_mlp(T, HIDDEN, FFN, "swiglu", torch.bfloat16, seed=0)  # replicated input
+    m = DistTPMLP(HIDDEN, FFN, P, "swiglu", device=dev)
+    m.load_weights(inp.W1, inp.W2)
+    X_h, dY_h = inp.X.pin_memory(), inp.dY.pin_memory()
+    del inp
+    X, dY = X_h.to(dev), dY_h.to(dev)
+    m.alloc(T)
+    stream = torch.cuda.current_stream()
+    pl = m.plan
+    gemm_calls = ("column_fwd", "row_fwd_reduce", "row_bwd", "column_bwd_reduce")
+    orig = {n: getattr(pl, n) for n in gemm_calls}
+    gemm_ev, comm_ev = [], []
+
+    def timed(fn, bucket):
+        def wrapper(*a, **k):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            out = fn(*a, **k)
+            e1.record(stream)
+            bucket.append((e0, e1))
+            return out
+        return wrapper
+
+    import megatron_tensor_transformer_gemm_b200.dist as D
+    orig_sum = D.sum_over_ranks
+
+    def step(instrument=False):
+        for n in gemm_calls:
+            setattr(pl, n, timed(orig[n], gemm_ev) if instrument else orig[n])
+        D.sum_over_ranks = timed(orig_sum, comm_ev) if instrument else orig_sum
+        m.forward(X)
+        m.backward(dY)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    tp.launch_count(reset=True)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        step(instrument=True)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    launches = tp.launch_count(reset=True)
+    barrier(world)
+    clk = clocks.stop()
+    for n in gemm_calls:
+        setattr(pl, n, orig[n])
+    D.sum_over_ranks = orig_sum
+    flops = m.flops(T)
+    ms = max_over_ranks(s0.elapsed_time(s1), world)
+    value = flops * args.steps / (ms / 1e3) / 1e12
+    gemm_ms = sum(a.elapsed_time(b) for a, b in gemm_ev)
+    comm_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in comm_ev), world)
+    gemm_tflops = (flops / world) * args.steps / (gemm_ms / 1e3) / 1e12
+    # end to end: every rank copies X and dY in from pinned memory and Y and dX out
+    Y_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
+    dX_h = torch.empty(T, HIDDEN, dtype=torch.bfloat16).pin_memory()
+    e2e = None
+    if not args.skip_e2e:
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            X.copy_(X_h, non_blocking=True)
+            dY.copy_(dY_h, non_blocking=True)
+            Y = m.forward(X)
+            Y_h.copy_(Y, non_blocking=True)
+            dX = m.backward(dY)
+            dX_h.copy_(dX, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        nb = X_h.numel() * 2
+        e2e = {"value": flops * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * nb * world, "d2h_bytes_per_step": 2 * nb * world,
+               "ms_per_step": e2e_ms / args.steps}
+    status = tp.device_status()
+    if rank != 0:
+        return 0
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded tp_synth draws: X, dY ~ N(0,1), W ~ N(0,0.02))",
+        "config": {"workload": WORKLOAD.replace("on one GPU", f"over {world} GPUs"), "hidden": HIDDEN,
+                   "ffn": FFN, "tokens": T, "p": P, "act": "swiglu", "global_batch": 8, "seq_len": 4096,
+                   "parallelism": f"tp{world}: {P // world} of the {P} shards per GPU, NCCL all-reduce",
+                   "l2": "inputs larger than L2 (X and dY 268 MB each); no flush"},
+        "roofline": {"bound": "tensor", "kernel": "tp_gemm_kernel (tcgen05)", "achieved": gemm_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops"],
+                     "peak_kind": f"bf16 burst ({peaks['source']}), per GPU", "traffic": None},
+        "comm": {"collective": "NCCL all-reduce of Y and dX ([T, 4096] bf16) per step",
+                 "ms_per_step": comm_ms / args.steps,
+                 "bytes_per_rank_per_step": 2 * 2 * (world - 1) / world * T * HIDDEN * 2},
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "device_status": status,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def run_ours(args, world, rank, local):
     import torch
     import tp_synth
@@ -850,6 +977,9 @@ def main():
     ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm", "sp_hbm"],
                     default="mlp7b",
                     help="mlp7b (the metric's workload) or another config of the suite")
+    ap.add_argument("--replicas", action="store_true",
+                    help="N > 1: one independent replica per GPU (weak scaling) instead of the "
+                         "shards split over the GPUs")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph (other workloads)")
     args = ap.parse_args()
@@ -861,7 +991,8 @@ def main():
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
     world, rank, local = dist_setup()
     if args.workload == "mlp7b":
-        rc = run_ours(args, world, rank, local)
+        rc = run_dist(args, world, rank, local) if world > 1 and not args.replicas else \
+            run_ours(args, world, rank, local)
     elif args.workload in ("vocab", "norm", "sp_hbm"):
         rc = run_hbm(args, world, rank, local)
     else:
