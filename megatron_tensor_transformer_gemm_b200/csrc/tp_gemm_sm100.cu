@@ -10,6 +10,10 @@
 //   EPI_DSWIGLU    dZ = [acc*u*SiLU'(g) | acc*SiLU(g)]   row layer backward
 // (TP walkthrough 2kiu.com §2.1-§2.2 and §3.2; 张量并行 wiki, 两种切法.)
 //
+// Tile layouts: a CTA pair (cta_group::2) on a 256 x 256 tile by default; for
+// problems whose 256 x 256 tiles would leave SMs idle, the host may instead
+// run 128-column tiles, one CTA per 128-row tile, or both (choose_layout).
+//
 // Design (per CTA, one CTA per SM, persistent over a static tile schedule):
 //   warp 0      TMA producer: 128B-swizzled A and B tiles into a 4-stage ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
@@ -85,6 +89,8 @@ struct alignas(64) GemmParams {
   GroupArgs g[TP_MAX_SHARDS];
   int ngroups;
   int total_tiles;
+  int tile_n;      // output columns per tile: BN, or BN / 2 (SwiGLU pairs; narrow launches)
+  int narrow_all;  // every tile runs as an N = BN / 2 MMA (small problems: twice the tiles)
   int a_mn;
   int b_mn;
   int epi;
@@ -119,7 +125,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, 
 // CTA pair each CTA then supplies BN / 4 rows of B (its half of the narrow N).
 // SwiGLU tiles (gate and up halves of one B tile) never run narrow.
 __device__ __forceinline__ bool narrow_tile(const GemmParams& p, const GroupArgs& ga, int n0) {
-  return p.epi != tpi::EPI_SWIGLU && ga.N - n0 <= BN / 2;
+  return p.epi != tpi::EPI_SWIGLU && (p.narrow_all || ga.N - n0 <= BN / 2);
 }
 
 // ------------------------------------------------------------- epilogue math
@@ -338,9 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       decode_tile(p, t, g, mt, nt);
       const GroupArgs& ga = p.g[g];
       const int m0 = mt * C::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
-      const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
+      const int n0 = nt * p.tile_n;
       // this CTA's B rows (in a narrow tile of a pair, each CTA's first BN / 4)
       const int nb0 = n0 + static_cast<int>(rank) * (narrow_tile(p, ga, n0) ? BN / (2 * PAIR) : C::B_ROWS);
+      // A narrow launch loads only the B rows its MMAs read (half a B stage);
+      // a ragged narrow tile of a full-width launch loads the full stage.
+      const uint32_t b_bytes = p.narrow_all ? C::B_BYTES / 2 : C::B_BYTES;
+      const int b_blocks = (p.narrow_all ? C::B_ROWS / 2 : C::B_ROWS) / 64;  // MN-major 64-column blocks
       const int nseg = p.kcat ? p.kcat : 1;
       for (int sg = 0; sg < nseg && ok; ++sg) {
         const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
           uint8_t* a_dst = sA + stage * C::A_BYTES;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
           if (PAIR == 1) {
-            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full[stage], C::A_BYTES + b_bytes);
             if (!p.a_mn) {
               tma_load_2d(a_dst, &p.tmA[gi], &full[stage], k0, m0);
             } else {
@@ -368,14 +378,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
             } else if (!p.b_mn) {
               tma_load_2d(b_dst, &p.tmB[gi], &full[stage], k0, n0);
             } else {
-#pragma unroll
-              for (int c = 0; c < BN / 64; ++c)
+              for (int c = 0; c < b_blocks; ++c)
                 tma_load_2d(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], &full[stage], n0 + c * 64, k0);
             }
           } else {
             // Both CTAs' copies complete on the leader's full barrier, which
             // expects the bytes of the whole pair.
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], PAIR * C::STAGE_BYTES);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], PAIR * (C::A_BYTES + b_bytes));
             const uint32_t fb = map_shared(smem_u32(&full[stage]), 0);
             if (!p.a_mn) {
               tma_load_2d_pair(a_dst, &p.tmA[gi], fb, k0, m0);
@@ -390,8 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
             } else if (!p.b_mn) {
               tma_load_2d_pair(b_dst, &p.tmB[gi], fb, k0, nb0);
             } else {
-#pragma unroll
-              for (int c = 0; c < C::B_ROWS / 64; ++c)
+              for (int c = 0; c < b_blocks; ++c)
                 tma_load_2d_pair(b_dst + c * MN_BLOCK_BYTES, &p.tmB[gi], fb, nb0 + c * 64, k0);
             }
           }
@@ -423,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       int g, mt, nt;
       decode_tile(p, t, g, mt, nt);
       const uint32_t idesc =
-          narrow_tile(p, p.g[g], nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN)) ? idesc_narrow : idesc_full;
+          narrow_tile(p, p.g[g], nt * p.tile_n) ? idesc_narrow : idesc_full;
       int num_kb = p.g[g].num_kb;
       if (p.kcat) {
         num_kb = 0;
@@ -485,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) break;
       tc_fence_after();
       const int row = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32 + lane;
-      const int n0 = nt * (p.epi == tpi::EPI_SWIGLU ? BN / 2 : BN);
+      const int n0 = nt * p.tile_n;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       epilogue_tile(p, ga, taddr, row, n0, half, narrow_tile(p, ga, n0));
@@ -543,24 +551,95 @@ tp_status encode_gateup(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint
   return TP_OK;
 }
 
-// CTA pairing of the bf16 GEMM: 2 (cta_group::2, 256-row tiles) unless the
-// environment variable TP_GEMM_CTA_PAIR is "1" (one CTA per 128-row tile).
-int gemm_pair() {
+// CTA pairing forced by the environment variable TP_GEMM_CTA_PAIR ("1": one
+// CTA per 128-row tile, "2": CTA pairs with 256-row tiles); 0 = chosen per launch.
+int forced_pair() {
   const char* e = getenv("TP_GEMM_CTA_PAIR");
-  return (e && e[0] == '1') ? 1 : 2;
+  if (e && e[0] == '1') return 1;
+  if (e && e[0] == '2') return 2;
+  return 0;
+}
+
+// Tile width forced by TP_GEMM_NARROW ("0": 256-column tiles, "1": 128-column
+// tiles everywhere); -1 = chosen per launch. SwiGLU launches ignore it.
+int forced_narrow() {
+  const char* e = getenv("TP_GEMM_NARROW");
+  if (e && e[0] == '0') return 0;
+  if (e && e[0] == '1') return 1;
+  return -1;
+}
+
+// Tile layout of one launch: CTA pairing and tile width.
+struct Layout {
+  int pair;     // 1 or 2 CTAs per tile
+  bool narrow;  // every tile N = BN / 2 (SwiGLU tiles are always 128 gate/up pairs)
+};
+
+// The layout with the least estimated time. A launch lasts as long as its
+// busiest SM: ceil(tiles / units) waves of the average tile, where a tile's
+// cost on each of its SMs is its MMA width times its K blocks. Layouts that
+// move more operand bytes per FLOP (one CTA instead of a pair, N = 128
+// instead of 256) carry a factor, so they win only when they fill more SMs:
+// small problems, whose 256 x 256 tiles leave most of the GPU idle.
+Layout choose_layout(const GemmBatch& b, int sms) {
+  const bool swiglu = b.epi == tpi::EPI_SWIGLU;
+  const int nout = b.kcat ? 1 : b.n;
+  int64_t kb_cat = 0;
+  if (b.kcat)
+    for (int i = 0; i < b.n; ++i) kb_cat += (b.g[i].K + BK - 1) / BK;
+  const int fp = forced_pair();
+  const int fn = swiglu ? 0 : forced_narrow();
+  Layout best{2, false};
+  double best_cost = -1.0;
+  for (int pair = 2; pair >= 1; --pair) {
+    if (fp && pair != fp) continue;
+    for (int nar = 0; nar <= (swiglu ? 0 : 1); ++nar) {
+      if (fn >= 0 && nar != fn) continue;
+      const int tile_m = BM * pair;
+      const int tn = (swiglu || nar) ? BN / 2 : BN;
+      double work = 0.0;
+      int64_t tiles = 0;
+      for (int i = 0; i < nout; ++i) {
+        const GemmProblem& o = b.g[i];
+        const int64_t mt = (o.M + tile_m - 1) / tile_m;
+        const int64_t nt = (o.N + tn - 1) / tn;
+        const int64_t kb = b.kcat ? kb_cat : (o.K + BK - 1) / BK;
+        const int last = o.N - static_cast<int>(nt - 1) * tn;  // columns of the last N tile
+        const int mma_n = swiglu ? BN : (nar ? BN / 2 : BN);
+        const int last_n = (!swiglu && last <= BN / 2) ? BN / 2 : mma_n;
+        tiles += mt * nt;
+        work += static_cast<double>(mt) * kb * ((nt - 1) * mma_n + last_n);
+      }
+      const int64_t units = std::max(1, sms / pair);
+      const double waves = static_cast<double>((tiles + units - 1) / units);
+      const double factor = (pair == 2 ? 1.0 : 1.08) * (nar ? 1.10 : 1.0);
+      const double cost = waves * (work / static_cast<double>(std::max<int64_t>(tiles, 1))) * factor;
+      if (best_cost < 0.0 || cost < best_cost) {
+        best_cost = cost;
+        best = Layout{pair, nar != 0};
+      }
+    }
+  }
+  return best;
 }
 
 template <int PAIR>
 tp_status launch_kernel(const GemmParams& p, int tiles, int sms, cudaStream_t st) {
   using C = Cfg<PAIR>;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[PAIR - 1]) {
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return tpi::fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  if (!attr_set[dev][PAIR - 1]) {
     tp_status s = tpi::cuda_status(
         cudaFuncSetAttribute(tp_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES),
         "cudaFuncSetAttribute(gemm smem)");
     if (s != TP_OK) return s;
-    attr_set[PAIR - 1] = true;
+    attr_set[dev][PAIR - 1] = true;
   }
   const int clusters = std::max(1, std::min(tiles, sms / PAIR));
   cudaLaunchConfig_t cfg{};
@@ -605,13 +684,19 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   std::lock_guard<std::mutex> lk(mu);
   memset(&p, 0, sizeof(p));
   const bool swiglu = b.epi == EPI_SWIGLU;
-  const int tile_n = swiglu ? BN / 2 : BN;
-  const int pair = gemm_pair();
-  const int tile_m = BM * pair;
   if (b.kcat && b.epi != EPI_STORE)
     return fail(TP_ERR_ARG, "K-concatenated GEMM supports the plain epilogue only");
-  int tiles = 0;
   const int nout = b.kcat ? 1 : b.n;
+  for (int i = 0; i < nout; ++i)
+    if (b.g[i].M <= 0 || b.g[i].N <= 0)
+      return fail(TP_ERR_ARG, "GEMM %d has an empty output (%d x %d)", i, b.g[i].M, b.g[i].N);
+  const int sms = device_sms();
+  const Layout lay = choose_layout(b, sms);
+  const int pair = lay.pair;
+  const int tile_n = (swiglu || lay.narrow) ? BN / 2 : BN;
+  const int tile_m = BM * pair;
+  const int b_box = (lay.narrow ? BN / 2 : BN) / pair;  // K-major B rows per CTA
+  int tiles = 0;
   for (int i = 0; i < b.n; ++i) {
     const GemmProblem& g = b.g[i];
     const GemmProblem& o = b.kcat ? b.g[0] : g;  // the output this segment feeds
@@ -651,7 +736,7 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     if (s != TP_OK) return s;
     // B operand
     if (swiglu) s = encode_gateup(enc, &p.tmB[i], g.B, g.K, o.nh, g.ldb);
-    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, o.N, g.ldb, BN / pair);
+    else if (!b.b_mn) s = encode_2d(enc, &p.tmB[i], g.B, g.K, o.N, g.ldb, b_box);
     else s = encode_2d(enc, &p.tmB[i], g.B, o.N, g.K, g.ldb, BK);
     if (s != TP_OK) return s;
   }
@@ -667,14 +752,16 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   }
   p.ngroups = nout;
   p.total_tiles = tiles;
+  p.tile_n = tile_n;
+  p.narrow_all = lay.narrow ? 1 : 0;
   p.a_mn = b.a_mn;
   p.b_mn = b.b_mn;
   p.epi = b.epi;
   p.out_f32 = b.out_f32;
   s = device_status_word(&p.status);
   if (s != TP_OK) return s;
-  if (pair == 2) return launch_kernel<2>(p, tiles, device_sms(), st);
-  return launch_kernel<1>(p, tiles, device_sms(), st);
+  if (pair == 2) return launch_kernel<2>(p, tiles, sms, st);
+  return launch_kernel<1>(p, tiles, sms, st);
 }
 
 }  // namespace tpi

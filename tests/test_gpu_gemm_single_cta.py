@@ -1,6 +1,8 @@
-"""The GEMM parity tests again with the one-CTA-per-tile kernel
-(TP_GEMM_CTA_PAIR=1) instead of the default CTA-pair (cta_group::2) kernel,
-in a subprocess so the choice is made before the library's first launch."""
+"""The GEMM parity tests again under each forced tile layout: one CTA per
+128-row tile (TP_GEMM_CTA_PAIR=1) instead of CTA pairs, and 128-column tiles
+everywhere (TP_GEMM_NARROW=1) with either pairing. Each runs in a subprocess so
+the choice is made before the library's first launch. The default run of
+test_gpu_gemm.py lets the library choose per launch."""
 import os
 import subprocess
 import sys
@@ -12,8 +14,9 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_gemm_suite_with_single_cta_tiles():
-    env = dict(os.environ, TP_GEMM_CTA_PAIR="1")
+@pytest.mark.parametrize("pair,narrow", [("1", "0"), ("2", "0"), ("2", "1"), ("1", "1")])
+def test_gemm_suite_under_forced_layouts(pair, narrow):
+    env = dict(os.environ, TP_GEMM_CTA_PAIR=pair, TP_GEMM_NARROW=narrow)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_gpu_gemm.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
