@@ -569,58 +569,34 @@ tp_status tp_column_fwd(tp_plan* plan, tp_which which, int64_t T, const void* X,
     g.ldb = cs.k;
     g.bias = bias ? bias[i] : nullptr;
   }
-  if (plan->dtype == TP_BF16) {
-    if (act == TP_ACT_NONE) {
-      b.epi = EPI_STORE;
-      for (int i = 0; i < p; ++i) {
-        b.g[i].N = cs.n_w;
-        b.g[i].D = H[i];
-        b.g[i].ldd = cs.n_h;
-      }
-    } else if (act == TP_ACT_GELU) {
-      b.epi = EPI_BIAS_GELU;
-      for (int i = 0; i < p; ++i) {
-        b.g[i].N = cs.n_w;
-        b.g[i].D = Z ? Z[i] : nullptr;
-        b.g[i].ldd = cs.n_w;
-        b.g[i].D2 = H[i];
-        b.g[i].ldd2 = cs.n_h;
-      }
-    } else {
-      b.epi = EPI_SWIGLU;
-      for (int i = 0; i < p; ++i) {
-        b.g[i].N = cs.n_h;  // gate/up pairs
-        b.g[i].nh = cs.n_h;
-        b.g[i].D = Z ? Z[i] : nullptr;
-        b.g[i].ldd = cs.n_w;
-        b.g[i].D2 = H[i];
-        b.g[i].ldd2 = cs.n_h;
-      }
+  if (act == TP_ACT_NONE) {
+    b.epi = EPI_STORE;
+    for (int i = 0; i < p; ++i) {
+      b.g[i].N = cs.n_w;
+      b.g[i].D = H[i];
+      b.g[i].ldd = cs.n_h;
     }
-    return launch_gemm_bf16(b, st);
+  } else if (act == TP_ACT_GELU) {
+    b.epi = EPI_BIAS_GELU;
+    for (int i = 0; i < p; ++i) {
+      b.g[i].N = cs.n_w;
+      b.g[i].D = Z ? Z[i] : nullptr;
+      b.g[i].ldd = cs.n_w;
+      b.g[i].D2 = H[i];
+      b.g[i].ldd2 = cs.n_h;
+    }
+  } else {
+    b.epi = EPI_SWIGLU;
+    for (int i = 0; i < p; ++i) {
+      b.g[i].N = cs.n_h;  // gate/up pairs
+      b.g[i].nh = cs.n_h;
+      b.g[i].D = Z ? Z[i] : nullptr;
+      b.g[i].ldd = cs.n_w;
+      b.g[i].D2 = H[i];
+      b.g[i].ldd2 = cs.n_h;
+    }
   }
-  // fp32: the GEMM writes the pre-activation, an element-wise kernel the activation.
-  b.epi = EPI_STORE;
-  float* zbuf = nullptr;
-  if (act != TP_ACT_NONE && !Z) {
-    void* ws = nullptr;
-    TP_TRY(workspace(plan, static_cast<size_t>(T) * cs.n_w * sizeof(float), &ws));
-    zbuf = static_cast<float*>(ws);
-  }
-  for (int i = 0; i < p; ++i) {
-    GemmBatch one = b;
-    one.n = 1;
-    one.g[0] = b.g[i];
-    one.g[0].N = cs.n_w;
-    void* zi = act == TP_ACT_NONE ? H[i] : (Z ? Z[i] : zbuf);
-    one.g[0].D = zi;
-    one.g[0].ldd = cs.n_w;
-    TP_TRY(launch_gemm_f32(one, st));
-    if (act != TP_ACT_NONE)
-      TP_TRY(launch_act_fwd(act, static_cast<const float*>(zi), T, cs.n_h, cs.n_w,
-                            static_cast<float*>(H[i]), cs.n_h, st));
-  }
-  return TP_OK;
+  return run_gemm(plan, b, st);
 }
 
 tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
@@ -663,7 +639,6 @@ static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
                                        void* Y, void* const* Y_seq, bool scatter, cudaStream_t st) {
   TP_TRY(check_plan(plan));
   TP_TRY(check_T(T));
-  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "the fused reduce runs on bf16 plans");
   int k = 0;
   TP_TRY(row_k(plan, which, &k));
   const int p = plan->p, h = plan->hidden;
@@ -708,7 +683,7 @@ static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
       b.res_seq[j] = residual_seq ? residual_seq[j] : nullptr;
     }
   }
-  return launch_gemm_bf16(b, st);
+  return run_gemm(plan, b, st);
 }
 
 tp_status tp_row_fwd_reduce(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
@@ -1065,31 +1040,8 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
     g.ldaux = nz;
     g.nh = k;
   }
-  if (plan->dtype == TP_BF16) {
-    b.epi = act == TP_ACT_GELU ? EPI_DGELU : act == TP_ACT_SWIGLU ? EPI_DSWIGLU : EPI_STORE;
-    TP_TRY(launch_gemm_bf16(b, st));
-  } else {
-    b.epi = EPI_STORE;
-    float* dh = nullptr;
-    if (act == TP_ACT_SWIGLU) {
-      void* ws = nullptr;
-      TP_TRY(workspace(plan, static_cast<size_t>(T) * k * sizeof(float), &ws));
-      dh = static_cast<float*>(ws);
-    }
-    for (int i = 0; i < p; ++i) {
-      GemmBatch one = b;
-      one.n = 1;
-      one.g[0] = b.g[i];
-      void* dst = act == TP_ACT_SWIGLU ? static_cast<void*>(dh) : dZ[i];
-      one.g[0].D = dst;
-      one.g[0].ldd = act == TP_ACT_SWIGLU ? k : nz;
-      TP_TRY(launch_gemm_f32(one, st));
-      if (act != TP_ACT_NONE)
-        TP_TRY(launch_act_bwd(act, static_cast<const float*>(dst), T, k,
-                              static_cast<const float*>(Z[i]), nz, static_cast<float*>(dZ[i]), nz,
-                              st));
-    }
-  }
+  b.epi = act == TP_ACT_GELU ? EPI_DGELU : act == TP_ACT_SWIGLU ? EPI_DSWIGLU : EPI_STORE;
+  TP_TRY(run_gemm(plan, b, st));
   if (dW) {
     // dW_i [h, k] = dY^T H_i: A(m, t) = dY[t, m] (MN-major), B(n, t) = H_i[t, n] (MN-major).
     GemmBatch w{};
@@ -1128,7 +1080,6 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   TP_TRY(col_shape(plan, which, &cs));
   const int p = plan->p, h = plan->hidden;
   const int n = cs.n_w;
-  if (mode != 0 && plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "the fused reduce runs on bf16 plans");
   TP_TRY(check_ptrs(dZ, p, "dZ", false));
   TP_TRY(check_ptrs(W, p, "W", false));
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dW), p, "dW", true));

@@ -107,12 +107,6 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
                                   const float* mean, const float* rstd, tp_dtype dt,
                                   cudaStream_t st, int accumulate = 0);
 
-// Element-wise activation kernels for the fp32 path (tp_gemm_simt.cu).
-tp_status launch_act_fwd(tp_act act, const float* Z, int64_t T, int64_t nh, int64_t ldz, float* H,
-                         int64_t ldh, cudaStream_t st);
-tp_status launch_act_bwd(tp_act act, const float* dH, int64_t T, int64_t nh, const float* Z,
-                         int64_t ldz, float* dZ, int64_t lddz, cudaStream_t st);
-
 // ------------------------------------------------------------------- GEMM
 // One GEMM problem of a grouped launch: D[M, N] = A[M, K] . B[N, K]^T.
 // A element (m, k) lives at A + m*lda + k when !a_mn (K-major) and at
@@ -163,7 +157,7 @@ struct GemmBatch {
 
 // bf16 tcgen05 tensor-core path (tp_gemm_sm100.cu).
 tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st);
-// fp32 FMA path (tp_gemm_simt.cu): EPI_STORE only (activations run separately).
+// fp32 FMA path (tp_gemm_simt.cu): the same epilogues, grouping and K concatenation.
 tp_status launch_gemm_f32(const GemmBatch& b, cudaStream_t st);
 
 // Attention core (tp_attention.cu).

@@ -185,6 +185,33 @@ def test_tiny_fp32_mlp_forward_backward():
     assert_close(m.db2[None, :], g["db2"][None, :], TOL_F32, "db2")
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["partials", "fused"])
+@pytest.mark.parametrize("act,bias", [("gelu", True), ("swiglu", False), ("none", True)])
+def test_fp32_mlp_every_epilogue(act, bias, fused):
+    """fp32 plans run the same fused epilogues as bf16 (bias + GELU, SwiGLU with
+    paired gate/up accumulators, their derivatives) in one grouped FMA launch,
+    and the shard sums fused into the row and dX GEMMs; ragged tiles (T = 200,
+    ffn/p = 72)."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    T, h, f, p = 200, 96, 288, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.float32, seed=17, bias=bias)
+    m = TPMLP(h, f, p, act, "f32", bias=bias, fused=fused)
+    m.load_weights(dev(inp.W1), dev(inp.W2), dev(inp.b1), dev(inp.b2))
+    Y = m.forward(dev(inp.X))
+    dX = m.backward(dev(inp.dY))
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    b1, b2 = (O.f64(inp.b1), O.f64(inp.b2)) if bias else (None, None)
+    ref = O.mlp_fwd(X, W1, b1, W2, b2, act)
+    g = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
+    assert_close(Y, ref["Y"], TOL_F32, "Y")
+    assert_close(dX, g["dX"], TOL_F32, "dX")
+    for i in range(p):
+        assert_close(m.dW1[i], _shard_w1(g["dW1"], act, p, i), TOL_F32, f"dW1 shard {i}")
+        assert_close(m.dW2[i], O.shard_cols(g["dW2"], p, i), TOL_F32, f"dW2 shard {i}")
+        if act != "none":
+            assert_close(m.Z[i], _shard_w1(ref["Z"].T, act, p, i).T, TOL_F32, f"Z shard {i}")
+
+
 @pytest.mark.parametrize("act,bias", [("gelu", True), ("swiglu", False)])
 def test_bf16_mlp_end_to_end_small(act, bias):
     """Whole sharded MLP (forward + backward through TPMLP) against the unsharded
