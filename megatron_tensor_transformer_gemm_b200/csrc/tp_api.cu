@@ -257,6 +257,37 @@ tp_status run_gemm(const tp_plan* plan, const GemmBatch& b, cudaStream_t st) {
   return launch_gemm_f32(b, st);
 }
 
+// A weight-gradient batch (every problem the same shape, outputs D[i] dense
+// [M, N] in the plan dtype). Problems with few output tiles and a long K (the
+// token dim) leave most SMs idle, so for bf16 plans, when the estimate says so,
+// the GEMM splits K: split s writes fp32 partials of every D[i] into the plan's
+// workspace and one reduce sums the splits in order into D[i].
+tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st) {
+  if (plan->dtype != TP_BF16) return run_gemm(plan, w, st);
+  const int s = gemm_split_k(w);
+  if (s <= 1 || s > TP_MAX_SHARDS) return launch_gemm_bf16(w, st);
+  const int n = w.n;
+  const int64_t M = w.g[0].M, N = w.g[0].N, mn = M * N, elems = n * mn;
+  for (int i = 0; i < n; ++i)
+    if (w.g[i].ldd != N) return launch_gemm_bf16(w, st);
+  void* ws = nullptr;
+  TP_TRY(workspace(plan, static_cast<size_t>(s) * elems * sizeof(float), &ws));
+  float* part = static_cast<float*>(ws);
+  MutPtrArray outs{};
+  for (int i = 0; i < n; ++i) {
+    outs.p[i] = w.g[i].D;
+    w.g[i].D = part + i * mn;
+  }
+  w.ksplit = s;
+  w.split_stride = elems;
+  w.out_f32 = true;
+  TP_TRY(launch_gemm_bf16(w, st));
+  PtrArray P{};
+  for (int j = 0; j < s; ++j) P.p[j] = part + j * elems;
+  return launch_reduce(P, s, nullptr, nullptr, PtrArray{}, false, outs, true, n, n * M, N, TP_F32,
+                       TP_BF16, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -1062,7 +1093,7 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
       g.D = dW[i];
       g.ldd = k;
     }
-    TP_TRY(run_gemm(plan, w, st));
+    TP_TRY(run_wgrad(plan, w, st));
   }
   if (dbias) TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, st));
   return TP_OK;
@@ -1113,7 +1144,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
       g.D = dW[i];
       g.ldd = h;
     }
-    TP_TRY(run_gemm(plan, w, st));
+    TP_TRY(run_wgrad(plan, w, st));
   }
   if (dX_out) {
     // dX_i [T, h] = dZ_i W_i: A = dZ_i (K-major), B(c, j) = W_i[j, c] (MN-major).

@@ -106,10 +106,23 @@ struct alignas(64) GemmParams {
   int rows_per_out;
   void* out_seq[TP_MAX_SHARDS];
   const void* res_seq[TP_MAX_SHARDS];
+  // Split K (ksplit > 1, EPI_STORE with fp32 outputs): every output tile runs
+  // ksplit times, split s over K blocks [s * kb_per_split, ...) writing its
+  // fp32 partial at D + s * split_stride; a reduce kernel sums the splits.
+  int ksplit;
+  int base_tiles;
+  int kb_per_split;
+  int64_t split_stride;
   unsigned* status;
 };
 
-__device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, int& mt, int& nt) {
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, int& mt, int& nt,
+                                            int& ks) {
+  ks = 0;
+  if (p.ksplit > 1) {
+    ks = t / p.base_tiles;
+    t -= ks * p.base_tiles;
+  }
   g = 0;
 #pragma unroll 1
   for (int i = 1; i < p.ngroups; ++i)
@@ -117,6 +130,19 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, 
   const int local = t - p.g[g].tile_begin;
   mt = local / p.g[g].tiles_n;
   nt = local - mt * p.g[g].tiles_n;
+}
+
+// K blocks of a tile: [kb0, kb0 + nkb) of its problem (the split's share
+// under split K, else all of them).
+__device__ __forceinline__ void kb_range(const GemmParams& p, const GroupArgs& ga, int ks, int& kb0,
+                                         int& nkb) {
+  if (p.ksplit > 1) {
+    kb0 = ks * p.kb_per_split;
+    nkb = min(p.kb_per_split, ga.num_kb - kb0);
+  } else {
+    kb0 = 0;
+    nkb = ga.num_kb;
+  }
 }
 
 // A tile with at most BN / 2 valid columns left (the ragged last N tile of a
@@ -171,7 +197,7 @@ __device__ __forceinline__ void load_row_chunk_bf16(const void* base, int64_t ld
 
 // Columns [half * BN/2, (half + 1) * BN/2) of the accumulator row this thread owns.
 __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t taddr, int row,
-                              int n0, int half, bool narrow) {
+                              int n0, int half, bool narrow, int ks) {
   const bool row_ok = row < ga.M;
   if (p.epi == tpi::EPI_SWIGLU) {
     // Accumulator columns [0,128) = gate units n0.., [128,256) = the same up units;
@@ -213,6 +239,7 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
           for (int i = 0; i < 32; ++i) v[i] += b[i];
         }
         void* dst = ga.D;
+        if (ks) dst = static_cast<float*>(dst) + ks * p.split_stride;  // split K: fp32 partials
         const void* res = ga.aux;
         int orow = row;
         if (p.scatter) {
@@ -340,9 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
     bool ok = true;
     for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
-      int g, mt, nt;
-      decode_tile(p, t, g, mt, nt);
+      int g, mt, nt, ks;
+      decode_tile(p, t, g, mt, nt, ks);
       const GroupArgs& ga = p.g[g];
+      int kb_first, kb_count;
+      kb_range(p, ga, ks, kb_first, kb_count);
       const int m0 = mt * C::TILE_M + static_cast<int>(rank) * BM;  // this CTA's A rows
       const int n0 = nt * p.tile_n;
       // this CTA's B rows (in a narrow tile of a pair, each CTA's first BN / 4)
@@ -354,13 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int nseg = p.kcat ? p.kcat : 1;
       for (int sg = 0; sg < nseg && ok; ++sg) {
         const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
-        const int nkb = p.kcat ? p.seg_kb[sg] : ga.num_kb;
+        const int nkb = p.kcat ? p.seg_kb[sg] : kb_count;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          const int k0 = kb * BK;
+          const int k0 = (p.kcat ? kb : kb_first + kb) * BK;
           uint8_t* a_dst = sA + stage * C::A_BYTES;
           uint8_t* b_dst = sB + stage * C::B_BYTES;
           if (PAIR == 1) {
@@ -428,11 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
-      int g, mt, nt;
-      decode_tile(p, t, g, mt, nt);
+      int g, mt, nt, ks;
+      decode_tile(p, t, g, mt, nt, ks);
       const uint32_t idesc =
           narrow_tile(p, p.g[g], nt * p.tile_n) ? idesc_narrow : idesc_full;
-      int num_kb = p.g[g].num_kb;
+      int kb_first, num_kb;
+      kb_range(p, p.g[g], ks, kb_first, num_kb);
       if (p.kcat) {
         num_kb = 0;
         for (int sg = 0; sg < p.kcat; ++sg) num_kb += p.seg_kb[sg];
@@ -486,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     uint32_t acc_phase = 0;
     const uint32_t tempty_leader = PAIR == 2 ? map_shared(smem_u32(&tempty[0]), 0) : 0u;
     for (int t = first_tile; t < p.total_tiles; t += tile_stride) {
-      int g, mt, nt;
-      decode_tile(p, t, g, mt, nt);
+      int g, mt, nt, ks;
+      decode_tile(p, t, g, mt, nt, ks);
       const GroupArgs& ga = p.g[g];
       // warp-uniform: the epilogue's tcgen05.ld is warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) break;
@@ -496,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int n0 = nt * p.tile_n;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_tile(p, ga, taddr, row, n0, half, narrow_tile(p, ga, n0));
+      epilogue_tile(p, ga, taddr, row, n0, half, narrow_tile(p, ga, n0), ks);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -581,8 +611,9 @@ struct Layout {
 // move more operand bytes per FLOP (one CTA instead of a pair, N = 128
 // instead of 256) carry a factor, so they win only when they fill more SMs:
 // small problems, whose 256 x 256 tiles leave most of the GPU idle.
-Layout choose_layout(const GemmBatch& b, int sms) {
+Layout choose_layout(const GemmBatch& b, int sms, double* cost_out = nullptr) {
   const bool swiglu = b.epi == tpi::EPI_SWIGLU;
+  const int ks = b.ksplit > 1 ? b.ksplit : 1;
   const int nout = b.kcat ? 1 : b.n;
   int64_t kb_cat = 0;
   if (b.kcat)
@@ -603,12 +634,13 @@ Layout choose_layout(const GemmBatch& b, int sms) {
         const GemmProblem& o = b.g[i];
         const int64_t mt = (o.M + tile_m - 1) / tile_m;
         const int64_t nt = (o.N + tn - 1) / tn;
-        const int64_t kb = b.kcat ? kb_cat : (o.K + BK - 1) / BK;
+        const int64_t kb_all = b.kcat ? kb_cat : (o.K + BK - 1) / BK;
+        const int64_t kb = (kb_all + ks - 1) / ks;  // K blocks of one split
         const int last = o.N - static_cast<int>(nt - 1) * tn;  // columns of the last N tile
         const int mma_n = swiglu ? BN : (nar ? BN / 2 : BN);
         const int last_n = (!swiglu && last <= BN / 2) ? BN / 2 : mma_n;
-        tiles += mt * nt;
-        work += static_cast<double>(mt) * kb * ((nt - 1) * mma_n + last_n);
+        tiles += mt * nt * ks;
+        work += static_cast<double>(mt) * ks * kb * ((nt - 1) * mma_n + last_n);
       }
       const int64_t units = std::max(1, sms / pair);
       const double waves = static_cast<double>((tiles + units - 1) / units);
@@ -620,6 +652,7 @@ Layout choose_layout(const GemmBatch& b, int sms) {
       }
     }
   }
+  if (cost_out) *cost_out = best_cost;
   return best;
 }
 
@@ -691,6 +724,13 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     if (b.g[i].M <= 0 || b.g[i].N <= 0)
       return fail(TP_ERR_ARG, "GEMM %d has an empty output (%d x %d)", i, b.g[i].M, b.g[i].N);
   const int sms = device_sms();
+  int ksplit = b.ksplit > 1 ? b.ksplit : 1;
+  if (ksplit > 1) {
+    if (b.kcat || b.scatter_n || b.epi != EPI_STORE || !b.out_f32)
+      return fail(TP_ERR_ARG, "split K needs plain fp32 outputs (no K concatenation or scatter)");
+    for (int i = 1; i < b.n; ++i)
+      if (b.g[i].K != b.g[0].K) return fail(TP_ERR_ARG, "split K needs every problem with the same K");
+  }
   const Layout lay = choose_layout(b, sms);
   const int pair = lay.pair;
   const int tile_n = (swiglu || lay.narrow) ? BN / 2 : BN;
@@ -750,6 +790,18 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
       p.res_seq[j] = b.res_seq[j];
     }
   }
+  if (ksplit > 1) {
+    const int nkb = (b.g[0].K + BK - 1) / BK;
+    const int kbps = (nkb + ksplit - 1) / ksplit;
+    if ((nkb + kbps - 1) / kbps != ksplit)
+      return fail(TP_ERR_ARG, "split K of %d over %d K blocks leaves a split empty", ksplit, nkb);
+    if (static_cast<int64_t>(tiles) * ksplit > 0x7fffffffLL) return fail(TP_ERR_UNSUPPORTED, "too many GEMM tiles");
+    p.ksplit = ksplit;
+    p.base_tiles = tiles;
+    p.kb_per_split = kbps;
+    p.split_stride = b.split_stride;
+    tiles *= ksplit;
+  }
   p.ngroups = nout;
   p.total_tiles = tiles;
   p.tile_n = tile_n;
@@ -762,6 +814,43 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   if (s != TP_OK) return s;
   if (pair == 2) return launch_kernel<2>(p, tiles, sms, st);
   return launch_kernel<1>(p, tiles, sms, st);
+}
+
+int gemm_split_k(const GemmBatch& b) {
+  if (b.kcat || b.scatter_n || b.epi != EPI_STORE || b.n < 1) return 1;
+  for (int i = 1; i < b.n; ++i)
+    if (b.g[i].K != b.g[0].K || b.g[i].M != b.g[0].M || b.g[i].N != b.g[0].N) return 1;
+  const int sms = device_sms();
+  const int nkb = (b.g[0].K + BK - 1) / BK;
+  if (const char* e = getenv("TP_GEMM_SPLITK")) {  // forced split (tests): 1..16
+    const int f = std::max(1, std::min(16, std::min(nkb, atoi(e))));
+    const int kbps = (nkb + f - 1) / f;
+    return (nkb + kbps - 1) / kbps;
+  }
+  // Cost units of choose_layout: one K block of one column on a 128-row slab
+  // of one SM (16 KFLOP, about 1.25 ns at the clocks seen under load). The
+  // reduce reads the fp32 partials once and writes the outputs once at about
+  // 6 KB per unit, plus about 2 us of launch and ramp.
+  const double out_bytes = static_cast<double>(b.n) * b.g[0].M * b.g[0].N;
+  GemmBatch t = b;
+  t.out_f32 = true;
+  t.ksplit = 1;
+  double best_cost = 0.0;
+  choose_layout(t, sms, &best_cost);
+  int best = 1;
+  for (int s = 2; s <= 16; s *= 2) {
+    if (nkb < 4 * s) break;  // at least four K blocks per split
+    t.ksplit = s;
+    double c = 0.0;
+    choose_layout(t, sms, &c);
+    c += (out_bytes * (4.0 * s + 2.0)) / 6000.0 + 1600.0;
+    if (c < 0.9 * best_cost) {
+      best_cost = c;
+      best = s;
+    }
+  }
+  const int kbps = (nkb + best - 1) / best;
+  return (nkb + kbps - 1) / kbps;  // every split gets at least one K block
 }
 
 }  // namespace tpi

@@ -153,10 +153,18 @@ struct GemmBatch {
   int64_t rows_per_out;
   void* out_seq[TP_MAX_SHARDS];
   const void* res_seq[TP_MAX_SHARDS];
+  // Split K (bf16 path, EPI_STORE, fp32 outputs, every problem with the same
+  // K): ksplit > 1 runs each output tile ksplit times over consecutive K
+  // ranges, split s writing its fp32 partial at g[i].D + s * split_stride.
+  int ksplit;
+  int64_t split_stride;
 };
 
 // bf16 tcgen05 tensor-core path (tp_gemm_sm100.cu).
 tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st);
+// The K split that minimises the estimated time of a batch of plain bf16-output
+// GEMMs of equal shape, counting the fp32 partials' reduce (1 = no split, <= 16).
+int gemm_split_k(const GemmBatch& b);
 // fp32 FMA path (tp_gemm_simt.cu): the same epilogues, grouping and K concatenation.
 tp_status launch_gemm_f32(const GemmBatch& b, cudaStream_t st);
 

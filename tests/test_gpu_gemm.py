@@ -3,6 +3,8 @@
 Shapes span several 128x256 tiles and end in ragged tails in M (tokens), N
 (output features) and K (reduction), including a final K block that is
 partly out of bounds."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -12,6 +14,8 @@ import tp_synth
 from gpu_helpers import TOL_BF16, TOL_F32, assert_close, dev
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _tp():
@@ -377,3 +381,38 @@ def test_host_step_pipeline_matches_direct_steps():
     for (Yr, dXr), (Yh, dXh) in zip(ref, outs):
         assert torch.equal(Yr, Yh)
         assert torch.equal(dXr, dXh)
+
+
+@pytest.mark.parametrize("splits", ["2", "3", "16"])
+def test_weight_gradients_with_split_k(splits):
+    """Weight gradients whose K (the token dim) is split over several tile
+    passes writing fp32 partials, summed in order by the reduce kernel into
+    each shard's dW: forced split counts, ragged K (T = 1000: 16 K blocks, the
+    last one partial), GELU and SwiGLU, in a subprocess so the forced split is
+    read by a fresh library."""
+    import subprocess
+    import sys
+    code = f"""
+import sys; sys.path.insert(0, {ROOT!r}); sys.path.insert(0, {os.path.join(ROOT, 'tests')!r})
+import numpy as np, torch, oracle as O, tp_synth
+from gpu_helpers import TOL_BF16, assert_close, dev
+from megatron_tensor_transformer_gemm_b200.block import TPMLP
+for act in ("gelu", "swiglu"):
+    T, h, f, p = 1000, 256, 512, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=23)
+    m = TPMLP(h, f, p, act, "bf16", fused=True)
+    m.load_weights(dev(inp.W1), dev(inp.W2))
+    m.forward(dev(inp.X)); m.backward(dev(inp.dY))
+    X, W1, W2, dY = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    ref = O.mlp_fwd(X, W1, None, W2, None, act)
+    g = O.mlp_bwd(X, W1, W2, ref["Z"], ref["H"], dY, act)
+    for i in range(p):
+        sh1 = O.shard_gate_up(g["dW1"], p, i) if act == "swiglu" else O.shard_rows(g["dW1"], p, i)
+        assert_close(m.dW1[i], sh1, TOL_BF16, f"dW1 shard {{i}}")
+        assert_close(m.dW2[i], O.shard_cols(g["dW2"], p, i), TOL_BF16, f"dW2 shard {{i}}")
+print("ok")
+"""
+    env = dict(os.environ, TP_GEMM_SPLITK=splits)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
