@@ -466,11 +466,25 @@ def run_ours(args, world, rank, local):
     if not args.skip_e2e:
         e2e = run_e2e(m, X_h, dY_h, T, flops, args, world, stream)
     coll = None if args.skip_collectives else time_sp_collectives(peaks, stream, rank)
+    others = None
+    if not args.skip_workloads and world == 1:
+        # free the 7B buffers first; every other configuration, briefly
+        del m, X, dY
+        torch.cuda.empty_cache()
+        others = {}
+        for wl, graph in (("sp", False), ("attn", False), ("stack", True)):
+            sub = argparse.Namespace(**vars(args))
+            sub.workload, sub.steps, sub.warmup, sub.graph = wl, 10, 3, graph
+            o = measure_other(sub, world, rank, local, sample_clocks=False)
+            keep = ("value", "unit", "ms_per_step", "frac_of_burst_peak", "roofline", "gpu_launches",
+                    "device_status")
+            others[wl] = {"workload": o["config"]["workload"], "cuda_graph": graph,
+                          **{k: o[k] for k in keep}}
     status = tp.device_status()
     if rank != 0:
         return 0
     return report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks,
-                  red_gbs, red_bytes, e2e, launches, clk, status, red_where, coll)
+                  red_gbs, red_bytes, e2e, launches, clk, status, red_where, coll, others)
 
 
 def time_standalone_reduce(pl, T, steps, stream):
@@ -612,7 +626,7 @@ def measured_traffic(T, variant):
 
 
 def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks, red_gbs,
-           red_bytes, e2e, launches, clk, status, red_where, coll):
+           red_bytes, e2e, launches, clk, status, red_where, coll, others=None):
     traffic, per_launch = measured_traffic(T, args.variant) or (None, None)
     alg = gemm_algorithmic_bytes(T, HIDDEN, FFN)
     alg_mean = sum(alg) / len(alg)
@@ -648,6 +662,7 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
                    "frac_of_8TBs": red_gbs / 8000.0, "bytes_per_launch": red_bytes,
                    "measured": red_where},
         "collectives": coll,
+        "workloads": others,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
@@ -659,11 +674,21 @@ def report(args, world, T, ms, value, flops, gemm_tflops, n_gemm_launches, peaks
 
 
 def run_other(args, world, rank, local):
+    """--workload attn|sp|stack: one of the other configurations, printed as
+    the JSON line of measure_other."""
+    out = measure_other(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def measure_other(args, world, rank, local, sample_clocks=True):
     """Device-timed throughput of the other workloads (parity cases of the
-    suite), printed in the same JSON form: the attention block forward
-    (hidden 4096, 32 heads x 128, seq 4096, batch 2, p 8), the Megatron-SP
-    SwiGLU MLP fwd+bwd (hidden 8192, ffn 28672, seq 8192, p 8) and the
-    12-layer stack fwd+bwd (hidden 512, MLP 2048, 8 heads, tokens 8x512, p 4)."""
+    suite): the attention block forward (hidden 4096, 32 heads x 128, seq
+    4096, batch 2, p 8) with its attention core forward and backward timed
+    alone, the Megatron-SP SwiGLU MLP fwd+bwd (hidden 8192, ffn 28672, seq
+    8192, p 8) and the 12-layer stack fwd+bwd (hidden 512, MLP 2048, 8 heads,
+    tokens 8x512, p 4). Returns the JSON-line dict."""
     import torch
     import tp_synth
     from megatron_tensor_transformer_gemm_b200 import tp
@@ -733,7 +758,8 @@ def run_other(args, world, rank, local):
             step()
         torch.cuda.synchronize()
     clocks = ClockSampler(local)
-    clocks.start()
+    if sample_clocks:
+        clocks.start()
     barrier(world)
     torch.cuda.synchronize()
     tp.launch_count(reset=True)
@@ -747,7 +773,7 @@ def run_other(args, world, rank, local):
     launches = tp.launch_count(reset=True)
     if graph is not None:
         launches = graph.launches * args.steps  # replays launch the captured kernels
-    clk = clocks.stop()
+    clk = clocks.stop() if sample_clocks else None
     value, ms = aggregate(flops, args.steps, e0.elapsed_time(e1), world)
     roof = None
     if core is not None:
@@ -782,17 +808,19 @@ def run_other(args, world, rank, local):
             roof["backward"] = {"kernel": "attn_bwd_prep + attn_bwd_dkdv + attn_bwd_dq (tcgen05)",
                                 "achieved": achb, "unit": "TFLOP/s", "frac": achb / peaks["bf16_tflops"],
                                 "flops_per_launch_set": 2.5 * core_flops}
-    if rank != 0:
-        return 0
-    print(json.dumps({"metric": f"{args.workload} TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",
-                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                      "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-                      "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded tp_synth)",
-                      "config": {"workload": name, "variant": args.variant,
-                                 "cuda_graph": bool(args.graph)}, "roofline": roof,
-                      "gpu_launches": launches, "clocks": clk,
-                      "device_status": tp.device_status()}), flush=True)
-    return 0
+    out = {"metric": f"{args.workload} TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded tp_synth)",
+           "config": {"workload": name, "variant": args.variant,
+                      "cuda_graph": bool(args.graph)}, "roofline": roof,
+           "frac_of_burst_peak": value / peaks["bf16_tflops"],
+           "gpu_launches": launches, "clocks": clk,
+           "device_status": tp.device_status()}
+    if graph is not None:
+        del graph
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_hbm(args, world, rank, local):
@@ -970,6 +998,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--skip-collectives", action="store_true",
                     help="skip the Megatron-SP collective GB/s measurements")
+    ap.add_argument("--skip-workloads", action="store_true",
+                    help="skip the brief runs of the other configurations (SP, attention, stack)")
     ap.add_argument("--variant", choices=["fused", "partials", "overlap"], default="fused",
                     help="sum over shards inside the GEMMs (fused), via p partials + reduce, "
                          "or partials with each token block's reduce overlapped with the next "
