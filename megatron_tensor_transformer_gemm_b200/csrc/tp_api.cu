@@ -1175,8 +1175,9 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     TP_TRY(run_gemm(plan, d, st));
   }
   if (dbias)
-    for (int i = 0; i < p; ++i)
-      TP_TRY(launch_column_sum(plan, dZ[i], T, n, n, dbias[i], 0, plan->dtype, st));
+    TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p),
+                                     p, T, n, n, to_marr(reinterpret_cast<void* const*>(dbias), p), 0,
+                                     plan->dtype, st));
   return TP_OK;
 }
 

@@ -75,6 +75,10 @@ tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_
                         tp_dtype dt, cudaStream_t st);
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
                             float* out, int accumulate, tp_dtype dt, cudaStream_t st);
+// The same for n inputs of one shape at once (one pass-1 and one pass-2 launch).
+tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
+                                    int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
+                                    tp_dtype dt, cudaStream_t st);
 
 // LayerNorm (tp_layernorm.cu).
 tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,

@@ -263,6 +263,56 @@ __global__ void colsum_pass2(const float* part, int splits, int64_t cols, float*
   out[c] = accumulate ? out[c] + s : s;
 }
 
+// Column sums of n same-shape inputs in one launch (blockIdx.z = input):
+// pass 1 as colsum_pass1 over X.p[z], partials at part + z * splits * cols.
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_grouped_pass1(const __grid_constant__ PtrArray X,
+                                                            int64_t ld, int64_t rows, int64_t vpr,
+                                                            int64_t rows_per_split, float* part,
+                                                            int64_t cols) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[8][32 * V + 1];
+  const T* x = static_cast<const T*>(X.p[blockIdx.z]);
+  float* pz = part + static_cast<int64_t>(blockIdx.z) * gridDim.y * cols;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(rows, r0 + rows_per_split);
+  float acc[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) acc[k] = 0.f;
+  if (cv < vpr) {
+    for (int64_t r = r0 + ty; r < r1; r += 8) {
+      float f[V];
+      Vec<T>::load(ld_stream(x + r * ld + cv * V), f);
+#pragma unroll
+      for (int k = 0; k < V; ++k) acc[k] += f[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < V; ++k) red[ty][tx * V + k] = acc[k];
+  __syncthreads();
+  for (int c = threadIdx.x; c < 32 * V; c += 256) {
+    float sum = 0.f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) sum += red[y][c];
+    const int64_t col = static_cast<int64_t>(blockIdx.x) * 32 * V + c;
+    if (col < cols) pz[static_cast<int64_t>(blockIdx.y) * cols + col] = sum;
+  }
+}
+
+// Pass 2 of the grouped sums: out.p[blockIdx.y][c] (+)= sum over splits in order.
+__global__ void colsum_grouped_pass2(const float* part, int splits, int64_t cols,
+                                     const __grid_constant__ MutPtrArray out, int accumulate) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const float* pz = part + static_cast<int64_t>(blockIdx.y) * splits * cols;
+  float sum = 0.f;
+  for (int k = 0; k < splits; ++k) sum += pz[static_cast<int64_t>(k) * cols + c];
+  float* o = static_cast<float*>(out.p[blockIdx.y]);
+  o[c] = accumulate ? o[c] + sum : sum;
+}
+
 // Block shape for row-walking kernels: x covers column vectors, y rows.
 void row_walk_shape(int64_t vpr, int64_t rows, dim3* grid, dim3* block) {
   int bx = static_cast<int>(std::min<int64_t>(kThreads, ((vpr + 31) / 32) * 32));
@@ -380,6 +430,36 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
   colsum_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
       part, static_cast<int>(splits), cols, out, accumulate);
   return after_launch("column_sum/pass2");
+}
+
+tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
+                                    int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
+                                    tp_dtype dt, cudaStream_t st) {
+  if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "column sums of %d inputs", n);
+  const int V = dt == TP_BF16 ? 8 : 4;
+  const int64_t vpr = cols / V;
+  const int gx = static_cast<int>((vpr + 31) / 32);
+  int64_t splits = std::max<int64_t>(1, (static_cast<int64_t>(sm_count()) * 8) / (gx * n));
+  splits = std::min<int64_t>(splits, std::max<int64_t>(1, (rows + 63) / 64));
+  splits = std::min<int64_t>(splits, 1024);
+  const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
+  splits = rows > 0 ? (rows + rps - 1) / rps : 0;
+  void* ws = nullptr;
+  tp_status s = workspace(plan, static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float), &ws);
+  if (s != TP_OK) return s;
+  float* part = static_cast<float*>(ws);
+  if (rows > 0) {
+    dim3 grid(gx, static_cast<unsigned>(splits), static_cast<unsigned>(n));
+    if (dt == TP_BF16)
+      colsum_grouped_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(x, ld, rows, vpr, rps, part, cols);
+    else
+      colsum_grouped_pass1<float><<<grid, 256, 0, st>>>(x, ld, rows, vpr, rps, part, cols);
+    s = after_launch("column_sum_grouped/pass1");
+    if (s != TP_OK) return s;
+  }
+  colsum_grouped_pass2<<<dim3(static_cast<unsigned>((cols + 255) / 256), static_cast<unsigned>(n)), 256, 0,
+                         st>>>(part, static_cast<int>(splits), cols, out, accumulate);
+  return after_launch("column_sum_grouped/pass2");
 }
 
 }  // namespace tpi
