@@ -326,3 +326,18 @@ def test_bounded_wait_times_out_and_reports():
     plan.reduce_partials(16, [dev(x) for x in P], dev(b), None, Y)
     assert_bitexact(Y, O.reduce_partials([O.f64(x) for x in P], O.f64(b)), "reduce after a timeout")
     assert tp.device_status(plan=plan) == "TP_OK"
+
+
+@pytest.mark.parametrize("n,t,h", [(8, 600, 1032), (3, 1000, 4096), (2, 64, 8192)])
+def test_all_gather_bulk_copy_bitexact(n, t, h):
+    """The sequence all-gather of shards of 1 MB and more runs as bulk copies of
+    32 KB chunks through shared memory; shard sizes that end in a partial chunk
+    (600 rows x 2064 bytes) and shards of exactly 1 MB are copied bit for bit."""
+    tp = _tp()
+    g = torch.Generator().manual_seed(n * t + h)
+    xs = [torch.randn(t, h, generator=g).to(torch.bfloat16) for _ in range(n)]
+    plan = tp.Plan(h, 0, 0, 1, "bf16", "none")
+    out = torch.full((n * t, h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    plan.all_gather_seq(n * t, [dev(x) for x in xs], out)
+    assert torch.equal(out.cpu(), torch.cat(xs, 0))
+    assert tp.device_status() == "TP_OK"
