@@ -17,6 +17,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -39,10 +40,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct BwdParams {
   CUtensorMap tm_qkv[TP_MAX_SHARDS];  // {3*Hl*d, batch, seq}, box {64, 1, 128}
   CUtensorMap tm_do[TP_MAX_SHARDS];   // {Hl*d, batch, seq}, box {64, 1, 128}
+  CUtensorMap tm_q64[TP_MAX_SHARDS];  // the same QKV, box {64, 1, 64}
+  CUtensorMap tm_do64[TP_MAX_SHARDS]; // the same dO, box {64, 1, 64}
   void* dqkv[TP_MAX_SHARDS];
   const float* lse[TP_MAX_SHARDS];
-  const float* dvec[TP_MAX_SHARDS];
+  const float* dvec[TP_MAX_SHARDS];   // D, [batch * hl][seq_pad]
+  const float* lse2[TP_MAX_SHARDS];   // lse * log2(e), [batch * hl][seq_pad]
   int p, batch, seq, hl, nq, nkv;
+  int seq_pad;                        // seq rounded up to a multiple of 64
   float scale_log2;  // log2(e) / sqrt(d)
   float scale;       // 1 / sqrt(d)
   unsigned* status;
@@ -85,10 +90,12 @@ __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, __nv_bfloat16
   }
 }
 
-// D[row] = sum_c dO[row, c] * O[row, c] for every (shard, b, head, q).
+// D[row] = sum_c dO[row, c] * O[row, c] for every (shard, b, head, q), and
+// lse2[row] = lse[row] * log2(e); both into [batch * hl][seq_pad] arrays.
 __global__ void attn_bwd_prep(const __grid_constant__ PtrArray O, const __grid_constant__ PtrArray dO,
-                              const __grid_constant__ MutPtrArray dvec, int p, int batch, int seq,
-                              int hl, int d) {
+                              const __grid_constant__ PtrArray LSE, const __grid_constant__ MutPtrArray dvec,
+                              const __grid_constant__ MutPtrArray lse2, int p, int batch, int seq,
+                              int seq_pad, int hl, int d) {
   const int64_t rows_per_shard = static_cast<int64_t>(batch) * hl * seq;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x & 31;
@@ -110,7 +117,11 @@ __global__ void attn_bwd_prep(const __grid_constant__ PtrArray O, const __grid_c
   }
 #pragma unroll
   for (int k = 16; k > 0; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
-  if (lane == 0) static_cast<float*>(dvec.p[shard])[(static_cast<int64_t>(b) * hl + hh) * seq + q] = s;
+  if (lane == 0) {
+    const int64_t bh = static_cast<int64_t>(b) * hl + hh;
+    static_cast<float*>(dvec.p[shard])[bh * seq_pad + q] = s;
+    static_cast<float*>(lse2.p[shard])[bh * seq_pad + q] = static_cast<const float*>(LSE.p[shard])[bh * seq + q] * kLog2e;
+  }
 }
 
 // Row r of this CTA's 128 x 128 (query x key) block, 32-column chunks
@@ -282,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
     const int r = lg * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const float* lse = p.lse[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
-    const float* dv = p.dvec[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
+    const float* dv = p.dvec[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq_pad;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int q = (j + it) * BQ + r;
@@ -305,6 +316,257 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_consta
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
       tc_fence_after();
       const int key = k0 + r;  // accumulator lane = key row
+      __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
+                            (static_cast<int64_t>(key) * p.batch + b) * (3 * hl_d) + hh * D;
+      const bool st_ok = key < p.seq;
+      if (half == 0) tmem_row_to_global<D>(tdV + lane_off, base + 2 * hl_d, 1.f, st_ok);
+      else tmem_row_to_global<D>(tdK + lane_off, base + hl_d, p.scale, st_ok);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK / dV with keys as the MMA rows and 64-query sub-tiles, two in flight.
+// One CTA per 128-key block of one (shard, batch, head). For each sub-tile of
+// 64 queries that sees the block:
+//   S^T = K Q_s^T and dP^T = V dO_s^T      (M = 128 keys, N = 64 queries)
+//   P^T = exp2(S^T * scale * log2e - lse2), dS^T = P^T * (dP^T - D)  (element-wise)
+//   dV += P^T dO_s, dK += dS^T Q_s         (M = 128 keys, N = d, K = 64 queries)
+// TMEM holds dV and dK (d columns each) and two (S^T, dP^T) pairs of 64
+// columns each, so the MMAs of sub-tile i + 1 (and the dV / dK MMAs of i - 1)
+// run while the element-wise warps turn sub-tile i into P^T and dS^T.
+// Q_s, dO_s and their 64 values of lse2 and D stream through ST stages.
+template <int D, int ST>
+struct DkdvStSmem {
+  static constexpr int KV = 128 * D * 2;    // one [128 x D] bf16 tile
+  static constexpr int QS = 64 * D * 2;     // one [64 x D] bf16 sub-tile
+  static constexpr int CH = 64 * 128;       // a 64-row 128B-swizzle column chunk of a sub-tile
+  static constexpr int PT = 128 * 128;      // [128 keys x 64 queries] bf16 (one swizzle chunk)
+  static constexpr int TOTAL = 1024 + 2 * KV + 2 * ST * QS + 4 * PT + ST * 512 + 256;
+};
+
+template <int D, int ST>
+__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_constant__ BwdParams p) {
+  using SM = DkdvStSmem<D, ST>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + SM::KV;
+  uint8_t* sQ = sV + SM::KV;           // [ST]
+  uint8_t* sdO = sQ + ST * SM::QS;     // [ST]
+  uint8_t* sP = sdO + ST * SM::QS;     // [2] P^T buffers
+  uint8_t* sdS = sP + 2 * SM::PT;      // [2] dS^T buffers
+  float* sL = reinterpret_cast<float*>(sdS + 2 * SM::PT);  // [ST][64] lse2 then [ST][64] D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sL + ST * 128);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = kv_full + 1;      // [ST]
+  uint64_t* q_empty = q_full + ST;     // [ST]
+  uint64_t* s_full = q_empty + ST;     // [2]
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* pds_empty = p_full + 2;    // [2]
+  uint64_t* acc_full = pds_empty + 2;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = p.p * p.batch * p.hl;
+  const int j = static_cast<int>(blockIdx.x) / per;  // key block; j = 0 has the most work
+  int rest = static_cast<int>(blockIdx.x) % per;
+  const int hh = rest % p.hl;
+  rest /= p.hl;
+  const int b = rest % p.batch;
+  const int shard = rest / p.batch;
+  const int k0 = j * BKV;
+  const int nsub = (p.seq + 63) / 64 - 2 * j;  // 64-query sub-tiles 2j .. that see this key block
+  const int hl_d = p.hl * D;
+  const int64_t bh = static_cast<int64_t>(b) * p.hl + hh;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 8);
+      mbar_init(&pds_empty[x], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tdV = tmem, tdK = tmem + D;
+  const uint32_t tS0 = tmem + 2 * D;  // buffer x: S^T at tS0 + 128 x, dP^T at tS0 + 128 x + 64
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    const CUtensorMap* tq = &p.tm_qkv[shard];
+    const CUtensorMap* tq64 = &p.tm_q64[shard];
+    const CUtensorMap* tdo64 = &p.tm_do64[shard];
+    tma_prefetch_desc(tq);
+    tma_prefetch_desc(tq64);
+    tma_prefetch_desc(tdo64);
+    mbar_arrive_expect_tx(kv_full, 2 * SM::KV);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sK + c * 128 * 128, tq, kv_full, hl_d + hh * D + c * 64, b, k0);
+      tma_load_3d(sV + c * 128 * 128, tq, kv_full, 2 * hl_d + hh * D + c * 64, b, k0);
+    }
+    const float* lse2 = p.lse2[shard] + bh * p.seq_pad;
+    const float* dv = p.dvec[shard] + bh * p.seq_pad;
+    int last_par[ST];
+    for (int s = 0; s < ST; ++s) last_par[s] = -1;
+    for (int it = 0; it < nsub; ++it) {
+      const int st = it % ST;
+      const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
+      if (!mbar_wait(&q_empty[st], ph ^ 1u, abort_flag, p.status)) break;
+      const int q0 = (2 * j + it) * 64;
+      mbar_arrive_expect_tx(&q_full[st], 2 * SM::QS + 512);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sQ + st * SM::QS + c * SM::CH, tq64, &q_full[st], hh * D + c * 64, b, q0);
+        tma_load_3d(sdO + st * SM::QS + c * SM::CH, tdo64, &q_full[st], hh * D + c * 64, b, q0);
+      }
+      bulk_load(sL + st * 128, lse2 + q0, 256, &q_full[st]);
+      bulk_load(sL + st * 128 + 64, dv + q0, 256, &q_full[st]);
+      last_par[st] = static_cast<int>(ph);
+    }
+    mbar_wait(kv_full, 0, abort_flag, p.status);
+    for (int s = 0; s < ST; ++s)
+      if (last_par[s] >= 0) mbar_wait(&q_full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t id_s = idesc_bf16(BKV, 64, false, false);  // M = 128 keys, N = 64 queries
+    const uint32_t id_acc = idesc_bf16(BKV, D, false, true);  // M = 128 keys, N = d, B MN-major
+    const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+    bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
+    // dV += P^T dO_s and dK += dS^T Q_s of sub-tile `it` (buffer it & 1)
+    auto acc_mmas = [&](int it) -> bool {
+      const int x = it & 1, st = it % ST;
+      if (!mbar_wait(&p_full[x], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, p.status)) return false;
+      tc_fence_after();
+      const uint32_t p_base = smem_u32(sP + x * SM::PT), ds_base = smem_u32(sdS + x * SM::PT);
+      const uint32_t q_base = smem_u32(sQ + st * SM::QS), do_base = smem_u32(sdO + st * SM::QS);
+#pragma unroll
+      for (int kk = 0; kk < 64 / 16; ++kk) {  // K = the sub-tile's 64 queries
+        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+        tc_mma_bf16(tdV, smem_desc_sw128(p_base + kk * 32, 16, 1024),
+                    smem_desc_sw128(do_base + kk * 2048, SM::CH, 1024), id_acc, acc);
+        tc_mma_bf16(tdK, smem_desc_sw128(ds_base + kk * 32, 16, 1024),
+                    smem_desc_sw128(q_base + kk * 2048, SM::CH, 1024), id_acc, acc);
+      }
+      tc_commit(&q_empty[st]);
+      tc_commit(&pds_empty[x]);
+      return true;
+    };
+    for (int it = 0; ok && it < nsub; ++it) {
+      const int st = it % ST, x = it & 1;
+      if (!mbar_wait(&q_full[st], static_cast<uint32_t>(it / ST) & 1u, abort_flag, p.status)) break;
+      tc_fence_after();
+      // buffer x was last read by the element-wise pass of it - 2, whose
+      // completion acc_mmas(it - 2) already waited for
+      const uint32_t q_base = smem_u32(sQ + st * SM::QS), do_base = smem_u32(sdO + st * SM::QS);
+      const uint32_t tS = tS0 + 128 * x, tdP = tS + 64;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t aoff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+        const uint32_t boff = (kk / 4) * SM::CH + (kk % 4) * 32;
+        tc_mma_bf16(tS, smem_desc_sw128(k_base + aoff, 16, 1024), smem_desc_sw128(q_base + boff, 16, 1024),
+                    id_s, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t aoff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
+        const uint32_t boff = (kk / 4) * SM::CH + (kk % 4) * 32;
+        tc_mma_bf16(tdP, smem_desc_sw128(v_base + aoff, 16, 1024), smem_desc_sw128(do_base + boff, 16, 1024),
+                    id_s, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(&s_full[x]);
+      if (it > 0 && !acc_mmas(it - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && nsub > 0) ok = acc_mmas(nsub - 1);
+    tc_commit(acc_full);
+    tc_commit(drain);
+    mbar_wait(drain, 0, abort_flag, p.status);
+  } else if (warp >= 2) {
+    // --------------------------------------------------------- element-wise
+    const int lg = warp & 3;
+    const int half = (warp - 2) / 4;  // query columns [32 half, 32 half + 32) of a sub-tile
+    const int r = lg * 32 + lane;     // key row of the block
+    const int key = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < nsub; ++it) {
+      const int x = it & 1, st = it % ST;
+      const uint32_t ph2 = static_cast<uint32_t>(it >> 1) & 1u;
+      // warp-uniform: the tcgen05.ld below is warp-collective
+      const bool got = mbar_wait(&s_full[x], ph2, abort_flag, p.status) &&
+                       mbar_wait(&pds_empty[x], ph2 ^ 1u, abort_flag, p.status) &&
+                       mbar_wait(&q_full[st], static_cast<uint32_t>(it / ST) & 1u, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tS = tS0 + 128 * x, tdP = tS + 64;
+      float sv[32], dp[32];
+      tmem_ld32(tS + lane_off + half * 32, sv);
+      tmem_ld32(tdP + lane_off + half * 32, dp);
+      tc_wait_ld();
+      const float* l2 = sL + st * 128 + half * 32;
+      const float* dd = l2 + 64;
+      const int qb = (2 * j + it) * 64 + half * 32;  // query of column 0 of this half
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int qa = qb + e;
+        const bool v0 = key <= qa && qa < p.seq && key < p.seq;
+        const bool v1 = key <= qa + 1 && qa + 1 < p.seq && key < p.seq;
+        const float p0 = v0 ? exp2f(sv[e] * p.scale_log2 - l2[e]) : 0.f;
+        const float p1 = v1 ? exp2f(sv[e + 1] * p.scale_log2 - l2[e + 1]) : 0.f;
+        pk[e / 2] = pack_bf16x2(p0, p1);
+        dk[e / 2] = pack_bf16x2(v0 ? p0 * (dp[e] - dd[e]) : 0.f, v1 ? p1 * (dp[e + 1] - dd[e + 1]) : 0.f);
+      }
+      // row r of the [128 keys x 64 queries] K-major tiles: 16-byte chunks
+      // 4 half .. 4 half + 3 of its 128-byte swizzled row
+      uint8_t* prow = sP + x * SM::PT + r * 128;
+      uint8_t* drow = sdS + x * SM::PT + r * 128;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int qv = half * 4 + v;
+        *reinterpret_cast<uint4*>(prow + ((qv ^ (r & 7)) << 4)) =
+            make_uint4(pk[v * 4 + 0], pk[v * 4 + 1], pk[v * 4 + 2], pk[v * 4 + 3]);
+        *reinterpret_cast<uint4*>(drow + ((qv ^ (r & 7)) << 4)) =
+            make_uint4(dk[v * 4 + 0], dk[v * 4 + 1], dk[v * 4 + 2], dk[v * 4 + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[x]);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
+      tc_fence_after();
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
                             (static_cast<int64_t>(key) * p.batch + b) * (3 * hl_d) + hh * D;
       const bool st_ok = key < p.seq;
@@ -459,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
     const int q = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
     const float* lse = p.lse[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
-    const float* dv = p.dvec[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
+    const float* dv = p.dvec[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq_pad;
     const float lse2 = q < p.seq ? lse[q] * kLog2e : 0.f;
     const float Dq = q < p.seq ? dv[q] : 0.f;
     bool ok = true;
@@ -496,23 +758,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
 
 // STK / STQ: stages of the streamed Q, dO blocks (dK/dV kernel) and K, V
 // blocks (dQ kernel); as many as fit the 227 KB of shared memory.
-template <int D, int STK, int STQ>
+template <int D, int STK, int STS, int STQ>
 tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
-  static_assert(DkdvSmem<D, STK>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448,
+  static_assert(DkdvSmem<D, STK>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448 &&
+                    DkdvStSmem<D, STS>::TOTAL <= 232448,
                 "shared memory of the backward kernels");
-  static bool attr = false;
-  if (!attr) {
+  constexpr int kMaxDev = 64;
+  static bool attr[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return tpi::fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  if (!attr[dev]) {
     tp_status s = tpi::cuda_status(
         cudaFuncSetAttribute(attn_bwd_dkdv<D, STK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DkdvSmem<D, STK>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
     if (s != TP_OK) return s;
+    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dkdv_st<D, STS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              DkdvStSmem<D, STS>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
+    if (s != TP_OK) return s;
     s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq<D, STQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               DqSmem<D, STQ>::TOTAL), "cudaFuncSetAttribute(attention dq)");
     if (s != TP_OK) return s;
-    attr = true;
+    attr[dev] = true;
   }
   const int per = prm.p * prm.batch * prm.hl;
-  attn_bwd_dkdv<D, STK><<<prm.nkv * per, kThreads, DkdvSmem<D, STK>::TOTAL, st>>>(prm);
+  const char* e = getenv("TP_ATTN_BWD_DKDV");
+  if (e && e[0] == '1') {
+    attn_bwd_dkdv<D, STK><<<prm.nkv * per, kThreads, DkdvSmem<D, STK>::TOTAL, st>>>(prm);
+  } else {
+    attn_bwd_dkdv_st<D, STS><<<prm.nkv * per, kThreads, DkdvStSmem<D, STS>::TOTAL, st>>>(prm);
+  }
   tp_status s = tpi::after_launch("attention_bwd dK/dV (tcgen05)");
   if (s != TP_OK) return s;
   attn_bwd_dq<D, STQ><<<prm.nq * per, kThreads, DqSmem<D, STQ>::TOTAL, st>>>(prm);
@@ -528,17 +805,22 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
                                const MutPtrArray& dqkv, cudaStream_t st) {
   const int p = plan->p, d = plan->head_dim, hl = plan->heads / plan->p;
   const int64_t rows_per_shard = static_cast<int64_t>(batch) * hl * seq;
+  const int seq_pad = (seq + 63) / 64 * 64;
+  const int64_t padded_per_shard = static_cast<int64_t>(batch) * hl * seq_pad;
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(rows_per_shard * p) * sizeof(float), &ws);
+  tp_status s = workspace(plan, static_cast<size_t>(2 * padded_per_shard * p) * sizeof(float), &ws);
   if (s != TP_OK) return s;
   static BwdParams prm;
   static std::mutex mu;
   std::lock_guard<std::mutex> lk(mu);
   memset(&prm, 0, sizeof(prm));
-  MutPtrArray dvec{};
+  MutPtrArray dvec{}, lse2{};
+  PtrArray lse_in{};
   const int64_t C = 3LL * hl * d;
   for (int i = 0; i < p; ++i) {
-    dvec.p[i] = static_cast<float*>(ws) + i * rows_per_shard;
+    dvec.p[i] = static_cast<float*>(ws) + i * padded_per_shard;
+    lse2.p[i] = static_cast<float*>(ws) + (p + i) * padded_per_shard;
+    lse_in.p[i] = lse[i];
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(batch), static_cast<cuuint64_t>(seq)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * batch};
     cuuint32_t box[3] = {64, 1, 128};
@@ -548,6 +830,12 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
     cuuint64_t strides2[2] = {static_cast<cuuint64_t>(hl) * d * 2, static_cast<cuuint64_t>(hl) * d * 2 * batch};
     s = encode_bf16(&prm.tm_do[i], dO.p[i], 3, dims2, strides2, box, "dO");
     if (s != TP_OK) return s;
+    cuuint32_t box64[3] = {64, 1, 64};
+    s = encode_bf16(&prm.tm_q64[i], qkv.p[i], 3, dims, strides, box64, "QKV (bwd, 64 rows)");
+    if (s != TP_OK) return s;
+    s = encode_bf16(&prm.tm_do64[i], dO.p[i], 3, dims2, strides2, box64, "dO (64 rows)");
+    if (s != TP_OK) return s;
+    prm.lse2[i] = static_cast<const float*>(lse2.p[i]);
     prm.dqkv[i] = dqkv.p[i];
     prm.lse[i] = lse[i];
     prm.dvec[i] = static_cast<const float*>(dvec.p[i]);
@@ -558,6 +846,7 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   prm.hl = hl;
   prm.nq = (seq + BQ - 1) / BQ;
   prm.nkv = (seq + BKV - 1) / BKV;
+  prm.seq_pad = seq_pad;
   prm.scale = 1.f / sqrtf(static_cast<float>(d));
   prm.scale_log2 = kLog2e * prm.scale;
   s = device_status_word(&prm.status);
@@ -565,11 +854,12 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   const int64_t warps = rows_per_shard * p;
   if (warps * 32 / 256 + 1 > 0x7fffffffLL || static_cast<int64_t>(prm.nq) * p * batch * hl > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "attention backward grid too large");
-  attn_bwd_prep<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dO, dvec, p, batch, seq, hl, d);
+  attn_bwd_prep<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dO, lse_in, dvec, lse2, p,
+                                                                                 batch, seq, seq_pad, hl, d);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;
-  if (d == 64) return launch_bwd_d<64, 2, 2>(prm, st);
-  if (d == 128) return launch_bwd_d<128, 1, 2>(prm, st);
+  if (d == 64) return launch_bwd_d<64, 2, 4, 2>(prm, st);
+  if (d == 128) return launch_bwd_d<128, 1, 3, 2>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
 }
 
