@@ -243,19 +243,20 @@ __global__ void __launch_bounds__(256) ln_bwd_param_pass1(const T* x, const T* d
   }
 }
 
-// Sums of the per-CTA partials part[k][0|1][c] over k for kPass2Cols columns
-// c0 + lane: warp w takes k = w, w + 8, ... in increasing order, then the
-// eight warps' sums are added in warp order (fixed order: deterministic).
-// Lane 0..31 of warp 0 returns true with the column's two sums.
+// Sums of the per-CTA partials part[k][0|1][c] over k in [k0, k1) for
+// kPass2Cols columns c0 + lane: warp w takes k = k0 + w, k0 + w + 8, ... in
+// increasing order, then the eight warps' sums are added in warp order (fixed
+// order: deterministic). Lane 0..31 of warp 0 returns true with the column's
+// two sums.
 constexpr int kPass2Cols = 32;
-__device__ __forceinline__ bool param_colsum(const float* part, int splits, int64_t cols, int64_t c,
-                                             float* sg_out, float* sb_out) {
+__device__ __forceinline__ bool param_colsum_range(const float* part, int k0, int k1, int64_t cols,
+                                                   int64_t c, float* sg_out, float* sb_out) {
   __shared__ float rg[8][32], rb[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float sg = 0.f, sb = 0.f;
   if (c < cols) {
 #pragma unroll 4
-    for (int k = warp; k < splits; k += 8) {
+    for (int k = k0 + warp; k < k1; k += 8) {
       sg += part[(static_cast<int64_t>(k) * 2 + 0) * cols + c];
       sb += part[(static_cast<int64_t>(k) * 2 + 1) * cols + c];
     }
@@ -274,6 +275,25 @@ __device__ __forceinline__ bool param_colsum(const float* part, int splits, int6
   *sg_out = sg;
   *sb_out = sb;
   return true;
+}
+__device__ __forceinline__ bool param_colsum(const float* part, int splits, int64_t cols, int64_t c,
+                                             float* sg_out, float* sb_out) {
+  return param_colsum_range(part, 0, splits, cols, c, sg_out, sb_out);
+}
+
+// Many partials (one per CTA of a wide persistent grid): first sum them in
+// groups of kParamGroup consecutive k, each group by its own CTAs in the fixed
+// order above, into inter[g][0|1][c]; pass 2 then sums the groups in order.
+constexpr int kParamGroup = 64;
+__global__ void __launch_bounds__(256) param_group_sum(const float* part, int splits, int64_t cols,
+                                                       float* inter) {
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
+  const int g = static_cast<int>(blockIdx.y);
+  const int k1 = min(splits, (g + 1) * kParamGroup);
+  float sg, sb;
+  if (!param_colsum_range(part, g * kParamGroup, k1, cols, c, &sg, &sb)) return;
+  inter[(static_cast<int64_t>(g) * 2 + 0) * cols + c] = sg;
+  inter[(static_cast<int64_t>(g) * 2 + 1) * cols + c] = sb;
 }
 
 // 256 threads per CTA, kPass2Cols columns per CTA.
@@ -794,10 +814,12 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   }
 #undef TP_NH_GRID
   if (s != TP_OK) return s;
+  const int groups = grid > 2 * kParamGroup ? static_cast<int>((grid + kParamGroup - 1) / kParamGroup) : 0;
   void* ws = nullptr;
-  s = workspace(plan, static_cast<size_t>(grid) * 2 * h * sizeof(float), &ws);
+  s = workspace(plan, static_cast<size_t>(grid + groups) * 2 * h * sizeof(float), &ws);
   if (s != TP_OK) return s;
   float* part = static_cast<float*>(ws);
+  float* inter = part + grid * 2 * h;
   if (rows > 0) {
 #define TP_NH_BWD(T, TH, VP, R)                                                               \
   norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R><<<static_cast<unsigned>(grid), TH,   \
@@ -814,8 +836,17 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
     s = after_launch("norm_sharded_bwd");
     if (s != TP_OK) return s;
   }
-  norm_hsh_param_pass2<<<static_cast<unsigned>((h + kPass2Cols - 1) / kPass2Cols), 256, 0, st>>>(
-      part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg, db, accumulate);
+  const unsigned cblocks = static_cast<unsigned>((h + kPass2Cols - 1) / kPass2Cols);
+  if (rows > 0 && groups > 0) {
+    param_group_sum<<<dim3(cblocks, static_cast<unsigned>(groups)), 256, 0, st>>>(
+        part, static_cast<int>(grid), h, inter);
+    s = after_launch("norm_sharded_bwd/param groups");
+    if (s != TP_OK) return s;
+    norm_hsh_param_pass2<<<cblocks, 256, 0, st>>>(inter, groups, hs, h, dg, db, accumulate);
+  } else {
+    norm_hsh_param_pass2<<<cblocks, 256, 0, st>>>(part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg,
+                                                  db, accumulate);
+  }
   return after_launch("norm_sharded_bwd/param");
 }
 

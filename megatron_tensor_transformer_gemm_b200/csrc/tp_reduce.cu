@@ -330,6 +330,7 @@ __global__ void colsum_pass2(const float* part, int splits, int64_t cols, float*
   const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   float s = 0.f;
+#pragma unroll 8
   for (int k = 0; k < splits; ++k) s += part[static_cast<int64_t>(k) * cols + c];
   out[c] = accumulate ? out[c] + s : s;
 }
@@ -379,6 +380,7 @@ __global__ void colsum_grouped_pass2(const float* part, int splits, int64_t cols
   if (c >= cols) return;
   const float* pz = part + static_cast<int64_t>(blockIdx.y) * splits * cols;
   float sum = 0.f;
+#pragma unroll 8
   for (int k = 0; k < splits; ++k) sum += pz[static_cast<int64_t>(k) * cols + c];
   float* o = static_cast<float*>(out.p[blockIdx.y]);
   o[c] = accumulate ? o[c] + sum : sum;
