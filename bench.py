@@ -541,6 +541,11 @@ def time_sp_collectives(peaks, stream, rank):
         ("ln_all_gather", "ln_fwd_kernel (S1 LayerNorm fused with the sequence all-gather)",
          lambda: plan.layernorm_all_gather_seq(T, xs, gam, bet, full, mean, rstd), 2 * T * h * 2 + T * 8),
     ]
+    # reference only (not on the path): a plain device copy of the same bytes,
+    # the ceiling an all-gather of this size meets
+    src_full = torch.randn(T, h, generator=g).to(bf).to(dev)
+    cases.append(("copy_reference", "torch copy_ of [8192, 8192] bf16 (reference, not on the path)",
+                  lambda: full.copy_(src_full), 2 * T * h * 2))
     res = {}
     reps = 10
     for key, kname, fn, nbytes in cases:
@@ -564,7 +569,7 @@ def time_sp_collectives(peaks, stream, rank):
                     "bytes_per_launch": nbytes, "frac": gbs / peaks["hbm_gbs"],
                     "frac_of_8TBs": gbs / 8000.0}
         del graph
-    del parts, outs, full, xs
+    del parts, outs, full, xs, src_full
     torch.cuda.empty_cache()
     return res
 

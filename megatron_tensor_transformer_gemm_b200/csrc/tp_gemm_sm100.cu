@@ -14,7 +14,8 @@
 // problems whose 256 x 256 tiles would leave SMs idle, the host may instead
 // run 128-column tiles, one CTA per 128-row tile, or both (choose_layout).
 //
-// Design (per CTA, one CTA per SM, persistent over a static tile schedule):
+// Design (per CTA, one CTA per SM, persistent; tiles drawn in order from an
+// atomic counter, see the tile ring below):
 //   warp 0      TMA producer: 128B-swizzled A and B tiles into a 4-stage ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..9  epilogue: tcgen05.ld TMEM -> registers -> fused math -> HBM;
@@ -50,7 +51,7 @@ constexpr int UMMA_K = 16;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int TMEM_COLS = 512;
-constexpr int kBarBytes = 256;
+constexpr int kBarBytes = 512;  // barriers, TMEM slot, abort flag, tile ring
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64-wide MN block of an MN-major tile
 
 // Per-CTA tile geometry. PAIR = 1: one CTA computes a 128 x 256 tile.
@@ -113,6 +114,10 @@ struct alignas(64) GemmParams {
   int base_tiles;
   int kb_per_split;
   int64_t split_stride;
+  // Dynamic tile schedule: {next tile, CTAs finished}, zero at launch; the
+  // leader CTA of each pair takes tiles with atomicAdd, the last CTA to finish
+  // sets both back to zero.
+  unsigned* sched;
   unsigned* status;
 };
 
@@ -299,6 +304,67 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
   }
 }
 
+// ------------------------------------------------------------ tile ring
+// The persistent CTAs take tiles in order from one atomic counter, so the
+// tiles in flight at any moment are a window of consecutive indices (the
+// operands they share stay in L2) and a CTA that drew narrow or short tiles
+// simply takes more: no pair waits at the end for one whose static share
+// held more work. The leader CTA's producer draws each tile and publishes it
+// through a ring of kRing slots in both CTAs of the pair; every consumer (the
+// MMA issuer, the epilogue warps, the peer's producer) reads each entry once
+// and arrives on the leader's `empty` barrier of that slot. -1 ends the list.
+constexpr int kRing = 8;
+struct TileRing {
+  volatile int* slot;
+  uint64_t* full;
+  uint64_t* empty;
+};
+// Consumers of each entry: per CTA of the pair, the MMA issuer (leader) or
+// the producer (peer), plus the epilogue warps.
+constexpr int kRingConsumers = 1 + kEpiWarps;
+
+template <int PAIR>
+__device__ __forceinline__ bool ring_put(const TileRing& r, int k, int v, volatile int* abort,
+                                         unsigned* status) {
+  const int s = k % kRing;
+  const uint32_t par = static_cast<uint32_t>(k / kRing) & 1u;
+  if (!mbar_wait_cl(&r.empty[s], par ^ 1u, abort, status)) return false;
+  r.slot[s] = v;
+  if (PAIR == 2) {
+    st_shared_cluster_u32(map_shared(smem_u32(const_cast<int*>(&r.slot[s])), 1), static_cast<uint32_t>(v));
+    mbar_arrive_cluster(map_shared(smem_u32(&r.full[s]), 1));
+  }
+  mbar_arrive_release_cluster(&r.full[s]);
+  return true;
+}
+// One consumer thread: entry k (-2 when the wait gave up).
+template <int PAIR>
+__device__ __forceinline__ int ring_take(const TileRing& r, int k, uint32_t rank, volatile int* abort,
+                                         unsigned* status) {
+  const int s = k % kRing;
+  const uint32_t par = static_cast<uint32_t>(k / kRing) & 1u;
+  if (!mbar_wait_cl(&r.full[s], par, abort, status)) return -2;
+  const int v = r.slot[s];
+  if (PAIR == 2 && rank != 0) mbar_arrive_cluster(map_shared(smem_u32(&r.empty[s]), 0));
+  else mbar_arrive_release_cluster(&r.empty[s]);
+  return v;
+}
+// A whole warp: every lane reads entry k, lane 0 arrives once for the warp.
+template <int PAIR>
+__device__ __forceinline__ int ring_take_warp(const TileRing& r, int k, uint32_t rank, int lane,
+                                              volatile int* abort, unsigned* status) {
+  const int s = k % kRing;
+  const uint32_t par = static_cast<uint32_t>(k / kRing) & 1u;
+  if (!__all_sync(0xffffffffu, mbar_wait_cl(&r.full[s], par, abort, status))) return -2;
+  const int v = r.slot[s];
+  __syncwarp();
+  if (lane == 0) {
+    if (PAIR == 2 && rank != 0) mbar_arrive_cluster(map_shared(smem_u32(&r.empty[s]), 0));
+    else mbar_arrive_release_cluster(&r.empty[s]);
+  }
+  return v;
+}
+
 // -------------------------------------------------------------------- kernel
 template <int PAIR>
 __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -316,12 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  TileRing ring;
+  ring.full = drain + 2;
+  ring.empty = ring.full + kRing;
+  ring.slot = reinterpret_cast<volatile int*>(ring.empty + kRing);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;  // 0 = MMA leader of the pair
-  const int first_tile = static_cast<int>(blockIdx.x) / PAIR;
-  const int tile_stride = static_cast<int>(gridDim.x) / PAIR;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -333,6 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       mbar_init(&tempty[a], PAIR * kEpiWarps);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&ring.full[r], 1);
+      mbar_init(&ring.empty[r], PAIR * kRingConsumers);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -366,7 +438,19 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
 #pragma unroll
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
     bool ok = true;
-    for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
+    int kseq = 0;
+    int next = rank == 0 ? static_cast<int>(atomicAdd(p.sched, 1u)) : 0;
+    for (;;) {
+      int t;
+      if (rank == 0) {  // draw the next tile and publish it (or the end)
+        t = next;
+        if (t < p.total_tiles) next = static_cast<int>(atomicAdd(p.sched, 1u));
+        if (!ring_put<PAIR>(ring, kseq, t < p.total_tiles ? t : -1, abort_flag, p.status)) break;
+      } else {
+        t = ring_take<PAIR>(ring, kseq, rank, abort_flag, p.status);
+      }
+      ++kseq;
+      if (t < 0 || t >= p.total_tiles) break;
       int g, mt, nt, ks;
       decode_tile(p, t, g, mt, nt, ks);
       const GroupArgs& ga = p.g[g];
@@ -439,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
           }
         }
       }
+      if (!ok) break;
     }
     // Drain: every copy of this CTA (and, for the leader, of the pair) has
     // landed before the CTA exits. The peer's copies complete on the leader's
@@ -456,7 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = first_tile; t < p.total_tiles && ok; t += tile_stride) {
+    for (int kseq = 0;; ++kseq) {
+      const int t = ring_take<PAIR>(ring, kseq, rank, abort_flag, p.status);
+      if (t < 0) break;
       int g, mt, nt, ks;
       decode_tile(p, t, g, mt, nt, ks);
       const uint32_t idesc =
@@ -515,7 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     int acc = 0;
     uint32_t acc_phase = 0;
     const uint32_t tempty_leader = PAIR == 2 ? map_shared(smem_u32(&tempty[0]), 0) : 0u;
-    for (int t = first_tile; t < p.total_tiles; t += tile_stride) {
+    for (int kseq = 0;; ++kseq) {
+      const int t = ring_take_warp<PAIR>(ring, kseq, rank, lane, abort_flag, p.status);
+      if (t < 0) break;
       int g, mt, nt, ks;
       decode_tile(p, t, g, mt, nt, ks);
       const GroupArgs& ga = p.g[g];
@@ -541,6 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   if (PAIR == 2) cluster_sync_all();  // neither CTA leaves while its pair may still signal it
+  if (threadIdx.x == 0) {
+    // every draw of this CTA is done: the last CTA to get here re-arms the counter
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
@@ -693,6 +790,46 @@ tp_status launch_kernel(const GemmParams& p, int tiles, int sms, cudaStream_t st
   return tpi::after_launch(PAIR == 2 ? "gemm_bf16 (tcgen05, CTA pair)" : "gemm_bf16 (tcgen05)");
 }
 
+// Dynamic-schedule counters: two words per launch, zero at rest (each launch
+// sets its pair back to zero as it ends). Eager launches take slots
+// [0, kEagerSlots) in turn; launches recorded into a CUDA graph take slots
+// from [kEagerSlots, kSchedSlots), so a replayed graph never shares a counter
+// with an eager launch. Two launches running at the same time must not share
+// a slot: eager launches are kEagerSlots launches apart before one repeats,
+// and a captured graph must not run concurrently with another replay of
+// itself.
+constexpr int kSchedSlots = 4096, kEagerSlots = 1024;
+__device__ unsigned g_sched[2 * kSchedSlots];
+
+tp_status sched_slot(cudaStream_t st, unsigned** out) {
+  constexpr int kMaxDev = 64;
+  static unsigned* base[kMaxDev] = {};
+  static unsigned next_eager[kMaxDev] = {}, next_graph[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return tpi::fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  if (!base[dev]) {
+    void* ptr = nullptr;
+    tp_status s = tpi::cuda_status(cudaGetSymbolAddress(&ptr, g_sched), "cudaGetSymbolAddress(scheduler)");
+    if (s != TP_OK) return s;
+    base[dev] = static_cast<unsigned*>(ptr);
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    cs = cudaStreamCaptureStatusNone;
+  }
+  unsigned slot;
+  if (cs == cudaStreamCaptureStatusActive)
+    slot = kEagerSlots + next_graph[dev]++ % (kSchedSlots - kEagerSlots);
+  else
+    slot = next_eager[dev]++ % kEagerSlots;
+  *out = base[dev] + 2 * slot;
+  return TP_OK;
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -811,6 +948,8 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   p.epi = b.epi;
   p.out_f32 = b.out_f32;
   s = device_status_word(&p.status);
+  if (s != TP_OK) return s;
+  s = sched_slot(st, &p.sched);
   if (s != TP_OK) return s;
   if (pair == 2) return launch_kernel<2>(p, tiles, sms, st);
   return launch_kernel<1>(p, tiles, sms, st);

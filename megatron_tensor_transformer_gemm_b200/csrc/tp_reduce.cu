@@ -8,7 +8,6 @@
 // vector and the output pointer arithmetic are computed once per thread and
 // every warp touches 512 contiguous bytes per row: coalesced 128-bit traffic.
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -192,76 +191,6 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
     const int64_t lr = r - static_cast<int64_t>(j) * rows_per_src;
     const uint4 v = ld_stream(static_cast<const uint4*>(src.p[j]) + lr * vpr + cv);
     D[r * vpr + cv] = v;
-  }
-}
-
-// The sequence all-gather as n contiguous copies (shard j's bytes land at
-// dst + j * shard_bytes): persistent CTAs, one issuing thread each, move
-// kGatherChunk-byte chunks by bulk copy global -> shared -> global with
-// kGatherStages loads in flight per CTA, so each SM keeps
-// kGatherStages * kGatherChunk bytes of reads outstanding and the stores leave
-// as whole-chunk bulk writes. Chunk c of the CTA's stride covers bytes
-// [o, o + 32 KB) of shard c / chunks_per_shard. Every wait is bounded.
-constexpr int kGatherChunk = 32768;
-constexpr int kGatherStages = 6;
-
-__global__ void __launch_bounds__(32, 1) gather_bulk_kernel(const __grid_constant__ PtrArray src,
-                                                            int n, char* dst, int64_t shard_bytes,
-                                                            int64_t chunks_per_shard, unsigned* status) {
-  extern __shared__ __align__(128) uint8_t gsm[];
-  __shared__ uint64_t bars[kGatherStages];
-  __shared__ int abort_flag;
-  if (threadIdx.x != 0) return;
-  for (int st = 0; st < kGatherStages; ++st) tpd::mbar_init(&bars[st], 1);
-  abort_flag = 0;
-  tpd::fence_barrier_init();
-  const int64_t total = static_cast<int64_t>(n) * chunks_per_shard;
-  const int64_t c0 = blockIdx.x, stride = gridDim.x;
-  const int64_t mine = c0 < total ? (total - 1 - c0) / stride + 1 : 0;
-  auto chunk = [&](int64_t k, const char*& from, char*& to, uint32_t& bytes) {
-    const int64_t c = c0 + k * stride;
-    const int j = static_cast<int>(c / chunks_per_shard);
-    const int64_t o = (c - static_cast<int64_t>(j) * chunks_per_shard) * kGatherChunk;
-    const int64_t left = shard_bytes - o;
-    bytes = static_cast<uint32_t>(left < kGatherChunk ? left : kGatherChunk);
-    from = static_cast<const char*>(src.p[j]) + o;
-    to = dst + static_cast<int64_t>(j) * shard_bytes + o;
-  };
-  auto load = [&](int64_t k) {
-    const char* from;
-    char* to;
-    uint32_t bytes;
-    chunk(k, from, to, bytes);
-    const int st = static_cast<int>(k % kGatherStages);
-    tpd::mbar_arrive_expect_tx(&bars[st], bytes);
-    tpd::bulk_load(gsm + st * kGatherChunk, from, bytes, &bars[st]);
-  };
-  int64_t issued = 0;
-  for (; issued < mine && issued < kGatherStages; ++issued) load(issued);
-  int64_t k = 0;
-  for (; k < mine; ++k) {
-    const int st = static_cast<int>(k % kGatherStages);
-    if (!tpd::mbar_wait(&bars[st], static_cast<uint32_t>(k / kGatherStages) & 1u, &abort_flag, status))
-      break;
-    const char* from;
-    char* to;
-    uint32_t bytes;
-    chunk(k, from, to, bytes);
-    tpd::bulk_store(to, gsm + st * kGatherChunk, bytes);
-    tpd::bulk_commit();
-    if (issued < mine) {
-      tpd::bulk_wait_read<0>();  // this stage's store has read it
-      load(issued++);
-    }
-  }
-  tpd::bulk_wait_all();
-  // After a time-out, give the loads still in flight one more bounded wait so
-  // none lands in shared memory after the CTA has gone.
-  if (k < mine) {
-    int flag = 0;
-    for (int64_t q = k; q < issued; ++q)
-      tpd::mbar_wait(&bars[q % kGatherStages], static_cast<uint32_t>(q / kGatherStages) & 1u, &flag,
-                     nullptr);
   }
 }
 
@@ -467,23 +396,6 @@ tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* 
 tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
                         tp_dtype dt, cudaStream_t st) {
   const int64_t vpr = cols * static_cast<int64_t>(dsize(dt)) / 16;
-  const int64_t shard_bytes = (T / n) * vpr * 16;
-  const char* e = getenv("TP_GATHER");
-  const bool bulk = !(e && e[0] == 'v') && shard_bytes >= (1 << 20);
-  if (bulk) {
-    constexpr int smem = kGatherStages * kGatherChunk;
-    const int64_t cps = (shard_bytes + kGatherChunk - 1) / kGatherChunk;
-    int64_t grid = 0;
-    tp_status s = persistent_grid(reinterpret_cast<const void*>(gather_bulk_kernel), 32, smem,
-                                  cps * n, &grid);
-    if (s != TP_OK) return s;
-    unsigned* status = nullptr;
-    s = device_status_word(&status);
-    if (s != TP_OK) return s;
-    gather_bulk_kernel<<<static_cast<unsigned>(grid), 32, smem, st>>>(src, n, static_cast<char*>(dst),
-                                                                     shard_bytes, cps, status);
-    return after_launch("all_gather_seq (bulk)");
-  }
   dim3 grid, block;
   row_walk_shape(vpr, T, &grid, &block);
   gather_kernel<<<grid, block, 0, st>>>(src, dst, T, vpr, T / n);

@@ -329,10 +329,9 @@ def test_bounded_wait_times_out_and_reports():
 
 
 @pytest.mark.parametrize("n,t,h", [(8, 600, 1032), (3, 1000, 4096), (2, 64, 8192)])
-def test_all_gather_bulk_copy_bitexact(n, t, h):
-    """The sequence all-gather of shards of 1 MB and more runs as bulk copies of
-    32 KB chunks through shared memory; shard sizes that end in a partial chunk
-    (600 rows x 2064 bytes) and shards of exactly 1 MB are copied bit for bit."""
+def test_all_gather_large_shards_bitexact(n, t, h):
+    """The sequence all-gather of shards of 1 MB and more (600 rows x 2064
+    bytes, 1000 x 8192 bytes, exactly 1 MB) is copied bit for bit."""
     tp = _tp()
     g = torch.Generator().manual_seed(n * t + h)
     xs = [torch.randn(t, h, generator=g).to(torch.bfloat16) for _ in range(n)]
