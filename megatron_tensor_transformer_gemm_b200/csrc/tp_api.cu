@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -32,6 +33,7 @@ namespace tp_selftest {
 // on an mbarrier that expects one arrival which never comes: the wait gives
 // up after limit_ns, sets the status word and the kernel returns.
 __global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns, int* gave_up) {
+  tpd::pdl_entry();
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x != 0) return;
@@ -56,6 +58,14 @@ tp_status fail(tp_status s, const char* fmt, ...) {
 tp_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return TP_OK;
   return fail(TP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TP_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 tp_status after_launch(const char* what, int launches) {
@@ -426,7 +436,7 @@ tp_status tp_selftest_wait_timeout(int64_t limit_ns, int* gave_up, void* stream)
     return fail(TP_ERR_ALIGN, "gave_up is not 4-byte aligned");
   unsigned* addr = nullptr;
   TP_TRY(device_status_word(&addr));
-  tp_selftest::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(addr, static_cast<uint64_t>(limit_ns), gave_up);
+  (void)tpi::launch(tp_selftest::selftest_wait_kernel, dim3(1), dim3(32), 0, as_stream(stream), addr, static_cast<uint64_t>(limit_ns), gave_up);
   return after_launch("selftest_wait_timeout");
 }
 

@@ -81,6 +81,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  tpd::pdl_entry();
   using SM = AttnSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -416,7 +417,7 @@ tp_status launch_fwd_d(AttnParams& prm, cudaStream_t st) {
     attr = true;
   }
   const int grid = prm.n_pairs * prm.p * prm.batch * prm.heads_local;
-  attn_fwd_kernel<D><<<grid, kThreads, smem, st>>>(prm);
+  (void)tpi::launch(attn_fwd_kernel<D>, dim3(grid), dim3(kThreads), smem, st, prm);
   return tpi::after_launch("attention_fwd (tcgen05)");
 }
 

@@ -96,6 +96,7 @@ __global__ void attn_bwd_prep(const __grid_constant__ PtrArray O, const __grid_c
                               const __grid_constant__ PtrArray LSE, const __grid_constant__ MutPtrArray dvec,
                               const __grid_constant__ MutPtrArray lse2, int p, int batch, int seq,
                               int seq_pad, int hl, int d) {
+  tpd::pdl_entry();
   const int64_t rows_per_shard = static_cast<int64_t>(batch) * hl * seq;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x & 31;
@@ -160,6 +161,7 @@ struct DkdvSmem {
 
 template <int D, int ST>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_constant__ BwdParams p) {
+  tpd::pdl_entry();
   using SM = DkdvSmem<D, ST>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -353,6 +355,7 @@ struct DkdvStSmem {
 
 template <int D, int ST>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_constant__ BwdParams p) {
+  tpd::pdl_entry();
   using SM = DkdvStSmem<D, ST>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -590,6 +593,7 @@ struct DqSmem {
 
 template <int D, int ST>
 __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant__ BwdParams p) {
+  tpd::pdl_entry();
   using SM = DqSmem<D, ST>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -786,13 +790,13 @@ tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
   const int per = prm.p * prm.batch * prm.hl;
   const char* e = getenv("TP_ATTN_BWD_DKDV");
   if (e && e[0] == '1') {
-    attn_bwd_dkdv<D, STK><<<prm.nkv * per, kThreads, DkdvSmem<D, STK>::TOTAL, st>>>(prm);
+    (void)tpi::launch(attn_bwd_dkdv<D, STK>, dim3(prm.nkv * per), dim3(kThreads), DkdvSmem<D, STK>::TOTAL, st, prm);
   } else {
-    attn_bwd_dkdv_st<D, STS><<<prm.nkv * per, kThreads, DkdvStSmem<D, STS>::TOTAL, st>>>(prm);
+    (void)tpi::launch(attn_bwd_dkdv_st<D, STS>, dim3(prm.nkv * per), dim3(kThreads), DkdvStSmem<D, STS>::TOTAL, st, prm);
   }
   tp_status s = tpi::after_launch("attention_bwd dK/dV (tcgen05)");
   if (s != TP_OK) return s;
-  attn_bwd_dq<D, STQ><<<prm.nq * per, kThreads, DqSmem<D, STQ>::TOTAL, st>>>(prm);
+  (void)tpi::launch(attn_bwd_dq<D, STQ>, dim3(prm.nq * per), dim3(kThreads), DqSmem<D, STQ>::TOTAL, st, prm);
   return tpi::after_launch("attention_bwd dQ (tcgen05)");
 }
 
@@ -854,7 +858,7 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   const int64_t warps = rows_per_shard * p;
   if (warps * 32 / 256 + 1 > 0x7fffffffLL || static_cast<int64_t>(prm.nq) * p * batch * hl > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "attention backward grid too large");
-  attn_bwd_prep<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(o, dO, lse_in, dvec, lse2, p,
+  (void)tpi::launch(attn_bwd_prep, dim3(static_cast<unsigned>((warps * 32 + 255) / 256)), dim3(256), 0, st, o, dO, lse_in, dvec, lse2, p,
                                                                                  batch, seq, seq_pad, hl, d);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;

@@ -29,6 +29,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch, at the start of every kernel of the library
+// (before any global memory access): wait until the kernel before this one on
+// the stream has completed and its writes are visible, then let the next
+// kernel's launch begin (its CTAs take SMs as this grid's CTAs leave).
+__device__ __forceinline__ void pdl_entry() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -370,6 +379,10 @@ __device__ __forceinline__ float gelu_grad_f(float z) {
          z * 0.39894228040143268f * expf(-0.5f * z * z);
 }
 __device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + expf(-z)); }
+// The logistic sigmoid from the hardware exponential and an approximate
+// division, for epilogues whose results are rounded to bf16 (a few fp32 ulp
+// of error against the 2^-8 of the rounding); 1/(1+inf) gives 0.
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 __device__ __forceinline__ float silu_f(float z) { return z * sigmoid_f(z); }
 __device__ __forceinline__ float silu_grad_f(float z) {
   float s = sigmoid_f(z);

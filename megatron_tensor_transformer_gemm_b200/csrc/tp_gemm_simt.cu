@@ -65,6 +65,7 @@ __device__ __forceinline__ float load_b(const F32Group& g, int b_mn, int n, int 
 // 256 threads; each computes a 4x4 block of the 64x64 output tile (two
 // blocks, gate and up, for SwiGLU). blockIdx.z = group (shard).
 __global__ void __launch_bounds__(256) sgemm_kernel(const __grid_constant__ F32Params p) {
+  tpd::pdl_entry();
   __shared__ float As[TK][TM + 4];
   __shared__ float Bs[TK][TN + 4];
   __shared__ float Us[TK][TN + 4];
@@ -223,7 +224,7 @@ tp_status launch_gemm_f32(const GemmBatch& b, cudaStream_t st) {
     }
   }
   dim3 grid((nmax + TN - 1) / TN, (mmax + TM - 1) / TM, nout);
-  sgemm_kernel<<<grid, 256, 0, st>>>(p);
+  (void)tpi::launch(sgemm_kernel, dim3(grid), dim3(256), 0, st, p);
   return after_launch("gemm_f32");
 }
 

@@ -221,7 +221,7 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
         }
         float h[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
+        for (int i = 0; i < 32; ++i) h[i] = g[i] * sigmoid_fast(g[i]) * u[i];
         store_row_chunk_bf16(ga.D2, ga.ldd2, row, j0, ga.N, h);
       }
     }
@@ -291,8 +291,10 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
                             ga.N, zu);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          dg[i] = v[i] * zu[i] * silu_grad_f(zg[i]);
-          v[i] = v[i] * silu_f(zg[i]);
+          // one sigmoid per element: SiLU(g) = g s, SiLU'(g) = s (1 + g (1 - s))
+          const float sg = sigmoid_fast(zg[i]);
+          dg[i] = v[i] * zu[i] * (sg * (1.0f + zg[i] * (1.0f - sg)));
+          v[i] = v[i] * (zg[i] * sg);
         }
         store_row_chunk_bf16(ga.D, ga.ldd, row, j0, ga.N, dg);
         store_row_chunk_bf16(static_cast<__nv_bfloat16*>(ga.D) + ga.nh, ga.ldd, row, j0, ga.N, v);
@@ -429,6 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   if (PAIR == 2) cluster_sync_all();  // the peer's barriers are initialised before any signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only shared memory, TMEM and the kernel
+  // parameters, so it overlapped the previous kernel's tail.
+  pdl_entry();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------- producer
@@ -777,13 +782,15 @@ tp_status launch_kernel(const GemmParams& p, int tiles, int sms, cudaStream_t st
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = PAIR;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = tpi::pdl_enabled() ? 2 : 1;
   tp_status s = tpi::cuda_status(cudaLaunchKernelEx(&cfg, tp_gemm_kernel<PAIR>, p),
                                  "cudaLaunchKernelEx(gemm)");
   if (s != TP_OK) return s;

@@ -27,6 +27,31 @@ struct tp_plan {
 
 namespace tpi {
 
+// Programmatic dependent launch: every kernel of the library begins with
+// pdl_entry() (tp_device.cuh) before it touches global memory, so a launch
+// may start while the kernel before it on the stream finishes, and its
+// wait resolves when that kernel has completed and its writes are visible.
+// On unless the environment variable TP_PDL is "0".
+bool pdl_enabled();
+
+// Launch `kernel` on `st` with the programmatic-serialization attribute (when
+// enabled). Launch errors surface through cudaGetLastError as with <<<>>>.
+template <typename... Exp, typename... Act>
+inline cudaError_t launch(void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Act&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Act&&>(args)...);
+}
+
 // Record `fmt` as this thread's last error and return `s`.
 tp_status fail(tp_status s, const char* fmt, ...);
 // TP_OK if e == cudaSuccess, else TP_ERR_CUDA with the CUDA error text.

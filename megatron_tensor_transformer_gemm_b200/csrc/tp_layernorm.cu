@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__
                                                          int64_t cols, const T* gamma,
                                                          const T* beta, T* y, float* mean_out,
                                                          float* rstd_out) {
+  tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   constexpr int W = THREADS / 32;
   __shared__ float red1[W], red2[W];
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(THREADS) ln_bwd_dx_kernel(const T* x, const T*
                                                             const T* dy, const float* mean_in,
                                                             const float* rstd_in, T* dx,
                                                             int64_t cols) {
+  tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   __shared__ float red[THREADS / 32];
   const int64_t r = blockIdx.x;
@@ -199,6 +201,7 @@ __global__ void __launch_bounds__(256) ln_bwd_param_pass1(const T* x, const T* d
                                                           const float* rstd_in, int64_t rows,
                                                           int64_t cols, int64_t rps,
                                                           float* part) {
+  tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   __shared__ float red[2][8][32 * V + 1];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -287,6 +290,7 @@ __device__ __forceinline__ bool param_colsum(const float* part, int splits, int6
 constexpr int kParamGroup = 64;
 __global__ void __launch_bounds__(256) param_group_sum(const float* part, int splits, int64_t cols,
                                                        float* inter) {
+  tpd::pdl_entry();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
   const int g = static_cast<int>(blockIdx.y);
   const int k1 = min(splits, (g + 1) * kParamGroup);
@@ -299,6 +303,7 @@ __global__ void __launch_bounds__(256) param_group_sum(const float* part, int sp
 // 256 threads per CTA, kPass2Cols columns per CTA.
 __global__ void __launch_bounds__(256) ln_bwd_param_pass2(const float* part, int splits, int64_t cols,
                                                           float* dgamma, float* dbeta, int accumulate) {
+  tpd::pdl_entry();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
   float sg, sb;
   if (!param_colsum(part, splits, cols, c, &sg, &sb)) return;
@@ -336,7 +341,7 @@ tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_sr
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "LayerNorm row too long (%lld)", (long long)cols);
   const int th = threads_for(vpr);
 #define TP_LN_FWD(T, TH)                                                                        \
-  ln_fwd_kernel<T, TH><<<static_cast<unsigned>(rows), TH, 0, st>>>(                            \
+  (void)tpi::launch(ln_fwd_kernel<T, TH>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st,                             \
       x_seq, rows_per_src, cols, static_cast<const T*>(gamma), static_cast<const T*>(beta),     \
       static_cast<T*>(y), mean, rstd)
   if (dt == TP_BF16) {
@@ -387,7 +392,7 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
   if (rows > 0) {
     const int th = threads_for(vpr);
 #define TP_LN_BWD(T, TH)                                                                        \
-  ln_bwd_dx_kernel<T, TH><<<static_cast<unsigned>(rows), TH, 0, st>>>(                         \
+  (void)tpi::launch(ln_bwd_dx_kernel<T, TH>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st,                          \
       static_cast<const T*>(x), static_cast<const T*>(gamma), static_cast<const T*>(dy), mean,  \
       rstd, static_cast<T*>(dx), cols)
     if (dt == TP_BF16) {
@@ -404,17 +409,17 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
     if (s != TP_OK) return s;
     dim3 grid(gx, static_cast<unsigned>(splits));
     if (dt == TP_BF16)
-      ln_bwd_param_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(
+      (void)tpi::launch(ln_bwd_param_pass1<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, 
           static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy), mean, rstd,
           rows, cols, rps, part);
     else
-      ln_bwd_param_pass1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x),
+      (void)tpi::launch(ln_bwd_param_pass1<float>, dim3(grid), dim3(256), 0, st, static_cast<const float*>(x),
                                                       static_cast<const float*>(dy), mean, rstd,
                                                       rows, cols, rps, part);
     s = after_launch("layernorm_bwd/param1");
     if (s != TP_OK) return s;
   }
-  ln_bwd_param_pass2<<<static_cast<unsigned>((cols + kPass2Cols - 1) / kPass2Cols), 256, 0, st>>>(
+  (void)tpi::launch(ln_bwd_param_pass2, dim3(static_cast<unsigned>((cols + kPass2Cols - 1) / kPass2Cols)), dim3(256), 0, st, 
       part, static_cast<int>(splits), cols, dgamma, dbeta, accumulate);
   return after_launch("layernorm_bwd/param2");
 }
@@ -497,6 +502,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
     const __grid_constant__ PtrArray B, const __grid_constant__ MutPtrArray Y, int vps, int64_t h,
     float* mean_out, float* rstd_out) {
+  tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   constexpr int W = THREADS / 32;
   __shared__ float2 red[W];
@@ -586,6 +592,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int p, int vps,
     int64_t hs, int64_t h, int64_t rows, const float* mean_in, const float* rstd_in,
     float* part, unsigned* status) {
+  tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   extern __shared__ __align__(128) uint8_t sbuf[];
   __shared__ uint64_t bar[STAGES];
@@ -709,6 +716,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
 __global__ void __launch_bounds__(256) norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
                                                             const __grid_constant__ MutPtrArray dg,
                                                             const __grid_constant__ MutPtrArray db, int accumulate) {
+  tpd::pdl_entry();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
   float sg, sb;
   if (!param_colsum(part, splits, h, c, &sg, &sb)) return;
@@ -764,7 +772,7 @@ tp_status launch_norm_sharded_fwd(bool rms, const PtrArray& X, const PtrArray& G
   const int vps = static_cast<int>(hs / V);
   const int th = threads_for(vpr);
 #define TP_NH_FWD(T, TH, R)                                                                      \
-  norm_hsh_row_fwd_kernel<T, TH, R><<<static_cast<unsigned>(rows), TH, 0, st>>>(X, G, B, Y, vps, h, \
+  (void)tpi::launch(norm_hsh_row_fwd_kernel<T, TH, R>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st, X, G, B, Y, vps, h, \
                                                                                mean, rstd)
 #define TP_NH_FWD_TH(T, R)          \
   do {                              \
@@ -822,8 +830,8 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   float* inter = part + grid * 2 * h;
   if (rows > 0) {
 #define TP_NH_BWD(T, TH, VP, R)                                                               \
-  norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R><<<static_cast<unsigned>(grid), TH,   \
-                                                            smem, st>>>(                       \
+  (void)tpi::launch(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R>, dim3(static_cast<unsigned>(grid)), dim3(TH), \
+                                                            smem, st,                        \
       X, G, DY, DX, p, vps, hs, h, rows, mean, rstd, part, status)
     if (dt == TP_BF16) {
       if (rms) { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
@@ -838,13 +846,13 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   }
   const unsigned cblocks = static_cast<unsigned>((h + kPass2Cols - 1) / kPass2Cols);
   if (rows > 0 && groups > 0) {
-    param_group_sum<<<dim3(cblocks, static_cast<unsigned>(groups)), 256, 0, st>>>(
+    (void)tpi::launch(param_group_sum, dim3(dim3(cblocks, static_cast<unsigned>(groups))), dim3(256), 0, st, 
         part, static_cast<int>(grid), h, inter);
     s = after_launch("norm_sharded_bwd/param groups");
     if (s != TP_OK) return s;
-    norm_hsh_param_pass2<<<cblocks, 256, 0, st>>>(inter, groups, hs, h, dg, db, accumulate);
+    (void)tpi::launch(norm_hsh_param_pass2, dim3(cblocks), dim3(256), 0, st, inter, groups, hs, h, dg, db, accumulate);
   } else {
-    norm_hsh_param_pass2<<<cblocks, 256, 0, st>>>(part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg,
+    (void)tpi::launch(norm_hsh_param_pass2, dim3(cblocks), dim3(256), 0, st, part, rows > 0 ? static_cast<int>(grid) : 0, hs, h, dg,
                                                   db, accumulate);
   }
   return after_launch("norm_sharded_bwd/param");

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
                                                           const __grid_constant__ MutPtrArray out,
                                                           int scatter, int64_t rows, int64_t vpr,
                                                           int64_t rows_per_out) {
+  tpd::pdl_entry();
   constexpr int V = Vec<OT>::N;
   constexpr int W = V * static_cast<int>(sizeof(PT)) / 16;
   constexpr int VP = Vec<PT>::N;  // partial elements per 16-byte load
@@ -181,6 +182,7 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
 // X_full rows [j*rows_per_src, ...) = src.p[j] rows; 16-byte vectors.
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ PtrArray src, void* dst, int64_t rows,
                                                           int64_t vpr, int64_t rows_per_src) {
+  tpd::pdl_entry();
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (cv >= vpr) return;
   const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.y;
@@ -197,6 +199,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
 // Strided 2-D copy of 16-byte vectors.
 __global__ void copy2d_vec_kernel(const uint4* src, int64_t sld, uint4* dst, int64_t dld,
                                   int64_t rows, int64_t vpr) {
+  tpd::pdl_entry();
   const int64_t total = rows * vpr;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -209,6 +212,7 @@ __global__ void copy2d_vec_kernel(const uint4* src, int64_t sld, uint4* dst, int
 template <typename E>
 __global__ void copy2d_elem_kernel(const E* src, int64_t sld, E* dst, int64_t dld, int64_t rows,
                                    int64_t cols) {
+  tpd::pdl_entry();
   const int64_t total = rows * cols;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -224,6 +228,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) colsum_pass1(const T* x, int64_t ld, int64_t rows,
                                                     int64_t vpr, int64_t rows_per_split,
                                                     float* part, int64_t cols) {
+  tpd::pdl_entry();
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -256,6 +261,7 @@ __global__ void __launch_bounds__(256) colsum_pass1(const T* x, int64_t ld, int6
 // Column sums, pass 2: out[c] (+)= sum over splits in order.
 __global__ void colsum_pass2(const float* part, int splits, int64_t cols, float* out,
                              int accumulate) {
+  tpd::pdl_entry();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   float s = 0.f;
@@ -271,6 +277,7 @@ __global__ void __launch_bounds__(256) colsum_grouped_pass1(const __grid_constan
                                                             int64_t ld, int64_t rows, int64_t vpr,
                                                             int64_t rows_per_split, float* part,
                                                             int64_t cols) {
+  tpd::pdl_entry();
   constexpr int V = Vec<T>::N;
   __shared__ float red[8][32 * V + 1];
   const T* x = static_cast<const T*>(X.p[blockIdx.z]);
@@ -305,6 +312,7 @@ __global__ void __launch_bounds__(256) colsum_grouped_pass1(const __grid_constan
 // Pass 2 of the grouped sums: out.p[blockIdx.y][c] (+)= sum over splits in order.
 __global__ void colsum_grouped_pass2(const float* part, int splits, int64_t cols,
                                      const __grid_constant__ MutPtrArray out, int accumulate) {
+  tpd::pdl_entry();
   const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   const float* pz = part + static_cast<int64_t>(blockIdx.y) * splits * cols;
@@ -341,18 +349,18 @@ tp_status launch_copy_2d(const void* src, int64_t src_ld, void* dst, int64_t dst
     const int64_t vpr = cols * esize / 16;
     const int64_t total = rows * vpr;
     int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 16LL));
-    copy2d_vec_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(src),
+    (void)tpi::launch(copy2d_vec_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const uint4*>(src),
                                               src_ld * esize / 16, static_cast<uint4*>(dst),
                                               dst_ld * esize / 16, rows, vpr);
   } else {
     const int64_t total = rows * cols;
     int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sm_count() * 16LL));
     if (esize == 2)
-      copy2d_elem_kernel<uint16_t><<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(src),
+      (void)tpi::launch(copy2d_elem_kernel<uint16_t>, dim3(blocks), dim3(256), 0, st, static_cast<const uint16_t*>(src),
                                                            src_ld, static_cast<uint16_t*>(dst),
                                                            dst_ld, rows, cols);
     else if (esize == 4)
-      copy2d_elem_kernel<uint32_t><<<blocks, 256, 0, st>>>(static_cast<const uint32_t*>(src),
+      (void)tpi::launch(copy2d_elem_kernel<uint32_t>, dim3(blocks), dim3(256), 0, st, static_cast<const uint32_t*>(src),
                                                            src_ld, static_cast<uint32_t*>(dst),
                                                            dst_ld, rows, cols);
     else
@@ -374,7 +382,7 @@ tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* 
   const int scatter = out_is_seq ? 1 : 0;
   const int64_t T_rows = T;
 #define TP_REDUCE_LAUNCH(PT, OT, NM)                                                            \
-  reduce_kernel<PT, OT, NM><<<grid, block, 0, st>>>(P, n, static_cast<const OT*>(bias),          \
+  (void)tpi::launch(reduce_kernel<PT, OT, NM>, dim3(grid), dim3(block), 0, st, P, n, static_cast<const OT*>(bias),          \
                                                     static_cast<const OT*>(residual),            \
                                                     residual_seq, rs, out, scatter, T_rows, vpr, \
                                                     rows_per_out)
@@ -398,7 +406,7 @@ tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_
   const int64_t vpr = cols * static_cast<int64_t>(dsize(dt)) / 16;
   dim3 grid, block;
   row_walk_shape(vpr, T, &grid, &block);
-  gather_kernel<<<grid, block, 0, st>>>(src, dst, T, vpr, T / n);
+  (void)tpi::launch(gather_kernel, dim3(grid), dim3(block), 0, st, src, dst, T, vpr, T / n);
   return after_launch("all_gather_seq");
 }
 
@@ -419,17 +427,17 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
   if (rows > 0) {
     dim3 grid(gx, static_cast<unsigned>(splits));
     if (dt == TP_BF16)
-      colsum_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), ld,
+      (void)tpi::launch(colsum_pass1<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), ld,
                                                         rows, vpr, rps, part, cols);
     else
-      colsum_pass1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), ld, rows, vpr, rps,
+      (void)tpi::launch(colsum_pass1<float>, dim3(grid), dim3(256), 0, st, static_cast<const float*>(x), ld, rows, vpr, rps,
                                                 part, cols);
     s = after_launch("column_sum/pass1");
     if (s != TP_OK) return s;
   } else {
     splits = 0;
   }
-  colsum_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+  (void)tpi::launch(colsum_pass2, dim3(static_cast<unsigned>((cols + 255) / 256)), dim3(256), 0, st, 
       part, static_cast<int>(splits), cols, out, accumulate);
   return after_launch("column_sum/pass2");
 }
@@ -453,14 +461,13 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
   if (rows > 0) {
     dim3 grid(gx, static_cast<unsigned>(splits), static_cast<unsigned>(n));
     if (dt == TP_BF16)
-      colsum_grouped_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(x, ld, rows, vpr, rps, part, cols);
+      (void)tpi::launch(colsum_grouped_pass1<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, ld, rows, vpr, rps, part, cols);
     else
-      colsum_grouped_pass1<float><<<grid, 256, 0, st>>>(x, ld, rows, vpr, rps, part, cols);
+      (void)tpi::launch(colsum_grouped_pass1<float>, dim3(grid), dim3(256), 0, st, x, ld, rows, vpr, rps, part, cols);
     s = after_launch("column_sum_grouped/pass1");
     if (s != TP_OK) return s;
   }
-  colsum_grouped_pass2<<<dim3(static_cast<unsigned>((cols + 255) / 256), static_cast<unsigned>(n)), 256, 0,
-                         st>>>(part, static_cast<int>(splits), cols, out, accumulate);
+  (void)tpi::launch(colsum_grouped_pass2, dim3(dim3(static_cast<unsigned>((cols + 255) / 256), static_cast<unsigned>(n))), dim3(256), 0, st, part, static_cast<int>(splits), cols, out, accumulate);
   return after_launch("column_sum_grouped/pass2");
 }
 
@@ -543,15 +550,15 @@ extern "C" tp_status tp_column_sum_static(int64_t rows, int64_t cols, tp_dtype d
     // nothing left from an earlier call is ever read.
     dim3 grid(gx, static_cast<unsigned>(splits));
     if (dtype == TP_BF16)
-      colsum_pass1<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+      (void)tpi::launch(colsum_pass1<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
                                                         cols, rows, vpr, rps, part, cols);
     else
-      colsum_pass1<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), cols, rows, vpr,
+      (void)tpi::launch(colsum_pass1<float>, dim3(grid), dim3(256), 0, st, static_cast<const float*>(x), cols, rows, vpr,
                                                 rps, part, cols);
     s = after_launch("column_sum_static/pass1");
     if (s != TP_OK) return s;
   }
-  colsum_pass2<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(
+  (void)tpi::launch(colsum_pass2, dim3(static_cast<unsigned>((cols + 255) / 256)), dim3(256), 0, st, 
       part, static_cast<int>(splits), cols, out, accumulate);
   return after_launch("column_sum_static/pass2");
 }

@@ -30,6 +30,7 @@ constexpr unsigned kStatusBadIndex = 2u;
 __global__ void embed_fwd_kernel(const int32_t* ids, const __grid_constant__ PtrArray E, int vocab,
                                  int64_t Vs, int64_t T, int64_t vpr, uint4* Y,
                                  unsigned* status) {
+  tpd::pdl_entry();
   const int64_t total = T * vpr;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -70,6 +71,7 @@ __device__ __forceinline__ bool valid_id(int id, int vocab) { return id >= 0 && 
 __global__ void __launch_bounds__(kTokBlock) emb_bucket_count(const int32_t* ids, int64_t ntok,
                                                               int vocab, int nb, int nblk,
                                                               int* cnt) {
+  tpd::pdl_entry();
   __shared__ int hist[kEmbMaxBuckets];
   for (int i = threadIdx.x; i < nb; i += kTokBlock) hist[i] = 0;
   __syncthreads();
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kTokBlock) emb_bucket_count(const int32_t* ids
 // Thread b: bucket b's counts over the blocks become their exclusive prefix
 // (in place); tot[b] = the bucket's total.
 __global__ void __launch_bounds__(256) emb_bucket_prefix(int* cnt, int nb, int nblk, int* tot) {
+  tpd::pdl_entry();
   const int b = blockIdx.x * 256 + threadIdx.x;
   if (b >= nb) return;
   int run = 0;
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(256) emb_bucket_prefix(int* cnt, int nb, int n
 // owns the contiguous chunk [tid * C, (tid + 1) * C), C a multiple of 4, read
 // and written as 16-byte vectors (a is 16-byte aligned).
 __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
+  tpd::pdl_entry();
   __shared__ int wsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t C = ((n + 1023) / 1024 + 3) / 4 * 4;
@@ -157,6 +161,7 @@ __global__ void __launch_bounds__(1024) emb_scan(int* a, int64_t n) {
 __global__ void __launch_bounds__(kTokBlock) emb_bucket_scatter(const int32_t* ids, int64_t ntok,
                                                                 int vocab, int nb, const int* off,
                                                                 const int* tot, int2* sorted) {
+  tpd::pdl_entry();
   __shared__ int seen[kEmbMaxBuckets];
   for (int i = threadIdx.x; i < nb; i += kTokBlock) seen[i] = 0;
   __syncthreads();
@@ -269,6 +274,7 @@ template <typename T>
 __global__ void __launch_bounds__(kAccThreads, 2) emb_bucket_accum(
     const int2* sorted, const int* tot, const T* dY, int64_t h, int64_t Vs, int64_t Vp,
     const __grid_constant__ MutPtrArray dE) {
+  tpd::pdl_entry();
   constexpr int E = 16 / sizeof(T);
   __shared__ int ltok[kListChunk];
   __shared__ int lrow[kListChunk];
@@ -477,6 +483,7 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_kernel(
     const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
     int vocab, const int32_t* labels, float scale, float* loss, float* lse_out,
     unsigned* status) {
+  tpd::pdl_entry();
   constexpr int N = Vec<T>::N;
   constexpr float kLog2e = 1.4426950408889634f;
   __shared__ float red[THREADS / 32 + 1];
@@ -582,6 +589,7 @@ __global__ void __launch_bounds__(THREADS) vocab_ce_pipe_kernel(
     const __grid_constant__ PtrArray L, const __grid_constant__ MutPtrArray G, int p, int64_t Vs,
     int vocab, int64_t T_rows, uint32_t stage_bytes, const int32_t* labels, float scale,
     float* loss, float* lse_out, unsigned* status) {
+  tpd::pdl_entry();
   constexpr int N = Vec<T>::N;
   constexpr float kLog2e = 1.4426950408889634f;
   extern __shared__ __align__(128) uint8_t sbuf[];
@@ -796,7 +804,7 @@ tp_status launch_ce_pipe(const PtrArray& L, const MutPtrArray& G, int p, int64_t
   int64_t grid = 1;
   tp_status r = tpi::persistent_grid(reinterpret_cast<const void*>(fn), THREADS, smem, T, &grid);
   if (r != TP_OK) return r;
-  fn<<<static_cast<unsigned>(grid), THREADS, smem, st>>>(L, G, p, Vs, vocab, T, stage_bytes, labels,
+  (void)tpi::launch(fn, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem, st, L, G, p, Vs, vocab, T, stage_bytes, labels,
                                                          scale, loss, lse, status);
   return TP_OK;
 }
@@ -823,7 +831,7 @@ tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab,
   const int64_t vpr = h * static_cast<int64_t>(dsize(dt)) / 16;
   const int64_t total = T * vpr;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, sms() * 16LL));
-  embed_fwd_kernel<<<blocks, 256, 0, st>>>(ids, E, vocab, Vs, T, vpr, static_cast<uint4*>(Y), status);
+  (void)tpi::launch(embed_fwd_kernel, dim3(blocks), dim3(256), 0, st, ids, E, vocab, Vs, T, vpr, static_cast<uint4*>(Y), status);
   return after_launch("embedding_fwd");
 }
 
@@ -852,16 +860,16 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
   int2* sorted = reinterpret_cast<int2*>(tot + round4(nb + 1));
   tp_status s = TP_OK;
   if (T > 0) {
-    emb_bucket_count<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, nblk, cnt);
+    (void)tpi::launch(emb_bucket_count, dim3(nblk), dim3(kTokBlock), 0, st, ids, T, vocab, nb, nblk, cnt);
     s = after_launch("embedding_bwd count");
     if (s != TP_OK) return s;
-    emb_bucket_prefix<<<(nb + 255) / 256, 256, 0, st>>>(cnt, nb, nblk, tot);
+    (void)tpi::launch(emb_bucket_prefix, dim3((nb + 255) / 256), dim3(256), 0, st, cnt, nb, nblk, tot);
     s = after_launch("embedding_bwd prefix");
     if (s != TP_OK) return s;
-    emb_scan<<<1, 1024, 0, st>>>(tot, nb);
+    (void)tpi::launch(emb_scan, dim3(1), dim3(1024), 0, st, tot, nb);
     s = after_launch("embedding_bwd scan");
     if (s != TP_OK) return s;
-    emb_bucket_scatter<<<nblk, kTokBlock, 0, st>>>(ids, T, vocab, nb, cnt, tot, sorted);
+    (void)tpi::launch(emb_bucket_scatter, dim3(nblk), dim3(kTokBlock), 0, st, ids, T, vocab, nb, cnt, tot, sorted);
     s = after_launch("embedding_bwd scatter");
     if (s != TP_OK) return s;
   } else {
@@ -870,10 +878,10 @@ tp_status launch_embedding_bwd(const int32_t* ids, int64_t T, const void* dY, in
   }
   const unsigned grid = static_cast<unsigned>(nb);
   if (dt == TP_BF16)
-    emb_bucket_accum<__nv_bfloat16><<<grid, kAccThreads, 0, st>>>(
+    (void)tpi::launch(emb_bucket_accum<__nv_bfloat16>, dim3(grid), dim3(kAccThreads), 0, st, 
         sorted, tot, static_cast<const __nv_bfloat16*>(dY), h, Vs, Vp, dE);
   else
-    emb_bucket_accum<float><<<grid, kAccThreads, 0, st>>>(sorted, tot, static_cast<const float*>(dY), h, Vs,
+    (void)tpi::launch(emb_bucket_accum<float>, dim3(grid), dim3(kAccThreads), 0, st, sorted, tot, static_cast<const float*>(dY), h, Vs,
                                                          Vp, dE);
   return after_launch("embedding_bwd accumulate");
 }
@@ -897,10 +905,10 @@ tp_status launch_vocab_ce(const PtrArray& L, const MutPtrArray& G, int p, int64_
     s = dt == TP_BF16 ? launch_ce_pipe<__nv_bfloat16, 1024, 2, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st)
                       : launch_ce_pipe<float, 1024, 2, 0>(L, G, p, Vs, vocab, labels, scale, loss, lse, T, sb, status, st);
   } else if (dt == TP_BF16) {
-    vocab_ce_kernel<__nv_bfloat16, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(
+    (void)tpi::launch(vocab_ce_kernel<__nv_bfloat16, 256>, dim3(static_cast<unsigned>(T)), dim3(256), 0, st, 
         L, G, p, Vs, vocab, labels, scale, loss, lse, status);
   } else {
-    vocab_ce_kernel<float, 256><<<static_cast<unsigned>(T), 256, 0, st>>>(L, G, p, Vs, vocab, labels,
+    (void)tpi::launch(vocab_ce_kernel<float, 256>, dim3(static_cast<unsigned>(T)), dim3(256), 0, st, L, G, p, Vs, vocab, labels,
                                                                          scale, loss, lse, status);
   }
   if (s != TP_OK) return s;
