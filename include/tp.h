@@ -380,11 +380,14 @@ TP_API tp_status tp_all_gather_seq_bwd(tp_plan* plan, int64_t T, int n, const vo
  * xhat)) with g = dy * gamma and xhat = (x - mean) * rstd; dgamma = sum_rows
  * dy * xhat, dbeta = sum_rows dy, [hidden] fp32 (deterministic; when
  * accumulate != 0 they are added to the existing contents, so the sequence
- * shards' sums can be chained). mean/rstd from the forward. Uses the plan's
+ * shards' sums can be chained). mean/rstd from the forward. dres (NULL ok,
+ * [rows, hidden], may alias dx) is added to dx: the gradient of the residual
+ * branch around a pre-LN sublayer (x1 = x + f(LN(x)) gives dx = dres +
+ * LN'(x)^T df), so the sum needs no launch of its own. Uses the plan's
  * device workspace for per-CTA partials. */
 TP_API tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
-                           const void* dy, const float* mean, const float* rstd, void* dx,
-                           float* dgamma, float* dbeta, int accumulate, void* stream);
+                           const void* dy, const float* mean, const float* rstd, const void* dres,
+                           void* dx, float* dgamma, float* dbeta, int accumulate, void* stream);
 
 /* Backward of tp_norm_sharded_fwd: dX[i] [rows, hidden/p]; dgamma[i] (and
  * dbeta[i] for LayerNorm; NULL array ok) [hidden/p] fp32 sums over rows

@@ -431,8 +431,7 @@ class TPLayer:
         self.x1, self.y = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
         self.m1, self.r1 = _empty((T,), f32, dev), _empty((T,), f32, dev)
         self.m2, self.r2 = _empty((T,), f32, dev), _empty((T,), f32, dev)
-        self.dx1_ln, self.dx1 = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
-        self.dx_ln, self.dx = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
+        self.dx1, self.dx = _empty((T, h), bf, dev), _empty((T, h), bf, dev)
         self.dln1_g, self.dln1_b = _empty((h,), f32, dev), _empty((h,), f32, dev)
         self.dln2_g, self.dln2_b = _empty((h,), f32, dev), _empty((h,), f32, dev)
 
@@ -451,13 +450,12 @@ class TPLayer:
         T = batch * seq
         ln = self.ln
         du2 = self.mlp.backward(dy)
-        ln.layernorm_bwd(T, self.x1, self.ln2_g, du2, self.m2, self.r2, self.dx1_ln,
-                         self.dln2_g, self.dln2_b)
-        ln.reduce_partials(T, [dy, self.dx1_ln], None, None, self.dx1)        # residual branch
+        # dx1 = dy (residual branch) + LN2 backward, in one launch
+        ln.layernorm_bwd(T, self.x1, self.ln2_g, du2, self.m2, self.r2, self.dx1,
+                         self.dln2_g, self.dln2_b, dres=dy)
         du1 = self.attn.backward(self.dx1, batch, seq)
-        ln.layernorm_bwd(T, self.x, self.ln1_g, du1, self.m1, self.r1, self.dx_ln,
-                         self.dln1_g, self.dln1_b)
-        ln.reduce_partials(T, [self.dx1, self.dx_ln], None, None, self.dx)
+        ln.layernorm_bwd(T, self.x, self.ln1_g, du1, self.m1, self.r1, self.dx,
+                         self.dln1_g, self.dln1_b, dres=self.dx1)
         return self.dx
 
 

@@ -853,8 +853,8 @@ tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, const voi
 }
 
 tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
-                           const void* dy, const float* mean, const float* rstd, void* dx,
-                           float* dgamma, float* dbeta, int accumulate, void* stream) {
+                           const void* dy, const float* mean, const float* rstd, const void* dres,
+                           void* dx, float* dgamma, float* dbeta, int accumulate, void* stream) {
   TP_TRY(check_plan(plan));
   TP_TRY(check_T(rows));
   TP_TRY(check_ptr(x, "x"));
@@ -865,9 +865,10 @@ tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const voi
   TP_TRY(check_ptr(dx, "dx"));
   TP_TRY(check_ptr(dgamma, "dgamma"));
   TP_TRY(check_ptr(dbeta, "dbeta"));
+  if (dres) TP_TRY(check_ptr(dres, "dres"));
   TP_TRY(check_ln(plan));
-  return launch_layernorm_bwd(plan, x, gamma, dy, mean, rstd, dx, dgamma, dbeta, accumulate, rows,
-                              plan->hidden, plan->dtype, as_stream(stream));
+  return launch_layernorm_bwd(plan, x, gamma, dy, mean, rstd, dres, dx, dgamma, dbeta, accumulate,
+                              rows, plan->hidden, plan->dtype, as_stream(stream));
 }
 
 tp_status tp_plan_set_vocab(tp_plan* plan, int vocab, int* vocab_padded) {

@@ -110,9 +110,9 @@ tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_sr
                                const void* gamma, const void* beta, void* y, float* mean,
                                float* rstd, tp_dtype dt, cudaStream_t st);
 tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, const void* dy,
-                               const float* mean, const float* rstd, void* dx, float* dgamma,
-                               float* dbeta, int accumulate, int64_t rows, int64_t cols,
-                               tp_dtype dt, cudaStream_t st);
+                               const float* mean, const float* rstd, const void* dres, void* dx,
+                               float* dgamma, float* dbeta, int accumulate, int64_t rows,
+                               int64_t cols, tp_dtype dt, cudaStream_t st);
 
 // Vocab-parallel embedding and cross-entropy (tp_vocab.cu).
 tp_status launch_embedding_fwd(const int32_t* ids, const PtrArray& E, int vocab, int64_t Vs,
@@ -134,7 +134,8 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
                                   const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
                                   const MutPtrArray& db, int p, int64_t rows, int64_t h,
                                   const float* mean, const float* rstd, tp_dtype dt,
-                                  cudaStream_t st, int accumulate = 0);
+                                  cudaStream_t st, int accumulate = 0,
+                                  const PtrArray& DRES = PtrArray{});
 
 // ------------------------------------------------------------------- GEMM
 // One GEMM problem of a grouped launch: D[M, N] = A[M, K] . B[N, K]^T.

@@ -152,8 +152,8 @@ __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__
 template <typename T, int THREADS>
 __global__ void __launch_bounds__(THREADS) ln_bwd_dx_kernel(const T* x, const T* gamma,
                                                             const T* dy, const float* mean_in,
-                                                            const float* rstd_in, T* dx,
-                                                            int64_t cols) {
+                                                            const float* rstd_in, const T* dres,
+                                                            T* dx, int64_t cols) {
   tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   __shared__ float red[THREADS / 32];
@@ -188,6 +188,12 @@ __global__ void __launch_bounds__(THREADS) ln_bwd_dx_kernel(const T* x, const T*
       float o[V];
 #pragma unroll
       for (int k = 0; k < V; ++k) o[k] = rstd * (gy[i][k] - m1 - xh[i][k] * m2);
+      if (dres) {
+        float rr[V];
+        LnVec<T>::load(dres + r * cols + static_cast<int64_t>(c) * V, rr);
+#pragma unroll
+        for (int k = 0; k < V; ++k) o[k] += rr[k];
+      }
       LnVec<T>::store(dx + r * cols + static_cast<int64_t>(c) * V, o);
     }
   }
@@ -358,9 +364,9 @@ tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_sr
 }
 
 tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, const void* dy,
-                               const float* mean, const float* rstd, void* dx, float* dgamma,
-                               float* dbeta, int accumulate, int64_t rows, int64_t cols,
-                               tp_dtype dt, cudaStream_t st) {
+                               const float* mean, const float* rstd, const void* dres, void* dx,
+                               float* dgamma, float* dbeta, int accumulate, int64_t rows,
+                               int64_t cols, tp_dtype dt, cudaStream_t st) {
   // The backward formula takes the saved mean and rstd, so a LayerNorm over the
   // whole row is the hidden-sharded one with a single shard: its one-pass,
   // staged kernel serves whenever the row fits it.
@@ -373,8 +379,10 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
     DX.p[0] = dx;
     dg.p[0] = dgamma;
     db.p[0] = dbeta;
+    PtrArray R{};
+    R.p[0] = dres;
     return launch_norm_sharded_bwd(plan, false, X, G, DY, DX, dg, db, 1, rows, cols, mean, rstd, dt, st,
-                                   accumulate);
+                                   accumulate, R);
   }
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
@@ -394,7 +402,7 @@ tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, 
 #define TP_LN_BWD(T, TH)                                                                        \
   (void)tpi::launch(ln_bwd_dx_kernel<T, TH>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st,                          \
       static_cast<const T*>(x), static_cast<const T*>(gamma), static_cast<const T*>(dy), mean,  \
-      rstd, static_cast<T*>(dx), cols)
+      rstd, static_cast<const T*>(dres), static_cast<T*>(dx), cols)
     if (dt == TP_BF16) {
       if (th == 64) TP_LN_BWD(__nv_bfloat16, 64);
       else if (th == 128) TP_LN_BWD(__nv_bfloat16, 128);
@@ -589,9 +597,9 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
 template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
 __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
-    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX, int p, int vps,
-    int64_t hs, int64_t h, int64_t rows, const float* mean_in, const float* rstd_in,
-    float* part, unsigned* status) {
+    const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX,
+    const __grid_constant__ PtrArray DRES, int p, int vps, int64_t hs, int64_t h, int64_t rows,
+    const float* mean_in, const float* rstd_in, float* part, unsigned* status) {
   tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   extern __shared__ __align__(128) uint8_t sbuf[];
@@ -633,6 +641,20 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     if (r >= rows) break;
     const int st = static_cast<int>(k % STAGES);
     const float mean = RMS ? 0.f : mean_in[r], rstd = rstd_in[r];
+    // a gradient to add to dx (the residual branch), read now so the loads
+    // are in flight during the row's sums
+    uint4 rv[VPT];
+    if (DRES.p[0]) {
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int c = threadIdx.x + i * THREADS;
+        rv[i] = make_uint4(0, 0, 0, 0);
+        if (c < vpr) {
+          const int sh = c / vps, lc = c - sh * vps;
+          rv[i] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const T*>(DRES.p[sh]) + r * hs) + lc);
+        }
+      }
+    }
     // a thread whose wait gave up computes on an unfinished stage; the sum's
     // barrier then stops every thread before anything is written
     const bool ok = tpd::mbar_wait(&bar[st], static_cast<uint32_t>(k / STAGES) & 1u, &abort_flag, status);
@@ -671,6 +693,12 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
         LnVec<T>::unpack(gp[i], g);
 #pragma unroll
         for (int e = 0; e < V; ++e) o[e] = rstd * (d[e] * g[e] - m1 - (x[e] - mean) * rstd * m2);
+        if (DRES.p[0]) {
+          float rr[V];
+          LnVec<T>::unpack(rv[i], rr);
+#pragma unroll
+          for (int e = 0; e < V; ++e) o[e] += rr[e];
+        }
         LnVec<T>::store(const_cast<uint4*>(xrow) + c, o);  // dx replaces x in the stage
       }
     }
@@ -796,7 +824,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
                                   const PtrArray& DY, const MutPtrArray& DX, const MutPtrArray& dg,
                                   const MutPtrArray& db, int p, int64_t rows, int64_t h,
                                   const float* mean, const float* rstd, tp_dtype dt,
-                                  cudaStream_t st, int accumulate) {
+                                  cudaStream_t st, int accumulate, const PtrArray& DRES) {
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = h / V, hs = h / p;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "norm row too long (%lld)", (long long)h);
@@ -832,7 +860,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
 #define TP_NH_BWD(T, TH, VP, R)                                                               \
   (void)tpi::launch(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R>, dim3(static_cast<unsigned>(grid)), dim3(TH), \
                                                             smem, st,                        \
-      X, G, DY, DX, p, vps, hs, h, rows, mean, rstd, part, status)
+      X, G, DY, DX, DRES, p, vps, hs, h, rows, mean, rstd, part, status)
     if (dt == TP_BF16) {
       if (rms) { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
       else { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, false); }

@@ -75,7 +75,7 @@ _SIGS = {
     "tp_column_bwd": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_reduce_scatter_seq_bwd": (_int, [_plan_p, _i64, _int, _vpp, _vp, _vp]),
     "tp_all_gather_seq_bwd": (_int, [_plan_p, _i64, _int, _vpp, _vpp, _vp]),
-    "tp_layernorm_bwd": (_int, [_plan_p, _i64, _vp, _vp, _vp, _fp, _fp, _vp, _fp, _fp, _int, _vp]),
+    "tp_layernorm_bwd": (_int, [_plan_p, _i64, _vp, _vp, _vp, _fp, _fp, _vp, _vp, _fp, _fp, _int, _vp]),
     "tp_attention_bwd": (_int, [_plan_p, _int, _int, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_column_sum": (_int, [_plan_p, _i64, _i64, _vp, _fp, _int, _vp]),
     "tp_column_sum_static": (_int, [_i64, _i64, _int, _vp, _fp, _int, _vp]),
@@ -300,9 +300,10 @@ class Plan:
                                         _arr(dX_seq), _stream(stream)), "tp_all_gather_seq_bwd")
 
     def layernorm_bwd(self, rows, x, gamma, dy, mean, rstd, dx, dgamma, dbeta, accumulate=False,
-                      stream=None):
+                      stream=None, dres=None):
+        """dres (optional): a gradient added to dx (the residual branch)."""
         check(lib.tp_layernorm_bwd(self._h, rows, _ptr(x), _ptr(gamma), _ptr(dy), _ptr(mean),
-                                   _ptr(rstd), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
+                                   _ptr(rstd), _ptr(dres), _ptr(dx), _ptr(dgamma), _ptr(dbeta),
                                    1 if accumulate else 0, _stream(stream)), "tp_layernorm_bwd")
 
     def attention_bwd(self, batch, seq, QKV, O, dO, LSE, dQKV, stream=None):

@@ -189,6 +189,13 @@ def test_layernorm_fwd_bwd(h, dtype):
     plan.layernorm_bwd(rows, dev(x), dev(gamma), dev(dy), mean, rstd, dx, dg, db, accumulate=True)
     assert_close(dg[None, :], 2 * rdg[None, :], 1e-3, "LN dgamma accumulated")
     assert_close(db[None, :], 2 * rdb[None, :], 1e-3, "LN dbeta accumulated")
+    # the residual branch's gradient added in the same launch, also in place (dres is dx)
+    dres = torch.randn(rows, h, generator=g).to(tdt)
+    plan.layernorm_bwd(rows, dev(x), dev(gamma), dev(dy), mean, rstd, dx, dg, db, dres=dev(dres))
+    assert_close(dx, rdx + O.f64(dres), tol, "LN dx + dres")
+    inplace = dev(dres)
+    plan.layernorm_bwd(rows, dev(x), dev(gamma), dev(dy), mean, rstd, inplace, dg, db, dres=inplace)
+    assert_close(inplace, rdx + O.f64(dres), tol, "LN dx + dres in place")
 
 
 @pytest.mark.parametrize("n", [1, 4, 8])
