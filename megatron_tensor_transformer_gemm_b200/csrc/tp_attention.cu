@@ -47,7 +47,6 @@ constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int CHUNK_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-atom column)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // raise the reference max when exceeded by > 2^8
-constexpr int kFmaExpPairs = 1;   // of every 4 pairs of scores, this many use exp2_fma
 
 struct AttnParams {
   CUtensorMap tm[TP_MAX_SHARDS];  // QKV_i as {3*Hl*d, batch, seq}, box {64, 1, 128}
@@ -328,16 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int i = v * 8 + 2 * w;
-            // One pair in four takes the FMA-pipe exp2, so the transcendental
-            // unit (also busy with the bf16 packing) no longer bounds the loop.
-            float a, bb;
-            if (w < kFmaExpPairs) {
-              a = exp2_fma(fmaf(sv[cc][i], sc, -m));
-              bb = exp2_fma(fmaf(sv[cc][i + 1], sc, -m));
-            } else {
-              a = ex2(fmaf(sv[cc][i], sc, -m));
-              bb = ex2(fmaf(sv[cc][i + 1], sc, -m));
-            }
+            float a = ex2(fmaf(sv[cc][i], sc, -m));
+            float bb = ex2(fmaf(sv[cc][i + 1], sc, -m));
             if (!full) {
               a = (cc * 32 + i <= kmax) ? a : 0.f;
               bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;

@@ -389,24 +389,6 @@ __device__ __forceinline__ float silu_grad_f(float z) {
   return s * (1.0f + z * (1.0f - s));
 }
 
-// 2^x on the FMA and integer pipes (no transcendental or conversion unit), for
-// softmax exponents x <= 8; x below -125 is clamped, giving about 2^-125 where
-// the hardware ex2 flushes to 0. Cody-Waite style split x = n + f with
-// n = round(x) taken by the 1.5 * 2^23 magic addition (n lands in the low
-// mantissa bits of t), 2^f for f in [-1/2, 1/2] by a cubic fitted here by
-// iteratively reweighted least squares to the relative error (max 7.5e-5,
-// far below a bf16 ulp), and n added to the exponent field of 2^f.
-constexpr float kExp2C0 = 0.999928057f, kExp2C1 = 0.693260968f, kExp2C2 = 0.242611110f,
-                kExp2C3 = 0.0551716052f;
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  const float q = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

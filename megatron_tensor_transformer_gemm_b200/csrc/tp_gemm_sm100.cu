@@ -118,6 +118,7 @@ struct alignas(64) GemmParams {
   // leader CTA of each pair takes tiles with atomicAdd, the last CTA to finish
   // sets both back to zero.
   unsigned* sched;
+  int dyn_sched;  // 1: draw tiles from *sched; 0: cluster c takes c, c + clusters, ...
   unsigned* status;
 };
 
@@ -444,12 +445,14 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
     bool ok = true;
     int kseq = 0;
-    int next = rank == 0 ? static_cast<int>(atomicAdd(p.sched, 1u)) : 0;
+    const int cluster = static_cast<int>(blockIdx.x) / PAIR, clusters = static_cast<int>(gridDim.x) / PAIR;
+    int next = rank != 0 ? 0 : p.dyn_sched ? static_cast<int>(atomicAdd(p.sched, 1u)) : cluster;
     for (;;) {
       int t;
       if (rank == 0) {  // draw the next tile and publish it (or the end)
         t = next;
-        if (t < p.total_tiles) next = static_cast<int>(atomicAdd(p.sched, 1u));
+        if (t < p.total_tiles)
+          next = p.dyn_sched ? static_cast<int>(atomicAdd(p.sched, 1u)) : next + clusters;
         if (!ring_put<PAIR>(ring, kseq, t < p.total_tiles ? t : -1, abort_flag, p.status)) break;
       } else {
         t = ring_take<PAIR>(ring, kseq, rank, abort_flag, p.status);
@@ -635,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   if (PAIR == 2) cluster_sync_all();  // neither CTA leaves while its pair may still signal it
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && p.dyn_sched) {
     // every draw of this CTA is done: the last CTA to get here re-arms the counter
     __threadfence();
     if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
@@ -837,6 +840,16 @@ tp_status sched_slot(cudaStream_t st, unsigned** out) {
   return TP_OK;
 }
 
+// Dynamic tile schedule for a launch of `tiles` tiles on `units` CTA pairs (or
+// CTAs): on unless TP_GEMM_SCHED is "static" ("dynamic" forces it on).
+bool dynamic_schedule(int tiles, int units) {
+  (void)tiles;
+  (void)units;
+  const char* e = getenv("TP_GEMM_SCHED");
+  if (e && e[0] == 's') return false;
+  return true;
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -956,8 +969,11 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   p.out_f32 = b.out_f32;
   s = device_status_word(&p.status);
   if (s != TP_OK) return s;
-  s = sched_slot(st, &p.sched);
-  if (s != TP_OK) return s;
+  p.dyn_sched = dynamic_schedule(tiles, sms / pair) ? 1 : 0;
+  if (p.dyn_sched) {
+    s = sched_slot(st, &p.sched);
+    if (s != TP_OK) return s;
+  }
   if (pair == 2) return launch_kernel<2>(p, tiles, sms, st);
   return launch_kernel<1>(p, tiles, sms, st);
 }

@@ -14,9 +14,13 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("pair,narrow", [("1", "0"), ("2", "0"), ("2", "1"), ("1", "1")])
-def test_gemm_suite_under_forced_layouts(pair, narrow):
-    env = dict(os.environ, TP_GEMM_CTA_PAIR=pair, TP_GEMM_NARROW=narrow)
+@pytest.mark.parametrize("pair,narrow,sched", [("1", "0", "dynamic"), ("2", "0", "dynamic"),
+                                               ("2", "1", "dynamic"), ("1", "1", "dynamic"),
+                                               ("2", "0", "static")])
+def test_gemm_suite_under_forced_layouts(pair, narrow, sched):
+    """sched: tiles drawn from the launch's atomic counter (dynamic) or taken
+    by a fixed stride per CTA pair (static)."""
+    env = dict(os.environ, TP_GEMM_CTA_PAIR=pair, TP_GEMM_NARROW=narrow, TP_GEMM_SCHED=sched)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_gpu_gemm.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
