@@ -4,20 +4,19 @@
 //   dV = P^T dO;  dP = dO V^T;  dS = P * (dP - D),  D = rowsum(dO * O)
 //   dQ = dS K / sqrt(d);  dK = dS^T Q / sqrt(d)
 // Three launches, deterministic (no atomics):
-//   attn_bwd_prep   D for every query row (one warp per row)
-//   attn_bwd_dkdv   one CTA per 128-key block: loops over the query blocks that
-//                   see it; S and dP in TMEM, P and dS written to shared memory
-//                   (128B-swizzled, query rows), then read back MN-major as P^T
-//                   and dS^T for dV += P^T dO and dK += dS^T Q (TMEM accumulators)
-//   attn_bwd_dq     one CTA per 128-query block: loops over its key blocks;
-//                   dS to shared memory (K-major) for dQ += dS K (TMEM)
+//   attn_bwd_prep     D and lse * log2(e) for every query row (one warp per row)
+//   attn_bwd_dkdv_st  one CTA per 128-key block, keys as the MMA rows: loops
+//                     over the 64-query sub-tiles that see it, S^T and dP^T in
+//                     TMEM (two sub-tiles in flight), P^T and dS^T written to
+//                     shared memory for dV += P^T dO and dK += dS^T Q (TMEM)
+//   attn_bwd_dq       one CTA per 128-query block: loops over its key blocks;
+//                     dS to shared memory (K-major) for dQ += dS K (TMEM)
 // Warp roles in both main kernels: warp 0 TMA, warp 1 TMEM + MMA issue, warps
 // 2..9 the element-wise work (softmax recompute, dS, epilogue), two warps per
 // TMEM lane quarter, each on half of the 128 columns. Waits are bounded.
 #include <cuda.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -150,186 +149,6 @@ __device__ __forceinline__ void p_ds_row(uint32_t tS, uint32_t tdP, uint32_t lan
     }
     if (sP) store_row32_sw128(sP, r, c, pk);
     store_row32_sw128(sdS, r, c, dk);
-  }
-}
-
-template <int D, int ST>
-struct DkdvSmem {
-  static constexpr int T = BQ * D * 2;  // one [128 x D] bf16 tile
-  static constexpr int TOTAL = 1024 + 2 * T + 2 * ST * T + 2 * CHUNK * 2 + 256;
-};
-
-template <int D, int ST>
-__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv(const __grid_constant__ BwdParams p) {
-  tpd::pdl_entry();
-  using SM = DkdvSmem<D, ST>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + SM::T;
-  uint8_t* sQ = sV + SM::T;          // [ST]
-  uint8_t* sdO = sQ + ST * SM::T;    // [ST]
-  uint8_t* sP = sdO + ST * SM::T;    // 2 chunks
-  uint8_t* sdS = sP + 2 * CHUNK;     // 2 chunks
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + 2 * CHUNK);
-  uint64_t* kv_full = bars;
-  uint64_t* q_full = kv_full + 1;   // [ST]
-  uint64_t* q_empty = q_full + ST;  // [ST]
-  uint64_t* s_full = q_empty + ST;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* pds_empty = p_full + 1;
-  uint64_t* acc_full = pds_empty + 1;
-  uint64_t* drain = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = p.p * p.batch * p.hl;
-  const int j = static_cast<int>(blockIdx.x) / per;  // key block; j = 0 has the most work
-  int rest = static_cast<int>(blockIdx.x) % per;
-  const int hh = rest % p.hl;
-  rest /= p.hl;
-  const int b = rest % p.batch;
-  const int shard = rest / p.batch;
-  const int k0 = j * BKV;
-  const int n_iter = p.nq - j;  // query blocks j .. nq-1 see this key block
-  const int hl_d = p.hl * D;
-  const CUtensorMap* tq = &p.tm_qkv[shard];
-  const CUtensorMap* tdo = &p.tm_do[shard];
-
-  if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
-    }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
-    mbar_init(pds_empty, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
-
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(tq);
-    tma_prefetch_desc(tdo);
-    mbar_arrive_expect_tx(kv_full, 2 * SM::T);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sK + c * CHUNK, tq, kv_full, hl_d + hh * D + c * 64, b, k0);
-      tma_load_3d(sV + c * CHUNK, tq, kv_full, 2 * hl_d + hh * D + c * 64, b, k0);
-    }
-    int last_par[ST];
-    for (int s = 0; s < ST; ++s) last_par[s] = -1;
-    for (int it = 0; it < n_iter; ++it) {
-      const int st = it % ST;
-      const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
-      if (!mbar_wait(&q_empty[st], ph ^ 1u, abort_flag, p.status)) break;
-      const int q0 = (j + it) * BQ;
-      mbar_arrive_expect_tx(&q_full[st], 2 * SM::T);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sQ + st * SM::T + c * CHUNK, tq, &q_full[st], hh * D + c * 64, b, q0);
-        tma_load_3d(sdO + st * SM::T + c * CHUNK, tdo, &q_full[st], hh * D + c * 64, b, q0);
-      }
-      last_par[st] = static_cast<int>(ph);
-    }
-    mbar_wait(kv_full, 0, abort_flag, p.status);
-    for (int s = 0; s < ST; ++s)
-      if (last_par[s] >= 0) mbar_wait(&q_full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
-  } else if (warp == 1 && lane == 0) {
-    const uint32_t id_s = idesc_bf16(BQ, BKV, false, false);
-    const uint32_t id_acc = idesc_bf16(BKV, D, true, true);
-    const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
-    const uint32_t p_base = smem_u32(sP), ds_base = smem_u32(sdS);
-    bool ok = mbar_wait(kv_full, 0, abort_flag, p.status);
-    for (int it = 0; ok && it < n_iter; ++it) {
-      const int st = it % ST;
-      if (!mbar_wait(&q_full[st], static_cast<uint32_t>(it / ST) & 1u, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t q_base = smem_u32(sQ + st * SM::T), do_base = smem_u32(sdO + st * SM::T);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk / 4) * CHUNK + (kk % 4) * 32;
-        tc_mma_bf16(tS, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
-                    id_s, kk > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk / 4) * CHUNK + (kk % 4) * 32;
-        tc_mma_bf16(tdP, smem_desc_sw128(do_base + off, 16, 1024), smem_desc_sw128(v_base + off, 16, 1024),
-                    id_s, kk > 0 ? 1u : 0u);
-      }
-      tc_commit(s_full);
-      if (!mbar_wait(p_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status)) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < BQ / 16; ++kk) {  // K = queries
-        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_bf16(tdV, smem_desc_sw128(p_base + kk * 2048, CHUNK, 1024),
-                    smem_desc_sw128(do_base + kk * 2048, CHUNK, 1024), id_acc, acc);
-        tc_mma_bf16(tdK, smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
-                    smem_desc_sw128(q_base + kk * 2048, CHUNK, 1024), id_acc, acc);
-      }
-      tc_commit(&q_empty[st]);
-      tc_commit(pds_empty);
-    }
-    tc_commit(acc_full);
-    tc_commit(drain);
-    mbar_wait(drain, 0, abort_flag, p.status);
-  } else if (warp >= 2) {
-    const int lg = warp & 3;
-    const int half = (warp - 2) / 4;
-    const int r = lg * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-    const float* lse = p.lse[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq;
-    const float* dv = p.dvec[shard] + (static_cast<int64_t>(b) * p.hl + hh) * p.seq_pad;
-    bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int q = (j + it) * BQ + r;
-      const float lse2 = q < p.seq ? lse[q] * kLog2e : 0.f;
-      const float Dq = q < p.seq ? dv[q] : 0.f;
-      // warp-uniform: p_ds_row's tcgen05.ld is warp-collective
-      const bool got = mbar_wait(s_full, static_cast<uint32_t>(it) & 1u, abort_flag, p.status) &&
-                       mbar_wait(pds_empty, (static_cast<uint32_t>(it) & 1u) ^ 1u, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      p_ds_row(tS, tdP, lane_off, r, q, k0, p.seq, p.scale_log2, lse2, Dq, sP, sdS, 2 * half);
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
-      tc_fence_after();
-      const int key = k0 + r;  // accumulator lane = key row
-      __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
-                            (static_cast<int64_t>(key) * p.batch + b) * (3 * hl_d) + hh * D;
-      const bool st_ok = key < p.seq;
-      if (half == 0) tmem_row_to_global<D>(tdV + lane_off, base + 2 * hl_d, 1.f, st_ok);
-      else tmem_row_to_global<D>(tdK + lane_off, base + hl_d, p.scale, st_ok);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -760,240 +579,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
   }
 }
 
-// ---------------------------------------------------------------------------
-// dQ with 64-key sub-blocks, two in flight. One CTA per 128-query tile of one
-// (shard, batch, head); for each sub-block of 64 keys the tile sees:
-//   S = Q K_s^T and dP = dO V_s^T          (M = 128 queries, N = 64 keys)
-//   dS = exp2(S * scale * log2e - lse2) * (dP - D)   (element-wise, thread = query row)
-//   dQ += dS K_s                           (N = d, K = 64 keys; K_s read MN-major)
-// TMEM holds dQ (d columns) and two (S, dP) pairs of 64 columns, so the MMAs of
-// sub-block j + 1 (and the dQ MMAs of j - 1) run while the element-wise warps
-// work on j. K_s, V_s stream through ST stages.
-template <int D, int ST>
-struct DqStSmem {
-  static constexpr int QT = 128 * D * 2;  // Q or dO tile [128 x D]
-  static constexpr int KS = 64 * D * 2;   // K or V sub-block [64 x D]
-  static constexpr int CH = 64 * 128;     // a 64-row 128B-swizzle column chunk of a sub-block
-  static constexpr int DS = 128 * 128;    // dS [128 queries x 64 keys] bf16 (one swizzle chunk)
-  static constexpr int TOTAL = 1024 + 2 * QT + 2 * ST * KS + 2 * DS + 256;
-};
-
-template <int D, int ST>
-__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_st(const __grid_constant__ BwdParams p) {
-  using SM = DqStSmem<D, ST>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + SM::QT;
-  uint8_t* sK = sdO + SM::QT;        // [ST]
-  uint8_t* sV = sK + ST * SM::KS;    // [ST]
-  uint8_t* sdS = sV + ST * SM::KS;   // [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + 2 * SM::DS);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = q_full + 1;     // [ST]
-  uint64_t* kv_empty = kv_full + ST;  // [ST]
-  uint64_t* s_full = kv_empty + ST;   // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* ds_empty = p_full + 2;    // [2]
-  uint64_t* acc_full = ds_empty + 2;
-  uint64_t* drain = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = p.p * p.batch * p.hl;
-  const int i = p.nq - 1 - static_cast<int>(blockIdx.x) / per;  // heaviest query tiles first
-  int rest = static_cast<int>(blockIdx.x) % per;
-  const int hh = rest % p.hl;
-  rest /= p.hl;
-  const int b = rest % p.batch;
-  const int shard = rest / p.batch;
-  const int q0 = i * BQ;
-  const int nsub = min(2 * i + 2, (p.seq + 63) / 64);  // 64-key sub-blocks 0 .. that the tile sees
-  const int hl_d = p.hl * D;
-  const int64_t bh = static_cast<int64_t>(b) * p.hl + hh;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 8);
-      mbar_init(&ds_empty[x], 1);
-    }
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  pdl_entry();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tdQ = tmem;
-  const uint32_t tS0 = tmem + D;  // buffer x: S at tS0 + 128 x, dP at tS0 + 128 x + 64
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    const CUtensorMap* tq = &p.tm_qkv[shard];
-    const CUtensorMap* tdo = &p.tm_do[shard];
-    const CUtensorMap* tq64 = &p.tm_q64[shard];
-    tma_prefetch_desc(tq);
-    tma_prefetch_desc(tdo);
-    tma_prefetch_desc(tq64);
-    mbar_arrive_expect_tx(q_full, 2 * SM::QT);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sQ + c * 128 * 128, tq, q_full, hh * D + c * 64, b, q0);
-      tma_load_3d(sdO + c * 128 * 128, tdo, q_full, hh * D + c * 64, b, q0);
-    }
-    int last_par[ST];
-    for (int s = 0; s < ST; ++s) last_par[s] = -1;
-    for (int it = 0; it < nsub; ++it) {
-      const int st = it % ST;
-      const uint32_t ph = static_cast<uint32_t>(it / ST) & 1u;
-      if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag, p.status)) break;
-      const int kb0 = it * 64;
-      mbar_arrive_expect_tx(&kv_full[st], 2 * SM::KS);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK + st * SM::KS + c * SM::CH, tq64, &kv_full[st], hl_d + hh * D + c * 64, b, kb0);
-        tma_load_3d(sV + st * SM::KS + c * SM::CH, tq64, &kv_full[st], 2 * hl_d + hh * D + c * 64, b, kb0);
-      }
-      last_par[st] = static_cast<int>(ph);
-    }
-    mbar_wait(q_full, 0, abort_flag, p.status);
-    for (int s = 0; s < ST; ++s)
-      if (last_par[s] >= 0) mbar_wait(&kv_full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------- MMA issuer
-    const uint32_t id_s = idesc_bf16(BQ, 64, false, false);  // M = 128 queries, N = 64 keys
-    const uint32_t id_dq = idesc_bf16(BQ, D, false, true);   // N = d, B (K_s) MN-major
-    const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sdO);
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-    // dQ += dS K_s of sub-block j (buffer j & 1)
-    auto acc_mma = [&](int j) -> bool {
-      const int x = j & 1, st = j % ST;
-      if (!mbar_wait(&p_full[x], static_cast<uint32_t>(j >> 1) & 1u, abort_flag, p.status)) return false;
-      tc_fence_after();
-      const uint32_t ds_base = smem_u32(sdS + x * SM::DS), k_base = smem_u32(sK + st * SM::KS);
-#pragma unroll
-      for (int kk = 0; kk < 64 / 16; ++kk)  // K = the sub-block's 64 keys
-        tc_mma_bf16(tdQ, smem_desc_sw128(ds_base + kk * 32, 16, 1024),
-                    smem_desc_sw128(k_base + kk * 2048, SM::CH, 1024), id_dq, (j > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(&kv_empty[st]);
-      tc_commit(&ds_empty[x]);
-      return true;
-    };
-    for (int it = 0; ok && it < nsub; ++it) {
-      const int st = it % ST, x = it & 1;
-      if (!mbar_wait(&kv_full[st], static_cast<uint32_t>(it / ST) & 1u, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t k_base = smem_u32(sK + st * SM::KS), v_base = smem_u32(sV + st * SM::KS);
-      const uint32_t tS = tS0 + 128 * x, tdP = tS + 64;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t aoff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-        const uint32_t boff = (kk / 4) * SM::CH + (kk % 4) * 32;
-        tc_mma_bf16(tS, smem_desc_sw128(q_base + aoff, 16, 1024), smem_desc_sw128(k_base + boff, 16, 1024),
-                    id_s, kk > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t aoff = (kk / 4) * (128 * 128) + (kk % 4) * 32;
-        const uint32_t boff = (kk / 4) * SM::CH + (kk % 4) * 32;
-        tc_mma_bf16(tdP, smem_desc_sw128(do_base + aoff, 16, 1024), smem_desc_sw128(v_base + boff, 16, 1024),
-                    id_s, kk > 0 ? 1u : 0u);
-      }
-      tc_commit(&s_full[x]);
-      if (it > 0 && !acc_mma(it - 1)) {
-        ok = false;
-        break;
-      }
-    }
-    if (ok && nsub > 0) ok = acc_mma(nsub - 1);
-    tc_commit(acc_full);
-    tc_commit(drain);
-    mbar_wait(drain, 0, abort_flag, p.status);
-  } else if (warp >= 2) {
-    // --------------------------------------------------------- element-wise
-    const int lg = warp & 3;
-    const int half = (warp - 2) / 4;  // key columns [32 half, 32 half + 32) of a sub-block
-    const int r = lg * 32 + lane;     // query row of the tile
-    const int q = q0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-    const float lse2 = q < p.seq ? p.lse2[shard][bh * p.seq_pad + q] : 0.f;
-    const float Dq = q < p.seq ? p.dvec[shard][bh * p.seq_pad + q] : 0.f;
-    bool ok = true;
-    for (int it = 0; it < nsub; ++it) {
-      const int x = it & 1;
-      const uint32_t ph2 = static_cast<uint32_t>(it >> 1) & 1u;
-      // warp-uniform: the tcgen05.ld below is warp-collective
-      const bool got = mbar_wait(&s_full[x], ph2, abort_flag, p.status) &&
-                       mbar_wait(&ds_empty[x], ph2 ^ 1u, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t tS = tS0 + 128 * x, tdP = tS + 64;
-      float sv[32], dp[32];
-      tmem_ld32(tS + lane_off + half * 32, sv);
-      tmem_ld32(tdP + lane_off + half * 32, dp);
-      tc_wait_ld();
-      const int kb = it * 64 + half * 32;  // key of column 0 of this half
-      uint32_t dk[16];
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const bool v0 = kb + e <= q && kb + e < p.seq && q < p.seq;
-        const bool v1 = kb + e + 1 <= q && kb + e + 1 < p.seq && q < p.seq;
-        const float p0 = v0 ? exp2f(sv[e] * p.scale_log2 - lse2) : 0.f;
-        const float p1 = v1 ? exp2f(sv[e + 1] * p.scale_log2 - lse2) : 0.f;
-        dk[e / 2] = pack_bf16x2(v0 ? p0 * (dp[e] - Dq) : 0.f, v1 ? p1 * (dp[e + 1] - Dq) : 0.f);
-      }
-      uint8_t* drow = sdS + x * SM::DS + r * 128;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int qv = half * 4 + v;
-        *reinterpret_cast<uint4*>(drow + ((qv ^ (r & 7)) << 4)) =
-            make_uint4(dk[v * 4 + 0], dk[v * 4 + 1], dk[v * 4 + 2], dk[v * 4 + 3]);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[x]);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
-      tc_fence_after();
-      __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
-                            (static_cast<int64_t>(q) * p.batch + b) * (3 * hl_d) + hh * D;
-      // each column half of warps stores half of dQ's D columns
-      tmem_row_to_global<D / 2>(tdQ + lane_off + half * (D / 2), base + half * (D / 2), p.scale, q < p.seq);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// STK / STQ: stages of the streamed Q, dO blocks (dK/dV kernel) and K, V
-// blocks (dQ kernel); as many as fit the 227 KB of shared memory.
-template <int D, int STK, int STS, int STQ, int STQS>
+// STS: stages of the streamed 64-query Q, dO sub-tiles (dK/dV kernel); STQ:
+// stages of the streamed 128-key K, V blocks (dQ kernel); as many as fit the
+// 227 KB of shared memory.
+template <int D, int STS, int STQ>
 tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
-  static_assert(DkdvSmem<D, STK>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448 &&
-                    DkdvStSmem<D, STS>::TOTAL <= 232448 && DqStSmem<D, STQS>::TOTAL <= 232448,
+  static_assert(DkdvStSmem<D, STS>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448,
                 "shared memory of the backward kernels");
   constexpr int kMaxDev = 64;
   static bool attr[kMaxDev] = {};
@@ -1004,35 +595,20 @@ tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
   }
   if (!attr[dev]) {
     tp_status s = tpi::cuda_status(
-        cudaFuncSetAttribute(attn_bwd_dkdv<D, STK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DkdvSmem<D, STK>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
-    if (s != TP_OK) return s;
-    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dkdv_st<D, STS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              DkdvStSmem<D, STS>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
+        cudaFuncSetAttribute(attn_bwd_dkdv_st<D, STS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvStSmem<D, STS>::TOTAL), "cudaFuncSetAttribute(attention dkdv)");
     if (s != TP_OK) return s;
     s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq<D, STQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               DqSmem<D, STQ>::TOTAL), "cudaFuncSetAttribute(attention dq)");
     if (s != TP_OK) return s;
-    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq_st<D, STQS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              DqStSmem<D, STQS>::TOTAL), "cudaFuncSetAttribute(attention dq)");
-    if (s != TP_OK) return s;
     attr[dev] = true;
   }
   const int per = prm.p * prm.batch * prm.hl;
-  const char* e = getenv("TP_ATTN_BWD_DKDV");
-  if (e && e[0] == '1') {
-    (void)tpi::launch(attn_bwd_dkdv<D, STK>, dim3(prm.nkv * per), dim3(kThreads), DkdvSmem<D, STK>::TOTAL, st, prm);
-  } else {
-    (void)tpi::launch(attn_bwd_dkdv_st<D, STS>, dim3(prm.nkv * per), dim3(kThreads), DkdvStSmem<D, STS>::TOTAL, st, prm);
-  }
+  (void)tpi::launch(attn_bwd_dkdv_st<D, STS>, dim3(prm.nkv * per), dim3(kThreads), DkdvStSmem<D, STS>::TOTAL, st,
+                    prm);
   tp_status s = tpi::after_launch("attention_bwd dK/dV (tcgen05)");
   if (s != TP_OK) return s;
-  const char* eq = getenv("TP_ATTN_BWD_DQ");
-  if (eq && eq[0] == '1')
-    (void)tpi::launch(attn_bwd_dq<D, STQ>, dim3(prm.nq * per), dim3(kThreads), DqSmem<D, STQ>::TOTAL, st, prm);
-  else
-    (void)tpi::launch(attn_bwd_dq_st<D, STQS>, dim3(prm.nq * per), dim3(kThreads), DqStSmem<D, STQS>::TOTAL, st,
-                      prm);
+  (void)tpi::launch(attn_bwd_dq<D, STQ>, dim3(prm.nq * per), dim3(kThreads), DqSmem<D, STQ>::TOTAL, st, prm);
   return tpi::after_launch("attention_bwd dQ (tcgen05)");
 }
 
@@ -1098,8 +674,8 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
                                                                                  batch, seq, seq_pad, hl, d);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;
-  if (d == 64) return launch_bwd_d<64, 2, 4, 2, 4>(prm, st);
-  if (d == 128) return launch_bwd_d<128, 1, 3, 2, 4>(prm, st);
+  if (d == 64) return launch_bwd_d<64, 4, 2>(prm, st);
+  if (d == 128) return launch_bwd_d<128, 3, 2>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
 }
 

@@ -114,9 +114,10 @@ struct alignas(64) GemmParams {
   int base_tiles;
   int kb_per_split;
   int64_t split_stride;
-  // Dynamic tile schedule: {next tile, CTAs finished}, zero at launch; the
-  // leader CTA of each pair takes tiles with atomicAdd, the last CTA to finish
-  // sets both back to zero.
+  // Dynamic tile schedule: {draws, pairs done drawing}, zero at launch. Pair c
+  // (or CTA c) starts on tile c; its leader then draws tile clusters + n with
+  // n = atomicAdd(draws, 1) until one comes back past the end, and the last
+  // pair to get there sets both words back to zero.
   unsigned* sched;
   int dyn_sched;  // 1: draw tiles from *sched; 0: cluster c takes c, c + clusters, ...
   unsigned* status;
@@ -326,6 +327,19 @@ struct TileRing {
 // the producer (peer), plus the epilogue warps.
 constexpr int kRingConsumers = 1 + kEpiWarps;
 
+// Called once by each leader that drew (a draw returned past the end, or it
+// gave up): the last of the pairs that draw sets the slot back to zero. Every
+// draw of every pair has returned by then, since each pair's last draw
+// returned before it counted itself out.
+__device__ __forceinline__ void sched_done_drawing(const GemmParams& p, int clusters) {
+  const unsigned drawers = static_cast<unsigned>(min(clusters, p.total_tiles));
+  __threadfence();  // this pair's draws are performed before it counts itself out
+  if (atomicAdd(p.sched + 1, 1u) == drawers - 1) {
+    atomicExch(p.sched, 0u);
+    atomicExch(p.sched + 1, 0u);
+  }
+}
+
 template <int PAIR>
 __device__ __forceinline__ bool ring_put(const TileRing& r, int k, int v, volatile int* abort,
                                          unsigned* status) {
@@ -446,13 +460,26 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     bool ok = true;
     int kseq = 0;
     const int cluster = static_cast<int>(blockIdx.x) / PAIR, clusters = static_cast<int>(gridDim.x) / PAIR;
-    int next = rank != 0 ? 0 : p.dyn_sched ? static_cast<int>(atomicAdd(p.sched, 1u)) : cluster;
+    // The first tile needs no draw, so the first copies start at once; each
+    // draw is issued a tile ahead and its result first read one tile later.
+    int next = cluster;
+    bool drawing = false;  // a draw of this pair is outstanding or came back empty
+    bool done_drawing = !p.dyn_sched || cluster >= p.total_tiles;
     for (;;) {
       int t;
       if (rank == 0) {  // draw the next tile and publish it (or the end)
         t = next;
-        if (t < p.total_tiles)
-          next = p.dyn_sched ? static_cast<int>(atomicAdd(p.sched, 1u)) : next + clusters;
+        if (t < p.total_tiles) {
+          if (p.dyn_sched) {
+            next = clusters + static_cast<int>(atomicAdd(p.sched, 1u));
+            drawing = true;
+          } else {
+            next += clusters;
+          }
+        } else if (drawing && !done_drawing) {
+          sched_done_drawing(p, clusters);
+          done_drawing = true;
+        }
         if (!ring_put<PAIR>(ring, kseq, t < p.total_tiles ? t : -1, abort_flag, p.status)) break;
       } else {
         t = ring_take<PAIR>(ring, kseq, rank, abort_flag, p.status);
@@ -533,6 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       }
       if (!ok) break;
     }
+    // A leader that left early (bounded wait gave up) still counts itself out,
+    // so the counters of this slot return to zero.
+    if (rank == 0 && !done_drawing) sched_done_drawing(p, clusters);
     // Drain: every copy of this CTA (and, for the leader, of the pair) has
     // landed before the CTA exits. The peer's copies complete on the leader's
     // barriers, which the leader drains.
@@ -638,14 +668,6 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   if (PAIR == 2) cluster_sync_all();  // neither CTA leaves while its pair may still signal it
-  if (threadIdx.x == 0 && p.dyn_sched) {
-    // every draw of this CTA is done: the last CTA to get here re-arms the counter
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-      atomicExch(p.sched, 0u);
-      atomicExch(p.sched + 1, 0u);
-    }
-  }
   if (warp == 1) {
     tc_fence_after();
     if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
@@ -841,13 +863,13 @@ tp_status sched_slot(cudaStream_t st, unsigned** out) {
 }
 
 // Dynamic tile schedule for a launch of `tiles` tiles on `units` CTA pairs (or
-// CTAs): on unless TP_GEMM_SCHED is "static" ("dynamic" forces it on).
+// CTAs): on when some unit takes more than one tile (with one tile each, the
+// first tiles are the whole schedule). TP_GEMM_SCHED=static / dynamic forces it.
 bool dynamic_schedule(int tiles, int units) {
-  (void)tiles;
-  (void)units;
   const char* e = getenv("TP_GEMM_SCHED");
   if (e && e[0] == 's') return false;
-  return true;
+  if (e && e[0] == 'd') return true;
+  return tiles > units;
 }
 
 int device_sms() {

@@ -180,32 +180,20 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
 }
 
 // X_full rows [j*rows_per_src, ...) = src.p[j] rows; 16-byte vectors. A thread
-// owns one column vector and walks the rows of each shard in turn (no
-// division per row), four rows per step with the four loads issued before
-// the stores, so four 16-byte loads per thread are in flight.
-__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ PtrArray src, int n,
-                                                          void* dst, int64_t vpr,
-                                                          int64_t rows_per_src) {
+// owns one column vector and walks the rows of the full output with the grid's
+// row stride, reading each from the shard that holds it (streaming loads: the
+// shards are read once).
+__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ PtrArray src, void* dst,
+                                                          int64_t rows, int64_t vpr, int64_t rows_per_src) {
   tpd::pdl_entry();
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (cv >= vpr) return;
   const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.y;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y;
-  for (int j = 0; j < n; ++j) {
-    const uint4* S = static_cast<const uint4*>(src.p[j]) + cv;
-    uint4* D = static_cast<uint4*>(dst) + static_cast<int64_t>(j) * rows_per_src * vpr + cv;
-    int64_t r = r0;
-    for (; r + 3 * stride < rows_per_src; r += 4 * stride) {
-      const uint4 a = ld_stream(S + r * vpr);
-      const uint4 b = ld_stream(S + (r + stride) * vpr);
-      const uint4 c = ld_stream(S + (r + 2 * stride) * vpr);
-      const uint4 d = ld_stream(S + (r + 3 * stride) * vpr);
-      D[r * vpr] = a;
-      D[(r + stride) * vpr] = b;
-      D[(r + 2 * stride) * vpr] = c;
-      D[(r + 3 * stride) * vpr] = d;
-    }
-    for (; r < rows_per_src; r += stride) D[r * vpr] = ld_stream(S + r * vpr);
+  uint4* D = static_cast<uint4*>(dst);
+  for (int64_t r = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; r < rows; r += stride) {
+    const int j = static_cast<int>(r / rows_per_src);
+    const int64_t lr = r - static_cast<int64_t>(j) * rows_per_src;
+    D[r * vpr + cv] = ld_stream(static_cast<const uint4*>(src.p[j]) + lr * vpr + cv);
   }
 }
 
@@ -419,7 +407,7 @@ tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_
   const int64_t vpr = cols * static_cast<int64_t>(dsize(dt)) / 16;
   dim3 grid, block;
   row_walk_shape(vpr, T, &grid, &block);
-  (void)tpi::launch(gather_kernel, dim3(grid), dim3(block), 0, st, src, n, dst, vpr, T / n);
+  (void)tpi::launch(gather_kernel, dim3(grid), dim3(block), 0, st, src, dst, T, vpr, T / n);
   return after_launch("all_gather_seq");
 }
 
