@@ -594,7 +594,9 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_row_fwd_kernel(
 // column partials dgamma = sum dy * xhat and dbeta = sum dy in registers and
 // writes them once: part[b][0][col], part[b][1][col]. A second kernel sums the
 // partials over b in order, so the parameter gradients are deterministic.
-template <typename T, int THREADS, int VPT, int STAGES, bool RMS>
+// RES: DRES holds a gradient to add to dx (the residual branch); a separate
+// instance, so the plain one keeps its register count (and its residency).
+template <typename T, int THREADS, int VPT, int STAGES, bool RMS, bool RES>
 __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     const __grid_constant__ PtrArray X, const __grid_constant__ PtrArray G,
     const __grid_constant__ PtrArray DY, const __grid_constant__ MutPtrArray DX,
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
     // a gradient to add to dx (the residual branch), read now so the loads
     // are in flight during the row's sums
     uint4 rv[VPT];
-    if (DRES.p[0]) {
+    if (RES) {
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const int c = threadIdx.x + i * THREADS;
@@ -693,7 +695,7 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
         LnVec<T>::unpack(gp[i], g);
 #pragma unroll
         for (int e = 0; e < V; ++e) o[e] = rstd * (d[e] * g[e] - m1 - (x[e] - mean) * rstd * m2);
-        if (DRES.p[0]) {
+        if (RES) {
           float rr[V];
           LnVec<T>::unpack(rv[i], rr);
 #pragma unroll
@@ -781,6 +783,10 @@ constexpr int kNormBwdStages = 3;
   else if (vpt == 2) LAUNCH(T, 256, 2, R);           \
   else if (vpt == 4) LAUNCH(T, 256, 4, R);           \
   else LAUNCH(T, 256, 8, R)
+// The backward's instances also differ by whether a residual gradient is added.
+#define TP_NH_BWD_DISPATCH(LAUNCH, T, R)                                 \
+  if (res) { TP_NH_DISPATCH(LAUNCH##_RES, T, R); }                       \
+  else { TP_NH_DISPATCH(LAUNCH##_PLAIN, T, R); }
 
 // Persistent grid for a staged row kernel: as many CTAs as are resident at
 // once (at most one per row), with its dynamic shared memory opted in.
@@ -838,17 +844,22 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   // The grid (and so the partials' size) depends only on the kernel, not on
   // the data: size it first, then the workspace.
   int64_t grid = 1;
-#define TP_NH_GRID(T, TH, VP, R)                                                          \
-  s = pipe_grid(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R>, TH, smem,         \
+  const bool res = DRES.p[0] != nullptr;
+#define TP_NH_GRID_(T, TH, VP, R, RES)                                                          \
+  s = pipe_grid(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R, RES>, TH, smem,          \
                 std::max<int64_t>(rows, 1), &grid)
+#define TP_NH_GRID_RES(T, TH, VP, R) TP_NH_GRID_(T, TH, VP, R, true)
+#define TP_NH_GRID_PLAIN(T, TH, VP, R) TP_NH_GRID_(T, TH, VP, R, false)
   if (dt == TP_BF16) {
-    if (rms) { TP_NH_DISPATCH(TP_NH_GRID, __nv_bfloat16, true); }
-    else { TP_NH_DISPATCH(TP_NH_GRID, __nv_bfloat16, false); }
+    if (rms) { TP_NH_BWD_DISPATCH(TP_NH_GRID, __nv_bfloat16, true); }
+    else { TP_NH_BWD_DISPATCH(TP_NH_GRID, __nv_bfloat16, false); }
   } else {
-    if (rms) { TP_NH_DISPATCH(TP_NH_GRID, float, true); }
-    else { TP_NH_DISPATCH(TP_NH_GRID, float, false); }
+    if (rms) { TP_NH_BWD_DISPATCH(TP_NH_GRID, float, true); }
+    else { TP_NH_BWD_DISPATCH(TP_NH_GRID, float, false); }
   }
-#undef TP_NH_GRID
+#undef TP_NH_GRID_PLAIN
+#undef TP_NH_GRID_RES
+#undef TP_NH_GRID_
   if (s != TP_OK) return s;
   const int groups = grid > 2 * kParamGroup ? static_cast<int>((grid + kParamGroup - 1) / kParamGroup) : 0;
   void* ws = nullptr;
@@ -857,18 +868,22 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   float* part = static_cast<float*>(ws);
   float* inter = part + grid * 2 * h;
   if (rows > 0) {
-#define TP_NH_BWD(T, TH, VP, R)                                                               \
-  (void)tpi::launch(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R>, dim3(static_cast<unsigned>(grid)), dim3(TH), \
-                                                            smem, st,                        \
-      X, G, DY, DX, DRES, p, vps, hs, h, rows, mean, rstd, part, status)
+#define TP_NH_BWD_(T, TH, VP, R, RES)                                                                 \
+  (void)tpi::launch(norm_hsh_bwd_fused_kernel<T, TH, VP, kNormBwdStages, R, RES>,                    \
+                    dim3(static_cast<unsigned>(grid)), dim3(TH), smem, st, X, G, DY, DX, DRES, p, vps, \
+                    hs, h, rows, mean, rstd, part, status)
+#define TP_NH_BWD_RES(T, TH, VP, R) TP_NH_BWD_(T, TH, VP, R, true)
+#define TP_NH_BWD_PLAIN(T, TH, VP, R) TP_NH_BWD_(T, TH, VP, R, false)
     if (dt == TP_BF16) {
-      if (rms) { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
-      else { TP_NH_DISPATCH(TP_NH_BWD, __nv_bfloat16, false); }
+      if (rms) { TP_NH_BWD_DISPATCH(TP_NH_BWD, __nv_bfloat16, true); }
+      else { TP_NH_BWD_DISPATCH(TP_NH_BWD, __nv_bfloat16, false); }
     } else {
-      if (rms) { TP_NH_DISPATCH(TP_NH_BWD, float, true); }
-      else { TP_NH_DISPATCH(TP_NH_BWD, float, false); }
+      if (rms) { TP_NH_BWD_DISPATCH(TP_NH_BWD, float, true); }
+      else { TP_NH_BWD_DISPATCH(TP_NH_BWD, float, false); }
     }
-#undef TP_NH_BWD
+#undef TP_NH_BWD_PLAIN
+#undef TP_NH_BWD_RES
+#undef TP_NH_BWD_
     s = after_launch("norm_sharded_bwd");
     if (s != TP_OK) return s;
   }
@@ -886,6 +901,7 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
   return after_launch("norm_sharded_bwd/param");
 }
 
+#undef TP_NH_BWD_DISPATCH
 #undef TP_NH_DISPATCH
 
 }  // namespace tpi
