@@ -53,6 +53,10 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int TMEM_COLS = 512;
 constexpr int kBarBytes = 512;  // barriers, TMEM slot, abort flag, tile ring
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64-wide MN block of an MN-major tile
+// TMA epilogue staging: per epilogue warp two [32 rows x 32 bf16] tiles.
+constexpr int kEpiTile = 32 * 64;
+constexpr int kEpiBuf = 2 * kEpiTile;
+constexpr int kEpiBytes = kEpiWarps * kEpiBuf;
 
 // Per-CTA tile geometry. PAIR = 1: one CTA computes a 128 x 256 tile.
 // PAIR = 2: a (2,1,1) cluster computes a 256 x 256 tile with cta_group::2
@@ -65,7 +69,8 @@ struct Cfg {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = PAIR == 1 ? 4 : 6;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + kBarBytes;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + kEpiBytes + kBarBytes;
+  static_assert(SMEM_BYTES <= 232448, "shared memory of the GEMM kernel");
 };
 
 struct GroupArgs {
@@ -120,8 +125,16 @@ struct alignas(64) GemmParams {
   // pair to get there sets both words back to zero.
   unsigned* sched;
   int dyn_sched;  // 1: draw tiles from *sched; 0: cluster c takes c, c + clusters, ...
+  // TMA epilogue (tma_epi = 1; bf16 outputs, no scatter, no split K): per
+  // output problem, tmE views D and tmX the staged input (Z of the dGELU /
+  // dSwiGLU epilogues, or the residual) as {columns, halves, rows} with a
+  // {32, 1, 32} box and 64-byte swizzle; halves = 2 splits [gate | up] at nh.
+  int tma_epi;
+  CUtensorMap tmE[TP_MAX_SHARDS];
+  CUtensorMap tmX[TP_MAX_SHARDS];
   unsigned* status;
 };
+static_assert(sizeof(GemmParams) <= 32764, "kernel parameter space");
 
 __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, int& mt, int& nt,
                                             int& ks) {
@@ -308,6 +321,237 @@ __device__ void epilogue_tile(const GemmParams& p, const GroupArgs& ga, uint32_t
   }
 }
 
+// ------------------------------------------------------ TMA epilogue
+// Each epilogue warp stages its 32 rows x 32 columns of a chunk in its own two
+// [32 x 64 B] tiles of shared memory, 64-byte swizzled: the 16-byte piece q of
+// row r sits at r * 64 + ((q ^ ((r >> 1) & 3)) << 4), so a warp reading or
+// writing one piece of each of its rows touches every bank once per 128 bytes.
+// Inputs (the aux Z, or the residual) arrive by TMA load, outputs leave by TMA
+// store (clipped at the tensor's edges), and a thread touches only its own
+// row. Global memory sees whole 64-byte row segments instead of the 16-byte
+// pieces of 32 rows that one vector store per row gives.
+__device__ __forceinline__ uint32_t sw64(uint32_t tile, int r, int q) {
+  return tile + static_cast<uint32_t>(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ void stage_read(uint32_t tile, int r, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = ld_shared_v4(sw64(tile, r, q));
+    const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y), c = unpack_bf16x2(u.z),
+                 d = unpack_bf16x2(u.w);
+    v[q * 8 + 0] = a.x; v[q * 8 + 1] = a.y; v[q * 8 + 2] = b.x; v[q * 8 + 3] = b.y;
+    v[q * 8 + 4] = c.x; v[q * 8 + 5] = c.y; v[q * 8 + 6] = d.x; v[q * 8 + 7] = d.y;
+  }
+}
+__device__ __forceinline__ void stage_write(uint32_t tile, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    st_shared_v4(sw64(tile, r, q), make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]),
+                                              pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
+                                              pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]),
+                                              pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7])));
+}
+
+// Staged inputs per chunk: Z's gate and up halves (dSwiGLU), Z (dGELU), the
+// residual (plain store with aux), or none.
+__device__ __forceinline__ int epi_inputs(const GemmParams& p, const GroupArgs& ga) {
+  if (p.epi == tpi::EPI_DSWIGLU) return 2;
+  if (p.epi == tpi::EPI_DGELU) return 1;
+  if (p.epi == tpi::EPI_STORE) return ga.aux ? 1 : 0;
+  return 0;  // the forward activations stage outputs only
+}
+
+// Per-warp state of the TMA epilogue (lane 0 issues every copy).
+struct EpiStage {
+  uint8_t* buf;   // kEpiBuf bytes: tiles 0 and 1
+  uint64_t* bar;  // completes the staged inputs of a chunk
+  uint32_t phase;
+  int slot;       // plain stores alternate between the two tiles
+};
+
+// Lane 0: load chunk j0's inputs into the stage (the tiles are free once this
+// thread's earlier stores have read them).
+__device__ __forceinline__ void epi_issue_inputs(const GemmParams& p, int gi, int nin, int j0, int row0,
+                                                 EpiStage& es) {
+  const bool plain = p.epi == tpi::EPI_STORE;
+  uint8_t* t = es.buf + (plain ? es.slot * kEpiTile : 0);
+  // plain stores alternate tiles: the store two chunks back must have read this one
+  if (plain) bulk_wait_read<1>();
+  else bulk_wait_read<0>();
+  mbar_arrive_expect_tx(es.bar, static_cast<uint32_t>(nin * kEpiTile));
+  tma_load_3d(t, &p.tmX[gi], es.bar, j0, 0, row0);
+  if (nin == 2) tma_load_3d(t + kEpiTile, &p.tmX[gi], es.bar, j0, 1, row0);
+}
+
+// Forward activation epilogues through the stage (nothing staged in): SwiGLU
+// stores Z = [g | u] (when requested, through tmE) and H = SiLU(g) u (tmX);
+// bias + GELU stores Z (when requested, tmE) and H = GELU(Z) (tmX).
+__device__ void epilogue_fwd_tma(const GemmParams& p, const GroupArgs& ga, int gi, uint32_t taddr, int row0,
+                                 int n0, int half, bool narrow, int lane, EpiStage& es) {
+  uint8_t* t = es.buf;
+  const uint32_t t0 = smem_u32(t), t1 = t0 + kEpiTile;
+  if (p.epi == tpi::EPI_SWIGLU) {
+    // accumulator columns [0, 128) = gate units n0.., [128, 256) = the same up
+    // units; this warp takes units [half * 64, half * 64 + 64)
+#pragma unroll 1
+    for (int c = half * 2; c < half * 2 + 2; ++c) {
+      const int j0 = n0 + c * 32;
+      if (j0 >= ga.N) break;  // warp-uniform
+      float g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tc_wait_ld();
+      if (lane == 0) bulk_wait_read<0>();  // the last chunk's stores have read both tiles
+      __syncwarp();
+      if (ga.D) {
+        stage_write(t0, lane, g);
+        stage_write(t1, lane, u);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&p.tmE[gi], t, j0, 0, row0);
+          bulk_commit();
+          tma_store_3d(&p.tmE[gi], t + kEpiTile, j0, 1, row0);
+          bulk_commit();
+          bulk_wait_read<1>();  // tile 0 has been read
+        }
+        __syncwarp();
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = g[i] * sigmoid_fast(g[i]) * u[i];
+      stage_write(t0, lane, g);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&p.tmX[gi], t, j0, 0, row0);
+        bulk_commit();
+      }
+    }
+    return;
+  }
+  // bias + GELU: Z to tile 0, H to tile 1
+  const int cpw = narrow ? BN / 128 : BN / 64;
+#pragma unroll 1
+  for (int c = half * cpw; c < (half + 1) * cpw; ++c) {
+    const int j0 = n0 + c * 32;
+    if (j0 >= ga.N) break;  // warp-uniform
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tc_wait_ld();
+    if (ga.bias) {
+      float bb[32];
+      load_row_chunk_bf16(ga.bias, 0, 0, j0, ga.N, bb);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += bb[i];
+    }
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+    if (ga.D) stage_write(t0, lane, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+    stage_write(t1, lane, v);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (ga.D) tma_store_3d(&p.tmE[gi], t, j0, 0, row0);
+      tma_store_3d(&p.tmX[gi], t + kEpiTile, j0, 0, row0);
+      bulk_commit();
+    }
+  }
+}
+
+// The tile's epilogue through the stage; `pre`: the first chunk's inputs are
+// already in flight. Returns false if a bounded wait gave up.
+__device__ bool epilogue_tile_tma(const GemmParams& p, const GroupArgs& ga, int gi, uint32_t taddr, int row0,
+                                  int n0, int half, bool narrow, bool pre, int lane, EpiStage& es,
+                                  volatile int* abort, unsigned* status) {
+  const int cpw = narrow ? BN / 128 : BN / 64;  // 32-column chunks per warp half
+  const int nin = epi_inputs(p, ga);
+  const bool plain = p.epi == tpi::EPI_STORE;
+  bool first = true;
+#pragma unroll 1
+  for (int c = half * cpw; c < (half + 1) * cpw; ++c) {
+    const int j0 = n0 + c * 32;
+    if (j0 >= ga.N) break;  // warp-uniform
+    uint8_t* t = es.buf + (plain ? es.slot * kEpiTile : 0);
+    if (lane == 0) {
+      if (nin > 0) {
+        if (!(first && pre)) epi_issue_inputs(p, gi, nin, j0, row0, es);
+      } else {
+        bulk_wait_read<1>();  // the store issued from this tile two chunks ago has read it
+      }
+    }
+    __syncwarp();  // the tile is free before any lane writes it
+    first = false;
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tc_wait_ld();
+    if (nin > 0) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(es.bar, es.phase, abort, status));
+      es.phase ^= 1u;
+      if (!ok) {
+        if (lane == 0) {  // let the copies in flight land before the CTA may exit (bounded)
+          volatile int none = 0;
+          mbar_wait(es.bar, es.phase ^ 1u, &none, nullptr, 1000000ull);
+        }
+        return false;
+      }
+    }
+    const uint32_t t0 = smem_u32(t), t1 = t0 + kEpiTile;
+    switch (p.epi) {
+      case tpi::EPI_DSWIGLU: {
+        float zg[32], zu[32];
+        stage_read(t0, lane, zg);
+        stage_read(t1, lane, zu);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          // one sigmoid per element: SiLU(g) = g s, SiLU'(g) = s (1 + g (1 - s))
+          const float sg = sigmoid_fast(zg[i]);
+          const float dg = v[i] * zu[i] * (sg * (1.0f + zg[i] * (1.0f - sg)));
+          zu[i] = v[i] * (zg[i] * sg);
+          zg[i] = dg;
+        }
+        stage_write(t0, lane, zg);
+        stage_write(t1, lane, zu);
+        break;
+      }
+      case tpi::EPI_DGELU: {
+        float z[32];
+        stage_read(t0, lane, z);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= gelu_grad_f(z[i]);
+        stage_write(t0, lane, v);
+        break;
+      }
+      default: {  // plain store: + bias, + residual
+        if (ga.bias) {
+          float bb[32];
+          load_row_chunk_bf16(ga.bias, 0, 0, j0, ga.N, bb);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += bb[i];
+        }
+        if (nin > 0) {
+          float r[32];
+          stage_read(t0, lane, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += r[i];
+        }
+        stage_write(t0, lane, v);
+        break;
+      }
+    }
+    fence_proxy_async_smem();  // this lane's writes are visible to the TMA store
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(&p.tmE[gi], t, j0, 0, row0);
+      if (nin == 2) tma_store_3d(&p.tmE[gi], t + kEpiTile, j0, 1, row0);
+      bulk_commit();
+    }
+    if (plain) es.slot ^= 1;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------ tile ring
 // The persistent CTAs take tiles in order from one atomic counter, so the
 // tiles in flight at any moment are a window of consecutive indices (the
@@ -392,7 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint8_t* sE = smem + STAGES * C::STAGE_BYTES;  // TMA epilogue stages, kEpiBuf per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -403,6 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
   ring.full = drain + 2;
   ring.empty = ring.full + kRing;
   ring.slot = reinterpret_cast<volatile int*>(ring.empty + kRing);
+  uint64_t* ebar = reinterpret_cast<uint64_t*>(const_cast<int*>(ring.slot) + kRing);  // [kEpiWarps]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -422,6 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       mbar_init(&ring.full[r], 1);
       mbar_init(&ring.empty[r], PAIR * kRingConsumers);
     }
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&ebar[w], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -430,6 +677,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     for (int g = 0; g < nmaps; ++g) {
       tma_prefetch_desc(&p.tmA[g]);
       tma_prefetch_desc(&p.tmB[g]);
+    }
+    if (p.tma_epi) {
+      const bool fwd = p.epi == tpi::EPI_SWIGLU || p.epi == tpi::EPI_BIAS_GELU;
+      for (int g = 0; g < p.ngroups; ++g) {  // only the views the launch encoded
+        if (!fwd || p.g[g].D) tma_prefetch_desc(&p.tmE[g]);
+        if (fwd || epi_inputs(p, p.g[g]) > 0) tma_prefetch_desc(&p.tmX[g]);
+      }
     }
   }
   if (warp == 1) {
@@ -495,10 +749,13 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int n0 = nt * p.tile_n;
       // this CTA's B rows (in a narrow tile of a pair, each CTA's first BN / 4)
       const int nb0 = n0 + static_cast<int>(rank) * (narrow_tile(p, ga, n0) ? BN / (2 * PAIR) : C::B_ROWS);
-      // A narrow launch loads only the B rows its MMAs read (half a B stage);
-      // a ragged narrow tile of a full-width launch loads the full stage.
-      const uint32_t b_bytes = p.narrow_all ? C::B_BYTES / 2 : C::B_BYTES;
-      const int b_blocks = (p.narrow_all ? C::B_ROWS / 2 : C::B_ROWS) / 64;  // MN-major 64-column blocks
+      // A narrow tile loads only the B rows its MMAs read (half a B stage):
+      // always for MN-major B (64-column blocks, one copy each); for K-major
+      // B only in a narrow launch, whose tensor map has the half-height box
+      // (a ragged narrow tile of a full-width launch loads the full box).
+      const bool half_b = p.narrow_all || (p.b_mn && narrow_tile(p, ga, n0));
+      const uint32_t b_bytes = half_b ? C::B_BYTES / 2 : C::B_BYTES;
+      const int b_blocks = (half_b ? C::B_ROWS / 2 : C::B_ROWS) / 64;  // MN-major 64-column blocks
       const int nseg = p.kcat ? p.kcat : 1;
       for (int sg = 0; sg < nseg && ok; ++sg) {
         const int gi = p.kcat ? sg : g;  // tensor maps of this K segment
@@ -640,20 +897,40 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
     int acc = 0;
     uint32_t acc_phase = 0;
     const uint32_t tempty_leader = PAIR == 2 ? map_shared(smem_u32(&tempty[0]), 0) : 0u;
+    EpiStage es{sE + (warp - 2) * kEpiBuf, &ebar[warp - 2], 0u, 0};
+    bool ok = true;
     for (int kseq = 0;; ++kseq) {
       const int t = ring_take_warp<PAIR>(ring, kseq, rank, lane, abort_flag, p.status);
       if (t < 0) break;
       int g, mt, nt, ks;
       decode_tile(p, t, g, mt, nt, ks);
       const GroupArgs& ga = p.g[g];
-      // warp-uniform: the epilogue's tcgen05.ld is warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) break;
-      tc_fence_after();
-      const int row = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32 + lane;
+      const int row0 = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32;
       const int n0 = nt * p.tile_n;
+      const bool narrow = narrow_tile(p, ga, n0);
+      // TMA epilogue: the first chunk's inputs load while the MMAs finish
+      const int gi = p.kcat ? 0 : g;
+      const bool pre = p.tma_epi && epi_inputs(p, ga) > 0 && n0 + half * (narrow ? BN / 4 : BN / 2) < ga.N;
+      if (pre && lane == 0) epi_issue_inputs(p, gi, epi_inputs(p, ga), n0 + half * (narrow ? BN / 4 : BN / 2), row0, es);
+      // warp-uniform: the epilogue's tcgen05.ld is warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) {
+        if (pre && lane == 0) {  // the prefetched copies land before the CTA may exit (bounded)
+          volatile int none = 0;
+          mbar_wait(es.bar, es.phase, &none, nullptr, 1000000ull);
+        }
+        break;
+      }
+      tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      epilogue_tile(p, ga, taddr, row, n0, half, narrow_tile(p, ga, n0), ks);
+      if (p.tma_epi && (p.epi == tpi::EPI_SWIGLU || p.epi == tpi::EPI_BIAS_GELU)) {
+        epilogue_fwd_tma(p, ga, gi, taddr, row0, n0, half, narrow, lane, es);
+      } else if (p.tma_epi) {
+        ok = epilogue_tile_tma(p, ga, gi, taddr, row0, n0, half, narrow, pre, lane, es, abort_flag, p.status);
+      } else {
+        epilogue_tile(p, ga, taddr, row0 + lane, n0, half, narrow, ks);
+      }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -663,6 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (p.tma_epi && lane == 0) bulk_wait_all();  // every store of this warp has landed
   }
 
   tc_fence_before();
@@ -706,6 +984,45 @@ tp_status encode_gateup(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return tpi::fail(TP_ERR_CUDA, "cuTensorMapEncodeTiled(3d gate/up) failed: %d", (int)r);
   return TP_OK;
+}
+
+// {cols, halves, rows} view of a bf16 epilogue output or staged input with a
+// {32, 1, 32} box and 64-byte swizzle (the TMA epilogue's staging tiles).
+// halves = 2 views [gate | up] of width cols = nh at a column offset of nh.
+tp_status encode_epi(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t halves,
+                     uint64_t half_stride, uint64_t rows, int64_t ld) {
+  cuuint64_t dims[3] = {cols, halves, rows};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(half_stride) * 2, static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[3] = {32, 1, 32};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TP_OK : TP_ERR_CUDA;
+}
+
+// The TMA epilogue serves bf16 outputs of the plain, dGELU and dSwiGLU
+// epilogues without row scatter or split K, on 16-byte aligned outputs and
+// inputs (and, for dSwiGLU, halves of a multiple of 8 columns).
+// TP_GEMM_TMA_EPI=0 keeps every launch on the direct epilogue.
+bool tma_epilogue_ok(const GemmBatch& b, int nout, int ksplit) {
+  const char* e = getenv("TP_GEMM_TMA_EPI");
+  if (e && e[0] == '0') return false;
+  if (b.out_f32 || ksplit > 1 || b.scatter_n > 0) return false;
+  const bool fwd = b.epi == tpi::EPI_SWIGLU || b.epi == tpi::EPI_BIAS_GELU;
+  const bool bwd = b.epi == tpi::EPI_DGELU || b.epi == tpi::EPI_DSWIGLU;
+  if (!fwd && !bwd && b.epi != tpi::EPI_STORE) return false;
+  const bool halves = b.epi == tpi::EPI_SWIGLU || b.epi == tpi::EPI_DSWIGLU;
+  for (int i = 0; i < nout; ++i) {
+    const GemmProblem& o = b.g[i];
+    const void* out = fwd ? o.D2 : o.D;  // the output every tile writes
+    if (!out || reinterpret_cast<uintptr_t>(out) % 16) return false;
+    if (fwd && o.D && reinterpret_cast<uintptr_t>(o.D) % 16) return false;
+    if (bwd && !o.aux) return false;
+    if (!fwd && o.aux && reinterpret_cast<uintptr_t>(o.aux) % 16) return false;
+    if (halves && (o.nh % 8 || o.N != o.nh)) return false;
+  }
+  return true;
 }
 
 // CTA pairing forced by the environment variable TP_GEMM_CTA_PAIR ("1": one
@@ -980,6 +1297,23 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     p.kb_per_split = kbps;
     p.split_stride = b.split_stride;
     tiles *= ksplit;
+  }
+  if (tma_epilogue_ok(b, nout, ksplit)) {
+    p.tma_epi = 1;
+    const bool sw = b.epi == tpi::EPI_DSWIGLU || b.epi == tpi::EPI_SWIGLU;
+    const bool fwd = b.epi == tpi::EPI_SWIGLU || b.epi == tpi::EPI_BIAS_GELU;
+    const uint64_t halves = sw ? 2 : 1;
+    for (int i = 0; i < nout && p.tma_epi; ++i) {
+      const GemmProblem& o = b.g[i];
+      bool good = true;
+      // tmE: D (Z in the forward activations, where it may be absent)
+      if (o.D) good = encode_epi(enc, &p.tmE[i], o.D, o.N, halves, sw ? o.nh : o.ldd, o.M, o.ldd) == TP_OK;
+      // tmX: H (forward activations) or the staged input
+      if (good && fwd) good = encode_epi(enc, &p.tmX[i], o.D2, o.N, 1, o.ldd2, o.M, o.ldd2) == TP_OK;
+      else if (good && o.aux)
+        good = encode_epi(enc, &p.tmX[i], o.aux, o.N, halves, sw ? o.nh : o.ldaux, o.M, o.ldaux) == TP_OK;
+      if (!good) p.tma_epi = 0;  // a view the encoder refuses: the direct epilogue serves
+    }
   }
   p.ngroups = nout;
   p.total_tiles = tiles;
