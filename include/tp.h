@@ -413,7 +413,11 @@ TP_API tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void*
                            const float* const* LSE, void* const* dQKV, void* stream);
 
 /* Column sums over rows: out[c] = sum_r x[r, c] in fp32 (fixed order;
- * accumulate != 0 adds to out). x [rows, cols] in the plan dtype. */
+ * accumulate != 0 adds to out). x [rows, cols] in the plan dtype. One launch:
+ * blocks sum row splits into the plan's workspace and the last block of each
+ * column slab adds the splits in order. The plan's first reduction on a
+ * device allocates its workspace and arrival counters, so it must not be the
+ * first call inside a stream capture (TP_ERR_ARG). */
 TP_API tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const void* x, float* out,
                         int accumulate, void* stream);
 

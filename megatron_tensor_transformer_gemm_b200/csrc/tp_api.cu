@@ -160,6 +160,42 @@ tp_status workspace(tp_plan* plan, size_t bytes, void** out) {
   return TP_OK;
 }
 
+tp_status plan_counters(tp_plan* plan, cudaStream_t st, unsigned** out) {
+  int dev = 0;
+  tp_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != TP_OK) return s;
+  if (plan->cnt && plan->cnt_device == dev) {
+    *out = plan->cnt;
+    return TP_OK;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return fail(TP_ERR_ARG, "the plan's first reduction on a device must run before a stream capture");
+  }
+  if (plan->cnt) {  // moved to another device
+    cudaDeviceSynchronize();
+    cudaSetDevice(plan->cnt_device);
+    cudaFree(plan->cnt);
+    cudaSetDevice(dev);
+    plan->cnt = nullptr;
+  }
+  void* p = nullptr;
+  s = cuda_status(cudaMalloc(&p, kPlanCounters * sizeof(unsigned)), "cudaMalloc(counters)");
+  if (s != TP_OK) return s;
+  // zero, and finished, before any kernel on any stream can use them
+  s = cuda_status(cudaMemsetAsync(p, 0, kPlanCounters * sizeof(unsigned), st), "cudaMemsetAsync(counters)");
+  if (s == TP_OK) s = cuda_status(cudaStreamSynchronize(st), "cudaStreamSynchronize(counters)");
+  if (s != TP_OK) {
+    cudaFree(p);
+    return s;
+  }
+  plan->cnt = static_cast<unsigned*>(p);
+  plan->cnt_device = dev;
+  *out = plan->cnt;
+  return TP_OK;
+}
+
 tp_status check_ptr(const void* p, const char* name) {
   if (!p) return fail(TP_ERR_ARG, "%s is NULL", name);
   if (!aligned16(p)) return fail(TP_ERR_ALIGN, "%s (%p) is not 16-byte aligned", name, p);
@@ -367,21 +403,28 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   plan->ws = nullptr;
   plan->ws_bytes = 0;
   plan->ws_device = -1;
+  plan->cnt = nullptr;
+  plan->cnt_device = -1;
   *out = plan;
   return TP_OK;
 }
 
 void tp_plan_destroy(tp_plan* plan) {
   if (!plan) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
   if (plan->ws) {
-    int cur = 0;
-    cudaGetDevice(&cur);
     cudaSetDevice(plan->ws_device);
     cudaDeviceSynchronize();
     cudaFree(plan->ws);
-    cudaSetDevice(cur);
-    cudaGetLastError();
   }
+  if (plan->cnt) {
+    cudaSetDevice(plan->cnt_device);
+    cudaDeviceSynchronize();
+    cudaFree(plan->cnt);
+  }
+  cudaSetDevice(cur);
+  cudaGetLastError();
   delete plan;
 }
 

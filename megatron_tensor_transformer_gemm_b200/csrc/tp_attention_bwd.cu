@@ -4,7 +4,7 @@
 //   dV = P^T dO;  dP = dO V^T;  dS = P * (dP - D),  D = rowsum(dO * O)
 //   dQ = dS K / sqrt(d);  dK = dS^T Q / sqrt(d)
 // Three launches, deterministic (no atomics):
-//   attn_bwd_prep     D and lse * log2(e) for every query row (one warp per row)
+//   attn_bwd_prep     D and lse * log2(e) for every query row (d / 8 threads per row)
 //   attn_bwd_dkdv_st  one CTA per 128-key block, keys as the MMA rows: loops
 //                     over the 64-query sub-tiles that see it, S^T and dP^T in
 //                     TMEM (two sub-tiles in flight), P^T and dS^T written to
@@ -91,34 +91,44 @@ __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, __nv_bfloat16
 
 // D[row] = sum_c dO[row, c] * O[row, c] for every (shard, b, head, q), and
 // lse2[row] = lse[row] * log2(e); both into [batch * hl][seq_pad] arrays.
+// A row is G = d / 8 threads, each loading 16 bytes of O and of dO; the G
+// products are summed by shuffles in a fixed order.
+template <int G>
 __global__ void attn_bwd_prep(const __grid_constant__ PtrArray O, const __grid_constant__ PtrArray dO,
                               const __grid_constant__ PtrArray LSE, const __grid_constant__ MutPtrArray dvec,
                               const __grid_constant__ MutPtrArray lse2, int p, int batch, int seq,
-                              int seq_pad, int hl, int d) {
+                              int seq_pad, int hl) {
   tpd::pdl_entry();
+  constexpr int d = 8 * G;
   const int64_t rows_per_shard = static_cast<int64_t>(batch) * hl * seq;
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows_per_shard * p) return;
-  const int shard = static_cast<int>(row / rows_per_shard);
-  int64_t rest = row - shard * rows_per_shard;
-  const int q = static_cast<int>(rest % seq);
-  rest /= seq;
-  const int hh = static_cast<int>(rest % hl);
-  const int b = static_cast<int>(rest / hl);
-  const int64_t off = (static_cast<int64_t>(q) * batch + b) * hl * d + static_cast<int64_t>(hh) * d;
-  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(O.p[shard]) + off;
-  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(dO.p[shard]) + off;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = t / G;
+  const int part = static_cast<int>(t % G);
+  const bool live = row < rows_per_shard * p;  // whole groups share one row
   float s = 0.f;
-  for (int c = lane * 2; c < d; c += 64) {
-    const float2 a = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(o + c));
-    const float2 bb = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(g + c));
-    s += a.x * bb.x + a.y * bb.y;
+  int shard = 0, q = 0;
+  int64_t bh = 0;
+  if (live) {
+    shard = static_cast<int>(row / rows_per_shard);
+    int64_t rest = row - shard * rows_per_shard;
+    q = static_cast<int>(rest % seq);
+    rest /= seq;
+    const int hh = static_cast<int>(rest % hl);
+    const int b = static_cast<int>(rest / hl);
+    bh = static_cast<int64_t>(b) * hl + hh;
+    const int64_t off = (static_cast<int64_t>(q) * batch + b) * hl * d + static_cast<int64_t>(hh) * d + part * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(O.p[shard]) + off);
+    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dO.p[shard]) + off);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x = unpack_bf16x2(av[k]), y = unpack_bf16x2(gv[k]);
+      s += x.x * y.x + x.y * y.y;
+    }
   }
 #pragma unroll
-  for (int k = 16; k > 0; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
-  if (lane == 0) {
-    const int64_t bh = static_cast<int64_t>(b) * hl + hh;
+  for (int k = G / 2; k > 0; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k, G);
+  if (live && part == 0) {
     static_cast<float*>(dvec.p[shard])[bh * seq_pad + q] = s;
     static_cast<float*>(lse2.p[shard])[bh * seq_pad + q] = static_cast<const float*>(LSE.p[shard])[bh * seq + q] * kLog2e;
   }
@@ -670,8 +680,14 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   const int64_t warps = rows_per_shard * p;
   if (warps * 32 / 256 + 1 > 0x7fffffffLL || static_cast<int64_t>(prm.nq) * p * batch * hl > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "attention backward grid too large");
-  (void)tpi::launch(attn_bwd_prep, dim3(static_cast<unsigned>((warps * 32 + 255) / 256)), dim3(256), 0, st, o, dO, lse_in, dvec, lse2, p,
-                                                                                 batch, seq, seq_pad, hl, d);
+  const int G = d / 8;  // threads per row
+  const unsigned pblocks = static_cast<unsigned>((rows_per_shard * p * G + 255) / 256);
+  if (d == 64)
+    (void)tpi::launch(attn_bwd_prep<8>, dim3(pblocks), dim3(256), 0, st, o, dO, lse_in, dvec, lse2, p, batch, seq,
+                      seq_pad, hl);
+  else
+    (void)tpi::launch(attn_bwd_prep<16>, dim3(pblocks), dim3(256), 0, st, o, dO, lse_in, dvec, lse2, p, batch, seq,
+                      seq_pad, hl);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;
   if (d == 64) return launch_bwd_d<64, 4, 2>(prm, st);

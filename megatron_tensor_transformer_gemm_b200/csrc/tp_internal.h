@@ -23,6 +23,10 @@ struct tp_plan {
   void* ws;
   size_t ws_bytes;
   int ws_device;
+  // Arrival counters of single-launch reductions (zero at rest: the last
+  // block of each reduction sets its counter back), allocated on first need.
+  unsigned* cnt;
+  int cnt_device;
 };
 
 namespace tpi {
@@ -73,6 +77,11 @@ tp_status persistent_grid(const void* kernel, int threads, int smem, int64_t uni
 tp_status device_status_word(unsigned** out);
 // Scratch of at least `bytes` on the current device, owned by the plan.
 tp_status workspace(tp_plan* plan, size_t bytes, void** out);
+// The plan's kPlanCounters arrival counters on the current device (zero at
+// rest). The first call on a device allocates and zeroes them (not allowed
+// while `st` is being captured).
+constexpr int kPlanCounters = 4096;
+tp_status plan_counters(tp_plan* plan, cudaStream_t st, unsigned** out);
 
 // Validation helpers: each returns TP_OK or records an error.
 tp_status check_ptr(const void* p, const char* name);

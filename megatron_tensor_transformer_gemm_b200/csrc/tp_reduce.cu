@@ -324,6 +324,71 @@ __global__ void colsum_grouped_pass2(const float* part, int splits, int64_t cols
   o[c] = accumulate ? o[c] + sum : sum;
 }
 
+// Column sums of n same-shape inputs in one launch: every block sums its split
+// of rows for 32*V columns of input blockIdx.z into part (as pass 1 above),
+// and the last block to finish a (column slab, input) pair, counted on
+// counters[z * gridDim.x + x], adds that slab's partials over the splits in
+// split order and writes out.p[z] (so the sums are deterministic), then sets
+// its counter back to zero.
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_fused(const __grid_constant__ PtrArray X, int64_t ld,
+                                                    int64_t rows, int64_t vpr, int64_t rows_per_split,
+                                                    float* part, int64_t cols,
+                                                    const __grid_constant__ MutPtrArray out,
+                                                    int accumulate, unsigned* counters) {
+  tpd::pdl_entry();
+  constexpr int V = Vec<T>::N;
+  __shared__ float red[8][32 * V + 1];
+  __shared__ int last;
+  const int splits = static_cast<int>(gridDim.y);
+  const T* x = static_cast<const T*>(X.p[blockIdx.z]);
+  float* pz = part + static_cast<int64_t>(blockIdx.z) * splits * cols;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + tx;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(rows, r0 + rows_per_split);
+  float acc[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) acc[k] = 0.f;
+  if (cv < vpr) {
+    for (int64_t r = r0 + ty; r < r1; r += 8) {
+      float f[V];
+      Vec<T>::load(ld_stream(x + r * ld + cv * V), f);
+#pragma unroll
+      for (int k = 0; k < V; ++k) acc[k] += f[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < V; ++k) red[ty][tx * V + k] = acc[k];
+  __syncthreads();
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 32 * V;
+  for (int c = threadIdx.x; c < 32 * V; c += 256) {
+    float sum = 0.f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) sum += red[y][c];
+    if (col0 + c < cols) pz[static_cast<int64_t>(blockIdx.y) * cols + col0 + c] = sum;
+  }
+  __threadfence();  // this block's partials are visible before it is counted
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned* ctr = counters + static_cast<int64_t>(blockIdx.z) * gridDim.x + blockIdx.x;
+    last = atomicAdd(ctr, 1u) == static_cast<unsigned>(splits - 1);
+    if (last) atomicExch(ctr, 0u);  // no other block of this slab counts again
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  float* o = static_cast<float*>(out.p[blockIdx.z]);
+  for (int c = threadIdx.x; c < 32 * V; c += 256) {
+    const int64_t col = col0 + c;
+    if (col >= cols) continue;
+    float sum = 0.f;
+#pragma unroll 16
+    for (int k = 0; k < splits; ++k) sum += __ldcg(pz + static_cast<int64_t>(k) * cols + col);
+    o[col] = accumulate ? o[col] + sum : sum;
+  }
+}
+
 // Block shape for row-walking kernels: x covers column vectors, y rows.
 void row_walk_shape(int64_t vpr, int64_t rows, dim3* grid, dim3* block) {
   int bx = static_cast<int>(std::min<int64_t>(kThreads, ((vpr + 31) / 32) * 32));
@@ -413,6 +478,13 @@ tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_
 
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
                             float* out, int accumulate, tp_dtype dt, cudaStream_t st) {
+  if (rows > 0) {  // one launch: the grouped form with one input
+    PtrArray X{};
+    MutPtrArray O{};
+    X.p[0] = x;
+    O.p[0] = out;
+    return launch_column_sum_grouped(plan, X, 1, rows, cols, ld, O, accumulate, dt, st);
+  }
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   const int gx = static_cast<int>((vpr + 31) / 32);
@@ -459,6 +531,20 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
   tp_status s = workspace(plan, static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float), &ws);
   if (s != TP_OK) return s;
   float* part = static_cast<float*>(ws);
+  if (rows > 0 && static_cast<int64_t>(gx) * n <= kPlanCounters) {
+    // one launch: the last block of each column slab finishes it
+    unsigned* ctr = nullptr;
+    s = plan_counters(plan, st, &ctr);
+    if (s != TP_OK) return s;
+    dim3 grid(gx, static_cast<unsigned>(splits), static_cast<unsigned>(n));
+    if (dt == TP_BF16)
+      (void)tpi::launch(colsum_fused<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, ld, rows, vpr, rps, part, cols,
+                        out, accumulate, ctr);
+    else
+      (void)tpi::launch(colsum_fused<float>, dim3(grid), dim3(256), 0, st, x, ld, rows, vpr, rps, part, cols, out,
+                        accumulate, ctr);
+    return after_launch("column_sum_grouped");
+  }
   if (rows > 0) {
     dim3 grid(gx, static_cast<unsigned>(splits), static_cast<unsigned>(n));
     if (dt == TP_BF16)

@@ -152,6 +152,45 @@ def test_column_sum(rows, cols):
     assert_bitexact(out, 2 * O.bias_grad(O.f64(x)), "column sum accumulate")
 
 
+def test_column_sum_one_launch_rearms_its_counters():
+    """The single-launch column sum counts each column slab's finished blocks
+    on the plan's counters, and the last block sets its counter back: many
+    sums of changing shapes on one plan (eager and replayed from a CUDA graph)
+    must each be exact. Integer inputs make every order give the same sum."""
+    tp = _tp()
+    plan = tp.Plan(8, 0, 0, 1, "bf16", "none")
+    shapes = [(4096, 512), (37, 8), (4096, 1536), (1000, 136), (64, 4096), (5000, 2048)]
+    for rep in range(3):
+        for rows, cols in shapes:
+            g = torch.Generator().manual_seed(rows * 7 + cols + rep)
+            x = torch.randint(-4, 5, (rows, cols), generator=g).to(torch.bfloat16)
+            out = torch.empty(cols, dtype=torch.float32, device="cuda")
+            plan.column_sum(rows, cols, dev(x), out)
+            assert_bitexact(out, O.bias_grad(O.f64(x)), f"column sum {rows}x{cols} rep {rep}")
+    rows, cols = 4096, 1536
+    g = torch.Generator().manual_seed(99)
+    x = dev(torch.randint(-4, 5, (rows, cols), generator=g).to(torch.bfloat16))
+    out = torch.zeros(cols, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        plan.column_sum(rows, cols, x, out, stream=s)  # first use on this stream, before capture
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            plan.column_sum(rows, cols, x, out, accumulate=True, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(4):
+        gr.replay()
+    torch.cuda.synchronize()
+    assert_bitexact(out, 5 * O.bias_grad(O.f64(host(x))), "column sum replayed")
+    # fp32 inputs take the same kernel
+    xf = torch.randint(-9, 10, (3000, 264), generator=g).to(torch.float32)
+    plan32 = tp.Plan(8, 0, 0, 1, "f32", "none")
+    outf = torch.empty(264, dtype=torch.float32, device="cuda")
+    plan32.column_sum(3000, 264, dev(xf), outf)
+    assert_bitexact(outf, O.bias_grad(O.f64(xf)), "column sum fp32")
+
+
 @pytest.mark.parametrize("h", [512, 4096, 8192, 136, 16384])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_layernorm_fwd_bwd(h, dtype):
