@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <tuple>
 #include <new>
@@ -296,6 +297,84 @@ MutPtrArray to_marr(void* const* a, int n) {
   for (int i = 0; i < n && a; ++i) r.p[i] = a[i];
   return r;
 }
+
+// A backward call's activation-gradient GEMM (dX or dH) and its weight
+// gradient read the same inputs and write different outputs. When either
+// leaves SMs idle (small problems: a few tiles per launch), the activation
+// gradient runs on a side stream of the device beside the weight gradient:
+// fork (the side stream waits for the caller's stream), the GEMM on the side
+// stream, then the caller's stream waits for it before the call returns. The
+// side GEMM uses no workspace (the weight gradient's split-K partials and the
+// bias sums do, on the caller's stream). Works inside stream capture (the
+// fork and join become graph edges). TP_BWD_CONCURRENT=0 keeps one stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+tp_status side_stream(SideStream** out) {
+  constexpr int kMaxDev = 64;
+  static SideStream side[kMaxDev];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return fail(TP_ERR_NO_DEVICE, "no current CUDA device");
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  SideStream& sd = side[dev];
+  if (!sd.s) {
+    SideStream n;
+    tp_status r = cuda_status(cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking), "cudaStreamCreate(side)");
+    if (r == TP_OK) r = cuda_status(cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming), "cudaEventCreate(fork)");
+    if (r == TP_OK) r = cuda_status(cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming), "cudaEventCreate(join)");
+    if (r != TP_OK) {
+      if (n.join) cudaEventDestroy(n.join);
+      if (n.fork) cudaEventDestroy(n.fork);
+      if (n.s) cudaStreamDestroy(n.s);
+      return r;
+    }
+    sd = n;
+  }
+  *out = &sd;
+  return TP_OK;
+}
+
+bool concurrent_bwd(const tp_plan* plan, const GemmBatch& act_grad, const GemmBatch& wgrad) {
+  if (plan->dtype != TP_BF16) return false;
+  const char* e = getenv("TP_BWD_CONCURRENT");
+  if (e && e[0] == '0') return false;
+  return !gemm_fills_gpu(act_grad) || !gemm_fills_gpu(wgrad);
+}
+
+// Runs `act_grad` on the side stream (forked from st) and, when it goes out
+// of scope, makes st wait for it: every return path of the call joins.
+class SideGemm {
+ public:
+  SideGemm(const tp_plan* plan, const GemmBatch& act_grad, cudaStream_t st) : st_(st) {
+    status_ = side_stream(&sd_);
+    if (status_ != TP_OK) return;
+    status_ = cuda_status(cudaEventRecord(sd_->fork, st), "cudaEventRecord(fork)");
+    if (status_ == TP_OK) status_ = cuda_status(cudaStreamWaitEvent(sd_->s, sd_->fork, 0), "cudaStreamWaitEvent(fork)");
+    if (status_ != TP_OK) {
+      sd_ = nullptr;
+      return;
+    }
+    status_ = plan->dtype == TP_BF16 ? launch_gemm_bf16(act_grad, sd_->s) : launch_gemm_f32(act_grad, sd_->s);
+    const tp_status r = cuda_status(cudaEventRecord(sd_->join, sd_->s), "cudaEventRecord(join)");
+    if (status_ == TP_OK) status_ = r;
+    if (r != TP_OK) sd_ = nullptr;
+  }
+  ~SideGemm() {
+    if (sd_) cudaStreamWaitEvent(st_, sd_->join, 0);
+  }
+  tp_status status() const { return status_; }
+
+ private:
+  SideStream* sd_ = nullptr;
+  cudaStream_t st_;
+  tp_status status_ = TP_OK;
+};
 
 // Launch grouped GEMMs in the plan dtype; fp32 takes EPI_STORE only.
 tp_status run_gemm(const tp_plan* plan, const GemmBatch& b, cudaStream_t st) {
@@ -1126,10 +1205,9 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
     g.nh = k;
   }
   b.epi = act == TP_ACT_GELU ? EPI_DGELU : act == TP_ACT_SWIGLU ? EPI_DSWIGLU : EPI_STORE;
-  TP_TRY(run_gemm(plan, b, st));
+  GemmBatch w{};
   if (dW) {
     // dW_i [h, k] = dY^T H_i: A(m, t) = dY[t, m] (MN-major), B(n, t) = H_i[t, n] (MN-major).
-    GemmBatch w{};
     w.n = p;
     w.a_mn = true;
     w.b_mn = true;
@@ -1147,8 +1225,16 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
       g.D = dW[i];
       g.ldd = k;
     }
-    TP_TRY(run_wgrad(plan, w, st));
   }
+  // dH beside the weight gradient (joined when this call returns), or before it
+  std::unique_ptr<SideGemm> side;
+  if (dW && concurrent_bwd(plan, b, w)) {
+    side.reset(new SideGemm(plan, b, st));
+    TP_TRY(side->status());
+  } else {
+    TP_TRY(run_gemm(plan, b, st));
+  }
+  if (dW) TP_TRY(run_wgrad(plan, w, st));
   if (dbias) TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, st));
   return TP_OK;
 }
@@ -1178,9 +1264,9 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
   if (mode == 0) TP_TRY(check_row_bytes(h, plan->partial_dtype, "hidden (dX partials)"));
   if (T == 0) return TP_OK;
+  GemmBatch w{};
   if (dW) {
     // dW_i [n, h] = dZ_i^T X: A(m, t) = dZ_i[t, m] (MN-major), B(c, t) = X[t, c] (MN-major).
-    GemmBatch w{};
     w.n = p;
     w.a_mn = true;
     w.b_mn = true;
@@ -1198,11 +1284,10 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
       g.D = dW[i];
       g.ldd = h;
     }
-    TP_TRY(run_wgrad(plan, w, st));
   }
+  GemmBatch d{};
   if (dX_out) {
     // dX_i [T, h] = dZ_i W_i: A = dZ_i (K-major), B(c, j) = W_i[j, c] (MN-major).
-    GemmBatch d{};
     d.n = p;
     d.a_mn = false;
     d.b_mn = true;
@@ -1226,8 +1311,15 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
       d.rows_per_out = T / p;
       for (int j = 0; j < p; ++j) d.out_seq[j] = dX_out[j];
     }
-    TP_TRY(run_gemm(plan, d, st));
   }
+  // dX beside the weight gradient (joined when this call returns), or after it
+  std::unique_ptr<SideGemm> side;
+  if (dW && dX_out && concurrent_bwd(plan, d, w)) {
+    side.reset(new SideGemm(plan, d, st));
+    TP_TRY(side->status());
+  }
+  if (dW) TP_TRY(run_wgrad(plan, w, st));
+  if (dX_out && !side) TP_TRY(run_gemm(plan, d, st));
   if (dbias)
     TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p),
                                      p, T, n, n, to_marr(reinterpret_cast<void* const*>(dbias), p), 0,

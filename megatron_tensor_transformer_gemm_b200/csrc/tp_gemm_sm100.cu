@@ -1334,6 +1334,18 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
   return launch_kernel<1>(p, tiles, sms, st);
 }
 
+bool gemm_fills_gpu(const GemmBatch& b) {
+  const int sms = device_sms();
+  const Layout lay = choose_layout(b, sms);
+  const bool swiglu = b.epi == EPI_SWIGLU;
+  const int tile_m = BM * lay.pair, tn = (swiglu || lay.narrow) ? BN / 2 : BN;
+  const int nout = b.kcat ? 1 : b.n;
+  int64_t tiles = 0;
+  for (int i = 0; i < nout; ++i)
+    tiles += static_cast<int64_t>((b.g[i].M + tile_m - 1) / tile_m) * ((b.g[i].N + tn - 1) / tn);
+  return tiles * (b.ksplit > 1 ? b.ksplit : 1) >= sms / lay.pair;
+}
+
 int gemm_split_k(const GemmBatch& b) {
   if (b.kcat || b.scatter_n || b.epi != EPI_STORE || b.n < 1) return 1;
   for (int i = 1; i < b.n; ++i)

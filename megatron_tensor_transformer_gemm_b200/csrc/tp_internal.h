@@ -201,6 +201,9 @@ struct GemmBatch {
 
 // bf16 tcgen05 tensor-core path (tp_gemm_sm100.cu).
 tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st);
+// Whether a bf16 launch of b has at least as many tiles as CTA units (pairs or
+// CTAs) on this device, i.e. leaves no SM idle in its first wave.
+bool gemm_fills_gpu(const GemmBatch& b);
 // The K split that minimises the estimated time of a batch of plain bf16-output
 // GEMMs of equal shape, counting the fp32 partials' reduce (1 = no split, <= 16).
 int gemm_split_k(const GemmBatch& b);

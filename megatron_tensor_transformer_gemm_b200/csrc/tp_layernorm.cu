@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(256) ln_bwd_param_pass1(const T* x, const T* d
 // order: deterministic). Lane 0..31 of warp 0 returns true with the column's
 // two sums.
 constexpr int kPass2Cols = 32;
+template <bool CG = false>  // CG: load through L2 only (partials other blocks of this launch wrote)
 __device__ __forceinline__ bool param_colsum_range(const float* part, int k0, int k1, int64_t cols,
                                                    int64_t c, float* sg_out, float* sb_out) {
   __shared__ float rg[8][32], rb[8][32];
@@ -266,8 +267,9 @@ __device__ __forceinline__ bool param_colsum_range(const float* part, int k0, in
   if (c < cols) {
 #pragma unroll 4
     for (int k = k0 + warp; k < k1; k += 8) {
-      sg += part[(static_cast<int64_t>(k) * 2 + 0) * cols + c];
-      sb += part[(static_cast<int64_t>(k) * 2 + 1) * cols + c];
+      const float* pg = part + (static_cast<int64_t>(k) * 2 + 0) * cols + c;
+      sg += CG ? __ldcg(pg) : *pg;
+      sb += CG ? __ldcg(pg + cols) : pg[cols];
     }
   }
   rg[warp][lane] = sg;
@@ -741,6 +743,44 @@ __global__ void __launch_bounds__(THREADS) norm_hsh_bwd_fused_kernel(
   }
 }
 
+// Groups and final sum in one launch: block (x, g) sums group g of the
+// partials for kPass2Cols columns into inter[g] (as param_group_sum); the last
+// group block of each column block, counted on counters[x], then adds the
+// groups in order (deterministic) and writes dgamma / dbeta of those columns
+// (as norm_hsh_param_pass2), and sets its counter back to zero.
+__global__ void __launch_bounds__(256) norm_hsh_param_groups_final(
+    const float* part, int splits, int64_t hs, int64_t h, float* inter, const __grid_constant__ MutPtrArray dg,
+    const __grid_constant__ MutPtrArray db, int accumulate, unsigned* counters) {
+  tpd::pdl_entry();
+  __shared__ int last;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPass2Cols + (threadIdx.x & 31);
+  const int g = static_cast<int>(blockIdx.y), groups = static_cast<int>(gridDim.y);
+  const int k1 = min(splits, (g + 1) * kParamGroup);
+  float sg, sb;
+  if (param_colsum_range(part, g * kParamGroup, k1, h, c, &sg, &sb)) {
+    inter[(static_cast<int64_t>(g) * 2 + 0) * h + c] = sg;
+    inter[(static_cast<int64_t>(g) * 2 + 1) * h + c] = sb;
+  }
+  __threadfence();  // this block's group sums are visible before it is counted
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    last = atomicAdd(counters + blockIdx.x, 1u) == static_cast<unsigned>(groups - 1);
+    if (last) atomicExch(counters + blockIdx.x, 0u);
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (!param_colsum_range<true>(inter, 0, groups, h, c, &sg, &sb)) return;
+  const int sh = static_cast<int>(c / hs);
+  const int64_t lc = c - sh * hs;
+  float* gp = static_cast<float*>(dg.p[sh]) + lc;
+  *gp = accumulate ? *gp + sg : sg;
+  if (db.p[sh]) {
+    float* bp = static_cast<float*>(db.p[sh]) + lc;
+    *bp = accumulate ? *bp + sb : sb;
+  }
+}
+
 // dgamma[c] (and dbeta[c]) = the fixed-order sum over the CTAs' partials
 // (added to the existing value when accumulate is set).
 __global__ void __launch_bounds__(256) norm_hsh_param_pass2(const float* part, int splits, int64_t hs, int64_t h,
@@ -888,7 +928,13 @@ tp_status launch_norm_sharded_bwd(tp_plan* plan, bool rms, const PtrArray& X, co
     if (s != TP_OK) return s;
   }
   const unsigned cblocks = static_cast<unsigned>((h + kPass2Cols - 1) / kPass2Cols);
-  if (rows > 0 && groups > 0) {
+  if (rows > 0 && groups > 0 && cblocks <= static_cast<unsigned>(kPlanCounters)) {
+    unsigned* ctr = nullptr;
+    s = plan_counters(plan, st, &ctr);
+    if (s != TP_OK) return s;
+    (void)tpi::launch(norm_hsh_param_groups_final, dim3(cblocks, static_cast<unsigned>(groups)), dim3(256), 0, st,
+                      part, static_cast<int>(grid), hs, h, inter, dg, db, accumulate, ctr);
+  } else if (rows > 0 && groups > 0) {
     (void)tpi::launch(param_group_sum, dim3(dim3(cblocks, static_cast<unsigned>(groups))), dim3(256), 0, st, 
         part, static_cast<int>(grid), h, inter);
     s = after_launch("norm_sharded_bwd/param groups");
