@@ -810,7 +810,7 @@ def measure_other(args, world, rank, local, sample_clocks=True):
             c1.record(stream)
             torch.cuda.synchronize()
             achb = 2.5 * core_flops * args.steps / (c0.elapsed_time(c1) / 1e3) / 1e12
-            roof["backward"] = {"kernel": "attn_bwd_prep + attn_bwd_dkdv_st + attn_bwd_dq (tcgen05)",
+            roof["backward"] = {"kernel": "attn_bwd_prep + attn_bwd_dkdv_st + attn_bwd_dq_gemm (tcgen05)",
                                 "achieved": achb, "unit": "TFLOP/s", "frac": achb / peaks["bf16_tflops"],
                                 "flops_per_launch_set": 2.5 * core_flops}
     out = {"metric": f"{args.workload} TFLOP/s on 1 B200", "value": value, "unit": "TFLOP/s",

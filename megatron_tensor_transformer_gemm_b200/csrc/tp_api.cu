@@ -387,9 +387,14 @@ tp_status run_gemm(const tp_plan* plan, const GemmBatch& b, cudaStream_t st) {
 // token dim) leave most SMs idle, so for bf16 plans, when the estimate says so,
 // the GEMM splits K: split s writes fp32 partials of every D[i] into the plan's
 // workspace and one reduce sums the splits in order into D[i].
-tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st) {
+// allow_split = false when another GEMM shares the GPU with this one (the
+// split's estimate assumes every SM; measured on the 12-layer stack beside
+// the side stream's GEMM: no split 240.1 TFLOP/s, split 237.8, and 48 fewer
+// launches a step).
+tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st, bool allow_split = true) {
   if (plan->dtype != TP_BF16) return run_gemm(plan, w, st);
-  const int s = gemm_split_k(w);
+  // a split forced through TP_GEMM_SPLITK (tests) applies in either case
+  const int s = allow_split || getenv("TP_GEMM_SPLITK") ? gemm_split_k(w) : 1;
   if (s <= 1 || s > TP_MAX_SHARDS) return launch_gemm_bf16(w, st);
   const int n = w.n;
   const int64_t M = w.g[0].M, N = w.g[0].N, mn = M * N, elems = n * mn;
@@ -1234,7 +1239,7 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
   } else {
     TP_TRY(run_gemm(plan, b, st));
   }
-  if (dW) TP_TRY(run_wgrad(plan, w, st));
+  if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
   if (dbias) TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, st));
   return TP_OK;
 }
@@ -1318,7 +1323,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     side.reset(new SideGemm(plan, d, st));
     TP_TRY(side->status());
   }
-  if (dW) TP_TRY(run_wgrad(plan, w, st));
+  if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
   if (dX_out && !side) TP_TRY(run_gemm(plan, d, st));
   if (dbias)
     TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p),

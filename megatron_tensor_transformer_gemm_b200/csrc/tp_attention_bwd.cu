@@ -17,6 +17,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "tp_device.cuh"
@@ -49,6 +50,13 @@ struct BwdParams {
   int seq_pad;                        // seq rounded up to a multiple of 64
   float scale_log2;  // log2(e) / sqrt(d)
   float scale;       // 1 / sqrt(d)
+  // store_ds: the dK/dV kernel also stores dS^T to the workspace, viewed as
+  // {queries, keys, shard * batch * hl} (query rows padded to seq_pad), and
+  // dQ = dS K runs as a GEMM over it (attn_bwd_dq_gemm) instead of recomputing
+  // S and dP (attn_bwd_dq).
+  int store_ds;
+  CUtensorMap tm_ds_st;  // box {64, 32, 1}: one warp pair's 32 key rows of a sub-tile
+  CUtensorMap tm_ds_ld;  // box {64, 64, 1}
   unsigned* status;
 };
 
@@ -205,7 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
   uint64_t* pds_empty = p_full + 2;    // [2]
   uint64_t* acc_full = pds_empty + 2;
   uint64_t* drain = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ds_written = drain + 1;    // [4] per lane quarter: both column halves written
+  uint64_t* ds_read = ds_written + 4;  // [4] per lane quarter: the slab's earlier store has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ds_read + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -234,6 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&ds_written[q], 2);  // lane 0 of each of the two warps
+      mbar_init(&ds_read[q], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -380,6 +394,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
         pk[e / 2] = pack_bf16x2(p0, p1);
         dk[e / 2] = pack_bf16x2(v0 ? p0 * (dp[e] - dd[e]) : 0.f, v1 ? p1 * (dp[e + 1] - dd[e + 1]) : 0.f);
       }
+      if (p.store_ds && it >= 2) {
+        // buffer x's dS^T slab was stored at it - 2; that store must have
+        // read it before the rewrite (the half-0 warp's lane 0 issued it)
+        bool rd = true;
+        if (half == 0) {
+          if (lane == 0) {
+            bulk_wait_read<1>();
+            mbar_arrive(&ds_read[lg]);
+          }
+          __syncwarp();
+        } else {
+          rd = mbar_wait(&ds_read[lg], static_cast<uint32_t>(it & 1), abort_flag, p.status);
+        }
+        if (!__all_sync(0xffffffffu, rd)) {
+          ok = false;
+          break;
+        }
+      }
       // row r of the [128 keys x 64 queries] K-major tiles: 16-byte chunks
       // 4 half .. 4 half + 3 of its 128-byte swizzled row
       uint8_t* prow = sP + x * SM::PT + r * 128;
@@ -396,7 +428,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x]);
+      if (p.store_ds) {
+        // rows [32 lg, 32 lg + 32) of dS^T, both column halves written: the
+        // half-0 warp's lane 0 stores them (keys k0 + 32 lg.., this sub-tile's 64 queries)
+        if (lane == 0) mbar_arrive(&ds_written[lg]);
+        if (half == 0 && lane == 0 &&
+            mbar_wait(&ds_written[lg], static_cast<uint32_t>(it & 1), abort_flag, p.status)) {
+          tma_store_3d(&p.tm_ds_st, sdS + x * SM::PT + lg * 32 * 128, (2 * j + it) * 64, k0 + lg * 32,
+                       static_cast<int>((static_cast<int64_t>(shard) * p.batch + b) * p.hl + hh));
+          bulk_commit();
+        }
+      }
     }
+    if (p.store_ds && half == 0 && lane == 0) bulk_wait_all();  // every dS^T store has landed
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
       tc_fence_after();
       __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
@@ -589,12 +633,144 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq(const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------
+// dQ = dS K / sqrt(d) as a GEMM over the dS^T the dK/dV kernel stored: one CTA
+// per 128-query block of one (shard, batch, head), looping over the 64-key
+// blocks that reach it (causal: keys < q0 + 128). Per key block, dS (two
+// 64-query blocks of dS^T, read MN-major) and K (D/64 blocks, MN-major) arrive
+// by TMA into one of ST stages, and dQ += dS K accumulates in TMEM (M = 128
+// queries, N = d, K = 64 keys); the epilogue scales and stores dQ. Entries of
+// dS^T above the diagonal inside a stored tile are zeros (P is masked there).
+template <int D, int ST>
+struct DqgSmem {
+  static constexpr int A = 64 * BQ * 2;  // dS^T [64 keys x 128 queries]
+  static constexpr int B = 64 * D * 2;   // K [64 keys x D]
+  static constexpr int STAGE = A + B;
+  static constexpr int TOTAL = 1024 + ST * STAGE + 256;
+};
+
+template <int D, int ST>
+__global__ void __launch_bounds__(kThreads, 2) attn_bwd_dq_gemm(const __grid_constant__ BwdParams p) {
+  tpd::pdl_entry();
+  using SM = DqgSmem<D, ST>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sA = smem;                 // [ST]
+  uint8_t* sB = sA + ST * SM::A;      // [ST]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + ST * SM::B);  // [ST]
+  uint64_t* empty = full + ST;        // [ST]
+  uint64_t* acc_full = empty + ST;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = p.p * p.batch * p.hl;
+  const int i = p.nq - 1 - static_cast<int>(blockIdx.x) / per;  // heaviest query blocks first
+  int rest = static_cast<int>(blockIdx.x) % per;
+  const int hh = rest % p.hl;
+  rest /= p.hl;
+  const int b = rest % p.batch;
+  const int shard = rest / p.batch;
+  const int q0 = i * BQ;
+  const int n_kb = min(2 * i + 2, (p.seq + 63) / 64);  // 64-key blocks with keys < q0 + 128
+  const int hl_d = p.hl * D;
+  const int bhg = static_cast<int>((static_cast<int64_t>(shard) * p.batch + b) * p.hl + hh);
+  constexpr uint32_t kCols = D < 32 ? 32 : D;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tdQ = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    const CUtensorMap* tk = &p.tm_q64[shard];  // QKV, box {64, 1, 64}: 64 keys x 64 of K's columns
+    tma_prefetch_desc(tk);
+    tma_prefetch_desc(&p.tm_ds_ld);
+    int last_par[ST];
+    for (int s = 0; s < ST; ++s) last_par[s] = -1;
+    for (int kb = 0; kb < n_kb; ++kb) {
+      const int st = kb % ST;
+      const uint32_t ph = static_cast<uint32_t>(kb / ST) & 1u;
+      if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) break;
+      mbar_arrive_expect_tx(&full[st], SM::A + SM::B);
+#pragma unroll
+      for (int c = 0; c < BQ / 64; ++c)
+        tma_load_3d(sA + st * SM::A + c * (64 * 128), &p.tm_ds_ld, &full[st], q0 + c * 64, kb * 64, bhg);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_3d(sB + st * SM::B + c * (64 * 128), tk, &full[st], hl_d + hh * D + c * 64, b, kb * 64);
+      last_par[st] = static_cast<int>(ph);
+    }
+    for (int s = 0; s < ST; ++s)
+      if (last_par[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(last_par[s]), abort_flag, p.status);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t id = idesc_bf16(BQ, D, true, true);  // A = dS (MN-major), B = K (MN-major)
+    bool ok = true;
+    for (int kb = 0; kb < n_kb; ++kb) {
+      const int st = kb % ST;
+      if (!mbar_wait(&full[st], static_cast<uint32_t>(kb / ST) & 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(sA + st * SM::A), b_base = smem_u32(sB + st * SM::B);
+#pragma unroll
+      for (int kk = 0; kk < 64 / 16; ++kk)  // K = 64 keys, 16 per MMA: 16 rows of 128 bytes
+        tc_mma_bf16(tdQ, smem_desc_sw128(a_base + kk * 2048, 64 * 128, 1024),
+                    smem_desc_sw128(b_base + kk * 2048, 64 * 128, 1024), id, (kb | kk) != 0 ? 1u : 0u);
+      tc_commit(&empty[st]);
+    }
+    (void)ok;
+    tc_commit(acc_full);
+    tc_commit(drain);
+    mbar_wait(drain, 0, abort_flag, p.status);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------- epilogue
+    const int lg = warp & 3;
+    const int half = (warp - 2) / 4;
+    const int q = q0 + lg * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+    if (n_kb > 0 && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.status))) {
+      tc_fence_after();
+      __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.dqkv[shard]) +
+                            (static_cast<int64_t>(q) * p.batch + b) * (3 * hl_d) + hh * D;
+      // each column half of warps stores half of dQ's D columns
+      tmem_row_to_global<D / 2>(tdQ + lane_off + half * (D / 2), base + half * (D / 2), p.scale, q < p.seq);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tdQ, kCols);
+  }
+}
+
 // STS: stages of the streamed 64-query Q, dO sub-tiles (dK/dV kernel); STQ:
 // stages of the streamed 128-key K, V blocks (dQ kernel); as many as fit the
 // 227 KB of shared memory.
-template <int D, int STS, int STQ>
+template <int D, int STS, int STQ, int STG>
 tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
-  static_assert(DkdvStSmem<D, STS>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448,
+  static_assert(DkdvStSmem<D, STS>::TOTAL <= 232448 && DqSmem<D, STQ>::TOTAL <= 232448 &&
+                    2 * DqgSmem<D, STG>::TOTAL <= 232448,
                 "shared memory of the backward kernels");
   constexpr int kMaxDev = 64;
   static bool attr[kMaxDev] = {};
@@ -611,6 +787,9 @@ tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
     s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq<D, STQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               DqSmem<D, STQ>::TOTAL), "cudaFuncSetAttribute(attention dq)");
     if (s != TP_OK) return s;
+    s = tpi::cuda_status(cudaFuncSetAttribute(attn_bwd_dq_gemm<D, STG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              DqgSmem<D, STG>::TOTAL), "cudaFuncSetAttribute(attention dq gemm)");
+    if (s != TP_OK) return s;
     attr[dev] = true;
   }
   const int per = prm.p * prm.batch * prm.hl;
@@ -618,7 +797,11 @@ tp_status launch_bwd_d(const BwdParams& prm, cudaStream_t st) {
                     prm);
   tp_status s = tpi::after_launch("attention_bwd dK/dV (tcgen05)");
   if (s != TP_OK) return s;
-  (void)tpi::launch(attn_bwd_dq<D, STQ>, dim3(prm.nq * per), dim3(kThreads), DqSmem<D, STQ>::TOTAL, st, prm);
+  if (prm.store_ds)
+    (void)tpi::launch(attn_bwd_dq_gemm<D, STG>, dim3(prm.nq * per), dim3(kThreads), DqgSmem<D, STG>::TOTAL, st,
+                      prm);
+  else
+    (void)tpi::launch(attn_bwd_dq<D, STQ>, dim3(prm.nq * per), dim3(kThreads), DqSmem<D, STQ>::TOTAL, st, prm);
   return tpi::after_launch("attention_bwd dQ (tcgen05)");
 }
 
@@ -633,8 +816,16 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
   const int64_t rows_per_shard = static_cast<int64_t>(batch) * hl * seq;
   const int seq_pad = (seq + 63) / 64 * 64;
   const int64_t padded_per_shard = static_cast<int64_t>(batch) * hl * seq_pad;
+  // workspace: D and lse2 ([p][batch * hl][seq_pad] fp32 each), then, when dQ
+  // runs as a GEMM over the stored dS^T, dS^T [p * batch * hl][seq_pad keys][seq_pad queries]
+  // bf16 (up to kDsBytesMax; longer sequences recompute S and dP in attn_bwd_dq).
+  constexpr size_t kDsBytesMax = size_t(8) << 30;
+  const size_t vec_bytes = (static_cast<size_t>(2 * padded_per_shard * p) * sizeof(float) + 1023) / 1024 * 1024;
+  const size_t ds_bytes = static_cast<size_t>(p) * batch * hl * seq_pad * seq_pad * 2;
+  const char* e_ds = getenv("TP_ATTN_BWD_DS");
+  const bool store_ds = !(e_ds && e_ds[0] == '0') && ds_bytes <= kDsBytesMax;
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(2 * padded_per_shard * p) * sizeof(float), &ws);
+  tp_status s = workspace(plan, vec_bytes + (store_ds ? ds_bytes : 0), &ws);
   if (s != TP_OK) return s;
   static BwdParams prm;
   static std::mutex mu;
@@ -666,6 +857,18 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
     prm.lse[i] = lse[i];
     prm.dvec[i] = static_cast<const float*>(dvec.p[i]);
   }
+  prm.store_ds = store_ds ? 1 : 0;
+  if (store_ds) {
+    void* ds = static_cast<uint8_t*>(ws) + vec_bytes;
+    cuuint64_t dd[3] = {static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(seq),
+                        static_cast<cuuint64_t>(p) * batch * hl};
+    cuuint64_t ds_str[2] = {static_cast<cuuint64_t>(seq_pad) * 2, static_cast<cuuint64_t>(seq_pad) * seq_pad * 2};
+    cuuint32_t box_st[3] = {64, 32, 1}, box_ld[3] = {64, 64, 1};
+    s = encode_bf16(&prm.tm_ds_st, ds, 3, dd, ds_str, box_st, "dS^T (stores)");
+    if (s != TP_OK) return s;
+    s = encode_bf16(&prm.tm_ds_ld, ds, 3, dd, ds_str, box_ld, "dS^T (loads)");
+    if (s != TP_OK) return s;
+  }
   prm.p = p;
   prm.batch = batch;
   prm.seq = seq;
@@ -690,8 +893,8 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
                       seq_pad, hl);
   s = after_launch("attention_bwd prep");
   if (s != TP_OK) return s;
-  if (d == 64) return launch_bwd_d<64, 4, 2>(prm, st);
-  if (d == 128) return launch_bwd_d<128, 3, 2>(prm, st);
+  if (d == 64) return launch_bwd_d<64, 4, 2, 4>(prm, st);
+  if (d == 128) return launch_bwd_d<128, 3, 2, 3>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
 }
 

@@ -90,14 +90,19 @@ def test_attention_block_full_size_sampled(fused):
     assert _tp().device_status() == "TP_OK"
 
 
+@pytest.mark.parametrize("ds", ["1", "0"])
 @pytest.mark.parametrize("batch,seq,heads,d,p", [
     (2, 300, 4, 64, 2),
     (1, 256, 2, 128, 1),
     (3, 129, 8, 64, 4),
+    (1, 520, 2, 128, 2),
 ])
-def test_attention_bwd_local_heads(batch, seq, heads, d, p):
+def test_attention_bwd_local_heads(batch, seq, heads, d, p, ds, monkeypatch):
     """dQ, dK, dV of each shard's heads from independent Q, K, V, dO; O and LSE
-    come from the GPU forward of those inputs (the oracle computes its own)."""
+    come from the GPU forward of those inputs (the oracle computes its own).
+    ds = "1": dQ as a GEMM over the dS^T the dK/dV kernel stores; "0": dQ
+    recomputing S and dP (TP_ATTN_BWD_DS=0, read at each call)."""
+    monkeypatch.setenv("TP_ATTN_BWD_DS", ds)
     tp = _tp()
     h = heads * d
     Q, K, V, dO = tp_synth.draw_qkv_activations(batch, seq, heads, d, torch.bfloat16, seed=seq + 7)
