@@ -384,15 +384,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
       const float* dd = l2 + 64;
       const int qb = (2 * j + it) * 64 + half * 32;  // query of column 0 of this half
       uint32_t pk[16], dk[16];
+      // below the diagonal and inside the sequence for the whole warp (every
+      // key <= the first query, the last query < seq): no masks
+      if (__all_sync(0xffffffffu, key <= qb && qb + 31 < p.seq)) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int qa = qb + e;
-        const bool v0 = key <= qa && qa < p.seq && key < p.seq;
-        const bool v1 = key <= qa + 1 && qa + 1 < p.seq && key < p.seq;
-        const float p0 = v0 ? exp2f(sv[e] * p.scale_log2 - l2[e]) : 0.f;
-        const float p1 = v1 ? exp2f(sv[e + 1] * p.scale_log2 - l2[e + 1]) : 0.f;
-        pk[e / 2] = pack_bf16x2(p0, p1);
-        dk[e / 2] = pack_bf16x2(v0 ? p0 * (dp[e] - dd[e]) : 0.f, v1 ? p1 * (dp[e + 1] - dd[e + 1]) : 0.f);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 L = *reinterpret_cast<const float4*>(l2 + e);
+          const float4 Dq = *reinterpret_cast<const float4*>(dd + e);
+          const float p0 = ex2(fmaf(sv[e], p.scale_log2, -L.x)), p1 = ex2(fmaf(sv[e + 1], p.scale_log2, -L.y));
+          const float p2 = ex2(fmaf(sv[e + 2], p.scale_log2, -L.z)), p3 = ex2(fmaf(sv[e + 3], p.scale_log2, -L.w));
+          pk[e / 2] = pack_bf16x2(p0, p1);
+          pk[e / 2 + 1] = pack_bf16x2(p2, p3);
+          dk[e / 2] = pack_bf16x2(p0 * (dp[e] - Dq.x), p1 * (dp[e + 1] - Dq.y));
+          dk[e / 2 + 1] = pack_bf16x2(p2 * (dp[e + 2] - Dq.z), p3 * (dp[e + 3] - Dq.w));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int qa = qb + e;
+          const bool v0 = key <= qa && qa < p.seq && key < p.seq;
+          const bool v1 = key <= qa + 1 && qa + 1 < p.seq && key < p.seq;
+          const float p0 = v0 ? ex2(fmaf(sv[e], p.scale_log2, -l2[e])) : 0.f;
+          const float p1 = v1 ? ex2(fmaf(sv[e + 1], p.scale_log2, -l2[e + 1])) : 0.f;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+          dk[e / 2] = pack_bf16x2(v0 ? p0 * (dp[e] - dd[e]) : 0.f, v1 ? p1 * (dp[e + 1] - dd[e + 1]) : 0.f);
+        }
       }
       if (p.store_ds && it >= 2) {
         // buffer x's dS^T slab was stored at it - 2; that store must have

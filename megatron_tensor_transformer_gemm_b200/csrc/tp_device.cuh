@@ -414,6 +414,14 @@ __device__ __forceinline__ float silu_grad_f(float z) {
   return s * (1.0f + z * (1.0f - s));
 }
 
+// 2^x by the hardware approximation (denormal results flush to 0): the
+// attention kernels' exponentials, whose arguments are <= 2^3 after the max.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
