@@ -320,6 +320,16 @@ TP_API tp_status tp_attention_fwd(tp_plan* plan, int batch, int seq, const void*
 
 /* ------------------------------------------------------------ backward */
 
+/* Streams of the backward calls: tp_row_bwd (dZ and dW) and the column
+ * backward calls (dX and dW) issue two GEMMs that read the same inputs. When
+ * either leaves SMs idle (few output tiles), the activation-gradient GEMM runs
+ * on a side stream the library creates per device, forked from `stream` by an
+ * event, and `stream` waits for it before the call returns: the results are
+ * ordered on `stream` as with one stream, also inside a stream capture (the
+ * fork and join become graph edges). Environment TP_BWD_CONCURRENT=0 keeps
+ * every launch on `stream`. Calls on one plan must not overlap in time (they
+ * share the plan's workspace). */
+
 /* Row layer backward for every shard ([TP-scratch] §四: the input gradient of
  * the row layer needs no reduction; dY is replicated).
  *   dY [T, hidden]; H[i] the row input of shard i; W[i] the row shard.

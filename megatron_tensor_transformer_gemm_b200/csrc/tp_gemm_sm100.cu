@@ -129,7 +129,10 @@ struct alignas(64) GemmParams {
   // output problem, tmE views D and tmX the staged input (Z of the dGELU /
   // dSwiGLU epilogues, or the residual) as {columns, halves, rows} with a
   // {32, 1, 32} box and 64-byte swizzle; halves = 2 splits [gate | up] at nh.
+  // With the row scatter, tmE[j] / tmX[j] view sequence shard j's output /
+  // residual ({N, 1, rows_per_out}) and scatter_res says whether residuals come.
   int tma_epi;
+  int scatter_res;
   CUtensorMap tmE[TP_MAX_SHARDS];
   CUtensorMap tmX[TP_MAX_SHARDS];
   unsigned* status;
@@ -357,7 +360,7 @@ __device__ __forceinline__ void stage_write(uint32_t tile, int r, const float (&
 __device__ __forceinline__ int epi_inputs(const GemmParams& p, const GroupArgs& ga) {
   if (p.epi == tpi::EPI_DSWIGLU) return 2;
   if (p.epi == tpi::EPI_DGELU) return 1;
-  if (p.epi == tpi::EPI_STORE) return ga.aux ? 1 : 0;
+  if (p.epi == tpi::EPI_STORE) return (p.scatter ? p.scatter_res : ga.aux != nullptr) ? 1 : 0;
   return 0;  // the forward activations stage outputs only
 }
 
@@ -678,7 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       tma_prefetch_desc(&p.tmA[g]);
       tma_prefetch_desc(&p.tmB[g]);
     }
-    if (p.tma_epi) {
+    if (p.tma_epi && p.scatter) {
+      for (int j = 0; j * p.rows_per_out < p.g[0].M && j < TP_MAX_SHARDS; ++j) {
+        tma_prefetch_desc(&p.tmE[j]);
+        if (p.scatter_res) tma_prefetch_desc(&p.tmX[j]);
+      }
+    } else if (p.tma_epi) {
       const bool fwd = p.epi == tpi::EPI_SWIGLU || p.epi == tpi::EPI_BIAS_GELU;
       for (int g = 0; g < p.ngroups; ++g) {  // only the views the launch encoded
         if (!fwd || p.g[g].D) tma_prefetch_desc(&p.tmE[g]);
@@ -908,10 +916,20 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       const int row0 = mt * C::TILE_M + static_cast<int>(rank) * BM + lg * 32;
       const int n0 = nt * p.tile_n;
       const bool narrow = narrow_tile(p, ga, n0);
+      // TMA views: the output problem's, or with the row scatter the view of
+      // the sequence shard holding these 32 rows (whole: rows_per_out is a
+      // multiple of 32), at its local row; warps past the last row store nothing
+      int gi = p.kcat ? 0 : g, trow = row0;
+      bool tma_rows = true;
+      if (p.scatter) {
+        tma_rows = row0 < ga.M;
+        gi = tma_rows ? row0 / p.rows_per_out : 0;
+        trow = row0 - gi * p.rows_per_out;
+      }
       // TMA epilogue: the first chunk's inputs load while the MMAs finish
-      const int gi = p.kcat ? 0 : g;
-      const bool pre = p.tma_epi && epi_inputs(p, ga) > 0 && n0 + half * (narrow ? BN / 4 : BN / 2) < ga.N;
-      if (pre && lane == 0) epi_issue_inputs(p, gi, epi_inputs(p, ga), n0 + half * (narrow ? BN / 4 : BN / 2), row0, es);
+      const bool pre = p.tma_epi && tma_rows && epi_inputs(p, ga) > 0 &&
+                       n0 + half * (narrow ? BN / 4 : BN / 2) < ga.N;
+      if (pre && lane == 0) epi_issue_inputs(p, gi, epi_inputs(p, ga), n0 + half * (narrow ? BN / 4 : BN / 2), trow, es);
       // warp-uniform: the epilogue's tcgen05.ld is warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status))) {
         if (pre && lane == 0) {  // the prefetched copies land before the CTA may exit (bounded)
@@ -923,10 +941,12 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      if (p.tma_epi && (p.epi == tpi::EPI_SWIGLU || p.epi == tpi::EPI_BIAS_GELU)) {
-        epilogue_fwd_tma(p, ga, gi, taddr, row0, n0, half, narrow, lane, es);
+      if (p.tma_epi && !tma_rows) {
+        // past the last row of a scattered launch: nothing to store
+      } else if (p.tma_epi && (p.epi == tpi::EPI_SWIGLU || p.epi == tpi::EPI_BIAS_GELU)) {
+        epilogue_fwd_tma(p, ga, gi, taddr, trow, n0, half, narrow, lane, es);
       } else if (p.tma_epi) {
-        ok = epilogue_tile_tma(p, ga, gi, taddr, row0, n0, half, narrow, pre, lane, es, abort_flag, p.status);
+        ok = epilogue_tile_tma(p, ga, gi, taddr, trow, n0, half, narrow, pre, lane, es, abort_flag, p.status);
       } else {
         epilogue_tile(p, ga, taddr, row0 + lane, n0, half, narrow, ks);
       }
@@ -1008,7 +1028,19 @@ tp_status encode_epi(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_
 bool tma_epilogue_ok(const GemmBatch& b, int nout, int ksplit) {
   const char* e = getenv("TP_GEMM_TMA_EPI");
   if (e && e[0] == '0') return false;
-  if (b.out_f32 || ksplit > 1 || b.scatter_n > 0) return false;
+  if (b.out_f32 || ksplit > 1) return false;
+  if (b.scatter_n > 0) {  // plain stores into sequence shards of whole 32-row warp slabs
+    if (b.epi != tpi::EPI_STORE || b.rows_per_out % 32 || b.scatter_n > TP_MAX_SHARDS ||
+        static_cast<int64_t>(b.scatter_n) * b.rows_per_out != b.g[0].M)
+      return false;
+    const bool res = b.res_seq[0] != nullptr;
+    for (int j = 0; j < b.scatter_n; ++j) {
+      if (!b.out_seq[j] || reinterpret_cast<uintptr_t>(b.out_seq[j]) % 16) return false;
+      if ((b.res_seq[j] != nullptr) != res) return false;
+      if (res && reinterpret_cast<uintptr_t>(b.res_seq[j]) % 16) return false;
+    }
+    return true;
+  }
   const bool fwd = b.epi == tpi::EPI_SWIGLU || b.epi == tpi::EPI_BIAS_GELU;
   const bool bwd = b.epi == tpi::EPI_DGELU || b.epi == tpi::EPI_DSWIGLU;
   if (!fwd && !bwd && b.epi != tpi::EPI_STORE) return false;
@@ -1298,7 +1330,17 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     p.split_stride = b.split_stride;
     tiles *= ksplit;
   }
-  if (tma_epilogue_ok(b, nout, ksplit)) {
+  if (b.scatter_n > 0 && tma_epilogue_ok(b, nout, ksplit)) {
+    p.tma_epi = 1;
+    p.scatter_res = b.res_seq[0] != nullptr ? 1 : 0;
+    const GemmProblem& o = b.g[0];
+    for (int j = 0; j < b.scatter_n && p.tma_epi; ++j) {
+      bool good = encode_epi(enc, &p.tmE[j], b.out_seq[j], o.N, 1, o.ldd, b.rows_per_out, o.ldd) == TP_OK;
+      if (good && p.scatter_res)
+        good = encode_epi(enc, &p.tmX[j], b.res_seq[j], o.N, 1, o.ldaux, b.rows_per_out, o.ldaux) == TP_OK;
+      if (!good) p.tma_epi = 0;
+    }
+  } else if (tma_epilogue_ok(b, nout, ksplit)) {
     p.tma_epi = 1;
     const bool sw = b.epi == tpi::EPI_DSWIGLU || b.epi == tpi::EPI_SWIGLU;
     const bool fwd = b.epi == tpi::EPI_SWIGLU || b.epi == tpi::EPI_BIAS_GELU;

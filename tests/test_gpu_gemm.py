@@ -241,7 +241,8 @@ def test_bf16_mlp_end_to_end_small(act, bias):
     assert_close(dW2, g["dW2"], TOL_BF16, "dW2")
 
 
-@pytest.mark.parametrize("T,K,h,p", [(300, 264, 192, 2), (257, 1376, 512, 8), (64, 128, 256, 1)])
+@pytest.mark.parametrize("T,K,h,p", [(300, 264, 192, 2), (257, 1376, 512, 8), (64, 128, 256, 1),
+                                     (512, 264, 192, 4), (320, 136, 280, 5)])
 def test_row_forward_fused_reduce(T, K, h, p):
     """The row GEMM with the shard sum fused: sum_i H_i W2_i^T + b + residual."""
     tp = _tp()
@@ -268,7 +269,8 @@ def test_row_forward_fused_reduce(T, K, h, p):
             assert_close(Ys[j], refs[j], TOL_BF16, f"fused RS shard {j}")
 
 
-@pytest.mark.parametrize("T,h,f,p,act", [(300, 192, 528, 2, "gelu"), (256, 256, 272, 2, "swiglu")])
+@pytest.mark.parametrize("T,h,f,p,act", [(300, 192, 528, 2, "gelu"), (256, 256, 272, 2, "swiglu"),
+                                        (384, 192, 528, 3, "gelu")])
 def test_column_backward_fused_reduce(T, h, f, p, act):
     tp = _tp()
     g = torch.Generator().manual_seed(T + 12)
