@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
         for (int c = 0; c < BKV / 32; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, sv[c][i]);
+          for (int i = 0; i < 32; i += 2) mx = max3(mx, sv[c][i], sv[c][i + 1]);
       } else {
 #pragma unroll
         for (int c = 0; c < BKV / 32; ++c)
@@ -321,15 +321,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int i = v * 8 + 2 * w;
-            float a = ex2(fmaf(sv[cc][i], sc, -m));
-            float bb = ex2(fmaf(sv[cc][i + 1], sc, -m));
+            const float2 x = fma2_bcast(sv[cc][i], sv[cc][i + 1], sc, -m);  // scaled score - m
+            float a = ex2(x.x);
+            float bb = ex2(x.y);
             if (!full) {
               a = (cc * 32 + i <= kmax) ? a : 0.f;
               bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
             }
             pk[w] = pack_bf16x2(a, bb);
-            const float2 f = unpack_bf16x2(pk[w]);  // the row sum uses the rounded P of the PV MMA
-            rs += f.x + f.y;
+            // the row sum uses the rounded P of the PV MMA (bf16 widening is exact)
+            { const float2 f = unpack_bf16x2(pk[w]); rs += f.x + f.y; }
           }
           const int qv = (cc % 2) * 4 + v;
           *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);

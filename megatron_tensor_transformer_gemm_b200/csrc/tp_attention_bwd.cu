@@ -387,16 +387,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkdv_st(const __grid_con
       // below the diagonal and inside the sequence for the whole warp (every
       // key <= the first query, the last query < seq): no masks
       if (__all_sync(0xffffffffu, key <= qb && qb + 31 < p.seq)) {
+        const float sc = p.scale_log2;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 L = *reinterpret_cast<const float4*>(l2 + e);
           const float4 Dq = *reinterpret_cast<const float4*>(dd + e);
-          const float p0 = ex2(fmaf(sv[e], p.scale_log2, -L.x)), p1 = ex2(fmaf(sv[e + 1], p.scale_log2, -L.y));
-          const float p2 = ex2(fmaf(sv[e + 2], p.scale_log2, -L.z)), p3 = ex2(fmaf(sv[e + 3], p.scale_log2, -L.w));
+          // pairs of columns in packed fp32 (one instruction per pair)
+          const float2 x01 = fma2(sv[e], sv[e + 1], sc, sc, -L.x, -L.y);
+          const float2 x23 = fma2(sv[e + 2], sv[e + 3], sc, sc, -L.z, -L.w);
+          const float p0 = ex2(x01.x), p1 = ex2(x01.y), p2 = ex2(x23.x), p3 = ex2(x23.y);
           pk[e / 2] = pack_bf16x2(p0, p1);
           pk[e / 2 + 1] = pack_bf16x2(p2, p3);
-          dk[e / 2] = pack_bf16x2(p0 * (dp[e] - Dq.x), p1 * (dp[e + 1] - Dq.y));
-          dk[e / 2 + 1] = pack_bf16x2(p2 * (dp[e + 2] - Dq.z), p3 * (dp[e + 3] - Dq.w));
+          const float2 d01 = submul2(dp[e], dp[e + 1], Dq.x, Dq.y, p0, p1);
+          const float2 d23 = submul2(dp[e + 2], dp[e + 3], Dq.z, Dq.w, p2, p3);
+          dk[e / 2] = pack_bf16x2(d01.x, d01.y);
+          dk[e / 2 + 1] = pack_bf16x2(d23.x, d23.y);
         }
       } else {
 #pragma unroll

@@ -414,6 +414,48 @@ __device__ __forceinline__ float silu_grad_f(float z) {
   return s * (1.0f + z * (1.0f - s));
 }
 
+// Packed fp32 pairs (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+// (a0, a1) * (b, b) + (c, c), each lane rounded once as fmaf
+__device__ __forceinline__ float2 fma2_bcast(float a0, float a1, float b, float c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_pack(a0, a1)), "l"(f2_pack(b, b)), "l"(f2_pack(c, c)));
+  return f2_unpack(r);
+}
+// (a0, a1) * (b0, b1) + (c0, c1), each lane rounded once as fmaf
+__device__ __forceinline__ float2 fma2(float a0, float a1, float b0, float b1, float c0, float c1) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_pack(a0, a1)), "l"(f2_pack(b0, b1)), "l"(f2_pack(c0, c1)));
+  return f2_unpack(r);
+}
+// (a0 - b0, a1 - b1) * (c0, c1), each operation rounded as in fp32
+__device__ __forceinline__ float2 submul2(float a0, float a1, float b0, float b1, float c0, float c1) {
+  uint64_t d, r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a0, a1)), "l"(f2_pack(b0, b1)));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(d), "l"(f2_pack(c0, c1)));
+  return f2_unpack(r);
+}
+// (a0 + b0, a1 + b1), each lane rounded as an fp32 add
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x by the hardware approximation (denormal results flush to 0): the
 // attention kernels' exponentials, whose arguments are <= 2^3 after the max.
 __device__ __forceinline__ float ex2(float x) {
