@@ -347,8 +347,9 @@ bool concurrent_bwd(const tp_plan* plan, const GemmBatch& act_grad, const GemmBa
   return !gemm_fills_gpu(act_grad) || !gemm_fills_gpu(wgrad);
 }
 
-// Runs `act_grad` on the side stream (forked from st) and, when it goes out
-// of scope, makes st wait for it: every return path of the call joins.
+// Runs `act_grad` on the side stream (forked from st); more work may follow
+// it there (stream()). When it goes out of scope, st waits for everything
+// issued on the side stream: every return path of the call joins.
 class SideGemm {
  public:
   SideGemm(const tp_plan* plan, const GemmBatch& act_grad, cudaStream_t st) : st_(st) {
@@ -361,14 +362,15 @@ class SideGemm {
       return;
     }
     status_ = plan->dtype == TP_BF16 ? launch_gemm_bf16(act_grad, sd_->s) : launch_gemm_f32(act_grad, sd_->s);
-    const tp_status r = cuda_status(cudaEventRecord(sd_->join, sd_->s), "cudaEventRecord(join)");
-    if (status_ == TP_OK) status_ = r;
-    if (r != TP_OK) sd_ = nullptr;
   }
   ~SideGemm() {
-    if (sd_) cudaStreamWaitEvent(st_, sd_->join, 0);
+    if (!sd_) return;
+    if (cudaEventRecord(sd_->join, sd_->s) == cudaSuccess) cudaStreamWaitEvent(st_, sd_->join, 0);
+    else cudaStreamSynchronize(sd_->s);  // cannot join by event: finish the side work now
+    cudaGetLastError();
   }
   tp_status status() const { return status_; }
+  cudaStream_t stream() const { return sd_ ? sd_->s : st_; }
 
  private:
   SideStream* sd_ = nullptr;
@@ -391,15 +393,30 @@ tp_status run_gemm(const tp_plan* plan, const GemmBatch& b, cudaStream_t st) {
 // split's estimate assumes every SM; measured on the 12-layer stack beside
 // the side stream's GEMM: no split 240.1 TFLOP/s, split 237.8, and 48 fewer
 // launches a step).
-tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st, bool allow_split = true) {
-  if (plan->dtype != TP_BF16) return run_gemm(plan, w, st);
+// The K split run_wgrad takes for w (1: none).
+int wgrad_split(const tp_plan* plan, const GemmBatch& w, bool allow_split) {
+  if (plan->dtype != TP_BF16) return 1;
   // a split forced through TP_GEMM_SPLITK (tests) applies in either case
   const int s = allow_split || getenv("TP_GEMM_SPLITK") ? gemm_split_k(w) : 1;
-  if (s <= 1 || s > TP_MAX_SHARDS) return launch_gemm_bf16(w, st);
+  if (s <= 1 || s > TP_MAX_SHARDS) return 1;
+  for (int i = 0; i < w.n; ++i)
+    if (w.g[i].ldd != w.g[0].N) return 1;
+  return s;
+}
+// Workspace bytes run_wgrad uses for w (its split's fp32 partials), rounded up to 256.
+size_t wgrad_workspace(const tp_plan* plan, const GemmBatch& w, bool allow_split) {
+  const int s = wgrad_split(plan, w, allow_split);
+  if (s <= 1) return 0;
+  const size_t b = static_cast<size_t>(s) * w.n * w.g[0].M * w.g[0].N * sizeof(float);
+  return (b + 255) / 256 * 256;
+}
+
+tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st, bool allow_split = true) {
+  if (plan->dtype != TP_BF16) return run_gemm(plan, w, st);
+  const int s = wgrad_split(plan, w, allow_split);
+  if (s <= 1) return launch_gemm_bf16(w, st);
   const int n = w.n;
   const int64_t M = w.g[0].M, N = w.g[0].N, mn = M * N, elems = n * mn;
-  for (int i = 0; i < n; ++i)
-    if (w.g[i].ldd != N) return launch_gemm_bf16(w, st);
   void* ws = nullptr;
   TP_TRY(workspace(plan, static_cast<size_t>(s) * elems * sizeof(float), &ws));
   float* part = static_cast<float*>(ws);
@@ -1239,8 +1256,12 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
   } else {
     TP_TRY(run_gemm(plan, b, st));
   }
+  // The bias gradient reads only dY: beside the weight gradient too (after dH on
+  // the side stream, its partials past the weight gradient's workspace).
+  if (dbias)
+    TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, side ? side->stream() : st,
+                             side ? wgrad_workspace(plan, w, false) : 0));
   if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
-  if (dbias) TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, st));
   return TP_OK;
 }
 
@@ -1323,12 +1344,14 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     side.reset(new SideGemm(plan, d, st));
     TP_TRY(side->status());
   }
+  // The bias gradients read only dZ: beside the weight gradient too (after dX on
+  // the side stream, their partials past the weight gradient's workspace).
+  if (dbias)
+    TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p), p, T, n, n,
+                                     to_marr(reinterpret_cast<void* const*>(dbias), p), 0, plan->dtype,
+                                     side ? side->stream() : st, side ? wgrad_workspace(plan, w, false) : 0));
   if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
   if (dX_out && !side) TP_TRY(run_gemm(plan, d, st));
-  if (dbias)
-    TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p),
-                                     p, T, n, n, to_marr(reinterpret_cast<void* const*>(dbias), p), 0,
-                                     plan->dtype, st));
   return TP_OK;
 }
 

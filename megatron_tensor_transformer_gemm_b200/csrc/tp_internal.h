@@ -107,12 +107,15 @@ tp_status launch_reduce(const PtrArray& P, int n, const void* bias, const void* 
                         tp_dtype dt, cudaStream_t st);
 tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_t cols,
                         tp_dtype dt, cudaStream_t st);
+// ws_offset: the partials start this many bytes into the plan's workspace
+// (a multiple of 256), leaving the bytes before it to concurrent work.
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
-                            float* out, int accumulate, tp_dtype dt, cudaStream_t st);
-// The same for n inputs of one shape at once (one pass-1 and one pass-2 launch).
+                            float* out, int accumulate, tp_dtype dt, cudaStream_t st,
+                            size_t ws_offset = 0);
+// The same for n inputs of one shape at once (one launch).
 tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
                                     int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
-                                    tp_dtype dt, cudaStream_t st);
+                                    tp_dtype dt, cudaStream_t st, size_t ws_offset = 0);
 
 // LayerNorm (tp_layernorm.cu).
 tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,

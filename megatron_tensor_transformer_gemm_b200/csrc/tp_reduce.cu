@@ -477,13 +477,13 @@ tp_status launch_gather(const PtrArray& src, int n, void* dst, int64_t T, int64_
 }
 
 tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t cols, int64_t ld,
-                            float* out, int accumulate, tp_dtype dt, cudaStream_t st) {
+                            float* out, int accumulate, tp_dtype dt, cudaStream_t st, size_t ws_offset) {
   if (rows > 0) {  // one launch: the grouped form with one input
     PtrArray X{};
     MutPtrArray O{};
     X.p[0] = x;
     O.p[0] = out;
-    return launch_column_sum_grouped(plan, X, 1, rows, cols, ld, O, accumulate, dt, st);
+    return launch_column_sum_grouped(plan, X, 1, rows, cols, ld, O, accumulate, dt, st, ws_offset);
   }
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
@@ -494,9 +494,9 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
   const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
   splits = rows > 0 ? (rows + rps - 1) / rps : 1;
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(splits) * cols * sizeof(float), &ws);
+  tp_status s = workspace(plan, ws_offset + static_cast<size_t>(splits) * cols * sizeof(float), &ws);
   if (s != TP_OK) return s;
-  float* part = static_cast<float*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_offset);
   if (rows > 0) {
     dim3 grid(gx, static_cast<unsigned>(splits));
     if (dt == TP_BF16)
@@ -517,7 +517,7 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
 
 tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
                                     int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
-                                    tp_dtype dt, cudaStream_t st) {
+                                    tp_dtype dt, cudaStream_t st, size_t ws_offset) {
   if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "column sums of %d inputs", n);
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
@@ -528,9 +528,9 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
   const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
   splits = rows > 0 ? (rows + rps - 1) / rps : 0;
   void* ws = nullptr;
-  tp_status s = workspace(plan, static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float), &ws);
+  tp_status s = workspace(plan, ws_offset + static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float), &ws);
   if (s != TP_OK) return s;
-  float* part = static_cast<float*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_offset);
   if (rows > 0 && static_cast<int64_t>(gx) * n <= kPlanCounters) {
     // one launch: the last block of each column slab finishes it
     unsigned* ctr = nullptr;
