@@ -748,8 +748,9 @@ def measure_other(args, world, rank, local, sample_clocks=True):
             for lay in lays:
                 x = lay.forward(x, b, s_)
             g = dYd
-            for lay in reversed(lays):
-                g = lay.backward(g, b, s_)
+            for lay in reversed(lays):  # weight gradients joined once, after the last layer
+                g = lay.backward(g, b, s_, join=False)
+            tp.backward_join()
         name = "12-layer block stack fwd+bwd: hidden 512, MLP 2048, 8 heads x 64, tokens 8x512, p=4"
         core, core_flops = None, None
     for _ in range(args.warmup):

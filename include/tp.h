@@ -330,6 +330,23 @@ TP_API tp_status tp_attention_fwd(tp_plan* plan, int batch, int seq, const void*
  * every launch on `stream`. Calls on one plan must not overlap in time (they
  * share the plan's workspace). */
 
+/* Deferred backward (a scheduling option; the results are the same): with
+ * on != 0, the plan's bf16 tp_row_bwd and column backward calls run the
+ * activation gradient (dZ / dX) on `stream` and put the weight gradient (no K
+ * split) and the bias sums on the device's side stream, forked from `stream`
+ * at the call, and do NOT join them: dW and dbias are valid on a stream only
+ * after tp_backward_join on it. They read the call's inputs (dY, H, X, dZ)
+ * when they run, so those buffers must stay unchanged until the join, and the
+ * call's dW / dbias must not be read before it. Deferred bias sums use scratch
+ * of their own, so later calls of the same plan may run meanwhile. TP_ERR_ARG
+ * if plan is NULL. */
+TP_API tp_status tp_set_backward_defer(tp_plan* plan, int on);
+
+/* Make `stream` wait for all work issued so far on the current device's side
+ * stream (the deferred weight gradients and bias sums of every plan). An
+ * event wait: it returns at once on the host, and works inside a capture. */
+TP_API tp_status tp_backward_join(void* stream);
+
 /* Row layer backward for every shard ([TP-scratch] §四: the input gradient of
  * the row layer needs no reduction; dY is replicated).
  *   dY [T, hidden]; H[i] the row input of shard i; W[i] the row shard.

@@ -22,7 +22,7 @@ from __future__ import annotations
 
 import torch
 
-from .tp import Plan
+from .tp import Plan, backward_join
 
 
 def _empty(shape, dtype, device):
@@ -403,6 +403,9 @@ class TPLayer:
         self.h = hidden
         self.attn = TPAttention(hidden, heads, p, device, bias=True, fused=fused)
         self.mlp = TPMLP(hidden, ffn, p, "gelu", "bf16", device, bias=True, fused=fused)
+        # weight gradients and bias sums off the critical path (joined in backward)
+        self.attn.plan.set_backward_defer(True)
+        self.mlp.plan.set_backward_defer(True)
         self.ln = Plan(hidden, 0, 0, 1, "bf16", "none")  # LayerNorm / elementwise calls
         self.device = torch.device(device)
         dev = self.device
@@ -446,7 +449,10 @@ class TPLayer:
         self.mlp.forward(self.u2, residual=self.x1, out=self.y)
         return self.y
 
-    def backward(self, dy: torch.Tensor, batch: int, seq: int):
+    def backward(self, dy: torch.Tensor, batch: int, seq: int, join: bool = True):
+        """join=False leaves this layer's weight gradients and bias sums
+        running on the side stream (a caller that backpropagates several
+        layers joins once, with tp.backward_join(), before reading them)."""
         T = batch * seq
         ln = self.ln
         du2 = self.mlp.backward(dy)
@@ -456,6 +462,8 @@ class TPLayer:
         du1 = self.attn.backward(self.dx1, batch, seq)
         ln.layernorm_bwd(T, self.x, self.ln1_g, du1, self.m1, self.r1, self.dx,
                          self.dln1_g, self.dln1_b, dres=self.dx1)
+        if join:
+            backward_join()
         return self.dx
 
 

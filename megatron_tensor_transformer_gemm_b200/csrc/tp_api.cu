@@ -182,10 +182,10 @@ tp_status plan_counters(tp_plan* plan, cudaStream_t st, unsigned** out) {
     plan->cnt = nullptr;
   }
   void* p = nullptr;
-  s = cuda_status(cudaMalloc(&p, kPlanCounters * sizeof(unsigned)), "cudaMalloc(counters)");
+  s = cuda_status(cudaMalloc(&p, 2 * kPlanCounters * sizeof(unsigned)), "cudaMalloc(counters)");
   if (s != TP_OK) return s;
   // zero, and finished, before any kernel on any stream can use them
-  s = cuda_status(cudaMemsetAsync(p, 0, kPlanCounters * sizeof(unsigned), st), "cudaMemsetAsync(counters)");
+  s = cuda_status(cudaMemsetAsync(p, 0, 2 * kPlanCounters * sizeof(unsigned), st), "cudaMemsetAsync(counters)");
   if (s == TP_OK) s = cuda_status(cudaStreamSynchronize(st), "cudaStreamSynchronize(counters)");
   if (s != TP_OK) {
     cudaFree(p);
@@ -194,6 +194,33 @@ tp_status plan_counters(tp_plan* plan, cudaStream_t st, unsigned** out) {
   plan->cnt = static_cast<unsigned*>(p);
   plan->cnt_device = dev;
   *out = plan->cnt;
+  return TP_OK;
+}
+
+tp_status workspace2(tp_plan* plan, size_t bytes, void** out) {
+  int dev = 0;
+  tp_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != TP_OK) return s;
+  if (plan->ws2 && (plan->ws2_bytes < bytes || plan->ws2_device != dev)) {
+    cudaDeviceSynchronize();  // side-stream work may still use the old block
+    int cur = dev;
+    if (plan->ws2_device != dev) cudaSetDevice(plan->ws2_device);
+    cudaFree(plan->ws2);
+    if (plan->ws2_device != dev) cudaSetDevice(cur);
+    plan->ws2 = nullptr;
+    plan->ws2_bytes = 0;
+  }
+  if (!plan->ws2) {
+    size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+    s = cuda_status(cudaMalloc(&plan->ws2, want), "cudaMalloc(side workspace)");
+    if (s != TP_OK) {
+      plan->ws2 = nullptr;
+      return s;
+    }
+    plan->ws2_bytes = want;
+    plan->ws2_device = dev;
+  }
+  *out = plan->ws2;
   return TP_OK;
 }
 
@@ -506,6 +533,10 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   plan->ws_device = -1;
   plan->cnt = nullptr;
   plan->cnt_device = -1;
+  plan->defer_bwd = 0;
+  plan->ws2 = nullptr;
+  plan->ws2_bytes = 0;
+  plan->ws2_device = -1;
   *out = plan;
   return TP_OK;
 }
@@ -524,9 +555,28 @@ void tp_plan_destroy(tp_plan* plan) {
     cudaDeviceSynchronize();
     cudaFree(plan->cnt);
   }
+  if (plan->ws2) {
+    cudaSetDevice(plan->ws2_device);
+    cudaDeviceSynchronize();
+    cudaFree(plan->ws2);
+  }
   cudaSetDevice(cur);
   cudaGetLastError();
   delete plan;
+}
+
+tp_status tp_set_backward_defer(tp_plan* plan, int on) {
+  TP_TRY(check_plan(plan));
+  plan->defer_bwd = on ? 1 : 0;
+  return TP_OK;
+}
+
+tp_status tp_backward_join(void* stream) {
+  SideStream* sd = nullptr;
+  TP_TRY(side_stream(&sd));
+  cudaStream_t st = as_stream(stream);
+  TP_TRY(cuda_status(cudaEventRecord(sd->join, sd->s), "cudaEventRecord(join)"));
+  return cuda_status(cudaStreamWaitEvent(st, sd->join, 0), "cudaStreamWaitEvent(join)");
 }
 
 tp_status tp_plan_describe(const tp_plan* plan, char* buf, size_t n) {
@@ -1248,6 +1298,24 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
       g.ldd = k;
     }
   }
+  if (plan->defer_bwd && plan->dtype == TP_BF16 && (dW || dbias)) {
+    // Deferred: dH on the caller's stream, dW and db on the side stream,
+    // joined by tp_backward_join (dW without a K split: no shared scratch).
+    SideStream* sd = nullptr;
+    TP_TRY(side_stream(&sd));
+    TP_TRY(cuda_status(cudaEventRecord(sd->fork, st), "cudaEventRecord(fork)"));
+    TP_TRY(cuda_status(cudaStreamWaitEvent(sd->s, sd->fork, 0), "cudaStreamWaitEvent(fork)"));
+    TP_TRY(run_gemm(plan, b, st));
+    if (dW) TP_TRY(launch_gemm_bf16(w, sd->s));
+    if (dbias) {
+      PtrArray X{};
+      MutPtrArray O{};
+      X.p[0] = dY;
+      O.p[0] = dbias;
+      TP_TRY(launch_column_sum_deferred(plan, X, 1, T, h, h, O, plan->dtype, sd->s));
+    }
+    return TP_OK;
+  }
   // dH beside the weight gradient (joined when this call returns), or before it
   std::unique_ptr<SideGemm> side;
   if (dW && concurrent_bwd(plan, b, w)) {
@@ -1337,6 +1405,20 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
       d.rows_per_out = T / p;
       for (int j = 0; j < p; ++j) d.out_seq[j] = dX_out[j];
     }
+  }
+  if (plan->defer_bwd && plan->dtype == TP_BF16 && (dW || dbias)) {
+    // Deferred: dX on the caller's stream, dW and db on the side stream,
+    // joined by tp_backward_join (dW without a K split: no shared scratch).
+    SideStream* sd = nullptr;
+    TP_TRY(side_stream(&sd));
+    TP_TRY(cuda_status(cudaEventRecord(sd->fork, st), "cudaEventRecord(fork)"));
+    TP_TRY(cuda_status(cudaStreamWaitEvent(sd->s, sd->fork, 0), "cudaStreamWaitEvent(fork)"));
+    if (dX_out) TP_TRY(run_gemm(plan, d, st));
+    if (dW) TP_TRY(launch_gemm_bf16(w, sd->s));
+    if (dbias)
+      TP_TRY(launch_column_sum_deferred(plan, to_arr(dZ, p), p, T, n, n,
+                                        to_marr(reinterpret_cast<void* const*>(dbias), p), plan->dtype, sd->s));
+    return TP_OK;
   }
   // dX beside the weight gradient (joined when this call returns), or after it
   std::unique_ptr<SideGemm> side;

@@ -24,9 +24,16 @@ struct tp_plan {
   size_t ws_bytes;
   int ws_device;
   // Arrival counters of single-launch reductions (zero at rest: the last
-  // block of each reduction sets its counter back), allocated on first need.
+  // block of each reduction sets its counter back), allocated on first need;
+  // the upper half serves work deferred to the side stream.
   unsigned* cnt;
   int cnt_device;
+  // Deferred backward (tp_set_backward_defer): weight gradients and bias sums
+  // run on the device's side stream, with scratch of their own (ws2).
+  int defer_bwd;
+  void* ws2;
+  size_t ws2_bytes;
+  int ws2_device;
 };
 
 namespace tpi {
@@ -82,6 +89,9 @@ tp_status workspace(tp_plan* plan, size_t bytes, void** out);
 // while `st` is being captured).
 constexpr int kPlanCounters = 4096;
 tp_status plan_counters(tp_plan* plan, cudaStream_t st, unsigned** out);
+// Scratch for the work a deferred backward puts on the side stream (never
+// shared with the caller's stream).
+tp_status workspace2(tp_plan* plan, size_t bytes, void** out);
 
 // Validation helpers: each returns TP_OK or records an error.
 tp_status check_ptr(const void* p, const char* name);
@@ -116,6 +126,11 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
 tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
                                     int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
                                     tp_dtype dt, cudaStream_t st, size_t ws_offset = 0);
+// Column sums deferred to the side stream: partials in workspace2, counters in
+// the upper half of the plan's counters.
+tp_status launch_column_sum_deferred(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
+                                     int64_t cols, int64_t ld, const MutPtrArray& out, tp_dtype dt,
+                                     cudaStream_t st);
 
 // LayerNorm (tp_layernorm.cu).
 tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,

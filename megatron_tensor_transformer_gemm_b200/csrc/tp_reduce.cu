@@ -515,9 +515,11 @@ tp_status launch_column_sum(tp_plan* plan, const void* x, int64_t rows, int64_t 
   return after_launch("column_sum/pass2");
 }
 
-tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
-                                    int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
-                                    tp_dtype dt, cudaStream_t st, size_t ws_offset) {
+// The grouped column sums with their scratch chosen by the caller: `deferred`
+// takes the side workspace and the upper half of the plan's counters.
+static tp_status column_sum_grouped_impl(tp_plan* plan, const PtrArray& x, int n, int64_t rows, int64_t cols,
+                                         int64_t ld, const MutPtrArray& out, int accumulate, tp_dtype dt,
+                                         cudaStream_t st, size_t ws_offset, bool deferred) {
   if (n < 1 || n > TP_MAX_SHARDS) return fail(TP_ERR_ARG, "column sums of %d inputs", n);
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
@@ -527,8 +529,9 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
   splits = std::min<int64_t>(splits, 1024);
   const int64_t rps = rows > 0 ? (rows + splits - 1) / splits : 1;
   splits = rows > 0 ? (rows + rps - 1) / rps : 0;
+  const size_t bytes = ws_offset + static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float);
   void* ws = nullptr;
-  tp_status s = workspace(plan, ws_offset + static_cast<size_t>(std::max<int64_t>(splits, 1)) * cols * n * sizeof(float), &ws);
+  tp_status s = deferred ? workspace2(plan, bytes, &ws) : workspace(plan, bytes, &ws);
   if (s != TP_OK) return s;
   float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_offset);
   if (rows > 0 && static_cast<int64_t>(gx) * n <= kPlanCounters) {
@@ -536,6 +539,7 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
     unsigned* ctr = nullptr;
     s = plan_counters(plan, st, &ctr);
     if (s != TP_OK) return s;
+    if (deferred) ctr += kPlanCounters;
     dim3 grid(gx, static_cast<unsigned>(splits), static_cast<unsigned>(n));
     if (dt == TP_BF16)
       (void)tpi::launch(colsum_fused<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, ld, rows, vpr, rps, part, cols,
@@ -556,6 +560,18 @@ tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int
   }
   (void)tpi::launch(colsum_grouped_pass2, dim3(dim3(static_cast<unsigned>((cols + 255) / 256), static_cast<unsigned>(n))), dim3(256), 0, st, part, static_cast<int>(splits), cols, out, accumulate);
   return after_launch("column_sum_grouped/pass2");
+}
+
+tp_status launch_column_sum_grouped(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
+                                    int64_t cols, int64_t ld, const MutPtrArray& out, int accumulate,
+                                    tp_dtype dt, cudaStream_t st, size_t ws_offset) {
+  return column_sum_grouped_impl(plan, x, n, rows, cols, ld, out, accumulate, dt, st, ws_offset, false);
+}
+
+tp_status launch_column_sum_deferred(tp_plan* plan, const PtrArray& x, int n, int64_t rows,
+                                     int64_t cols, int64_t ld, const MutPtrArray& out, tp_dtype dt,
+                                     cudaStream_t st) {
+  return column_sum_grouped_impl(plan, x, n, rows, cols, ld, out, 0, dt, st, 0, true);
 }
 
 }  // namespace tpi

@@ -89,6 +89,8 @@ _SIGS = {
     "tp_row_fwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _vp, _vpp, _vpp, _vp]),
     "tp_column_bwd_reduce": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp]),
     "tp_column_bwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_set_backward_defer": (_int, [_plan_p, _int]),
+    "tp_backward_join": (_int, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -107,6 +109,12 @@ def check(status: int, func: str) -> None:
 
 def launch_count(reset: bool = False) -> int:
     return int(lib.tp_launch_count(1 if reset else 0))
+
+
+def backward_join(stream=None) -> None:
+    """tp_backward_join: the stream waits for the deferred weight gradients
+    and bias sums of every plan (see Plan.set_backward_defer)."""
+    check(lib.tp_backward_join(_stream(stream)), "tp_backward_join")
 
 
 def _ptr(t) -> int | None:
@@ -309,6 +317,11 @@ class Plan:
     def attention_bwd(self, batch, seq, QKV, O, dO, LSE, dQKV, stream=None):
         check(lib.tp_attention_bwd(self._h, batch, seq, _arr(QKV), _arr(O), _arr(dO), _arr(LSE),
                                    _arr(dQKV), _stream(stream)), "tp_attention_bwd")
+
+    def set_backward_defer(self, on: bool = True):
+        """tp_set_backward_defer: this plan's backward calls leave their weight
+        gradients and bias sums on the side stream until backward_join()."""
+        check(lib.tp_set_backward_defer(self._h, 1 if on else 0), "tp_set_backward_defer")
 
     def column_sum(self, rows, cols, x, out, accumulate=False, stream=None):
         check(lib.tp_column_sum(self._h, rows, cols, _ptr(x), _ptr(out), 1 if accumulate else 0,

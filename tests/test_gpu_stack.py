@@ -163,3 +163,43 @@ def test_stack_step_replayed_as_cuda_graph_matches_eager():
     assert torch.equal(out["y"], y_eager)
     assert torch.equal(out["dx"], dx_eager)
     assert torch.equal(lays[0].mlp.dW1[0], w_eager)
+
+
+def test_deferred_weight_gradients_joined_once():
+    """TPLayer leaves its weight gradients and bias sums on the side stream
+    (tp_set_backward_defer). Backpropagating three layers with one join at the
+    end gives the gradients, bit for bit, of joining after every layer, and,
+    within the bf16 tolerance, those of the plans with deferral off (every
+    backward GEMM joined inside its call)."""
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from gpu_helpers import TOL_BF16, assert_close
+    X, layers, dY = tp_synth.draw_block_stack(3, BATCH, SEQ, H_, F_, torch.bfloat16, seed=9,
+                                              ln_affine_random=True)
+    lays = [_gpu_layer(prm, 2) for prm in layers]
+
+    def run(join_each):
+        x = dev(X)
+        for lay in lays:
+            x = lay.forward(x, BATCH, SEQ)
+        g = dev(dY)
+        for lay in reversed(lays):
+            g = lay.backward(g, BATCH, SEQ, join=join_each)
+        if not join_each:
+            tp.backward_join()
+        torch.cuda.synchronize()
+        out = [g.clone()]
+        for lay in lays:
+            out += [t.clone() for t in (lay.mlp.dW1[0], lay.mlp.dW2[1], lay.attn.dWqkv[1], lay.attn.dWo[0])]
+            out += [lay.mlp.db2.clone()[None, :], lay.attn.dbo.clone()[None, :], lay.mlp.db1[1].clone()[None, :]]
+        return out
+
+    each = run(True)
+    once = run(False)
+    for a, b in zip(each, once):
+        assert torch.equal(a, b)
+    for lay in lays:
+        lay.attn.plan.set_backward_defer(False)
+        lay.mlp.plan.set_backward_defer(False)
+    immediate = run(True)
+    for i, (a, b) in enumerate(zip(each, immediate)):
+        assert_close(a, host(b).astype(np.float64), TOL_BF16, f"gradient {i}")
