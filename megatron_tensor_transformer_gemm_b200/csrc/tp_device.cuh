@@ -396,12 +396,28 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t mask) 
 }
 
 // ----------------------------------------------------------------- numerics
+// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
+// 7.1.26 (absolute error <= 1.5e-7 for x >= 0; odd symmetry for x < 0), given
+// e = exp(-x^2): erf(|x|) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) e,
+// t = 1 / (1 + p |x|).
+__device__ __forceinline__ float erf_as(float x, float e) {
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, fabsf(x), 1.0f));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f),
+               0.254829592f);
+  return copysignf(fmaf(-poly, e, 1.0f), x);
+}
+// GELU(z) = z Phi(z) = z (1 + erf(z / sqrt 2)) / 2; GELU'(z) = Phi(z) + z phi(z).
+// Both share exp(-z^2 / 2): the erf's exp(-x^2) at x = z / sqrt 2 is the
+// density's exponential, so one fast exponential serves both terms.
 __device__ __forceinline__ float gelu_f(float z) {
-  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+  const float x = z * 0.70710678118654752f;
+  return 0.5f * z * (1.0f + erf_as(x, __expf(-x * x)));
 }
 __device__ __forceinline__ float gelu_grad_f(float z) {
-  return 0.5f * (1.0f + erff(z * 0.70710678118654752f)) +
-         z * 0.39894228040143268f * expf(-0.5f * z * z);
+  const float x = z * 0.70710678118654752f;
+  const float e = __expf(-x * x);
+  return 0.5f * (1.0f + erf_as(x, e)) + z * 0.39894228040143268f * e;
 }
 __device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + expf(-z)); }
 // The logistic sigmoid from the hardware exponential and an approximate
