@@ -251,7 +251,7 @@ def run_dist(args, world, rank, local):
     dev = torch.device("cuda", local)
     T = args.tokens
     inp = tp_synth.draw_mlp(T, HIDDEN, FFN, "swiglu", torch.bfloat16, seed=0)  # replicated input
-    m = DistTPMLP(HIDDEN, FFN, P, "swiglu", device=dev)
+    m = DistTPMLP(HIDDEN, FFN, P, "swiglu", device=dev, comm=args.comm)
     m.load_weights(inp.W1, inp.W2)
     X_h, dY_h = inp.X.pin_memory(), inp.dY.pin_memory()
     del inp
@@ -259,7 +259,9 @@ def run_dist(args, world, rank, local):
     m.alloc(T)
     stream = torch.cuda.current_stream()
     pl = m.plan
-    gemm_calls = ("column_fwd", "row_fwd_reduce", "row_bwd", "column_bwd_reduce")
+    peer = args.comm == "peer"
+    gemm_calls = ("column_fwd", "row_fwd_push_peer", "row_bwd", "column_bwd_push_peer") if peer else \
+        ("column_fwd", "row_fwd_reduce", "row_bwd", "column_bwd_reduce")
     orig = {n: getattr(pl, n) for n in gemm_calls}
     gemm_ev, comm_ev = [], []
 
@@ -276,11 +278,15 @@ def run_dist(args, world, rank, local):
 
     import megatron_tensor_transformer_gemm_b200.dist as D
     orig_sum = D.sum_over_ranks
+    orig_peer = m.peer.reduce if peer else None
 
     def step(instrument=False):
         for n in gemm_calls:
             setattr(pl, n, timed(orig[n], gemm_ev) if instrument else orig[n])
-        D.sum_over_ranks = timed(orig_sum, comm_ev) if instrument else orig_sum
+        if peer:   # the reduce + wait steps (the pushes are inside the GEMMs)
+            m.peer.reduce = timed(orig_peer, comm_ev) if instrument else orig_peer
+        else:
+            D.sum_over_ranks = timed(orig_sum, comm_ev) if instrument else orig_sum
         m.forward(X)
         m.backward(dY)
 
@@ -306,6 +312,8 @@ def run_dist(args, world, rank, local):
     for n in gemm_calls:
         setattr(pl, n, orig[n])
     D.sum_over_ranks = orig_sum
+    if peer:
+        m.peer.reduce = orig_peer
     flops = m.flops(T)
     ms = max_over_ranks(s0.elapsed_time(s1), world)
     value = flops * args.steps / (ms / 1e3) / 1e12
@@ -337,6 +345,9 @@ def run_dist(args, world, rank, local):
                "h2d_bytes_per_step": 2 * nb * world, "d2h_bytes_per_step": 2 * nb * world,
                "ms_per_step": e2e_ms / args.steps}
     status = tp.device_status()
+    barrier(world)   # no rank frees its peer memory while another may still write into it
+    if peer:
+        m.close_peer()
     if rank != 0:
         return 0
     out = {
@@ -346,12 +357,15 @@ def run_dist(args, world, rank, local):
         "data": "synthetic (seeded tp_synth draws: X, dY ~ N(0,1), W ~ N(0,0.02))",
         "config": {"workload": WORKLOAD.replace("on one GPU", f"over {world} GPUs"), "hidden": HIDDEN,
                    "ffn": FFN, "tokens": T, "p": P, "act": "swiglu", "global_batch": 8, "seq_len": 4096,
-                   "parallelism": f"tp{world}: {P // world} of the {P} shards per GPU, NCCL all-reduce",
+                   "parallelism": f"tp{world}: {P // world} of the {P} shards per GPU, "
+                                  + ("peer-memory all-reduce" if peer else "NCCL all-reduce"),
                    "l2": "inputs larger than L2 (X and dY 268 MB each); no flush"},
         "roofline": {"bound": "tensor", "kernel": "tp_gemm_kernel (tcgen05)", "achieved": gemm_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops"],
                      "peak_kind": f"bf16 burst ({peaks['source']}), per GPU", "traffic": None},
-        "comm": {"collective": "NCCL all-reduce of Y and dX ([T, 4096] bf16) per step",
+        "comm": {"collective": ("peer memory: row blocks pushed from the GEMM epilogues into the owners' "
+                                "receive buffers, reduced once and pushed to every rank (all-reduce of Y and dX)")
+                 if peer else "NCCL all-reduce of Y and dX ([T, 4096] bf16) per step",
                  "ms_per_step": comm_ms / args.steps,
                  "bytes_per_rank_per_step": 2 * 2 * (world - 1) / world * T * HIDDEN * 2},
         "e2e": e2e, "gpu_launches": launches, "clocks": clk, "device_status": status,
@@ -829,6 +843,97 @@ def measure_other(args, world, rank, local, sample_clocks=True):
     return out
 
 
+def run_peer_emul(args, world, rank, local):
+    """The peer-memory all-reduce of the 7B row layer (hidden 4096, ffn 11008,
+    tokens 8x4096) with 8 ranks of one shard each emulated on this GPU: every
+    rank's receive buffer, flags and output are local, and each step is taken
+    for all 8 ranks before the next (push GEMMs, then reduces, then waits), so
+    no kernel waits for a later launch. Times each step over the 8 ranks
+    beside the single-GPU fused row GEMM of the same FLOPs; the reduce's
+    algorithmic bytes per rank: 8 slots read + 8 output blocks written."""
+    import torch
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.dist import bf16_view
+
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    T, h, f, W = args.tokens, HIDDEN, FFN, P
+    t, fp = T // W, f // W
+    g = torch.Generator(device="cpu").manual_seed(2000 + rank)
+    H = [torch.randn(T, fp, generator=g).to(torch.bfloat16).to(dev) for _ in range(W)]
+    W2 = [(torch.randn(h, fp, generator=g) * 0.02).to(torch.bfloat16).to(dev) for _ in range(W)]
+    fused = tp.Plan(h, f, 0, W, "bf16", "none")
+    Y = torch.empty(T, h, dtype=torch.bfloat16, device=dev)
+    plans = [tp.Plan(h, fp, 0, 1, "bf16", "none") for _ in range(W)]
+    mem, outs = [], []
+    try:
+        for _ in range(W):
+            mem.append(tp.peer_alloc(tp.PEER_FLAG_BYTES + 2 * T * h)[0])
+            outs.append(tp.peer_alloc(2 * T * h)[0])
+        grp = [tp.peer_group(W, r, T * h, mem, [q + tp.PEER_FLAG_BYTES for q in mem]) for r in range(W)]
+        blocks = [[q + r * t * h * 2 for q in outs] for r in range(W)]
+        epoch = 1
+        steps = {
+            "fused row GEMM, one GPU (tp_row_fwd_reduce, 8 shards in one accumulator)":
+                lambda: fused.row_fwd_reduce("mlp", T, H, W2, None, None, Y),
+            "push: 8 x tp_gemm_kernel (1 shard each, row blocks stored into 8 receive buffers) + peer_signal":
+                lambda: [plans[r].row_fwd_push_peer("mlp", T, [H[r]], [W2[r]], grp[r], epoch) for r in range(W)],
+            "reduce: 8 x peer_reduce_kernel (8 slots summed, block pushed to 8 outputs) + peer_signal":
+                lambda: [tp.peer_reduce(grp[r], T, h, None, None, blocks[r], epoch) for r in range(W)],
+            "wait: 8 x peer_wait_kernel":
+                lambda: [tp.peer_wait(grp[r], epoch) for r in range(W)],
+        }
+        for fn in steps.values():
+            for _ in range(args.warmup):
+                fn()
+        torch.cuda.synchronize()
+        if tp.lib.tp_get_device_status(None, None) != 0:
+            raise SystemExit("a peer wait gave up in the warm-up")
+        clocks = ClockSampler(local)
+        clocks.start()
+        tp.launch_count(reset=True)
+        per = []
+        for name, fn in steps.items():
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            per.append({"step": name, "ms": e0.elapsed_time(e1) / args.steps})
+        launches = tp.launch_count(reset=True)
+        clk = clocks.stop()
+        status = tp.device_status()
+    finally:
+        torch.cuda.synchronize()
+        for q in mem + outs:
+            tp.peer_free(q)
+    flops = 2.0 * T * h * f
+    red_bytes = W * (W * t * h * 2 + W * t * h * 2)
+    per[0]["tflops"] = flops / (per[0]["ms"] / 1e3) / 1e12
+    per[1]["tflops"] = flops / (per[1]["ms"] / 1e3) / 1e12
+    per[2]["bytes"] = red_bytes
+    per[2]["gbs"] = red_bytes / (per[2]["ms"] / 1e3) / 1e9
+    if rank != 0:
+        return 0
+    gbs = per[2]["gbs"]
+    print(json.dumps({
+        "metric": "peer all-reduce steps of the 7B row layer, 8 ranks emulated on 1 B200: reduce GB/s",
+        "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(x["ms"] for x in per[1:]), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch draws)",
+        "config": {"workload": f"row layer hidden {h}, ffn {f}, tokens {T}, 8 ranks x 1 shard, emulated on one GPU "
+                               "(peer stores land in local HBM; NVLink is not exercised)",
+                   "l2": "every buffer set larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "kernel": "peer_reduce_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"HBM copy ({peaks['source']})",
+                     "traffic": None},
+        "steps_timed": per, "gpu_launches": launches, "clocks": clk, "device_status": status}), flush=True)
+    return 0
+
+
 def run_hbm(args, world, rank, local):
     """Device-timed HBM throughput of the memory-bound rows, each kernel timed
     on its own over the same buffers (algorithmic bytes / event time; sp_hbm:
@@ -1010,12 +1115,15 @@ def main():
                     help="sum over shards inside the GEMMs (fused), via p partials + reduce, "
                          "or partials with each token block's reduce overlapped with the next "
                          "block's GEMM (overlap)")
-    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm", "sp_hbm"],
+    ap.add_argument("--workload", choices=["mlp7b", "attn", "sp", "stack", "vocab", "norm", "sp_hbm", "peer"],
                     default="mlp7b",
                     help="mlp7b (the metric's workload) or another config of the suite")
     ap.add_argument("--replicas", action="store_true",
                     help="N > 1: one independent replica per GPU (weak scaling) instead of the "
                          "shards split over the GPUs")
+    ap.add_argument("--comm", choices=["nccl", "peer"], default="nccl",
+                    help="N > 1, mlp7b: the all-reduces of Y and dX through NCCL, or through libtp's "
+                         "peer-memory steps (push from the GEMM epilogue, reduce, wait)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph (other workloads)")
     args = ap.parse_args()
@@ -1031,6 +1139,8 @@ def main():
             run_ours(args, world, rank, local)
     elif args.workload in ("vocab", "norm", "sp_hbm"):
         rc = run_hbm(args, world, rank, local)
+    elif args.workload == "peer":
+        rc = run_peer_emul(args, world, rank, local)
     else:
         rc = run_other(args, world, rank, local)
     if world > 1:

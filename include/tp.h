@@ -479,6 +479,90 @@ TP_API tp_status tp_column_sum(tp_plan* plan, int64_t rows, int64_t cols, const 
 TP_API tp_status tp_column_sum_static(int64_t rows, int64_t cols, tp_dtype dtype, const void* x,
                                       float* out, int accumulate, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Across GPUs over peer memory: the p shards split over `world` ranks (one
+ * process per GPU), every rank's buffers mapped into every other rank's
+ * address space with CUDA IPC. The row layer's all-reduce ([TP-blog] §4.1:
+ * each GPU holds a partial sum and every GPU needs the full result) is split
+ * into a reduce-scatter and an all-gather ([TP-wiki] 序列维度的补充：
+ * Megatron-SP: all-reduce = reduce-scatter + all-gather at the same traffic),
+ * and the reduce-scatter's transfer is fused into the GEMM that produces the
+ * partial sum. Three asynchronous calls on the caller's stream, each taken by
+ * every rank with the same `epoch` (a counter that starts at 1 and grows by
+ * one per all-reduce; the group's flag words start at zero):
+ *   1. push    tp_row_fwd_push_peer / tp_column_bwd_push_peer: the GEMM sums
+ *              this rank's shards in its accumulator and its epilogue stores
+ *              row block j (rows [j*T/world, (j+1)*T/world)) straight into
+ *              rank j's receive buffer, slot <rank>, with plain stores through
+ *              the peer mapping; then this rank's "arrived" flag is raised on
+ *              every rank.
+ *   2. reduce  tp_peer_reduce: waits until every rank's block has arrived,
+ *              sums the world slots in rank order in fp32, adds bias and
+ *              residual once, rounds once, stores the block to each of the
+ *              n_out destinations (every rank's output at this rank's rows:
+ *              the all-gather; or this rank's sequence shard only: the
+ *              Megatron-SP reduce-scatter), then raises this rank's "done"
+ *              flag on every rank.
+ *   3. wait    tp_peer_wait: waits until every rank's "done" flag is up: all
+ *              of this rank's output blocks have been written, and every rank
+ *              has finished reading its receive buffer, so the next push may
+ *              begin.
+ * Waits are bounded (tp_peer_set_wait_limit, default 5 s): a rank that never
+ * arrives makes the waiting kernel set TP_ERR_TIMEOUT in the device status
+ * word and return. bf16 plans only. No call here issues a TMA load, and no
+ * library kernel is given a peer's memory. */
+#define TP_PEER_HANDLE_BYTES 64
+#define TP_PEER_FLAG_WORDS (2 * TP_MAX_SHARDS) /* [0, MAX): arrived from rank s; [MAX, 2 MAX): done */
+#define TP_PEER_FLAG_BYTES 256                  /* flag words padded to keep what follows aligned */
+
+typedef struct tp_peer_group {
+  int world;                      /* ranks, 1..TP_MAX_SHARDS */
+  int rank;                       /* this rank, 0..world-1 */
+  int64_t recv_elems;             /* capacity of each receive buffer, in elements */
+  uint32_t* flags[TP_MAX_SHARDS]; /* rank d's TP_PEER_FLAG_WORDS flag words (device, zeroed) */
+  void* recv[TP_MAX_SHARDS];      /* rank d's receive buffer (device): world slots of [T/world, hidden] */
+} tp_peer_group;
+
+/* Device memory that other processes can map: `bytes` (> 0) from cudaMalloc
+ * on the current device, zero-filled, its IPC handle written to `handle`
+ * (TP_PEER_HANDLE_BYTES host bytes). Free with tp_peer_free. */
+TP_API tp_status tp_peer_alloc(size_t bytes, void** ptr, void* handle);
+TP_API tp_status tp_peer_free(void* ptr);
+/* Map another process's tp_peer_alloc memory (its handle bytes) into this
+ * process; unmap with tp_peer_close. A handle from this same process is
+ * refused by CUDA (TP_ERR_CUDA): a rank uses its own pointer directly. */
+TP_API tp_status tp_peer_open(const void* handle, void** ptr);
+TP_API tp_status tp_peer_close(void* ptr);
+/* Wait limit of the peer waits in nanoseconds, (0, 60e9]; 0 restores the
+ * default. Applies to launches made after the call, from any thread. */
+TP_API tp_status tp_peer_set_wait_limit(int64_t ns);
+
+/* Step 1 for the row layer: Y_r = sum over this rank's p shards of H[i]
+ * W[i]^T (fp32 accumulator, rounded once to bf16), row block j pushed into
+ * g->recv[j] slot g->rank ([T/world, hidden] at element offset
+ * rank*(T/world)*hidden). No bias or residual here (step 2 adds them once).
+ * T % world == 0 and T*hidden <= g->recv_elems. */
+TP_API tp_status tp_row_fwd_push_peer(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                                      const void* const* W, const tp_peer_group* g, uint32_t epoch,
+                                      void* stream);
+/* Step 1 for the column layer's backward ([TP-scratch] §四: the input
+ * gradient is all-reduced): dW[i], dbias[i] as in tp_column_bwd, and dX_r =
+ * sum over this rank's shards of dZ[i] W[i] pushed by row block as above. */
+TP_API tp_status tp_column_bwd_push_peer(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                                         const void* const* dZ, const void* const* W, void* const* dW,
+                                         float* const* dbias, const tp_peer_group* g, uint32_t epoch,
+                                         void* stream);
+/* Step 2: out[k] [T/world, hidden] = sum_{s<world} slot s of this rank's
+ * receive buffer (fp32, in order 0..world-1) + bias [hidden] (NULL ok) +
+ * residual [T/world, hidden] (this rank's rows; NULL ok), rounded to bf16,
+ * for k < n_out (1 <= n_out <= TP_MAX_SHARDS; out is a host array of device
+ * pointers, local or peer). hidden % 8 == 0. */
+TP_API tp_status tp_peer_reduce(const tp_peer_group* g, int64_t T, int hidden, const void* bias,
+                                const void* residual, int n_out, void* const* out, uint32_t epoch,
+                                void* stream);
+/* Step 3: the stream waits (on the device) for every rank's step 2. */
+TP_API tp_status tp_peer_wait(const tp_peer_group* g, uint32_t epoch, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -254,12 +254,6 @@ tp_status check_row_bytes(int64_t cols, tp_dtype t, const char* name) {
 
 using namespace tpi;
 
-#define TP_TRY(expr)                   \
-  do {                                 \
-    tp_status _s = (expr);             \
-    if (_s != TP_OK) return _s;        \
-  } while (0)
-
 namespace {
 
 tp_status check_plan(const tp_plan* plan) {
@@ -868,10 +862,36 @@ tp_status tp_row_fwd_partial(tp_plan* plan, tp_which which, int64_t T, const voi
 
 // Row GEMM with the shard sum fused (K-concatenated over shards), writing the
 // full output or (scatter) its sequence shards.
+// With a peer group (peer != NULL, scatter false, no bias or residual) row
+// block j goes to slot <rank> of rank j's receive buffer with plain stores.
+static tp_status check_peer_push(const tp_plan* plan, const tp_peer_group* g, int64_t T) {
+  TP_TRY(check_peer_group(g));
+  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "peer pushes need a bf16 plan");
+  if (T % g->world)
+    return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by world = %d", (long long)T, g->world);
+  if (T * plan->hidden > g->recv_elems)
+    return fail(TP_ERR_ARG, "T x hidden = %lld exceeds the receive buffers (%lld elements)",
+                (long long)(T * plan->hidden), (long long)g->recv_elems);
+  return TP_OK;
+}
+
+static void peer_push_targets(GemmBatch& b, const tp_peer_group* g, int64_t T, int h) {
+  const int64_t t = T / g->world;
+  b.scatter_n = g->world;
+  b.rows_per_out = t;
+  b.plain_stores = true;
+  for (int j = 0; j < g->world; ++j) {
+    b.out_seq[j] = static_cast<__nv_bfloat16*>(g->recv[j]) + static_cast<int64_t>(g->rank) * t * h;
+    b.res_seq[j] = nullptr;
+  }
+  b.g[0].D = b.out_seq[0];
+}
+
 static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
                                        const void* const* H, const void* const* W, const void* bias,
                                        const void* residual, const void* const* residual_seq,
-                                       void* Y, void* const* Y_seq, bool scatter, cudaStream_t st) {
+                                       void* Y, void* const* Y_seq, bool scatter, cudaStream_t st,
+                                       const tp_peer_group* peer = nullptr) {
   TP_TRY(check_plan(plan));
   TP_TRY(check_T(T));
   int k = 0;
@@ -882,7 +902,9 @@ static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
   if (bias) TP_TRY(check_ptr(bias, "bias"));
   TP_TRY(check_row_bytes(k, plan->dtype, "row shard width"));
   TP_TRY(check_row_bytes(h, plan->dtype, "hidden"));
-  if (scatter) {
+  if (peer) {
+    TP_TRY(check_peer_push(plan, peer, T));
+  } else if (scatter) {
     if (T % p) return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by p = %d", (long long)T, p);
     TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(Y_seq), p, "Y_seq", false));
     TP_TRY(check_ptrs(residual_seq, p, "residual_seq", true));
@@ -910,7 +932,9 @@ static tp_status row_fwd_reduce_common(tp_plan* plan, tp_which which, int64_t T,
   b.g[0].bias = bias;
   b.g[0].aux = scatter ? nullptr : residual;
   b.g[0].ldaux = h;
-  if (scatter) {
+  if (peer) {
+    peer_push_targets(b, peer, T, h);
+  } else if (scatter) {
     b.scatter_n = p;
     b.rows_per_out = T / p;
     for (int j = 0; j < p; ++j) {
@@ -934,6 +958,15 @@ tp_status tp_row_fwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_t T
                                         void* const* Y_seq, void* stream) {
   return row_fwd_reduce_common(plan, which, T, H, W, bias, nullptr, residual_seq, nullptr, Y_seq,
                                true, as_stream(stream));
+}
+
+tp_status tp_row_fwd_push_peer(tp_plan* plan, tp_which which, int64_t T, const void* const* H,
+                               const void* const* W, const tp_peer_group* g, uint32_t epoch,
+                               void* stream) {
+  const cudaStream_t st = as_stream(stream);
+  TP_TRY(row_fwd_reduce_common(plan, which, T, H, W, nullptr, nullptr, nullptr, nullptr, nullptr,
+                               false, st, g));
+  return launch_peer_signal(g, g->rank, epoch, st);
 }
 
 static tp_status reduce_common(tp_plan* plan, int64_t T, int n, const void* const* P,
@@ -1334,11 +1367,12 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
 }
 
 // dX mode: 0 = partials (dX_out[i] per shard), 1 = summed (dX_out[0] full),
-// 2 = summed and scattered by sequence (dX_out[j] = rows of shard j).
+// 2 = summed and scattered by sequence (dX_out[j] = rows of shard j),
+// 3 = summed and pushed by row block into the peer group's receive buffers.
 static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, const void* X,
                                    const void* const* dZ, const void* const* W, void* const* dW,
                                    float* const* dbias, void* const* dX_out, int mode,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const tp_peer_group* peer = nullptr) {
   TP_TRY(check_plan(plan));
   TP_TRY(check_T(T));
   ColShape cs{};
@@ -1350,7 +1384,8 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dW), p, "dW", true));
   TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dbias), p, "dbias", true));
   const int nout = mode == 1 ? 1 : p;
-  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX_out), nout, "dX", mode == 0));
+  if (mode == 3) TP_TRY(check_peer_push(plan, peer, T));
+  else TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(dX_out), nout, "dX", mode == 0));
   if (mode == 2 && T % p)
     return fail(TP_ERR_DIVISIBILITY, "T = %lld is not divisible by p = %d", (long long)T, p);
   if (dW) TP_TRY(check_ptr(X, "X"));
@@ -1380,7 +1415,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     }
   }
   GemmBatch d{};
-  if (dX_out) {
+  if (dX_out || mode == 3) {
     // dX_i [T, h] = dZ_i W_i: A = dZ_i (K-major), B(c, j) = W_i[j, c] (MN-major).
     d.n = p;
     d.a_mn = false;
@@ -1397,15 +1432,18 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
       g.lda = n;
       g.B = W[i];
       g.ldb = h;
-      g.D = mode == 0 ? dX_out[i] : dX_out[0];
+      g.D = mode == 3 ? nullptr : mode == 0 ? dX_out[i] : dX_out[0];
       g.ldd = h;
     }
     if (mode == 2) {
       d.scatter_n = p;
       d.rows_per_out = T / p;
       for (int j = 0; j < p; ++j) d.out_seq[j] = dX_out[j];
+    } else if (mode == 3) {
+      peer_push_targets(d, peer, T, h);
     }
   }
+  const bool has_dx = dX_out || mode == 3;
   if (plan->defer_bwd && plan->dtype == TP_BF16 && (dW || dbias)) {
     // Deferred: dX on the caller's stream, dW and db on the side stream,
     // joined by tp_backward_join (dW without a K split: no shared scratch).
@@ -1413,7 +1451,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     TP_TRY(side_stream(&sd));
     TP_TRY(cuda_status(cudaEventRecord(sd->fork, st), "cudaEventRecord(fork)"));
     TP_TRY(cuda_status(cudaStreamWaitEvent(sd->s, sd->fork, 0), "cudaStreamWaitEvent(fork)"));
-    if (dX_out) TP_TRY(run_gemm(plan, d, st));
+    if (has_dx) TP_TRY(run_gemm(plan, d, st));
     if (dW) TP_TRY(launch_gemm_bf16(w, sd->s));
     if (dbias)
       TP_TRY(launch_column_sum_deferred(plan, to_arr(dZ, p), p, T, n, n,
@@ -1422,7 +1460,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   }
   // dX beside the weight gradient (joined when this call returns), or after it
   std::unique_ptr<SideGemm> side;
-  if (dW && dX_out && concurrent_bwd(plan, d, w)) {
+  if (dW && has_dx && concurrent_bwd(plan, d, w)) {
     side.reset(new SideGemm(plan, d, st));
     TP_TRY(side->status());
   }
@@ -1433,7 +1471,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
                                      to_marr(reinterpret_cast<void* const*>(dbias), p), 0, plan->dtype,
                                      side ? side->stream() : st, side ? wgrad_workspace(plan, w, false) : 0));
   if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
-  if (dX_out && !side) TP_TRY(run_gemm(plan, d, st));
+  if (has_dx && !side) TP_TRY(run_gemm(plan, d, st));
   return TP_OK;
 }
 
@@ -1456,6 +1494,15 @@ tp_status tp_column_bwd_reduce_scatter_seq(tp_plan* plan, tp_which which, int64_
                                            float* const* dbias, void* const* dX_seq,
                                            void* stream) {
   return column_bwd_common(plan, which, T, X, dZ, W, dW, dbias, dX_seq, 2, as_stream(stream));
+}
+
+tp_status tp_column_bwd_push_peer(tp_plan* plan, tp_which which, int64_t T, const void* X,
+                                  const void* const* dZ, const void* const* W, void* const* dW,
+                                  float* const* dbias, const tp_peer_group* g, uint32_t epoch,
+                                  void* stream) {
+  const cudaStream_t st = as_stream(stream);
+  TP_TRY(column_bwd_common(plan, which, T, X, dZ, W, dW, dbias, nullptr, 3, st, g));
+  return launch_peer_signal(g, g->rank, epoch, st);
 }
 
 }  // extern "C"

@@ -1028,7 +1028,7 @@ tp_status encode_epi(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, uint64_
 bool tma_epilogue_ok(const GemmBatch& b, int nout, int ksplit) {
   const char* e = getenv("TP_GEMM_TMA_EPI");
   if (e && e[0] == '0') return false;
-  if (b.out_f32 || ksplit > 1) return false;
+  if (b.out_f32 || ksplit > 1 || b.plain_stores) return false;
   if (b.scatter_n > 0) {  // plain stores into sequence shards of whole 32-row warp slabs
     if (b.epi != tpi::EPI_STORE || b.rows_per_out % 32 || b.scatter_n > TP_MAX_SHARDS ||
         static_cast<int64_t>(b.scatter_n) * b.rows_per_out != b.g[0].M)

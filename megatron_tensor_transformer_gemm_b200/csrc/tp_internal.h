@@ -210,6 +210,9 @@ struct GemmBatch {
   int64_t rows_per_out;
   void* out_seq[TP_MAX_SHARDS];
   const void* res_seq[TP_MAX_SHARDS];
+  // Outputs that may be another GPU's memory (a peer group's receive
+  // buffers): the epilogue writes them with plain stores, never TMA.
+  bool plain_stores;
   // Split K (bf16 path, EPI_STORE, fp32 outputs, every problem with the same
   // K): ksplit > 1 runs each output tile ksplit times over consecutive K
   // ranges, split s writing its fp32 partial at g[i].D + s * split_stride.
@@ -228,6 +231,11 @@ int gemm_split_k(const GemmBatch& b);
 // fp32 FMA path (tp_gemm_simt.cu): the same epilogues, grouping and K concatenation.
 tp_status launch_gemm_f32(const GemmBatch& b, cudaStream_t st);
 
+// Peer-memory steps (tp_peer.cu): validation of a peer group, and the flag
+// raise that follows a grid which wrote into other ranks' memory.
+tp_status check_peer_group(const tp_peer_group* g);
+tp_status launch_peer_signal(const tp_peer_group* g, int word, uint32_t epoch, cudaStream_t st);
+
 // Attention core (tp_attention.cu).
 tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const PtrArray& qkv,
                                const MutPtrArray& o, float* const* lse, cudaStream_t st);
@@ -236,3 +244,10 @@ tp_status launch_attention_bwd(tp_plan* plan, int batch, int seq, const PtrArray
                                const MutPtrArray& dqkv, cudaStream_t st);
 
 }  // namespace tpi
+
+// Return the status of `expr` from the enclosing function unless it is TP_OK.
+#define TP_TRY(expr)            \
+  do {                          \
+    tp_status _s = (expr);      \
+    if (_s != TP_OK) return _s; \
+  } while (0)

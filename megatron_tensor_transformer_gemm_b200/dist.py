@@ -20,12 +20,23 @@ its local GEMM epilogue, every other rank contributes its bare partial sum
 The collective steps (sum_over_ranks, scatter_seq_sum, gather_seq) and the
 weight slicing are plain torch.distributed / tensor code, independent of the
 device, so they run unchanged on CPU gloo ranks.
+
+comm="peer" replaces the all-reduces (and the Megatron-SP reduce-scatters) of
+Y and dX by libtp's peer-memory steps: the row GEMM (and the column
+backward's dX GEMM) stores each row block of its local sum straight into the
+owning rank's receive buffer from its epilogue, the owner sums the world
+slots once and pushes its block to every rank's output (non-SP) or keeps it
+(SP), and a device-side wait closes the exchange ("张量并行", Megatron-SP:
+all-reduce = reduce-scatter + all-gather). The buffers are mapped between the
+processes with CUDA IPC (PeerMemory); bias and residual are added once, in
+the owner's reduce.
 """
 from __future__ import annotations
 
 import torch
 import torch.distributed as dist
 
+from . import tp
 from .tp import Plan
 
 
@@ -88,6 +99,102 @@ def gather_seq(shard: torch.Tensor, out: torch.Tensor, group=None) -> torch.Tens
     return out
 
 
+# ------------------------------------------------------------- peer memory
+
+class _DevView:
+    """A raw device range as a __cuda_array_interface__ of int16 (bf16 bits)."""
+
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = {"shape": (nbytes // 2,), "typestr": "<i2", "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
+def bf16_view(ptr: int, shape, device) -> torch.Tensor:
+    """A bf16 tensor over the device range at `ptr` (not owned: the memory
+    must outlive the tensor)."""
+    n = 1
+    for x in shape:
+        n *= x
+    t = torch.as_tensor(_DevView(ptr, 2 * n), device=device)
+    return t.view(torch.bfloat16).view(*shape)
+
+
+class PeerMemory:
+    """`nbytes` of device memory on every rank of `group`, each rank's block
+    mapped into every other rank's process (tp_peer_alloc, the IPC handles
+    all-gathered, tp_peer_open). ptrs[d] is rank d's block as seen here;
+    ptrs[rank] is this rank's own. close() unmaps and frees; tensors made by
+    bf16() do not own the memory and must not outlive it."""
+
+    def __init__(self, nbytes: int, group=None, device=None):
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.nbytes = nbytes
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.local, handle = tp.peer_alloc(nbytes)
+        handles = [None] * self.world
+        if self.world > 1:
+            dist.all_gather_object(handles, handle, group=group)
+        else:
+            handles[0] = handle
+        self.ptrs, self._opened = [], []
+        try:
+            for d, h in enumerate(handles):
+                if d == self.rank:
+                    self.ptrs.append(self.local)
+                else:
+                    ptr = tp.peer_open(h)
+                    self._opened.append(ptr)
+                    self.ptrs.append(ptr)
+        except Exception:
+            self.close()
+            raise
+
+    def bf16(self, offset: int, shape) -> torch.Tensor:
+        """A bf16 tensor over this rank's block at byte `offset`."""
+        n = 1
+        for x in shape:
+            n *= x
+        if offset % 16 or offset + 2 * n > self.nbytes:
+            raise ValueError("view outside the peer block or not 16-byte aligned")
+        return bf16_view(self.local + offset, shape, self.device)
+
+    def close(self):
+        for ptr in self._opened:
+            tp.peer_close(ptr)
+        self._opened = []
+        if self.local:
+            tp.peer_free(self.local)
+            self.local = 0
+
+
+class PeerGroup:
+    """The flag words and receive buffers of one exchange between the ranks
+    of `group` (tp_peer_group), for up to recv_elems elements per rank, and
+    the epoch counter every rank advances in step."""
+
+    def __init__(self, recv_elems: int, group=None, device=None):
+        self.mem = PeerMemory(tp.PEER_FLAG_BYTES + 2 * recv_elems, group, device)
+        self.world, self.rank = self.mem.world, self.mem.rank
+        self.recv_elems = recv_elems
+        self.c = tp.peer_group(self.world, self.rank, recv_elems, self.mem.ptrs,
+                               [q + tp.PEER_FLAG_BYTES for q in self.mem.ptrs])
+        self.epoch = 0
+
+    def next_epoch(self) -> int:
+        self.epoch = (self.epoch + 1) & 0xFFFFFFFF
+        return self.epoch
+
+    def reduce(self, T: int, hidden: int, bias, residual, out, epoch: int):
+        """tp_peer_reduce then tp_peer_wait: this rank's row block of the sum
+        over ranks (+ bias + residual) into every pointer of `out`."""
+        tp.peer_reduce(self.c, T, hidden, bias, residual, out, epoch)
+        tp.peer_wait(self.c, epoch)
+
+    def close(self):
+        self.mem.close()
+
+
 # ------------------------------------------------------------------- the layer
 
 class DistTPMLP:
@@ -98,7 +205,12 @@ class DistTPMLP:
     output is the rank's sequence shard of Y."""
 
     def __init__(self, hidden: int, ffn: int, p: int, act: str = "swiglu", group=None,
-                 device="cuda", bias: bool = False, sequence_parallel: bool = False):
+                 device="cuda", bias: bool = False, sequence_parallel: bool = False,
+                 comm: str = "nccl"):
+        if comm not in ("nccl", "peer"):
+            raise ValueError(f"comm must be 'nccl' or 'peer', not {comm!r}")
+        self.comm = comm
+        self.peer = self.Ymem = self.dXmem = None
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -151,8 +263,18 @@ class DistTPMLP:
         self.dW2 = [torch.empty_like(w) for w in self.W2]
         self.db1 = [torch.empty(self.n1, dtype=torch.float32, device=dev) for _ in range(pl)] if self.bias else None
         self.db2 = torch.empty(h, dtype=torch.float32, device=dev) if self.bias else None
-        self.Yp = torch.empty(T, h, dtype=bf, device=dev)     # local sum, then the all-reduced Y
-        self.dXp = torch.empty(T, h, dtype=bf, device=dev)
+        if self.comm == "peer":
+            self.close_peer()
+            self.peer = PeerGroup(T * h, self.group, dev)
+            if not self.sp:   # outputs the other ranks push their row blocks into
+                self.Ymem = PeerMemory(2 * T * h, self.group, dev)
+                self.dXmem = PeerMemory(2 * T * h, self.group, dev)
+                self.Yp, self.dXp = self.Ymem.bf16(0, (T, h)), self.dXmem.bf16(0, (T, h))
+            else:
+                self.Yp = self.dXp = None
+        else:
+            self.Yp = torch.empty(T, h, dtype=bf, device=dev)     # local sum, then the all-reduced Y
+            self.dXp = torch.empty(T, h, dtype=bf, device=dev)
         if self.sp:
             self.Xn = torch.empty(t, h, dtype=bf, device=dev)   # LayerNorm of the local shard
             self.U = torch.empty(T, h, dtype=bf, device=dev)    # gathered LayerNorm output
@@ -183,6 +305,16 @@ class DistTPMLP:
             Xin = X
         self.X = Xin
         pl.column_fwd("mlp", T, Xin, self.W1, self.b1, self.Z if self.act != "none" else None, self.H)
+        if self.comm == "peer":
+            e = self.peer.next_epoch()
+            pl.row_fwd_push_peer("mlp", T, self.H, self.W2, self.peer.c, e)
+            t, r = T // self.world, self.rank
+            if self.sp:
+                self.peer.reduce(T, self.h, self.b2, residual, [self.Y_seq], e)
+                return self.Y_seq
+            res = residual[r * t:(r + 1) * t] if residual is not None else None
+            self.peer.reduce(T, self.h, self.b2, res, self._blocks(self.Ymem, T), e)
+            return self.Yp
         res = None if self.sp else once_on_rank0(residual, self.rank)
         pl.row_fwd_reduce("mlp", T, self.H, self.W2, once_on_rank0(self.b2, self.rank), res, self.Yp)
         if self.sp:
@@ -205,6 +337,19 @@ class DistTPMLP:
             dYf = dY
         pl.row_bwd("mlp", T, dYf, self.H, self.W2, self.Z if self.act != "none" else None, self.dZ,
                    self.dW2, self.db2)
+        if self.comm == "peer":
+            e = self.peer.next_epoch()
+            pl.column_bwd_push_peer("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.peer.c, e)
+            if not self.sp:
+                self.peer.reduce(T, self.h, None, None, self._blocks(self.dXmem, T), e)
+                return self.dXp
+            self.peer.reduce(T, self.h, None, None, [self.dU_seq], e)
+            t = T // self.world
+            self.ln.layernorm_bwd(t, self.X_in, self.gamma, self.dU_seq, self.mean, self.rstd,
+                                  self.dX_seq, self.dgamma, self.dbeta)
+            sum_over_ranks(self.dgamma, g)
+            sum_over_ranks(self.dbeta, g)
+            return self.dX_seq
         pl.column_bwd_reduce("mlp", T, self.X, self.dZ, self.W1, self.dW1, self.db1, self.dXp)
         if not self.sp:
             return sum_over_ranks(self.dXp, g)
@@ -215,6 +360,17 @@ class DistTPMLP:
         sum_over_ranks(self.dgamma, g)
         sum_over_ranks(self.dbeta, g)
         return self.dX_seq
+
+    def _blocks(self, mem: PeerMemory, T: int) -> list:
+        """This rank's row block of the [T, h] output on every rank."""
+        off = self.rank * (T // self.world) * self.h * 2
+        return [q + off for q in mem.ptrs]
+
+    def close_peer(self):
+        for m in (self.peer, self.Ymem, self.dXmem):
+            if m is not None:
+                m.close()
+        self.peer = self.Ymem = self.dXmem = None
 
     def flops(self, T: int) -> float:
         """Useful FLOPs of one forward + backward of the whole layer (all ranks)."""

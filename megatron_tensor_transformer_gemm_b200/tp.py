@@ -48,6 +48,20 @@ _i64 = ctypes.c_int64
 _int = ctypes.c_int
 _fp = ctypes.c_void_p  # float* (device)
 _plan_p = ctypes.c_void_p
+_u32 = ctypes.c_uint32
+
+PEER_HANDLE_BYTES = 64
+PEER_FLAG_BYTES = 256
+
+
+class PeerGroupC(ctypes.Structure):
+    """tp_peer_group: this rank's view of every rank's flag words and
+    receive buffer (device pointers, local or mapped from a peer)."""
+    _fields_ = [("world", ctypes.c_int), ("rank", ctypes.c_int), ("recv_elems", ctypes.c_int64),
+                ("flags", ctypes.c_void_p * MAX_SHARDS), ("recv", ctypes.c_void_p * MAX_SHARDS)]
+
+
+_peer_p = ctypes.POINTER(PeerGroupC)
 
 _SIGS = {
     "tp_plan_create": (_int, [_int, _int, _int, _int, _int, _int, _int, ctypes.POINTER(_plan_p)]),
@@ -91,6 +105,15 @@ _SIGS = {
     "tp_column_bwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_set_backward_defer": (_int, [_plan_p, _int]),
     "tp_backward_join": (_int, [_vp]),
+    "tp_peer_alloc": (_int, [ctypes.c_size_t, _vpp, _vp]),
+    "tp_peer_free": (_int, [_vp]),
+    "tp_peer_open": (_int, [_vp, _vpp]),
+    "tp_peer_close": (_int, [_vp]),
+    "tp_peer_set_wait_limit": (_int, [_i64]),
+    "tp_row_fwd_push_peer": (_int, [_plan_p, _int, _i64, _vpp, _vpp, _peer_p, _u32, _vp]),
+    "tp_column_bwd_push_peer": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _peer_p, _u32, _vp]),
+    "tp_peer_reduce": (_int, [_peer_p, _i64, _int, _vp, _vp, _int, _vpp, _u32, _vp]),
+    "tp_peer_wait": (_int, [_peer_p, _u32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -115,6 +138,57 @@ def backward_join(stream=None) -> None:
     """tp_backward_join: the stream waits for the deferred weight gradients
     and bias sums of every plan (see Plan.set_backward_defer)."""
     check(lib.tp_backward_join(_stream(stream)), "tp_backward_join")
+
+
+def peer_alloc(nbytes: int) -> tuple[int, bytes]:
+    """tp_peer_alloc: zeroed device memory other processes can map; returns
+    (device pointer, IPC handle bytes)."""
+    ptr = ctypes.c_void_p()
+    h = ctypes.create_string_buffer(PEER_HANDLE_BYTES)
+    check(lib.tp_peer_alloc(nbytes, ctypes.byref(ptr), h), "tp_peer_alloc")
+    return ptr.value, h.raw
+
+
+def peer_free(ptr: int) -> None:
+    check(lib.tp_peer_free(ptr), "tp_peer_free")
+
+
+def peer_open(handle: bytes) -> int:
+    """tp_peer_open: map another process's peer memory; returns its pointer here."""
+    if len(handle) != PEER_HANDLE_BYTES:
+        raise ValueError(f"a peer handle has {PEER_HANDLE_BYTES} bytes, got {len(handle)}")
+    ptr = ctypes.c_void_p()
+    check(lib.tp_peer_open(ctypes.create_string_buffer(handle, PEER_HANDLE_BYTES), ctypes.byref(ptr)),
+          "tp_peer_open")
+    return ptr.value
+
+
+def peer_close(ptr: int) -> None:
+    check(lib.tp_peer_close(ptr), "tp_peer_close")
+
+
+def peer_set_wait_limit(ns: int) -> None:
+    check(lib.tp_peer_set_wait_limit(int(ns)), "tp_peer_set_wait_limit")
+
+
+def peer_group(world: int, rank: int, recv_elems: int, flags: Sequence[int], recv: Sequence[int]) -> PeerGroupC:
+    """A tp_peer_group from per-rank device pointers."""
+    g = PeerGroupC()
+    g.world, g.rank, g.recv_elems = world, rank, recv_elems
+    for d in range(world):
+        g.flags[d] = flags[d]
+        g.recv[d] = recv[d]
+    return g
+
+
+def peer_reduce(g: PeerGroupC, T: int, hidden: int, bias, residual, out: Sequence, epoch: int,
+                stream=None) -> None:
+    check(lib.tp_peer_reduce(ctypes.byref(g), T, hidden, _ptr(bias), _ptr(residual), len(out), _arr(out),
+                             epoch, _stream(stream)), "tp_peer_reduce")
+
+
+def peer_wait(g: PeerGroupC, epoch: int, stream=None) -> None:
+    check(lib.tp_peer_wait(ctypes.byref(g), epoch, _stream(stream)), "tp_peer_wait")
 
 
 def _ptr(t) -> int | None:
@@ -292,6 +366,15 @@ class Plan:
     def column_bwd_reduce(self, which, T, X, dZ, W, dW=None, dbias=None, dX=None, stream=None):
         check(lib.tp_column_bwd_reduce(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
                                        _arr(dbias), _ptr(dX), _stream(stream)), "tp_column_bwd_reduce")
+
+    def row_fwd_push_peer(self, which, T, H, W, g: PeerGroupC, epoch: int, stream=None):
+        check(lib.tp_row_fwd_push_peer(self._h, WHICH[which], T, _arr(H), _arr(W), ctypes.byref(g), epoch,
+                                       _stream(stream)), "tp_row_fwd_push_peer")
+
+    def column_bwd_push_peer(self, which, T, X, dZ, W, dW, dbias, g: PeerGroupC, epoch: int, stream=None):
+        check(lib.tp_column_bwd_push_peer(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
+                                          _arr(dbias), ctypes.byref(g), epoch, _stream(stream)),
+              "tp_column_bwd_push_peer")
 
     def column_bwd_reduce_scatter_seq(self, which, T, X, dZ, W, dW=None, dbias=None, dX_seq=None,
                                       stream=None):

@@ -213,3 +213,38 @@ def test_layernorm_row_limits(dtype, hidden):
         assert L.tp_layernorm_all_gather_seq(h, 4, 1, _arr([FAKE]), FAKE, FAKE, FAKE, None, None, None) == 5
     finally:
         p.close()
+
+
+def test_peer_calls_validate_before_any_launch(plan):
+    """The peer-memory steps check the group, the sizes and the pointers on
+    the host (no device needed for these errors)."""
+    L, h = tp.lib, plan.handle
+    W = _arr([FAKE, FAKE])
+    ok = tp.peer_group(2, 1, 64 * 256, [FAKE, FAKE + 4096], [FAKE + 256, FAKE + 8192])
+    assert L.tp_peer_reduce(None, 64, 256, None, None, 1, _arr([FAKE]), 1, None) == 1
+    bad = tp.peer_group(2, 2, 64 * 256, [FAKE, FAKE], [FAKE, FAKE])      # rank outside [0, world)
+    assert L.tp_peer_reduce(ctypes.byref(bad), 64, 256, None, None, 1, _arr([FAKE]), 1, None) == 1
+    bad = tp.peer_group(2, 0, 64 * 256, [FAKE, 0], [FAKE, FAKE])         # a NULL flag pointer
+    assert L.tp_peer_wait(ctypes.byref(bad), 1, None) == 1
+    bad = tp.peer_group(2, 0, 64 * 256, [FAKE, FAKE + 8], [FAKE, FAKE])  # misaligned flags
+    assert L.tp_peer_wait(ctypes.byref(bad), 1, None) == 3
+    assert L.tp_peer_reduce(ctypes.byref(ok), 63, 256, None, None, 1, _arr([FAKE]), 1, None) == 2   # T % world
+    assert L.tp_peer_reduce(ctypes.byref(ok), 128, 256, None, None, 1, _arr([FAKE]), 1, None) == 1  # capacity
+    assert "exceeds the receive buffers" in tp.last_error()
+    assert L.tp_peer_reduce(ctypes.byref(ok), 64, 100, None, None, 1, _arr([FAKE]), 1, None) == 3   # hidden % 8
+    assert L.tp_peer_reduce(ctypes.byref(ok), 64, 256, None, None, 0, _arr([FAKE]), 1, None) == 1   # n_out
+    assert L.tp_peer_reduce(ctypes.byref(ok), 64, 256, FAKE + 2, None, 1, _arr([FAKE]), 1, None) == 3
+    assert L.tp_row_fwd_push_peer(h, 0, 63, W, W, ctypes.byref(ok), 1, None) == 2
+    assert L.tp_row_fwd_push_peer(h, 0, 64, W, W, None, 1, None) == 1
+    assert L.tp_column_bwd_push_peer(h, 0, 128, FAKE, W, W, None, None, ctypes.byref(ok), 1, None) == 1
+    f32 = tp.Plan(256, 512, 0, 2, "f32", "gelu")
+    try:
+        assert L.tp_row_fwd_push_peer(f32.handle, 0, 64, W, W, ctypes.byref(ok), 1, None) == 4
+    finally:
+        f32.close()
+    assert L.tp_peer_set_wait_limit(-5) == 1
+    assert L.tp_peer_set_wait_limit(61 * 10**9) == 1
+    assert L.tp_peer_set_wait_limit(0) == 0
+    with pytest.raises(ValueError):
+        tp.peer_open(b"short")
+    assert L.tp_peer_alloc(0, ctypes.byref(ctypes.c_void_p()), ctypes.create_string_buffer(64)) == 1

@@ -100,3 +100,53 @@ def test_dist_mlp_gelu_bias_single_rank(nccl_group):
     assert_close(d.db2[None, :], gr["db2"][None, :], 1e-4, "db2")
     for j, i in enumerate(d.shards):
         assert_close(d.db1[j][None, :], O.shard_vec(gr["db1"], p, i)[None, :], TOL_BF16, f"db1 {i}")
+
+
+@pytest.mark.parametrize("sp", [False, True])
+def test_dist_mlp_peer_comm_single_rank(nccl_group, sp):
+    """comm="peer": the all-reduces (SP: reduce-scatters) of Y and dX through
+    the peer-memory steps (push from the GEMM epilogue, reduce, wait) on a
+    one-rank group, against the oracle; a second step repeats the first."""
+    from megatron_tensor_transformer_gemm_b200.dist import DistTPMLP
+    if sp:
+        seq, h, f, p = 256, 512, 1536, 4
+        X, g, b, W1, W2, dY = tp_synth.draw_sp_mlp(seq, h, f, p, torch.bfloat16, seed=14, ln_affine_random=True)
+        d = DistTPMLP(h, f, p, "swiglu", group=nccl_group, sequence_parallel=True, comm="peer")
+        d.load_weights(W1, W2)
+        d.gamma.copy_(dev(g))
+        d.beta.copy_(dev(b))
+        try:
+            Y = d.forward(dev(X)).clone()
+            dX = d.backward(dev(dY)).clone()
+            Y2 = d.forward(dev(X)).clone()
+            dX2 = d.backward(dev(dY)).clone()
+            Xo, go, bo, W1o, W2o, dYo = (O.f64(t) for t in (X, g, b, W1, W2, dY))
+            ref = O.sp_mlp_fwd(Xo, go, bo, W1o, W2o)
+            rb = O.sp_mlp_bwd(Xo, go, W1o, W2o, ref, dYo)
+            assert_close(Y, ref["Y"], TOL_BF16, "Y")
+            assert_close(dX, rb["dX"], TOL_BF16, "dX")
+            assert torch.equal(Y, Y2) and torch.equal(dX, dX2)
+        finally:
+            d.close_peer()
+        return
+    T, h, f, p = 384, 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, "gelu", torch.bfloat16, seed=15, bias=True)
+    d = DistTPMLP(h, f, p, "gelu", group=nccl_group, bias=True, comm="peer")
+    d.load_weights(inp.W1, inp.W2, inp.b1, dev(inp.b2))
+    res = (dev(inp.X) * 0.5).contiguous()
+    try:
+        Y = d.forward(dev(inp.X), residual=res).clone()
+        dX = d.backward(dev(inp.dY)).clone()
+        Y2 = d.forward(dev(inp.X), residual=res).clone()
+        dX2 = d.backward(dev(inp.dY)).clone()
+        from megatron_tensor_transformer_gemm_b200 import tp
+        torch.cuda.synchronize()
+        assert tp.lib.tp_get_device_status(None, None) == 0
+        Xo, W1, W2, dYo = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+        ref = O.mlp_fwd(Xo, W1, O.f64(inp.b1), W2, O.f64(inp.b2), "gelu", residual=O.f64(res))
+        gr = O.mlp_bwd(Xo, W1, W2, ref["Z"], ref["H"], dYo, "gelu")
+        assert_close(Y, ref["Y"], TOL_BF16, "Y")
+        assert_close(dX, gr["dX"], TOL_BF16, "dX")
+        assert torch.equal(Y, Y2) and torch.equal(dX, dX2)
+    finally:
+        d.close_peer()
