@@ -14,9 +14,13 @@
 //               tile's MMAs run while the other tile's softmax works
 //   warps 2..5  softmax of tile A, warps 6..9 of tile B: thread r owns query
 //               row r; its 128 scores of a block come from TMEM in one read
-//               (row max, then exp2 and the row sum), P rounded to bf16 and written to shared
-//               memory in the 128-byte-swizzled K-major layout of the PV MMA.
-//               Only the diagonal block (and a ragged last block) is masked.
+//               (row max, then exp2 and the row sum), P rounded to bf16 and written back
+//               into the first 64 columns of the tile's S in TMEM (two keys per column),
+//               where the PV MMA reads it as its A operand, so P takes no shared-memory
+//               bandwidth from the MMAs' Q, K and V operands (PT = false, selected with
+//               TP_ATTN_P_SMEM=1, keeps the earlier form: P in shared memory,
+//               128-byte-swizzled K-major). Only the diagonal block (and a ragged last
+//               block) is masked.
 // O accumulates in TMEM across key blocks. P is taken relative to a reference
 // max m that is raised (and O, l rescaled in place) only when a row's max
 // exceeds it by more than 2^8; P <= 2^8 stays exact in fp32/bf16 range and the
@@ -58,13 +62,15 @@ struct AttnParams {
   unsigned* status;
 };
 
-template <int D>
+template <int D, bool PT>
 struct AttnSmem {
   static constexpr int Q_BYTES = BQ * D * 2;
   static constexpr int KV_BYTES = BKV * D * 2;
-  static constexpr int P_BYTES = BQ * BKV * 2;
-  static constexpr int KV_SLOTS = 3;
+  static constexpr int P_BYTES = PT ? 0 : BQ * BKV * 2;
+  static constexpr int KV_SLOTS = PT ? 5 : 3;  // the shared memory P no longer takes
   static constexpr int TOTAL = 1024 + 2 * Q_BYTES + KV_SLOTS * KV_BYTES + 2 * P_BYTES + 256;
+  static_assert(TOTAL <= 232448, "attention forward shared memory");
+  static_assert((1 + 2 * KV_SLOTS + 7) * 8 + 8 <= 256, "barrier area");
 };
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -72,10 +78,10 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 
-template <int D>
+template <int D, bool PT>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   tpd::pdl_entry();
-  using SM = AttnSmem<D>;
+  using SM = AttnSmem<D, PT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -84,13 +90,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint8_t* sP = sKV + SM::KV_SLOTS * SM::KV_BYTES;  // [2] tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SM::P_BYTES);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [KV_SLOTS]
-  uint64_t* kv_empty = bars + 4;  // [KV_SLOTS]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;    // [2]
-  uint64_t* o_done = bars + 11;   // [2]
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* kv_full = bars + 1;                  // [KV_SLOTS]
+  uint64_t* kv_empty = kv_full + SM::KV_SLOTS;   // [KV_SLOTS]
+  uint64_t* s_full = kv_empty + SM::KV_SLOTS;    // [2]
+  uint64_t* p_full = s_full + 2;                 // [2]
+  uint64_t* o_done = p_full + 2;                 // [2]
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,7 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // S of tile t in columns [128 t, 128 t + 128); O of tile t in [256 + D t, 256 + D (t + 1)).
+  // S of tile t in columns [128 t, 128 t + 128) (PT: its P in the first 64 of them, written
+  // after S is read; the MMAs issue PV(j) before S(j + 1), and tcgen05.mma executes in issue
+  // order, so S(j + 1) overwrites P(j) only after PV(j) has read it); O of tile t in
+  // [256 + D t, 256 + D (t + 1)).
 
   if (warp == kProducerWarp && lane == 0) {
     // ------------------------------------------------------------- producer
@@ -195,9 +204,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const uint32_t v_base = smem_u32(sKV + slot_of(2 * j + 1) * SM::KV_BYTES);
 #pragma unroll
       for (int kk = 0; kk < BKV / 16; ++kk) {
-        const uint64_t adesc = smem_desc_sw128(p_base + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
         const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, CHUNK_BYTES, 1024);
-        tc_mma_bf16(tmem + 256 + D * t, adesc, bdesc, idesc_o, (first && kk == 0) ? 0u : 1u);
+        if (PT) {  // A = P from TMEM: keys 16 kk .. 16 kk + 15 in columns 8 kk .. 8 kk + 7
+          tc_mma_bf16_ts(tmem + 256 + D * t, tmem + 128 * t + 8 * kk, bdesc, idesc_o,
+                         (first && kk == 0) ? 0u : 1u);
+        } else {
+          const uint64_t adesc = smem_desc_sw128(p_base + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
+          tc_mma_bf16(tmem + 256 + D * t, adesc, bdesc, idesc_o, (first && kk == 0) ? 0u : 1u);
+        }
       }
       tc_commit(&o_done[t]);
     };
@@ -313,29 +327,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       float rs = 0.f;
       const float sc = p.scale_log2;
 #pragma unroll
-      for (int cc = 0; cc < BKV / 32; ++cc) {
-        uint8_t* rowp = sPt + (cc / 2) * CHUNK_BYTES + r * 128;
+      for (int cc = 0; cc < BKV / 32; ++cc) {  // 32 keys -> 16 packed words
+        uint32_t pw[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {  // 8 columns -> one 16-byte store of P
-          uint32_t pk[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int i = v * 8 + 2 * w;
-            const float2 x = fma2_bcast(sv[cc][i], sv[cc][i + 1], sc, -m);  // scaled score - m
-            float a = ex2(x.x);
-            float bb = ex2(x.y);
-            if (!full) {
-              a = (cc * 32 + i <= kmax) ? a : 0.f;
-              bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
-            }
-            pk[w] = pack_bf16x2(a, bb);
-            // the row sum uses the rounded P of the PV MMA (bf16 widening is exact)
-            { const float2 f = unpack_bf16x2(pk[w]); rs += f.x + f.y; }
+        for (int i = 0; i < 32; i += 2) {
+          const float2 x = fma2_bcast(sv[cc][i], sv[cc][i + 1], sc, -m);  // scaled score - m
+          float a = ex2(x.x);
+          float bb = ex2(x.y);
+          if (!full) {
+            a = (cc * 32 + i <= kmax) ? a : 0.f;
+            bb = (cc * 32 + i + 1 <= kmax) ? bb : 0.f;
           }
-          const int qv = (cc % 2) * 4 + v;
-          *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          const uint32_t w = pack_bf16x2(a, bb);
+          pw[i / 2] = w;
+          // the row sum uses the rounded P of the PV MMA (bf16 widening is exact)
+          const float2 f = unpack_bf16x2(w);
+          rs += f.x + f.y;
+        }
+        if (PT) {
+          tmem_st16u(tS + 16 * cc, pw);
+        } else {
+          uint8_t* rowp = sPt + (cc / 2) * CHUNK_BYTES + r * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {  // 8 keys -> one 16-byte store of P
+            const int qv = (cc % 2) * 4 + v;
+            *reinterpret_cast<uint4*>(rowp + ((qv ^ (r & 7)) << 4)) =
+                make_uint4(pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
+          }
         }
       }
+      if (PT) tc_wait_st();  // P is in TMEM before the MMA warp is told
       if (rescale) {
         // O of the previous blocks (stable: their P.V is done) to the new reference.
 #pragma unroll 1
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         tc_wait_st();
       }
       l = l * alpha + rs;
-      fence_async_smem();
+      if (!PT) fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
@@ -391,20 +412,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   }
 }
 
-template <int D>
+template <int D, bool PT>
 tp_status launch_fwd_d(AttnParams& prm, cudaStream_t st) {
   static bool attr = false;
-  const int smem = AttnSmem<D>::TOTAL;
+  const int smem = AttnSmem<D, PT>::TOTAL;
   if (!attr) {
     tp_status s = tpi::cuda_status(
-        cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+        cudaFuncSetAttribute(attn_fwd_kernel<D, PT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
         "cudaFuncSetAttribute(attention)");
     if (s != TP_OK) return s;
     attr = true;
   }
   const int grid = prm.n_pairs * prm.p * prm.batch * prm.heads_local;
-  (void)tpi::launch(attn_fwd_kernel<D>, dim3(grid), dim3(kThreads), smem, st, prm);
+  (void)tpi::launch(attn_fwd_kernel<D, PT>, dim3(grid), dim3(kThreads), smem, st, prm);
   return tpi::after_launch("attention_fwd (tcgen05)");
+}
+
+// P in TMEM (default) or, with TP_ATTN_P_SMEM=1, in shared memory.
+bool p_in_tmem() {
+  static const bool on = [] {
+    const char* e = getenv("TP_ATTN_P_SMEM");
+    return !(e && e[0] == '1');
+  }();
+  return on;
 }
 
 }  // namespace
@@ -442,8 +472,8 @@ tp_status launch_attention_fwd(const tp_plan* plan, int batch, int seq, const Pt
   if (s != TP_OK) return s;
   if (static_cast<int64_t>(prm.n_pairs) * p * batch * hl > 0x7fffffffLL)
     return fail(TP_ERR_UNSUPPORTED, "attention grid too large");
-  if (d == 64) return launch_fwd_d<64>(prm, st);
-  if (d == 128) return launch_fwd_d<128>(prm, st);
+  if (d == 64) return p_in_tmem() ? launch_fwd_d<64, true>(prm, st) : launch_fwd_d<64, false>(prm, st);
+  if (d == 128) return p_in_tmem() ? launch_fwd_d<128, true>(prm, st) : launch_fwd_d<128, false>(prm, st);
   return fail(TP_ERR_UNSUPPORTED, "head_dim %d", d);
 }
 

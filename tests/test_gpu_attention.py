@@ -123,3 +123,19 @@ def test_attention_bwd_local_heads(batch, seq, heads, d, p, ds, monkeypatch):
     for name, idx, ref in (("dQ", 0, rq), ("dK", 1, rk), ("dV", 2, rv)):
         g = np.concatenate([x[:, :, idx, :] for x in got], axis=2)
         assert_close(g.reshape(seq * batch, h), ref.reshape(seq * batch, h), TOL_BF16, name)
+
+
+def test_attention_fwd_p_in_shared_memory():
+    """The forward's earlier form (TP_ATTN_P_SMEM=1: P through shared memory
+    instead of TMEM) on the same forward cases, in a subprocess so the choice
+    is made before the library's first launch."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(root, "tests", "test_gpu_attention.py"), "-k",
+                        "fwd_local_heads or growing_scores"],
+                       cwd=root, env=dict(os.environ, TP_ATTN_P_SMEM="1"), capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-2000:]
