@@ -104,18 +104,13 @@ __device__ __forceinline__ void acc8(float (&a)[8], const uint4& u) {
 // res[r, :], rounded to bf16, for every destination k. A thread owns one
 // 16-byte vector (8 columns) of a row and walks the slot's rows and vectors
 // with the grid's stride, two vectors per step with all their loads issued
-// before the sums. Thread 0 of each CTA first waits for every source's block.
+// before the sums. Each CTA first waits for every source's block: thread s
+// polls source s's word, so the system-scope acquire loads overlap.
 template <int NMAX>
 __global__ void __launch_bounds__(256) peer_reduce_kernel(const __grid_constant__ ReduceParams p) {
   tpd::pdl_entry();
-  __shared__ int ready;
-  if (threadIdx.x == 0) {
-    bool ok = true;
-    for (int s = 0; s < p.world && ok; ++s) ok = wait_flag(p.arrived + s, p.epoch, p.limit_ns, p.status);
-    ready = ok ? 1 : 0;
-  }
-  __syncthreads();
-  if (!ready) return;
+  const bool ok = threadIdx.x >= p.world || wait_flag(p.arrived + threadIdx.x, p.epoch, p.limit_ns, p.status);
+  if (!__syncthreads_and(ok)) return;
   const int64_t total = p.t * p.vpr;
   const int64_t slot = p.t * p.vpr * 8;  // elements per slot
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
