@@ -164,15 +164,6 @@ __global__ void __launch_bounds__(256) peer_reduce_kernel(const __grid_constant_
   }
 }
 
-int sm_count_now() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return 148;
-  }
-  return n > 0 ? n : 148;
-}
-
 }  // namespace
 
 namespace tpi {
@@ -285,12 +276,19 @@ tp_status tp_peer_reduce(const tp_peer_group* g, int64_t T, int hidden, const vo
   p.epoch = epoch;
   p.limit_ns = g_peer_wait_ns.load();
   p.status = status;
-  const int64_t vec = p.t * p.vpr;
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((vec + 511) / 512, sm_count_now() * 8LL));
-  if (g->world <= 2) (void)launch(peer_reduce_kernel<2>, dim3(grid), dim3(256), 0, st, p);
-  else if (g->world <= 4) (void)launch(peer_reduce_kernel<4>, dim3(grid), dim3(256), 0, st, p);
-  else if (g->world <= 8) (void)launch(peer_reduce_kernel<8>, dim3(grid), dim3(256), 0, st, p);
-  else (void)launch(peer_reduce_kernel<TP_MAX_SHARDS>, dim3(grid), dim3(256), 0, st, p);
+  // one CTA per 512 vectors (two per thread), at most as many as are resident at once
+  // (SM count and occupancy cached per device)
+  const int64_t units = std::max<int64_t>(1, (p.t * p.vpr + 511) / 512);
+  auto run = [&](auto kernel) -> tp_status {
+    int64_t grid = 1;
+    TP_TRY(persistent_grid(reinterpret_cast<const void*>(kernel), 256, 0, units, &grid));
+    (void)launch(kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, p);
+    return TP_OK;
+  };
+  if (g->world <= 2) TP_TRY(run(peer_reduce_kernel<2>));
+  else if (g->world <= 4) TP_TRY(run(peer_reduce_kernel<4>));
+  else if (g->world <= 8) TP_TRY(run(peer_reduce_kernel<8>));
+  else TP_TRY(run(peer_reduce_kernel<TP_MAX_SHARDS>));
   TP_TRY(after_launch("peer_reduce"));
   return launch_peer_signal(g, TP_MAX_SHARDS + g->rank, epoch, st);
 }
