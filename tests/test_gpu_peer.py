@@ -254,3 +254,32 @@ def test_peer_memory_maps_into_another_process():
     finally:
         torch.cuda.synchronize()
         tp.peer_free(ptr)
+
+
+def test_peer_steps_at_the_edges():
+    """T = 0 still takes every flag step (the epochs stay in step across the
+    ranks), and the largest group, 16 emulated ranks of one shard each, sums
+    and gathers like the smaller ones."""
+    from megatron_tensor_transformer_gemm_b200 import tp
+    world, T, h, f = 16, 512, 128, 512
+    inp = tp_synth.draw_mlp(T, h, f, "gelu", torch.bfloat16, seed=61)
+    em = EmulatedRanks(world, 1, T, h, f, "gelu", inp)
+    try:
+        X = dev(inp.X)
+        # an empty exchange first: no rows, but every rank's flags advance to epoch 1
+        for r, k in enumerate(em.ranks):
+            k["plan"].row_fwd_push_peer("mlp", 0, k["H"], k["W2"], em.g[r], 1)
+        for r in range(world):
+            tp.peer_reduce(em.g[r], 0, h, None, None, em.blocks(em.Yptr, r), 1)
+        for r in range(world):
+            tp.peer_wait(em.g[r], 1)
+        assert em.status() == 0
+        em.forward(X, None, None, epoch=2)
+        assert em.status() == 0
+        Xo, W1, W2 = (O.f64(v) for v in (inp.X, inp.W1, inp.W2))
+        ref = O.mlp_fwd(Xo, W1, None, W2, None, "gelu")
+        for r in range(world):
+            assert torch.equal(em.Y[r], em.Y[0])
+        assert_close(em.Y[0], ref["Y"], TOL_BF16, "Y")
+    finally:
+        em.close()
