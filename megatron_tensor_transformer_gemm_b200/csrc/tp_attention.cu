@@ -4,15 +4,16 @@
 //
 // One CTA computes two adjacent 128-query tiles (A = 2i, B = 2i + 1) of one
 // (shard, batch, head); both read every K/V block once from shared memory:
-//   warp 0      TMA producer: both Q tiles, then K_0, V_0, K_1, V_1, ... into a
-//               ring of three K/V buffers (item n waits only for item n - 3 to
-//               be released, so V_j lands while block j - 1 is still in flight)
-//               from a 3-D tensor map over the sequence-major
-//               [seq, batch, 3*heads_local*d] QKV of the shard
-//   warp 1      TMEM allocator + MMA issuer, ping-pong order: S_A(0), S_B(0),
+//   warp 8      TMA producer: both Q tiles, then K_0, V_0, K_1, V_1, ... into a
+//               ring of K/V buffers (five with P in TMEM, three with P in shared
+//               memory; item n waits only for item n - slots to be released, so
+//               V_j lands while block j - 1 is still in flight) from a 3-D
+//               tensor map over the sequence-major [seq, batch, 3*heads_local*d]
+//               QKV of the shard
+//   warp 9      TMEM allocator + MMA issuer, ping-pong order: S_A(0), S_B(0),
 //               then per block PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one
 //               tile's MMAs run while the other tile's softmax works
-//   warps 2..5  softmax of tile A, warps 6..9 of tile B: thread r owns query
+//   warps 0..3  softmax of tile A, warps 4..7 of tile B: thread r owns query
 //               row r; its 128 scores of a block come from TMEM in one read
 //               (row max, then exp2 and the row sum), P rounded to bf16 and written back
 //               into the first 64 columns of the tile's S in TMEM (two keys per column),
