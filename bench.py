@@ -48,16 +48,31 @@ METRIC = "sharded MLP fwd+bwd TFLOP/s at p shards on 1 B200; partial-reduce HBM 
 WORKLOAD = "7B-shaped SwiGLU MLP fwd+bwd: hidden 4096, ffn 11008, tokens 8x4096, p=8 shards on one GPU"
 
 
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
 def load_peaks():
+    """The measured peaks file (copy GB/s, bf16 TFLOP/s burst and sustained)
+    when present and readable, else the fallback figures; a figure the file
+    lacks is taken from the fallback (the sustained one scaled from the
+    measured burst), and `source` says which."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as fh:
             d = json.load(fh)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+        got = {k: float(d[k]) for k in FALLBACK_PEAKS if isinstance(d.get(k), (int, float)) and d[k] > 0}
     except Exception:
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-                "source": "fallback"}
+        got = {}
+    if not got:
+        return dict(FALLBACK_PEAKS, source="fallback")
+    out = dict(FALLBACK_PEAKS)
+    out.update(got)
+    if "bf16_tflops_sustained" not in got and "bf16_tflops" in got:
+        out["bf16_tflops_sustained"] = got["bf16_tflops"] * (FALLBACK_PEAKS["bf16_tflops_sustained"] /
+                                                             FALLBACK_PEAKS["bf16_tflops"])
+    missing = [k for k in FALLBACK_PEAKS if k not in got]
+    out["source"] = "measured" if not missing else "measured (" + ", ".join(missing) + " from the fallback)"
+    return out
 
 
 def mlp_flops(T, h, f):
