@@ -563,6 +563,28 @@ TP_API tp_status tp_peer_reduce(const tp_peer_group* g, int64_t T, int hidden, c
 /* Step 3: the stream waits (on the device) for every rank's step 2. */
 TP_API tp_status tp_peer_wait(const tp_peer_group* g, uint32_t epoch, void* stream);
 
+/* The Megatron-SP all-gather along the sequence ([TP-wiki] Megatron-SP: the
+ * next layer's column GEMM needs the whole sequence) over peer memory, in two
+ * of the steps above: this rank's shard is stored into out[d] (rank d's
+ * gathered buffer at this rank's rows, [rows, cols]) for every d < world with
+ * plain stores, then this rank's "done" word is raised on every rank; then
+ * tp_peer_wait (step 3, same epoch) waits until every rank's shard has
+ * arrived. A gathered buffer is written by the next all-gather's pushes, so
+ * its readers must have finished by then: in a layer they do, because the
+ * exchange that follows them (the reduce-scatter and its wait) cannot finish
+ * on any rank before every rank has passed them. x and out[d] bf16, dense,
+ * cols % 8 == 0. */
+TP_API tp_status tp_all_gather_push_peer(const tp_peer_group* g, int64_t rows, int cols, const void* x,
+                                         void* const* out, uint32_t epoch, void* stream);
+/* The same with the LayerNorm of the shard fused in ([TP-blog] §3.3, as
+ * tp_layernorm_fwd: x [rows, hidden] of this rank, gamma, beta [hidden], mean
+ * and rstd [rows] fp32 (NULL ok)): each normalised row is pushed to every
+ * rank's gathered buffer. bf16 plans only. */
+TP_API tp_status tp_layernorm_all_gather_push_peer(tp_plan* plan, const tp_peer_group* g, int64_t rows,
+                                                   const void* x, const void* gamma, const void* beta,
+                                                   void* const* out, float* mean, float* rstd,
+                                                   uint32_t epoch, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1079,6 +1079,31 @@ tp_status tp_layernorm_all_gather_seq(tp_plan* plan, int64_t T, int n, const voi
                               rstd, plan->dtype, as_stream(stream));
 }
 
+tp_status tp_layernorm_all_gather_push_peer(tp_plan* plan, const tp_peer_group* g, int64_t rows,
+                                           const void* x, const void* gamma, const void* beta,
+                                           void* const* out, float* mean, float* rstd, uint32_t epoch,
+                                           void* stream) {
+  TP_TRY(check_plan(plan));
+  TP_TRY(check_T(rows));
+  TP_TRY(check_peer_group(g));
+  if (plan->dtype != TP_BF16) return fail(TP_ERR_DTYPE, "peer pushes need a bf16 plan");
+  TP_TRY(check_ptr(x, "x"));
+  TP_TRY(check_ptr(gamma, "gamma"));
+  TP_TRY(check_ptr(beta, "beta"));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(out), g->world, "out", false));
+  TP_TRY(check_ln(plan));
+  const cudaStream_t st = as_stream(stream);
+  if (rows > 0) {
+    PtrArray xs{};
+    xs.p[0] = x;
+    MutPtrArray dst{};
+    for (int d = 0; d < g->world; ++d) dst.p[d] = out[d];
+    TP_TRY(launch_layernorm_fwd(xs, 1, rows, plan->hidden, gamma, beta, nullptr, mean, rstd, plan->dtype,
+                                st, &dst, g->world));
+  }
+  return launch_peer_signal(g, TP_MAX_SHARDS + g->rank, epoch, st);
+}
+
 tp_status tp_layernorm_bwd(tp_plan* plan, int64_t rows, const void* x, const void* gamma,
                            const void* dy, const float* mean, const float* rstd, const void* dres,
                            void* dx, float* dgamma, float* dbeta, int accumulate, void* stream) {

@@ -135,7 +135,8 @@ tp_status launch_column_sum_deferred(tp_plan* plan, const PtrArray& x, int n, in
 // LayerNorm (tp_layernorm.cu).
 tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,
                                const void* gamma, const void* beta, void* y, float* mean,
-                               float* rstd, tp_dtype dt, cudaStream_t st);
+                               float* rstd, tp_dtype dt, cudaStream_t st,
+                               const MutPtrArray* ydst = nullptr, int n_dst = 0);
 tp_status launch_layernorm_bwd(tp_plan* plan, const void* x, const void* gamma, const void* dy,
                                const float* mean, const float* rstd, const void* dres, void* dx,
                                float* dgamma, float* dbeta, int accumulate, int64_t rows,

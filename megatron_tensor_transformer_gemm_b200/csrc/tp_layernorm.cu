@@ -13,6 +13,7 @@
 
 namespace {
 
+using tpi::MutPtrArray;
 using tpi::PtrArray;
 
 constexpr float kEps = 1e-5f;
@@ -71,11 +72,13 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // The slice stays packed in registers; the mean and the biased variance about
 // it are two exact passes over those registers, each summed over the CTA with
 // one barrier (each sum has a buffer of its own, and a CTA takes one row).
-template <typename T, int THREADS>
+// Row r of y goes to ydst.p[0] (MULTI = false) or to each of the n_dst outputs
+// (MULTI: an all-gather pushed into other GPUs' buffers over peer memory).
+template <typename T, int THREADS, bool MULTI>
 __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__ PtrArray src, int64_t rows_per_src,
                                                          int64_t cols, const T* gamma,
-                                                         const T* beta, T* y, float* mean_out,
-                                                         float* rstd_out) {
+                                                         const T* beta, const __grid_constant__ MutPtrArray ydst,
+                                                         int n_dst, float* mean_out, float* rstd_out) {
   tpd::pdl_entry();
   constexpr int V = LnVec<T>::N;
   constexpr int W = THREADS / 32;
@@ -128,7 +131,7 @@ __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__
 #pragma unroll
   for (int w = 0; w < W; ++w) u += red2[w];
   const float rstd = rsqrtf(u * inv_h + kEps);
-  uint4* yr = reinterpret_cast<uint4*>(y + r * cols);
+  uint4* y1 = reinterpret_cast<uint4*>(static_cast<T*>(ydst.p[0]) + r * cols);
 #pragma unroll
   for (int i = 0; i < kVptMax; ++i) {
     const int c = threadIdx.x + i * THREADS;
@@ -139,7 +142,12 @@ __global__ void __launch_bounds__(THREADS) ln_fwd_kernel(const __grid_constant__
       LnVec<T>::load(beta + static_cast<int64_t>(c) * V, b);
 #pragma unroll
       for (int e = 0; e < V; ++e) o[e] = (v[e] - mean) * rstd * g[e] + b[e];
-      LnVec<T>::store(yr + c, o);
+      if (MULTI) {
+        for (int d = 0; d < n_dst; ++d)
+          LnVec<T>::store(reinterpret_cast<uint4*>(static_cast<T*>(ydst.p[d]) + r * cols) + c, o);
+      } else {
+        LnVec<T>::store(y1 + c, o);
+      }
     }
   }
   if (threadIdx.x == 0) {
@@ -341,17 +349,28 @@ namespace tpi {
 
 tp_status launch_layernorm_fwd(const PtrArray& x_seq, int n, int64_t rows_per_src, int64_t cols,
                                const void* gamma, const void* beta, void* y, float* mean,
-                               float* rstd, tp_dtype dt, cudaStream_t st) {
+                               float* rstd, tp_dtype dt, cudaStream_t st, const MutPtrArray* ydst,
+                               int n_dst) {
   const int64_t rows = rows_per_src * n;
   if (rows == 0) return TP_OK;
   const int V = dt == TP_BF16 ? 8 : 4;
   const int64_t vpr = cols / V;
   if (vpr > 256 * kVptMax) return fail(TP_ERR_UNSUPPORTED, "LayerNorm row too long (%lld)", (long long)cols);
   const int th = threads_for(vpr);
+  MutPtrArray dst{};
+  if (ydst && n_dst > 0) {
+    dst = *ydst;
+  } else {
+    dst.p[0] = y;
+    n_dst = 1;
+  }
 #define TP_LN_FWD(T, TH)                                                                        \
-  (void)tpi::launch(ln_fwd_kernel<T, TH>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st,                             \
-      x_seq, rows_per_src, cols, static_cast<const T*>(gamma), static_cast<const T*>(beta),     \
-      static_cast<T*>(y), mean, rstd)
+  (void)(n_dst > 1 ? tpi::launch(ln_fwd_kernel<T, TH, true>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st, \
+                                 x_seq, rows_per_src, cols, static_cast<const T*>(gamma),       \
+                                 static_cast<const T*>(beta), dst, n_dst, mean, rstd)           \
+                   : tpi::launch(ln_fwd_kernel<T, TH, false>, dim3(static_cast<unsigned>(rows)), dim3(TH), 0, st, \
+                                 x_seq, rows_per_src, cols, static_cast<const T*>(gamma),       \
+                                 static_cast<const T*>(beta), dst, n_dst, mean, rstd))
   if (dt == TP_BF16) {
     if (th == 64) TP_LN_FWD(__nv_bfloat16, 64);
     else if (th == 128) TP_LN_FWD(__nv_bfloat16, 128);

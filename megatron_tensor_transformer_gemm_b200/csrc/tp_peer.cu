@@ -164,6 +164,27 @@ __global__ void __launch_bounds__(256) peer_reduce_kernel(const __grid_constant_
   }
 }
 
+struct PushParams {
+  const uint4* src;  // [rows, cols] bf16 as 16-byte vectors, dense
+  uint4* out[TP_MAX_SHARDS];
+  int n_out, rank;
+  int64_t total;     // vectors
+};
+
+// out[k][v] = src[v] for every destination, in rotated order as in the reduce.
+__global__ void __launch_bounds__(256) peer_push_kernel(const __grid_constant__ PushParams p) {
+  tpd::pdl_entry();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < p.total; v += stride) {
+    const uint4 x = __ldcs(p.src + v);
+    for (int k = 0; k < p.n_out; ++k) {
+      int d = p.rank + 1 + k;
+      while (d >= p.n_out) d -= p.n_out;
+      p.out[d][v] = x;
+    }
+  }
+}
+
 }  // namespace
 
 namespace tpi {
@@ -290,6 +311,31 @@ tp_status tp_peer_reduce(const tp_peer_group* g, int64_t T, int hidden, const vo
   else if (g->world <= 8) TP_TRY(run(peer_reduce_kernel<8>));
   else TP_TRY(run(peer_reduce_kernel<TP_MAX_SHARDS>));
   TP_TRY(after_launch("peer_reduce"));
+  return launch_peer_signal(g, TP_MAX_SHARDS + g->rank, epoch, st);
+}
+
+tp_status tp_all_gather_push_peer(const tp_peer_group* g, int64_t rows, int cols, const void* x,
+                                  void* const* out, uint32_t epoch, void* stream) {
+  TP_TRY(check_peer_group(g));
+  if (rows < 0) return fail(TP_ERR_ARG, "rows = %lld", (long long)rows);
+  if (cols <= 0 || cols % 8)
+    return fail(TP_ERR_ALIGN, "cols = %d is not a positive multiple of 8 (16-byte rows)", cols);
+  TP_TRY(check_ptr(x, "x"));
+  TP_TRY(check_ptrs(reinterpret_cast<const void* const*>(out), g->world, "out", false));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rows > 0) {
+    PushParams p{};
+    p.src = static_cast<const uint4*>(x);
+    for (int d = 0; d < g->world; ++d) p.out[d] = static_cast<uint4*>(out[d]);
+    p.n_out = g->world;
+    p.rank = g->rank;
+    p.total = rows * (cols / 8);
+    int64_t grid = 1;
+    TP_TRY(persistent_grid(reinterpret_cast<const void*>(peer_push_kernel), 256, 0,
+                           std::max<int64_t>(1, (p.total + 255) / 256), &grid));
+    (void)launch(peer_push_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, p);
+    TP_TRY(after_launch("peer_push"));
+  }
   return launch_peer_signal(g, TP_MAX_SHARDS + g->rank, epoch, st);
 }
 

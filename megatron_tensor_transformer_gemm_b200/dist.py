@@ -27,7 +27,9 @@ backward's dX GEMM) stores each row block of its local sum straight into the
 owning rank's receive buffer from its epilogue, the owner sums the world
 slots once and pushes its block to every rank's output (non-SP) or keeps it
 (SP), and a device-side wait closes the exchange ("张量并行", Megatron-SP:
-all-reduce = reduce-scatter + all-gather). The buffers are mapped between the
+all-reduce = reduce-scatter + all-gather). Under SP the all-gathers go the same
+way: the LayerNorm kernel pushes each normalised row into every rank's
+gathered input, and dY's shard is pushed likewise. The buffers are mapped between the
 processes with CUDA IPC (PeerMemory); bias and residual are added once, in
 the owner's reduce.
 """
@@ -210,7 +212,7 @@ class DistTPMLP:
         if comm not in ("nccl", "peer"):
             raise ValueError(f"comm must be 'nccl' or 'peer', not {comm!r}")
         self.comm = comm
-        self.peer = self.Ymem = self.dXmem = None
+        self.peer = self.Ymem = self.dXmem = self.Umem = self.dYmem = None
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -270,18 +272,22 @@ class DistTPMLP:
                 self.Ymem = PeerMemory(2 * T * h, self.group, dev)
                 self.dXmem = PeerMemory(2 * T * h, self.group, dev)
                 self.Yp, self.dXp = self.Ymem.bf16(0, (T, h)), self.dXmem.bf16(0, (T, h))
-            else:
+            else:             # gathered inputs the other ranks push their sequence shards into
                 self.Yp = self.dXp = None
+                self.Umem = PeerMemory(2 * T * h, self.group, dev)
+                self.dYmem = PeerMemory(2 * T * h, self.group, dev)
         else:
             self.Yp = torch.empty(T, h, dtype=bf, device=dev)     # local sum, then the all-reduced Y
             self.dXp = torch.empty(T, h, dtype=bf, device=dev)
         if self.sp:
             self.Xn = torch.empty(t, h, dtype=bf, device=dev)   # LayerNorm of the local shard
-            self.U = torch.empty(T, h, dtype=bf, device=dev)    # gathered LayerNorm output
+            self.U = (self.Umem.bf16(0, (T, h)) if self.comm == "peer" else
+                      torch.empty(T, h, dtype=bf, device=dev))  # gathered LayerNorm output
             self.mean = torch.empty(t, dtype=torch.float32, device=dev)
             self.rstd = torch.empty(t, dtype=torch.float32, device=dev)
             self.Y_seq = torch.empty(t, h, dtype=bf, device=dev)
-            self.dY_full = torch.empty(T, h, dtype=bf, device=dev)
+            self.dY_full = (self.dYmem.bf16(0, (T, h)) if self.comm == "peer" else
+                            torch.empty(T, h, dtype=bf, device=dev))
             self.dU_seq = torch.empty(t, h, dtype=bf, device=dev)
             self.dX_seq = torch.empty(t, h, dtype=bf, device=dev)
             self.dgamma = torch.empty(h, dtype=torch.float32, device=dev)
@@ -296,8 +302,14 @@ class DistTPMLP:
             T = t * self.world
             self.alloc(T)
             self.X_in = X
-            self.ln.layernorm_fwd(t, X, self.gamma, self.beta, self.Xn, self.mean, self.rstd)
-            gather_seq(self.Xn, self.U, g)
+            if self.comm == "peer":   # LayerNorm pushed into every rank's U at this rank's rows
+                e = self.peer.next_epoch()
+                self.ln.layernorm_all_gather_push_peer(self.peer.c, t, X, self.gamma, self.beta,
+                                                       self._blocks(self.Umem, T), self.mean, self.rstd, e)
+                tp.peer_wait(self.peer.c, e)
+            else:
+                self.ln.layernorm_fwd(t, X, self.gamma, self.beta, self.Xn, self.mean, self.rstd)
+                gather_seq(self.Xn, self.U, g)
             Xin = self.U
         else:
             T = X.shape[0]
@@ -331,7 +343,12 @@ class DistTPMLP:
         pl, g = self.plan, self.group
         T = self._T
         if self.sp:
-            gather_seq(dY, self.dY_full, g)
+            if self.comm == "peer":
+                e = self.peer.next_epoch()
+                tp.all_gather_push_peer(self.peer.c, T // self.world, self.h, dY, self._blocks(self.dYmem, T), e)
+                tp.peer_wait(self.peer.c, e)
+            else:
+                gather_seq(dY, self.dY_full, g)
             dYf = self.dY_full
         else:
             dYf = dY
@@ -367,10 +384,10 @@ class DistTPMLP:
         return [q + off for q in mem.ptrs]
 
     def close_peer(self):
-        for m in (self.peer, self.Ymem, self.dXmem):
+        for m in (self.peer, self.Ymem, self.dXmem, self.Umem, self.dYmem):
             if m is not None:
                 m.close()
-        self.peer = self.Ymem = self.dXmem = None
+        self.peer = self.Ymem = self.dXmem = self.Umem = self.dYmem = None
 
     def flops(self, T: int) -> float:
         """Useful FLOPs of one forward + backward of the whole layer (all ranks)."""

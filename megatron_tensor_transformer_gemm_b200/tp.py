@@ -114,6 +114,8 @@ _SIGS = {
     "tp_column_bwd_push_peer": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _peer_p, _u32, _vp]),
     "tp_peer_reduce": (_int, [_peer_p, _i64, _int, _vp, _vp, _int, _vpp, _u32, _vp]),
     "tp_peer_wait": (_int, [_peer_p, _u32, _vp]),
+    "tp_all_gather_push_peer": (_int, [_peer_p, _i64, _int, _vp, _vpp, _u32, _vp]),
+    "tp_layernorm_all_gather_push_peer": (_int, [_plan_p, _peer_p, _i64, _vp, _vp, _vp, _vpp, _fp, _fp, _u32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -189,6 +191,11 @@ def peer_reduce(g: PeerGroupC, T: int, hidden: int, bias, residual, out: Sequenc
 
 def peer_wait(g: PeerGroupC, epoch: int, stream=None) -> None:
     check(lib.tp_peer_wait(ctypes.byref(g), epoch, _stream(stream)), "tp_peer_wait")
+
+
+def all_gather_push_peer(g: PeerGroupC, rows: int, cols: int, x, out: Sequence, epoch: int, stream=None) -> None:
+    check(lib.tp_all_gather_push_peer(ctypes.byref(g), rows, cols, _ptr(x), _arr(out), epoch, _stream(stream)),
+          "tp_all_gather_push_peer")
 
 
 def _ptr(t) -> int | None:
@@ -366,6 +373,12 @@ class Plan:
     def column_bwd_reduce(self, which, T, X, dZ, W, dW=None, dbias=None, dX=None, stream=None):
         check(lib.tp_column_bwd_reduce(self._h, WHICH[which], T, _ptr(X), _arr(dZ), _arr(W), _arr(dW),
                                        _arr(dbias), _ptr(dX), _stream(stream)), "tp_column_bwd_reduce")
+
+    def layernorm_all_gather_push_peer(self, g: PeerGroupC, rows, x, gamma, beta, out, mean=None, rstd=None,
+                                       epoch: int = 0, stream=None):
+        check(lib.tp_layernorm_all_gather_push_peer(self._h, ctypes.byref(g), rows, _ptr(x), _ptr(gamma), _ptr(beta),
+                                                    _arr(out), _ptr(mean), _ptr(rstd), epoch, _stream(stream)),
+              "tp_layernorm_all_gather_push_peer")
 
     def row_fwd_push_peer(self, which, T, H, W, g: PeerGroupC, epoch: int, stream=None):
         check(lib.tp_row_fwd_push_peer(self._h, WHICH[which], T, _arr(H), _arr(W), ctypes.byref(g), epoch,

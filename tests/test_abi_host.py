@@ -248,3 +248,16 @@ def test_peer_calls_validate_before_any_launch(plan):
     with pytest.raises(ValueError):
         tp.peer_open(b"short")
     assert L.tp_peer_alloc(0, ctypes.byref(ctypes.c_void_p()), ctypes.create_string_buffer(64)) == 1
+
+
+def test_peer_all_gather_calls_validate(plan):
+    L, h = tp.lib, plan.handle
+    ok = tp.peer_group(2, 0, 64 * 256, [FAKE, FAKE + 4096], [FAKE + 256, FAKE + 8192])
+    assert L.tp_all_gather_push_peer(None, 8, 256, FAKE, _arr([FAKE, FAKE]), 1, None) == 1
+    assert L.tp_all_gather_push_peer(ctypes.byref(ok), 8, 100, FAKE, _arr([FAKE, FAKE]), 1, None) == 3
+    assert L.tp_all_gather_push_peer(ctypes.byref(ok), 8, 256, FAKE, _arr([FAKE, 0]), 1, None) == 1
+    assert L.tp_all_gather_push_peer(ctypes.byref(ok), -1, 256, FAKE, _arr([FAKE, FAKE]), 1, None) == 1
+    assert L.tp_layernorm_all_gather_push_peer(h, ctypes.byref(ok), 8, FAKE, FAKE, FAKE,
+                                               _arr([FAKE, FAKE + 2]), None, None, 1, None) == 3
+    assert L.tp_layernorm_all_gather_push_peer(h, None, 8, FAKE, FAKE, FAKE,
+                                               _arr([FAKE, FAKE]), None, None, 1, None) == 1

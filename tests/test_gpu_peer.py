@@ -283,3 +283,57 @@ def test_peer_steps_at_the_edges():
         assert_close(em.Y[0], ref["Y"], TOL_BF16, "Y")
     finally:
         em.close()
+
+
+@pytest.mark.parametrize("world,t,h", [(2, 64, 256), (3, 40, 128), (8, 32, 512)])
+def test_peer_all_gathers_emulated(world, t, h):
+    """The Megatron-SP all-gathers over peer memory with `world` emulated
+    ranks (all pushes, then all waits): every rank's gathered buffer equals
+    the concatenation of the shards bit for bit (tp_all_gather_push_peer), and
+    with the LayerNorm fused in (tp_layernorm_all_gather_push_peer) equals the
+    single-GPU LayerNorm + all-gather bit for bit (same arithmetic) and the
+    oracle's LayerNorm within the bf16 tolerance; mean and rstd match too."""
+    from megatron_tensor_transformer_gemm_b200 import tp
+    from megatron_tensor_transformer_gemm_b200.dist import bf16_view
+    T = world * t
+    gen = torch.Generator().manual_seed(70 + world)
+    xs = [torch.randn(t, h, generator=gen).to(torch.bfloat16).cuda() for _ in range(world)]
+    gamma = (1 + 0.1 * torch.randn(h, generator=gen)).to(torch.bfloat16).cuda()
+    beta = (0.1 * torch.randn(h, generator=gen)).to(torch.bfloat16).cuda()
+    mem = [tp.peer_alloc(tp.PEER_FLAG_BYTES + 2 * T * h)[0] for _ in range(world)]
+    outs = [tp.peer_alloc(2 * T * h)[0] for _ in range(world)]
+    try:
+        g = [tp.peer_group(world, r, T * h, mem, [q + tp.PEER_FLAG_BYTES for q in mem]) for r in range(world)]
+        U = [bf16_view(q, (T, h), "cuda") for q in outs]
+        blocks = lambda r: [q + r * t * h * 2 for q in outs]
+        for r in range(world):
+            tp.all_gather_push_peer(g[r], t, h, xs[r], blocks(r), 1)
+        for r in range(world):
+            tp.peer_wait(g[r], 1)
+        torch.cuda.synchronize()
+        assert tp.lib.tp_get_device_status(None, None) == 0
+        full = torch.cat(xs)
+        for r in range(world):
+            assert torch.equal(U[r], full), f"rank {r}'s gathered buffer"
+        plan = tp.Plan(h, 0, 0, 1, "bf16", "none")
+        mean = [torch.empty(t, dtype=torch.float32, device="cuda") for _ in range(world)]
+        rstd = [torch.empty(t, dtype=torch.float32, device="cuda") for _ in range(world)]
+        for r in range(world):
+            plan.layernorm_all_gather_push_peer(g[r], t, xs[r], gamma, beta, blocks(r), mean[r], rstd[r], 2)
+        for r in range(world):
+            tp.peer_wait(g[r], 2)
+        ref = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+        mref = torch.empty(T, dtype=torch.float32, device="cuda")
+        rref = torch.empty(T, dtype=torch.float32, device="cuda")
+        plan.layernorm_all_gather_seq(T, xs, gamma, beta, ref, mref, rref)
+        torch.cuda.synchronize()
+        assert tp.lib.tp_get_device_status(None, None) == 0
+        for r in range(world):
+            assert torch.equal(U[r], ref), f"rank {r}'s LayerNorm all-gather"
+        assert torch.equal(torch.cat(mean), mref) and torch.equal(torch.cat(rstd), rref)
+        y, _, _ = O.layernorm_fwd(O.f64(full), O.f64(gamma), O.f64(beta))
+        assert_close(U[0], y, TOL_BF16, "LayerNorm")
+    finally:
+        torch.cuda.synchronize()
+        for q in mem + outs:
+            tp.peer_free(q)
