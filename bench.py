@@ -404,7 +404,8 @@ def run_ours(args, world, rank, local):
     dY_h = inp.dY.pin_memory()
     fused = args.variant == "fused"
     m = TPMLP(HIDDEN, FFN, P, "swiglu", "bf16", dev, fused=fused,
-              overlap_chunks=4 if args.variant == "overlap" else 0)
+              overlap_chunks=4 if args.variant == "overlap" else 0,
+              group_wgrad=args.wgrad_grouping)
     m.load_weights(inp.W1.to(dev), inp.W2.to(dev))
     del inp
     X = X_h.to(dev)
@@ -1139,6 +1140,9 @@ def main():
     ap.add_argument("--comm", choices=["nccl", "peer"], default="nccl",
                     help="N > 1, mlp7b: the all-reduces of Y and dX through NCCL, or through libtp's "
                          "peer-memory steps (push from the GEMM epilogue, reduce, wait)")
+    ap.add_argument("--wgrad-grouping", action="store_true",
+                    help="mlp7b: launch the row and column backward's weight gradients as one "
+                         "grouped GEMM instead of two")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph (other workloads)")
     args = ap.parse_args()

@@ -347,6 +347,19 @@ TP_API tp_status tp_set_backward_defer(tp_plan* plan, int on);
  * event wait: it returns at once on the host, and works inside a capture. */
 TP_API tp_status tp_backward_join(void* stream);
 
+/* Grouped weight gradients (on != 0): tp_row_bwd leaves its weight-gradient
+ * GEMM (dW_i = dY^T H_i) waiting in the plan, and the next tp_column_bwd*
+ * call on the same plan and stream launches it together with its own
+ * (dW_i = dZ_i^T X) as one grouped GEMM over both shard sets: the same tiles
+ * and results, one partly empty last wave instead of two. Until then dW of
+ * the row backward is not written, and its inputs dY and H must stay
+ * unchanged. tp_flush_wgrad launches a waiting one alone (on the stream it was
+ * issued on); so does any backward call that cannot take it along (another
+ * stream, the deferred mode, a GEMM on the side stream, no dW), and switching
+ * grouping off. bf16 plans; fp32 plans run every GEMM at once. */
+TP_API tp_status tp_set_wgrad_grouping(tp_plan* plan, int on);
+TP_API tp_status tp_flush_wgrad(tp_plan* plan);
+
 /* Row layer backward for every shard ([TP-scratch] §四: the input gradient of
  * the row layer needs no reduction; dY is replicated).
  *   dY [T, hidden]; H[i] the row input of shard i; W[i] the row shard.

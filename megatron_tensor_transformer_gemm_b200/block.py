@@ -33,19 +33,25 @@ class TPMLP:
     """One MLP sublayer split over p shards that all live on ``device``."""
 
     def __init__(self, hidden: int, ffn: int, p: int, act: str = "gelu", dtype: str = "bf16",
-                 device="cuda", bias: bool = False, fused: bool = False, overlap_chunks: int = 0):
+                 device="cuda", bias: bool = False, fused: bool = False, overlap_chunks: int = 0,
+                 group_wgrad: bool = False):
         """fused: sum the shards inside the row GEMM and the column-backward dX
         GEMM (tp_row_fwd_reduce / tp_column_bwd_reduce) instead of writing p
         partials and reducing them (tp_row_fwd_partial + tp_reduce_partials).
         overlap_chunks > 1 (partials only): split the tokens into that many
         blocks and reduce block c on a second stream while the GEMM of block
         c + 1 runs (the compute / communication overlap of "从零实现 Tensor
-        Parallel" §三, with the local reduce in place of the collective)."""
+        Parallel" §三, with the local reduce in place of the collective).
+        group_wgrad: the row and column backward's weight gradients run as one
+        grouped launch (tp_set_wgrad_grouping; backward() issues both). Off by
+        default: on the 7B step it measured slower than two launches."""
         self.h, self.f, self.p, self.act = hidden, ffn, p, act
         self.fused = fused
         self.chunks = overlap_chunks if (overlap_chunks > 1 and not fused) else 0
         self._side = None
         self.plan = Plan(hidden, ffn, 0, p, dtype, act)
+        if group_wgrad:
+            self.plan.set_wgrad_grouping(True)
         self.dt = self.plan.torch_dtype
         self.device = torch.device(device)
         self.bias = bias

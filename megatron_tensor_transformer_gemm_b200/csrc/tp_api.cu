@@ -456,6 +456,49 @@ tp_status run_wgrad(tp_plan* plan, GemmBatch w, cudaStream_t st, bool allow_spli
                        TP_BF16, st);
 }
 
+// Launch the weight gradients a row backward left waiting, alone, on the
+// stream it was issued on.
+tp_status flush_wgrad(tp_plan* plan) {
+  if (!plan->wg_pend) return TP_OK;
+  std::unique_ptr<GemmBatch> w(plan->wg_pend);
+  plan->wg_pend = nullptr;
+  return run_wgrad(plan, *w, plan->wg_st);
+}
+
+// Whether two weight-gradient batches can run as one launch: the same
+// operand layouts, epilogue and output type, the same K (tokens), room for
+// both in one batch, and the same stream.
+bool wgrad_mergeable(const GemmBatch& a, const GemmBatch& b, cudaStream_t sa, cudaStream_t sb) {
+  return sa == sb && a.n + b.n <= TP_MAX_SHARDS && a.a_mn == b.a_mn && a.b_mn == b.b_mn &&
+         a.epi == b.epi && a.out_f32 == b.out_f32 && !a.kcat && !b.kcat && a.scatter_n == 0 &&
+         b.scatter_n == 0 && a.g[0].K == b.g[0].K;
+}
+
+// The weight-gradient step of a backward call: with grouping on, a row
+// backward's batch waits for the next column backward, which launches both
+// in one grouped GEMM (one partly empty last wave instead of two).
+tp_status issue_wgrad(tp_plan* plan, const GemmBatch& w, cudaStream_t st, bool allow_split, bool row) {
+  if (plan->group_wgrad && plan->dtype == TP_BF16 && allow_split) {
+    if (row) {
+      TP_TRY(flush_wgrad(plan));
+      plan->wg_pend = new (std::nothrow) GemmBatch(w);
+      if (!plan->wg_pend) return fail(TP_ERR_ARG, "out of host memory for a pending weight gradient");
+      plan->wg_st = st;
+      return TP_OK;
+    }
+    if (plan->wg_pend && wgrad_mergeable(*plan->wg_pend, w, plan->wg_st, st)) {
+      std::unique_ptr<GemmBatch> pend(plan->wg_pend);
+      plan->wg_pend = nullptr;
+      GemmBatch m = *pend;
+      for (int i = 0; i < w.n; ++i) m.g[m.n + i] = w.g[i];
+      m.n += w.n;
+      return run_wgrad(plan, m, st);
+    }
+  }
+  TP_TRY(flush_wgrad(plan));
+  return run_wgrad(plan, w, st, allow_split);
+}
+
 }  // namespace
 
 extern "C" {
@@ -531,12 +574,17 @@ tp_status tp_plan_create(int hidden, int ffn, int heads, int p, tp_dtype dtype, 
   plan->ws2 = nullptr;
   plan->ws2_bytes = 0;
   plan->ws2_device = -1;
+  plan->group_wgrad = 0;
+  plan->wg_pend = nullptr;
+  plan->wg_st = nullptr;
   *out = plan;
   return TP_OK;
 }
 
 void tp_plan_destroy(tp_plan* plan) {
   if (!plan) return;
+  delete plan->wg_pend;  // a weight gradient still waiting is dropped, not launched
+  plan->wg_pend = nullptr;
   int cur = 0;
   cudaGetDevice(&cur);
   if (plan->ws) {
@@ -562,6 +610,18 @@ void tp_plan_destroy(tp_plan* plan) {
 tp_status tp_set_backward_defer(tp_plan* plan, int on) {
   TP_TRY(check_plan(plan));
   plan->defer_bwd = on ? 1 : 0;
+  return TP_OK;
+}
+
+tp_status tp_flush_wgrad(tp_plan* plan) {
+  TP_TRY(check_plan(plan));
+  return flush_wgrad(plan);
+}
+
+tp_status tp_set_wgrad_grouping(tp_plan* plan, int on) {
+  TP_TRY(check_plan(plan));
+  if (!on) TP_TRY(flush_wgrad(plan));
+  plan->group_wgrad = on ? 1 : 0;
   return TP_OK;
 }
 
@@ -1359,6 +1419,7 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
   if (plan->defer_bwd && plan->dtype == TP_BF16 && (dW || dbias)) {
     // Deferred: dH on the caller's stream, dW and db on the side stream,
     // joined by tp_backward_join (dW without a K split: no shared scratch).
+    TP_TRY(flush_wgrad(plan));
     SideStream* sd = nullptr;
     TP_TRY(side_stream(&sd));
     TP_TRY(cuda_status(cudaEventRecord(sd->fork, st), "cudaEventRecord(fork)"));
@@ -1387,7 +1448,7 @@ tp_status tp_row_bwd(tp_plan* plan, tp_which which, int64_t T, const void* dY,
   if (dbias)
     TP_TRY(launch_column_sum(plan, dY, T, h, h, dbias, 0, plan->dtype, side ? side->stream() : st,
                              side ? wgrad_workspace(plan, w, false) : 0));
-  if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
+  if (dW) TP_TRY(issue_wgrad(plan, w, st, !side, true));
   return TP_OK;
 }
 
@@ -1472,6 +1533,7 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
   if (plan->defer_bwd && plan->dtype == TP_BF16 && (dW || dbias)) {
     // Deferred: dX on the caller's stream, dW and db on the side stream,
     // joined by tp_backward_join (dW without a K split: no shared scratch).
+    TP_TRY(flush_wgrad(plan));
     SideStream* sd = nullptr;
     TP_TRY(side_stream(&sd));
     TP_TRY(cuda_status(cudaEventRecord(sd->fork, st), "cudaEventRecord(fork)"));
@@ -1495,7 +1557,8 @@ static tp_status column_bwd_common(tp_plan* plan, tp_which which, int64_t T, con
     TP_TRY(launch_column_sum_grouped(plan, to_arr(dZ, p), p, T, n, n,
                                      to_marr(reinterpret_cast<void* const*>(dbias), p), 0, plan->dtype,
                                      side ? side->stream() : st, side ? wgrad_workspace(plan, w, false) : 0));
-  if (dW) TP_TRY(run_wgrad(plan, w, st, !side));
+  if (dW) TP_TRY(issue_wgrad(plan, w, st, !side, false));
+  else TP_TRY(flush_wgrad(plan));
   if (has_dx && !side) TP_TRY(run_gemm(plan, d, st));
   return TP_OK;
 }

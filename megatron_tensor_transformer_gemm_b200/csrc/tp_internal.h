@@ -8,6 +8,10 @@
 
 #include "tp.h"
 
+namespace tpi {
+struct GemmBatch;
+}
+
 struct tp_plan {
   int hidden;
   int ffn;
@@ -34,6 +38,12 @@ struct tp_plan {
   void* ws2;
   size_t ws2_bytes;
   int ws2_device;
+  // Grouped weight gradients (tp_set_wgrad_grouping): the row backward's
+  // weight-gradient batch waits here (launched by the next column backward
+  // together with its own, or by tp_flush_wgrad) on stream wg_st.
+  int group_wgrad;
+  tpi::GemmBatch* wg_pend;  // NULL when nothing waits
+  cudaStream_t wg_st;
 };
 
 namespace tpi {

@@ -104,6 +104,8 @@ _SIGS = {
     "tp_column_bwd_reduce": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp]),
     "tp_column_bwd_reduce_scatter_seq": (_int, [_plan_p, _int, _i64, _vp, _vpp, _vpp, _vpp, _vpp, _vpp, _vp]),
     "tp_set_backward_defer": (_int, [_plan_p, _int]),
+    "tp_set_wgrad_grouping": (_int, [_plan_p, _int]),
+    "tp_flush_wgrad": (_int, [_plan_p]),
     "tp_backward_join": (_int, [_vp]),
     "tp_peer_alloc": (_int, [ctypes.c_size_t, _vpp, _vp]),
     "tp_peer_free": (_int, [_vp]),
@@ -413,6 +415,14 @@ class Plan:
     def attention_bwd(self, batch, seq, QKV, O, dO, LSE, dQKV, stream=None):
         check(lib.tp_attention_bwd(self._h, batch, seq, _arr(QKV), _arr(O), _arr(dO), _arr(LSE),
                                    _arr(dQKV), _stream(stream)), "tp_attention_bwd")
+
+    def set_wgrad_grouping(self, on: bool = True):
+        """tp_set_wgrad_grouping: the row backward's weight gradients wait for
+        the next column backward and run in one grouped launch with its own."""
+        check(lib.tp_set_wgrad_grouping(self._h, 1 if on else 0), "tp_set_wgrad_grouping")
+
+    def flush_wgrad(self):
+        check(lib.tp_flush_wgrad(self._h), "tp_flush_wgrad")
 
     def set_backward_defer(self, on: bool = True):
         """tp_set_backward_defer: this plan's backward calls leave their weight

@@ -261,3 +261,12 @@ def test_peer_all_gather_calls_validate(plan):
                                                _arr([FAKE, FAKE + 2]), None, None, 1, None) == 3
     assert L.tp_layernorm_all_gather_push_peer(h, None, 8, FAKE, FAKE, FAKE,
                                                _arr([FAKE, FAKE]), None, None, 1, None) == 1
+
+
+def test_wgrad_grouping_calls_validate(plan):
+    L = tp.lib
+    assert L.tp_set_wgrad_grouping(None, 1) == 1
+    assert L.tp_flush_wgrad(None) == 1
+    assert L.tp_set_wgrad_grouping(plan.handle, 1) == 0
+    assert L.tp_flush_wgrad(plan.handle) == 0          # nothing waits: no device call
+    assert L.tp_set_wgrad_grouping(plan.handle, 0) == 0

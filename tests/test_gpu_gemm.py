@@ -418,3 +418,65 @@ print("ok")
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
                        text=True, timeout=600)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("fused,act,T", [(True, "swiglu", 520), (False, "gelu", 384), (True, "gelu", 256)])
+def test_grouped_weight_gradients_match_separate(fused, act, T, monkeypatch):
+    """tp_set_wgrad_grouping: the row backward's dW2 waits and runs in one
+    grouped launch with the column backward's dW1; every gradient is bit for
+    bit the one the separate launches give (same tiles, same K order). The
+    backward calls are kept on one stream (at these small sizes they would
+    otherwise put the activation gradient beside the weight gradient, which
+    launches the weight gradient at once)."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    monkeypatch.setenv("TP_BWD_CONCURRENT", "0")
+    h, f, p = 256, 1024, 4
+    inp = tp_synth.draw_mlp(T, h, f, act, torch.bfloat16, seed=81)
+    outs = []
+    for grouped in (False, True):
+        m = TPMLP(h, f, p, act, "bf16", fused=fused, group_wgrad=grouped)
+        m.load_weights(dev(inp.W1), dev(inp.W2))
+        m.forward(dev(inp.X))
+        dX = m.backward(dev(inp.dY)).clone()
+        torch.cuda.synchronize()
+        outs.append((dX, [w.clone() for w in m.dW1], [w.clone() for w in m.dW2]))
+    (dX0, dW10, dW20), (dX1, dW11, dW21) = outs
+    assert torch.equal(dX0, dX1)
+    for i in range(p):
+        assert torch.equal(dW10[i], dW11[i]), f"dW1 shard {i}"
+        assert torch.equal(dW20[i], dW21[i]), f"dW2 shard {i}"
+    Xo, W1, W2, dYo = (O.f64(t) for t in (inp.X, inp.W1, inp.W2, inp.dY))
+    ref = O.mlp_fwd(Xo, W1, None, W2, None, act)
+    gr = O.mlp_bwd(Xo, W1, W2, ref["Z"], ref["H"], dYo, act)
+    for i in range(p):
+        assert_close(dW21[i], O.shard_cols(gr["dW2"], p, i), TOL_BF16, f"dW2 {i}")
+
+
+def test_pending_weight_gradient_flushes(monkeypatch):
+    """A row backward's waiting weight gradient is written by tp_flush_wgrad
+    alone, and by switching grouping off."""
+    from megatron_tensor_transformer_gemm_b200.block import TPMLP
+    monkeypatch.setenv("TP_BWD_CONCURRENT", "0")
+    T, h, f, p = 256, 256, 1024, 2
+    inp = tp_synth.draw_mlp(T, h, f, "gelu", torch.bfloat16, seed=82)
+    m = TPMLP(h, f, p, "gelu", "bf16", fused=True, group_wgrad=False)
+    m.load_weights(dev(inp.W1), dev(inp.W2))
+    m.forward(dev(inp.X))
+    dY = dev(inp.dY)
+    m.plan.row_bwd("mlp", T, dY, m.H, m.W2, m.Z, m.dZ, m.dW2, None)
+    ref = [w.clone() for w in m.dW2]
+    for grouped_flush in ("flush", "off"):
+        m.plan.set_wgrad_grouping(True)
+        for w in m.dW2:
+            w.zero_()
+        m.plan.row_bwd("mlp", T, dY, m.H, m.W2, m.Z, m.dZ, m.dW2, None)
+        torch.cuda.synchronize()
+        assert all(float(w.abs().max()) == 0.0 for w in m.dW2), "dW2 written before the flush"
+        if grouped_flush == "flush":
+            m.plan.flush_wgrad()
+        else:
+            m.plan.set_wgrad_grouping(False)
+        torch.cuda.synchronize()
+        for i in range(p):
+            assert torch.equal(m.dW2[i], ref[i])
+    m.plan.set_wgrad_grouping(False)
