@@ -133,6 +133,9 @@ struct alignas(64) GemmParams {
   // residual ({N, 1, rows_per_out}) and scatter_res says whether residuals come.
   int tma_epi;
   int scatter_res;
+  // Plain stores through the stage (plain_staged = 1): outputs that may be
+  // another GPU's memory, EPI_STORE, bf16, no bias, residual or split.
+  int plain_staged;
   CUtensorMap tmE[TP_MAX_SHARDS];
   CUtensorMap tmX[TP_MAX_SHARDS];
   unsigned* status;
@@ -353,6 +356,46 @@ __device__ __forceinline__ void stage_write(uint32_t tile, int r, const float (&
                                               pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
                                               pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]),
                                               pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7])));
+}
+
+// Plain-store epilogue through the stage (outputs that may be another GPU's
+// memory take no TMA): each 32 x 32 chunk of the warp's rows is written to
+// the stage by row, then read back four lanes to a row, so that one warp
+// store writes eight whole 64-byte row segments instead of 16-byte pieces of
+// 32 rows. EPI_STORE with bf16 outputs, no bias or residual, optionally
+// scattered by row to out_seq (any rows_per_out).
+__device__ void epilogue_plain_staged(const GemmParams& p, const GroupArgs& ga, uint32_t taddr, int row0,
+                                      int n0, int half, bool narrow, int lane, uint32_t tile) {
+  const int cpw = narrow ? BN / 128 : BN / 64;  // 32-column chunks per warp half
+  const int q = lane & 3, rsub = lane >> 2;     // this lane's piece and row within each group of 8
+#pragma unroll 1
+  for (int c = half * cpw; c < (half + 1) * cpw; ++c) {
+    const int j0 = n0 + c * 32;
+    if (j0 >= ga.N) break;  // warp-uniform
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tc_wait_ld();
+    stage_write(tile, lane, v);
+    __syncwarp();
+    const int col = j0 + q * 8;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int r = it * 8 + rsub, row = row0 + r;
+      const uint4 u = ld_shared_v4(sw64(tile, r, q));
+      if (row < ga.M && col < ga.N) {
+        __nv_bfloat16* base;
+        if (p.scatter) {
+          const int jb = row / p.rows_per_out;
+          base = static_cast<__nv_bfloat16*>(p.out_seq[jb]) +
+                 static_cast<int64_t>(row - jb * p.rows_per_out) * ga.ldd;
+        } else {
+          base = static_cast<__nv_bfloat16*>(ga.D) + static_cast<int64_t>(row) * ga.ldd;
+        }
+        *reinterpret_cast<uint4*>(base + col) = u;
+      }
+    }
+    __syncwarp();  // every lane has read the stage before the next chunk rewrites it
+  }
 }
 
 // Staged inputs per chunk: Z's gate and up halves (dSwiGLU), Z (dGELU), the
@@ -947,6 +990,8 @@ __global__ void __launch_bounds__(kThreads, 1) tp_gemm_kernel(const __grid_const
         epilogue_fwd_tma(p, ga, gi, taddr, trow, n0, half, narrow, lane, es);
       } else if (p.tma_epi) {
         ok = epilogue_tile_tma(p, ga, gi, taddr, trow, n0, half, narrow, pre, lane, es, abort_flag, p.status);
+      } else if (p.plain_staged) {
+        epilogue_plain_staged(p, ga, taddr, row0, n0, half, narrow, lane, smem_u32(es.buf));
       } else {
         epilogue_tile(p, ga, taddr, row0 + lane, n0, half, narrow, ks);
       }
@@ -1329,6 +1374,14 @@ tp_status launch_gemm_bf16(const GemmBatch& b, cudaStream_t st) {
     p.kb_per_split = kbps;
     p.split_stride = b.split_stride;
     tiles *= ksplit;
+  }
+  if (b.plain_stores && b.epi == tpi::EPI_STORE && !b.out_f32 && ksplit <= 1) {
+    bool plain = true;
+    for (int i = 0; i < nout; ++i)
+      if (b.g[i].bias || b.g[i].aux || b.g[i].ldd % 8) plain = false;
+    for (int j = 0; j < b.scatter_n; ++j)
+      if (b.res_seq[j] || reinterpret_cast<uintptr_t>(b.out_seq[j]) % 16) plain = false;
+    p.plain_staged = plain ? 1 : 0;
   }
   if (b.scatter_n > 0 && tma_epilogue_ok(b, nout, ksplit)) {
     p.tma_epi = 1;
