@@ -508,7 +508,7 @@ def run_ours(args, world, rank, local):
             o = measure_other(sub, world, rank, local, sample_clocks=False)
             keep = ("value", "unit", "ms_per_step", "frac_of_burst_peak", "roofline", "gpu_launches",
                     "device_status")
-            others[wl] = {"workload": o["config"]["workload"], "cuda_graph": graph,
+            others[wl] = {"workload": o["config"]["workload"], "cuda_graph": graph, "l2": o["config"]["l2"],
                           **{k: o[k] for k in keep}}
     status = tp.device_status()
     if rank != 0:
@@ -741,6 +741,7 @@ def measure_other(args, world, rank, local, sample_clocks=True):
         flops = blk.flops_fwd(b, s)
         step = lambda: blk.forward(X, b, s, residual=X)
         name = "attention block fwd: hidden 4096, 32 heads x 128, seq 4096, batch 2, p=8, causal"
+        l2 = "inputs larger than L2 (X 67 MB, Wqkv 101 MB, the shards' QKV 201 MB); no flush"
         # attention-core launches alone, for the roofline of the dominant kernel
         core = lambda: blk.plan.attention_fwd(b, s, blk.QKV, blk.O, blk.LSE)
         core_flops = 4.0 * b * H * (s * (s + 1) / 2) * (h // H)
@@ -758,6 +759,7 @@ def measure_other(args, world, rank, local, sample_clocks=True):
             sp.forward(Xs)
             sp.backward(dYs)
         name = "Megatron-SP SwiGLU MLP fwd+bwd: hidden 8192, ffn 28672, seq 8192, batch 1, p=8"
+        l2 = "inputs larger than L2 (W1 940 MB, W2 470 MB, gathered X 134 MB); no flush"
         core, core_flops = None, None
     else:
         L, b, s_, h, f, H, p = 12, 8, 512, 512, 2048, 8, 4
@@ -782,6 +784,9 @@ def measure_other(args, world, rank, local, sample_clocks=True):
                 g = lay.backward(g, b, s_, join=False)
             tp.backward_join()
         name = "12-layer block stack fwd+bwd: hidden 512, MLP 2048, 8 heads x 64, tokens 8x512, p=4"
+        # a layer keeps about 65 MB of activations for its backward (LN outputs, QKV,
+        # attention output, Z and H of the MLP), so the step's data is well over L2
+        l2 = "a step touches about 0.8 GB (12 layers' saved activations), larger than L2; no flush"
         core, core_flops = None, None
     for _ in range(args.warmup):
         step()
@@ -849,7 +854,7 @@ def measure_other(args, world, rank, local, sample_clocks=True):
            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded tp_synth)",
            "config": {"workload": name, "variant": args.variant,
-                      "cuda_graph": bool(args.graph)}, "roofline": roof,
+                      "cuda_graph": bool(args.graph), "l2": l2}, "roofline": roof,
            "frac_of_burst_peak": value / peaks["bf16_tflops"],
            "gpu_launches": launches, "clocks": clk,
            "device_status": tp.device_status()}
