@@ -320,7 +320,9 @@ TP_API tp_status tp_attention_fwd(tp_plan* plan, int batch, int seq, const void*
 
 /* ------------------------------------------------------------ backward */
 
-/* Streams of the backward calls: tp_row_bwd (dZ and dW) and the column
+/* Streams of the backward calls (scheduling only: the pages' backward
+ * ([TP-scratch] §四) fixes what is computed, not the launch order, and has no
+ * counterpart of these switches): tp_row_bwd (dZ and dW) and the column
  * backward calls (dX and dW) issue two GEMMs that read the same inputs. When
  * either leaves SMs idle (few output tiles), the activation-gradient GEMM runs
  * on a side stream the library creates per device, forked from `stream` by an
@@ -453,7 +455,11 @@ TP_API tp_status tp_attention_bwd(tp_plan* plan, int batch, int seq, const void*
                            const float* const* LSE, void* const* dQKV, void* stream);
 
 /* Column sums over rows: out[c] = sum_r x[r, c] in fp32 (fixed order;
- * accumulate != 0 adds to out). x [rows, cols] in the plan dtype. One launch:
+ * accumulate != 0 adds to out) -- the bias gradient of a layer, db = the sum
+ * over tokens of its output gradient ([TP-basics] 实现细节: the row bias is
+ * one full vector, so its gradient is the column sum of dY once; the column
+ * bias shard i gets the column sums of dZ_i). x [rows, cols] in the plan
+ * dtype. One launch:
  * blocks sum row splits into the plan's workspace and the last block of each
  * column slab adds the splits in order. The plan's first reduction on a
  * device allocates its workspace and arrival counters, so it must not be the
@@ -536,7 +542,10 @@ typedef struct tp_peer_group {
   void* recv[TP_MAX_SHARDS];      /* rank d's receive buffer (device): world slots of [T/world, hidden] */
 } tp_peer_group;
 
-/* Device memory that other processes can map: `bytes` (> 0) from cudaMalloc
+/* Buffers of the exchange above ([TP-blog] §4.1: every GPU holds a partial
+ * sum that the others need; here each rank's receive buffer and flag words,
+ * mapped into the other ranks' processes).
+ * Device memory that other processes can map: `bytes` (> 0) from cudaMalloc
  * on the current device, zero-filled, its IPC handle written to `handle`
  * (TP_PEER_HANDLE_BYTES host bytes). Free with tp_peer_free. */
 TP_API tp_status tp_peer_alloc(size_t bytes, void** ptr, void* handle);
