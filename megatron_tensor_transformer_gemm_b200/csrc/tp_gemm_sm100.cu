@@ -1132,6 +1132,13 @@ struct Layout {
 // move more operand bytes per FLOP (one CTA instead of a pair, N = 128
 // instead of 256) carry a factor, so they win only when they fill more SMs:
 // small problems, whose 256 x 256 tiles leave most of the GPU idle.
+// CTA pairs are considered only for launches of at least one 256 x 256 tile
+// per SM (two waves of pairs): below that the launch is a wave or two of
+// short tiles, where what a pair saves in operand reads is less than what it
+// costs to start and to keep two SMs in step. Measured on the 12-layer stack
+// at hidden 512 (every GEMM 16-128 such tiles): single CTAs took the step
+// from 3.63 to 3.51 ms; the larger workloads' launches (512 and more tiles)
+// keep their pairs.
 Layout choose_layout(const GemmBatch& b, int sms, double* cost_out = nullptr) {
   const bool swiglu = b.epi == tpi::EPI_SWIGLU;
   const int ks = b.ksplit > 1 ? b.ksplit : 1;
@@ -1141,10 +1148,14 @@ Layout choose_layout(const GemmBatch& b, int sms, double* cost_out = nullptr) {
     for (int i = 0; i < b.n; ++i) kb_cat += (b.g[i].K + BK - 1) / BK;
   const int fp = forced_pair();
   const int fn = swiglu ? 0 : forced_narrow();
+  int64_t pair_tiles = 0;  // 256 x 256 tiles of the launch
+  for (int i = 0; i < nout; ++i)
+    pair_tiles += static_cast<int64_t>((b.g[i].M + 2 * BM - 1) / (2 * BM)) * ((b.g[i].N + BN - 1) / BN) * ks;
   Layout best{2, false};
   double best_cost = -1.0;
   for (int pair = 2; pair >= 1; --pair) {
     if (fp && pair != fp) continue;
+    if (!fp && pair == 2 && pair_tiles < sms) continue;
     for (int nar = 0; nar <= (swiglu ? 0 : 1); ++nar) {
       if (fn >= 0 && nar != fn) continue;
       const int tile_m = BM * pair;
