@@ -783,3 +783,73 @@ def test_mutant_padding_included_fails_the_ce_pin():
     bad, _ = O.cross_entropy(z, labels, 16)   # padding columns wrongly in the softmax
     good, _ = O.cross_entropy(z, labels, V)
     assert not np.allclose(bad, good)
+
+
+# ---- the attention sublayer and the pre-LN layer, by their special cases
+
+def _attn_params(h):
+    return randn(3 * h, h, std=0.5), 0.1 * randn(3 * h), randn(h, h, std=0.5), 0.1 * randn(h)
+
+
+def test_attn_sublayer_one_position_passes_v_through():
+    # One position per sequence: the causal softmax runs over a single score
+    # and equals 1, so the attention output is V itself and the sublayer is
+    # (u Wv^T + bv) Wo^T + bo, with Wv the last h rows of Wqkv.
+    batch, h, H = 3, 4, 2
+    u = randn(batch, h)
+    Wqkv, bqkv, Wo, bo = _attn_params(h)
+    a = O.attn_sublayer_fwd(u, Wqkv, bqkv, Wo, bo, batch, H)
+    V = u @ Wqkv[2 * h:].T + bqkv[2 * h:]
+    np.testing.assert_allclose(a["Y"], V @ Wo.T + bo, rtol=1e-12, atol=1e-12)
+
+
+def test_attn_sublayer_equal_scores_average_the_values_so_far():
+    # Wq = 0, bq = 0: every score is 0, so causal attention at position i is the
+    # plain mean of V over positions 0..i (the diagonal included).
+    batch, s, h, H = 2, 5, 4, 2
+    u = randn(s * batch, h)
+    Wqkv, bqkv, Wo, bo = _attn_params(h)
+    Wqkv[:h] = 0.0
+    bqkv[:h] = 0.0
+    a = O.attn_sublayer_fwd(u, Wqkv, bqkv, Wo, bo, batch, H)
+    V = (u @ Wqkv[2 * h:].T + bqkv[2 * h:]).reshape(s, batch, h)
+    want = np.stack([V[:i + 1].mean(axis=0) for i in range(s)]).reshape(s * batch, h)
+    np.testing.assert_allclose(a["O"], want, rtol=1e-12, atol=1e-12)
+
+
+def test_attn_sublayer_is_causal():
+    # Changing the tokens of the last position leaves every earlier row as it
+    # was and changes the last one (rows are position-major: row = pos * batch + b).
+    batch, s, h, H = 2, 4, 4, 2
+    u = randn(s * batch, h)
+    Wqkv, bqkv, Wo, bo = _attn_params(h)
+    y0 = O.attn_sublayer_fwd(u, Wqkv, bqkv, Wo, bo, batch, H)["Y"]
+    u2 = u.copy()
+    u2[(s - 1) * batch:] += randn(batch, h)
+    y1 = O.attn_sublayer_fwd(u2, Wqkv, bqkv, Wo, bo, batch, H)["Y"]
+    np.testing.assert_allclose(y1[:(s - 1) * batch], y0[:(s - 1) * batch], rtol=0, atol=1e-14)
+    assert np.abs(y1[(s - 1) * batch:] - y0[(s - 1) * batch:]).max() > 1e-3
+
+
+def test_layer_fwd_zero_sublayers_are_residual_identities():
+    batch, s, h, f, H = 2, 3, 4, 8, 2
+    x = randn(batch * s, h)
+    P = _layer_params(h, f, H)
+    # both sublayers' output projections zero: each adds nothing
+    Z = dict(P, Wo=np.zeros_like(P["Wo"]), bo=np.zeros_like(P["bo"]),
+             W2=np.zeros_like(P["W2"]), b2=np.zeros_like(P["b2"]))
+    assert np.array_equal(O.layer_fwd(x, Z, batch, H)["y"], x)
+    # only the MLP zero: y = x + Attn(LN1(x))
+    A = dict(P, W2=np.zeros_like(P["W2"]), b2=np.zeros_like(P["b2"]))
+    u1 = O.layernorm_fwd(x, P["ln1_g"], P["ln1_b"])[0]
+    att = O.attn_sublayer_fwd(u1, P["Wqkv"], P["bqkv"], P["Wo"], P["bo"], batch, H)["Y"]
+    np.testing.assert_allclose(O.layer_fwd(x, A, batch, H)["y"], x + att, rtol=1e-13, atol=1e-13)
+    # both on: the MLP reads LN2 of the attention's residual sum, not of x
+    full = O.layer_fwd(x, P, batch, H)
+    x1 = x + att
+    u2 = O.layernorm_fwd(x1, P["ln2_g"], P["ln2_b"])[0]
+    mlp = O.mlp_fwd(u2, P["W1"], P["b1"], P["W2"], P["b2"], "gelu")["Y"]
+    np.testing.assert_allclose(full["y"], x1 + mlp, rtol=1e-13, atol=1e-13)
+    wrong = O.mlp_fwd(O.layernorm_fwd(x, P["ln2_g"], P["ln2_b"])[0], P["W1"], P["b1"], P["W2"], P["b2"],
+                      "gelu")["Y"]
+    assert np.abs(full["y"] - (x1 + wrong)).max() > 1e-3
