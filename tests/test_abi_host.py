@@ -270,3 +270,21 @@ def test_wgrad_grouping_calls_validate(plan):
     assert L.tp_set_wgrad_grouping(plan.handle, 1) == 0
     assert L.tp_flush_wgrad(plan.handle) == 0          # nothing waits: no device call
     assert L.tp_set_wgrad_grouping(plan.handle, 0) == 0
+
+
+def test_static_column_sum_validates_before_any_device_call():
+    """The allocation-free column sum rejects bad arguments on the host, and
+    column counts beyond its fixed scratch (512 Ki floats) with a clear error."""
+    f = tp.lib.tp_column_sum_static
+    assert f(4, 8, 7, FAKE, FAKE, 0, None) == 4                 # unknown dtype
+    assert f(-1, 8, 1, FAKE, FAKE, 0, None) == 1                # rows < 0
+    assert f(4, 0, 1, FAKE, FAKE, 0, None) == 1                 # cols = 0
+    assert f(4, 524288 + 8, 1, FAKE, FAKE, 0, None) == 5        # beyond the static scratch
+    assert "524288" in tp.last_error()
+    assert f(4, 8, 1, None, FAKE, 0, None) == 1                 # x NULL with rows > 0
+    assert f(4, 8, 1, FAKE, None, 0, None) == 1                 # out NULL
+    assert f(4, 8, 1, FAKE + 2, FAKE, 0, None) == 3             # x not 16-byte aligned
+    assert f(4, 12, 1, FAKE, FAKE, 0, None) == 3                # a bf16 row of 24 bytes
+    if not torch.cuda.is_available():
+        # valid arguments reach the device lookup, which fails on the host
+        assert f(4, 8, 1, FAKE, FAKE, 0, None) in (6, 8)
